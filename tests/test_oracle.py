@@ -1,0 +1,339 @@
+"""Pins for the oracle: each check is independent of the oracle's own formulas (hand-packed blocks
+with hand-computed values, an independent GGUF decoder, closed forms, finite differences,
+brute-force loops), so a dropped term, a wrong sign or index, or a transposed operand fails one."""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import gguf_blocks as gb
+from oracle import lora_linear as ll
+from oracle import moe as om
+from quantized_base_lora_tma_b200 import inputs as inp
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _hand_blocks():
+    out = []
+    with open(os.path.join(GOLDEN, "gguf_hand_blocks.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            t, hx, vals = [p.strip() for p in line.split("|")]
+            raw = np.frombuffer(bytes.fromhex(hx.replace(" ", "")), np.uint8)
+            out.append((t, raw, np.array([float(v) for v in vals.split()])))
+    return out
+
+
+@pytest.mark.parametrize("case", range(4))
+def test_hand_packed_q4_0_q8_0(case):
+    t, raw, want = _hand_blocks()[case]
+    qt = {"q4_0": gb.Q4_0, "q8_0": gb.Q8_0}[t]
+    got = gb.decode_exact(qt, raw, 1, 32)[0]
+    assert np.array_equal(got, want)
+
+
+def _hand_q4_k(d16, dmin16, sc, m, q):
+    """Pack one Q4_K superblock byte by byte from (sc, m, q) chosen by hand."""
+    S = [0] * 12
+    for j in range(4):
+        S[j] = (sc[j] & 63) | ((sc[j + 4] >> 4) << 6)
+        S[j + 4] = (m[j] & 63) | ((m[j + 4] >> 4) << 6)
+        S[j + 8] = (sc[j + 4] & 15) | ((m[j + 4] & 15) << 4)
+    qs = []
+    for i in range(4):
+        qs += [q[2 * i][l] | (q[2 * i + 1][l] << 4) for l in range(32)]
+    raw = bytes([d16 & 255, d16 >> 8, dmin16 & 255, dmin16 >> 8] + S + qs)
+    assert len(raw) == 144
+    return np.frombuffer(raw, np.uint8)
+
+
+def test_hand_packed_q4_k_high_bit_split():
+    # Scales and mins >= 16 in sub-blocks 4..7 exercise the split of their top 2 bits into S[0..7].
+    sc = [1, 2, 3, 4, 17, 33, 50, 63]
+    m = [0, 1, 2, 3, 16, 31, 47, 62]
+    q = [[(l + j) % 16 for l in range(32)] for j in range(8)]
+    raw = _hand_q4_k(0x3C00, 0x3800, sc, m, q)          # d = 1.0, dmin = 0.5
+    # the 12 scale bytes, worked out by hand
+    assert list(raw[4:16]) == [0x41, 0x82, 0xC3, 0xC4, 0x40, 0x41, 0x82, 0xC3, 0x01, 0xF1, 0xF2, 0xEF]
+    got = gb.decode_exact(gb.Q4_K, raw, 1, 256)[0].reshape(8, 32)
+    want = np.array([[1.0 * sc[j] * q[j][l] - 0.5 * m[j] for l in range(32)] for j in range(8)])
+    assert np.array_equal(got, want)
+
+
+def _random_blocks(qtype, nblocks, rng):
+    bb = {gb.Q4_0: 18, gb.Q8_0: 34, gb.Q4_K: 144}[qtype]
+    raw = rng.integers(0, 256, size=(nblocks, bb), dtype=np.uint8)
+    # finite fp16 scales only (random bytes could spell Inf/NaN)
+    n_h = 2 if qtype == gb.Q4_K else 1
+    for h in range(n_h):
+        d = (rng.standard_normal(nblocks) * 0.01).astype(np.float16)
+        d[::7] = np.float16(6.0e-8)                    # include subnormal scales
+        raw[:, 2 * h:2 * h + 2] = d.view(np.uint8).reshape(-1, 2)
+    return raw
+
+
+@pytest.mark.parametrize("qtype,gtype", [(gb.Q4_0, "Q4_0"), (gb.Q8_0, "Q8_0"), (gb.Q4_K, "Q4_K")])
+def test_decode_matches_gguf_py(qtype, gtype):
+    """Independent codebase: gguf-py's dequantize (fp32) must equal the fp32 rounding of the exact
+    decode, element by element."""
+    gguf = pytest.importorskip("gguf")
+    from gguf import quants
+    rng = np.random.default_rng(7)
+    qk = {gb.Q4_0: 32, gb.Q8_0: 32, gb.Q4_K: 256}[qtype]
+    rows, cols = 16, 4 * qk if qtype == gb.Q4_K else 16 * qk
+    raw = _random_blocks(qtype, rows * cols // qk, rng).reshape(rows, -1)
+    want = quants.dequantize(raw, getattr(gguf.GGMLQuantizationType, gtype)).astype(np.float32)
+    got = gb.deq_f32(qtype, raw, rows, cols).astype(np.float32)
+    assert np.array_equal(got.view(np.uint32), want.reshape(rows, cols).view(np.uint32))
+
+
+def test_decode_value_grid_closed_form():
+    """Q4_0 values lie on d*{-8..7}; Q8_0 on d*{-128..127}."""
+    rng = np.random.default_rng(3)
+    for qt, lo, hi in [(gb.Q4_0, -8, 7), (gb.Q8_0, -128, 127)]:
+        raw = _random_blocks(qt, 64, rng)
+        d = raw[:, 0:2].copy().view(np.float16).astype(np.float64).ravel()
+        w = gb.decode_exact(qt, raw, 64, 32)
+        k = w / np.where(d == 0, 1, d)[:, None]
+        assert np.all(k == np.round(k)) and k.min() >= lo and k.max() <= hi
+
+
+@pytest.mark.parametrize("gtype", ["Q4_0", "Q8_0"])
+def test_packers_match_gguf_py_bytes(gtype):
+    """The input encoders agree byte for byte with gguf-py's quantize (pins the input recipe)."""
+    gguf = pytest.importorskip("gguf")
+    from gguf import quants
+    rng = np.random.default_rng(11)
+    x = (rng.standard_normal((32, 512)) * 0.02).astype(np.float32)
+    x[3, :32] = 0.0
+    qt = {"Q4_0": inp.Q4_0, "Q8_0": inp.Q8_0}[gtype]
+    assert np.array_equal(inp.pack(qt, x), quants.quantize(x, getattr(gguf.GGMLQuantizationType, gtype)))
+
+
+@pytest.mark.parametrize("qtype", [inp.Q4_0, inp.Q8_0, inp.Q4_K])
+def test_pack_roundtrip_error_bound(qtype):
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal((8, 512)) * 0.02).astype(np.float32)
+    w = gb.decode_exact(qtype, inp.pack(qtype, x), 8, 512)
+    err = np.abs(w - x)
+    if qtype == inp.Q4_K:
+        assert err.max() < 0.2 * (x.max() - x.min()) / 15 * 8
+    else:
+        qk = 32
+        d = np.abs(inp.pack(qtype, x).reshape(-1, 18 if qtype == inp.Q4_0 else 34)[:, :2].copy()
+                   .view(np.float16).astype(np.float64)).ravel()
+        # half a step (a whole step at Q4_0's clipped top end) plus the fp16 rounding of d,
+        # which the quantizer does not see: at most |q| * 2^-11 * |d|
+        bound = d * (1 + 8 * 2.0 ** -11) if qtype == inp.Q4_0 else d * (0.5 + 127 * 2.0 ** -11)
+        assert np.all(err.reshape(-1, qk) <= bound[:, None] * (1 + 1e-6) + 1e-12)
+
+
+def test_round_bf16_ties_and_torch():
+    one = 1.0
+    assert gb.round_bf16(np.array([one + 2 ** -8]))[0] == 1.0                  # tie -> even
+    assert gb.round_bf16(np.array([one + 3 * 2 ** -8]))[0] == one + 2 ** -6    # tie -> even (up)
+    assert gb.round_bf16(np.array([one + 2 ** -8 + 2 ** -20]))[0] == one + 2 ** -7
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal(100000).astype(np.float32)
+    want = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(gb.round_bf16(x.astype(np.float64)), want)
+
+
+# ------------------------------------------------------------------------------------------------
+# dense linear
+# ------------------------------------------------------------------------------------------------
+def _small_linear(M=5, K=256, N=7, r=3, qtype=inp.Q4_0, seed=0):
+    c = inp.linear_case(M, K, N, qtype, r, 2.0 * r, seed)
+    f = gb.bf16_bits_to_f64
+    return c, f(c.X), f(c.dY), f(c.A), f(c.B)
+
+
+def test_linear_b_zero_is_base_gemm():
+    """B = 0: Y is the dequantized base GEMM (computed here with gguf-py's decoder and torch),
+    dA = 0 exactly and dB = s dY^T (X A^T)."""
+    gguf = pytest.importorskip("gguf")
+    from gguf import quants
+    c, X, dY, A, B = _small_linear(M=9, K=512, N=33)
+    B0 = np.zeros_like(B)
+    W = ll.weights(c.qtype, c.wq, c.N, c.K)
+    Y, H = ll.linear_fwd(W, X, A, B0, c.scale)
+    Wg = quants.dequantize(c.wq, gguf.GGMLQuantizationType.Q4_0).astype(np.float32)
+    Wg = torch.from_numpy(Wg).to(torch.bfloat16).double()
+    Yt = torch.nn.functional.linear(torch.from_numpy(X), Wg).numpy()
+    assert np.allclose(Y, Yt, rtol=0, atol=1e-12)
+    dX, dA, dB, G = ll.linear_bwd(W, X, dY, A, B0, c.scale, H)
+    assert np.all(dA == 0) and np.all(G == 0)
+    dB_t = c.scale * torch.einsum("mn,mj->nj", torch.from_numpy(dY),
+                                  torch.einsum("mk,jk->mj", torch.from_numpy(X), torch.from_numpy(A)))
+    assert np.allclose(dB, dB_t.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_linear_lora_selector_closed_form():
+    """A picks X's first r columns and B = c*[I_r; 0]: the LoRA term is s*c*X[:, n] for n < r and 0
+    beyond, so a transposed operand, a missing s or a wrong index shows."""
+    c, X, dY, A, B = _small_linear(M=6, K=256, N=9, r=3)
+    r = c.r
+    A = np.zeros_like(A); A[np.arange(r), np.arange(r)] = 1.0
+    B = np.zeros_like(B); B[np.arange(r), np.arange(r)] = 0.75
+    W0 = np.zeros((c.N, c.K))
+    Y, H = ll.linear_fwd(W0, X, A, B, c.scale)
+    want = np.zeros((c.M, c.N)); want[:, :r] = c.scale * 0.75 * X[:, :r]
+    assert np.array_equal(Y, want)
+    assert np.array_equal(H, X[:, :r])
+
+
+@pytest.mark.parametrize("qtype", [inp.Q4_0, inp.Q8_0, inp.Q4_K])
+def test_linear_grads_finite_differences(qtype):
+    """Central differences of L = sum(dY * Y) against the analytic dX, dA, dB (fp64, exact decode)."""
+    c, X, dY, A, B = _small_linear(M=3, K=256, N=5, r=2, qtype=qtype)
+    s = c.scale
+    W = ll.weights(qtype, c.wq, c.N, c.K, round_weights=False)
+
+    def loss(X_, A_, B_):
+        return float((dY * ll.linear_fwd(W, X_, A_, B_, s)[0]).sum())
+
+    dX, dA, dB, _ = ll.linear_bwd(W, X, dY, A, B, s)
+    h = 1e-4
+    rng = np.random.default_rng(1)
+    for name, T, grad in [("X", X, dX), ("A", A, dA), ("B", B, dB)]:
+        for _ in range(12):
+            i = tuple(rng.integers(0, n) for n in T.shape)
+            Tp, Tm = T.copy(), T.copy()
+            Tp[i] += h; Tm[i] -= h
+            args_p = {"X": X, "A": A, "B": B}; args_m = dict(args_p)
+            args_p[name] = Tp; args_m[name] = Tm
+            fd = (loss(args_p["X"], args_p["A"], args_p["B"]) - loss(args_m["X"], args_m["A"], args_m["B"])) / (2 * h)
+            assert abs(fd - grad[i]) <= 1e-6 * max(1.0, abs(grad[i])), (name, i, fd, grad[i])
+
+
+# ------------------------------------------------------------------------------------------------
+# routing
+# ------------------------------------------------------------------------------------------------
+def test_route_invariants_and_brute_force():
+    rng = np.random.default_rng(2)
+    T, E, k = 50, 16, 4
+    logits = gb.bf16_bits_to_f64(inp.to_bf16_bits(rng.standard_normal((T, E)).astype(np.float32)))
+    logits[3, :] = logits[3, 0]          # a token with all-equal logits
+    logits[4, 5] = logits[4, 9] = 10.0   # a tie at the top
+    idx, w, counts, offsets, perm, inv = om.route(logits, k)
+    assert counts.sum() == T * k and offsets[-1] == T * k and np.all(np.diff(offsets) == counts)
+    assert np.array_equal(np.sort(perm), np.arange(T * k))
+    assert np.array_equal(perm[inv], np.arange(T * k))
+    assert np.allclose(w.sum(axis=1), 1.0, atol=1e-15)
+    assert list(idx[3]) == [0, 1, 2, 3]
+    assert list(idx[4][:2]) == [5, 9]
+    for t in range(T):
+        assert len(set(idx[t])) == k
+        # brute force: repeatedly take the largest remaining logit, lowest index on ties
+        rem = list(range(E)); sel = []
+        for _ in range(k):
+            best = rem[0]
+            for e in rem:
+                if logits[t, e] > logits[t, best]:
+                    best = e
+            sel.append(best); rem.remove(best)
+        assert list(idx[t]) == sel
+        ex = [math.exp(logits[t, e]) for e in sel]
+        assert np.allclose(w[t], np.array(ex) / sum(ex), rtol=1e-13)
+    # pairs sorted by (expert, token, slot)
+    keys = [(idx[p // k, p % k], p // k, p % k) for p in perm]
+    assert keys == sorted(keys)
+
+
+# ------------------------------------------------------------------------------------------------
+# MoE
+# ------------------------------------------------------------------------------------------------
+def _small_moe(T=6, H=256, I=256, E=4, k=2, r=2, qtype=inp.Q4_0, seed=0):
+    c = inp.moe_case(T, H, I, E, k, qtype, r, 2.0 * r, seed)
+    f = gb.bf16_bits_to_f64
+    return c, f(c.X), f(c.dY), f(c.logits), f(c.A_gu), f(c.B_gu), f(c.A_d), f(c.B_d)
+
+
+def _brute_token_ffn(x, Wgu, Wd, Agu, Bgu, Ad, Bd, s, I):
+    """One token through one expert, written as explicit per-element sums (no matmul)."""
+    H = x.shape[0]
+    r = Agu.shape[0]
+    hg = [sum(x[kk] * Agu[j, kk] for kk in range(H)) for j in range(r)]
+    gu = [sum(x[kk] * Wgu[n, kk] for kk in range(H)) + s * sum(hg[j] * Bgu[n, j] for j in range(r))
+          for n in range(2 * I)]
+    h = [gu[i] / (1 + math.exp(-gu[i])) * gu[I + i] for i in range(I)]
+    hd = [sum(h[i] * Ad[j, i] for i in range(I)) for j in range(r)]
+    return np.array([sum(h[i] * Wd[n, i] for i in range(I)) + s * sum(hd[j] * Bd[n, j] for j in range(r))
+                     for n in range(H)])
+
+
+def test_moe_fwd_vs_per_token_brute_force():
+    c, X, dY, L, Agu, Bgu, Ad, Bd = _small_moe(T=5, H=256, I=256, E=4, k=2)
+    Wgu, Wd = om.expert_weights(c.qtype, c.w_gu, c.w_d, c.H, c.I, round_weights=False)
+    idx, w, counts, offsets, perm, inv = om.route(L, c.k)
+    Y, _ = om.moe_fwd(Wgu, Wd, X, idx, w, counts, offsets, perm, Agu, Bgu, Ad, Bd, c.scale, mirror=False)
+    for t in [0, 3]:
+        want = np.zeros(c.H)
+        for j in range(c.k):
+            e = idx[t, j]
+            want += w[t, j] * _brute_token_ffn(X[t], Wgu[e], Wd[e], Agu[e], Bgu[e], Ad[e], Bd[e], c.scale, c.I)
+        assert np.allclose(Y[t], want, rtol=1e-10, atol=1e-12)
+
+
+def test_moe_single_expert_is_dense_swiglu_with_lora():
+    """E = 1, k = 1: the layer is one dense SwiGLU FFN built from the dense LoRA linear oracle."""
+    c, X, dY, L, Agu, Bgu, Ad, Bd = _small_moe(T=7, E=1, k=1)
+    Wgu, Wd = om.expert_weights(c.qtype, c.w_gu, c.w_d, c.H, c.I)
+    idx, w, counts, offsets, perm, inv = om.route(L, 1)
+    assert np.all(w == 1.0)
+    Y, saved = om.moe_fwd(Wgu, Wd, X, idx, w, counts, offsets, perm, Agu, Bgu, Ad, Bd, c.scale, mirror=False)
+    gu, _ = ll.linear_fwd(Wgu[0], X, Agu[0], Bgu[0], c.scale)
+    g, u = gu[:, :c.I], gu[:, c.I:]
+    sig = 1 / (1 + np.exp(-g))
+    h = g * sig * u
+    o, _ = ll.linear_fwd(Wd[0], h, Ad[0], Bd[0], c.scale)
+    assert np.allclose(Y, o, rtol=1e-12, atol=1e-12)
+    gr = om.moe_bwd(Wgu, Wd, X, dY, idx, w, counts, offsets, perm, Agu, Bgu, Ad, Bd, c.scale, saved, mirror=False)
+    dh, dAd, dBd, _ = ll.linear_bwd(Wd[0], h, dY, Ad[0], Bd[0], c.scale)
+    dgu = np.concatenate([dh * u * sig * (1 + g * (1 - sig)), dh * g * sig], axis=1)
+    dX, dAgu, dBgu, _ = ll.linear_bwd(Wgu[0], X, dgu, Agu[0], Bgu[0], c.scale)
+    for got, want in [(gr["dX"], dX), (gr["dA_d"][0], dAd), (gr["dB_d"][0], dBd),
+                      (gr["dA_gu"][0], dAgu), (gr["dB_gu"][0], dBgu)]:
+        assert np.allclose(got, want, rtol=1e-11, atol=1e-12)
+    assert np.allclose(gr["d_logits_sel"], 0.0)      # one selected expert: weight is constant 1
+
+
+def test_moe_grads_finite_differences():
+    c, X, dY, L, Agu, Bgu, Ad, Bd = _small_moe(T=4, H=256, I=256, E=3, k=2, r=2)
+    # separate the logits so that small perturbations never change the selection
+    L = L + np.arange(c.E)[None, :] * 0.0 + np.array([[0.0, 0.7, 1.9]])
+    Wgu, Wd = om.expert_weights(c.qtype, c.w_gu, c.w_d, c.H, c.I, round_weights=False)
+    s = c.scale
+
+    def run(X_, L_, Agu_, Bgu_, Ad_, Bd_):
+        idx, w, counts, offsets, perm, inv = om.route(L_, c.k)
+        Y, saved = om.moe_fwd(Wgu, Wd, X_, idx, w, counts, offsets, perm, Agu_, Bgu_, Ad_, Bd_, s, mirror=False)
+        return Y, saved, (idx, w, counts, offsets, perm)
+
+    Y, saved, (idx, w, counts, offsets, perm) = run(X, L, Agu, Bgu, Ad, Bd)
+    gr = om.moe_bwd(Wgu, Wd, X, dY, idx, w, counts, offsets, perm, Agu, Bgu, Ad, Bd, s, saved, mirror=False)
+    dL = om.scatter_d_logits(idx, gr["d_logits_sel"], c.E)
+    names = ["X", "L", "Agu", "Bgu", "Ad", "Bd"]
+    vals = dict(X=X, L=L, Agu=Agu, Bgu=Bgu, Ad=Ad, Bd=Bd)
+    grads = dict(X=gr["dX"], L=dL, Agu=gr["dA_gu"], Bgu=gr["dB_gu"], Ad=gr["dA_d"], Bd=gr["dB_d"])
+    rng = np.random.default_rng(4)
+    h = 1e-5
+    for name in names:
+        T = vals[name]
+        for _ in range(6):
+            i = tuple(rng.integers(0, n) for n in T.shape)
+            if name in ("Bgu", "Agu", "Ad", "Bd") and counts[i[0]] == 0:
+                continue
+            out = []
+            for sgn in (1, -1):
+                v = dict(vals)
+                v[name] = T.copy(); v[name][i] += sgn * h
+                out.append(float((dY * run(v["X"], v["L"], v["Agu"], v["Bgu"], v["Ad"], v["Bd"])[0]).sum()))
+            fd = (out[0] - out[1]) / (2 * h)
+            g = grads[name][i]
+            assert abs(fd - g) <= 1e-5 * max(1.0, abs(g)), (name, i, fd, g)
