@@ -1,0 +1,123 @@
+/*
+ * qlora.h — C ABI of the frozen-GGUF-base + LoRA layer library for NVIDIA B200 (sm_100a).
+ *
+ * The layer is the one the LoRA-over-GGUF training recipe runs in every projection: a frozen,
+ * block-quantized base weight (GGUF Q8_0, Q4_0 or Q4_K) plus a trainable rank-r adapter, dense and
+ * as routed per-expert SwiGLU MoE ("Things involved in the training" of Show HN: LoRA over GGUF:
+ * MMQ and grouped MMQ, the fast LoRA backward formula for linear and MoE layers, MoE routing, the
+ * GGUF dequant function). With s = alpha / r:
+ *
+ *   forward   Y  = X deq(W)^T + s (X A^T) B^T             H = X A^T is returned for the backward
+ *   backward  dX = dY deq(W) + s (dY B) A,  dA = s (dY B)^T X,  dB = s dY^T H;  W is never updated
+ *
+ * Conventions for every entry point
+ *   - All tensor arguments are DEVICE pointers to row-major, contiguous buffers that the caller
+ *     allocated and owns; the library never allocates, frees or synchronises. Work is enqueued on
+ *     `stream` (a cudaStream_t passed as void*, NULL = legacy default stream) and is asynchronous:
+ *     results are valid after the caller synchronises that stream.
+ *   - bf16 tensors are IEEE bfloat16 (uint16 storage). Packed weights are GGUF blocks in file
+ *     order: a weight [rows x cols] is `rows` packed rows of cols/QK blocks each (QK = 32 for
+ *     Q4_0/Q8_0, 256 for Q4_K; 18, 34, 144 bytes per block). Expert stacks are [E][rows][...].
+ *   - Every pointer must be 16-byte aligned; the packed weight rows, X, dY, A and B rows must make
+ *     every row start 16-byte aligned (guaranteed by the shape rules below).
+ *   - Return value: a ql_status. Argument errors are detected on the host before anything is
+ *     launched. Launch failures return QL_ERR_CUDA. Faults inside kernels surface at the caller's
+ *     synchronisation as CUDA errors; a device-side wait that exceeds its bound (about one second)
+ *     sets a device status word, read with qlora_device_status().
+ *   - Workspace: entry points that need scratch take (ws, ws_bytes); the required size comes from
+ *     the matching *_workspace_bytes() query. The caller owns it; its contents on entry do not
+ *     matter.
+ */
+#ifndef QLORA_H
+#define QLORA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+#if defined(__GNUC__)
+#pragma GCC visibility push(default)
+#endif
+
+/* GGML type ids of the supported block formats. */
+typedef enum { QL_Q4_0 = 2, QL_Q8_0 = 8, QL_Q4_K = 12 } ql_qtype;
+
+/* Element type of an output tensor. */
+typedef enum { QL_F32 = 0, QL_BF16 = 1 } ql_dtype;
+
+typedef enum {
+  QL_OK = 0,
+  QL_ERR_INVALID_ARG = 1, /* null pointer, bad enum, non-positive size */
+  QL_ERR_UNSUPPORTED = 2, /* a qtype / rank / expert count this build does not handle */
+  QL_ERR_SHAPE = 3,       /* a size rule is broken (e.g. K % 256 != 0) */
+  QL_ERR_ALIGNMENT = 4,   /* a pointer is not 16-byte aligned */
+  QL_ERR_WORKSPACE = 5,   /* ws is NULL or smaller than the query says */
+  QL_ERR_CUDA = 6,        /* a CUDA runtime / driver call failed */
+  QL_ERR_TIMEOUT = 7      /* a device-side bounded wait gave up (device status word) */
+} ql_status;
+
+/* Human-readable name of a status code. Never NULL. */
+const char* qlora_status_string(int status);
+
+/* Number of the library's own kernel launches since load (all entry points, all streams). */
+uint64_t qlora_launch_count(void);
+
+/* Reads the device status word of the current device (synchronises the device first). Returns
+ * QL_OK or the first recorded device-side error (QL_ERR_TIMEOUT); *site (nullable) receives the
+ * code of the wait that gave up. reset != 0 clears the word afterwards. */
+int qlora_device_status(int* site, int reset);
+
+/* Self-check of the bounded-wait path: launches one block that waits on a barrier nothing ever
+ * arrives at, with a limit of `limit_us` microseconds (1..2000000). The wait gives up, records
+ * QL_ERR_TIMEOUT in the device status word and the kernel returns normally. */
+int qlora_selftest_wait_timeout(int64_t limit_us, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * gguf_dequant — expand packed GGUF rows to fp32 or bf16.
+ * The pages' recipe runs a standalone GGUF dequant function (Show HN: LoRA over GGUF, "Other
+ * notes"); the layer's own kernels never call this: they expand blocks in shared memory.
+ *   qtype     QL_Q4_0 | QL_Q8_0 | QL_Q4_K
+ *   wq        [rows][cols/QK blocks] packed bytes
+ *   rows      > 0
+ *   cols      > 0, multiple of 256
+ *   out       [rows x cols] of out_dtype. fp32 output is the exact decode rounded once to fp32;
+ *             bf16 output is that fp32 value rounded to nearest-even bf16.
+ * ------------------------------------------------------------------------------------------- */
+int gguf_dequant(int qtype, const void* wq, int64_t rows, int64_t cols, void* out, int out_dtype,
+                 void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Dense layer (one projection). Shapes: X [M x K] bf16, W packed [N rows x K], A [r x K] bf16,
+ * B [N x r] bf16, dY [M x N] bf16. Rules: M >= 1; K % 256 == 0; N % 64 == 0; 1 <= r <= 64.
+ * ------------------------------------------------------------------------------------------- */
+
+/* Scratch bytes needed by qlora_linear_fwd / qlora_linear_bwd for these sizes. */
+size_t qlora_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
+
+/* Forward: Y = X deq(W)^T + scale (X A^T) B^T.
+ *   Y      [M x N] of y_dtype (QL_F32 or QL_BF16; bf16 is the fp32 result rounded once)
+ *   H      [M x r] fp32, receives X A^T (without scale) for the backward; required
+ *   Computes deq(W) tile by tile in shared memory; no full-precision weight is written to HBM. */
+int qlora_linear_fwd(int qtype, const void* wq, int64_t N, int64_t K, const void* X, int64_t M,
+                     const void* A, const void* B, int r, float scale, void* Y, int y_dtype, float* H,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/* Backward:
+ *   dX  [M x K] of dx_dtype, = dY deq(W) + G A with G = scale dY B; nullable (skips dX)
+ *   dA  [r x K] fp32, = G^T X (overwritten)
+ *   dB  [N x r] fp32, = scale dY^T H (overwritten)
+ *   H   [M x r] fp32 from the forward. */
+int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void* X, const void* dY,
+                     int64_t M, const void* A, const void* B, int r, float scale, const float* H,
+                     void* dX, int dx_dtype, float* dA, float* dB, void* ws, size_t ws_bytes,
+                     void* stream);
+
+#if defined(__GNUC__)
+#pragma GCC visibility pop
+#endif
+#ifdef __cplusplus
+}
+#endif
+#endif /* QLORA_H */

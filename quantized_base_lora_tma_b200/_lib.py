@@ -1,0 +1,132 @@
+"""ctypes binding of libqlora.so: the C ABI in include/qlora.h, same names, argument marshalling only.
+
+Tensors are torch tensors on the GPU (torch supplies device memory and streams); every number the
+layer computes comes from the library's kernels. If the library is not built, loading fails loudly:
+there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libqlora.so")
+
+Q4_0, Q8_0, Q4_K = 2, 8, 12
+QL_F32, QL_BF16 = 0, 1
+QL_OK = 0
+STATUS = {0: "QL_OK", 1: "QL_ERR_INVALID_ARG", 2: "QL_ERR_UNSUPPORTED", 3: "QL_ERR_SHAPE",
+          4: "QL_ERR_ALIGNMENT", 5: "QL_ERR_WORKSPACE", 6: "QL_ERR_CUDA", 7: "QL_ERR_TIMEOUT"}
+
+_c_i64 = ctypes.c_int64
+_c_vp = ctypes.c_void_p
+_c_int = ctypes.c_int
+_c_f = ctypes.c_float
+_c_sz = ctypes.c_size_t
+
+# name -> (restype, argtypes); must match include/qlora.h
+SIGNATURES = {
+    "qlora_status_string": (ctypes.c_char_p, [_c_int]),
+    "qlora_launch_count": (ctypes.c_uint64, []),
+    "qlora_device_status": (_c_int, [ctypes.POINTER(_c_int), _c_int]),
+    "qlora_selftest_wait_timeout": (_c_int, [_c_i64, _c_vp]),
+    "gguf_dequant": (_c_int, [_c_int, _c_vp, _c_i64, _c_i64, _c_vp, _c_int, _c_vp]),
+    "qlora_linear_workspace_bytes": (_c_sz, [_c_i64, _c_i64, _c_i64, _c_int]),
+    "qlora_linear_fwd": (_c_int, [_c_int, _c_vp, _c_i64, _c_i64, _c_vp, _c_i64, _c_vp, _c_vp, _c_int, _c_f,
+                                  _c_vp, _c_int, _c_vp, _c_vp, _c_sz, _c_vp]),
+    "qlora_linear_bwd": (_c_int, [_c_int, _c_vp, _c_i64, _c_i64, _c_vp, _c_vp, _c_i64, _c_vp, _c_vp, _c_int,
+                                  _c_f, _c_vp, _c_vp, _c_int, _c_vp, _c_vp, _c_vp, _c_sz, _c_vp]),
+}
+
+_lib = None
+
+
+class QloraError(RuntimeError):
+    def __init__(self, code: int, where: str = ""):
+        self.code = code
+        super().__init__(f"{where}: {STATUS.get(code, code)}")
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is not built; run `python -m quantized_base_lora_tma_b200.build`")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(l, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = l
+    return _lib
+
+
+def _p(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor arguments must be CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("tensor arguments must be contiguous")
+    return _c_vp(t.data_ptr())
+
+
+def _s(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return _c_vp(stream.cuda_stream)
+
+
+def _dt(t):
+    if t.dtype == torch.float32:
+        return QL_F32
+    if t.dtype == torch.bfloat16:
+        return QL_BF16
+    raise ValueError(f"unsupported output dtype {t.dtype}")
+
+
+def _check(rc, where):
+    if rc != QL_OK:
+        raise QloraError(rc, where)
+
+
+def qlora_status_string(code: int) -> str:
+    return lib().qlora_status_string(code).decode()
+
+
+def qlora_launch_count() -> int:
+    return int(lib().qlora_launch_count())
+
+
+def qlora_device_status(reset: bool = False):
+    site = _c_int(0)
+    rc = lib().qlora_device_status(ctypes.byref(site), 1 if reset else 0)
+    return rc, site.value
+
+
+def qlora_selftest_wait_timeout(limit_us: int, stream=None):
+    _check(lib().qlora_selftest_wait_timeout(limit_us, _s(stream)), "qlora_selftest_wait_timeout")
+
+
+def gguf_dequant(qtype, wq, rows, cols, out, stream=None):
+    _check(lib().gguf_dequant(qtype, _p(wq), rows, cols, _p(out), _dt(out), _s(stream)), "gguf_dequant")
+
+
+def qlora_linear_workspace_bytes(M, N, K, r) -> int:
+    return int(lib().qlora_linear_workspace_bytes(M, N, K, r))
+
+
+def qlora_linear_fwd(qtype, wq, N, K, X, A, B, r, scale, Y, H, ws, stream=None):
+    M = X.shape[0]
+    _check(lib().qlora_linear_fwd(qtype, _p(wq), N, K, _p(X), M, _p(A), _p(B), r, scale, _p(Y), _dt(Y), _p(H),
+                                  _p(ws), ws.numel() * ws.element_size(), _s(stream)), "qlora_linear_fwd")
+
+
+def qlora_linear_bwd(qtype, wq, N, K, X, dY, A, B, r, scale, H, dX, dA, dB, ws, stream=None):
+    M = X.shape[0]
+    dxt = _dt(dX) if dX is not None else QL_F32
+    _check(lib().qlora_linear_bwd(qtype, _p(wq), N, K, _p(X), _p(dY), M, _p(A), _p(B), r, scale, _p(H), _p(dX),
+                                  dxt, _p(dA), _p(dB), _p(ws), ws.numel() * ws.element_size(), _s(stream)),
+           "qlora_linear_bwd")

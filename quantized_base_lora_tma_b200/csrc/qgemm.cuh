@@ -1,0 +1,490 @@
+// Dequant-in-shared-memory tcgen05 GEMM: D[M, Nd] = A[M, Kd] * deq(W)^T-or-deq(W) (+ LoRA k-blocks).
+//
+// This is the base matmul of the layer ("MMQ and grouped MMQ like llama.cpp", Show HN: LoRA over
+// GGUF, "Things involved in the training"; the fused dequant-matmul that expands packed weights on
+// chip without an fp16 intermediate in memory, ai-manual.ru, "Fused dequant-matmul и MoE kernels").
+// It is designed for sm_100a rather than after those kernels:
+//
+//   * TMA copies packed GGUF groups (256 weights of a row, 272 or 144 bytes) of W into a shared
+//     memory ring; dequant warps expand them to bf16 directly in the 128-byte-swizzled canonical
+//     UMMA layout of the B operand; the full-precision weight never exists in HBM.
+//   * Forward (TRANS = false): B[n, k] = deq(W)[n, k], K-major, tile 128 x 128.
+//     Input-gradient (TRANS = true): B[k, n] = deq(W)[n, k] with the reduction over W's rows; the
+//     same decode writes an MN-major tile, tile 128 x 256.
+//   * The A operand (X or dY rows) arrives by TMA with the 128-byte swizzle.
+//   * One elected thread issues tcgen05.mma (bf16 x bf16 -> fp32) into a double-buffered TMEM
+//     accumulator; four epilogue warps drain it with tcgen05.ld while the next tile accumulates.
+//   * The rank-r adapter product is folded in as extra 64-wide k-blocks: A-side [hi(v) | lo(v)]
+//     (a bf16 pair whose sum carries v = s*H or G to ~2^-16 relative), B-side [Bop | Bop]; so the
+//     LoRA term is accumulated by the tensor core into the same TMEM tile, in fp32.
+//   * Grouped mode walks a device-side list of (expert, 128-row block) segments of a routed batch.
+//   * Persistent: one CTA per SM loops over tiles. Every wait is bounded (ptx.cuh).
+#pragma once
+#include <cuda_bf16.h>
+
+#include "decode.cuh"
+#include "ptx.cuh"
+
+namespace qlora {
+
+enum EpiKind { EPI_STORE = 0, EPI_SWIGLU = 1, EPI_PAIR_OUT = 2, EPI_SWIGLU_BWD = 3 };
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kNumEpiWarps = 4;   // warps 0..3 (TMEM lane quadrants 0..3)
+constexpr int kWarpTmaA = 4;
+constexpr int kWarpMma = 5;
+constexpr int kWarpTmaW = 6;
+constexpr int kWarpDq0 = 7;
+constexpr int kNumDqWarps = 8;
+constexpr int kGemmThreads = (kWarpDq0 + kNumDqWarps) * 32;  // 480
+
+struct GemmParams {
+  int M;           // rows of the A operand (tokens; routed pairs in grouped mode)
+  int Nd;          // output columns
+  int Kd;          // quantized reduction length
+  int n_lora_kb;   // extra 64-wide LoRA k-blocks
+  int num_n_tiles;
+  int num_m_blocks;  // dense mode: ceil(M / 128)
+  // weight rows
+  int w_rows_per_expert;  // rows of W per expert (grouped); 0 in dense mode
+  int lb_rows_per_expert; // rows of the LoRA B operand per expert (grouped)
+  int I;                  // SwiGLU: width of the gate (and up) half
+  // grouped
+  int E;                  // 0 = dense
+  const int* seg_off;     // [E+1] first pair row of each expert
+  const int* mblk_off;    // [E+1] prefix sum of ceil(count_e / 128)
+  // epilogue
+  void* out;
+  int out_dtype;
+  long ldo;
+  __nv_bfloat16* out_g;        // SWIGLU: g, u, h [M x I]; SWIGLU_BWD: d[g|u] [M x 2I] in out_g
+  __nv_bfloat16* out_u;
+  __nv_bfloat16* out_h;
+  const __nv_bfloat16* in_g;   // SWIGLU_BWD: saved g, u, h [M x I]
+  const __nv_bfloat16* in_u;
+  const __nv_bfloat16* in_h;
+  const float* row_w;          // PAIR_OUT, SWIGLU_BWD: routing weight per row
+  float* dw_part;              // SWIGLU_BWD: [M x num_n_tiles] partial <dh_u, h>
+};
+
+template <int QT, bool TRANS>
+struct GemmCfg {
+  static constexpr int BN = TRANS ? 256 : 128;
+  static constexpr int GB = QTraits<QT>::kGroupBytes;
+  static constexpr int A_BYTES = kBM * kBK * 2;              // 16 KB
+  static constexpr int B_BYTES = BN * kBK * 2;               // 16 / 32 KB
+  static constexpr int RAW_ROWS = TRANS ? 64 : 128;          // W rows per raw chunk
+  static constexpr int RAW_BYTES = RAW_ROWS * GB;
+  static constexpr int STAGES = TRANS ? 3 : 4;
+  static constexpr int RAW_SLOTS = TRANS ? (GB > 200 ? 4 : 6) : (GB > 200 ? 2 : 3);
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+  static constexpr int OFF_RAW = OFF_B + STAGES * B_BYTES;
+  static constexpr int OFF_BAR = OFF_RAW + RAW_SLOTS * RAW_BYTES;
+  // barriers: full[S], empty[S], raw_full[R], raw_empty[R], tfull[2], tempty[2], drain, tmem ptr
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * RAW_SLOTS + 5;
+  static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16 + 1024;  // + alignment slack
+  static constexpr int TMEM_COLS = 2 * BN;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(RAW_BYTES % 128 == 0, "raw slot alignment");
+};
+
+struct TileInfo {
+  int row0;     // first A row
+  int row_end;  // one past the last valid row
+  int nb;       // output column block
+  int e;        // expert (0 in dense mode)
+};
+
+__device__ __forceinline__ bool gemm_tile(const GemmParams& p, int t, TileInfo& ti) {
+  if (p.E == 0) {
+    if (t >= p.num_m_blocks * p.num_n_tiles) return false;
+    const int mb = t % p.num_m_blocks;
+    ti.nb = t / p.num_m_blocks;
+    ti.row0 = mb * kBM;
+    ti.row_end = p.M;
+    ti.e = 0;
+    return true;
+  }
+  const int total_mb = __ldg(p.mblk_off + p.E);
+  if (t >= total_mb * p.num_n_tiles) return false;
+  const int gm = t % total_mb;
+  ti.nb = t / total_mb;
+  // last expert e with mblk_off[e] <= gm
+  int lo = 0, hi = p.E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(p.mblk_off + mid) <= gm) lo = mid; else hi = mid - 1;
+  }
+  ti.e = lo;
+  ti.row0 = __ldg(p.seg_off + lo) + (gm - __ldg(p.mblk_off + lo)) * kBM;
+  ti.row_end = __ldg(p.seg_off + lo + 1);
+  return true;
+}
+
+// All 32 lanes wait; the outcome is made warp-uniform.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int site) {
+  const bool r = mbar_wait(bar, parity, site);
+  return __all_sync(0xffffffffu, r);
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
+
+template <int QT, bool TRANS, int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    qgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
+                 const __grid_constant__ CUtensorMap tmLA, const __grid_constant__ CUtensorMap tmLB,
+                 const GemmParams p) {
+  using C = GemmCfg<QT, TRANS>;
+  constexpr int BN = C::BN;
+  extern __shared__ uint8_t smem_raw_[];
+  const uint32_t base_u32 = (smem_u32(smem_raw_) + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw_ + (base_u32 - smem_u32(smem_raw_));
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const uint32_t sA = base_u32 + C::OFF_A;
+  const uint32_t sB = base_u32 + C::OFF_B;
+  const uint32_t sRaw = base_u32 + C::OFF_RAW;
+  const uint32_t bar0 = base_u32 + C::OFF_BAR;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
+  auto rfull_bar = [&](int s) { return bar0 + 8u * (2 * C::STAGES + s); };
+  auto rempty_bar = [&](int s) { return bar0 + 8u * (2 * C::STAGES + C::RAW_SLOTS + s); };
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 2 * C::RAW_SLOTS + b); };
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 2 * C::RAW_SLOTS + 2 + b); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * C::STAGES + 2 * C::RAW_SLOTS + 4);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + C::NUM_BARS * 8);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(full_bar(s), 1 + kNumDqWarps);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int s = 0; s < C::RAW_SLOTS; ++s) {
+      mbar_init(rfull_bar(s), 1);
+      mbar_init(rempty_bar(s), kNumDqWarps);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), kNumEpiWarps);
+    }
+    mbar_init(drain_bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == kWarpTmaA && lane == 0) {
+    prefetch_tmap(&tmA);
+    if (p.n_lora_kb) { prefetch_tmap(&tmLA); prefetch_tmap(&tmLB); }
+  }
+  if (warp == kWarpTmaW && lane == 0) prefetch_tmap(&tmW);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
+
+  const int kb_main = TRANS ? p.Kd / kBK : p.Kd / kBK;
+  const int kb_total = kb_main + p.n_lora_kb;
+  const int groups = p.Kd / 256;  // forward: raw chunks per tile
+
+  if (warp == kWarpTmaA) {
+    // ---------------- A operand (and LoRA operands) producer ----------------
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      int last_phase[8];
+      for (int s = 0; s < C::STAGES; ++s) last_phase[s] = -1;
+      TileInfo ti;
+      for (int t = blockIdx.x; ok && gemm_tile(p, t, ti); t += gridDim.x) {
+        for (int kb = 0; kb < kb_total; ++kb, ++it) {
+          const int s = it % C::STAGES;
+          const uint32_t ph = (it / C::STAGES) & 1;
+          if (!mbar_wait(empty_bar(s), ph ^ 1, 1)) { ok = false; break; }
+          if (kb < kb_main) {
+            mbar_arrive_expect_tx(full_bar(s), C::A_BYTES);
+            tma_load_2d(sA + s * C::A_BYTES, &tmA, full_bar(s), kb * kBK, ti.row0);
+          } else {
+            const int x = (kb - kb_main) * kBK;
+            mbar_arrive_expect_tx(full_bar(s), C::A_BYTES + C::B_BYTES);
+            tma_load_2d(sA + s * C::A_BYTES, &tmLA, full_bar(s), x, ti.row0);
+            const int lb0 = ti.e * p.lb_rows_per_expert;
+#pragma unroll
+            for (int i = 0; i < BN / 64; ++i) {
+              int y;
+              if (EPI == EPI_SWIGLU) y = lb0 + (i == 0 ? ti.nb * 64 : p.I + ti.nb * 64);
+              else y = lb0 + ti.nb * BN + 64 * i;
+              tma_load_2d(sB + s * C::B_BYTES + i * 64 * 128, &tmLB, full_bar(s), x, y);
+            }
+          }
+          last_phase[s] = (int)ph;
+        }
+      }
+      if (!ok) {  // let copies already issued land before the CTA can exit
+        for (int s = 0; s < C::STAGES; ++s)
+          if (last_phase[s] >= 0) mbar_wait(full_bar(s), (uint32_t)last_phase[s], 0, false, 2000000ull);
+      }
+    }
+  } else if (warp == kWarpTmaW) {
+    // ---------------- packed weight producer ----------------
+    if (lane == 0) {
+      int rc = 0;
+      bool ok = true;
+      int last_phase[8];
+      for (int s = 0; s < C::RAW_SLOTS; ++s) last_phase[s] = -1;
+      constexpr int GW = C::GB / 4;  // group width in 32-bit words
+      TileInfo ti;
+      for (int t = blockIdx.x; ok && gemm_tile(p, t, ti); t += gridDim.x) {
+        const int wbase = ti.e * p.w_rows_per_expert;
+        const int nchunks = TRANS ? kb_main : groups;
+        for (int c = 0; c < nchunks; ++c, ++rc) {
+          const int s = rc % C::RAW_SLOTS;
+          const uint32_t ph = (rc / C::RAW_SLOTS) & 1;
+          if (!mbar_wait(rempty_bar(s), ph ^ 1, 2)) { ok = false; break; }
+          mbar_arrive_expect_tx(rfull_bar(s), C::RAW_BYTES);
+          const uint32_t dst = sRaw + s * C::RAW_BYTES;
+          if (TRANS) {
+            tma_load_2d(dst, &tmW, rfull_bar(s), ti.nb * GW, wbase + c * 64);
+          } else {
+            int y0, y1;
+            if (EPI == EPI_SWIGLU) { y0 = wbase + ti.nb * 64; y1 = wbase + p.I + ti.nb * 64; }
+            else { y0 = wbase + ti.nb * 128; y1 = y0 + 64; }
+            tma_load_2d(dst, &tmW, rfull_bar(s), c * GW, y0);
+            tma_load_2d(dst + 64 * C::GB, &tmW, rfull_bar(s), c * GW, y1);
+          }
+          last_phase[s] = (int)ph;
+        }
+      }
+      if (!ok) {
+        for (int s = 0; s < C::RAW_SLOTS; ++s)
+          if (last_phase[s] >= 0) mbar_wait(rfull_bar(s), (uint32_t)last_phase[s], 0, false, 2000000ull);
+      }
+    }
+  } else if (warp == kWarpMma) {
+    // ---------------- tensor-core issuer ----------------
+    if (lane == 0) {
+      int it = 0, tc = 0;
+      bool ok = true;
+      bool issued = false;
+      TileInfo ti;
+      constexpr uint32_t idesc_main = idesc_bf16(kBM, BN, TRANS);
+      constexpr uint32_t idesc_kmaj = idesc_bf16(kBM, BN, false);
+      for (int t = blockIdx.x; ok && gemm_tile(p, t, ti); t += gridDim.x, ++tc) {
+        const int buf = tc & 1;
+        if (!mbar_wait(tempty_bar(buf), ((tc >> 1) & 1) ^ 1, 3)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * BN;
+        for (int kb = 0; kb < kb_total; ++kb, ++it) {
+          const int s = it % C::STAGES;
+          const uint32_t ph = (it / C::STAGES) & 1;
+          if (!mbar_wait(full_bar(s), ph, 4)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = sA + s * C::A_BYTES;
+          const uint32_t b0 = sB + s * C::B_BYTES;
+          const bool kmaj = !TRANS || kb >= kb_main;
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint64_t ad = smem_desc_sw128(a0 + 32 * k, 16, 1024);
+            uint64_t bd;
+            if (kmaj) bd = smem_desc_sw128(b0 + 32 * k, 16, 1024);
+            else bd = smem_desc_sw128(b0 + 8192 * k, 1024, 4096);
+            umma_bf16(d_tmem, ad, bd, kmaj ? idesc_kmaj : idesc_main, (kb | k) != 0);
+          }
+          umma_commit(empty_bar(s));
+          issued = true;
+        }
+        if (!ok) break;
+        umma_commit(tfull_bar(buf));
+      }
+      if (issued) {  // every MMA issued has completed before TMEM can be released
+        umma_commit(drain_bar);
+        mbar_wait(drain_bar, 0, 0, false, 2000000ull);
+      }
+    }
+  } else if (warp >= kWarpDq0) {
+    // ---------------- dequant workers ----------------
+    const int dq = threadIdx.x - kWarpDq0 * 32;  // 0..255
+    const int dw = warp - kWarpDq0;
+    int it = 0, rc = 0;
+    bool ok = true;
+    TileInfo ti;
+    for (int t = blockIdx.x; ok && gemm_tile(p, t, ti); t += gridDim.x) {
+      if (!TRANS) {
+        for (int g = 0; ok && g < groups; ++g, ++rc) {
+          const int rs = rc % C::RAW_SLOTS;
+          if (!warp_wait(rfull_bar(rs), (rc / C::RAW_SLOTS) & 1, 5)) { ok = false; break; }
+          const uint8_t* raw = smem + C::OFF_RAW + rs * C::RAW_BYTES;
+          for (int sub = 0; sub < 4; ++sub, ++it) {
+            const int s = it % C::STAGES;
+            if (!warp_wait(empty_bar(s), ((it / C::STAGES) & 1) ^ 1, 6)) { ok = false; break; }
+            uint8_t* sb = smem + C::OFF_B + s * C::B_BYTES;
+            const int c8 = dq & 7;
+            const int rb = dq >> 3;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int row = rb + 32 * i;
+              const uint4 v = decode8_bf16<QT>(raw + row * C::GB, 8 * sub + c8);
+              *reinterpret_cast<uint4*>(sb + row * 128 + ((c8 ^ (row & 7)) << 4)) = v;
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(full_bar(s));
+          }
+          __syncwarp();
+          if (ok && lane == 0) mbar_arrive(rempty_bar(rs));
+        }
+      } else {
+        for (int kb = 0; ok && kb < kb_main; ++kb, ++rc, ++it) {
+          const int rs = rc % C::RAW_SLOTS;
+          if (!warp_wait(rfull_bar(rs), (rc / C::RAW_SLOTS) & 1, 5)) { ok = false; break; }
+          const int s = it % C::STAGES;
+          if (!warp_wait(empty_bar(s), ((it / C::STAGES) & 1) ^ 1, 6)) { ok = false; break; }
+          const uint8_t* raw = smem + C::OFF_RAW + rs * C::RAW_BYTES;
+          uint8_t* sb = smem + C::OFF_B + s * C::B_BYTES;
+          const int gc = lane;
+#pragma unroll 4
+          for (int i = 0; i < 8; ++i) {
+            const int kk = dw + 8 * i;
+            const uint4 v = decode8_bf16<QT>(raw + kk * C::GB, gc);
+            const int off = (kk >> 3) * 4096 + (gc >> 3) * 1024 + (kk & 7) * 128 + (((gc & 7) ^ (kk & 7)) << 4);
+            *reinterpret_cast<uint4*>(sb + off) = v;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(full_bar(s));
+            mbar_arrive(rempty_bar(rs));
+          }
+        }
+      }
+      // LoRA k-blocks: operands come by TMA; the workers only account for their share.
+      for (int kb = kb_main; ok && kb < kb_total; ++kb, ++it) {
+        const int s = it % C::STAGES;
+        if (!warp_wait(empty_bar(s), ((it / C::STAGES) & 1) ^ 1, 7)) { ok = false; break; }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(full_bar(s));
+      }
+    }
+  } else if (warp < kNumEpiWarps) {
+    // ---------------- epilogue ----------------
+    int tc = 0;
+    TileInfo ti;
+    for (int t = blockIdx.x; gemm_tile(p, t, ti); t += gridDim.x, ++tc) {
+      const int buf = tc & 1;
+      if (!warp_wait(tfull_bar(buf), (tc >> 1) & 1, 8)) break;
+      tc_fence_after();
+      const int row = ti.row0 + warp * 32 + lane;
+      const bool valid = row < ti.row_end;
+      const uint32_t tbase = tmem_base + ((uint32_t)(warp * 32) << 16) + buf * BN;
+      if (EPI == EPI_STORE || EPI == EPI_PAIR_OUT) {
+        float wr = 1.0f;
+        if (EPI == EPI_PAIR_OUT && valid) wr = __ldg(p.row_w + row);
+#pragma unroll 1
+        for (int jc = 0; jc < BN / 32; ++jc) {
+          uint32_t v[32];
+          tmem_ld32(tbase + 32 * jc, v);
+          tmem_ld_wait();
+          const int col0 = ti.nb * BN + 32 * jc;
+          if (valid && col0 < p.Nd) {
+            if (p.out_dtype == QL_F32 && EPI == EPI_STORE) {
+              float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (long)row * p.ldo + col0);
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                o[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                   __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+            } else {
+              uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + (long)row * p.ldo + col0);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                float f[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) f[j] = wr * __uint_as_float(v[8 * i + j]);
+                o[i] = pack_bf16x8(f);
+              }
+            }
+          }
+        }
+      } else if (EPI == EPI_SWIGLU) {
+        // columns [0,64) of the tile are gate j = nb*64 + c, [64,128) are up for the same j
+#pragma unroll 1
+        for (int jp = 0; jp < 2; ++jp) {
+          uint32_t vg[32], vu[32];
+          tmem_ld32(tbase + 32 * jp, vg);
+          tmem_ld32(tbase + 64 + 32 * jp, vu);
+          tmem_ld_wait();
+          const int j0 = ti.nb * 64 + 32 * jp;
+          if (valid && j0 < p.I) {
+            const long o = (long)row * p.I + j0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              float g[8], u[8], h[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                g[j] = __uint_as_float(vg[8 * i + j]);
+                u[j] = __uint_as_float(vu[8 * i + j]);
+                h[j] = silu_f(g[j]) * u[j];
+              }
+              *reinterpret_cast<uint4*>(p.out_g + o + 8 * i) = pack_bf16x8(g);
+              *reinterpret_cast<uint4*>(p.out_u + o + 8 * i) = pack_bf16x8(u);
+              *reinterpret_cast<uint4*>(p.out_h + o + 8 * i) = pack_bf16x8(h);
+            }
+          }
+        }
+      } else if (EPI == EPI_SWIGLU_BWD) {
+        float wr = 0.0f, dwp = 0.0f;
+        if (valid) wr = __ldg(p.row_w + row);
+#pragma unroll 1
+        for (int jc = 0; jc < BN / 32; ++jc) {
+          uint32_t v[32];
+          tmem_ld32(tbase + 32 * jc, v);
+          tmem_ld_wait();
+          const int j0 = ti.nb * BN + 32 * jc;
+          if (valid && j0 < p.I) {
+            const long o = (long)row * p.I + j0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint4 gq = *reinterpret_cast<const uint4*>(p.in_g + o + 8 * i);
+              const uint4 uq = *reinterpret_cast<const uint4*>(p.in_u + o + 8 * i);
+              const uint4 hq = *reinterpret_cast<const uint4*>(p.in_h + o + 8 * i);
+              const __nv_bfloat16* gb = reinterpret_cast<const __nv_bfloat16*>(&gq);
+              const __nv_bfloat16* ub = reinterpret_cast<const __nv_bfloat16*>(&uq);
+              const __nv_bfloat16* hb = reinterpret_cast<const __nv_bfloat16*>(&hq);
+              float dg[8], du[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const float a = __uint_as_float(v[8 * i + j]);
+                const float g = __bfloat162float(gb[j]);
+                const float u = __bfloat162float(ub[j]);
+                dwp = fmaf(a, __bfloat162float(hb[j]), dwp);
+                const float dh = wr * a;
+                const float sg = 1.0f / (1.0f + expf(-g));
+                dg[j] = dh * u * sg * (1.0f + g * (1.0f - sg));
+                du[j] = dh * g * sg;
+              }
+              const long od = (long)row * 2 * p.I + j0 + 8 * i;
+              *reinterpret_cast<uint4*>(p.out_g + od) = pack_bf16x8(dg);
+              *reinterpret_cast<uint4*>(p.out_g + od + p.I) = pack_bf16x8(du);
+            }
+          }
+        }
+        if (valid) p.dw_part[(long)row * p.num_n_tiles + ti.nb] = dwp;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(buf));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace qlora

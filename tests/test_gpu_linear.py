@@ -1,0 +1,160 @@
+"""GPU parity: gguf_dequant and the dense layer (forward + backward) through the C ABI, against the
+oracle on the same seeded inputs."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import gguf_blocks as gb
+from oracle import lora_linear as ll
+from quantized_base_lora_tma_b200 import inputs as inp
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import quantized_base_lora_tma_b200 as ql
+    from tests.gpu_util import assert_close, bf16_f64, dev_bf16, dev_u8, f64
+
+
+@pytest.fixture(autouse=True)
+def _reset_status():
+    ql.qlora_device_status(reset=True)
+    yield
+    rc, site = ql.qlora_device_status(reset=True)
+    assert rc == 0, f"device status {rc} at site {site}"
+
+
+def _random_packed(qtype, rows, cols, rng):
+    w = (rng.standard_normal((rows, cols)) * 0.02).astype(np.float32)
+    raw = inp.pack(qtype, w)
+    if qtype != inp.Q4_K:  # sprinkle subnormal and zero scales
+        bb = inp.BLOCK_BYTES[qtype]
+        v = raw.reshape(-1, bb)
+        v[::5, 0:2] = np.frombuffer(np.float16(3.0e-6).tobytes(), np.uint8)
+        v[::13, 0:2] = 0
+    return raw
+
+
+@pytest.mark.parametrize("qtype", [inp.Q4_0, inp.Q8_0, inp.Q4_K])
+def test_dequant_bit_exact(qtype):
+    rng = np.random.default_rng(qtype)
+    rows, cols = 37, 768
+    raw = _random_packed(qtype, rows, cols, rng)
+    wq = dev_u8(raw)
+    for dt, ref in [(torch.float32, gb.deq_f32(qtype, raw, rows, cols)),
+                    (torch.bfloat16, gb.deq_bf16(qtype, raw, rows, cols))]:
+        out = torch.empty(rows, cols, dtype=dt, device="cuda")
+        ql.gguf_dequant(qtype, wq, rows, cols, out)
+        torch.cuda.synchronize()
+        got = f64(out)
+        assert np.array_equal(got, ref), f"{dt}: {np.sum(got != ref)} mismatches"
+
+
+def run_linear(c, y_dtype=torch.float32, dx_dtype=torch.float32, with_dx=True):
+    X, dY, A, B = dev_bf16(c.X), dev_bf16(c.dY), dev_bf16(c.A), dev_bf16(c.B)
+    wq = dev_u8(c.wq)
+    M, N, K, r = c.M, c.N, c.K, c.r
+    ws = torch.empty(ql.qlora_linear_workspace_bytes(M, N, K, r), dtype=torch.uint8, device="cuda")
+    Y = torch.full((M, N), float("nan"), dtype=y_dtype, device="cuda")
+    H = torch.empty(M, r, dtype=torch.float32, device="cuda")
+    ql.qlora_linear_fwd(c.qtype, wq, N, K, X, A, B, r, c.scale, Y, H, ws)
+    dX = torch.full((M, K), float("nan"), dtype=dx_dtype, device="cuda") if with_dx else None
+    dA = torch.empty(r, K, dtype=torch.float32, device="cuda")
+    dB = torch.empty(N, r, dtype=torch.float32, device="cuda")
+    ql.qlora_linear_bwd(c.qtype, wq, N, K, X, dY, A, B, r, c.scale, H, dX, dA, dB, ws)
+    torch.cuda.synchronize()
+    return Y, H, dX, dA, dB
+
+
+def oracle_linear(c, rows=None):
+    W = ll.weights(c.qtype, c.wq, c.N, c.K)
+    X, dY, A, B = bf16_f64(c.X), bf16_f64(c.dY), bf16_f64(c.A), bf16_f64(c.B)
+    H = X @ A.T
+    dX_rows = None
+    if rows is None:
+        Y, _ = ll.linear_fwd(W, X, A, B, c.scale)
+        dX, dA, dB, _ = ll.linear_bwd(W, X, dY, A, B, c.scale, H)
+        return Y, H, dX, dA, dB
+    Y, _ = ll.linear_fwd(W, X[rows], A, B, c.scale)
+    dX, _, _, _ = ll.linear_bwd(W, X[rows], dY[rows], A, B, c.scale, H[rows])
+    G = c.scale * (dY @ B)
+    dA = G.T @ X
+    dB = c.scale * (dY.T @ H)
+    return Y, H, dX, dA, dB
+
+
+SMALL = [
+    # (M, K, N, r): several tiles in every dimension and ragged tails
+    (300, 512, 384, 4),
+    (129, 768, 320, 16),
+    (1, 256, 64, 1),
+    (200, 256, 448, 40),   # r > 32: two LoRA k-blocks
+    (64, 1024, 128, 64),
+]
+
+
+@pytest.mark.parametrize("qtype", [inp.Q4_0, inp.Q8_0, inp.Q4_K])
+@pytest.mark.parametrize("shape", SMALL)
+def test_linear_parity_small(qtype, shape):
+    M, K, N, r = shape
+    c = inp.linear_case(M, K, N, qtype, r, 2.0 * r, seed=M + K + N + r)
+    Y, H, dX, dA, dB = run_linear(c)
+    Yr, Hr, dXr, dAr, dBr = oracle_linear(c)
+    for got, ref, name in [(Y, Yr, "Y"), (H, Hr, "H"), (dX, dXr, "dX"), (dA, dAr, "dA"), (dB, dBr, "dB")]:
+        assert_close(f64(got), ref, name)
+
+
+def test_linear_q4_0_64x256x512_bf16_outputs():
+    c = inp.q4_0_linear_64x256x512()
+    Y, H, dX, dA, dB = run_linear(c, torch.bfloat16, torch.bfloat16)
+    Yr, Hr, dXr, dAr, dBr = oracle_linear(c)
+    assert_close(f64(Y), Yr, "Y", bf16_out=True)
+    assert_close(f64(dX), dXr, "dX", bf16_out=True)
+    assert_close(f64(dA), dAr, "dA")
+    assert_close(f64(dB), dBr, "dB")
+
+
+def test_linear_b_zero_gives_exact_zero_dA():
+    c = inp.linear_case(130, 512, 256, inp.Q8_0, 8, 16.0, seed=3)
+    c.B[:] = 0
+    Y, H, dX, dA, dB = run_linear(c)
+    assert torch.count_nonzero(dA).item() == 0
+    Yr, Hr, dXr, dAr, dBr = oracle_linear(c)
+    assert_close(f64(Y), Yr, "Y")
+    assert_close(f64(dB), dBr, "dB")
+
+
+def test_linear_deterministic():
+    c = inp.linear_case(257, 512, 256, inp.Q4_K, 8, 16.0, seed=9)
+    a = [t.clone() for t in run_linear(c)]
+    b = run_linear(c)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+@pytest.mark.parametrize("name", ["dense_q8_0", "dense_q4_0", "gate_up_q4_k"])
+def test_linear_full_size_sampled(name):
+    """The benchmark's shapes and launch configuration: sampled rows of Y and dX, full dA and dB."""
+    c = {"dense_q8_0": lambda: inp.dense_proj_2048x4096x4096(inp.Q8_0),
+         "dense_q4_0": lambda: inp.dense_proj_2048x4096x4096(inp.Q4_0),
+         "gate_up_q4_k": inp.gate_up_q4_k_2048x2048x12288}[name]()
+    Y, H, dX, dA, dB = run_linear(c)
+    rows = np.sort(np.random.default_rng(1).choice(c.M, size=24, replace=False))
+    rows[0], rows[-1] = 0, c.M - 1
+    Yr, Hr, dXr, dAr, dBr = oracle_linear(c, rows)
+    assert_close(f64(Y)[rows], Yr, "Y")
+    assert_close(f64(H), Hr, "H")
+    assert_close(f64(dX)[rows], dXr, "dX")
+    assert_close(f64(dA), dAr, "dA")
+    assert_close(f64(dB), dBr, "dB")
+
+
+def test_bounded_wait_self_check():
+    ql.qlora_device_status(reset=True)
+    ql.qlora_selftest_wait_timeout(20000)
+    rc, site = ql.qlora_device_status(reset=True)
+    assert rc == 7 and site == 99
+    # the context is still usable
+    c = inp.linear_case(64, 256, 128, inp.Q4_0, 4, 8.0, seed=1)
+    Y, *_ = run_linear(c)
+    Yr, *_ = oracle_linear(c)
+    assert_close(f64(Y), Yr, "Y")
