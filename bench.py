@@ -1,0 +1,436 @@
+"""Benchmark of the frozen-GGUF-base + LoRA layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step is one forward + backward of the layer on one batch: for the default workload the
+2048-token dense projection K = N = 4096 with a Q8_0 base and a rank-16 adapter (alpha 32):
+H = X A^T, Y = X deq(W)^T + s H B^T, then G = s dY B, dX = dY deq(W) + G A, dA = G^T X,
+dB = s dY^T H. Inputs are seeded synthetic tensors of that shape (X, dY ~ N(0,1); W ~ N(0, 0.02)
+packed once; A ~ N(0, 1/K); B ~ N(0, 0.01)).
+
+Timing: W untimed warm-up steps, then K steps each bracketed by CUDA events on the launch stream;
+the L2 cache is flushed (a 256 MiB write) between steps, outside the events. With N > 1 each rank
+runs its own batch (weak scaling) and the adapter gradients are summed across ranks with one NCCL
+all-reduce per step (the data-parallel exchange); the step time is the max over ranks.
+
+The JSON line also carries: the dominant kernel's roofline (its algorithmic FLOPs over its
+event-timed duration against the measured bf16 peak), the end-to-end number through the public
+API with host buffers, the CPU oracle timed on a sample of the same workload, the count of the
+library's own kernel launches and the SM clocks sampled during the timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from quantized_base_lora_tma_b200 import inputs as inp  # noqa: E402
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "quantized-LoRA fwd+bwd tokens/s and TFLOP/s (% bf16 peak); small-M weight GB/s"
+
+WORKLOADS = {
+    "dense_q8_0": ("dense_proj_q8_0_2048x4096x4096_r16", lambda seed: inp.dense_proj_2048x4096x4096(inp.Q8_0, seed)),
+    "dense_q4_0": ("dense_proj_q4_0_2048x4096x4096_r16", lambda seed: inp.dense_proj_2048x4096x4096(inp.Q4_0, seed)),
+    "gate_up_q4_k": ("gate_up_q4_k_2048x2048x12288_r8", lambda seed: inp.gate_up_q4_k_2048x2048x12288(seed)),
+}
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "quantized_base_lora_tma_b200", "csrc")
+    for fn in sorted(os.listdir(d)):
+        with open(os.path.join(d, fn), "rb") as f:
+            h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d[workload][kernel]
+        if e.get("source_hash") == kernel_source_hash():
+            return float(e["dram_bytes"])
+    except Exception:
+        pass
+    return None
+
+
+# ------------------------------------------------------------------------------------------------
+# clocks
+# ------------------------------------------------------------------------------------------------
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML every `period` seconds while running."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80,
+    }
+
+    def __init__(self, device_index: int, period: float = 0.01):
+        self.period = period
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            pass
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------------------------
+# our implementation
+# ------------------------------------------------------------------------------------------------
+def bf16_dev(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+class DenseLayerRun:
+    """Device buffers and one fwd+bwd step of the dense layer through the C ABI."""
+
+    def __init__(self, case):
+        import quantized_base_lora_tma_b200 as ql
+        self.ql = ql
+        self.c = c = case
+        self.X = bf16_dev(c.X)
+        self.dY = bf16_dev(c.dY)
+        self.A = bf16_dev(c.A)
+        self.B = bf16_dev(c.B)
+        self.wq = torch.from_numpy(c.wq).cuda()
+        M, N, K, r = c.M, c.N, c.K, c.r
+        self.ws = torch.empty(ql.qlora_linear_workspace_bytes(M, N, K, r), dtype=torch.uint8, device="cuda")
+        self.Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        self.H = torch.empty(M, r, dtype=torch.float32, device="cuda")
+        self.dX = torch.empty(M, K, dtype=torch.bfloat16, device="cuda")
+        self.dA = torch.empty(r, K, dtype=torch.float32, device="cuda")
+        self.dB = torch.empty(N, r, dtype=torch.float32, device="cuda")
+
+    def step(self, X=None, dY=None):
+        c, ql = self.c, self.ql
+        X = self.X if X is None else X
+        dY = self.dY if dY is None else dY
+        ql.qlora_linear_fwd(c.qtype, self.wq, c.N, c.K, X, self.A, self.B, c.r, c.scale, self.Y, self.H, self.ws)
+        ql.qlora_linear_bwd(c.qtype, self.wq, c.N, c.K, X, dY, self.A, self.B, c.r, c.scale, self.H, self.dX,
+                            self.dA, self.dB, self.ws)
+
+    def flops(self):
+        c = self.c
+        base = 2 * 2.0 * c.M * c.N * c.K           # forward and input-gradient GEMMs (W is frozen)
+        lora = 6.0 * c.r * (c.K + c.N) * c.M
+        return base + lora
+
+    def gemm_flops(self, slot):
+        c = self.c
+        return 2.0 * c.M * c.N * c.K + 2.0 * c.M * c.r * (c.N if slot == 0 else c.K)
+
+
+def run_ours(args, rank, world, local_rank):
+    import quantized_base_lora_tma_b200 as ql
+    from quantized_base_lora_tma_b200 import build
+    build.build()
+    torch.cuda.set_device(local_rank)
+    wl_name, make = WORKLOADS[args.workload]
+    # weights identical on every rank (replicated frozen base); tokens differ per rank
+    case = make(0)
+    if rank != 0:
+        rng = np.random.default_rng(1000 + rank)
+        case.X = inp.to_bf16_bits(rng.standard_normal(case.X.shape, dtype=np.float32))
+        case.dY = inp.to_bf16_bits(rng.standard_normal(case.dY.shape, dtype=np.float32))
+    run = DenseLayerRun(case)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    ql.qlora_device_status(reset=True)
+
+    def allreduce_grads():
+        if world > 1:
+            torch.distributed.all_reduce(run.dA)
+            torch.distributed.all_reduce(run.dB)
+
+    for _ in range(args.warmup):
+        run.step()
+        allreduce_grads()
+    torch.cuda.synchronize()
+
+    # --- device-timed steps with per-kernel events for the two tensor-core GEMMs ---
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    gev = {s: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+           for s in (0, 1)}
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    launches0 = ql.qlora_launch_count()
+    sampler = ClockSampler(local_rank)
+    wall0 = time.perf_counter()
+    with sampler:
+        for i in range(K):
+            flush.zero_()
+            for s in (0, 1):
+                ql.qlora_set_kernel_events(s, gev[s][i][0], gev[s][i][1])
+            ev[i][0].record(stream)
+            run.step()
+            allreduce_grads()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    launches = ql.qlora_launch_count() - launches0
+    for s in (0, 1):
+        ql.qlora_set_kernel_events(s, None, None)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    st, site = ql.qlora_device_status(reset=True)
+    if st != 0:
+        raise RuntimeError(f"device status {st} at site {site}")
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    gemm_ms = {s: [a.elapsed_time(b) for a, b in gev[s]] for s in (0, 1)}
+    ms = statistics.mean(step_ms)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # --- end to end through the public API with host buffers ---
+    E = max(3, min(K, 50))
+    X_h = torch.from_numpy(np.ascontiguousarray(case.X).view(np.int16)).view(torch.bfloat16).pin_memory()
+    dY_h = torch.from_numpy(np.ascontiguousarray(case.dY).view(np.int16)).view(torch.bfloat16).pin_memory()
+    dA_h = torch.empty(run.dA.shape, dtype=torch.float32).pin_memory()
+    dB_h = torch.empty(run.dB.shape, dtype=torch.float32).pin_memory()
+    Xd = torch.empty_like(run.X)
+    dYd = torch.empty_like(run.dY)
+    e2e_ms = []
+    for i in range(E + 2):
+        flush.zero_()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        Xd.copy_(X_h, non_blocking=True)
+        dYd.copy_(dY_h, non_blocking=True)
+        run.step(Xd, dYd)
+        allreduce_grads()
+        dA_h.copy_(run.dA, non_blocking=True)
+        dB_h.copy_(run.dB, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= 2:
+            e2e_ms.append(a.elapsed_time(b))
+    e2e = statistics.mean(e2e_ms)
+    if world > 1:
+        t = torch.tensor([e2e], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e = float(t.item())
+
+    c = case
+    tokens = c.M * world
+    value = tokens / (ms / 1e3)
+    pk, pk_kind = peaks()
+    # dominant kernel: the tensor-core GEMM with the larger share of the step
+    g_mean = {s: statistics.mean(gemm_ms[s]) for s in (0, 1)}
+    dom = max(g_mean, key=g_mean.get)
+    dom_name = {0: "qgemm_fwd (dequant-in-SMEM tcgen05 GEMM, K-major)",
+                1: "qgemm_dx (dequant-in-SMEM tcgen05 GEMM, MN-major)"}[dom]
+    achieved = run.gemm_flops(dom) / (g_mean[dom] / 1e3) / 1e12
+    step_tflops = run.flops() / (ms / 1e3) / 1e12
+    traffic = profiled_traffic(args.workload, "qgemm_fwd" if dom == 0 else "qgemm_dx")
+    out = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) weights packed once to GGUF)",
+        "config": {"workload": wl_name, "tokens_per_gpu": c.M, "K": c.K, "N": c.N, "qtype": inp.QTYPE_NAMES[c.qtype],
+                   "rank": c.r, "alpha": c.alpha, "global_batch_tokens": tokens,
+                   "parallelism": f"dp{world}" if world > 1 else "single",
+                   "l2": "flushed between steps (256 MiB write outside the timed events)"},
+        "tflops": step_tflops,
+        "frac_of_bf16_peak": step_tflops / pk["bf16_tflops"],
+        "roofline": {"kernel": dom_name, "bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"], "traffic": traffic,
+                     "peak_kind": f"{pk_kind} burst bf16 (cuBLAS)",
+                     "kernel_ms": {"qgemm_fwd": g_mean[0], "qgemm_dx": g_mean[1]}},
+        "e2e": {"value": tokens / (e2e / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(run.X.numel() * 2 + run.dY.numel() * 2),
+                "d2h_bytes_per_step": int((run.dA.numel() + run.dB.numel()) * 4),
+                "ms_per_step": e2e},
+        "gpu_launches": int(launches),
+        "clocks": sampler.summary(),
+        "wall_s_timed_region": wall,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(case, target_s=args.cpu_seconds)
+    return out
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle (baseline leg and the reference arm)
+# ------------------------------------------------------------------------------------------------
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_step(case, rows):
+    """The oracle's forward + backward restricted to a sample of token rows (dA, dB over those rows)."""
+    from oracle import gguf_blocks as gb
+    from oracle import lora_linear as ll
+    W = ll.weights(case.qtype, case.wq, case.N, case.K)
+    X = gb.bf16_bits_to_f64(case.X[rows])
+    dY = gb.bf16_bits_to_f64(case.dY[rows])
+    A = gb.bf16_bits_to_f64(case.A)
+    B = gb.bf16_bits_to_f64(case.B)
+    Y, H = ll.linear_fwd(W, X, A, B, case.scale)
+    return ll.linear_bwd(W, X, dY, A, B, case.scale, H)
+
+
+def cpu_baseline(case, target_s=15.0, max_rows=None):
+    rows_total = case.M
+    n = 64
+    t0 = time.perf_counter()
+    oracle_step(case, np.arange(n))
+    t1 = time.perf_counter() - t0
+    n = int(min(rows_total if max_rows is None else max_rows, max(64, n * target_s / max(t1, 1e-3))))
+    t0 = time.perf_counter()
+    oracle_step(case, np.arange(n))
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"fp64 numpy oracle fwd+bwd on the first {n} of {rows_total} token rows "
+                      f"(weights decoded once per call), {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    wl_name, make = WORKLOADS[args.workload]
+    case = make(0)
+    cores = _blas_threads()
+    n = max(32, int(args.ref_rows))
+    for _ in range(args.warmup):
+        oracle_step(case, np.arange(n))
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle_step(case, np.arange(n))
+        times.append(time.perf_counter() - t0)
+    ms = statistics.mean(times) * 1e3
+    value = n / (ms / 1e3)
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl_name, "tokens_per_step_sample": n},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"fp64 numpy oracle fwd+bwd on {n} token rows per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="dense_q8_0", choices=sorted(WORKLOADS))
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-rows", type=int, default=128)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        out = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

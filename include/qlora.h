@@ -64,6 +64,14 @@ const char* qlora_status_string(int status);
 /* Number of the library's own kernel launches since load (all entry points, all streams). */
 uint64_t qlora_launch_count(void);
 
+/* Timing hook: when set, the library records `start` / `stop` (cudaEvent_t, as void*) on the
+ * launch stream right before / after every launch of the tensor-core GEMM kernel of a slot:
+ * 0 = dense forward GEMM, 1 = dense input-gradient GEMM, 2 = MoE gate/up GEMM, 3 = MoE down GEMM,
+ * 4 = MoE down input-gradient GEMM, 5 = MoE gate/up input-gradient GEMM. Both NULL clears the slot.
+ * The caller owns the events; they must outlive every launch made while they are set. Not
+ * thread-safe with concurrent calls that launch into the same slot. */
+int qlora_set_kernel_events(int slot, void* start, void* stop);
+
 /* Reads the device status word of the current device (synchronises the device first). Returns
  * QL_OK or the first recorded device-side error (QL_ERR_TIMEOUT); *site (nullable) receives the
  * code of the wait that gave up. reset != 0 clears the word afterwards. */

@@ -1,10 +1,10 @@
 """Frozen GGUF-quantized base + LoRA layer for NVIDIA B200 (sm_100a).
 
 The kernels live in ``libqlora.so`` (built from ``csrc/`` by ``build.py``) behind the C ABI of
-``include/qlora.h``; ``_lib`` binds that ABI with the same names. ``layer`` adds the buffer
-bookkeeping a training loop needs (outputs and workspace as torch tensors). ``inputs`` holds the
-seeded synthetic workloads and the offline GGUF packers.
+``include/qlora.h``; ``_lib`` binds that ABI with the same names (torch tensors in, argument
+marshalling only). ``inputs`` holds the seeded synthetic workloads and the offline GGUF packers.
 """
 from ._lib import (Q4_0, Q4_K, Q8_0, QL_BF16, QL_F32, QloraError, gguf_dequant, lib,  # noqa: F401
                    qlora_device_status, qlora_launch_count, qlora_linear_bwd, qlora_linear_fwd,
-                   qlora_linear_workspace_bytes, qlora_selftest_wait_timeout, qlora_status_string)
+                   qlora_linear_workspace_bytes, qlora_selftest_wait_timeout, qlora_set_kernel_events,
+                   qlora_status_string)

@@ -31,6 +31,7 @@ SIGNATURES = {
     "qlora_status_string": (ctypes.c_char_p, [_c_int]),
     "qlora_launch_count": (ctypes.c_uint64, []),
     "qlora_device_status": (_c_int, [ctypes.POINTER(_c_int), _c_int]),
+    "qlora_set_kernel_events": (_c_int, [_c_int, _c_vp, _c_vp]),
     "qlora_selftest_wait_timeout": (_c_int, [_c_i64, _c_vp]),
     "gguf_dequant": (_c_int, [_c_int, _c_vp, _c_i64, _c_i64, _c_vp, _c_int, _c_vp]),
     "qlora_linear_workspace_bytes": (_c_sz, [_c_i64, _c_i64, _c_i64, _c_int]),
@@ -104,6 +105,17 @@ def qlora_device_status(reset: bool = False):
     site = _c_int(0)
     rc = lib().qlora_device_status(ctypes.byref(site), 1 if reset else 0)
     return rc, site.value
+
+
+def qlora_set_kernel_events(slot: int, start=None, stop=None):
+    """start / stop: torch.cuda.Event (created with enable_timing=True) or None to clear."""
+    def h(e):
+        if e is None:
+            return None
+        if e.cuda_event == 0:          # torch creates the event lazily
+            e.record()
+        return _c_vp(e.cuda_event)
+    _check(lib().qlora_set_kernel_events(slot, h(start), h(stop)), "qlora_set_kernel_events")
 
 
 def qlora_selftest_wait_timeout(limit_us: int, stream=None):

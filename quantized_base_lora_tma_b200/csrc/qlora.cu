@@ -15,6 +15,15 @@ namespace qlora {
 
 static std::atomic<uint64_t> g_launches{0};
 
+// Optional timing events recorded around the tensor-core GEMM launches (slot 0: forward GEMM,
+// 1: input-gradient GEMM, 2..5: grouped GEMMs of the MoE layer), on the launch stream.
+constexpr int kEventSlots = 8;
+static cudaEvent_t g_ev[kEventSlots][2] = {};
+
+static void ev_record(int slot, int which, cudaStream_t st) {
+  if (slot >= 0 && slot < kEventSlots && g_ev[slot][which]) cudaEventRecord(g_ev[slot][which], st);
+}
+
 // ------------------------------------------------------------------------------------------------
 // Driver entry point for tensor-map encoding (no link-time dependency on libcuda).
 // ------------------------------------------------------------------------------------------------
@@ -94,23 +103,25 @@ static inline int launch_status() {
 // ------------------------------------------------------------------------------------------------
 template <int QT, bool TRANS, int EPI>
 static int launch_qgemm(const CUtensorMap& tA, const CUtensorMap& tW, const CUtensorMap& tLA, const CUtensorMap& tLB,
-                        const GemmParams& p, int grid, cudaStream_t st) {
+                        const GemmParams& p, int grid, cudaStream_t st, int slot) {
   using C = GemmCfg<QT, TRANS>;
   auto k = qgemm_kernel<QT, TRANS, EPI>;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return QL_ERR_CUDA;
+  ev_record(slot, 0, st);
   k<<<grid, kGemmThreads, C::SMEM_BYTES, st>>>(tA, tW, tLA, tLB, p);
   g_launches.fetch_add(1, std::memory_order_relaxed);
+  ev_record(slot, 1, st);
   return launch_status();
 }
 
 template <bool TRANS, int EPI>
 static int launch_qgemm_q(int qtype, const CUtensorMap& tA, const CUtensorMap& tW, const CUtensorMap& tLA,
-                          const CUtensorMap& tLB, const GemmParams& p, int grid, cudaStream_t st) {
+                          const CUtensorMap& tLB, const GemmParams& p, int grid, cudaStream_t st, int slot) {
   switch (qtype) {
-    case QL_Q8_0: return launch_qgemm<QL_Q8_0, TRANS, EPI>(tA, tW, tLA, tLB, p, grid, st);
-    case QL_Q4_0: return launch_qgemm<QL_Q4_0, TRANS, EPI>(tA, tW, tLA, tLB, p, grid, st);
-    case QL_Q4_K: return launch_qgemm<QL_Q4_K, TRANS, EPI>(tA, tW, tLA, tLB, p, grid, st);
+    case QL_Q8_0: return launch_qgemm<QL_Q8_0, TRANS, EPI>(tA, tW, tLA, tLB, p, grid, st, slot);
+    case QL_Q4_0: return launch_qgemm<QL_Q4_0, TRANS, EPI>(tA, tW, tLA, tLB, p, grid, st, slot);
+    case QL_Q4_K: return launch_qgemm<QL_Q4_K, TRANS, EPI>(tA, tW, tLA, tLB, p, grid, st, slot);
     default: return QL_ERR_UNSUPPORTED;
   }
 }
@@ -214,6 +225,14 @@ const char* qlora_status_string(int s) {
 
 uint64_t qlora_launch_count(void) { return g_launches.load(); }
 
+int qlora_set_kernel_events(int slot, void* start, void* stop) {
+  if (slot < 0 || slot >= kEventSlots) return QL_ERR_INVALID_ARG;
+  if ((start == nullptr) != (stop == nullptr)) return QL_ERR_INVALID_ARG;
+  g_ev[slot][0] = (cudaEvent_t)start;
+  g_ev[slot][1] = (cudaEvent_t)stop;
+  return QL_OK;
+}
+
 int qlora_device_status(int* site, int reset) {
   if (cudaDeviceSynchronize() != cudaSuccess) return QL_ERR_CUDA;
   DeviceStatus h;
@@ -299,7 +318,7 @@ int qlora_linear_fwd(int qtype, const void* wq, int64_t N, int64_t K, const void
   p.ldo = N;
   const int tiles = p.num_n_tiles * p.num_m_blocks;
   const int grid = std::min(tiles, num_sms());
-  return launch_qgemm_q<false, EPI_STORE>(qtype, tA, tW, tLA, tLB, p, grid, st);
+  return launch_qgemm_q<false, EPI_STORE>(qtype, tA, tW, tLA, tLB, p, grid, st, 0);
 }
 
 int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void* X, const void* dY, int64_t M,
@@ -348,7 +367,7 @@ int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void
     p.out_dtype = dx_dtype;
     p.ldo = K;
     const int tiles = p.num_n_tiles * p.num_m_blocks;
-    rc = launch_qgemm_q<true, EPI_STORE>(qtype, tA, tW, tLA, tLB, p, std::min(tiles, num_sms()), st);
+    rc = launch_qgemm_q<true, EPI_STORE>(qtype, tA, tW, tLA, tLB, p, std::min(tiles, num_sms()), st, 1);
     if (rc) return rc;
   }
   // dB = s dY^T H ; dA = G^T X
