@@ -122,6 +122,28 @@ int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void
                      void* dX, int dx_dtype, float* dA, float* dB, void* ws, size_t ws_bytes,
                      void* stream);
 
+/* Forward without allocation (no counterpart in the method's sources; a convenience of this
+ * library). Same arguments, results and rules as qlora_linear_fwd, minus (ws, ws_bytes).
+ *
+ * For callers that cannot allocate device memory: code running where every byte of the device
+ * pool is already owned by a caching allocator, or where a cudaMalloc (which can synchronise the
+ * whole device) is not acceptable, and that therefore cannot hand this library a workspace.
+ * Instead of a workspace it uses one static device array of 4 MiB that the library image itself
+ * reserves on every device that loads it (held until the process exits). The adapter operands need
+ * roundup(2*KL*M, 256) + 2*KL*N bytes of it, KL = 64 for r <= 32 and 128 for r <= 64 (so about
+ * M + N <= 32768 at r <= 32 and M + N <= 16384 at r <= 64); larger sizes return
+ * QL_ERR_WORKSPACE before any launch.
+ * It calls no allocation routine of any kind.
+ *
+ * The first call on each device looks up the array's device address (cudaGetSymbolAddress) while
+ * that device is current; make that first call before any stream capture. All calls on a device
+ * share the one array and leave their operands in it: two calls whose kernels overlap on the GPU
+ * (different streams, no ordering between them) race on it and may produce wrong results; calls
+ * on one stream, or otherwise ordered, are fine. Each call rewrites everything it reads. */
+int qlora_linear_fwd_noalloc(int qtype, const void* wq, int64_t N, int64_t K, const void* X, int64_t M,
+                             const void* A, const void* B, int r, float scale, void* Y, int y_dtype,
+                             float* H, void* stream);
+
 #if defined(__GNUC__)
 #pragma GCC visibility pop
 #endif

@@ -6,5 +6,6 @@ marshalling only). ``inputs`` holds the seeded synthetic workloads and the offli
 """
 from ._lib import (Q4_0, Q4_K, Q8_0, QL_BF16, QL_F32, QloraError, gguf_dequant, lib,  # noqa: F401
                    qlora_device_status, qlora_launch_count, qlora_linear_bwd, qlora_linear_fwd,
+                   qlora_linear_fwd_noalloc,
                    qlora_linear_workspace_bytes, qlora_selftest_wait_timeout, qlora_set_kernel_events,
                    qlora_status_string)

@@ -37,6 +37,8 @@ SIGNATURES = {
     "qlora_linear_workspace_bytes": (_c_sz, [_c_i64, _c_i64, _c_i64, _c_int]),
     "qlora_linear_fwd": (_c_int, [_c_int, _c_vp, _c_i64, _c_i64, _c_vp, _c_i64, _c_vp, _c_vp, _c_int, _c_f,
                                   _c_vp, _c_int, _c_vp, _c_vp, _c_sz, _c_vp]),
+    "qlora_linear_fwd_noalloc": (_c_int, [_c_int, _c_vp, _c_i64, _c_i64, _c_vp, _c_i64, _c_vp, _c_vp, _c_int,
+                                          _c_f, _c_vp, _c_int, _c_vp, _c_vp]),
     "qlora_linear_bwd": (_c_int, [_c_int, _c_vp, _c_i64, _c_i64, _c_vp, _c_vp, _c_i64, _c_vp, _c_vp, _c_int,
                                   _c_f, _c_vp, _c_vp, _c_int, _c_vp, _c_vp, _c_vp, _c_sz, _c_vp]),
 }
@@ -134,6 +136,13 @@ def qlora_linear_fwd(qtype, wq, N, K, X, A, B, r, scale, Y, H, ws, stream=None):
     M = X.shape[0]
     _check(lib().qlora_linear_fwd(qtype, _p(wq), N, K, _p(X), M, _p(A), _p(B), r, scale, _p(Y), _dt(Y), _p(H),
                                   _p(ws), ws.numel() * ws.element_size(), _s(stream)), "qlora_linear_fwd")
+
+
+def qlora_linear_fwd_noalloc(qtype, wq, N, K, X, A, B, r, scale, Y, H, stream=None):
+    """qlora_linear_fwd without a workspace: the library's own static device scratch is used."""
+    M = X.shape[0]
+    _check(lib().qlora_linear_fwd_noalloc(qtype, _p(wq), N, K, _p(X), M, _p(A), _p(B), r, scale, _p(Y), _dt(Y),
+                                          _p(H), _s(stream)), "qlora_linear_fwd_noalloc")
 
 
 def qlora_linear_bwd(qtype, wq, N, K, X, dY, A, B, r, scale, H, dX, dA, dB, ws, stream=None):

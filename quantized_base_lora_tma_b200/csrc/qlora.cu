@@ -6,6 +6,7 @@
 #include <atomic>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "qlora.h"
 #include "lora.cuh"
@@ -380,3 +381,80 @@ int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------------
+// Forward without any allocation: the adapter operands live in a static device array.
+// ------------------------------------------------------------------------------------------------
+namespace qlora {
+
+// Scratch of qlora_linear_fwd_noalloc: LA [M x KL] then LB [N x KL], bf16 (KL = 64 for r <= 32,
+// 128 for r <= 64). Every device that loads the library holds these 4 MiB until the process exits.
+constexpr size_t kStaticScratchBytes = (size_t)4 << 20;
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+static std::mutex g_static_scratch_mu;
+static void* g_static_scratch_dev[kMaxDevices] = {};
+
+// Device address of g_static_scratch on the current device; looked up on the first use per device.
+static int static_scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QL_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return QL_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+  if (g_static_scratch_dev[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress((void**)&ptr, g_static_scratch) != cudaSuccess || ptr == nullptr) return QL_ERR_CUDA;
+    g_static_scratch_dev[dev] = ptr;
+  }
+  *out = g_static_scratch_dev[dev];
+  return QL_OK;
+}
+
+}  // namespace qlora
+
+extern "C" int qlora_linear_fwd_noalloc(int qtype, const void* wq, int64_t N, int64_t K, const void* X, int64_t M,
+                                        const void* A, const void* B, int r, float scale, void* Y, int y_dtype,
+                                        float* H, void* stream) {
+  int rc = check_linear(qtype, wq, N, K, X, M, A, B, r);
+  if (rc != QL_OK) return rc;
+  if (!Y || !H) return QL_ERR_INVALID_ARG;
+  if (y_dtype != QL_F32 && y_dtype != QL_BF16) return QL_ERR_INVALID_ARG;
+  if (!aligned16(Y) || !aligned16(H)) return QL_ERR_ALIGNMENT;
+  const int KL = 2 * lora_rp(r);
+  const size_t la_bytes = al256((size_t)M * KL * 2);
+  const size_t need = la_bytes + (size_t)N * KL * 2;
+  if (need > kStaticScratchBytes) return QL_ERR_WORKSPACE;
+  void* base = nullptr;
+  rc = static_scratch_address(&base);
+  if (rc != QL_OK) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  // Both operands are rewritten in full (padding included) before the GEMM reads them, so what
+  // an earlier call left in the array does not matter.
+  __nv_bfloat16* LA = (__nv_bfloat16*)base;
+  __nv_bfloat16* LB = (__nv_bfloat16*)((uint8_t*)base + la_bytes);
+
+  rc = launch_lora_rows((const __nv_bfloat16*)X, K, (int)M, (int)K, (const __nv_bfloat16*)A, K, 1, 0, nullptr, r,
+                        1.0f, scale, H, LA, st);
+  if (rc) return rc;
+  rc = launch_lora_bop((const __nv_bfloat16*)B, r, 1, 0, (int)N, 1, r, LB, st);
+  if (rc) return rc;
+  CUtensorMap tA, tW, tLA, tLB;
+  const int64_t rb = packed_row_bytes(qtype, K);
+  if (!tmap_bf16_rows(&tA, X, K, M, 128) || !tmap_packed(&tW, wq, rb, N, group_bytes(qtype)) ||
+      !tmap_bf16_rows(&tLA, LA, KL, M, 128) || !tmap_bf16_rows(&tLB, LB, KL, N, 64))
+    return QL_ERR_CUDA;
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.M = (int)M;
+  p.Nd = (int)N;
+  p.Kd = (int)K;
+  p.n_lora_kb = KL / 64;
+  p.num_n_tiles = (int)((N + 127) / 128);
+  p.num_m_blocks = (int)((M + 127) / 128);
+  p.out = Y;
+  p.out_dtype = y_dtype;
+  p.ldo = N;
+  const int tiles = p.num_n_tiles * p.num_m_blocks;
+  return launch_qgemm_q<false, EPI_STORE>(qtype, tA, tW, tLA, tLB, p, std::min(tiles, num_sms()), st, 0);
+}
