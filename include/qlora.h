@@ -122,6 +122,62 @@ int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void
                      void* dX, int dx_dtype, float* dA, float* dB, void* ws, size_t ws_bytes,
                      void* stream);
 
+/* ---------------------------------------------------------------------------------------------
+ * Routed MoE layer with SwiGLU experts ("MoE routing", "grouped MMQ" and the fast LoRA backward
+ * "for linear layer and MoE layer" of Show HN: LoRA over GGUF, "Things involved in the training").
+ * Expert e: gate/up weight Wgu_e [2I x H] (rows [0, I) gate, [I, 2I) up), down weight Wd_e [H x I],
+ * packed and stacked [E][rows][...]; adapters A_gu [E][r][H], B_gu [E][2I][r], A_d [E][r][I],
+ * B_d [E][H][r] (bf16); s = scale.
+ *   gu = x Wgu^T + s (x A_gu^T) B_gu^T;  h = silu(gu[:I]) * gu[I:];  o = h Wd^T + s (h A_d^T) B_d^T
+ *   Y[t] = sum over the k selected slots (slot order) of w_tj * o_tj.
+ * Rules: 1 <= k <= min(E, 16); E <= 256; H % 256 == 0; I % 256 == 0; 1 <= r <= 64; T >= 1;
+ * T * ceil(E/32) <= 50000. P = T * k routed pairs.
+ * ------------------------------------------------------------------------------------------- */
+
+/* Routing. logits [T x E] bf16. Writes (device buffers of the caller):
+ *   topk_idx [T x k] int32   selected experts, descending logit, equal logits -> lower index
+ *   topk_w   [T x k] fp32    softmax over the k selected logits
+ *   counts   [E] int32, offsets [E+1] int32 (exclusive scan; offsets[E] = P)
+ *   perm     [P] int32       pairs t*k+j sorted by (expert, token, slot); inv_perm [P] its inverse
+ *   mblk     [E+1] int32     sum over earlier experts of ceil(counts/128): the grouped GEMMs' block list
+ * Indices, counts, offsets, perm, inv_perm and mblk are exact (no floating point decides them
+ * beyond comparisons of the bf16 logits). */
+int qlora_moe_route(const void* logits, int64_t T, int E, int k, int32_t* topk_idx, float* topk_w,
+                    int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv_perm, int32_t* mblk,
+                    void* stream);
+
+/* Bytes of the activations the forward saves for the backward (caller-owned buffer `saved`):
+ * g, u, h [P x I] bf16, the bf16 residual h - bf16(h) [P x I] and X A_gu^T, h A_d^T [P x r] fp32,
+ * in pair order. */
+size_t qlora_moe_saved_bytes(int64_t T, int k, int64_t H, int64_t I, int r);
+
+/* Scratch bytes for qlora_moe_fwd / qlora_moe_bwd with these sizes. */
+size_t qlora_moe_workspace_bytes(int64_t T, int k, int E, int64_t H, int64_t I, int r);
+
+/* Forward. X [T x H] bf16; the routing buffers as written by qlora_moe_route; Y [T x H] of y_dtype.
+ * The weighted per-pair outputs stay fp32 up to the slot-ordered fp32 sum; g, u, h are saved in
+ * bf16 (h from the fp32 g, u). */
+int qlora_moe_fwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H, int64_t I,
+                  const void* X, int64_t T, int k, const int32_t* topk_idx, const float* topk_w,
+                  const int32_t* offsets, const int32_t* perm, const int32_t* inv_perm,
+                  const int32_t* mblk, const void* A_gu, const void* B_gu, const void* A_d,
+                  const void* B_d, int r, float scale, void* Y, int y_dtype, void* saved,
+                  size_t saved_bytes, void* ws, size_t ws_bytes, void* stream);
+
+/* Backward. dY [T x H] bf16; saved from the forward. Writes dX [T x H] of dx_dtype (per-pair input
+ * gradients stay fp32 up to the slot-ordered sum; d[g|u] enters the gate/up input-gradient GEMM in
+ * bf16 and the adapter gradients as an fp32-accurate bf16 pair, like h), dA_gu [E][r][H], dB_gu [E][2I][r],
+ * dA_d [E][r][I], dB_d [E][H][r] (fp32, overwritten; experts without tokens get zeros) and, if
+ * d_logits is not NULL, the router-logit gradient [T x E] fp32 (zero off the selected experts). */
+int qlora_moe_bwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H, int64_t I,
+                  const void* X, const void* dY, int64_t T, int k, const int32_t* topk_idx,
+                  const float* topk_w, const int32_t* offsets, const int32_t* perm,
+                  const int32_t* inv_perm, const int32_t* mblk, const void* A_gu, const void* B_gu,
+                  const void* A_d, const void* B_d, int r, float scale, const void* saved,
+                  size_t saved_bytes, void* dX, int dx_dtype, float* dA_gu, float* dB_gu,
+                  float* dA_d, float* dB_d, float* d_logits, void* ws, size_t ws_bytes,
+                  void* stream);
+
 /* Forward without allocation (no counterpart in the method's sources; a convenience of this
  * library). Same arguments, results and rules as qlora_linear_fwd, minus (ws, ws_bytes).
  *
@@ -129,10 +185,10 @@ int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void
  * pool is already owned by a caching allocator, or where a cudaMalloc (which can synchronise the
  * whole device) is not acceptable, and that therefore cannot hand this library a workspace.
  * Instead of a workspace it uses one static device array of 4 MiB that the library image itself
- * reserves on every device that loads it (held until the process exits). The adapter operands need
- * roundup(2*KL*M, 256) + 2*KL*N bytes of it, KL = 64 for r <= 32 and 128 for r <= 64 (so about
- * M + N <= 32768 at r <= 32 and M + N <= 16384 at r <= 64); larger sizes return
- * QL_ERR_WORKSPACE before any launch.
+ * reserves on every device that loads it (held until the process exits). It holds the two adapter
+ * operands, roundup256(2*KL*M) + roundup256(2*KL*N) bytes with KL = 64 for r <= 32 and 128 for
+ * r <= 64 (about M + N <= 32768 at r <= 32, M + N <= 16384 at r <= 64); sizes that do not fit
+ * return QL_ERR_WORKSPACE before any launch.
  * It calls no allocation routine of any kind.
  *
  * The first call on each device looks up the array's device address (cudaGetSymbolAddress) while

@@ -30,9 +30,13 @@ weight), dw_tj = <dh_u, h>, dh = w_tj dh_u, sigma = 1/(1+exp(-g)):
   dA_d_e  = sum_p (s w_p dY_t B_d)^T h_p       dB_d_e  = s sum_p (w_p dY_t)^T (h_p A_d^T)
   d_logits on the k selected logits of token t: w_j (dw_j - sum_i w_i dw_i); zero elsewhere.
 
-Rounding points (``mirror=True``): the layer stores g, u, h, d[g|u], the weighted pair outputs
-w*o and the pair input-gradients dx_pair in bf16, and uses the stored g, u in the backward; the
-oracle rounds the same values at the same places. Weights are the bf16 decode. With
+Rounding points (``mirror=True``): the layer stores g, u, h and d[g|u] in bf16 and uses the stored
+g, u in the backward, and the bf16 h and d[g|u] in the matmuls that take them (the down projection
+and its adapter input h A_d^T; the gate/up input-gradient and its adapter input s d[g|u] B_gu); the
+oracle rounds the same values at the same places. The adapter gradients dA_d and dB_gu, which sum
+over an expert's pairs only, take h and d[g|u] at fp32 accuracy (the layer carries them as a bf16
+pair there), so the oracle uses the unrounded values for those two. The weighted pair outputs w*o
+and the pair input-gradients dx_pair are kept in fp32 (no rounding point). Weights are the bf16 decode. With
 ``mirror=False`` and ``round_weights=False`` the function is smooth (finite-difference checks).
 """
 from __future__ import annotations
@@ -71,30 +75,36 @@ def _sigmoid(g):
     return 1.0 / (1.0 + np.exp(-g))
 
 
-def expert_weights(qtype, w_gu, w_d, H, I, round_weights=True):
-    """Decoded (W_gu [E,2I,H], W_d [E,H,I])."""
+def expert_weights(qtype, w_gu, w_d, H, I, round_weights=True, experts=None):
+    """Decoded (W_gu [E,2I,H], W_d [E,H,I]). With `experts`, only those are decoded (the others
+    stay zero and must then be skipped by moe_fwd / moe_bwd through the same `experts`)."""
     dec = deq_bf16 if round_weights else decode_exact
     E = w_gu.shape[0]
-    Wgu = np.stack([dec(qtype, w_gu[e], 2 * I, H) for e in range(E)])
-    Wd = np.stack([dec(qtype, w_d[e], H, I) for e in range(E)])
-    return Wgu, Wd
+    if experts is None:
+        Wgu = np.stack([dec(qtype, w_gu[e], 2 * I, H) for e in range(E)])
+        Wd = np.stack([dec(qtype, w_d[e], H, I) for e in range(E)])
+        return Wgu, Wd
+    return ({e: dec(qtype, w_gu[e], 2 * I, H) for e in experts},
+            {e: dec(qtype, w_d[e], H, I) for e in experts})
 
 
-def moe_fwd(Wgu, Wd, X, idx, w, counts, offsets, perm, A_gu, B_gu, A_d, B_d, s, mirror=True):
-    """Grouped forward. Returns (Y [T,H], saved) where saved holds per-pair (perm order) tensors."""
+def moe_fwd(Wgu, Wd, X, idx, w, counts, offsets, perm, A_gu, B_gu, A_d, B_d, s, mirror=True, experts=None):
+    """Grouped forward. Returns (Y [T,H], saved) where saved holds per-pair (perm order) tensors.
+    With `experts`, only those experts' pairs are computed (Y is then complete only for tokens
+    whose selected experts all lie in the subset)."""
     rb = round_bf16 if mirror else (lambda v: v)
     T, H = X.shape
     k = idx.shape[1]
-    E, twoI, _ = Wgu.shape
-    I = twoI // 2
+    E = len(offsets) - 1
+    I = B_gu.shape[1] // 2
     P = T * k
     tok = perm // k
     slot = perm % k
     wp = w[tok, slot]
-    g = np.zeros((P, I)); u = np.zeros((P, I)); h = np.zeros((P, I))
+    g = np.zeros((P, I)); u = np.zeros((P, I)); h = np.zeros((P, I)); h_exact = np.zeros((P, I))
     Hgu = np.zeros((P, A_gu.shape[1])); Hd = np.zeros((P, A_d.shape[1]))
     pair_out = np.zeros((P, H))
-    for e in range(E):
+    for e in (range(E) if experts is None else experts):
         a, b = offsets[e], offsets[e + 1]
         if a == b:
             continue
@@ -102,29 +112,31 @@ def moe_fwd(Wgu, Wd, X, idx, w, counts, offsets, perm, A_gu, B_gu, A_d, B_d, s, 
         Hgu[a:b] = x @ A_gu[e].T
         gu = x @ Wgu[e].T + s * (Hgu[a:b] @ B_gu[e].T)
         ge, ue = gu[:, :I], gu[:, I:]
-        h[a:b] = rb(_silu(ge) * ue)
+        h_exact[a:b] = _silu(ge) * ue
+        h[a:b] = rb(h_exact[a:b])
         g[a:b] = rb(ge)
         u[a:b] = rb(ue)
         Hd[a:b] = h[a:b] @ A_d[e].T
         o = h[a:b] @ Wd[e].T + s * (Hd[a:b] @ B_d[e].T)
-        pair_out[a:b] = rb(wp[a:b, None] * o)
+        pair_out[a:b] = wp[a:b, None] * o
     Y = np.zeros((T, H))
     inv = np.empty(P, np.int64)
     inv[perm] = np.arange(P)
     for j in range(k):                                   # slot order
         Y += pair_out[inv[np.arange(T) * k + j]]
-    saved = dict(g=g, u=u, h=h, Hgu=Hgu, Hd=Hd, pair_out=pair_out)
+    saved = dict(g=g, u=u, h=h, h_exact=h_exact, Hgu=Hgu, Hd=Hd, pair_out=pair_out)
     return Y, saved
 
 
 def moe_bwd(Wgu, Wd, X, dY, idx, w, counts, offsets, perm, A_gu, B_gu, A_d, B_d, s, saved,
-            mirror=True):
-    """Grouped backward. Returns dict(dX, dA_gu, dB_gu, dA_d, dB_d, d_logits_sel [T,k], dw [T,k])."""
+            mirror=True, experts=None):
+    """Grouped backward. Returns dict(dX, dA_gu, dB_gu, dA_d, dB_d, d_logits_sel [T,k], dw [T,k]).
+    `experts` restricts the work as in moe_fwd."""
     rb = round_bf16 if mirror else (lambda v: v)
     T, H = X.shape
     k = idx.shape[1]
-    E, twoI, _ = Wgu.shape
-    I = twoI // 2
+    E = len(offsets) - 1
+    I = B_gu.shape[1] // 2
     P = T * k
     tok = perm // k
     slot = perm % k
@@ -134,7 +146,7 @@ def moe_bwd(Wgu, Wd, X, dY, idx, w, counts, offsets, perm, A_gu, B_gu, A_d, B_d,
     dA_d = np.zeros_like(A_d); dB_d = np.zeros_like(B_d)
     dw_p = np.zeros(P)
     dx_pair = np.zeros((P, H))
-    for e in range(E):
+    for e in (range(E) if experts is None else experts):
         a, b = offsets[e], offsets[e + 1]
         if a == b:
             continue
@@ -146,13 +158,14 @@ def moe_bwd(Wgu, Wd, X, dY, idx, w, counts, offsets, perm, A_gu, B_gu, A_d, B_d,
         sg = _sigmoid(g[a:b])
         dg = dh * u[a:b] * sg * (1.0 + g[a:b] * (1.0 - sg))
         du = dh * (g[a:b] * sg)
-        dgu = rb(np.concatenate([dg, du], axis=1))
-        dA_d[e] = (wp[a:b, None] * Gd).T @ h[a:b]
+        dgu_exact = np.concatenate([dg, du], axis=1)
+        dgu = rb(dgu_exact)
+        dA_d[e] = (wp[a:b, None] * Gd).T @ saved["h_exact"][a:b]
         dB_d[e] = s * ((wp[a:b, None] * dy).T @ Hd[a:b])
         Ggu = s * (dgu @ B_gu[e])
-        dx_pair[a:b] = rb(dgu @ Wgu[e] + Ggu @ A_gu[e])
+        dx_pair[a:b] = dgu @ Wgu[e] + Ggu @ A_gu[e]
         dA_gu[e] = Ggu.T @ X[tok[a:b]]
-        dB_gu[e] = s * (dgu.T @ Hgu[a:b])
+        dB_gu[e] = s * (dgu_exact.T @ Hgu[a:b])
     inv = np.empty(P, np.int64)
     inv[perm] = np.arange(P)
     dX = np.zeros((T, H))

@@ -37,6 +37,16 @@ SIGNATURES = {
     "qlora_linear_workspace_bytes": (_c_sz, [_c_i64, _c_i64, _c_i64, _c_int]),
     "qlora_linear_fwd": (_c_int, [_c_int, _c_vp, _c_i64, _c_i64, _c_vp, _c_i64, _c_vp, _c_vp, _c_int, _c_f,
                                   _c_vp, _c_int, _c_vp, _c_vp, _c_sz, _c_vp]),
+    "qlora_moe_route": (_c_int, [_c_vp, _c_i64, _c_int, _c_int, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp,
+                                 _c_vp]),
+    "qlora_moe_saved_bytes": (_c_sz, [_c_i64, _c_int, _c_i64, _c_i64, _c_int]),
+    "qlora_moe_workspace_bytes": (_c_sz, [_c_i64, _c_int, _c_int, _c_i64, _c_i64, _c_int]),
+    "qlora_moe_fwd": (_c_int, [_c_int, _c_vp, _c_vp, _c_int, _c_i64, _c_i64, _c_vp, _c_i64, _c_int, _c_vp, _c_vp,
+                               _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_f, _c_vp, _c_int,
+                               _c_vp, _c_sz, _c_vp, _c_sz, _c_vp]),
+    "qlora_moe_bwd": (_c_int, [_c_int, _c_vp, _c_vp, _c_int, _c_i64, _c_i64, _c_vp, _c_vp, _c_i64, _c_int, _c_vp,
+                               _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_f, _c_vp,
+                               _c_sz, _c_vp, _c_int, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_sz, _c_vp]),
     "qlora_linear_fwd_noalloc": (_c_int, [_c_int, _c_vp, _c_i64, _c_i64, _c_vp, _c_i64, _c_vp, _c_vp, _c_int,
                                           _c_f, _c_vp, _c_int, _c_vp, _c_vp]),
     "qlora_linear_bwd": (_c_int, [_c_int, _c_vp, _c_i64, _c_i64, _c_vp, _c_vp, _c_i64, _c_vp, _c_vp, _c_int,
@@ -151,3 +161,61 @@ def qlora_linear_bwd(qtype, wq, N, K, X, dY, A, B, r, scale, H, dX, dA, dB, ws, 
     _check(lib().qlora_linear_bwd(qtype, _p(wq), N, K, _p(X), _p(dY), M, _p(A), _p(B), r, scale, _p(H), _p(dX),
                                   dxt, _p(dA), _p(dB), _p(ws), ws.numel() * ws.element_size(), _s(stream)),
            "qlora_linear_bwd")
+
+
+class MoeRoute:
+    """Device buffers written by qlora_moe_route."""
+
+    def __init__(self, T, E, k, device="cuda"):
+        P = T * k
+        i32 = torch.int32
+        self.T, self.E, self.k = T, E, k
+        self.topk_idx = torch.empty(T, k, dtype=i32, device=device)
+        self.topk_w = torch.empty(T, k, dtype=torch.float32, device=device)
+        self.counts = torch.empty(E, dtype=i32, device=device)
+        self.offsets = torch.empty(E + 1, dtype=i32, device=device)
+        self.perm = torch.empty(P, dtype=i32, device=device)
+        self.inv_perm = torch.empty(P, dtype=i32, device=device)
+        self.mblk = torch.empty(E + 1, dtype=i32, device=device)
+
+
+def qlora_moe_route(logits, k, route=None, stream=None) -> MoeRoute:
+    T, E = logits.shape
+    if route is None:
+        route = MoeRoute(T, E, k, logits.device)
+    _check(lib().qlora_moe_route(_p(logits), T, E, k, _p(route.topk_idx), _p(route.topk_w), _p(route.counts),
+                                 _p(route.offsets), _p(route.perm), _p(route.inv_perm), _p(route.mblk), _s(stream)),
+           "qlora_moe_route")
+    return route
+
+
+def qlora_moe_saved_bytes(T, k, H, I, r) -> int:
+    return int(lib().qlora_moe_saved_bytes(T, k, H, I, r))
+
+
+def qlora_moe_workspace_bytes(T, k, E, H, I, r) -> int:
+    return int(lib().qlora_moe_workspace_bytes(T, k, E, H, I, r))
+
+
+def _nb(t):
+    return t.numel() * t.element_size()
+
+
+def qlora_moe_fwd(qtype, w_gu, w_d, E, H, I, X, route, A_gu, B_gu, A_d, B_d, r, scale, Y, saved, ws, stream=None):
+    T = X.shape[0]
+    R = route
+    _check(lib().qlora_moe_fwd(qtype, _p(w_gu), _p(w_d), E, H, I, _p(X), T, R.k, _p(R.topk_idx), _p(R.topk_w),
+                               _p(R.offsets), _p(R.perm), _p(R.inv_perm), _p(R.mblk), _p(A_gu), _p(B_gu), _p(A_d),
+                               _p(B_d), r, scale, _p(Y), _dt(Y), _p(saved), _nb(saved), _p(ws), _nb(ws), _s(stream)),
+           "qlora_moe_fwd")
+
+
+def qlora_moe_bwd(qtype, w_gu, w_d, E, H, I, X, dY, route, A_gu, B_gu, A_d, B_d, r, scale, saved, dX, dA_gu, dB_gu,
+                  dA_d, dB_d, d_logits, ws, stream=None):
+    T = X.shape[0]
+    R = route
+    _check(lib().qlora_moe_bwd(qtype, _p(w_gu), _p(w_d), E, H, I, _p(X), _p(dY), T, R.k, _p(R.topk_idx),
+                               _p(R.topk_w), _p(R.offsets), _p(R.perm), _p(R.inv_perm), _p(R.mblk), _p(A_gu), _p(B_gu),
+                               _p(A_d), _p(B_d), r, scale, _p(saved), _nb(saved), _p(dX), _dt(dX), _p(dA_gu),
+                               _p(dB_gu), _p(dA_d), _p(dB_d), _p(d_logits), _p(ws), _nb(ws), _s(stream)),
+           "qlora_moe_bwd")

@@ -32,6 +32,11 @@ struct QTraits<QL_Q4_K> {
   static constexpr int kGroupBytes = 144;
 };
 
+__device__ __forceinline__ uint32_t pack2_same(__nv_bfloat16 h) {
+  const uint32_t u = __bfloat16_as_ushort(h);
+  return u | (u << 16);
+}
+
 __device__ __forceinline__ float half_at(const uint8_t* p) {
   return __half2float(*reinterpret_cast<const __half*>(p));
 }
@@ -103,6 +108,165 @@ __device__ __forceinline__ void decode8<QL_Q4_K>(const uint8_t* g, int c, float 
     w[i] = fmaf(ds, (float)((q.x >> (8 * i + sh)) & 15u), dm);
     w[4 + i] = fmaf(ds, (float)((q.y >> (8 * i + sh)) & 15u), dm);
   }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Whole-unit decode to bf16 for the tensor-core producers: weights [32u, 32u + 32) of a group
+// (one Q8_0 / Q4_0 block, or one 32-weight sub-block of a Q4_K superblock) as four 16-byte chunks
+// of 8 bf16. Every result equals RNE_bf16 of the exact decoded value (which is exact in fp32).
+// Integer-to-float conversion uses the 2^23 magic: the float with bit pattern 0x4B000000 | b is
+// 2^23 + b for a byte b, so one byte permute plus one subtraction yields an exact small integer.
+// ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// 32 bytes starting at a 2-byte aligned address p, as 8 words (the read stays inside [p, p+32)
+// rounded out to whole words).
+__device__ __forceinline__ void load32_a2(const uint8_t* p, uint32_t (&x)[8]) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(a & ~(uintptr_t)3);
+  const uint32_t sh = (uint32_t)(a & 3) * 8u;
+  uint32_t v[9];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = w[i];
+  v[8] = sh ? w[8] : 0u;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) x[i] = __funnelshift_r(v[i], v[i + 1], sh);
+}
+
+// 16 bytes starting at a 2-byte aligned address p, as 4 words.
+__device__ __forceinline__ void load16_a2(const uint8_t* p, uint32_t (&x)[4]) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(a & ~(uintptr_t)3);
+  const uint32_t sh = (uint32_t)(a & 3) * 8u;
+  uint32_t v[5];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = w[i];
+  v[4] = sh ? w[4] : 0u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) x[i] = __funnelshift_r(v[i], v[i + 1], sh);
+}
+
+// Four bytes of a word (each the low 8 bits of 2^23 + b) -> four exact floats 2^23 + b.
+__device__ __forceinline__ void magic4(uint32_t x, float (&f)[4]) {
+#pragma unroll
+  for (int e = 0; e < 4; ++e) f[e] = __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7440u + e));
+}
+
+template <int QT>
+__device__ __forceinline__ void decode_unit_bf16(const uint8_t* g, int u, uint4 (&out)[4]);
+
+// Q8_0: w = d * q, q int8. Bytes are biased to q + 128 so that 2^23 + (q + 128) is the magic float.
+template <>
+__device__ __forceinline__ void decode_unit_bf16<QL_Q8_0>(const uint8_t* g, int u, uint4 (&out)[4]) {
+  const uint8_t* b = g + 34 * u;
+  const float d = half_at(b);
+  uint32_t x[8];
+  load32_a2(b + 2, x);
+  const float2 dd = make_float2(d, d);
+  const float2 bias = make_float2(-8388736.0f, -8388736.0f);  // -(2^23 + 128)
+  uint32_t o[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float f[4];
+    magic4(x[i] ^ 0x80808080u, f);
+    const float2 a = __fmul2_rn(__fadd2_rn(make_float2(f[0], f[1]), bias), dd);
+    const float2 c = __fmul2_rn(__fadd2_rn(make_float2(f[2], f[3]), bias), dd);
+    o[2 * i] = bf16x2_bits(a.x, a.y);
+    o[2 * i + 1] = bf16x2_bits(c.x, c.y);
+  }
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) out[cc] = make_uint4(o[4 * cc], o[4 * cc + 1], o[4 * cc + 2], o[4 * cc + 3]);
+}
+
+__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+
+// Q4_0: w = d * (q - 8). d (fp16, 11 significant bits) = d1 + d2 with d1 = bf16(d) and d2 = d - d1
+// (at most 3 significant bits, so exact in bf16). v = q - 8 is exact in bf16 and d2 * v has at most
+// 7 significant bits, so c = d2 * v is exact and one fused bf16 FMA d1 * v + c rounds d * v once:
+// the result is RNE_bf16 of the exact value. The bf16 magic 0x4300 | n is 128 + n for a nibble n.
+template <>
+__device__ __forceinline__ void decode_unit_bf16<QL_Q4_0>(const uint8_t* g, int u, uint4 (&out)[4]) {
+  const uint8_t* b = g + 18 * u;
+  const float d = half_at(b);
+  const __nv_bfloat16 d1 = __float2bfloat16_rn(d);
+  const __nv_bfloat16 d2 = __float2bfloat16_rn(d - __bfloat162float(d1));
+  const uint32_t D1 = pack2_same(d1), D2 = pack2_same(d2);
+  const uint32_t B136 = 0x43084308u;  // bf16 pair (136, 136)
+  uint32_t x[4];
+  load16_a2(b + 2, x);
+  uint32_t o[16];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {  // h = 0: low nibbles (weights 0..15), 1: high nibbles (16..31)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t w = h ? (x[i] >> 4) : x[i];
+#pragma unroll
+      for (int pr = 0; pr < 2; ++pr) {
+        const uint32_t t = __byte_perm(w, 0u, (uint32_t)(2 * pr) | 0x4000u | ((uint32_t)(2 * pr + 1) << 8) | 0x40u);
+        const uint32_t m = (t & 0x000F000Fu) | 0x43004300u;
+        const uint32_t v = bf16x2_sub(m, B136);
+        o[8 * h + 2 * i + pr] = bf16x2_fma(v, D1, bf16x2_mul(v, D2));
+      }
+    }
+  }
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) out[cc] = make_uint4(o[4 * cc], o[4 * cc + 1], o[4 * cc + 2], o[4 * cc + 3]);
+}
+
+// Q4_K sub-block u: w = (d*sc) * q - dmin*m with both products exact in fp32; one fp32 FMA rounds
+// the difference once, then one bf16 rounding.
+template <>
+__device__ __forceinline__ void decode_unit_bf16<QL_Q4_K>(const uint8_t* g, int u, uint4 (&out)[4]) {
+  const float d = half_at(g);
+  const float dmin = half_at(g + 2);
+  const uint8_t* S = g + 4;
+  const int j = u;
+  int sc, m;
+  if (j < 4) {
+    sc = S[j] & 63;
+    m = S[j + 4] & 63;
+  } else {
+    sc = (S[j + 4] & 15) | ((S[j - 4] >> 6) << 4);
+    m = (S[j + 4] >> 4) | ((S[j] >> 6) << 4);
+  }
+  const float ds = d * (float)sc;
+  const float dm = -(dmin * (float)m);
+  const uint4* qp = reinterpret_cast<const uint4*>(g + 16 + 32 * (j >> 1));
+  const uint4 q0 = qp[0], q1 = qp[1];
+  const uint32_t xs[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+  const uint32_t sh = (uint32_t)(j & 1) * 4u;
+  const float2 dsv = make_float2(ds, ds), dmv = make_float2(dm, dm);
+  const float2 bias = make_float2(-8388608.0f, -8388608.0f);  // -2^23
+  uint32_t o[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float f[4];
+    magic4((xs[i] >> sh) & 0x0F0F0F0Fu, f);
+    const float2 a = __ffma2_rn(__fadd2_rn(make_float2(f[0], f[1]), bias), dsv, dmv);
+    const float2 c = __ffma2_rn(__fadd2_rn(make_float2(f[2], f[3]), bias), dsv, dmv);
+    o[2 * i] = bf16x2_bits(a.x, a.y);
+    o[2 * i + 1] = bf16x2_bits(c.x, c.y);
+  }
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) out[cc] = make_uint4(o[4 * cc], o[4 * cc + 1], o[4 * cc + 2], o[4 * cc + 3]);
 }
 
 // 8 fp32 values -> 8 bf16 (round to nearest even) packed in 16 bytes.

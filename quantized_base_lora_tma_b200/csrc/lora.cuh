@@ -107,6 +107,644 @@ __global__ void __launch_bounds__(256) lora_rows_kernel(const __nv_bfloat16* __r
   }
 }
 
+// ------------------------------------------------------------------------------------------------
+// Tensor-core (mma.sync m16n8k16, bf16 in, fp32 accumulate) versions of the two adapter reductions.
+// These are small, bandwidth-bound contractions with r <= 64 output columns; the warp-level MMA
+// keeps them at memory speed without a CUDA-core FMA bottleneck.
+// ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t ldg_u32(const void* p) { return __ldg(reinterpret_cast<const uint32_t*>(p)); }
+
+__device__ __forceinline__ uint32_t pack2_bf16(__nv_bfloat16 lo, __nv_bfloat16 hi) {
+  return (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+}
+
+// Split-K partial row products: part[ks][m][j] = sum_{k in slice ks} Y[m, k] Z(j, k), j < 8*NT.
+// Z(j, k) = Z[j*zj + k*zk]. Grid (ceil(M/64), KS), 128 threads; warp w owns rows 64*bx + 16w.
+template <int NT>
+__global__ void __launch_bounds__(128) lora_rows_mma_kernel(const __nv_bfloat16* __restrict__ Y, long ldy, int M,
+                                                            int Kin, int kchunk, const __nv_bfloat16* __restrict__ Z,
+                                                            long zj, long zk, int r, float* __restrict__ part) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  const int m0 = blockIdx.x * 64 + warp * 16;
+  const int r0 = m0 + g, r1 = m0 + g + 8;
+  const int kb = blockIdx.y * kchunk;
+  const int ke = min(Kin, kb + kchunk);
+  float acc[NT][4];
+#pragma unroll
+  for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+  const __nv_bfloat16* y0 = Y + (long)min(r0, M - 1) * ldy;
+  const __nv_bfloat16* y1 = Y + (long)min(r1, M - 1) * ldy;
+  const bool v0 = r0 < M, v1 = r1 < M;
+#pragma unroll 4
+  for (int k = kb; k < ke; k += 16) {
+    const uint32_t a0 = v0 ? ldg_u32(y0 + k + 2 * c) : 0u;
+    const uint32_t a1 = v1 ? ldg_u32(y1 + k + 2 * c) : 0u;
+    const uint32_t a2 = v0 ? ldg_u32(y0 + k + 2 * c + 8) : 0u;
+    const uint32_t a3 = v1 ? ldg_u32(y1 + k + 2 * c + 8) : 0u;
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      const int n = 8 * t + g;
+      uint32_t b0 = 0u, b1 = 0u;
+      if (n < r) {
+        const __nv_bfloat16* zp = Z + (long)n * zj;
+        if (zk == 1) {
+          b0 = ldg_u32(zp + k + 2 * c);
+          b1 = ldg_u32(zp + k + 2 * c + 8);
+        } else {
+          b0 = pack2_bf16(zp[(long)(k + 2 * c) * zk], zp[(long)(k + 2 * c + 1) * zk]);
+          b1 = pack2_bf16(zp[(long)(k + 2 * c + 8) * zk], zp[(long)(k + 2 * c + 9) * zk]);
+        }
+      }
+      mma_16816(acc[t], a0, a1, a2, a3, b0, b1);
+    }
+  }
+  constexpr int RN = 8 * NT;
+  float* o = part + (long)blockIdx.y * M * RN;
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    const int j = 8 * t + 2 * c;
+    if (v0) *reinterpret_cast<float2*>(o + (long)r0 * RN + j) = make_float2(acc[t][0], acc[t][1]);
+    if (v1) *reinterpret_cast<float2*>(o + (long)r1 * RN + j) = make_float2(acc[t][2], acc[t][3]);
+  }
+}
+
+// Ordered sum of the split-K partials; writes out[m][j] = oscale * v (j < r) and the split
+// operand la[m] = [hi(lscale v) | lo(lscale v)] (zero padded to 2*RP columns).
+__global__ void lora_rows_reduce_kernel(const float* __restrict__ part, int KS, int M, int RN, int r, float oscale,
+                                        float lscale, float* __restrict__ out, __nv_bfloat16* __restrict__ la,
+                                        int RP) {
+  const long total = (long)M * RP;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total; i += (long)gridDim.x * blockDim.x) {
+    const int m = (int)(i / RP), j = (int)(i % RP);
+    float v = 0.f;
+    if (j < r)
+      for (int ks = 0; ks < KS; ++ks) v += part[((long)ks * M + m) * RN + j];
+    if (out != nullptr && j < r) out[(long)m * r + j] = oscale * v;
+    if (la != nullptr) {
+      const float x = lscale * v;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+      la[(long)m * 2 * RP + j] = j < r ? hi : __float2bfloat16(0.f);
+      la[(long)m * 2 * RP + RP + j] = j < r ? lo : __float2bfloat16(0.f);
+    }
+  }
+}
+
+// Column reductions on tensor cores: part[slice][c][j] = sum_{m in slice} Y[m][c] * Zs[m][j], where
+// Zs = Z * zw (optional per-row weight) is fed as a bf16 hi + lo pair (fp32-accurate).
+// A operand: Zs^T (rows j, k = m); B operand: Y (k = m, n = c) through ldmatrix.trans.
+// Grid (ceil(C/128), slices), 128 threads: warp w owns columns 128*bx + 32w .. +31.
+// Slices as in colred_partial_kernel. JT = ceil(r/16) tiles of 16 rows of j.
+template <int JT>
+__global__ void __launch_bounds__(128) colred_mma_kernel(const __nv_bfloat16* __restrict__ Y, long ldy, int Ccols,
+                                                         const float* __restrict__ Z, int r, int M,
+                                                         const float* __restrict__ zw, const int* __restrict__ seg_off,
+                                                         const int* __restrict__ mblk_off, int E,
+                                                         float* __restrict__ part,
+                                                         const __nv_bfloat16* __restrict__ Ylo) {
+  // Ylo (nullable): a second bf16 term of Y (Y = Y + Ylo to ~2^-16), same layout.
+  constexpr int YS = 128 + 8;  // padded row (bf16): 272 bytes, ldmatrix rows hit distinct banks
+  constexpr int HR = 32;       // rows staged per step
+  __shared__ __align__(16) __nv_bfloat16 ys[HR * YS];
+  __shared__ __align__(16) __nv_bfloat16 ysl[HR * YS];
+  __shared__ __align__(16) __nv_bfloat16 zh[JT * 16][HR + 8];
+  __shared__ __align__(16) __nv_bfloat16 zl[JT * 16][HR + 8];
+  const int slice = blockIdx.y;
+  int lo, hi;
+  if (E == 0) {
+    lo = slice * 128;
+    hi = min(M, lo + 128);
+  } else {
+    const int total = __ldg(mblk_off + E);
+    if (slice >= total) return;
+    int a = 0, b = E - 1;
+    while (a < b) {
+      const int mid = (a + b + 1) >> 1;
+      if (__ldg(mblk_off + mid) <= slice) a = mid; else b = mid - 1;
+    }
+    lo = __ldg(seg_off + a) + (slice - __ldg(mblk_off + a)) * 128;
+    hi = min(__ldg(seg_off + a + 1), lo + 128);
+  }
+  const int c0 = blockIdx.x * 128;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  const bool two = Ylo != nullptr;
+  float acc[JT][4][4];
+#pragma unroll
+  for (int jt = 0; jt < JT; ++jt)
+#pragma unroll
+    for (int t = 0; t < 4; ++t) acc[jt][t][0] = acc[jt][t][1] = acc[jt][t][2] = acc[jt][t][3] = 0.f;
+  const int wc = warp * 32;  // warp's first column within the CTA tile
+  for (int step = 0; step < 128 / HR; ++step) {
+    const int mb = lo + step * HR;
+    const int n = min(HR, hi - mb);
+    if (n <= 0) break;
+    uint4 yv[HR * 16 / 128], yl[HR * 16 / 128];
+#pragma unroll
+    for (int it = 0; it < HR * 16 / 128; ++it) {
+      const int i = threadIdx.x + 128 * it;
+      const int m = i >> 4, q = i & 15;
+      const bool in = m < n && c0 + 8 * q < Ccols;
+      const long o = (long)(mb + m) * ldy + c0 + 8 * q;
+      yv[it] = in ? __ldg(reinterpret_cast<const uint4*>(Y + o)) : make_uint4(0, 0, 0, 0);
+      yl[it] = (in && two) ? __ldg(reinterpret_cast<const uint4*>(Ylo + o)) : make_uint4(0, 0, 0, 0);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int it = 0; it < HR * 16 / 128; ++it) {
+      const int i = threadIdx.x + 128 * it;
+      *reinterpret_cast<uint4*>(ys + (i >> 4) * YS + 8 * (i & 15)) = yv[it];
+      *reinterpret_cast<uint4*>(ysl + (i >> 4) * YS + 8 * (i & 15)) = yl[it];
+    }
+    // stage Z^T as hi / lo bf16
+    for (int i = threadIdx.x; i < JT * 16 * HR; i += 128) {
+      const int j = i / HR, m = i % HR;
+      float z = 0.f;
+      if (m < n && j < r) {
+        z = Z[(long)(mb + m) * r + j];
+        if (zw != nullptr) z *= zw[mb + m];
+      }
+      const __nv_bfloat16 h = __float2bfloat16_rn(z);
+      zh[j][m] = h;
+      zl[j][m] = __float2bfloat16_rn(z - __bfloat162float(h));
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < HR; k += 16) {
+#pragma unroll
+      for (int term = 0; term < 2; ++term) {
+        if (term == 1 && !two) break;
+        const __nv_bfloat16* src = term ? ysl : ys;
+        // B fragments for 4 n8 tiles: two ldmatrix.x4.trans, each covering 2 tiles x k16
+        uint32_t b[4][2];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int mat = lane >> 3, rr = lane & 7;
+          const int krow = k + ((mat & 1) ? 8 : 0) + rr;
+          const int ncol = wc + 16 * h2 + ((mat & 2) ? 8 : 0);
+          const uint32_t addr = smem_u32(src + krow * YS + ncol);
+          uint32_t x0, x1, x2, x3;
+          asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                       : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3)
+                       : "r"(addr));
+          b[2 * h2][0] = x0;
+          b[2 * h2][1] = x1;
+          b[2 * h2 + 1][0] = x2;
+          b[2 * h2 + 1][1] = x3;
+        }
+#pragma unroll
+        for (int jt = 0; jt < JT; ++jt) {
+          const int j0 = 16 * jt;
+          const uint32_t ah0 = *reinterpret_cast<const uint32_t*>(&zh[j0 + g][k + 2 * c]);
+          const uint32_t ah1 = *reinterpret_cast<const uint32_t*>(&zh[j0 + g + 8][k + 2 * c]);
+          const uint32_t ah2 = *reinterpret_cast<const uint32_t*>(&zh[j0 + g][k + 2 * c + 8]);
+          const uint32_t ah3 = *reinterpret_cast<const uint32_t*>(&zh[j0 + g + 8][k + 2 * c + 8]);
+#pragma unroll
+          for (int t = 0; t < 4; ++t) mma_16816(acc[jt][t], ah0, ah1, ah2, ah3, b[t][0], b[t][1]);
+          if (term == 0) {  // Z_lo * Y (Z_lo * Y_lo is below fp32 resolution)
+            const uint32_t al0 = *reinterpret_cast<const uint32_t*>(&zl[j0 + g][k + 2 * c]);
+            const uint32_t al1 = *reinterpret_cast<const uint32_t*>(&zl[j0 + g + 8][k + 2 * c]);
+            const uint32_t al2 = *reinterpret_cast<const uint32_t*>(&zl[j0 + g][k + 2 * c + 8]);
+            const uint32_t al3 = *reinterpret_cast<const uint32_t*>(&zl[j0 + g + 8][k + 2 * c + 8]);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) mma_16816(acc[jt][t], al0, al1, al2, al3, b[t][0], b[t][1]);
+          }
+        }
+      }
+    }
+    __syncthreads();
+  }
+  // acc[jt][t]: rows j = 16jt + g (+8), columns c0 + wc + 8t + 2c (+1)
+#pragma unroll
+  for (int jt = 0; jt < JT; ++jt)
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int col = c0 + wc + 8 * t + 2 * c;
+      const int j0 = 16 * jt + g, j1 = j0 + 8;
+      float* o = part + (long)slice * Ccols * r;
+      if (col < Ccols) {
+        if (j0 < r) { o[(long)col * r + j0] = acc[jt][t][0]; o[(long)(col + 1) * r + j0] = acc[jt][t][1]; }
+        if (j1 < r) { o[(long)col * r + j1] = acc[jt][t][2]; o[(long)(col + 1) * r + j1] = acc[jt][t][3]; }
+      }
+    }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Cluster versions (dense layer): the split-K / split-M partials are summed through distributed
+// shared memory inside one kernel, in a fixed rank order (deterministic), so no reduction launch
+// and no partial buffer in HBM are needed.
+// ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ float ld_dsmem_f32(const float* local, uint32_t rank) {
+  uint32_t a = smem_u32(local), ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
+  return v;
+}
+
+struct BopArgs {            // LB[n] = [Z(n, :) | Z(n, :)], zero padded (nullptr Z = none)
+  const __nv_bfloat16* Z;
+  long zn, zjs;
+  int rows;
+};
+
+// Rows of out = Y Z^T for 64 rows per cluster column; cluster rank q sums k in
+// [q * kchunk, (q + 1) * kchunk). Z(j, k) = Z[j*zj + k*zk]. Writes out = oscale * sum (fp32 [M x r])
+// and la = split(lscale * sum). Every CTA also writes its share of the LB operand (bop).
+template <int NT>
+__global__ void __launch_bounds__(128) lora_rows_cluster_kernel(const __nv_bfloat16* __restrict__ Y, long ldy, int M,
+                                                                int Kin, int kchunk, const __nv_bfloat16* __restrict__ Z,
+                                                                long zj, long zk, int r, float oscale, float lscale,
+                                                                float* __restrict__ out, __nv_bfloat16* __restrict__ la,
+                                                                int RP, BopArgs bop, __nv_bfloat16* __restrict__ LB) {
+  constexpr int RN = 8 * NT;
+  constexpr int SK = 128;       // k per staged sub-chunk
+  constexpr int ZS = SK + 8;    // padded row of the staged Z tile (bf16)
+  __shared__ float part[64 * RN];
+  __shared__ __align__(16) __nv_bfloat16 zs[RN * ZS];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  const int KS = gridDim.y;
+  const uint32_t rank = cluster_ctarank();
+  const int m0 = blockIdx.x * 64 + warp * 16;
+  const int r0 = m0 + g, r1 = m0 + g + 8;
+  const bool v0 = r0 < M, v1 = r1 < M;
+  const __nv_bfloat16* y0 = Y + (long)min(r0, M - 1) * ldy;
+  const __nv_bfloat16* y1 = Y + (long)min(r1, M - 1) * ldy;
+  const int kb = (int)rank * kchunk;
+  const int ke = min(Kin, kb + kchunk);
+  float acc[NT][4];
+#pragma unroll
+  for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+  for (int k0 = kb; k0 < ke; k0 += SK) {
+    const int nk = min(SK, ke - k0);  // multiple of 32
+    // this sub-chunk's rows of Y, 16 bytes per lane per k32 step, issued before the staging wait
+    uint4 xa[SK / 32], xb[SK / 32];
+#pragma unroll
+    for (int q = 0; q < SK / 32; ++q) {
+      const int k = k0 + 32 * q + 8 * c;
+      const bool in = 32 * q < nk;
+      xa[q] = (v0 && in) ? __ldg(reinterpret_cast<const uint4*>(y0 + k)) : make_uint4(0, 0, 0, 0);
+      xb[q] = (v1 && in) ? __ldg(reinterpret_cast<const uint4*>(y1 + k)) : make_uint4(0, 0, 0, 0);
+    }
+    __syncthreads();
+    // stage Z(j, k0 .. k0+SK) as zs[j][k]
+    if (zk == 1) {
+      for (int i = threadIdx.x; i < RN * (SK / 8); i += 128) {
+        const int j = i / (SK / 8), q = i % (SK / 8);
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (j < r && 8 * q < nk) v = __ldg(reinterpret_cast<const uint4*>(Z + (long)j * zj + k0 + 8 * q));
+        *reinterpret_cast<uint4*>(zs + j * ZS + 8 * q) = v;
+      }
+    } else {
+      for (int i = threadIdx.x; i < RN * SK; i += 128) {
+        const int kk = i / RN, j = i % RN;  // consecutive threads read consecutive j of one k
+        __nv_bfloat16 v = __float2bfloat16(0.f);
+        if (j < r && kk < nk) v = Z[(long)j * zj + (long)(k0 + kk) * zk];
+        zs[j * ZS + kk] = v;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < SK / 32; ++q) {
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        const uint4 zq = *reinterpret_cast<const uint4*>(zs + (8 * t + g) * ZS + 32 * q + 8 * c);
+        mma_16816(acc[t], xa[q].x, xb[q].x, xa[q].y, xb[q].y, zq.x, zq.y);
+        mma_16816(acc[t], xa[q].z, xb[q].z, xa[q].w, xb[q].w, zq.z, zq.w);
+      }
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    const int j = 8 * t + 2 * c;
+    const int lr = warp * 16 + g;
+    part[lr * RN + j] = acc[t][0];
+    part[lr * RN + j + 1] = acc[t][1];
+    part[(lr + 8) * RN + j] = acc[t][2];
+    part[(lr + 8) * RN + j + 1] = acc[t][3];
+  }
+  cluster_sync_all();
+  // rank q reduces rows [q*64/KS, (q+1)*64/KS) of the cluster's 64 rows, over ranks in order
+  const int rows_per = (64 + KS - 1) / KS;
+  const int lr0 = (int)rank * rows_per;
+  for (int i = threadIdx.x; i < rows_per * RP; i += 128) {
+    const int lr = lr0 + i / RP, j = i % RP;
+    const int m = blockIdx.x * 64 + lr;
+    if (lr >= 64 || m >= M) continue;
+    float v = 0.f;
+    if (j < r)
+      for (int q = 0; q < KS; ++q) v += ld_dsmem_f32(&part[lr * RN + j], (uint32_t)q);
+    if (out != nullptr && j < r) out[(long)m * r + j] = oscale * v;
+    if (la != nullptr) {
+      const float x = lscale * v;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+      la[(long)m * 2 * RP + j] = j < r ? hi : __float2bfloat16(0.f);
+      la[(long)m * 2 * RP + RP + j] = j < r ? lo : __float2bfloat16(0.f);
+    }
+  }
+  // this CTA's share of LB: items of 8 columns
+  if (bop.Z != nullptr) {
+    const long items = (long)bop.rows * (2 * RP / 8);
+    const long cta = (long)blockIdx.y * gridDim.x + blockIdx.x;
+    const long ncta = (long)gridDim.x * gridDim.y;
+    for (long i = cta * 128 + threadIdx.x; i < items; i += ncta * 128) {
+      const int n = (int)(i / (2 * RP / 8));
+      const int j0 = (int)(i % (2 * RP / 8)) * 8;
+      __nv_bfloat16 v[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int j = (j0 + e) % RP;
+        v[e] = j < r ? bop.Z[(long)n * bop.zn + (long)j * bop.zjs] : __float2bfloat16(0.f);
+      }
+      *reinterpret_cast<uint4*>(LB + (long)n * 2 * RP + j0) = *reinterpret_cast<const uint4*>(v);
+    }
+  }
+  cluster_sync_all();  // no CTA leaves while a peer may still read its partials
+}
+
+// Two column-reduction problems in one launch (dense layer): problem p (blockIdx.x < nb0: p = 0)
+// computes out = scale * sum_m Y[m][c] Z[m][j] over all M rows; cluster rank q takes rows
+// [q * mchunk, (q + 1) * mchunk) and the ranks' partials are summed through DSMEM in rank order.
+// transpose = 0: out[c][j]; 1: out[j][c].
+struct ColredProblem {
+  const __nv_bfloat16* Y;
+  long ldy;
+  int C;
+  const float* Z;
+  float scale;
+  int transpose;
+  float* out;
+};
+
+template <int JT>
+__global__ void __launch_bounds__(128) colred_cluster_kernel(ColredProblem p0, ColredProblem p1, int nb0, int M,
+                                                             int r, int mchunk) {
+  constexpr int YS = 128 + 8;
+  constexpr int HR = 64;
+  constexpr int Y_BYTES = HR * YS * 2;
+  constexpr int Z_BYTES = JT * 16 * (HR + 8) * 2;
+  constexpr int P_BYTES = JT * 16 * (128 + 1) * 4;
+  constexpr int BUF = (Y_BYTES + 2 * Z_BYTES) > P_BYTES ? (Y_BYTES + 2 * Z_BYTES) : P_BYTES;
+  __shared__ __align__(16) uint8_t sbuf[BUF];
+  __nv_bfloat16* ys = reinterpret_cast<__nv_bfloat16*>(sbuf);
+  auto zh = reinterpret_cast<__nv_bfloat16(*)[HR + 8]>(sbuf + Y_BYTES);
+  auto zl = reinterpret_cast<__nv_bfloat16(*)[HR + 8]>(sbuf + Y_BYTES + Z_BYTES);
+  auto part = reinterpret_cast<float(*)[128 + 1]>(sbuf);  // reused after the main loop
+  const bool second = (int)blockIdx.x >= nb0;
+  const ColredProblem& P = second ? p1 : p0;
+  const int c0 = (second ? (int)blockIdx.x - nb0 : (int)blockIdx.x) * 128;
+  const uint32_t rank = cluster_ctarank();
+  const int CS = gridDim.y;
+  const int lo = (int)rank * mchunk;
+  const int hi = min(M, lo + mchunk);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  float acc[JT][4][4];
+#pragma unroll
+  for (int jt = 0; jt < JT; ++jt)
+#pragma unroll
+    for (int t = 0; t < 4; ++t) acc[jt][t][0] = acc[jt][t][1] = acc[jt][t][2] = acc[jt][t][3] = 0.f;
+  const int wc = warp * 32;
+  for (int mb = lo; mb < hi; mb += HR) {
+    const int n = min(HR, hi - mb);
+    uint4 yv[HR * 16 / 128];
+#pragma unroll
+    for (int it = 0; it < HR * 16 / 128; ++it) {
+      const int i = threadIdx.x + 128 * it;
+      const int m = i >> 4, q = i & 15;
+      yv[it] = (m < n && c0 + 8 * q < P.C)
+                   ? __ldg(reinterpret_cast<const uint4*>(P.Y + (long)(mb + m) * P.ldy + c0 + 8 * q))
+                   : make_uint4(0, 0, 0, 0);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int it = 0; it < HR * 16 / 128; ++it) {
+      const int i = threadIdx.x + 128 * it;
+      *reinterpret_cast<uint4*>(ys + (i >> 4) * YS + 8 * (i & 15)) = yv[it];
+    }
+    for (int i = threadIdx.x; i < JT * 16 * HR; i += 128) {
+      const int j = i / HR, m = i % HR;
+      float z = 0.f;
+      if (m < n && j < r) z = P.Z[(long)(mb + m) * r + j];
+      const __nv_bfloat16 h = __float2bfloat16_rn(z);
+      zh[j][m] = h;
+      zl[j][m] = __float2bfloat16_rn(z - __bfloat162float(h));
+    }
+    __syncthreads();
+#pragma unroll 2
+    for (int k = 0; k < HR; k += 16) {
+      uint32_t b[4][2];
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int mat = lane >> 3, rr = lane & 7;
+        const int krow = k + ((mat & 1) ? 8 : 0) + rr;
+        const int ncol = wc + 16 * h2 + ((mat & 2) ? 8 : 0);
+        const uint32_t addr = smem_u32(ys + krow * YS + ncol);
+        uint32_t x0, x1, x2, x3;
+        asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3)
+                     : "r"(addr));
+        b[2 * h2][0] = x0;
+        b[2 * h2][1] = x1;
+        b[2 * h2 + 1][0] = x2;
+        b[2 * h2 + 1][1] = x3;
+      }
+#pragma unroll
+      for (int jt = 0; jt < JT; ++jt) {
+        const int j0 = 16 * jt;
+        const uint32_t ah0 = *reinterpret_cast<const uint32_t*>(&zh[j0 + g][k + 2 * c]);
+        const uint32_t ah1 = *reinterpret_cast<const uint32_t*>(&zh[j0 + g + 8][k + 2 * c]);
+        const uint32_t ah2 = *reinterpret_cast<const uint32_t*>(&zh[j0 + g][k + 2 * c + 8]);
+        const uint32_t ah3 = *reinterpret_cast<const uint32_t*>(&zh[j0 + g + 8][k + 2 * c + 8]);
+        const uint32_t al0 = *reinterpret_cast<const uint32_t*>(&zl[j0 + g][k + 2 * c]);
+        const uint32_t al1 = *reinterpret_cast<const uint32_t*>(&zl[j0 + g + 8][k + 2 * c]);
+        const uint32_t al2 = *reinterpret_cast<const uint32_t*>(&zl[j0 + g][k + 2 * c + 8]);
+        const uint32_t al3 = *reinterpret_cast<const uint32_t*>(&zl[j0 + g + 8][k + 2 * c + 8]);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          mma_16816(acc[jt][t], ah0, ah1, ah2, ah3, b[t][0], b[t][1]);
+          mma_16816(acc[jt][t], al0, al1, al2, al3, b[t][0], b[t][1]);
+        }
+      }
+    }
+  }
+  __syncthreads();  // the staging buffers become the partial tile
+#pragma unroll
+  for (int jt = 0; jt < JT; ++jt)
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int col = wc + 8 * t + 2 * c;
+      const int j0 = 16 * jt + g;
+      part[j0][col] = acc[jt][t][0];
+      part[j0][col + 1] = acc[jt][t][1];
+      part[j0 + 8][col] = acc[jt][t][2];
+      part[j0 + 8][col + 1] = acc[jt][t][3];
+    }
+  cluster_sync_all();
+  // rank q reduces columns [q*128/CS, (q+1)*128/CS) over ranks in order
+  const int cols_per = (128 + CS - 1) / CS;
+  const int cl0 = (int)rank * cols_per;
+  for (int i = threadIdx.x; i < cols_per * r; i += 128) {
+    const int cl = cl0 + i / r, j = i % r;
+    const int col = c0 + cl;
+    if (cl >= 128 || col >= P.C) continue;
+    float v = 0.f;
+    for (int q = 0; q < CS; ++q) v += ld_dsmem_f32(&part[j][cl], (uint32_t)q);
+    const long o = P.transpose ? (long)j * P.C + col : (long)col * r + j;
+    P.out[o] = P.scale * v;
+  }
+  cluster_sync_all();
+}
+
+// Grouped (routed) row products: one CTA per 128-row block of an expert segment (the grouped
+// GEMM's block list), rows sharing one expert e: out[p] = oscale * Y[p] Z_e^T and
+// la[p] = split(lscale * Y[p] Z_e^T), Z_e(j, k) = Z[e*zes + j*zj + k*zk]. CTAs past the block
+// count exit. 256 threads: warp w owns rows 16w .. 16w + 15 of the block.
+template <int NT>
+__global__ void __launch_bounds__(256) lora_rows_seg_kernel(const __nv_bfloat16* __restrict__ Y, long ldy, int Kin,
+                                                            const __nv_bfloat16* __restrict__ Z, long zj, long zk,
+                                                            long zes, const int* __restrict__ seg_off,
+                                                            const int* __restrict__ mblk_off, int E, int r, float oscale,
+                                                            float lscale, float* __restrict__ out,
+                                                            __nv_bfloat16* __restrict__ la, int RP) {
+  constexpr int RN = 8 * NT;
+  constexpr int SK = 128;
+  constexpr int ZS = SK + 8;
+  __shared__ __align__(16) __nv_bfloat16 zs[RN * ZS];
+  const int total = __ldg(mblk_off + E);
+  const int blk = blockIdx.x;
+  if (blk >= total) return;
+  int a = 0, b = E - 1;
+  while (a < b) {
+    const int mid = (a + b + 1) >> 1;
+    if (__ldg(mblk_off + mid) <= blk) a = mid; else b = mid - 1;
+  }
+  const int e = a;
+  const int row_lo = __ldg(seg_off + e) + (blk - __ldg(mblk_off + e)) * 128;
+  const int row_hi = min(__ldg(seg_off + e + 1), row_lo + 128);
+  const __nv_bfloat16* Ze = Z + (long)e * zes;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  const int r0 = row_lo + warp * 16 + g, r1 = r0 + 8;
+  const bool v0 = r0 < row_hi, v1 = r1 < row_hi;
+  const __nv_bfloat16* y0 = Y + (long)(v0 ? r0 : row_lo) * ldy;
+  const __nv_bfloat16* y1 = Y + (long)(v1 ? r1 : row_lo) * ldy;
+  float acc[NT][4];
+#pragma unroll
+  for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+  for (int k0 = 0; k0 < Kin; k0 += SK) {
+    const int nk = min(SK, Kin - k0);
+    uint4 xa[SK / 32], xb[SK / 32];
+#pragma unroll
+    for (int q = 0; q < SK / 32; ++q) {
+      const int k = k0 + 32 * q + 8 * c;
+      const bool in = 32 * q < nk;
+      xa[q] = (v0 && in) ? __ldg(reinterpret_cast<const uint4*>(y0 + k)) : make_uint4(0, 0, 0, 0);
+      xb[q] = (v1 && in) ? __ldg(reinterpret_cast<const uint4*>(y1 + k)) : make_uint4(0, 0, 0, 0);
+    }
+    __syncthreads();
+    if (zk == 1) {
+      for (int i = threadIdx.x; i < RN * (SK / 8); i += 256) {
+        const int j = i / (SK / 8), q = i % (SK / 8);
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (j < r && 8 * q < nk) v = __ldg(reinterpret_cast<const uint4*>(Ze + (long)j * zj + k0 + 8 * q));
+        *reinterpret_cast<uint4*>(zs + j * ZS + 8 * q) = v;
+      }
+    } else {
+      for (int i = threadIdx.x; i < RN * SK; i += 256) {
+        const int kk = i / RN, j = i % RN;
+        __nv_bfloat16 v = __float2bfloat16(0.f);
+        if (j < r && kk < nk) v = Ze[(long)j * zj + (long)(k0 + kk) * zk];
+        zs[j * ZS + kk] = v;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < SK / 32; ++q) {
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        const uint4 zq = *reinterpret_cast<const uint4*>(zs + (8 * t + g) * ZS + 32 * q + 8 * c);
+        mma_16816(acc[t], xa[q].x, xb[q].x, xa[q].y, xb[q].y, zq.x, zq.y);
+        mma_16816(acc[t], xa[q].z, xb[q].z, xa[q].w, xb[q].w, zq.z, zq.w);
+      }
+    }
+  }
+  // C fragment: rows r0 / r1, columns 8t + 2c (+1)
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int row = hh ? r1 : r0;
+      if (!(hh ? v1 : v0)) continue;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int j = 8 * t + 2 * c + q;
+        const float v = acc[t][2 * hh + q];
+        if (out != nullptr && j < r) out[(long)row * r + j] = oscale * v;
+        if (la != nullptr && j < RP) {
+          const float x = lscale * v;
+          const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+          const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+          la[(long)row * 2 * RP + j] = j < r ? hi : __float2bfloat16(0.f);
+          la[(long)row * 2 * RP + RP + j] = j < r ? lo : __float2bfloat16(0.f);
+        }
+      }
+    }
+  }
+  // padding columns of la beyond RN (RP > RN happens for r <= 16: RN = 16, RP = 32)
+  if (la != nullptr && RP > RN) {
+    for (int i = threadIdx.x; i < 128 * (RP - RN); i += 256) {
+      const int lr = i / (RP - RN), j = RN + i % (RP - RN);
+      const int row = row_lo + lr;
+      if (row < row_hi) {
+        la[(long)row * 2 * RP + j] = __float2bfloat16(0.f);
+        la[(long)row * 2 * RP + RP + j] = __float2bfloat16(0.f);
+      }
+    }
+  }
+}
+
+// LB[e][n] = [Z_e(n, :) | Z_e(n, :)] zero padded to 2*RP columns; Z_e(n, j) = Z[e*zes + n*zn + j*zjs].
+// One thread per 8 output columns.
+__global__ void lora_bop_vec_kernel(const __nv_bfloat16* __restrict__ Z, long zn, long zjs, long zes, int rows, int nexp,
+                                    int r, int RP, __nv_bfloat16* __restrict__ LB) {
+  const int per_row = 2 * RP / 8;
+  const long items = (long)nexp * rows * per_row;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < items; i += (long)gridDim.x * blockDim.x) {
+    const long rn = i / per_row;
+    const int j0 = (int)(i % per_row) * 8;
+    const int n = (int)(rn % rows);
+    const int e = (int)(rn / rows);
+    __nv_bfloat16 v[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int j = (j0 + q) % RP;
+      v[q] = j < r ? Z[(long)e * zes + (long)n * zn + (long)j * zjs] : __float2bfloat16(0.f);
+    }
+    *reinterpret_cast<uint4*>(LB + rn * 2 * RP + j0) = *reinterpret_cast<const uint4*>(v);
+  }
+}
+
 // LB[e*rows + n][j] = LB[..][RP + j] = Z(e, n, j) = Z[e*zes + n*zn + j*zjs] for j < r, else 0.
 __global__ void lora_bop_kernel(const __nv_bfloat16* __restrict__ Z, long zn, long zjs, long zes, int rows,
                                 int nexp, int r, int RP, __nv_bfloat16* __restrict__ LB) {
@@ -204,25 +842,36 @@ __global__ void colred_reduce_kernel(const float* __restrict__ part, int Ccols, 
   }
 }
 
-// Standalone dequant: one thread per 8 consecutive weights.
+// Standalone dequant. fp32 output: one thread per 8 consecutive weights (decode8); bf16 output:
+// one thread per 32-weight unit through the same decoder the tensor-core producers use.
 template <int QT>
 __global__ void gguf_dequant_kernel(const uint8_t* __restrict__ wq, long rows, long cols, void* __restrict__ out,
                                     int out_dtype) {
   const long groups_per_row = cols / 256;
   const long row_bytes = groups_per_row * QTraits<QT>::kGroupBytes;
-  const long total = rows * (cols / 8);
-  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total; i += (long)gridDim.x * blockDim.x) {
-    const long row = i / (cols / 8);
-    const long c8 = i % (cols / 8);  // chunk of 8 within the row
-    const uint8_t* g = wq + row * row_bytes + (c8 / 32) * QTraits<QT>::kGroupBytes;
-    float w[8];
-    decode8<QT>(g, (int)(c8 % 32), w);
-    if (out_dtype == QL_F32) {
+  if (out_dtype == QL_F32) {
+    const long total = rows * (cols / 8);
+    for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total; i += (long)gridDim.x * blockDim.x) {
+      const long row = i / (cols / 8);
+      const long c8 = i % (cols / 8);  // chunk of 8 within the row
+      const uint8_t* g = wq + row * row_bytes + (c8 / 32) * QTraits<QT>::kGroupBytes;
+      float w[8];
+      decode8<QT>(g, (int)(c8 % 32), w);
       float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + row * cols + c8 * 8);
       o[0] = make_float4(w[0], w[1], w[2], w[3]);
       o[1] = make_float4(w[4], w[5], w[6], w[7]);
-    } else {
-      *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out) + row * cols + c8 * 8) = pack_bf16x8(w);
+    }
+  } else {
+    const long total = rows * (cols / 32);
+    for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total; i += (long)gridDim.x * blockDim.x) {
+      const long row = i / (cols / 32);
+      const long u = i % (cols / 32);  // unit of 32 within the row
+      const uint8_t* g = wq + row * row_bytes + (u / 8) * QTraits<QT>::kGroupBytes;
+      uint4 v[4];
+      decode_unit_bf16<QT>(g, (int)(u % 8), v);
+      uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out) + row * cols + u * 32);
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) o[cc] = v[cc];
     }
   }
 }

@@ -8,9 +8,10 @@
 //   * TMA copies packed GGUF groups (256 weights of a row, 272 or 144 bytes) of W into a shared
 //     memory ring; dequant warps expand them to bf16 directly in the 128-byte-swizzled canonical
 //     UMMA layout of the B operand; the full-precision weight never exists in HBM.
-//   * Forward (TRANS = false): B[n, k] = deq(W)[n, k], K-major, tile 128 x 128.
-//     Input-gradient (TRANS = true): B[k, n] = deq(W)[n, k] with the reduction over W's rows; the
-//     same decode writes an MN-major tile, tile 128 x 256.
+//   * Forward (TRANS = false): B[n, k] = deq(W)[n, k], K-major. Input-gradient (TRANS = true):
+//     B[k, n] = deq(W)[n, k] with the reduction over W's rows; the same decode writes an MN-major
+//     tile. Tiles are BM x 128 with BM = 128 * MS: with MS = 2 every dequantized B tile feeds two
+//     M = 128 MMAs (two TMEM accumulators), halving the dequant work per FLOP.
 //   * The A operand (X or dY rows) arrives by TMA with the 128-byte swizzle.
 //   * One elected thread issues tcgen05.mma (bf16 x bf16 -> fp32) into a double-buffered TMEM
 //     accumulator; four epilogue warps drain it with tcgen05.ld while the next tile accumulates.
@@ -29,7 +30,6 @@ namespace qlora {
 
 enum EpiKind { EPI_STORE = 0, EPI_SWIGLU = 1, EPI_PAIR_OUT = 2, EPI_SWIGLU_BWD = 3 };
 
-constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kNumEpiWarps = 4;   // warps 0..3 (TMEM lane quadrants 0..3)
 constexpr int kWarpTmaA = 4;
@@ -45,7 +45,7 @@ struct GemmParams {
   int Kd;          // quantized reduction length
   int n_lora_kb;   // extra 64-wide LoRA k-blocks
   int num_n_tiles;
-  int num_m_blocks;  // dense mode: ceil(M / 128)
+  int num_m_blocks;  // dense mode: ceil(M / BM)
   // weight rows
   int w_rows_per_expert;  // rows of W per expert (grouped); 0 in dense mode
   int lb_rows_per_expert; // rows of the LoRA B operand per expert (grouped)
@@ -53,7 +53,7 @@ struct GemmParams {
   // grouped
   int E;                  // 0 = dense
   const int* seg_off;     // [E+1] first pair row of each expert
-  const int* mblk_off;    // [E+1] prefix sum of ceil(count_e / 128)
+  const int* mblk_off;    // [E+1] prefix sum of ceil(count_e / BM)
   // epilogue
   void* out;
   int out_dtype;
@@ -61,6 +61,7 @@ struct GemmParams {
   __nv_bfloat16* out_g;        // SWIGLU: g, u, h [M x I]; SWIGLU_BWD: d[g|u] [M x 2I] in out_g
   __nv_bfloat16* out_u;
   __nv_bfloat16* out_h;
+  __nv_bfloat16* out_lo;       // SWIGLU: h - bf16(h); SWIGLU_BWD: d[g|u] - bf16(d[g|u]) (nullable)
   const __nv_bfloat16* in_g;   // SWIGLU_BWD: saved g, u, h [M x I]
   const __nv_bfloat16* in_u;
   const __nv_bfloat16* in_h;
@@ -68,15 +69,16 @@ struct GemmParams {
   float* dw_part;              // SWIGLU_BWD: [M x num_n_tiles] partial <dh_u, h>
 };
 
-template <int QT, bool TRANS>
+template <int QT, bool TRANS, int MS>
 struct GemmCfg {
-  static constexpr int BN = TRANS ? 256 : 128;
+  static constexpr int BM = 128 * MS;
+  static constexpr int BN = 128;
   static constexpr int GB = QTraits<QT>::kGroupBytes;
-  static constexpr int A_BYTES = kBM * kBK * 2;              // 16 KB
-  static constexpr int B_BYTES = BN * kBK * 2;               // 16 / 32 KB
-  static constexpr int RAW_ROWS = TRANS ? 64 : 128;          // W rows per raw chunk
+  static constexpr int A_BYTES = BM * kBK * 2;               // 16 / 32 KB
+  static constexpr int B_BYTES = BN * kBK * 2;               // 16 KB
+  static constexpr int RAW_ROWS = TRANS ? 64 : 128;          // W rows per raw chunk (one group each)
   static constexpr int RAW_BYTES = RAW_ROWS * GB;
-  static constexpr int STAGES = TRANS ? 3 : 4;
+  static constexpr int STAGES = MS == 2 ? 3 : 4;
   static constexpr int RAW_SLOTS = TRANS ? (GB > 200 ? 4 : 6) : (GB > 200 ? 2 : 3);
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
@@ -85,7 +87,9 @@ struct GemmCfg {
   // barriers: full[S], empty[S], raw_full[R], raw_empty[R], tfull[2], tempty[2], drain, tmem ptr
   static constexpr int NUM_BARS = 2 * STAGES + 2 * RAW_SLOTS + 5;
   static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16 + 1024;  // + alignment slack
-  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int ACC_COLS = MS * BN;   // TMEM columns of one tile's accumulators
+  static constexpr int TMEM_COLS = 512;      // two tiles in flight
+  static_assert(2 * ACC_COLS <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(RAW_BYTES % 128 == 0, "raw slot alignment");
 };
@@ -97,12 +101,13 @@ struct TileInfo {
   int e;        // expert (0 in dense mode)
 };
 
+template <int BM>
 __device__ __forceinline__ bool gemm_tile(const GemmParams& p, int t, TileInfo& ti) {
   if (p.E == 0) {
     if (t >= p.num_m_blocks * p.num_n_tiles) return false;
     const int mb = t % p.num_m_blocks;
     ti.nb = t / p.num_m_blocks;
-    ti.row0 = mb * kBM;
+    ti.row0 = mb * BM;
     ti.row_end = p.M;
     ti.e = 0;
     return true;
@@ -118,8 +123,9 @@ __device__ __forceinline__ bool gemm_tile(const GemmParams& p, int t, TileInfo& 
     if (__ldg(p.mblk_off + mid) <= gm) lo = mid; else hi = mid - 1;
   }
   ti.e = lo;
-  ti.row0 = __ldg(p.seg_off + lo) + (gm - __ldg(p.mblk_off + lo)) * kBM;
-  ti.row_end = __ldg(p.seg_off + lo + 1);
+  ti.row0 = __ldg(p.seg_off + lo) + (gm - __ldg(p.mblk_off + lo)) * BM;
+  ti.row_end = min(__ldg(p.seg_off + lo + 1), p.M);  // rows past M are never written
+  if (ti.row0 < 0) ti.row0 = 0;
   return true;
 }
 
@@ -129,15 +135,138 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int sit
   return __all_sync(0xffffffffu, r);
 }
 
+// 8 fp32 values as a bf16 pair per value: hi = RNE_bf16(f), lo = RNE_bf16(f - hi).
+__device__ __forceinline__ void split_bf16x8(const float (&f)[8], uint4& hi, uint4& lo) {
+  float h[8], l[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    h[j] = __bfloat162float(__float2bfloat16_rn(f[j]));
+    l[j] = f[j] - h[j];
+  }
+  hi = pack_bf16x8(h);
+  lo = pack_bf16x8(l);
+}
+
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
 
-template <int QT, bool TRANS, int EPI>
+// Epilogue of one accumulator row block: this thread owns output row `row` (valid or not: the
+// TMEM loads are warp-collective) and reads BN fp32 columns starting at TMEM address tbase.
+template <int EPI, int BN>
+__device__ __forceinline__ void epilogue_rows(const GemmParams& p, const TileInfo& ti, int row, bool valid,
+                                              uint32_t tbase) {
+  if (EPI == EPI_STORE || EPI == EPI_PAIR_OUT) {
+    float wr = 1.0f;
+    if (EPI == EPI_PAIR_OUT && valid) wr = __ldg(p.row_w + row);
+#pragma unroll 1
+    for (int jc = 0; jc < BN / 32; ++jc) {
+      uint32_t v[32];
+      tmem_ld32(tbase + 32 * jc, v);
+      tmem_ld_wait();
+      const int col0 = ti.nb * BN + 32 * jc;
+      if (valid && col0 < p.Nd) {
+        if (p.out_dtype == QL_F32) {
+          float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (long)row * p.ldo + col0);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            o[i] = make_float4(wr * __uint_as_float(v[4 * i]), wr * __uint_as_float(v[4 * i + 1]),
+                               wr * __uint_as_float(v[4 * i + 2]), wr * __uint_as_float(v[4 * i + 3]));
+        } else {
+          uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + (long)row * p.ldo + col0);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            float f[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) f[j] = wr * __uint_as_float(v[8 * i + j]);
+            o[i] = pack_bf16x8(f);
+          }
+        }
+      }
+    }
+  } else if (EPI == EPI_SWIGLU) {
+    // tile columns [0, BN/2) are gate j = nb*BN/2 + c, [BN/2, BN) are up for the same j
+#pragma unroll 1
+    for (int jp = 0; jp < BN / 64; ++jp) {
+      uint32_t vg[32], vu[32];
+      tmem_ld32(tbase + 32 * jp, vg);
+      tmem_ld32(tbase + BN / 2 + 32 * jp, vu);
+      tmem_ld_wait();
+      const int j0 = ti.nb * (BN / 2) + 32 * jp;
+      if (valid && j0 < p.I) {
+        const long o = (long)row * p.I + j0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float g[8], u[8], h[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            g[j] = __uint_as_float(vg[8 * i + j]);
+            u[j] = __uint_as_float(vu[8 * i + j]);
+            h[j] = silu_f(g[j]) * u[j];
+          }
+          *reinterpret_cast<uint4*>(p.out_g + o + 8 * i) = pack_bf16x8(g);
+          *reinterpret_cast<uint4*>(p.out_u + o + 8 * i) = pack_bf16x8(u);
+          uint4 hh, hl;
+          split_bf16x8(h, hh, hl);
+          *reinterpret_cast<uint4*>(p.out_h + o + 8 * i) = hh;
+          if (p.out_lo != nullptr) *reinterpret_cast<uint4*>(p.out_lo + o + 8 * i) = hl;
+        }
+      }
+    }
+  } else if (EPI == EPI_SWIGLU_BWD) {
+    float wr = 0.0f, dwp = 0.0f;
+    if (valid) wr = __ldg(p.row_w + row);
+#pragma unroll 1
+    for (int jc = 0; jc < BN / 32; ++jc) {
+      uint32_t v[32];
+      tmem_ld32(tbase + 32 * jc, v);
+      tmem_ld_wait();
+      const int j0 = ti.nb * BN + 32 * jc;
+      if (valid && j0 < p.I) {
+        const long o = (long)row * p.I + j0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 gq = *reinterpret_cast<const uint4*>(p.in_g + o + 8 * i);
+          const uint4 uq = *reinterpret_cast<const uint4*>(p.in_u + o + 8 * i);
+          const uint4 hq = *reinterpret_cast<const uint4*>(p.in_h + o + 8 * i);
+          const __nv_bfloat16* gb = reinterpret_cast<const __nv_bfloat16*>(&gq);
+          const __nv_bfloat16* ub = reinterpret_cast<const __nv_bfloat16*>(&uq);
+          const __nv_bfloat16* hb = reinterpret_cast<const __nv_bfloat16*>(&hq);
+          float dg[8], du[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float a = __uint_as_float(v[8 * i + j]);
+            const float g = __bfloat162float(gb[j]);
+            const float u = __bfloat162float(ub[j]);
+            dwp = fmaf(a, __bfloat162float(hb[j]), dwp);
+            const float dh = wr * a;
+            const float sg = 1.0f / (1.0f + expf(-g));
+            dg[j] = dh * u * sg * (1.0f + g * (1.0f - sg));
+            du[j] = dh * g * sg;
+          }
+          const long od = (long)row * 2 * p.I + j0 + 8 * i;
+          uint4 gh, gl, uh, ul;
+          split_bf16x8(dg, gh, gl);
+          split_bf16x8(du, uh, ul);
+          *reinterpret_cast<uint4*>(p.out_g + od) = gh;
+          *reinterpret_cast<uint4*>(p.out_g + od + p.I) = uh;
+          if (p.out_lo != nullptr) {
+            *reinterpret_cast<uint4*>(p.out_lo + od) = gl;
+            *reinterpret_cast<uint4*>(p.out_lo + od + p.I) = ul;
+          }
+        }
+      }
+    }
+    if (valid) p.dw_part[(long)row * p.num_n_tiles + ti.nb] = dwp;
+  }
+}
+
+template <int QT, bool TRANS, int EPI, int MS>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     qgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
                  const __grid_constant__ CUtensorMap tmLA, const __grid_constant__ CUtensorMap tmLB,
                  const GemmParams p) {
-  using C = GemmCfg<QT, TRANS>;
+  using C = GemmCfg<QT, TRANS, MS>;
   constexpr int BN = C::BN;
+  constexpr int BM = C::BM;
   extern __shared__ uint8_t smem_raw_[];
   const uint32_t base_u32 = (smem_u32(smem_raw_) + 1023u) & ~1023u;
   uint8_t* smem = smem_raw_ + (base_u32 - smem_u32(smem_raw_));
@@ -188,7 +317,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
 
-  const int kb_main = TRANS ? p.Kd / kBK : p.Kd / kBK;
+  const int kb_main = p.Kd / kBK;
   const int kb_total = kb_main + p.n_lora_kb;
   const int groups = p.Kd / 256;  // forward: raw chunks per tile
 
@@ -200,7 +329,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int last_phase[8];
       for (int s = 0; s < C::STAGES; ++s) last_phase[s] = -1;
       TileInfo ti;
-      for (int t = blockIdx.x; ok && gemm_tile(p, t, ti); t += gridDim.x) {
+      for (int t = blockIdx.x; ok && gemm_tile<BM>(p, t, ti); t += gridDim.x) {
         for (int kb = 0; kb < kb_total; ++kb, ++it) {
           const int s = it % C::STAGES;
           const uint32_t ph = (it / C::STAGES) & 1;
@@ -238,7 +367,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int s = 0; s < C::RAW_SLOTS; ++s) last_phase[s] = -1;
       constexpr int GW = C::GB / 4;  // group width in 32-bit words
       TileInfo ti;
-      for (int t = blockIdx.x; ok && gemm_tile(p, t, ti); t += gridDim.x) {
+      for (int t = blockIdx.x; ok && gemm_tile<BM>(p, t, ti); t += gridDim.x) {
         const int wbase = ti.e * p.w_rows_per_expert;
         const int nchunks = TRANS ? kb_main : groups;
         for (int c = 0; c < nchunks; ++c, ++rc) {
@@ -248,7 +377,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           mbar_arrive_expect_tx(rfull_bar(s), C::RAW_BYTES);
           const uint32_t dst = sRaw + s * C::RAW_BYTES;
           if (TRANS) {
-            tma_load_2d(dst, &tmW, rfull_bar(s), ti.nb * GW, wbase + c * 64);
+            tma_load_2d(dst, &tmW, rfull_bar(s), (ti.nb >> 1) * GW, wbase + c * 64);
           } else {
             int y0, y1;
             if (EPI == EPI_SWIGLU) { y0 = wbase + ti.nb * 64; y1 = wbase + p.I + ti.nb * 64; }
@@ -271,13 +400,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       bool issued = false;
       TileInfo ti;
-      constexpr uint32_t idesc_main = idesc_bf16(kBM, BN, TRANS);
-      constexpr uint32_t idesc_kmaj = idesc_bf16(kBM, BN, false);
-      for (int t = blockIdx.x; ok && gemm_tile(p, t, ti); t += gridDim.x, ++tc) {
+      constexpr uint32_t idesc_main = idesc_bf16(128, BN, TRANS);
+      constexpr uint32_t idesc_kmaj = idesc_bf16(128, BN, false);
+      for (int t = blockIdx.x; ok && gemm_tile<BM>(p, t, ti); t += gridDim.x, ++tc) {
         const int buf = tc & 1;
         if (!mbar_wait(tempty_bar(buf), ((tc >> 1) & 1) ^ 1, 3)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + buf * BN;
+        const uint32_t d_tmem = tmem_base + buf * C::ACC_COLS;
         for (int kb = 0; kb < kb_total; ++kb, ++it) {
           const int s = it % C::STAGES;
           const uint32_t ph = (it / C::STAGES) & 1;
@@ -288,11 +417,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const bool kmaj = !TRANS || kb >= kb_main;
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k) {
-            const uint64_t ad = smem_desc_sw128(a0 + 32 * k, 16, 1024);
             uint64_t bd;
             if (kmaj) bd = smem_desc_sw128(b0 + 32 * k, 16, 1024);
-            else bd = smem_desc_sw128(b0 + 8192 * k, 1024, 4096);
-            umma_bf16(d_tmem, ad, bd, kmaj ? idesc_kmaj : idesc_main, (kb | k) != 0);
+            else bd = smem_desc_sw128(b0 + 4096 * k, 1024, 2048);
+#pragma unroll
+            for (int h = 0; h < MS; ++h) {
+              const uint64_t ad = smem_desc_sw128(a0 + h * 16384 + 32 * k, 16, 1024);
+              umma_bf16(d_tmem + h * BN, ad, bd, kmaj ? idesc_kmaj : idesc_main, (kb | k) != 0);
+            }
           }
           umma_commit(empty_bar(s));
           issued = true;
@@ -308,11 +440,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp >= kWarpDq0) {
     // ---------------- dequant workers ----------------
     const int dq = threadIdx.x - kWarpDq0 * 32;  // 0..255
-    const int dw = warp - kWarpDq0;
     int it = 0, rc = 0;
     bool ok = true;
     TileInfo ti;
-    for (int t = blockIdx.x; ok && gemm_tile(p, t, ti); t += gridDim.x) {
+    for (int t = blockIdx.x; ok && gemm_tile<BM>(p, t, ti); t += gridDim.x) {
       if (!TRANS) {
         for (int g = 0; ok && g < groups; ++g, ++rc) {
           const int rs = rc % C::RAW_SLOTS;
@@ -322,13 +453,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int s = it % C::STAGES;
             if (!warp_wait(empty_bar(s), ((it / C::STAGES) & 1) ^ 1, 6)) { ok = false; break; }
             uint8_t* sb = smem + C::OFF_B + s * C::B_BYTES;
-            const int c8 = dq & 7;
-            const int rb = dq >> 3;
+            {
+              // one 32-weight unit per thread: row dq/2, units 2*sub + (dq&1) of the group
+              const int row = dq >> 1;
+              const int uh = dq & 1;
+              uint4 v[4];
+              decode_unit_bf16<QT>(raw + row * C::GB, 2 * sub + uh, v);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int row = rb + 32 * i;
-              const uint4 v = decode8_bf16<QT>(raw + row * C::GB, 8 * sub + c8);
-              *reinterpret_cast<uint4*>(sb + row * 128 + ((c8 ^ (row & 7)) << 4)) = v;
+              for (int cc = 0; cc < 4; ++cc) {
+                const int c8 = 4 * uh + cc;
+                *reinterpret_cast<uint4*>(sb + row * 128 + ((c8 ^ (row & 7)) << 4)) = v[cc];
+              }
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -345,13 +480,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (!warp_wait(empty_bar(s), ((it / C::STAGES) & 1) ^ 1, 6)) { ok = false; break; }
           const uint8_t* raw = smem + C::OFF_RAW + rs * C::RAW_BYTES;
           uint8_t* sb = smem + C::OFF_B + s * C::B_BYTES;
-          const int gc = lane;
-#pragma unroll 4
-          for (int i = 0; i < 8; ++i) {
-            const int kk = dw + 8 * i;
-            const uint4 v = decode8_bf16<QT>(raw + kk * C::GB, gc);
-            const int off = (kk >> 3) * 4096 + (gc >> 3) * 1024 + (kk & 7) * 128 + (((gc & 7) ^ (kk & 7)) << 4);
-            *reinterpret_cast<uint4*>(sb + off) = v;
+          {
+            // one 32-column unit per thread: row kk = dq/4 of the chunk, unit 4*(nb&1) + dq%4 of
+            // the group (the tile's 128 columns are half of the 256-column group)
+            const int kk = dq >> 2, ul = dq & 3;
+            uint4 v[4];
+            decode_unit_bf16<QT>(raw + kk * C::GB, 4 * (ti.nb & 1) + ul, v);
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              const int gc = 4 * ul + cc;  // 16-byte chunk within the tile's 128 columns
+              const int off = (kk >> 3) * 2048 + (gc >> 3) * 1024 + (kk & 7) * 128 + (((gc & 7) ^ (kk & 7)) << 4);
+              *reinterpret_cast<uint4*>(sb + off) = v[cc];
+            }
           }
           fence_proxy_async_smem();
           __syncwarp();
@@ -373,105 +513,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ---------------- epilogue ----------------
     int tc = 0;
     TileInfo ti;
-    for (int t = blockIdx.x; gemm_tile(p, t, ti); t += gridDim.x, ++tc) {
+    for (int t = blockIdx.x; gemm_tile<BM>(p, t, ti); t += gridDim.x, ++tc) {
       const int buf = tc & 1;
       if (!warp_wait(tfull_bar(buf), (tc >> 1) & 1, 8)) break;
       tc_fence_after();
-      const int row = ti.row0 + warp * 32 + lane;
-      const bool valid = row < ti.row_end;
-      const uint32_t tbase = tmem_base + ((uint32_t)(warp * 32) << 16) + buf * BN;
-      if (EPI == EPI_STORE || EPI == EPI_PAIR_OUT) {
-        float wr = 1.0f;
-        if (EPI == EPI_PAIR_OUT && valid) wr = __ldg(p.row_w + row);
 #pragma unroll 1
-        for (int jc = 0; jc < BN / 32; ++jc) {
-          uint32_t v[32];
-          tmem_ld32(tbase + 32 * jc, v);
-          tmem_ld_wait();
-          const int col0 = ti.nb * BN + 32 * jc;
-          if (valid && col0 < p.Nd) {
-            if (p.out_dtype == QL_F32 && EPI == EPI_STORE) {
-              float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (long)row * p.ldo + col0);
-#pragma unroll
-              for (int i = 0; i < 8; ++i)
-                o[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                   __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-            } else {
-              uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + (long)row * p.ldo + col0);
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                float f[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) f[j] = wr * __uint_as_float(v[8 * i + j]);
-                o[i] = pack_bf16x8(f);
-              }
-            }
-          }
-        }
-      } else if (EPI == EPI_SWIGLU) {
-        // columns [0,64) of the tile are gate j = nb*64 + c, [64,128) are up for the same j
-#pragma unroll 1
-        for (int jp = 0; jp < 2; ++jp) {
-          uint32_t vg[32], vu[32];
-          tmem_ld32(tbase + 32 * jp, vg);
-          tmem_ld32(tbase + 64 + 32 * jp, vu);
-          tmem_ld_wait();
-          const int j0 = ti.nb * 64 + 32 * jp;
-          if (valid && j0 < p.I) {
-            const long o = (long)row * p.I + j0;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              float g[8], u[8], h[8];
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                g[j] = __uint_as_float(vg[8 * i + j]);
-                u[j] = __uint_as_float(vu[8 * i + j]);
-                h[j] = silu_f(g[j]) * u[j];
-              }
-              *reinterpret_cast<uint4*>(p.out_g + o + 8 * i) = pack_bf16x8(g);
-              *reinterpret_cast<uint4*>(p.out_u + o + 8 * i) = pack_bf16x8(u);
-              *reinterpret_cast<uint4*>(p.out_h + o + 8 * i) = pack_bf16x8(h);
-            }
-          }
-        }
-      } else if (EPI == EPI_SWIGLU_BWD) {
-        float wr = 0.0f, dwp = 0.0f;
-        if (valid) wr = __ldg(p.row_w + row);
-#pragma unroll 1
-        for (int jc = 0; jc < BN / 32; ++jc) {
-          uint32_t v[32];
-          tmem_ld32(tbase + 32 * jc, v);
-          tmem_ld_wait();
-          const int j0 = ti.nb * BN + 32 * jc;
-          if (valid && j0 < p.I) {
-            const long o = (long)row * p.I + j0;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const uint4 gq = *reinterpret_cast<const uint4*>(p.in_g + o + 8 * i);
-              const uint4 uq = *reinterpret_cast<const uint4*>(p.in_u + o + 8 * i);
-              const uint4 hq = *reinterpret_cast<const uint4*>(p.in_h + o + 8 * i);
-              const __nv_bfloat16* gb = reinterpret_cast<const __nv_bfloat16*>(&gq);
-              const __nv_bfloat16* ub = reinterpret_cast<const __nv_bfloat16*>(&uq);
-              const __nv_bfloat16* hb = reinterpret_cast<const __nv_bfloat16*>(&hq);
-              float dg[8], du[8];
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                const float a = __uint_as_float(v[8 * i + j]);
-                const float g = __bfloat162float(gb[j]);
-                const float u = __bfloat162float(ub[j]);
-                dwp = fmaf(a, __bfloat162float(hb[j]), dwp);
-                const float dh = wr * a;
-                const float sg = 1.0f / (1.0f + expf(-g));
-                dg[j] = dh * u * sg * (1.0f + g * (1.0f - sg));
-                du[j] = dh * g * sg;
-              }
-              const long od = (long)row * 2 * p.I + j0 + 8 * i;
-              *reinterpret_cast<uint4*>(p.out_g + od) = pack_bf16x8(dg);
-              *reinterpret_cast<uint4*>(p.out_g + od + p.I) = pack_bf16x8(du);
-            }
-          }
-        }
-        if (valid) p.dw_part[(long)row * p.num_n_tiles + ti.nb] = dwp;
+      for (int h = 0; h < MS; ++h) {
+        const int row = ti.row0 + h * 128 + warp * 32 + lane;
+        const bool valid = row < ti.row_end;
+        const uint32_t tbase = tmem_base + ((uint32_t)(warp * 32) << 16) + buf * C::ACC_COLS + h * BN;
+        epilogue_rows<EPI, BN>(p, ti, row, valid, tbase);
       }
       tc_fence_before();
       __syncwarp();

@@ -11,6 +11,7 @@
 #include "qlora.h"
 #include "lora.cuh"
 #include "qgemm.cuh"
+#include "moe.cuh"
 
 namespace qlora {
 
@@ -102,11 +103,11 @@ static inline int launch_status() {
 // ------------------------------------------------------------------------------------------------
 // Launch helpers
 // ------------------------------------------------------------------------------------------------
-template <int QT, bool TRANS, int EPI>
+template <int QT, bool TRANS, int EPI, int MS>
 static int launch_qgemm(const CUtensorMap& tA, const CUtensorMap& tW, const CUtensorMap& tLA, const CUtensorMap& tLB,
                         const GemmParams& p, int grid, cudaStream_t st, int slot) {
-  using C = GemmCfg<QT, TRANS>;
-  auto k = qgemm_kernel<QT, TRANS, EPI>;
+  using C = GemmCfg<QT, TRANS, MS>;
+  auto k = qgemm_kernel<QT, TRANS, EPI, MS>;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return QL_ERR_CUDA;
   ev_record(slot, 0, st);
@@ -116,23 +117,52 @@ static int launch_qgemm(const CUtensorMap& tA, const CUtensorMap& tW, const CUte
   return launch_status();
 }
 
-template <bool TRANS, int EPI>
+template <bool TRANS, int EPI, int MS>
 static int launch_qgemm_q(int qtype, const CUtensorMap& tA, const CUtensorMap& tW, const CUtensorMap& tLA,
                           const CUtensorMap& tLB, const GemmParams& p, int grid, cudaStream_t st, int slot) {
   switch (qtype) {
-    case QL_Q8_0: return launch_qgemm<QL_Q8_0, TRANS, EPI>(tA, tW, tLA, tLB, p, grid, st, slot);
-    case QL_Q4_0: return launch_qgemm<QL_Q4_0, TRANS, EPI>(tA, tW, tLA, tLB, p, grid, st, slot);
-    case QL_Q4_K: return launch_qgemm<QL_Q4_K, TRANS, EPI>(tA, tW, tLA, tLB, p, grid, st, slot);
+    case QL_Q8_0: return launch_qgemm<QL_Q8_0, TRANS, EPI, MS>(tA, tW, tLA, tLB, p, grid, st, slot);
+    case QL_Q4_0: return launch_qgemm<QL_Q4_0, TRANS, EPI, MS>(tA, tW, tLA, tLB, p, grid, st, slot);
+    case QL_Q4_K: return launch_qgemm<QL_Q4_K, TRANS, EPI, MS>(tA, tW, tLA, tLB, p, grid, st, slot);
     default: return QL_ERR_UNSUPPORTED;
   }
 }
 
+// Split-K configuration of the row reductions (H = X A^T, G = s dY B).
+static void rows_split(int M, int Kin, int ks_cap, int* KS, int* kchunk) {
+  const int mblocks = (M + 63) / 64;
+  int ks = (4 * 148 + mblocks - 1) / mblocks;
+  ks = std::max(1, std::min(std::min(ks, ks_cap), std::min(16, Kin / 256)));
+  int kc = (Kin + ks - 1) / ks;
+  kc = (kc + 15) / 16 * 16;
+  *kchunk = kc;
+  *KS = (Kin + kc - 1) / kc;
+}
+
+// out = oscale * Y Z^T (fp32 [M x r]) and la = split(lscale * Y Z^T); dense Z(j, k) = Z[j*zj + k*zk].
+// Grouped use (row_exp != NULL, per-row expert) goes through the CUDA-core kernel.
 static int launch_lora_rows(const __nv_bfloat16* Y, long ldy, int M, int Kin, const __nv_bfloat16* Z, long zj, long zk,
                             long zes, const int* row_exp, int r, float oscale, float lscale, float* out,
-                            __nv_bfloat16* la, cudaStream_t st) {
+                            __nv_bfloat16* la, float* part, cudaStream_t st, int ks_cap = 16) {
   const int RP = lora_rp(r);
+  if (M <= 0) return QL_OK;
+  if (row_exp == nullptr) {
+    int KS, kchunk;
+    rows_split(M, Kin, ks_cap, &KS, &kchunk);
+    dim3 grid((M + 63) / 64, KS);
+    const int NT = r <= 16 ? 2 : (r <= 32 ? 4 : 8);
+    if (NT == 2) lora_rows_mma_kernel<2><<<grid, 128, 0, st>>>(Y, ldy, M, Kin, kchunk, Z, zj, zk, r, part);
+    else if (NT == 4) lora_rows_mma_kernel<4><<<grid, 128, 0, st>>>(Y, ldy, M, Kin, kchunk, Z, zj, zk, r, part);
+    else lora_rows_mma_kernel<8><<<grid, 128, 0, st>>>(Y, ldy, M, Kin, kchunk, Z, zj, zk, r, part);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (launch_status() != QL_OK) return QL_ERR_CUDA;
+    const long total = (long)M * RP;
+    const int g2 = (int)std::min<long>((total + 255) / 256, 148L * 16);
+    lora_rows_reduce_kernel<<<g2, 256, 0, st>>>(part, KS, M, 8 * NT, r, oscale, lscale, out, la, RP);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return launch_status();
+  }
   const int grid = (M + 7) / 8;
-  if (grid == 0) return QL_OK;
   if (r <= 16)
     lora_rows_kernel<16><<<grid, 256, 0, st>>>(Y, ldy, M, Kin, Z, zj, zk, zes, row_exp, r, oscale, lscale, out, la, RP);
   else if (r <= 32)
@@ -140,6 +170,80 @@ static int launch_lora_rows(const __nv_bfloat16* Y, long ldy, int M, int Kin, co
   else
     lora_rows_kernel<64><<<grid, 256, 0, st>>>(Y, ldy, M, Kin, Z, zj, zk, zes, row_exp, r, oscale, lscale, out, la, RP);
   g_launches.fetch_add(1, std::memory_order_relaxed);
+  return launch_status();
+}
+
+// Dense row reduction with the in-cluster split-K sum: out = oscale * Y Z^T, la = split(lscale *
+// Y Z^T) and, in the same launch, LB = [Zb | Zb] (bop).
+static int launch_rows_dense(const __nv_bfloat16* Y, long ldy, int M, int Kin, const __nv_bfloat16* Z, long zj,
+                             long zk, int r, float oscale, float lscale, float* out, __nv_bfloat16* la, BopArgs bop,
+                             __nv_bfloat16* LB, cudaStream_t st) {
+  if (M <= 0) return QL_OK;
+  const int RP = lora_rp(r);
+  int KS = std::max(1, std::min(8, Kin / 32));
+  int kchunk = (Kin + KS - 1) / KS;
+  kchunk = (kchunk + 31) / 32 * 32;
+  KS = (Kin + kchunk - 1) / kchunk;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((M + 63) / 64, KS, 1);
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = KS;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
+  if (r <= 16)
+    e = cudaLaunchKernelEx(&cfg, lora_rows_cluster_kernel<2>, Y, ldy, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out,
+                           la, RP, bop, LB);
+  else if (r <= 32)
+    e = cudaLaunchKernelEx(&cfg, lora_rows_cluster_kernel<4>, Y, ldy, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out,
+                           la, RP, bop, LB);
+  else
+    e = cudaLaunchKernelEx(&cfg, lora_rows_cluster_kernel<8>, Y, ldy, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out,
+                           la, RP, bop, LB);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  return launch_status();
+}
+
+// Two dense column reductions in one launch (dB and dA of the backward).
+static int launch_colred_dense(const ColredProblem& p0, const ColredProblem& p1, int M, int r, cudaStream_t st) {
+  int CS = std::max(1, std::min(8, (M + 63) / 64));
+  int mchunk = (M + CS - 1) / CS;
+  mchunk = (mchunk + 63) / 64 * 64;
+  CS = (M + mchunk - 1) / mchunk;
+  const int nb0 = (p0.C + 127) / 128, nb1 = (p1.C + 127) / 128;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nb0 + nb1, CS, 1);
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = CS;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const int JT = (r + 15) / 16;
+  cudaError_t e;
+  if (JT == 1) e = cudaLaunchKernelEx(&cfg, colred_cluster_kernel<1>, p0, p1, nb0, M, r, mchunk);
+  else if (JT == 2) e = cudaLaunchKernelEx(&cfg, colred_cluster_kernel<2>, p0, p1, nb0, M, r, mchunk);
+  else if (JT == 3) e = cudaLaunchKernelEx(&cfg, colred_cluster_kernel<3>, p0, p1, nb0, M, r, mchunk);
+  else e = cudaLaunchKernelEx(&cfg, colred_cluster_kernel<4>, p0, p1, nb0, M, r, mchunk);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
   return launch_status();
 }
 
@@ -156,15 +260,14 @@ static int launch_lora_bop(const __nv_bfloat16* Z, long zn, long zjs, long zes, 
 // out = scale * sum over slices of Y[m, c] Z[m, j]
 static int launch_colred(const __nv_bfloat16* Y, long ldy, int Ccols, const float* Z, int r, int M, const float* zw,
                          const int* seg_off, const int* mblk_off, int E, int max_slices, float* part, float scale,
-                         int transpose, float* out, cudaStream_t st) {
+                         int transpose, float* out, cudaStream_t st, const __nv_bfloat16* Ylo = nullptr) {
   if (max_slices <= 0) return QL_OK;
-  dim3 grid((Ccols + 255) / 256, max_slices);
-  if (r <= 16)
-    colred_partial_kernel<16><<<grid, 128, 0, st>>>(Y, ldy, Ccols, Z, r, M, zw, seg_off, mblk_off, E, part);
-  else if (r <= 32)
-    colred_partial_kernel<32><<<grid, 128, 0, st>>>(Y, ldy, Ccols, Z, r, M, zw, seg_off, mblk_off, E, part);
-  else
-    colred_partial_kernel<64><<<grid, 128, 0, st>>>(Y, ldy, Ccols, Z, r, M, zw, seg_off, mblk_off, E, part);
+  dim3 grid((Ccols + 127) / 128, max_slices);
+  const int JT = (r + 15) / 16;
+  if (JT == 1) colred_mma_kernel<1><<<grid, 128, 0, st>>>(Y, ldy, Ccols, Z, r, M, zw, seg_off, mblk_off, E, part, Ylo);
+  else if (JT == 2) colred_mma_kernel<2><<<grid, 128, 0, st>>>(Y, ldy, Ccols, Z, r, M, zw, seg_off, mblk_off, E, part, Ylo);
+  else if (JT == 3) colred_mma_kernel<3><<<grid, 128, 0, st>>>(Y, ldy, Ccols, Z, r, M, zw, seg_off, mblk_off, E, part, Ylo);
+  else colred_mma_kernel<4><<<grid, 128, 0, st>>>(Y, ldy, Ccols, Z, r, M, zw, seg_off, mblk_off, E, part, Ylo);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (launch_status() != QL_OK) return QL_ERR_CUDA;
   const long total = (long)(E == 0 ? 1 : E) * Ccols * r;
@@ -176,7 +279,7 @@ static int launch_colred(const __nv_bfloat16* Y, long ldy, int Ccols, const floa
 
 // Workspace layout of the dense layer (byte offsets, 256-aligned).
 struct LinearWs {
-  size_t la, lb, g, part, total;
+  size_t la, lb, g, total;
 };
 static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 static LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int r) {
@@ -187,7 +290,6 @@ static LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int r) {
   w.la = o; o = al256(o + (size_t)M * KL * 2);
   w.lb = o; o = al256(o + (size_t)NK * KL * 2);
   w.g = o; o = al256(o + (size_t)M * r * 4);
-  w.part = o; o = al256(o + (size_t)((M + 127) / 128) * NK * r * 4);
   w.total = o;
   return w;
 }
@@ -202,6 +304,111 @@ static int check_linear(int qtype, const void* wq, int64_t N, int64_t K, const v
   if (M > (1 << 30) || N > (1 << 24) || K > (1 << 24)) return QL_ERR_SHAPE;
   if (!aligned16(wq) || !aligned16(X) || !aligned16(A) || !aligned16(B)) return QL_ERR_ALIGNMENT;
   return QL_OK;
+}
+
+// ------------------------------------------------------------------------------------------------
+// MoE: workspace / saved layouts and launch helpers
+// ------------------------------------------------------------------------------------------------
+struct MoeSaved {
+  size_t g, u, h, hlo, hgu, hd, total;
+};
+static MoeSaved moe_saved(int64_t T, int k, int64_t H, int64_t I, int r) {
+  (void)H;
+  const size_t P = (size_t)T * k;
+  MoeSaved m;
+  size_t o = 0;
+  m.g = o; o = al256(o + P * I * 2);
+  m.u = o; o = al256(o + P * I * 2);
+  m.h = o; o = al256(o + P * I * 2);
+  m.hlo = o; o = al256(o + P * I * 2);
+  m.hgu = o; o = al256(o + P * r * 4);
+  m.hd = o; o = al256(o + P * r * 4);
+  m.total = o;
+  return m;
+}
+
+struct MoeWs {
+  size_t xp, yp, row_w, la, lb, g1, g2, dgu, dgulo, dwp, dxp, part, total;
+};
+static int moe_max_slices(int64_t P, int E) { return (int)((P + 127) / 128 + E); }
+static MoeWs moe_ws(int64_t T, int k, int E, int64_t H, int64_t I, int r) {
+  const size_t P = (size_t)T * k;
+  const size_t KL = 2 * lora_rp(r);
+  const size_t HI = (size_t)std::max<int64_t>(H, 2 * I);
+  MoeWs w;
+  size_t o = 0;
+  w.xp = o; o = al256(o + P * H * 2);
+  w.yp = o; o = al256(o + P * H * 4);
+  w.row_w = o; o = al256(o + P * 4);
+  w.la = o; o = al256(o + P * KL * 2);
+  w.lb = o; o = al256(o + (size_t)E * HI * KL * 2);
+  w.g1 = o; o = al256(o + P * r * 4);
+  w.g2 = o; o = al256(o + P * r * 4);
+  w.dgu = o; o = al256(o + P * 2 * I * 2);
+  w.dgulo = o; o = al256(o + P * 2 * I * 2);
+  w.dwp = o; o = al256(o + P * (I / 128) * 4);
+  w.dxp = o; o = al256(o + P * H * 4);
+  w.part = o; o = al256(o + (size_t)moe_max_slices(P, E) * HI * r * 4);
+  w.total = o;
+  return w;
+}
+
+static int check_moe(int qtype, const void* w_gu, const void* w_d, int E, int64_t H, int64_t I, const void* X, int64_t T,
+                     int k, int r) {
+  if (!w_gu || !w_d || !X) return QL_ERR_INVALID_ARG;
+  if (group_bytes(qtype) == 0) return QL_ERR_UNSUPPORTED;
+  if (E < 1 || E > kMaxExperts || k < 1 || k > kMaxTopK || k > E) return QL_ERR_UNSUPPORTED;
+  if (r < 1 || r > 64) return QL_ERR_UNSUPPORTED;
+  if (T < 1 || H < 1 || I < 1) return QL_ERR_INVALID_ARG;
+  if (H % 256 != 0 || I % 256 != 0) return QL_ERR_SHAPE;
+  if (T * k > (1 << 28) || H > (1 << 16) || I > (1 << 16)) return QL_ERR_SHAPE;
+  if (!aligned16(w_gu) || !aligned16(w_d) || !aligned16(X)) return QL_ERR_ALIGNMENT;
+  return QL_OK;
+}
+
+static int launch_rows_seg(const __nv_bfloat16* Y, long ldy, int Kin, const __nv_bfloat16* Z, long zj, long zk, long zes,
+                           const int* seg_off, const int* mblk, int E, int r, float oscale, float lscale, float* out,
+                           __nv_bfloat16* la, int max_slices, cudaStream_t st) {
+  const int RP = lora_rp(r);
+  if (r <= 16)
+    lora_rows_seg_kernel<2><<<max_slices, 256, 0, st>>>(Y, ldy, Kin, Z, zj, zk, zes, seg_off, mblk, E, r, oscale, lscale,
+                                                        out, la, RP);
+  else if (r <= 32)
+    lora_rows_seg_kernel<4><<<max_slices, 256, 0, st>>>(Y, ldy, Kin, Z, zj, zk, zes, seg_off, mblk, E, r, oscale, lscale,
+                                                        out, la, RP);
+  else
+    lora_rows_seg_kernel<8><<<max_slices, 256, 0, st>>>(Y, ldy, Kin, Z, zj, zk, zes, seg_off, mblk, E, r, oscale, lscale,
+                                                        out, la, RP);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return launch_status();
+}
+
+static int launch_bop_vec(const __nv_bfloat16* Z, long zn, long zjs, long zes, int rows, int nexp, int r,
+                          __nv_bfloat16* LB, cudaStream_t st) {
+  const int RP = lora_rp(r);
+  const long items = (long)nexp * rows * (2 * RP / 8);
+  const int grid = (int)std::min<long>((items + 255) / 256, (long)num_sms() * 8);
+  lora_bop_vec_kernel<<<grid, 256, 0, st>>>(Z, zn, zjs, zes, rows, nexp, r, RP, LB);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return launch_status();
+}
+
+static int launch_gather(const __nv_bfloat16* src, int cols, const int32_t* perm, int P, int k, __nv_bfloat16* dst,
+                         const float* topk_w, float* row_w, cudaStream_t st) {
+  const long total = (long)P * (cols / 8);
+  const int grid = (int)std::min<long>((total + 255) / 256, (long)num_sms() * 16);
+  moe_gather_rows_kernel<<<grid, 256, 0, st>>>(src, cols, perm, P, k, dst, topk_w, row_w);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return launch_status();
+}
+
+static int launch_combine(const float* rows, int cols, const int32_t* inv_perm, int T, int k, void* out,
+                          int out_dtype, cudaStream_t st) {
+  const long total = (long)T * (cols / 4);
+  const int grid = (int)std::min<long>((total + 255) / 256, (long)num_sms() * 16);
+  moe_combine_kernel<<<grid, 256, 0, st>>>(rows, cols, inv_perm, T, k, out, out_dtype);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return launch_status();
 }
 
 }  // namespace qlora
@@ -294,17 +501,15 @@ int qlora_linear_fwd(int qtype, const void* wq, int64_t N, int64_t K, const void
   __nv_bfloat16* LB = (__nv_bfloat16*)(wsb + w.lb);
   const int KL = 2 * lora_rp(r);
 
-  // H = X A^T (saved) and the split operand of s*H
-  rc = launch_lora_rows((const __nv_bfloat16*)X, K, (int)M, (int)K, (const __nv_bfloat16*)A, K, 1, 0, nullptr, r,
-                        1.0f, scale, H, LA, st);
-  if (rc) return rc;
-  rc = launch_lora_bop((const __nv_bfloat16*)B, r, 1, 0, (int)N, 1, r, LB, st);
+  // H = X A^T (saved), the split operand of s*H, and LB = [B | B]
+  rc = launch_rows_dense((const __nv_bfloat16*)X, K, (int)M, (int)K, (const __nv_bfloat16*)A, K, 1, r, 1.0f, scale, H,
+                         LA, BopArgs{(const __nv_bfloat16*)B, r, 1, (int)N}, LB, st);
   if (rc) return rc;
 
   CUtensorMap tA, tW, tLA, tLB;
   const int64_t rb = packed_row_bytes(qtype, K);
-  if (!tmap_bf16_rows(&tA, X, K, M, 128) || !tmap_packed(&tW, wq, rb, N, group_bytes(qtype)) ||
-      !tmap_bf16_rows(&tLA, LA, KL, M, 128) || !tmap_bf16_rows(&tLB, LB, KL, N, 64))
+  if (!tmap_bf16_rows(&tA, X, K, M, 256) || !tmap_packed(&tW, wq, rb, N, group_bytes(qtype)) ||
+      !tmap_bf16_rows(&tLA, LA, KL, M, 256) || !tmap_bf16_rows(&tLB, LB, KL, N, 64))
     return QL_ERR_CUDA;
   GemmParams p;
   memset(&p, 0, sizeof(p));
@@ -313,13 +518,240 @@ int qlora_linear_fwd(int qtype, const void* wq, int64_t N, int64_t K, const void
   p.Kd = (int)K;
   p.n_lora_kb = KL / 64;
   p.num_n_tiles = (int)((N + 127) / 128);
-  p.num_m_blocks = (int)((M + 127) / 128);
+  p.num_m_blocks = (int)((M + 255) / 256);
   p.out = Y;
   p.out_dtype = y_dtype;
   p.ldo = N;
   const int tiles = p.num_n_tiles * p.num_m_blocks;
   const int grid = std::min(tiles, num_sms());
-  return launch_qgemm_q<false, EPI_STORE>(qtype, tA, tW, tLA, tLB, p, grid, st, 0);
+  return launch_qgemm_q<false, EPI_STORE, 2>(qtype, tA, tW, tLA, tLB, p, grid, st, 0);
+}
+
+int qlora_moe_route(const void* logits, int64_t T, int E, int k, int32_t* topk_idx, float* topk_w, int32_t* counts,
+                    int32_t* offsets, int32_t* perm, int32_t* inv_perm, int32_t* mblk, void* stream) {
+  if (!logits || !topk_idx || !topk_w || !counts || !offsets || !perm || !inv_perm || !mblk) return QL_ERR_INVALID_ARG;
+  if (E < 1 || E > kMaxExperts || k < 1 || k > kMaxTopK || k > E) return QL_ERR_UNSUPPORTED;
+  if (T < 1) return QL_ERR_INVALID_ARG;
+  const int EW = (E + 31) / 32;
+  if (T * EW > 50000) return QL_ERR_SHAPE;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int grid = (int)((T * 32 + 255) / 256);
+  moe_topk_kernel<<<grid, 256, 0, st>>>((const __nv_bfloat16*)logits, (int)T, E, k, topk_idx, topk_w);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (launch_status() != QL_OK) return QL_ERR_CUDA;
+  const size_t smem = (size_t)T * EW * 4;
+  if (cudaFuncSetAttribute(moe_permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return QL_ERR_CUDA;
+  moe_permute_kernel<<<1, 1024, smem, st>>>(topk_idx, (int)T, E, k, counts, offsets, mblk, perm, inv_perm);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return launch_status();
+}
+
+size_t qlora_moe_saved_bytes(int64_t T, int k, int64_t H, int64_t I, int r) {
+  if (T < 1 || k < 1 || H < 1 || I < 1 || r < 1 || r > 64) return 0;
+  return moe_saved(T, k, H, I, r).total;
+}
+
+size_t qlora_moe_workspace_bytes(int64_t T, int k, int E, int64_t H, int64_t I, int r) {
+  if (T < 1 || k < 1 || E < 1 || H < 1 || I < 1 || r < 1 || r > 64) return 0;
+  return moe_ws(T, k, E, H, I, r).total;
+}
+
+int qlora_moe_fwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H, int64_t I, const void* X, int64_t T,
+                  int k, const int32_t* topk_idx, const float* topk_w, const int32_t* offsets, const int32_t* perm,
+                  const int32_t* inv_perm, const int32_t* mblk, const void* A_gu, const void* B_gu, const void* A_d,
+                  const void* B_d, int r, float scale, void* Y, int y_dtype, void* saved, size_t saved_bytes, void* ws,
+                  size_t ws_bytes, void* stream) {
+  int rc = check_moe(qtype, w_gu, w_d, E, H, I, X, T, k, r);
+  if (rc) return rc;
+  if (!topk_idx || !topk_w || !offsets || !perm || !inv_perm || !mblk || !A_gu || !B_gu || !A_d || !B_d || !Y || !saved)
+    return QL_ERR_INVALID_ARG;
+  if (y_dtype != QL_F32 && y_dtype != QL_BF16) return QL_ERR_INVALID_ARG;
+  if (!aligned16(A_gu) || !aligned16(B_gu) || !aligned16(A_d) || !aligned16(B_d) || !aligned16(Y) || !aligned16(saved))
+    return QL_ERR_ALIGNMENT;
+  const MoeSaved sv = moe_saved(T, k, H, I, r);
+  const MoeWs w = moe_ws(T, k, E, H, I, r);
+  if (saved_bytes < sv.total) return QL_ERR_WORKSPACE;
+  if (!ws || ws_bytes < w.total) return QL_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QL_ERR_ALIGNMENT;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int P = (int)(T * k);
+  const int KL = 2 * lora_rp(r);
+  const int ms = moe_max_slices(P, E);
+  uint8_t* wb = (uint8_t*)ws;
+  uint8_t* sb = (uint8_t*)saved;
+  __nv_bfloat16* Xp = (__nv_bfloat16*)(wb + w.xp);
+  float* pair_out = (float*)(wb + w.yp);
+  float* row_w = (float*)(wb + w.row_w);
+  __nv_bfloat16* LA = (__nv_bfloat16*)(wb + w.la);
+  __nv_bfloat16* LB = (__nv_bfloat16*)(wb + w.lb);
+  __nv_bfloat16* g = (__nv_bfloat16*)(sb + sv.g);
+  __nv_bfloat16* u = (__nv_bfloat16*)(sb + sv.u);
+  __nv_bfloat16* h = (__nv_bfloat16*)(sb + sv.h);
+  float* Hgu = (float*)(sb + sv.hgu);
+  float* Hd = (float*)(sb + sv.hd);
+  const int* off = offsets;
+
+  rc = launch_gather((const __nv_bfloat16*)X, (int)H, perm, P, k, Xp, topk_w, row_w, st);
+  if (rc) return rc;
+  // gate/up: Hgu = Xp A_gu^T (saved), LA = split(s Hgu), LB = [B_gu | B_gu]
+  rc = launch_rows_seg(Xp, H, (int)H, (const __nv_bfloat16*)A_gu, H, 1, (long)r * H, off, mblk, E, r, 1.0f, scale, Hgu,
+                       LA, ms, st);
+  if (rc) return rc;
+  rc = launch_bop_vec((const __nv_bfloat16*)B_gu, r, 1, (long)2 * I * r, (int)(2 * I), E, r, LB, st);
+  if (rc) return rc;
+  const int nsm = num_sms();
+  {
+    CUtensorMap tA, tW, tLA, tLB;
+    if (!tmap_bf16_rows(&tA, Xp, H, P, 128) ||
+        !tmap_packed(&tW, w_gu, packed_row_bytes(qtype, H), (uint64_t)E * 2 * I, group_bytes(qtype)) ||
+        !tmap_bf16_rows(&tLA, LA, KL, P, 128) || !tmap_bf16_rows(&tLB, LB, KL, (uint64_t)E * 2 * I, 64))
+      return QL_ERR_CUDA;
+    GemmParams p;
+    memset(&p, 0, sizeof(p));
+    p.M = P; p.Nd = (int)(2 * I); p.Kd = (int)H; p.n_lora_kb = KL / 64; p.num_n_tiles = (int)(I / 64);
+    p.w_rows_per_expert = (int)(2 * I); p.lb_rows_per_expert = (int)(2 * I); p.I = (int)I;
+    p.E = E; p.seg_off = off; p.mblk_off = mblk;
+    p.out_g = g; p.out_u = u; p.out_h = h; p.out_lo = (__nv_bfloat16*)(sb + sv.hlo);
+    rc = launch_qgemm_q<false, EPI_SWIGLU, 1>(qtype, tA, tW, tLA, tLB, p, nsm, st, 2);
+    if (rc) return rc;
+  }
+  // down: Hd = h A_d^T (saved), LA = split(s Hd), LB = [B_d | B_d]
+  rc = launch_rows_seg(h, I, (int)I, (const __nv_bfloat16*)A_d, I, 1, (long)r * I, off, mblk, E, r, 1.0f, scale, Hd, LA,
+                       ms, st);
+  if (rc) return rc;
+  rc = launch_bop_vec((const __nv_bfloat16*)B_d, r, 1, (long)H * r, (int)H, E, r, LB, st);
+  if (rc) return rc;
+  {
+    CUtensorMap tA, tW, tLA, tLB;
+    if (!tmap_bf16_rows(&tA, h, I, P, 128) ||
+        !tmap_packed(&tW, w_d, packed_row_bytes(qtype, I), (uint64_t)E * H, group_bytes(qtype)) ||
+        !tmap_bf16_rows(&tLA, LA, KL, P, 128) || !tmap_bf16_rows(&tLB, LB, KL, (uint64_t)E * H, 64))
+      return QL_ERR_CUDA;
+    GemmParams p;
+    memset(&p, 0, sizeof(p));
+    p.M = P; p.Nd = (int)H; p.Kd = (int)I; p.n_lora_kb = KL / 64; p.num_n_tiles = (int)(H / 128);
+    p.w_rows_per_expert = (int)H; p.lb_rows_per_expert = (int)H; p.I = (int)I;
+    p.E = E; p.seg_off = off; p.mblk_off = mblk;
+    p.out = pair_out; p.out_dtype = QL_F32; p.ldo = H; p.row_w = row_w;
+    rc = launch_qgemm_q<false, EPI_PAIR_OUT, 1>(qtype, tA, tW, tLA, tLB, p, nsm, st, 3);
+    if (rc) return rc;
+  }
+  return launch_combine(pair_out, (int)H, inv_perm, (int)T, k, Y, y_dtype, st);
+}
+
+int qlora_moe_bwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H, int64_t I, const void* X, const void* dY,
+                  int64_t T, int k, const int32_t* topk_idx, const float* topk_w, const int32_t* offsets,
+                  const int32_t* perm, const int32_t* inv_perm, const int32_t* mblk, const void* A_gu, const void* B_gu,
+                  const void* A_d, const void* B_d, int r, float scale, const void* saved, size_t saved_bytes, void* dX,
+                  int dx_dtype, float* dA_gu, float* dB_gu, float* dA_d, float* dB_d, float* d_logits, void* ws,
+                  size_t ws_bytes, void* stream) {
+  int rc = check_moe(qtype, w_gu, w_d, E, H, I, X, T, k, r);
+  if (rc) return rc;
+  if (!dY || !topk_idx || !topk_w || !offsets || !perm || !inv_perm || !mblk || !A_gu || !B_gu || !A_d || !B_d ||
+      !saved || !dX || !dA_gu || !dB_gu || !dA_d || !dB_d)
+    return QL_ERR_INVALID_ARG;
+  if (dx_dtype != QL_F32 && dx_dtype != QL_BF16) return QL_ERR_INVALID_ARG;
+  if (!aligned16(dY) || !aligned16(dX) || !aligned16(saved) || !aligned16(dA_gu) || !aligned16(dB_gu) ||
+      !aligned16(dA_d) || !aligned16(dB_d) || (d_logits && !aligned16(d_logits)))
+    return QL_ERR_ALIGNMENT;
+  const MoeSaved sv = moe_saved(T, k, H, I, r);
+  const MoeWs w = moe_ws(T, k, E, H, I, r);
+  if (saved_bytes < sv.total) return QL_ERR_WORKSPACE;
+  if (!ws || ws_bytes < w.total) return QL_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QL_ERR_ALIGNMENT;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int P = (int)(T * k);
+  const int KL = 2 * lora_rp(r);
+  const int ms = moe_max_slices(P, E);
+  uint8_t* wb = (uint8_t*)ws;
+  const uint8_t* sb = (const uint8_t*)saved;
+  __nv_bfloat16* Xp = (__nv_bfloat16*)(wb + w.xp);
+  __nv_bfloat16* dYp = (__nv_bfloat16*)(wb + w.yp);
+  float* row_w = (float*)(wb + w.row_w);
+  __nv_bfloat16* LA = (__nv_bfloat16*)(wb + w.la);
+  __nv_bfloat16* LB = (__nv_bfloat16*)(wb + w.lb);
+  float* Gd = (float*)(wb + w.g1);
+  float* Ggu = (float*)(wb + w.g2);
+  __nv_bfloat16* dgu = (__nv_bfloat16*)(wb + w.dgu);
+  __nv_bfloat16* dgu_lo = (__nv_bfloat16*)(wb + w.dgulo);
+  float* dwp = (float*)(wb + w.dwp);
+  float* dxp = (float*)(wb + w.dxp);
+  float* part = (float*)(wb + w.part);
+  const __nv_bfloat16* g = (const __nv_bfloat16*)(sb + sv.g);
+  const __nv_bfloat16* u = (const __nv_bfloat16*)(sb + sv.u);
+  const __nv_bfloat16* h = (const __nv_bfloat16*)(sb + sv.h);
+  const __nv_bfloat16* h_lo = (const __nv_bfloat16*)(sb + sv.hlo);
+  const float* Hgu = (const float*)(sb + sv.hgu);
+  const float* Hd = (const float*)(sb + sv.hd);
+  const int* off = offsets;
+  const int nsm = num_sms();
+
+  rc = launch_gather((const __nv_bfloat16*)X, (int)H, perm, P, k, Xp, topk_w, row_w, st);
+  if (rc) return rc;
+  rc = launch_gather((const __nv_bfloat16*)dY, (int)H, perm, P, k, dYp, nullptr, nullptr, st);
+  if (rc) return rc;
+  // down input-gradient: Gd = s dYp B_d, LA = split(Gd), LB[e][i] = [A_d^T | A_d^T]
+  rc = launch_rows_seg(dYp, H, (int)H, (const __nv_bfloat16*)B_d, 1, r, (long)H * r, off, mblk, E, r, scale, scale, Gd,
+                       LA, ms, st);
+  if (rc) return rc;
+  rc = launch_bop_vec((const __nv_bfloat16*)A_d, 1, I, (long)r * I, (int)I, E, r, LB, st);
+  if (rc) return rc;
+  {
+    CUtensorMap tA, tW, tLA, tLB;
+    if (!tmap_bf16_rows(&tA, dYp, H, P, 128) ||
+        !tmap_packed(&tW, w_d, packed_row_bytes(qtype, I), (uint64_t)E * H, group_bytes(qtype)) ||
+        !tmap_bf16_rows(&tLA, LA, KL, P, 128) || !tmap_bf16_rows(&tLB, LB, KL, (uint64_t)E * I, 64))
+      return QL_ERR_CUDA;
+    GemmParams p;
+    memset(&p, 0, sizeof(p));
+    p.M = P; p.Nd = (int)I; p.Kd = (int)H; p.n_lora_kb = KL / 64; p.num_n_tiles = (int)(I / 128);
+    p.w_rows_per_expert = (int)H; p.lb_rows_per_expert = (int)I; p.I = (int)I;
+    p.E = E; p.seg_off = off; p.mblk_off = mblk;
+    p.in_g = g; p.in_u = u; p.in_h = h; p.out_g = dgu; p.out_lo = dgu_lo; p.row_w = row_w; p.dw_part = dwp;
+    rc = launch_qgemm_q<true, EPI_SWIGLU_BWD, 1>(qtype, tA, tW, tLA, tLB, p, nsm, st, 4);
+    if (rc) return rc;
+  }
+  // down adapter gradients: dA_d = sum_p w_p Gd_p^T h_p ; dB_d = s sum_p w_p dYp_p^T Hd_p
+  rc = launch_colred(h, I, (int)I, Gd, r, P, row_w, off, mblk, E, ms, part, 1.0f, 1, dA_d, st, h_lo);
+  if (rc) return rc;
+  rc = launch_colred(dYp, H, (int)H, Hd, r, P, row_w, off, mblk, E, ms, part, scale, 0, dB_d, st);
+  if (rc) return rc;
+  // gate/up input-gradient: Ggu = s dgu B_gu, LA = split(Ggu), LB[e][hh] = [A_gu^T | A_gu^T]
+  rc = launch_rows_seg(dgu, 2 * I, (int)(2 * I), (const __nv_bfloat16*)B_gu, 1, r, (long)2 * I * r, off, mblk, E, r,
+                       scale, scale, Ggu, LA, ms, st);
+  if (rc) return rc;
+  rc = launch_bop_vec((const __nv_bfloat16*)A_gu, 1, H, (long)r * H, (int)H, E, r, LB, st);
+  if (rc) return rc;
+  {
+    CUtensorMap tA, tW, tLA, tLB;
+    if (!tmap_bf16_rows(&tA, dgu, 2 * I, P, 128) ||
+        !tmap_packed(&tW, w_gu, packed_row_bytes(qtype, H), (uint64_t)E * 2 * I, group_bytes(qtype)) ||
+        !tmap_bf16_rows(&tLA, LA, KL, P, 128) || !tmap_bf16_rows(&tLB, LB, KL, (uint64_t)E * H, 64))
+      return QL_ERR_CUDA;
+    GemmParams p;
+    memset(&p, 0, sizeof(p));
+    p.M = P; p.Nd = (int)H; p.Kd = (int)(2 * I); p.n_lora_kb = KL / 64; p.num_n_tiles = (int)(H / 128);
+    p.w_rows_per_expert = (int)(2 * I); p.lb_rows_per_expert = (int)H; p.I = (int)I;
+    p.E = E; p.seg_off = off; p.mblk_off = mblk;
+    p.out = dxp; p.out_dtype = QL_F32; p.ldo = H;
+    rc = launch_qgemm_q<true, EPI_STORE, 1>(qtype, tA, tW, tLA, tLB, p, nsm, st, 5);
+    if (rc) return rc;
+  }
+  rc = launch_combine(dxp, (int)H, inv_perm, (int)T, k, dX, dx_dtype, st);
+  if (rc) return rc;
+  // gate/up adapter gradients: dA_gu = sum_p Ggu_p^T Xp_p ; dB_gu = s sum_p dgu_p^T Hgu_p
+  rc = launch_colred(Xp, H, (int)H, Ggu, r, P, nullptr, off, mblk, E, ms, part, 1.0f, 1, dA_gu, st);
+  if (rc) return rc;
+  rc = launch_colred(dgu, 2 * I, (int)(2 * I), Hgu, r, P, nullptr, off, mblk, E, ms, part, scale, 0, dB_gu, st, dgu_lo);
+  if (rc) return rc;
+  if (d_logits != nullptr) {
+    moe_dw_dlogits_kernel<<<(int)((T + 127) / 128), 128, 0, st>>>(dwp, (int)(I / 128), inv_perm, topk_idx, topk_w,
+                                                                  (int)T, E, k, nullptr, d_logits);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return launch_status();
+  }
+  return QL_OK;
 }
 
 int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void* X, const void* dY, int64_t M,
@@ -339,22 +771,17 @@ int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void
   __nv_bfloat16* LA = (__nv_bfloat16*)(wsb + w.la);
   __nv_bfloat16* LB = (__nv_bfloat16*)(wsb + w.lb);
   float* G = (float*)(wsb + w.g);
-  float* part = (float*)(wsb + w.part);
   const int KL = 2 * lora_rp(r);
-  const int slices = (int)((M + 127) / 128);
 
-  // G = s dY B (kept in fp32) and its split operand
-  rc = launch_lora_rows((const __nv_bfloat16*)dY, N, (int)M, (int)N, (const __nv_bfloat16*)B, 1, r, 0, nullptr, r,
-                        scale, scale, G, LA, st);
+  // G = s dY B (kept in fp32), its split operand, and LB[k] = [A^T(k) | A^T(k)]
+  rc = launch_rows_dense((const __nv_bfloat16*)dY, N, (int)M, (int)N, (const __nv_bfloat16*)B, 1, r, r, scale, scale, G,
+                         LA, dX ? BopArgs{(const __nv_bfloat16*)A, 1, K, (int)K} : BopArgs{nullptr, 0, 0, 0}, LB, st);
   if (rc) return rc;
   if (dX) {
-    // LB[k] = [A^T(k) | A^T(k)]
-    rc = launch_lora_bop((const __nv_bfloat16*)A, 1, K, 0, (int)K, 1, r, LB, st);
-    if (rc) return rc;
     CUtensorMap tA, tW, tLA, tLB;
     const int64_t rb = packed_row_bytes(qtype, K);
-    if (!tmap_bf16_rows(&tA, dY, N, M, 128) || !tmap_packed(&tW, wq, rb, N, group_bytes(qtype)) ||
-        !tmap_bf16_rows(&tLA, LA, KL, M, 128) || !tmap_bf16_rows(&tLB, LB, KL, K, 64))
+    if (!tmap_bf16_rows(&tA, dY, N, M, 256) || !tmap_packed(&tW, wq, rb, N, group_bytes(qtype)) ||
+        !tmap_bf16_rows(&tLA, LA, KL, M, 256) || !tmap_bf16_rows(&tLB, LB, KL, K, 64))
       return QL_ERR_CUDA;
     GemmParams p;
     memset(&p, 0, sizeof(p));
@@ -362,22 +789,19 @@ int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void
     p.Nd = (int)K;
     p.Kd = (int)N;
     p.n_lora_kb = KL / 64;
-    p.num_n_tiles = (int)(K / 256);
-    p.num_m_blocks = slices;
+    p.num_n_tiles = (int)(K / 128);
+    p.num_m_blocks = (int)((M + 255) / 256);
     p.out = dX;
     p.out_dtype = dx_dtype;
     p.ldo = K;
     const int tiles = p.num_n_tiles * p.num_m_blocks;
-    rc = launch_qgemm_q<true, EPI_STORE>(qtype, tA, tW, tLA, tLB, p, std::min(tiles, num_sms()), st, 1);
+    rc = launch_qgemm_q<true, EPI_STORE, 2>(qtype, tA, tW, tLA, tLB, p, std::min(tiles, num_sms()), st, 1);
     if (rc) return rc;
   }
-  // dB = s dY^T H ; dA = G^T X
-  rc = launch_colred((const __nv_bfloat16*)dY, N, (int)N, H, r, (int)M, nullptr, nullptr, nullptr, 0, slices, part,
-                     scale, 0, dB, st);
-  if (rc) return rc;
-  rc = launch_colred((const __nv_bfloat16*)X, K, (int)K, G, r, (int)M, nullptr, nullptr, nullptr, 0, slices, part,
-                     1.0f, 1, dA, st);
-  return rc;
+  // dB = s dY^T H and dA = G^T X in one launch
+  const ColredProblem pb{(const __nv_bfloat16*)dY, N, (int)N, H, scale, 0, dB};
+  const ColredProblem pa{(const __nv_bfloat16*)X, K, (int)K, G, 1.0f, 1, dA};
+  return launch_colred_dense(pb, pa, (int)M, r, st);
 }
 
 }  // extern "C"
@@ -423,8 +847,8 @@ extern "C" int qlora_linear_fwd_noalloc(int qtype, const void* wq, int64_t N, in
   if (!aligned16(Y) || !aligned16(H)) return QL_ERR_ALIGNMENT;
   const int KL = 2 * lora_rp(r);
   const size_t la_bytes = al256((size_t)M * KL * 2);
-  const size_t need = la_bytes + (size_t)N * KL * 2;
-  if (need > kStaticScratchBytes) return QL_ERR_WORKSPACE;
+  const size_t lb_bytes = al256((size_t)N * KL * 2);
+  if (la_bytes + lb_bytes > kStaticScratchBytes) return QL_ERR_WORKSPACE;
   void* base = nullptr;
   rc = static_scratch_address(&base);
   if (rc != QL_OK) return rc;
@@ -434,15 +858,13 @@ extern "C" int qlora_linear_fwd_noalloc(int qtype, const void* wq, int64_t N, in
   __nv_bfloat16* LA = (__nv_bfloat16*)base;
   __nv_bfloat16* LB = (__nv_bfloat16*)((uint8_t*)base + la_bytes);
 
-  rc = launch_lora_rows((const __nv_bfloat16*)X, K, (int)M, (int)K, (const __nv_bfloat16*)A, K, 1, 0, nullptr, r,
-                        1.0f, scale, H, LA, st);
-  if (rc) return rc;
-  rc = launch_lora_bop((const __nv_bfloat16*)B, r, 1, 0, (int)N, 1, r, LB, st);
+  rc = launch_rows_dense((const __nv_bfloat16*)X, K, (int)M, (int)K, (const __nv_bfloat16*)A, K, 1, r, 1.0f, scale, H,
+                         LA, BopArgs{(const __nv_bfloat16*)B, r, 1, (int)N}, LB, st);
   if (rc) return rc;
   CUtensorMap tA, tW, tLA, tLB;
   const int64_t rb = packed_row_bytes(qtype, K);
-  if (!tmap_bf16_rows(&tA, X, K, M, 128) || !tmap_packed(&tW, wq, rb, N, group_bytes(qtype)) ||
-      !tmap_bf16_rows(&tLA, LA, KL, M, 128) || !tmap_bf16_rows(&tLB, LB, KL, N, 64))
+  if (!tmap_bf16_rows(&tA, X, K, M, 256) || !tmap_packed(&tW, wq, rb, N, group_bytes(qtype)) ||
+      !tmap_bf16_rows(&tLA, LA, KL, M, 256) || !tmap_bf16_rows(&tLB, LB, KL, N, 64))
     return QL_ERR_CUDA;
   GemmParams p;
   memset(&p, 0, sizeof(p));
@@ -451,10 +873,10 @@ extern "C" int qlora_linear_fwd_noalloc(int qtype, const void* wq, int64_t N, in
   p.Kd = (int)K;
   p.n_lora_kb = KL / 64;
   p.num_n_tiles = (int)((N + 127) / 128);
-  p.num_m_blocks = (int)((M + 127) / 128);
+  p.num_m_blocks = (int)((M + 255) / 256);
   p.out = Y;
   p.out_dtype = y_dtype;
   p.ldo = N;
   const int tiles = p.num_n_tiles * p.num_m_blocks;
-  return launch_qgemm_q<false, EPI_STORE>(qtype, tA, tW, tLA, tLB, p, std::min(tiles, num_sms()), st, 0);
+  return launch_qgemm_q<false, EPI_STORE, 2>(qtype, tA, tW, tLA, tLB, p, std::min(tiles, num_sms()), st, 0);
 }
