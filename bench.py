@@ -45,6 +45,8 @@ WORKLOADS = {
     "dense_q8_0": ("dense_proj_q8_0_2048x4096x4096_r16", lambda seed: inp.dense_proj_2048x4096x4096(inp.Q8_0, seed)),
     "dense_q4_0": ("dense_proj_q4_0_2048x4096x4096_r16", lambda seed: inp.dense_proj_2048x4096x4096(inp.Q4_0, seed)),
     "gate_up_q4_k": ("gate_up_q4_k_2048x2048x12288_r8", lambda seed: inp.gate_up_q4_k_2048x2048x12288(seed)),
+    "decode_q4_0_m1": ("decode_q4_0_1x8192x8192_r4", lambda seed: inp.decode_q4_0_8192(1, seed)),
+    "decode_q4_0_m16": ("decode_q4_0_16x8192x8192_r4", lambda seed: inp.decode_q4_0_8192(16, seed)),
 }
 
 
@@ -186,6 +188,124 @@ class DenseLayerRun:
         return 2.0 * c.M * c.N * c.K + 2.0 * c.M * c.r * (c.N if slot == 0 else c.K)
 
 
+class MoERun:
+    """Device buffers and one step (route + forward + backward) of the routed MoE layer."""
+
+    def __init__(self, case):
+        import quantized_base_lora_tma_b200 as ql
+        self.ql = ql
+        self.c = c = case
+        T, H, I, E, k, r = c.T, c.H, c.I, c.E, c.k, c.r
+        self.X, self.dY, self.logits = bf16_dev(c.X), bf16_dev(c.dY), bf16_dev(c.logits)
+        self.w_gu = torch.from_numpy(c.w_gu).cuda()
+        self.w_d = torch.from_numpy(c.w_d).cuda()
+        self.A_gu, self.B_gu = bf16_dev(c.A_gu), bf16_dev(c.B_gu)
+        self.A_d, self.B_d = bf16_dev(c.A_d), bf16_dev(c.B_d)
+        self.route = ql.MoeRoute(T, E, k)
+        self.saved = torch.empty(ql.qlora_moe_saved_bytes(T, k, H, I, r), dtype=torch.uint8, device="cuda")
+        self.ws = torch.empty(ql.qlora_moe_workspace_bytes(T, k, E, H, I, r), dtype=torch.uint8, device="cuda")
+        f32 = dict(dtype=torch.float32, device="cuda")
+        self.Y = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+        self.dX = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+        self.dA_gu = torch.empty(E, r, H, **f32)
+        self.dB_gu = torch.empty(E, 2 * I, r, **f32)
+        self.dA_d = torch.empty(E, r, I, **f32)
+        self.dB_d = torch.empty(E, H, r, **f32)
+        self.dL = torch.empty(T, E, **f32)
+
+    def step(self):
+        c, ql = self.c, self.ql
+        ql.qlora_moe_route(self.logits, c.k, self.route)
+        ql.qlora_moe_fwd(c.qtype, self.w_gu, self.w_d, c.E, c.H, c.I, self.X, self.route, self.A_gu, self.B_gu,
+                         self.A_d, self.B_d, c.r, c.scale, self.Y, self.saved, self.ws)
+        ql.qlora_moe_bwd(c.qtype, self.w_gu, self.w_d, c.E, c.H, c.I, self.X, self.dY, self.route, self.A_gu,
+                         self.B_gu, self.A_d, self.B_d, c.r, c.scale, self.saved, self.dX, self.dA_gu, self.dB_gu,
+                         self.dA_d, self.dB_d, self.dL, self.ws)
+
+    def flops(self):
+        c = self.c
+        P = c.T * c.k
+        return 12.0 * P * c.H * c.I + 6.0 * c.r * (2 * c.H + 3 * c.I) * P
+
+
+def time_steps(fn, steps, warmup, flush, slots=()):
+    """Mean device time (ms) of fn() over `steps` calls, L2 flushed before each; per-slot GEMM means."""
+    import quantized_base_lora_tma_b200 as ql
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    gev = {s: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+           for s in slots}
+    for i in range(steps):
+        flush.zero_()
+        for s in slots:
+            ql.qlora_set_kernel_events(s, gev[s][i][0], gev[s][i][1])
+        ev[i][0].record(stream)
+        fn()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    for s in slots:
+        ql.qlora_set_kernel_events(s, None, None)
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    return ms, {s: statistics.mean(a.elapsed_time(b) for a, b in gev[s]) for s in slots}
+
+
+def device_status_ok(where):
+    import quantized_base_lora_tma_b200 as ql
+    st, site = ql.qlora_device_status(reset=True)
+    if st != 0:
+        raise RuntimeError(f"device status {st} (wait site {site}) after {where}")
+
+
+def also_measurements(flush, steps, pk):
+    """Single-GPU measurements of the other shapes of the benchmark set (not the headline)."""
+    out = {}
+    # routed MoE layer, fwd + bwd incl. routing
+    c = inp.moe_q4_0_2048tok_128x768()
+    m = MoERun(c)
+    ms, g = time_steps(m.step, max(5, steps // 4), 3, flush, slots=(2, 3, 4, 5))
+    tf = m.flops() / (ms / 1e3) / 1e12
+    out["moe_q4_0_T2048_H2048_E128_I768_k8_r4"] = {
+        "tokens_per_s": c.T / (ms / 1e3), "ms_per_step": ms, "tflops": tf, "frac_of_bf16_peak": tf / pk["bf16_tflops"],
+        "gemm_ms": {"gate_up": g[2], "down": g[3], "down_dx": g[4], "gate_up_dx": g[5]},
+        "experts_touched": int((m.route.counts > 0).sum().item())}
+    device_status_ok("moe")
+    del m
+    torch.cuda.empty_cache()
+    # decode-shaped linear: weight streaming
+    for M in (1, 4, 16):
+        c = inp.decode_q4_0_8192(M)
+        d = DenseLayerRun(c)
+        wbytes = c.wq.nbytes
+        ms_f, gf = time_steps(lambda: d.ql.qlora_linear_fwd(c.qtype, d.wq, c.N, c.K, d.X, d.A, d.B, c.r, c.scale, d.Y,
+                                                           d.H, d.ws), steps, 3, flush, slots=(0,))
+        ms_b, gb = time_steps(lambda: d.ql.qlora_linear_bwd(c.qtype, d.wq, c.N, c.K, d.X, d.dY, d.A, d.B, c.r, c.scale,
+                                                           d.H, d.dX, d.dA, d.dB, d.ws), steps, 3, flush, slots=(1,))
+        act_f = c.M * (c.K + c.N) * 2
+        out[f"decode_q4_0_M{M}_8192x8192"] = {
+            "fwd_ms": ms_f, "bwd_ms": ms_b, "fwd_gemm_ms": gf[0], "dx_gemm_ms": gb[1],
+            "fwd_weight_gbs": (wbytes + act_f) / (ms_f / 1e3) / 1e9,
+            "dx_gemm_weight_gbs": (wbytes + act_f) / (gb[1] / 1e3) / 1e9,
+            "fwd_frac_of_hbm": (wbytes + act_f) / (ms_f / 1e3) / 1e9 / pk["hbm_gbs"]}
+        device_status_ok(f"decode M={M}")
+        del d
+    torch.cuda.empty_cache()
+    # the other dense shapes
+    for key in ("dense_q4_0", "gate_up_q4_k"):
+        name, make = WORKLOADS[key]
+        d = DenseLayerRun(make(0))
+        ms, g = time_steps(d.step, steps, 3, flush, slots=(0, 1))
+        tf = d.flops() / (ms / 1e3) / 1e12
+        out[name] = {"tokens_per_s": d.c.M / (ms / 1e3), "ms_per_step": ms, "tflops": tf,
+                     "frac_of_bf16_peak": tf / pk["bf16_tflops"], "gemm_ms": {"fwd": g[0], "dx": g[1]}}
+        device_status_ok(name)
+        del d
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, rank, world, local_rank):
     import quantized_base_lora_tma_b200 as ql
     from quantized_base_lora_tma_b200 import build
@@ -325,6 +445,8 @@ def run_ours(args, rank, world, local_rank):
         "clocks": sampler.summary(),
         "wall_s_timed_region": wall,
     }
+    if rank == 0 and world == 1 and not args.no_also:
+        out["also"] = also_measurements(flush, max(20, K // 4), pk)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(case, target_s=args.cpu_seconds)
     return out
@@ -407,6 +529,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-also", action="store_true", help="skip the other shapes of the benchmark set")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 

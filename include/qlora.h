@@ -130,8 +130,8 @@ int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void
  * B_d [E][H][r] (bf16); s = scale.
  *   gu = x Wgu^T + s (x A_gu^T) B_gu^T;  h = silu(gu[:I]) * gu[I:];  o = h Wd^T + s (h A_d^T) B_d^T
  *   Y[t] = sum over the k selected slots (slot order) of w_tj * o_tj.
- * Rules: 1 <= k <= min(E, 16); E <= 256; H % 256 == 0; I % 256 == 0; 1 <= r <= 64; T >= 1;
- * T * ceil(E/32) <= 50000. P = T * k routed pairs.
+ * Rules: 1 <= k <= min(E, 16); E <= 256; H % 256 == 0; I % 256 == 0; 1 <= r <= 64; T >= 1.
+ * P = T * k routed pairs.
  * ------------------------------------------------------------------------------------------- */
 
 /* Routing. logits [T x E] bf16. Writes (device buffers of the caller):

@@ -125,10 +125,12 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
 
 // 32 bytes starting at a 2-byte aligned address p, as 8 words (the read stays inside [p, p+32)
 // rounded out to whole words).
+// The aligned base is formed by pointer arithmetic on p (not through an integer), so the compiler
+// keeps p's address space (shared-memory loads stay LDS).
 __device__ __forceinline__ void load32_a2(const uint8_t* p, uint32_t (&x)[8]) {
-  const uintptr_t a = reinterpret_cast<uintptr_t>(p);
-  const uint32_t* w = reinterpret_cast<const uint32_t*>(a & ~(uintptr_t)3);
-  const uint32_t sh = (uint32_t)(a & 3) * 8u;
+  const uint32_t mis = (uint32_t)(reinterpret_cast<uintptr_t>(p) & 3u);
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(p - mis);
+  const uint32_t sh = mis * 8u;
   uint32_t v[9];
 #pragma unroll
   for (int i = 0; i < 8; ++i) v[i] = w[i];
@@ -139,9 +141,9 @@ __device__ __forceinline__ void load32_a2(const uint8_t* p, uint32_t (&x)[8]) {
 
 // 16 bytes starting at a 2-byte aligned address p, as 4 words.
 __device__ __forceinline__ void load16_a2(const uint8_t* p, uint32_t (&x)[4]) {
-  const uintptr_t a = reinterpret_cast<uintptr_t>(p);
-  const uint32_t* w = reinterpret_cast<const uint32_t*>(a & ~(uintptr_t)3);
-  const uint32_t sh = (uint32_t)(a & 3) * 8u;
+  const uint32_t mis = (uint32_t)(reinterpret_cast<uintptr_t>(p) & 3u);
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(p - mis);
+  const uint32_t sh = mis * 8u;
   uint32_t v[5];
 #pragma unroll
   for (int i = 0; i < 4; ++i) v[i] = w[i];

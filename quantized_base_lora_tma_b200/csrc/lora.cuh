@@ -366,6 +366,25 @@ struct BopArgs {            // LB[n] = [Z(n, :) | Z(n, :)], zero padded (nullptr
   int rows;
 };
 
+// This CTA's share (by its linear index in the grid) of LB, 8 columns per item.
+__device__ __forceinline__ void lora_bop_share(const BopArgs& bop, int r, int RP, __nv_bfloat16* __restrict__ LB) {
+  if (bop.Z == nullptr) return;
+  const long items = (long)bop.rows * (2 * RP / 8);
+  const long cta = (long)blockIdx.y * gridDim.x + blockIdx.x;
+  const long ncta = (long)gridDim.x * gridDim.y;
+  for (long i = cta * blockDim.x + threadIdx.x; i < items; i += ncta * blockDim.x) {
+    const int n = (int)(i / (2 * RP / 8));
+    const int j0 = (int)(i % (2 * RP / 8)) * 8;
+    __nv_bfloat16 v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int j = (j0 + e) % RP;
+      v[e] = j < r ? bop.Z[(long)n * bop.zn + (long)j * bop.zjs] : __float2bfloat16(0.f);
+    }
+    *reinterpret_cast<uint4*>(LB + (long)n * 2 * RP + j0) = *reinterpret_cast<const uint4*>(v);
+  }
+}
+
 // Rows of out = Y Z^T for 64 rows per cluster column; cluster rank q sums k in
 // [q * kchunk, (q + 1) * kchunk). Z(j, k) = Z[j*zj + k*zk]. Writes out = oscale * sum (fp32 [M x r])
 // and la = split(lscale * sum). Every CTA also writes its share of the LB operand (bop).
@@ -374,12 +393,18 @@ __global__ void __launch_bounds__(128) lora_rows_cluster_kernel(const __nv_bfloa
                                                                 int Kin, int kchunk, const __nv_bfloat16* __restrict__ Z,
                                                                 long zj, long zk, int r, float oscale, float lscale,
                                                                 float* __restrict__ out, __nv_bfloat16* __restrict__ la,
-                                                                int RP, BopArgs bop, __nv_bfloat16* __restrict__ LB) {
+                                                                int RP, BopArgs bop, __nv_bfloat16* __restrict__ LB,
+                                                                int row_blocks) {
+  // CTAs with blockIdx.x >= row_blocks (whole clusters) only write their share of LB.
   constexpr int RN = 8 * NT;
   constexpr int SK = 128;       // k per staged sub-chunk
   constexpr int ZS = SK + 8;    // padded row of the staged Z tile (bf16)
   __shared__ float part[64 * RN];
   __shared__ __align__(16) __nv_bfloat16 zs[RN * ZS];
+  if ((int)blockIdx.x >= row_blocks) {
+    lora_bop_share(bop, r, RP, LB);
+    return;
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
   const int KS = gridDim.y;
@@ -462,23 +487,7 @@ __global__ void __launch_bounds__(128) lora_rows_cluster_kernel(const __nv_bfloa
       la[(long)m * 2 * RP + RP + j] = j < r ? lo : __float2bfloat16(0.f);
     }
   }
-  // this CTA's share of LB: items of 8 columns
-  if (bop.Z != nullptr) {
-    const long items = (long)bop.rows * (2 * RP / 8);
-    const long cta = (long)blockIdx.y * gridDim.x + blockIdx.x;
-    const long ncta = (long)gridDim.x * gridDim.y;
-    for (long i = cta * 128 + threadIdx.x; i < items; i += ncta * 128) {
-      const int n = (int)(i / (2 * RP / 8));
-      const int j0 = (int)(i % (2 * RP / 8)) * 8;
-      __nv_bfloat16 v[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int j = (j0 + e) % RP;
-        v[e] = j < r ? bop.Z[(long)n * bop.zn + (long)j * bop.zjs] : __float2bfloat16(0.f);
-      }
-      *reinterpret_cast<uint4*>(LB + (long)n * 2 * RP + j0) = *reinterpret_cast<const uint4*>(v);
-    }
-  }
+  lora_bop_share(bop, r, RP, LB);
   cluster_sync_all();  // no CTA leaves while a peer may still read its partials
 }
 
@@ -839,6 +848,30 @@ __global__ void colred_reduce_kernel(const float* __restrict__ part, int Ccols, 
     const int c = (int)(cj / r), j = (int)(cj % r);
     const long o = transpose ? ((long)e * r + j) * Ccols + c : ((long)e * Ccols + c) * r + j;
     out[o] = scale * acc;
+  }
+}
+
+// Ordered sum of the split-K partials of a dense GEMM: out[m][n] = sum_ks part[ks][m][n].
+__global__ void split_reduce_kernel(const float* __restrict__ part, int ksplit, long stride, long count,
+                                    void* __restrict__ out, int out_dtype) {
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; 4 * i < count; i += (long)gridDim.x * blockDim.x) {
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int ks = 0; ks < ksplit; ++ks) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(part + ks * stride) + i);
+      a.x += v.x;
+      a.y += v.y;
+      a.z += v.z;
+      a.w += v.w;
+    }
+    if (out_dtype == QL_F32) {
+      reinterpret_cast<float4*>(out)[i] = a;
+    } else {
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(a.x, a.y), hi = __floats2bfloat162_rn(a.z, a.w);
+      uint2 r;
+      r.x = *reinterpret_cast<const uint32_t*>(&lo);
+      r.y = *reinterpret_cast<const uint32_t*>(&hi);
+      reinterpret_cast<uint2*>(out)[i] = r;
+    }
   }
 }
 

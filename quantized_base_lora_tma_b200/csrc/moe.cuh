@@ -20,7 +20,8 @@ constexpr int kMaxTopK = 16;
 
 // One warp per token. E <= 256, k <= 16.
 __global__ void moe_topk_kernel(const __nv_bfloat16* __restrict__ logits, int T, int E, int k,
-                                int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+                                int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+                                int32_t* __restrict__ counts) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= T) return;
@@ -67,63 +68,68 @@ __global__ void moe_topk_kernel(const __nv_bfloat16* __restrict__ logits, int T,
     for (int j = 0; j < k; ++j) {
       topk_idx[(long)warp * k + j] = sel_e[j];
       topk_w[(long)warp * k + j] = w[j] * inv;
+      atomicAdd(counts + sel_e[j], 1);  // a count: the order of the additions does not matter
     }
   }
 }
 
-// Single CTA (1024 threads): counts, offsets, mblk and the (expert, token, slot) permutation.
-// Shared memory: a T x ceil(E/32) bitmask of selections (dynamic).
-__global__ void __launch_bounds__(1024) moe_permute_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
-                                                           int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-                                                           int32_t* __restrict__ mblk, int32_t* __restrict__ perm,
-                                                           int32_t* __restrict__ inv_perm) {
-  extern __shared__ uint32_t sel[];  // [T][EW]
-  __shared__ int cnt[kMaxExperts];
-  __shared__ int off[kMaxExperts + 1];
-  const int EW = (E + 31) / 32;
-  for (int i = threadIdx.x; i < T * EW; i += blockDim.x) sel[i] = 0u;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
-  __syncthreads();
-  for (int i = threadIdx.x; i < T * k; i += blockDim.x) {
-    const int t = i / k;
-    const int e = topk_idx[i];
-    atomicOr(&sel[t * EW + (e >> 5)], 1u << (e & 31));
-    atomicAdd(&cnt[e], 1);
-  }
-  __syncthreads();
+// One CTA (1024 threads) per expert e: offsets[e] and mblk[e] from the counts of the experts before
+// it, then e's pairs in token order: perm[offsets[e] + rank] = t*k + j and its inverse, where rank
+// counts the earlier tokens that selected e (block-wide ballot prefix sums over 1024 tokens at a
+// time). CTA 0 also writes offsets[E] and mblk[E].
+__global__ void __launch_bounds__(1024) moe_place_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
+                                                         const int32_t* __restrict__ counts,
+                                                         int32_t* __restrict__ offsets, int32_t* __restrict__ mblk,
+                                                         int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm) {
+  __shared__ int s_base;
+  __shared__ int s_warp[32];
+  const int e = blockIdx.x;
   if (threadIdx.x == 0) {
     int o = 0, mb = 0;
-    for (int e = 0; e < E; ++e) {
-      off[e] = o;
-      offsets[e] = o;
-      counts[e] = cnt[e];
-      mblk[e] = mb;
-      o += cnt[e];
-      mb += (cnt[e] + 127) / 128;
+    for (int q = 0; q < e; ++q) {
+      const int c = counts[q];
+      o += c;
+      mb += (c + 127) / 128;
     }
-    off[E] = o;
-    offsets[E] = o;
-    mblk[E] = mb;
+    offsets[e] = o;
+    mblk[e] = mb;
+    if (e == 0) {
+      int ot = 0, mt = 0;
+      for (int q = 0; q < E; ++q) {
+        const int c = counts[q];
+        ot += c;
+        mt += (c + 127) / 128;
+      }
+      offsets[E] = ot;
+      mblk[E] = mt;
+    }
+    s_base = o;
   }
   __syncthreads();
-  // one warp per expert: walk the tokens in order, 32 at a time
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nwarps = blockDim.x >> 5;
-  for (int e = warp; e < E; e += nwarps) {
-    int base = off[e];
-    for (int t0 = 0; t0 < T; t0 += 32) {
-      const int t = t0 + lane;
-      const bool hit = t < T && ((sel[t * EW + (e >> 5)] >> (e & 31)) & 1u);
-      const uint32_t b = __ballot_sync(0xffffffffu, hit);
-      if (hit) {
-        int j = 0;
-        while (j < k && topk_idx[(long)t * k + j] != e) ++j;
-        const int pos = base + __popc(b & ((1u << lane) - 1u));
-        perm[pos] = t * k + j;
-        inv_perm[t * k + j] = pos;
-      }
-      base += __popc(b);
+  for (int t0 = 0; t0 < T; t0 += 1024) {
+    const int t = t0 + threadIdx.x;
+    int slot = -1;
+    if (t < T)
+      for (int j = 0; j < k; ++j)
+        if (topk_idx[(long)t * k + j] == e) slot = j;
+    const uint32_t b = __ballot_sync(0xffffffffu, slot >= 0);
+    if (lane == 0) s_warp[warp] = __popc(b);
+    __syncthreads();
+    int before = 0, total = 0;
+    for (int w = 0; w < 32; ++w) {
+      const int c = s_warp[w];
+      if (w < warp) before += c;
+      total += c;
     }
+    if (slot >= 0) {
+      const int pos = s_base + before + __popc(b & ((1u << lane) - 1u));
+      perm[pos] = t * k + slot;
+      inv_perm[t * k + slot] = pos;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) s_base += total;
+    __syncthreads();
   }
 }
 

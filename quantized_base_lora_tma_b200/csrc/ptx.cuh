@@ -84,11 +84,14 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int sit
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   uint32_t spins = 0;
+  // Giving up needs both the time limit and a floor of failed polls, so that a jump of the global
+  // timer alone can never end a wait that is still making progress.
+  const uint32_t min_spins = limit_ns >= 1000000ull ? 65536u : 64u;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((++spins & 63u) == 0) {
       if (honour_abort && dev_aborted()) return false;
-      if (globaltimer_ns() - t0 > limit_ns) {
+      if (spins >= min_spins && globaltimer_ns() - t0 > limit_ns) {
         if (honour_abort) dev_fail(QL_ERR_TIMEOUT, site);
         return false;
       }

@@ -36,8 +36,8 @@ constexpr int kWarpTmaA = 4;
 constexpr int kWarpMma = 5;
 constexpr int kWarpTmaW = 6;
 constexpr int kWarpDq0 = 7;
-constexpr int kNumDqWarps = 8;
-constexpr int kGemmThreads = (kWarpDq0 + kNumDqWarps) * 32;  // 480
+constexpr int kNumDqWarps = 16;  // two groups of eight, taking alternate stages
+constexpr int kGemmThreads = (kWarpDq0 + kNumDqWarps) * 32;  // 736
 
 struct GemmParams {
   int M;           // rows of the A operand (tokens; routed pairs in grouped mode)
@@ -46,6 +46,9 @@ struct GemmParams {
   int n_lora_kb;   // extra 64-wide LoRA k-blocks
   int num_n_tiles;
   int num_m_blocks;  // dense mode: ceil(M / BM)
+  int ksplit;        // dense mode: the K range of every output tile is split into ksplit parts
+  int kb_per_split;  // k-blocks per part (a multiple of 4 in forward mode: whole raw groups)
+  long split_stride; // ksplit > 1: part ks of the fp32 output starts at out + ks * split_stride
   // weight rows
   int w_rows_per_expert;  // rows of W per expert (grouped); 0 in dense mode
   int lb_rows_per_expert; // rows of the LoRA B operand per expert (grouped)
@@ -99,19 +102,33 @@ struct TileInfo {
   int row_end;  // one past the last valid row
   int nb;       // output column block
   int e;        // expert (0 in dense mode)
+  int ks;       // K part (0 without split)
+  int kb_lo;    // first quantized k-block of this tile's part
+  int kb_hi;    // one past the last
+  int lora;     // this part also accumulates the LoRA k-blocks
 };
 
 template <int BM>
 __device__ __forceinline__ bool gemm_tile(const GemmParams& p, int t, TileInfo& ti) {
+  const int kb_main = p.Kd / kBK;
   if (p.E == 0) {
-    if (t >= p.num_m_blocks * p.num_n_tiles) return false;
-    const int mb = t % p.num_m_blocks;
-    ti.nb = t / p.num_m_blocks;
+    if (t >= p.num_m_blocks * p.num_n_tiles * p.ksplit) return false;
+    ti.ks = t % p.ksplit;
+    const int rest = t / p.ksplit;
+    const int mb = rest % p.num_m_blocks;
+    ti.nb = rest / p.num_m_blocks;
     ti.row0 = mb * BM;
     ti.row_end = p.M;
     ti.e = 0;
+    ti.kb_lo = ti.ks * p.kb_per_split;
+    ti.kb_hi = min(kb_main, ti.kb_lo + p.kb_per_split);
+    ti.lora = ti.ks == p.ksplit - 1;
     return true;
   }
+  ti.ks = 0;
+  ti.kb_lo = 0;
+  ti.kb_hi = kb_main;
+  ti.lora = 1;
   const int total_mb = __ldg(p.mblk_off + p.E);
   if (t >= total_mb * p.num_n_tiles) return false;
   const int gm = t % total_mb;
@@ -157,6 +174,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, const TileInf
   if (EPI == EPI_STORE || EPI == EPI_PAIR_OUT) {
     float wr = 1.0f;
     if (EPI == EPI_PAIR_OUT && valid) wr = __ldg(p.row_w + row);
+    const bool split = p.ksplit > 1;  // fp32 partial of K part ti.ks
 #pragma unroll 1
     for (int jc = 0; jc < BN / 32; ++jc) {
       uint32_t v[32];
@@ -164,8 +182,9 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, const TileInf
       tmem_ld_wait();
       const int col0 = ti.nb * BN + 32 * jc;
       if (valid && col0 < p.Nd) {
-        if (p.out_dtype == QL_F32) {
-          float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (long)row * p.ldo + col0);
+        if (p.out_dtype == QL_F32 || split) {
+          float* base = reinterpret_cast<float*>(p.out) + (split ? ti.ks * p.split_stride : 0);
+          float4* o = reinterpret_cast<float4*>(base + (long)row * p.ldo + col0);
 #pragma unroll
           for (int i = 0; i < 8; ++i)
             o[i] = make_float4(wr * __uint_as_float(v[4 * i]), wr * __uint_as_float(v[4 * i + 1]),
@@ -289,12 +308,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(full_bar(s), 1 + kNumDqWarps);
+      mbar_init(full_bar(s), 1 + kNumDqWarps / 2);  // TMA + the warps of one group
       mbar_init(empty_bar(s), 1);
     }
     for (int s = 0; s < C::RAW_SLOTS; ++s) {
       mbar_init(rfull_bar(s), 1);
-      mbar_init(rempty_bar(s), kNumDqWarps);
+      mbar_init(rempty_bar(s), TRANS ? kNumDqWarps / 2 : kNumDqWarps);  // every reader of the chunk
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull_bar(b), 1);
@@ -318,8 +337,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
 
   const int kb_main = p.Kd / kBK;
-  const int kb_total = kb_main + p.n_lora_kb;
-  const int groups = p.Kd / 256;  // forward: raw chunks per tile
+  // k-block of step i of a tile: its quantized part first, then (if it carries them) the LoRA blocks
+  auto tile_steps = [&](const TileInfo& ti) { return (ti.kb_hi - ti.kb_lo) + (ti.lora ? p.n_lora_kb : 0); };
+  auto step_kb = [&](const TileInfo& ti, int i) {
+    const int nq = ti.kb_hi - ti.kb_lo;
+    return i < nq ? ti.kb_lo + i : kb_main + (i - nq);
+  };
 
   if (warp == kWarpTmaA) {
     // ---------------- A operand (and LoRA operands) producer ----------------
@@ -330,7 +353,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int s = 0; s < C::STAGES; ++s) last_phase[s] = -1;
       TileInfo ti;
       for (int t = blockIdx.x; ok && gemm_tile<BM>(p, t, ti); t += gridDim.x) {
-        for (int kb = 0; kb < kb_total; ++kb, ++it) {
+        const int nsteps = tile_steps(ti);
+        for (int i = 0; i < nsteps; ++i, ++it) {
+          const int kb = step_kb(ti, i);
           const int s = it % C::STAGES;
           const uint32_t ph = (it / C::STAGES) & 1;
           if (!mbar_wait(empty_bar(s), ph ^ 1, 1)) { ok = false; break; }
@@ -369,8 +394,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       TileInfo ti;
       for (int t = blockIdx.x; ok && gemm_tile<BM>(p, t, ti); t += gridDim.x) {
         const int wbase = ti.e * p.w_rows_per_expert;
-        const int nchunks = TRANS ? kb_main : groups;
-        for (int c = 0; c < nchunks; ++c, ++rc) {
+        const int c_lo = TRANS ? ti.kb_lo : ti.kb_lo / 4;
+        const int c_hi = TRANS ? ti.kb_hi : ti.kb_hi / 4;
+        for (int c = c_lo; c < c_hi; ++c, ++rc) {
           const int s = rc % C::RAW_SLOTS;
           const uint32_t ph = (rc / C::RAW_SLOTS) & 1;
           if (!mbar_wait(rempty_bar(s), ph ^ 1, 2)) { ok = false; break; }
@@ -407,7 +433,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (!mbar_wait(tempty_bar(buf), ((tc >> 1) & 1) ^ 1, 3)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * C::ACC_COLS;
-        for (int kb = 0; kb < kb_total; ++kb, ++it) {
+        const int nsteps = tile_steps(ti);
+        for (int i = 0; i < nsteps; ++i, ++it) {
+          const int kb = step_kb(ti, i);
           const int s = it % C::STAGES;
           const uint32_t ph = (it / C::STAGES) & 1;
           if (!mbar_wait(full_bar(s), ph, 4)) { ok = false; break; }
@@ -423,7 +451,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int h = 0; h < MS; ++h) {
               const uint64_t ad = smem_desc_sw128(a0 + h * 16384 + 32 * k, 16, 1024);
-              umma_bf16(d_tmem + h * BN, ad, bd, kmaj ? idesc_kmaj : idesc_main, (kb | k) != 0);
+              umma_bf16(d_tmem + h * BN, ad, bd, kmaj ? idesc_kmaj : idesc_main, (i | k) != 0);
             }
           }
           umma_commit(empty_bar(s));
@@ -439,24 +467,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp >= kWarpDq0) {
     // ---------------- dequant workers ----------------
-    const int dq = threadIdx.x - kWarpDq0 * 32;  // 0..255
+    // Two groups of eight warps take alternate stages, so one group's fence and barrier round
+    // trip overlaps the other group's decoding, and eight warps per group hide the latency of
+    // the decode's dependent chains. Each thread decodes one 32-weight unit per stage.
+    const int dq = threadIdx.x - kWarpDq0 * 32;  // 0..511
+    const int grp = dq >> 8;                     // stage parity this group handles
+    const int gt = dq & 255;                     // thread within the group
     int it = 0, rc = 0;
     bool ok = true;
     TileInfo ti;
     for (int t = blockIdx.x; ok && gemm_tile<BM>(p, t, ti); t += gridDim.x) {
       if (!TRANS) {
-        for (int g = 0; ok && g < groups; ++g, ++rc) {
+        for (int g = ti.kb_lo / 4; ok && g < ti.kb_hi / 4; ++g, ++rc) {
           const int rs = rc % C::RAW_SLOTS;
           if (!warp_wait(rfull_bar(rs), (rc / C::RAW_SLOTS) & 1, 5)) { ok = false; break; }
           const uint8_t* raw = smem + C::OFF_RAW + rs * C::RAW_BYTES;
           for (int sub = 0; sub < 4; ++sub, ++it) {
+            if ((it & 1) != grp) continue;
             const int s = it % C::STAGES;
             if (!warp_wait(empty_bar(s), ((it / C::STAGES) & 1) ^ 1, 6)) { ok = false; break; }
             uint8_t* sb = smem + C::OFF_B + s * C::B_BYTES;
             {
-              // one 32-weight unit per thread: row dq/2, units 2*sub + (dq&1) of the group
-              const int row = dq >> 1;
-              const int uh = dq & 1;
+              // row gt/2 of the tile, 32-weight unit 2*sub + gt%2 of the group
+              const int row = gt >> 1, uh = gt & 1;
               uint4 v[4];
               decode_unit_bf16<QT>(raw + row * C::GB, 2 * sub + uh, v);
 #pragma unroll
@@ -473,7 +506,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (ok && lane == 0) mbar_arrive(rempty_bar(rs));
         }
       } else {
-        for (int kb = 0; ok && kb < kb_main; ++kb, ++rc, ++it) {
+        for (int kb = ti.kb_lo; ok && kb < ti.kb_hi; ++kb, ++rc, ++it) {
+          if ((it & 1) != grp) continue;
           const int rs = rc % C::RAW_SLOTS;
           if (!warp_wait(rfull_bar(rs), (rc / C::RAW_SLOTS) & 1, 5)) { ok = false; break; }
           const int s = it % C::STAGES;
@@ -481,9 +515,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint8_t* raw = smem + C::OFF_RAW + rs * C::RAW_BYTES;
           uint8_t* sb = smem + C::OFF_B + s * C::B_BYTES;
           {
-            // one 32-column unit per thread: row kk = dq/4 of the chunk, unit 4*(nb&1) + dq%4 of
-            // the group (the tile's 128 columns are half of the 256-column group)
-            const int kk = dq >> 2, ul = dq & 3;
+            // 32-column unit: row kk = gt/4 of the chunk, unit 4*(nb&1) + gt%4 of the group
+            // (the tile's 128 columns are half of the 256-column group)
+            const int kk = gt >> 2, ul = gt & 3;
             uint4 v[4];
             decode_unit_bf16<QT>(raw + kk * C::GB, 4 * (ti.nb & 1) + ul, v);
 #pragma unroll
@@ -501,8 +535,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
-      // LoRA k-blocks: operands come by TMA; the workers only account for their share.
-      for (int kb = kb_main; ok && kb < kb_total; ++kb, ++it) {
+      // LoRA k-blocks: operands come by TMA; the group whose turn it is accounts for the stage.
+      for (int i = 0; ok && ti.lora && i < p.n_lora_kb; ++i, ++it) {
+        if ((it & 1) != grp) continue;
         const int s = it % C::STAGES;
         if (!warp_wait(empty_bar(s), ((it / C::STAGES) & 1) ^ 1, 7)) { ok = false; break; }
         __syncwarp();

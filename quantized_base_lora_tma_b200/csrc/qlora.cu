@@ -184,8 +184,13 @@ static int launch_rows_dense(const __nv_bfloat16* Y, long ldy, int M, int Kin, c
   int kchunk = (Kin + KS - 1) / KS;
   kchunk = (kchunk + 31) / 32 * 32;
   KS = (Kin + kchunk - 1) / kchunk;
+  // extra clusters for the LB operand when it outweighs the row work (small M)
+  const int row_blocks = (M + 63) / 64;
+  const long bop_items = bop.Z ? (long)bop.rows * (2 * RP / 8) : 0;
+  const long per_cluster = (long)KS * 128 * 4;
+  const int bop_blocks = (int)std::max<long>(0, (bop_items + per_cluster - 1) / per_cluster - row_blocks);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((M + 63) / 64, KS, 1);
+  cfg.gridDim = dim3(row_blocks + bop_blocks, KS, 1);
   cfg.blockDim = dim3(128, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
@@ -199,13 +204,13 @@ static int launch_rows_dense(const __nv_bfloat16* Y, long ldy, int M, int Kin, c
   cudaError_t e;
   if (r <= 16)
     e = cudaLaunchKernelEx(&cfg, lora_rows_cluster_kernel<2>, Y, ldy, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out,
-                           la, RP, bop, LB);
+                           la, RP, bop, LB, row_blocks);
   else if (r <= 32)
     e = cudaLaunchKernelEx(&cfg, lora_rows_cluster_kernel<4>, Y, ldy, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out,
-                           la, RP, bop, LB);
+                           la, RP, bop, LB, row_blocks);
   else
     e = cudaLaunchKernelEx(&cfg, lora_rows_cluster_kernel<8>, Y, ldy, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out,
-                           la, RP, bop, LB);
+                           la, RP, bop, LB, row_blocks);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -277,9 +282,92 @@ static int launch_colred(const __nv_bfloat16* Y, long ldy, int Ccols, const floa
   return launch_status();
 }
 
+// Tile plan of a dense GEMM: BM = 128 * MS rows per tile; K split into ksplit parts of
+// kb_per_split k-blocks (a multiple of 4 in forward mode) when the output has fewer tiles than
+// there are SMs (the small-M, weight-streaming regime).
+struct DensePlan {
+  int MS, ksplit, kbs, mblocks, ntiles;
+};
+static DensePlan plan_dense(int64_t M, int64_t Nd, int64_t Kd, bool trans, bool allow_split) {
+  DensePlan d;
+  d.MS = M > 128 ? 2 : 1;
+  d.mblocks = (int)((M + 128 * d.MS - 1) / (128 * d.MS));
+  d.ntiles = (int)((Nd + 127) / 128);
+  const int kb_main = (int)(Kd / 64);
+  const int unit = trans ? 1 : 4;
+  d.ksplit = 1;
+  d.kbs = kb_main;
+  const int tiles = d.mblocks * d.ntiles;
+  const int nsm = num_sms();
+  if (allow_split && tiles < nsm) {
+    int ks = std::min((4 * nsm + tiles - 1) / tiles, std::min(kb_main / unit, 32));
+    if (ks > 1) {
+      int kbs = (kb_main + ks - 1) / ks;
+      kbs = (kbs + unit - 1) / unit * unit;
+      d.kbs = kbs;
+      d.ksplit = (kb_main + kbs - 1) / kbs;
+    }
+  }
+  return d;
+}
+static size_t split_bytes(const DensePlan& d, int64_t M, int64_t Nd) {
+  return d.ksplit > 1 ? (size_t)d.ksplit * M * Nd * 4 : 0;
+}
+
+static int launch_split_reduce(const float* part, int ksplit, long stride, long count, void* out, int out_dtype,
+                               cudaStream_t st) {
+  const long vec = count / 4;
+  const int grid = (int)std::min<long>((vec + 255) / 256, (long)num_sms() * 8);
+  split_reduce_kernel<<<grid, 256, 0, st>>>(part, ksplit, stride, count, out, out_dtype);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return launch_status();
+}
+
+
+// One dense dequant GEMM (forward: TRANS = false, D = A deq(W)^T; input-gradient: TRANS = true,
+// D = A deq(W)) with its LoRA k-blocks, planned by plan_dense; with a K split the fp32 partials go
+// to split_buf and are summed in order into `out`.
+template <bool TRANS>
+static int launch_dense_gemm(int qtype, const void* A, int64_t M, int64_t Kd, const void* wq, int64_t w_rows,
+                             int64_t w_cols, const __nv_bfloat16* LA, const __nv_bfloat16* LB, int KL, int64_t Nd,
+                             void* out, int out_dtype, float* split_buf, bool allow_split, cudaStream_t st, int slot) {
+  const DensePlan d = plan_dense(M, Nd, Kd, TRANS, allow_split && split_buf != nullptr);
+  const uint32_t box = 128u * d.MS;
+  CUtensorMap tA, tW, tLA, tLB;
+  if (!tmap_bf16_rows(&tA, A, Kd, M, box) ||
+      !tmap_packed(&tW, wq, packed_row_bytes(qtype, w_cols), w_rows, group_bytes(qtype)) ||
+      !tmap_bf16_rows(&tLA, LA, KL, M, box) || !tmap_bf16_rows(&tLB, LB, KL, Nd, 64))
+    return QL_ERR_CUDA;
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.M = (int)M;
+  p.Nd = (int)Nd;
+  p.Kd = (int)Kd;
+  p.n_lora_kb = KL / 64;
+  p.num_n_tiles = d.ntiles;
+  p.num_m_blocks = d.mblocks;
+  p.ksplit = d.ksplit;
+  p.kb_per_split = d.kbs;
+  p.ldo = Nd;
+  if (d.ksplit > 1) {
+    p.out = split_buf;
+    p.out_dtype = QL_F32;
+    p.split_stride = (long)M * Nd;
+  } else {
+    p.out = out;
+    p.out_dtype = out_dtype;
+  }
+  const int tiles = d.mblocks * d.ntiles * d.ksplit;
+  const int grid = std::min(tiles, num_sms());
+  int rc = d.MS == 2 ? launch_qgemm_q<TRANS, EPI_STORE, 2>(qtype, tA, tW, tLA, tLB, p, grid, st, slot)
+                     : launch_qgemm_q<TRANS, EPI_STORE, 1>(qtype, tA, tW, tLA, tLB, p, grid, st, slot);
+  if (rc || d.ksplit == 1) return rc;
+  return launch_split_reduce(split_buf, d.ksplit, (long)M * Nd, (long)M * Nd, out, out_dtype, st);
+}
+
 // Workspace layout of the dense layer (byte offsets, 256-aligned).
 struct LinearWs {
-  size_t la, lb, g, total;
+  size_t la, lb, g, split, total;
 };
 static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 static LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int r) {
@@ -290,6 +378,9 @@ static LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int r) {
   w.la = o; o = al256(o + (size_t)M * KL * 2);
   w.lb = o; o = al256(o + (size_t)NK * KL * 2);
   w.g = o; o = al256(o + (size_t)M * r * 4);
+  const size_t sf = split_bytes(plan_dense(M, N, K, false, true), M, N);
+  const size_t sb = split_bytes(plan_dense(M, K, N, true, true), M, K);
+  w.split = o; o = al256(o + std::max(sf, sb));
   w.total = o;
   return w;
 }
@@ -506,25 +597,8 @@ int qlora_linear_fwd(int qtype, const void* wq, int64_t N, int64_t K, const void
                          LA, BopArgs{(const __nv_bfloat16*)B, r, 1, (int)N}, LB, st);
   if (rc) return rc;
 
-  CUtensorMap tA, tW, tLA, tLB;
-  const int64_t rb = packed_row_bytes(qtype, K);
-  if (!tmap_bf16_rows(&tA, X, K, M, 256) || !tmap_packed(&tW, wq, rb, N, group_bytes(qtype)) ||
-      !tmap_bf16_rows(&tLA, LA, KL, M, 256) || !tmap_bf16_rows(&tLB, LB, KL, N, 64))
-    return QL_ERR_CUDA;
-  GemmParams p;
-  memset(&p, 0, sizeof(p));
-  p.M = (int)M;
-  p.Nd = (int)N;
-  p.Kd = (int)K;
-  p.n_lora_kb = KL / 64;
-  p.num_n_tiles = (int)((N + 127) / 128);
-  p.num_m_blocks = (int)((M + 255) / 256);
-  p.out = Y;
-  p.out_dtype = y_dtype;
-  p.ldo = N;
-  const int tiles = p.num_n_tiles * p.num_m_blocks;
-  const int grid = std::min(tiles, num_sms());
-  return launch_qgemm_q<false, EPI_STORE, 2>(qtype, tA, tW, tLA, tLB, p, grid, st, 0);
+  return launch_dense_gemm<false>(qtype, X, M, K, wq, N, K, LA, LB, KL, N, Y, y_dtype, (float*)(wsb + w.split), true,
+                                  st, 0);
 }
 
 int qlora_moe_route(const void* logits, int64_t T, int E, int k, int32_t* topk_idx, float* topk_w, int32_t* counts,
@@ -532,17 +606,14 @@ int qlora_moe_route(const void* logits, int64_t T, int E, int k, int32_t* topk_i
   if (!logits || !topk_idx || !topk_w || !counts || !offsets || !perm || !inv_perm || !mblk) return QL_ERR_INVALID_ARG;
   if (E < 1 || E > kMaxExperts || k < 1 || k > kMaxTopK || k > E) return QL_ERR_UNSUPPORTED;
   if (T < 1) return QL_ERR_INVALID_ARG;
-  const int EW = (E + 31) / 32;
-  if (T * EW > 50000) return QL_ERR_SHAPE;
+  if (T > (1 << 24)) return QL_ERR_SHAPE;
   cudaStream_t st = (cudaStream_t)stream;
+  if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, st) != cudaSuccess) return QL_ERR_CUDA;
   const int grid = (int)((T * 32 + 255) / 256);
-  moe_topk_kernel<<<grid, 256, 0, st>>>((const __nv_bfloat16*)logits, (int)T, E, k, topk_idx, topk_w);
+  moe_topk_kernel<<<grid, 256, 0, st>>>((const __nv_bfloat16*)logits, (int)T, E, k, topk_idx, topk_w, counts);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (launch_status() != QL_OK) return QL_ERR_CUDA;
-  const size_t smem = (size_t)T * EW * 4;
-  if (cudaFuncSetAttribute(moe_permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return QL_ERR_CUDA;
-  moe_permute_kernel<<<1, 1024, smem, st>>>(topk_idx, (int)T, E, k, counts, offsets, mblk, perm, inv_perm);
+  moe_place_kernel<<<E, 1024, 0, st>>>(topk_idx, (int)T, E, k, counts, offsets, mblk, perm, inv_perm);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return launch_status();
 }
@@ -611,7 +682,7 @@ int qlora_moe_fwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
     memset(&p, 0, sizeof(p));
     p.M = P; p.Nd = (int)(2 * I); p.Kd = (int)H; p.n_lora_kb = KL / 64; p.num_n_tiles = (int)(I / 64);
     p.w_rows_per_expert = (int)(2 * I); p.lb_rows_per_expert = (int)(2 * I); p.I = (int)I;
-    p.E = E; p.seg_off = off; p.mblk_off = mblk;
+    p.E = E; p.seg_off = off; p.mblk_off = mblk; p.ksplit = 1;
     p.out_g = g; p.out_u = u; p.out_h = h; p.out_lo = (__nv_bfloat16*)(sb + sv.hlo);
     rc = launch_qgemm_q<false, EPI_SWIGLU, 1>(qtype, tA, tW, tLA, tLB, p, nsm, st, 2);
     if (rc) return rc;
@@ -632,7 +703,7 @@ int qlora_moe_fwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
     memset(&p, 0, sizeof(p));
     p.M = P; p.Nd = (int)H; p.Kd = (int)I; p.n_lora_kb = KL / 64; p.num_n_tiles = (int)(H / 128);
     p.w_rows_per_expert = (int)H; p.lb_rows_per_expert = (int)H; p.I = (int)I;
-    p.E = E; p.seg_off = off; p.mblk_off = mblk;
+    p.E = E; p.seg_off = off; p.mblk_off = mblk; p.ksplit = 1;
     p.out = pair_out; p.out_dtype = QL_F32; p.ldo = H; p.row_w = row_w;
     rc = launch_qgemm_q<false, EPI_PAIR_OUT, 1>(qtype, tA, tW, tLA, tLB, p, nsm, st, 3);
     if (rc) return rc;
@@ -707,7 +778,7 @@ int qlora_moe_bwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
     memset(&p, 0, sizeof(p));
     p.M = P; p.Nd = (int)I; p.Kd = (int)H; p.n_lora_kb = KL / 64; p.num_n_tiles = (int)(I / 128);
     p.w_rows_per_expert = (int)H; p.lb_rows_per_expert = (int)I; p.I = (int)I;
-    p.E = E; p.seg_off = off; p.mblk_off = mblk;
+    p.E = E; p.seg_off = off; p.mblk_off = mblk; p.ksplit = 1;
     p.in_g = g; p.in_u = u; p.in_h = h; p.out_g = dgu; p.out_lo = dgu_lo; p.row_w = row_w; p.dw_part = dwp;
     rc = launch_qgemm_q<true, EPI_SWIGLU_BWD, 1>(qtype, tA, tW, tLA, tLB, p, nsm, st, 4);
     if (rc) return rc;
@@ -733,7 +804,7 @@ int qlora_moe_bwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
     memset(&p, 0, sizeof(p));
     p.M = P; p.Nd = (int)H; p.Kd = (int)(2 * I); p.n_lora_kb = KL / 64; p.num_n_tiles = (int)(H / 128);
     p.w_rows_per_expert = (int)(2 * I); p.lb_rows_per_expert = (int)H; p.I = (int)I;
-    p.E = E; p.seg_off = off; p.mblk_off = mblk;
+    p.E = E; p.seg_off = off; p.mblk_off = mblk; p.ksplit = 1;
     p.out = dxp; p.out_dtype = QL_F32; p.ldo = H;
     rc = launch_qgemm_q<true, EPI_STORE, 1>(qtype, tA, tW, tLA, tLB, p, nsm, st, 5);
     if (rc) return rc;
@@ -778,24 +849,8 @@ int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void
                          LA, dX ? BopArgs{(const __nv_bfloat16*)A, 1, K, (int)K} : BopArgs{nullptr, 0, 0, 0}, LB, st);
   if (rc) return rc;
   if (dX) {
-    CUtensorMap tA, tW, tLA, tLB;
-    const int64_t rb = packed_row_bytes(qtype, K);
-    if (!tmap_bf16_rows(&tA, dY, N, M, 256) || !tmap_packed(&tW, wq, rb, N, group_bytes(qtype)) ||
-        !tmap_bf16_rows(&tLA, LA, KL, M, 256) || !tmap_bf16_rows(&tLB, LB, KL, K, 64))
-      return QL_ERR_CUDA;
-    GemmParams p;
-    memset(&p, 0, sizeof(p));
-    p.M = (int)M;
-    p.Nd = (int)K;
-    p.Kd = (int)N;
-    p.n_lora_kb = KL / 64;
-    p.num_n_tiles = (int)(K / 128);
-    p.num_m_blocks = (int)((M + 255) / 256);
-    p.out = dX;
-    p.out_dtype = dx_dtype;
-    p.ldo = K;
-    const int tiles = p.num_n_tiles * p.num_m_blocks;
-    rc = launch_qgemm_q<true, EPI_STORE, 2>(qtype, tA, tW, tLA, tLB, p, std::min(tiles, num_sms()), st, 1);
+    rc = launch_dense_gemm<true>(qtype, dY, M, N, wq, N, K, LA, LB, KL, K, dX, dx_dtype,
+                                 (float*)(wsb + w.split), true, st, 1);
     if (rc) return rc;
   }
   // dB = s dY^T H and dA = G^T X in one launch
@@ -861,22 +916,6 @@ extern "C" int qlora_linear_fwd_noalloc(int qtype, const void* wq, int64_t N, in
   rc = launch_rows_dense((const __nv_bfloat16*)X, K, (int)M, (int)K, (const __nv_bfloat16*)A, K, 1, r, 1.0f, scale, H,
                          LA, BopArgs{(const __nv_bfloat16*)B, r, 1, (int)N}, LB, st);
   if (rc) return rc;
-  CUtensorMap tA, tW, tLA, tLB;
-  const int64_t rb = packed_row_bytes(qtype, K);
-  if (!tmap_bf16_rows(&tA, X, K, M, 256) || !tmap_packed(&tW, wq, rb, N, group_bytes(qtype)) ||
-      !tmap_bf16_rows(&tLA, LA, KL, M, 256) || !tmap_bf16_rows(&tLB, LB, KL, N, 64))
-    return QL_ERR_CUDA;
-  GemmParams p;
-  memset(&p, 0, sizeof(p));
-  p.M = (int)M;
-  p.Nd = (int)N;
-  p.Kd = (int)K;
-  p.n_lora_kb = KL / 64;
-  p.num_n_tiles = (int)((N + 127) / 128);
-  p.num_m_blocks = (int)((M + 255) / 256);
-  p.out = Y;
-  p.out_dtype = y_dtype;
-  p.ldo = N;
-  const int tiles = p.num_n_tiles * p.num_m_blocks;
-  return launch_qgemm_q<false, EPI_STORE, 2>(qtype, tA, tW, tLA, tLB, p, std::min(tiles, num_sms()), st, 0);
+  // no K split here: its partials would need more scratch than the static array holds
+  return launch_dense_gemm<false>(qtype, X, M, K, wq, N, K, LA, LB, KL, N, Y, y_dtype, nullptr, false, st, 0);
 }

@@ -174,14 +174,20 @@ def _normal(rng, shape, std):
 
 
 def linear_case(M, K, N, qtype, r, alpha, seed=0, outlier_frac=0.0, w_std=0.02, b_std=0.01,
-                name=None) -> LinearCase:
-    """Draw order: X, dY, W, A, B, then (if outlier_frac > 0) the outlier rows of W (scaled x8)."""
+                name=None, weights_first=False) -> LinearCase:
+    """Draw order: X, dY, W, A, B, then (if outlier_frac > 0) the outlier rows of W (scaled x8).
+    With weights_first: W, A, B, then X, dY (the weights then do not depend on M)."""
     rng = np.random.default_rng(seed)
+    if weights_first:
+        W = _normal(rng, (N, K), w_std)
+        A = _normal(rng, (r, K), 1.0 / math.sqrt(K))
+        B = _normal(rng, (N, r), b_std)
     X = _normal(rng, (M, K), 1.0)
     dY = _normal(rng, (M, N), 1.0)
-    W = _normal(rng, (N, K), w_std)
-    A = _normal(rng, (r, K), 1.0 / math.sqrt(K))
-    B = _normal(rng, (N, r), b_std)
+    if not weights_first:
+        W = _normal(rng, (N, K), w_std)
+        A = _normal(rng, (r, K), 1.0 / math.sqrt(K))
+        B = _normal(rng, (N, r), b_std)
     meta = {}
     if outlier_frac > 0:
         n_out = int(round(outlier_frac * N))
@@ -203,6 +209,13 @@ def dense_proj_2048x4096x4096(qtype=Q8_0, seed=0):
     """Dense projection at one 2048-token chunk: K = N = 4096, rank 16, alpha 32."""
     return linear_case(2048, 4096, 4096, qtype, 16, 32.0, seed,
                        name=f"dense_proj_{QTYPE_NAMES[qtype]}_2048x4096x4096_r16")
+
+
+def decode_q4_0_8192(M, seed=0):
+    """Decode-shaped Q4_0 linear: K = N = 8192 at M tokens (M in {1, 4, 16} in the benchmark set),
+    rank 4, alpha 8; the weights are drawn first so they are the same for every M."""
+    return linear_case(M, 8192, 8192, Q4_0, 4, 8.0, seed, name=f"decode_q4_0_{M}x8192x8192_r4",
+                       weights_first=True)
 
 
 def gate_up_q4_k_2048x2048x12288(seed=0):

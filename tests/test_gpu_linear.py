@@ -89,6 +89,8 @@ SMALL = [
     (1, 256, 64, 1),
     (200, 256, 448, 40),   # r > 32: two LoRA k-blocks
     (64, 1024, 128, 64),
+    (16, 2048, 512, 8),    # small M: the K range is split across CTAs (fwd and dX)
+    (3, 1024, 1024, 4),
 ]
 
 
@@ -158,3 +160,53 @@ def test_bounded_wait_self_check():
     Y, *_ = run_linear(c)
     Yr, *_ = oracle_linear(c)
     assert_close(f64(Y), Yr, "Y")
+
+
+_W8192 = {}
+
+
+def _small_m_case(M):
+    c = inp.decode_q4_0_8192(M)
+    if "W" not in _W8192:
+        _W8192["W"] = (c.wq.copy(), ll.weights(c.qtype, c.wq, c.N, c.K))
+    assert np.array_equal(_W8192["W"][0], c.wq)
+    return c, _W8192["W"][1]
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_linear_decode_shape_q4_0_8192(M):
+    """Weight-streaming shape: Q4_0, K = N = 8192, M in {1, 4, 16}; full Y, dX, dA, dB."""
+    c, W = _small_m_case(M)
+    Y, H, dX, dA, dB = run_linear(c)
+    X, dY, A, B = bf16_f64(c.X), bf16_f64(c.dY), bf16_f64(c.A), bf16_f64(c.B)
+    Yr, Hr = ll.linear_fwd(W, X, A, B, c.scale)
+    dXr, dAr, dBr, _ = ll.linear_bwd(W, X, dY, A, B, c.scale, Hr)
+    for got, ref, name in [(Y, Yr, "Y"), (H, Hr, "H"), (dX, dXr, "dX"), (dA, dAr, "dA"), (dB, dBr, "dB")]:
+        assert_close(f64(got), ref, name)
+
+
+@pytest.mark.parametrize("qtype", [inp.Q4_0, inp.Q8_0, inp.Q4_K])
+def test_linear_repeated_launches_complete(qtype):
+    """Many back-to-back forward + backward calls (both GEMM directions, BM = 256 tiles) finish
+    without any bounded wait giving up, and give the same result every time."""
+    c = inp.linear_case(512, 2048, 1024, qtype, 8, 16.0, seed=31)
+    X, dY, A, B = dev_bf16(c.X), dev_bf16(c.dY), dev_bf16(c.A), dev_bf16(c.B)
+    wq = dev_u8(c.wq)
+    M, N, K, r = c.M, c.N, c.K, c.r
+    ws = torch.empty(ql.qlora_linear_workspace_bytes(M, N, K, r), dtype=torch.uint8, device="cuda")
+    Y = torch.empty(M, N, dtype=torch.float32, device="cuda")
+    H = torch.empty(M, r, dtype=torch.float32, device="cuda")
+    dX = torch.empty(M, K, dtype=torch.float32, device="cuda")
+    dA = torch.empty(r, K, dtype=torch.float32, device="cuda")
+    dB = torch.empty(N, r, dtype=torch.float32, device="cuda")
+    first = None
+    for i in range(60):
+        ql.qlora_linear_fwd(c.qtype, wq, N, K, X, A, B, r, c.scale, Y, H, ws)
+        ql.qlora_linear_bwd(c.qtype, wq, N, K, X, dY, A, B, r, c.scale, H, dX, dA, dB, ws)
+        if i == 0:
+            torch.cuda.synchronize()
+            first = (Y.clone(), dX.clone())
+    torch.cuda.synchronize()
+    rc, site = ql.qlora_device_status(reset=False)
+    assert rc == 0, f"bounded wait gave up at site {site}"
+    assert torch.equal(first[0], Y) and torch.equal(first[1], dX)
