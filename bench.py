@@ -228,6 +228,13 @@ class MoERun:
         return 12.0 * P * c.H * c.I + 6.0 * c.r * (2 * c.H + 3 * c.I) * P
 
 
+def allreduce_adapter_grads(grads):
+    """The data-parallel exchange of the layer: every rank holds the adapter gradients of its own
+    tokens; dA and dB are sums over tokens, so their sum over ranks is the full-batch gradient."""
+    for g in grads:
+        torch.distributed.all_reduce(g, op=torch.distributed.ReduceOp.SUM)
+
+
 def time_steps(fn, steps, warmup, flush, slots=()):
     """Mean device time (ms) of fn() over `steps` calls, L2 flushed before each; per-slot GEMM means."""
     import quantized_base_lora_tma_b200 as ql
@@ -325,8 +332,7 @@ def run_ours(args, rank, world, local_rank):
 
     def allreduce_grads():
         if world > 1:
-            torch.distributed.all_reduce(run.dA)
-            torch.distributed.all_reduce(run.dB)
+            allreduce_adapter_grads([run.dA, run.dB])
 
     for _ in range(args.warmup):
         run.step()
