@@ -147,8 +147,9 @@ __device__ __forceinline__ bool gemm_tile(const GemmParams& p, int t, TileInfo& 
 }
 
 // All 32 lanes wait; the outcome is made warp-uniform.
+template <bool CLUSTER = false>
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int site) {
-  const bool r = mbar_wait(bar, parity, site);
+  const bool r = mbar_wait<CLUSTER>(bar, parity, site);
   return __all_sync(0xffffffffu, r);
 }
 

@@ -1,0 +1,379 @@
+// Pair (two-CTA) dequant-in-shared-memory GEMM for the dense layer: D = A deq(W)^T (forward) or
+// A deq(W) (input gradient), plus the LoRA k-blocks, on 256 x 256 output tiles computed by a CTA pair
+// with tcgen05.mma.cta_group::2.
+//
+// Why pairs: with 128-wide N tiles every CTA streams its A rows once per 128 output columns and the
+// A ring cannot cover the TMA latency within shared memory. A pair tile holds A split by M (each CTA
+// its own 128 rows) and B split by N (each CTA dequantizes its own 128 W rows, or its own 128 of
+// the output columns in the input-gradient direction), so per SM the bytes moved per FLOP halve and
+// the freed shared memory deepens the ring. Each CTA keeps its own producers (TMA for its A rows and
+// its packed groups, sixteen dequant warps); the leader CTA (rank 0) issues the pair MMAs, which
+// read both CTAs' shared memory and write both CTAs' TMEM (each its own 128 rows x 256 columns).
+//
+// Barrier protocol (full barriers live in the leader):
+//   full[s]   leader: 1 arrive.expect_tx (both CTAs' TMA bytes, plus 16 signal bytes per peer
+//             dequant warp on quantized steps) + the leader's dequant group. The peer's TMA copies
+//             complete_tx on the leader's barrier; each peer dequant warp, once its part of the B half
+//             is written and fenced for the async proxy, signals by a 16-byte bulk copy into the
+//             leader that also completes tx there. Counting the peer through the copy engine keeps a
+//             cluster-scope release fence (which costs about a thousand cycles) off the per-stage path.
+//   empty[s]  each CTA: one pair commit arriving on both CTAs
+//   tfull[b]  each CTA: one pair commit arriving on both; tempty[b] leader: 4 + 4 epilogue warps
+// Every wait is bounded (ptx.cuh); both CTAs always reach the final cluster barrier.
+#pragma once
+#include "qgemm.cuh"
+
+namespace qlora {
+
+// Warp roles. The MMA issuer (warp 5) runs on scheduler 1 (warp % 4 == 1); no dequant warp is
+// placed there, so the issuer's short dependent chain between stages is not starved of issue slots
+// by decode arithmetic. Dequant warps are the warps 7..27 with warp % 4 != 1 (sixteen of them);
+// warps 9, 13, 17, 21, 25 have no role and wait at the final barrier.
+constexpr int kGemm2Warps = 28;
+constexpr int kGemm2Threads = kGemm2Warps * 32;  // 896
+__device__ __forceinline__ int gemm2_dq_warp(int warp) {  // ordinal of a dequant warp, or -1
+  if (warp < kWarpDq0 || (warp & 3) == 1) return -1;
+  const int q = warp - kWarpDq0;
+  return q - (q + 1) / 4;
+}
+
+template <int QT, bool TRANS>
+struct Gemm2Cfg {
+  static constexpr int BN = 256;                 // pair tile N (output columns)
+  static constexpr int HN = 128;                 // this CTA's half of N
+  static constexpr int GB = QTraits<QT>::kGroupBytes;
+  static constexpr int A_BYTES = 128 * kBK * 2;  // 16 KB
+  static constexpr int B_BYTES = HN * kBK * 2;   // 16 KB
+  static constexpr int RAW_ROWS = TRANS ? 64 : 128;
+  static constexpr int RAW_BYTES = RAW_ROWS * GB;
+  static constexpr int STAGES = TRANS ? (GB > 200 ? 4 : 5) : (GB > 200 ? 4 : 5);
+  static constexpr int RAW_SLOTS = TRANS ? (GB > 200 ? 5 : 6) : (GB > 200 ? 2 : 3);
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+  static constexpr int OFF_RAW = OFF_B + STAGES * B_BYTES;
+  static constexpr int OFF_BAR = OFF_RAW + RAW_SLOTS * RAW_BYTES;
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * RAW_SLOTS + 5;
+  static constexpr int SIG_BYTES = 16 * (kNumDqWarps / 2);  // peer dequant signals per quantized step
+  static constexpr int OFF_SIG = (OFF_BAR + NUM_BARS * 8 + 16 + 127) / 128 * 128;  // signal landing area
+  static constexpr int SMEM_BYTES = OFF_SIG + 16 * kNumDqWarps + 1024;
+  static constexpr int ACC_COLS = BN;
+  static constexpr int TMEM_COLS = 512;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(RAW_BYTES % 128 == 0, "raw slot alignment");
+};
+
+// Dense pair tiles: t -> (256-row block, 256-column block, K part).
+__device__ __forceinline__ bool gemm2_tile(const GemmParams& p, int t, TileInfo& ti) {
+  const int kb_main = p.Kd / kBK;
+  if (t >= p.num_m_blocks * p.num_n_tiles * p.ksplit) return false;
+  ti.ks = t % p.ksplit;
+  const int rest = t / p.ksplit;
+  const int mb = rest % p.num_m_blocks;
+  ti.nb = rest / p.num_m_blocks;
+  ti.row0 = mb * 256;
+  ti.row_end = p.M;
+  ti.e = 0;
+  ti.kb_lo = ti.ks * p.kb_per_split;
+  ti.kb_hi = min(kb_main, ti.kb_lo + p.kb_per_split);
+  ti.lora = ti.ks == p.ksplit - 1;
+  return true;
+}
+
+template <int QT, bool TRANS>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm2Threads, 1)
+    qgemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
+                  const __grid_constant__ CUtensorMap tmLA, const __grid_constant__ CUtensorMap tmLB,
+                  const GemmParams p) {
+  using C = Gemm2Cfg<QT, TRANS>;
+  constexpr int BN = C::BN;
+  extern __shared__ uint8_t smem_raw_[];
+  const uint32_t base_u32 = (smem_u32(smem_raw_) + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw_ + (base_u32 - smem_u32(smem_raw_));
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cta_rank_in_cluster();  // 0 = leader
+  const bool leader = rank == 0;
+  const int cid = blockIdx.x >> 1;
+  const int ncl = gridDim.x >> 1;
+
+  const uint32_t sA = base_u32 + C::OFF_A;
+  const uint32_t sB = base_u32 + C::OFF_B;
+  const uint32_t sRaw = base_u32 + C::OFF_RAW;
+  const uint32_t bar0 = base_u32 + C::OFF_BAR;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
+  auto rfull_bar = [&](int s) { return bar0 + 8u * (2 * C::STAGES + s); };
+  auto rempty_bar = [&](int s) { return bar0 + 8u * (2 * C::STAGES + C::RAW_SLOTS + s); };
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 2 * C::RAW_SLOTS + b); };
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 2 * C::RAW_SLOTS + 2 + b); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * C::STAGES + 2 * C::RAW_SLOTS + 4);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + C::NUM_BARS * 8);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(full_bar(s), 1 + kNumDqWarps / 2);  // leader TMA (+ peer signal bytes) + leader dequant group
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int s = 0; s < C::RAW_SLOTS; ++s) {
+      mbar_init(rfull_bar(s), 1);
+      mbar_init(rempty_bar(s), TRANS ? kNumDqWarps / 2 : kNumDqWarps);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), 2 * kNumEpiWarps);
+    }
+    mbar_init(drain_bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc_pair(smem_u32(tmem_holder), C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  if (warp == kWarpTmaA && lane == 0) {
+    prefetch_tmap(&tmA);
+    if (p.n_lora_kb) { prefetch_tmap(&tmLA); prefetch_tmap(&tmLB); }
+  }
+  if (warp == kWarpTmaW && lane == 0) prefetch_tmap(&tmW);
+  tc_fence_before();
+  __syncthreads();
+  cluster_arrive_wait();  // both CTAs' barriers exist before any cross-CTA arrival
+  tc_fence_after();
+  const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
+
+  const int kb_main = p.Kd / kBK;
+  auto tile_steps = [&](const TileInfo& ti) { return (ti.kb_hi - ti.kb_lo) + (ti.lora ? p.n_lora_kb : 0); };
+  auto step_kb = [&](const TileInfo& ti, int i) {
+    const int nq = ti.kb_hi - ti.kb_lo;
+    return i < nq ? ti.kb_lo + i : kb_main + (i - nq);
+  };
+  // the leader's copies of the full / tempty barriers, as cluster addresses
+  auto full_leader = [&](int s) { return map_to_rank(full_bar(s), 0); };
+  auto tempty_leader = [&](int b) { return map_to_rank(tempty_bar(b), 0); };
+
+  if (warp == kWarpTmaA) {
+    // ---------------- A rows (and LoRA operands) of this CTA ----------------
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      bool issued = false;
+      TileInfo ti;
+      for (int t = cid; ok && gemm2_tile(p, t, ti); t += ncl) {
+        const int nsteps = tile_steps(ti);
+        const int arow = ti.row0 + 128 * (int)rank;
+        for (int i = 0; i < nsteps; ++i, ++it) {
+          const int kb = step_kb(ti, i);
+          const int s = it % C::STAGES;
+          const uint32_t ph = (it / C::STAGES) & 1;
+          if (!mbar_wait(empty_bar(s), ph ^ 1, 11)) { ok = false; break; }
+          const uint32_t fb = full_leader(s);
+          if (kb < kb_main) {
+            if (leader) mbar_arrive_expect_tx(full_bar(s), 2 * C::A_BYTES + C::SIG_BYTES);
+            tma_load_2d_pair(sA + s * C::A_BYTES, &tmA, fb, kb * kBK, arow);
+          } else {
+            const int x = (kb - kb_main) * kBK;
+            if (leader) mbar_arrive_expect_tx(full_bar(s), 2 * (C::A_BYTES + C::B_BYTES));
+            tma_load_2d_pair(sA + s * C::A_BYTES, &tmLA, fb, x, arow);
+            const int lb = ti.nb * BN + C::HN * (int)rank;
+            tma_load_2d_pair(sB + s * C::B_BYTES, &tmLB, fb, x, lb);
+            tma_load_2d_pair(sB + s * C::B_BYTES + 64 * 128, &tmLB, fb, x, lb + 64);
+          }
+          issued = true;
+        }
+      }
+      // copies still in flight complete on the leader's barrier, which this CTA cannot wait on
+      // once the pipeline has given up: give them time to land before the CTA may exit
+      if (!ok && issued) spin_ns(2000000ull);
+    }
+  } else if (warp == kWarpTmaW) {
+    // ---------------- packed groups of this CTA's half ----------------
+    if (lane == 0) {
+      int rc = 0;
+      bool ok = true;
+      int last_phase[8];
+      for (int s = 0; s < C::RAW_SLOTS; ++s) last_phase[s] = -1;
+      constexpr int GW = C::GB / 4;
+      TileInfo ti;
+      for (int t = cid; ok && gemm2_tile(p, t, ti); t += ncl) {
+        const int c_lo = TRANS ? ti.kb_lo : ti.kb_lo / 4;
+        const int c_hi = TRANS ? ti.kb_hi : ti.kb_hi / 4;
+        for (int c = c_lo; c < c_hi; ++c, ++rc) {
+          const int s = rc % C::RAW_SLOTS;
+          const uint32_t ph = (rc / C::RAW_SLOTS) & 1;
+          if (!mbar_wait(rempty_bar(s), ph ^ 1, 12)) { ok = false; break; }
+          mbar_arrive_expect_tx(rfull_bar(s), C::RAW_BYTES);
+          const uint32_t dst = sRaw + s * C::RAW_BYTES;
+          if (TRANS) {
+            tma_load_2d(dst, &tmW, rfull_bar(s), ti.nb * GW, c * 64);
+          } else {
+            const int y0 = ti.nb * BN + C::HN * (int)rank;
+            tma_load_2d(dst, &tmW, rfull_bar(s), c * GW, y0);
+            tma_load_2d(dst + 64 * C::GB, &tmW, rfull_bar(s), c * GW, y0 + 64);
+          }
+          last_phase[s] = (int)ph;
+        }
+      }
+      if (!ok) {
+        for (int s = 0; s < C::RAW_SLOTS; ++s)
+          if (last_phase[s] >= 0) mbar_wait(rfull_bar(s), (uint32_t)last_phase[s], 0, false, 2000000ull);
+      }
+    }
+  } else if (warp == kWarpMma) {
+    // ---------------- pair MMA issuer (leader) ----------------
+    if (lane == 0 && leader) {
+      int s = 0, tc = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      bool issued = false;
+      TileInfo ti;
+      constexpr uint32_t idesc_main = idesc_bf16(256, BN, TRANS);
+      constexpr uint32_t idesc_kmaj = idesc_bf16(256, BN, false);
+      // descriptors of stage 0; stage s adds s * bytes / 16 to the start-address field
+      const uint64_t adesc0 = smem_desc_sw128(sA, 16, 1024);
+      const uint64_t bdesc0_k = smem_desc_sw128(sB, 16, 1024);
+      const uint64_t bdesc0_mn = smem_desc_sw128(sB, 1024, 2048);
+      for (int t = cid; ok && gemm2_tile(p, t, ti); t += ncl, ++tc) {
+        const int buf = tc & 1;
+        if (!mbar_wait<true>(tempty_bar(buf), ((tc >> 1) & 1) ^ 1, 13)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * C::ACC_COLS;
+        const int nq = ti.kb_hi - ti.kb_lo;
+        const int nsteps = tile_steps(ti);
+        for (int i = 0; i < nsteps; ++i) {
+          if (!mbar_wait(full_bar(s), ph, 14)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t ad = adesc0 + (uint64_t)(s * (C::A_BYTES >> 4));
+          const bool kmaj = !TRANS || i >= nq;
+          if (kmaj) {
+            const uint64_t bd = bdesc0_k + (uint64_t)(s * (C::B_BYTES >> 4));
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k)
+              umma_bf16_pair(d_tmem, ad + 2 * k, bd + 2 * k, idesc_kmaj, (i | k) != 0);
+          } else {
+            const uint64_t bd = bdesc0_mn + (uint64_t)(s * (C::B_BYTES >> 4));
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k)
+              umma_bf16_pair(d_tmem, ad + 2 * k, bd + 256 * k, idesc_main, (i | k) != 0);
+          }
+          umma_commit_pair_both(empty_bar(s));
+          issued = true;
+          if (++s == C::STAGES) { s = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit_pair_both(tfull_bar(buf));
+      }
+      if (issued) {
+        umma_commit_pair(map_to_rank(drain_bar, 0));
+        mbar_wait(drain_bar, 0, 0, false, 2000000ull);
+      }
+    }
+  } else if (gemm2_dq_warp(warp) >= 0) {
+    // ---------------- dequant workers: this CTA's half of B ----------------
+    const int dq = gemm2_dq_warp(warp) * 32 + lane;
+    const int grp = dq >> 8;
+    const int gt = dq & 255;
+    // this warp's 16-byte slot of the signal area (the same offset in both CTAs)
+    const uint32_t sig = base_u32 + C::OFF_SIG + 16u * (uint32_t)(dq >> 5);
+    auto signal_full = [&](int s) {
+      if (leader) mbar_arrive(full_bar(s));
+      else bulk_signal_peer(map_to_rank(sig, 0), sig, 16, full_leader(s));
+    };
+    int it = 0, rc = 0;
+    bool ok = true;
+    TileInfo ti;
+    for (int t = cid; ok && gemm2_tile(p, t, ti); t += ncl) {
+      if (!TRANS) {
+        for (int g = ti.kb_lo / 4; ok && g < ti.kb_hi / 4; ++g, ++rc) {
+          const int rs = rc % C::RAW_SLOTS;
+          if (!warp_wait(rfull_bar(rs), (rc / C::RAW_SLOTS) & 1, 15)) { ok = false; break; }
+          const uint8_t* raw = smem + C::OFF_RAW + rs * C::RAW_BYTES;
+          for (int sub = 0; sub < 4; ++sub, ++it) {
+            if ((it & 1) != grp) continue;
+            const int s = it % C::STAGES;
+            if (!warp_wait(empty_bar(s), ((it / C::STAGES) & 1) ^ 1, 16)) { ok = false; break; }
+            uint8_t* sb = smem + C::OFF_B + s * C::B_BYTES;
+            {
+              const int row = gt >> 1, uh = gt & 1;
+              uint4 v[4];
+              decode_unit_bf16<QT>(raw + row * C::GB, 2 * sub + uh, v);
+#pragma unroll
+              for (int cc = 0; cc < 4; ++cc) {
+                const int c8 = 4 * uh + cc;
+                *reinterpret_cast<uint4*>(sb + row * 128 + ((c8 ^ (row & 7)) << 4)) = v[cc];
+              }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) signal_full(s);
+          }
+          __syncwarp();
+          if (ok && lane == 0) mbar_arrive(rempty_bar(rs));
+        }
+      } else {
+        for (int kb = ti.kb_lo; ok && kb < ti.kb_hi; ++kb, ++rc, ++it) {
+          if ((it & 1) != grp) continue;
+          const int rs = rc % C::RAW_SLOTS;
+          if (!warp_wait(rfull_bar(rs), (rc / C::RAW_SLOTS) & 1, 15)) { ok = false; break; }
+          const int s = it % C::STAGES;
+          if (!warp_wait(empty_bar(s), ((it / C::STAGES) & 1) ^ 1, 16)) { ok = false; break; }
+          const uint8_t* raw = smem + C::OFF_RAW + rs * C::RAW_BYTES;
+          uint8_t* sb = smem + C::OFF_B + s * C::B_BYTES;
+          {
+            // this CTA's 128 output columns are half `rank` of the 256-column group
+            const int kk = gt >> 2, ul = gt & 3;
+            uint4 v[4];
+            decode_unit_bf16<QT>(raw + kk * C::GB, 4 * (int)rank + ul, v);
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              const int gc = 4 * ul + cc;
+              const int off = (kk >> 3) * 2048 + (gc >> 3) * 1024 + (kk & 7) * 128 + (((gc & 7) ^ (kk & 7)) << 4);
+              *reinterpret_cast<uint4*>(sb + off) = v[cc];
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            signal_full(s);
+            mbar_arrive(rempty_bar(rs));
+          }
+        }
+      }
+      for (int i = 0; ok && ti.lora && i < p.n_lora_kb; ++i, ++it) {
+        if ((it & 1) != grp) continue;
+        const int s = it % C::STAGES;
+        if (!warp_wait(empty_bar(s), ((it / C::STAGES) & 1) ^ 1, 17)) { ok = false; break; }
+        __syncwarp();
+        if (lane == 0 && leader) mbar_arrive(full_bar(s));  // the peer has nothing to signal here
+      }
+    }
+  } else if (warp < kNumEpiWarps) {
+    // ---------------- epilogue: this CTA's 128 rows x 256 columns ----------------
+    int tc = 0;
+    TileInfo ti;
+    for (int t = cid; gemm2_tile(p, t, ti); t += ncl, ++tc) {
+      const int buf = tc & 1;
+      if (!warp_wait(tfull_bar(buf), (tc >> 1) & 1, 18)) break;
+      tc_fence_after();
+      const int row = ti.row0 + 128 * (int)rank + warp * 32 + lane;
+      const bool valid = row < ti.row_end;
+      const uint32_t tbase = tmem_base + ((uint32_t)(warp * 32) << 16) + buf * C::ACC_COLS;
+      epilogue_rows<EPI_STORE, BN>(p, ti, row, valid, tbase);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader(buf));
+    }
+  }
+
+  tc_fence_before();
+  // after a wait gave up, copies issued before it (TMA loads, peer signals) may still be in flight
+  // towards either CTA's shared memory: let them land before the pair can exit
+  if (threadIdx.x == 0 && dev_aborted()) spin_ns(2000000ull);
+  __syncthreads();
+  cluster_arrive_wait();  // no CTA leaves while the pair MMAs or the peer may still touch it
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace qlora

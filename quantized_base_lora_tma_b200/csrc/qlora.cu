@@ -11,6 +11,7 @@
 #include "qlora.h"
 #include "lora.cuh"
 #include "qgemm.cuh"
+#include "qgemm2.cuh"
 #include "moe.cuh"
 
 namespace qlora {
@@ -124,6 +125,55 @@ static int launch_qgemm_q(int qtype, const CUtensorMap& tA, const CUtensorMap& t
     case QL_Q8_0: return launch_qgemm<QL_Q8_0, TRANS, EPI, MS>(tA, tW, tLA, tLB, p, grid, st, slot);
     case QL_Q4_0: return launch_qgemm<QL_Q4_0, TRANS, EPI, MS>(tA, tW, tLA, tLB, p, grid, st, slot);
     case QL_Q4_K: return launch_qgemm<QL_Q4_K, TRANS, EPI, MS>(tA, tW, tLA, tLB, p, grid, st, slot);
+    default: return QL_ERR_UNSUPPORTED;
+  }
+}
+
+// Pair-tile dense GEMM: clusters of two CTAs, one cluster per pair tile slot. The grid is capped at
+// the number of clusters that can be resident at once (a persistent kernel must never have CTAs
+// waiting for a free SM pair).
+template <int QT, bool TRANS>
+static int launch_qgemm2(const CUtensorMap& tA, const CUtensorMap& tW, const CUtensorMap& tLA, const CUtensorMap& tLB,
+                         const GemmParams& p, int tiles, cudaStream_t st, int slot) {
+  using C = Gemm2Cfg<QT, TRANS>;
+  auto k = qgemm2_kernel<QT, TRANS>;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+    return QL_ERR_CUDA;
+  static int max_clusters[16] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int& mc = max_clusters[dev & 15];
+  if (mc <= 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (num_sms() / 2));
+    cfg.blockDim = dim3(kGemm2Threads);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, k, &cfg) != cudaSuccess || n <= 0) return QL_ERR_CUDA;
+    mc = n;
+  }
+  const int clusters = std::min(tiles, mc);
+  ev_record(slot, 0, st);
+  k<<<2 * clusters, kGemm2Threads, C::SMEM_BYTES, st>>>(tA, tW, tLA, tLB, p);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  ev_record(slot, 1, st);
+  return launch_status();
+}
+
+template <bool TRANS>
+static int launch_qgemm2_q(int qtype, const CUtensorMap& tA, const CUtensorMap& tW, const CUtensorMap& tLA,
+                           const CUtensorMap& tLB, const GemmParams& p, int tiles, cudaStream_t st, int slot) {
+  switch (qtype) {
+    case QL_Q8_0: return launch_qgemm2<QL_Q8_0, TRANS>(tA, tW, tLA, tLB, p, tiles, st, slot);
+    case QL_Q4_0: return launch_qgemm2<QL_Q4_0, TRANS>(tA, tW, tLA, tLB, p, tiles, st, slot);
+    case QL_Q4_K: return launch_qgemm2<QL_Q4_K, TRANS>(tA, tW, tLA, tLB, p, tiles, st, slot);
     default: return QL_ERR_UNSUPPORTED;
   }
 }
@@ -282,25 +332,28 @@ static int launch_colred(const __nv_bfloat16* Y, long ldy, int Ccols, const floa
   return launch_status();
 }
 
-// Tile plan of a dense GEMM: BM = 128 * MS rows per tile; K split into ksplit parts of
-// kb_per_split k-blocks (a multiple of 4 in forward mode) when the output has fewer tiles than
-// there are SMs (the small-M, weight-streaming regime).
+// Tile plan of a dense GEMM. With more than 128 rows the tiles are pair tiles of 256 x 256 computed
+// by two CTAs (pair = true); otherwise 128 x 128 tiles on one CTA. K is split into ksplit parts of
+// kb_per_split k-blocks (a multiple of 4 in forward mode) when the output has fewer tiles than there
+// are tile slots (SMs, or SM pairs): the small-M, weight-streaming regime.
 struct DensePlan {
-  int MS, ksplit, kbs, mblocks, ntiles;
+  bool pair;
+  int ksplit, kbs, mblocks, ntiles;
 };
 static DensePlan plan_dense(int64_t M, int64_t Nd, int64_t Kd, bool trans, bool allow_split) {
   DensePlan d;
-  d.MS = M > 128 ? 2 : 1;
-  d.mblocks = (int)((M + 128 * d.MS - 1) / (128 * d.MS));
-  d.ntiles = (int)((Nd + 127) / 128);
+  d.pair = M > 128;
+  const int tm = d.pair ? 256 : 128, tn = d.pair ? 256 : 128;
+  d.mblocks = (int)((M + tm - 1) / tm);
+  d.ntiles = (int)((Nd + tn - 1) / tn);
   const int kb_main = (int)(Kd / 64);
   const int unit = trans ? 1 : 4;
   d.ksplit = 1;
   d.kbs = kb_main;
   const int tiles = d.mblocks * d.ntiles;
-  const int nsm = num_sms();
-  if (allow_split && tiles < nsm) {
-    int ks = std::min((4 * nsm + tiles - 1) / tiles, std::min(kb_main / unit, 32));
+  const int slots = d.pair ? num_sms() / 2 : num_sms();
+  if (allow_split && tiles < slots) {
+    int ks = std::min((4 * slots + tiles - 1) / tiles, std::min(kb_main / unit, 32));
     if (ks > 1) {
       int kbs = (kb_main + ks - 1) / ks;
       kbs = (kbs + unit - 1) / unit * unit;
@@ -332,7 +385,7 @@ static int launch_dense_gemm(int qtype, const void* A, int64_t M, int64_t Kd, co
                              int64_t w_cols, const __nv_bfloat16* LA, const __nv_bfloat16* LB, int KL, int64_t Nd,
                              void* out, int out_dtype, float* split_buf, bool allow_split, cudaStream_t st, int slot) {
   const DensePlan d = plan_dense(M, Nd, Kd, TRANS, allow_split && split_buf != nullptr);
-  const uint32_t box = 128u * d.MS;
+  const uint32_t box = 128u;
   CUtensorMap tA, tW, tLA, tLB;
   if (!tmap_bf16_rows(&tA, A, Kd, M, box) ||
       !tmap_packed(&tW, wq, packed_row_bytes(qtype, w_cols), w_rows, group_bytes(qtype)) ||
@@ -358,9 +411,9 @@ static int launch_dense_gemm(int qtype, const void* A, int64_t M, int64_t Kd, co
     p.out_dtype = out_dtype;
   }
   const int tiles = d.mblocks * d.ntiles * d.ksplit;
-  const int grid = std::min(tiles, num_sms());
-  int rc = d.MS == 2 ? launch_qgemm_q<TRANS, EPI_STORE, 2>(qtype, tA, tW, tLA, tLB, p, grid, st, slot)
-                     : launch_qgemm_q<TRANS, EPI_STORE, 1>(qtype, tA, tW, tLA, tLB, p, grid, st, slot);
+  int rc = d.pair ? launch_qgemm2_q<TRANS>(qtype, tA, tW, tLA, tLB, p, tiles, st, slot)
+                  : launch_qgemm_q<TRANS, EPI_STORE, 1>(qtype, tA, tW, tLA, tLB, p, std::min(tiles, num_sms()), st,
+                                                        slot);
   if (rc || d.ksplit == 1) return rc;
   return launch_split_reduce(split_buf, d.ksplit, (long)M * Nd, (long)M * Nd, out, out_dtype, st);
 }

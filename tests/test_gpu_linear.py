@@ -91,6 +91,8 @@ SMALL = [
     (64, 1024, 128, 64),
     (16, 2048, 512, 8),    # small M: the K range is split across CTAs (fwd and dX)
     (3, 1024, 1024, 4),
+    (1100, 512, 4096, 8),  # more pair tiles than SM pairs: forward without a K split
+    (1100, 4096, 512, 8),  # the same for the input-gradient GEMM
 ]
 
 
