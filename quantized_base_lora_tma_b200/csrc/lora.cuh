@@ -1,10 +1,14 @@
-// Adapter-side kernels of the layer (bandwidth-bound, CUDA cores, fp32 accumulation):
+// Adapter-side kernels of the layer (bandwidth-bound; warp-level bf16 MMA, fp32 accumulation):
 //
-//   lora_rows      out[m, j] = oscale * sum_k Y[m, k] Z(j, k)        H = X A^T,  G = s dY B
-//                  and the tensor-core operand LA[m] = [hi(v) | lo(v)], v = lscale * sum
-//   lora_bop       LB[n] = [Z(n, :) | Z(n, :)]                        B (forward) or A^T (dX)
-//   colred         part[slice, c, j] = sum_{m in slice} Y[m, c] Z[m, j]   then an ordered sum
-//                  over slices: dB = s dY^T H, dA = G^T X (deterministic: no atomics)
+//   rows     out[m, j] = oscale * sum_k Y[m, k] Z(j, k)        H = X A^T,  G = s dY B
+//            and the tensor-core operand LA[m] = [hi(v) | lo(v)], v = lscale * sum
+//   bop      LB[n] = [Z(n, :) | Z(n, :)]                        B (forward) or A^T (dX)
+//   colred   out[c, j] = sum_m Y[m, c] Z[m, j] over row slices, then an ordered sum over the
+//            slices: dB = dY^T split(s H), dA = split(G)^T X (deterministic: no atomics)
+//
+// Dense layer: lora_rows_cluster_kernel and colred_cluster_kernel stream their bf16 operand through
+// a cp.async ring and sum the slices in-cluster. Routed (grouped) layer: lora_rows_seg_kernel,
+// colred_mma_kernel + colred_reduce_kernel, lora_bop_vec_kernel.
 //
 // The fast LoRA backward these implement is the plain chain rule of the layer (Show HN: LoRA over
 // GGUF, "Things involved in the training": "Fast LoRA bwd formula like Unsloth for linear layer
@@ -27,86 +31,6 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 q, float (&f)[8]) {
   }
 }
 
-// Row-wise reduction against a small [r x Kin] operand Z(j, k) = Z[j*zj + k*zk].
-// One warp per row (ROWS rows per CTA of 8 warps); K in chunks of 256 staged in shared memory.
-// Grouped use: zexp[row] picks the expert (Z advances by z_exp_stride per expert); NULL = dense.
-// out: [M x r] fp32 (nullable); la: [M x 2RP] bf16 (nullable), RP = 32 * ceil(r / 32).
-template <int RM>
-__global__ void __launch_bounds__(256) lora_rows_kernel(const __nv_bfloat16* __restrict__ Y, long ldy, int M,
-                                                        int Kin, const __nv_bfloat16* __restrict__ Z, long zj,
-                                                        long zk, long z_exp_stride, const int* __restrict__ row_exp,
-                                                        int r, float oscale, float lscale, float* __restrict__ out,
-                                                        __nv_bfloat16* __restrict__ la, int RP) {
-  __shared__ __align__(16) __nv_bfloat16 zs[RM * 256];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * 8 + warp;
-  // rows of one CTA share an expert only in dense mode; grouped mode loads Z per warp
-  const bool grouped = row_exp != nullptr;
-  float acc[RM];
-#pragma unroll
-  for (int j = 0; j < RM; ++j) acc[j] = 0.f;
-  const int e = (grouped && row < M) ? __ldg(row_exp + row) : 0;
-  const __nv_bfloat16* Ze = Z + (long)e * z_exp_stride;
-  for (int k0 = 0; k0 < Kin; k0 += 256) {
-    if (!grouped) {
-      __syncthreads();
-      for (int idx = threadIdx.x; idx < r * 256; idx += 256) {
-        int j, kk;
-        if (zk == 1) { j = idx / 256; kk = idx % 256; } else { j = idx % r; kk = idx / r; }
-        const int k = k0 + kk;
-        zs[j * 256 + kk] = (k < Kin) ? Z[(long)j * zj + (long)k * zk] : __float2bfloat16(0.f);
-      }
-      __syncthreads();
-    }
-    if (row < M) {
-      const int k = k0 + 8 * lane;
-      if (k < Kin) {
-        float y[8];
-        bf16x8_to_f32(*reinterpret_cast<const uint4*>(Y + (long)row * ldy + k), y);
-#pragma unroll
-        for (int j = 0; j < RM; ++j) {
-          if (j < r) {
-            float z[8];
-            if (!grouped) {
-              bf16x8_to_f32(*reinterpret_cast<const uint4*>(zs + j * 256 + 8 * lane), z);
-            } else {
-#pragma unroll
-              for (int i = 0; i < 8; ++i) z[i] = __bfloat162float(Ze[(long)j * zj + (long)(k + i) * zk]);
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[j] = fmaf(y[i], z[i], acc[j]);
-          }
-        }
-      }
-    }
-  }
-  if (row >= M) return;
-#pragma unroll
-  for (int j = 0; j < RM; ++j) {
-    if (j < r) {
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
-    }
-  }
-  // lanes write distinct columns
-  for (int j = lane; j < 2 * RP; j += 32) {
-    float a = 0.f;
-#pragma unroll
-    for (int jj = 0; jj < RM; ++jj) if (jj == (j < RP ? j : j - RP)) a = acc[jj];
-    const int jr = j < RP ? j : j - RP;
-    if (out != nullptr && j < r) out[(long)row * r + j] = oscale * a;
-    if (la != nullptr) {
-      __nv_bfloat16 v = __float2bfloat16(0.f);
-      if (jr < r) {
-        const float x = lscale * a;
-        const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-        v = (j < RP) ? hi : __float2bfloat16_rn(x - __bfloat162float(hi));
-      }
-      la[(long)row * 2 * RP + j] = v;
-    }
-  }
-}
-
 // ------------------------------------------------------------------------------------------------
 // Tensor-core (mma.sync m16n8k16, bf16 in, fp32 accumulate) versions of the two adapter reductions.
 // These are small, bandwidth-bound contractions with r <= 64 output columns; the warp-level MMA
@@ -125,79 +49,6 @@ __device__ __forceinline__ uint32_t ldg_u32(const void* p) { return __ldg(reinte
 
 __device__ __forceinline__ uint32_t pack2_bf16(__nv_bfloat16 lo, __nv_bfloat16 hi) {
   return (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
-}
-
-// Split-K partial row products: part[ks][m][j] = sum_{k in slice ks} Y[m, k] Z(j, k), j < 8*NT.
-// Z(j, k) = Z[j*zj + k*zk]. Grid (ceil(M/64), KS), 128 threads; warp w owns rows 64*bx + 16w.
-template <int NT>
-__global__ void __launch_bounds__(128) lora_rows_mma_kernel(const __nv_bfloat16* __restrict__ Y, long ldy, int M,
-                                                            int Kin, int kchunk, const __nv_bfloat16* __restrict__ Z,
-                                                            long zj, long zk, int r, float* __restrict__ part) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, c = lane & 3;
-  const int m0 = blockIdx.x * 64 + warp * 16;
-  const int r0 = m0 + g, r1 = m0 + g + 8;
-  const int kb = blockIdx.y * kchunk;
-  const int ke = min(Kin, kb + kchunk);
-  float acc[NT][4];
-#pragma unroll
-  for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-  const __nv_bfloat16* y0 = Y + (long)min(r0, M - 1) * ldy;
-  const __nv_bfloat16* y1 = Y + (long)min(r1, M - 1) * ldy;
-  const bool v0 = r0 < M, v1 = r1 < M;
-#pragma unroll 4
-  for (int k = kb; k < ke; k += 16) {
-    const uint32_t a0 = v0 ? ldg_u32(y0 + k + 2 * c) : 0u;
-    const uint32_t a1 = v1 ? ldg_u32(y1 + k + 2 * c) : 0u;
-    const uint32_t a2 = v0 ? ldg_u32(y0 + k + 2 * c + 8) : 0u;
-    const uint32_t a3 = v1 ? ldg_u32(y1 + k + 2 * c + 8) : 0u;
-#pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      const int n = 8 * t + g;
-      uint32_t b0 = 0u, b1 = 0u;
-      if (n < r) {
-        const __nv_bfloat16* zp = Z + (long)n * zj;
-        if (zk == 1) {
-          b0 = ldg_u32(zp + k + 2 * c);
-          b1 = ldg_u32(zp + k + 2 * c + 8);
-        } else {
-          b0 = pack2_bf16(zp[(long)(k + 2 * c) * zk], zp[(long)(k + 2 * c + 1) * zk]);
-          b1 = pack2_bf16(zp[(long)(k + 2 * c + 8) * zk], zp[(long)(k + 2 * c + 9) * zk]);
-        }
-      }
-      mma_16816(acc[t], a0, a1, a2, a3, b0, b1);
-    }
-  }
-  constexpr int RN = 8 * NT;
-  float* o = part + (long)blockIdx.y * M * RN;
-#pragma unroll
-  for (int t = 0; t < NT; ++t) {
-    const int j = 8 * t + 2 * c;
-    if (v0) *reinterpret_cast<float2*>(o + (long)r0 * RN + j) = make_float2(acc[t][0], acc[t][1]);
-    if (v1) *reinterpret_cast<float2*>(o + (long)r1 * RN + j) = make_float2(acc[t][2], acc[t][3]);
-  }
-}
-
-// Ordered sum of the split-K partials; writes out[m][j] = oscale * v (j < r) and the split
-// operand la[m] = [hi(lscale v) | lo(lscale v)] (zero padded to 2*RP columns).
-__global__ void lora_rows_reduce_kernel(const float* __restrict__ part, int KS, int M, int RN, int r, float oscale,
-                                        float lscale, float* __restrict__ out, __nv_bfloat16* __restrict__ la,
-                                        int RP) {
-  const long total = (long)M * RP;
-  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total; i += (long)gridDim.x * blockDim.x) {
-    const int m = (int)(i / RP), j = (int)(i % RP);
-    float v = 0.f;
-    if (j < r)
-      for (int ks = 0; ks < KS; ++ks) v += part[((long)ks * M + m) * RN + j];
-    if (out != nullptr && j < r) out[(long)m * r + j] = oscale * v;
-    if (la != nullptr) {
-      const float x = lscale * v;
-      const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-      const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
-      la[(long)m * 2 * RP + j] = j < r ? hi : __float2bfloat16(0.f);
-      la[(long)m * 2 * RP + RP + j] = j < r ? lo : __float2bfloat16(0.f);
-    }
-  }
 }
 
 // Column reductions on tensor cores: part[slice][c][j] = sum_{m in slice} Y[m][c] * Zs[m][j], where
@@ -360,6 +211,19 @@ __device__ __forceinline__ float ld_dsmem_f32(const float* local, uint32_t rank)
   return v;
 }
 
+// sum over cluster ranks 0 .. n-1 (n <= 8) of the value at this shared address, added in rank
+// order; the remote loads are all issued before the first add
+__device__ __forceinline__ float cluster_sum_ordered(const float* local, int n) {
+  float x[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) x[q] = q < n ? ld_dsmem_f32(local, (uint32_t)q) : 0.f;
+  float v = 0.f;
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    if (q < n) v += x[q];
+  return v;
+}
+
 struct BopArgs {            // LB[n] = [Z(n, :) | Z(n, :)], zero padded (nullptr Z = none)
   const __nv_bfloat16* Z;
   long zn, zjs;
@@ -385,99 +249,165 @@ __device__ __forceinline__ void lora_bop_share(const BopArgs& bop, int r, int RP
   }
 }
 
-// Rows of out = Y Z^T for 64 rows per cluster column; cluster rank q sums k in
-// [q * kchunk, (q + 1) * kchunk). Z(j, k) = Z[j*zj + k*zk]. Writes out = oscale * sum (fp32 [M x r])
-// and la = split(lscale * sum). Every CTA also writes its share of the LB operand (bop).
+// ---- streamed tiles: 16-byte cp.async copies into a shared-memory ring ----------------------------
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  // src-size 0 fills the 16 bytes with zeros and reads nothing
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+constexpr int kRowsStages = 4;    // cp.async ring depth of the dense row products
+constexpr int kRowsTileK = 128;   // k per streamed tile (64 rows x 128 bf16)
+constexpr int kRowsYS = kRowsTileK + 8;  // padded tile row: ldmatrix rows land in distinct banks
+
+// Dynamic shared memory of lora_rows_cluster_kernel<NT> for a k range of kchunk.
+__host__ __device__ constexpr size_t rows_smem_bytes(int NT, int kchunk) {
+  return (size_t)kRowsStages * 64 * kRowsYS * 2 + (size_t)8 * NT * (kchunk + 8) * 2 + (size_t)64 * 8 * NT * 4;
+}
+
+// Rows of out = Y Z^T for 64 rows per cluster column (warp w owns rows 16w .. 16w+15); cluster rank
+// q sums k in [q * kchunk, (q + 1) * kchunk). Z(j, k) = Z[j*zj + k*zk] is staged once per CTA; the
+// rows of Y stream through a ring of 64 x 128 tiles (cp.async, kRowsStages deep) into ldmatrix-fed
+// mma.sync. The ranks' partials are summed through distributed shared memory in rank order.
+// Writes out = oscale * sum (fp32 [M x r]) and la = split(lscale * sum) ([M x 2RP] bf16); when
+// hin is given also hs = split(hscale * hin) for the same rows; every CTA also writes its share of
+// the LB operand (bop). CTAs with blockIdx.x >= row_blocks (whole clusters) only write LB.
 template <int NT>
-__global__ void __launch_bounds__(128) lora_rows_cluster_kernel(const __nv_bfloat16* __restrict__ Y, long ldy, int M,
-                                                                int Kin, int kchunk, const __nv_bfloat16* __restrict__ Z,
-                                                                long zj, long zk, int r, float oscale, float lscale,
-                                                                float* __restrict__ out, __nv_bfloat16* __restrict__ la,
-                                                                int RP, BopArgs bop, __nv_bfloat16* __restrict__ LB,
-                                                                int row_blocks) {
-  // CTAs with blockIdx.x >= row_blocks (whole clusters) only write their share of LB.
+__global__ void __launch_bounds__(128) lora_rows_cluster_kernel(
+    const __nv_bfloat16* __restrict__ Y, long ldy, int M, int Kin, int kchunk, const __nv_bfloat16* __restrict__ Z,
+    long zj, long zk, int r, float oscale, float lscale, float* __restrict__ out, __nv_bfloat16* __restrict__ la,
+    int RP, BopArgs bop, __nv_bfloat16* __restrict__ LB, int row_blocks, const float* __restrict__ hin, float hscale,
+    __nv_bfloat16* __restrict__ hs) {
   constexpr int RN = 8 * NT;
-  constexpr int SK = 128;       // k per staged sub-chunk
-  constexpr int ZS = SK + 8;    // padded row of the staged Z tile (bf16)
-  __shared__ float part[64 * RN];
-  __shared__ __align__(16) __nv_bfloat16 zs[RN * ZS];
+  constexpr int S = kRowsStages, TK = kRowsTileK, YS = kRowsYS;
+  extern __shared__ __align__(16) uint8_t rows_smem[];
   if ((int)blockIdx.x >= row_blocks) {
     lora_bop_share(bop, r, RP, LB);
     return;
   }
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, c = lane & 3;
+  const int ZS = kchunk + 8;
+  __nv_bfloat16* ring = reinterpret_cast<__nv_bfloat16*>(rows_smem);
+  __nv_bfloat16* zs = ring + S * 64 * YS;
+  float* part = reinterpret_cast<float*>(zs + RN * ZS);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int KS = gridDim.y;
   const uint32_t rank = cluster_ctarank();
-  const int m0 = blockIdx.x * 64 + warp * 16;
-  const int r0 = m0 + g, r1 = m0 + g + 8;
-  const bool v0 = r0 < M, v1 = r1 < M;
-  const __nv_bfloat16* y0 = Y + (long)min(r0, M - 1) * ldy;
-  const __nv_bfloat16* y1 = Y + (long)min(r1, M - 1) * ldy;
+  const int m0 = blockIdx.x * 64;
   const int kb = (int)rank * kchunk;
   const int ke = min(Kin, kb + kchunk);
-  float acc[NT][4];
+  const int nk = max(0, ke - kb);
+  const int ntiles = (nk + TK - 1) / TK;
+
+  auto issue = [&](int t) {
+    const uint32_t dst0 = smem_u32(ring + (t % S) * 64 * YS);
 #pragma unroll
-  for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-  for (int k0 = kb; k0 < ke; k0 += SK) {
-    const int nk = min(SK, ke - k0);  // multiple of 32
-    // this sub-chunk's rows of Y, 16 bytes per lane per k32 step, issued before the staging wait
-    uint4 xa[SK / 32], xb[SK / 32];
-#pragma unroll
-    for (int q = 0; q < SK / 32; ++q) {
-      const int k = k0 + 32 * q + 8 * c;
-      const bool in = 32 * q < nk;
-      xa[q] = (v0 && in) ? __ldg(reinterpret_cast<const uint4*>(y0 + k)) : make_uint4(0, 0, 0, 0);
-      xb[q] = (v1 && in) ? __ldg(reinterpret_cast<const uint4*>(y1 + k)) : make_uint4(0, 0, 0, 0);
+    for (int it = 0; it < 64 * (TK / 8) / 128; ++it) {
+      const int i = tid + 128 * it;
+      const int row = i / (TK / 8), q = i % (TK / 8);
+      const int k = kb + t * TK + 8 * q;
+      const bool v = (m0 + row < M) && (k < ke);
+      cp_async16(dst0 + (uint32_t)(row * YS + 8 * q) * 2, v ? (const void*)(Y + (long)(m0 + row) * ldy + k) : (const void*)Y,
+                 v);
     }
-    __syncthreads();
-    // stage Z(j, k0 .. k0+SK) as zs[j][k]
-    if (zk == 1) {
-      for (int i = threadIdx.x; i < RN * (SK / 8); i += 128) {
-        const int j = i / (SK / 8), q = i % (SK / 8);
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (j < r && 8 * q < nk) v = __ldg(reinterpret_cast<const uint4*>(Z + (long)j * zj + k0 + 8 * q));
-        *reinterpret_cast<uint4*>(zs + j * ZS + 8 * q) = v;
-      }
-    } else {
-      for (int i = threadIdx.x; i < RN * SK; i += 128) {
-        const int kk = i / RN, j = i % RN;  // consecutive threads read consecutive j of one k
-        __nv_bfloat16 v = __float2bfloat16(0.f);
-        if (j < r && kk < nk) v = Z[(long)j * zj + (long)(k0 + kk) * zk];
-        zs[j * ZS + kk] = v;
-      }
+  };
+  // the ring's first tiles are in flight while the LB share is written and Z is staged
+#pragma unroll
+  for (int t = 0; t < S - 1; ++t) {
+    if (t < ntiles) issue(t);
+    cp_async_commit();
+  }
+  lora_bop_share(bop, r, RP, LB);
+  if (zk == 1) {
+    for (int i = tid; i < RN * (kchunk / 8); i += 128) {
+      const int j = i / (kchunk / 8), q = i % (kchunk / 8);
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (j < r && 8 * q < nk) v = __ldg(reinterpret_cast<const uint4*>(Z + (long)j * zj + kb + 8 * q));
+      *reinterpret_cast<uint4*>(zs + j * ZS + 8 * q) = v;
     }
-    __syncthreads();
+  } else {
+    // strided Z: eight independent loads in flight per thread; consecutive threads read
+    // consecutive j of one k
+    const int total = kchunk * RN;
+    for (int i0 = tid; i0 < total; i0 += 128 * 8) {
+      __nv_bfloat16 v[8];
 #pragma unroll
-    for (int q = 0; q < SK / 32; ++q) {
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + 128 * u;
+        const int kk = i / RN, j = i % RN;
+        v[u] = (i < total && j < r && kk < nk) ? Z[(long)j * zj + (long)(kb + kk) * zk] : __float2bfloat16(0.f);
+      }
 #pragma unroll
-      for (int t = 0; t < NT; ++t) {
-        const uint4 zq = *reinterpret_cast<const uint4*>(zs + (8 * t + g) * ZS + 32 * q + 8 * c);
-        mma_16816(acc[t], xa[q].x, xb[q].x, xa[q].y, xb[q].y, zq.x, zq.y);
-        mma_16816(acc[t], xa[q].z, xb[q].z, xa[q].w, xb[q].w, zq.z, zq.w);
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + 128 * u;
+        if (i < total) zs[(i % RN) * ZS + i / RN] = v[u];
       }
     }
   }
+
+  float acc[NT][4];
 #pragma unroll
-  for (int t = 0; t < NT; ++t) {
-    const int j = 8 * t + 2 * c;
-    const int lr = warp * 16 + g;
-    part[lr * RN + j] = acc[t][0];
-    part[lr * RN + j + 1] = acc[t][1];
-    part[(lr + 8) * RN + j] = acc[t][2];
-    part[(lr + 8) * RN + j + 1] = acc[t][3];
+  for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+  // ldmatrix lane addresses: A = rows 16w + lane%16, k offset 8*(lane/16); B = Z rows (n) lane%8 +
+  // 8*(lane/16) of an n-tile pair, k offset 8*((lane/8)%2)
+  const int a_row = 16 * warp + (lane & 15), a_col = 8 * (lane >> 4);
+  const int b_row = (lane & 7) + 8 * (lane >> 4), b_col = 8 * ((lane >> 3) & 1);
+  for (int t = 0; t < ntiles; ++t) {
+    cp_async_wait<S - 2>();
+    __syncthreads();  // tile t visible to all; every thread is done with tile t - 1's slot
+    if (t + S - 1 < ntiles) issue(t + S - 1);
+    cp_async_commit();
+    const uint32_t abase = smem_u32(ring + (t % S) * 64 * YS + a_row * YS + a_col);
+    const uint32_t bbase = smem_u32(zs + b_row * ZS + t * TK + b_col);
+#pragma unroll
+    for (int k16 = 0; k16 < TK / 16; ++k16) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(abase + 32 * k16, a0, a1, a2, a3);
+#pragma unroll
+      for (int tp = 0; tp < NT / 2; ++tp) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(bbase + (uint32_t)(16 * tp * ZS) * 2 + 32 * k16, b0, b1, b2, b3);
+        mma_16816(acc[2 * tp], a0, a1, a2, a3, b0, b1);
+        mma_16816(acc[2 * tp + 1], a0, a1, a2, a3, b2, b3);
+      }
+    }
+  }
+  cp_async_wait<0>();
+  {
+    const int g = lane >> 2, c = lane & 3;
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      const int j = 8 * t + 2 * c;
+      const int lr = warp * 16 + g;
+      part[lr * RN + j] = acc[t][0];
+      part[lr * RN + j + 1] = acc[t][1];
+      part[(lr + 8) * RN + j] = acc[t][2];
+      part[(lr + 8) * RN + j + 1] = acc[t][3];
+    }
   }
   cluster_sync_all();
   // rank q reduces rows [q*64/KS, (q+1)*64/KS) of the cluster's 64 rows, over ranks in order
   const int rows_per = (64 + KS - 1) / KS;
   const int lr0 = (int)rank * rows_per;
-  for (int i = threadIdx.x; i < rows_per * RP; i += 128) {
+  for (int i = tid; i < rows_per * RP; i += 128) {
     const int lr = lr0 + i / RP, j = i % RP;
-    const int m = blockIdx.x * 64 + lr;
+    const int m = m0 + lr;
     if (lr >= 64 || m >= M) continue;
     float v = 0.f;
-    if (j < r)
-      for (int q = 0; q < KS; ++q) v += ld_dsmem_f32(&part[lr * RN + j], (uint32_t)q);
+    if (j < r) v = cluster_sum_ordered(&part[lr * RN + j], KS);
     if (out != nullptr && j < r) out[(long)m * r + j] = oscale * v;
     if (la != nullptr) {
       const float x = lscale * v;
@@ -486,39 +416,53 @@ __global__ void __launch_bounds__(128) lora_rows_cluster_kernel(const __nv_bfloa
       la[(long)m * 2 * RP + j] = j < r ? hi : __float2bfloat16(0.f);
       la[(long)m * 2 * RP + RP + j] = j < r ? lo : __float2bfloat16(0.f);
     }
+    if (hs != nullptr) {
+      const float x = j < r ? hscale * hin[(long)m * r + j] : 0.f;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+      hs[(long)m * 2 * RP + j] = hi;
+      hs[(long)m * 2 * RP + RP + j] = __float2bfloat16_rn(x - __bfloat162float(hi));
+    }
   }
-  lora_bop_share(bop, r, RP, LB);
   cluster_sync_all();  // no CTA leaves while a peer may still read its partials
 }
 
 // Two column-reduction problems in one launch (dense layer): problem p (blockIdx.x < nb0: p = 0)
-// computes out = scale * sum_m Y[m][c] Z[m][j] over all M rows; cluster rank q takes rows
-// [q * mchunk, (q + 1) * mchunk) and the ranks' partials are summed through DSMEM in rank order.
-// transpose = 0: out[c][j]; 1: out[j][c].
+// computes out = scale * sum_m Y[m][c] Z[m][j] over all M rows, for the 128 columns c of this CTA
+// (warp w: columns 32w .. 32w+31). Z is given as its bf16 split [M x 2RP] = [hi | lo] (the sum of
+// the two carries Z to about 2^-16 relative). Cluster rank q takes rows [q * mchunk, (q + 1) *
+// mchunk); 64-row tiles of Y and of the split Z stream through a cp.async ring into mma.sync
+// (A = Z^T by ldmatrix.trans, B = Y by ldmatrix.trans) and the ranks' partials are summed through
+// distributed shared memory in rank order. transpose = 0: out[c][j]; 1: out[j][c].
 struct ColredProblem {
   const __nv_bfloat16* Y;
   long ldy;
   int C;
-  const float* Z;
+  const __nv_bfloat16* Zs;
   float scale;
   int transpose;
   float* out;
 };
 
+constexpr int kColStages = 4;
+constexpr int kColYS = 128 + 8;  // padded row of a 64 x 128 Y tile (bf16)
+
+// Dynamic shared memory of colred_cluster_kernel: the ring, which later holds the partial tile
+// [16 * JT <= RP][129] fp32.
+__host__ __device__ constexpr size_t colred_smem_bytes(int RP) {
+  return (size_t)kColStages * 64 * (kColYS + 2 * RP + 8) * 2 > (size_t)RP * (128 + 1) * 4
+             ? (size_t)kColStages * 64 * (kColYS + 2 * RP + 8) * 2
+             : (size_t)RP * (128 + 1) * 4;
+}
+
 template <int JT>
 __global__ void __launch_bounds__(128) colred_cluster_kernel(ColredProblem p0, ColredProblem p1, int nb0, int M,
-                                                             int r, int mchunk) {
-  constexpr int YS = 128 + 8;
-  constexpr int HR = 64;
-  constexpr int Y_BYTES = HR * YS * 2;
-  constexpr int Z_BYTES = JT * 16 * (HR + 8) * 2;
-  constexpr int P_BYTES = JT * 16 * (128 + 1) * 4;
-  constexpr int BUF = (Y_BYTES + 2 * Z_BYTES) > P_BYTES ? (Y_BYTES + 2 * Z_BYTES) : P_BYTES;
-  __shared__ __align__(16) uint8_t sbuf[BUF];
-  __nv_bfloat16* ys = reinterpret_cast<__nv_bfloat16*>(sbuf);
-  auto zh = reinterpret_cast<__nv_bfloat16(*)[HR + 8]>(sbuf + Y_BYTES);
-  auto zl = reinterpret_cast<__nv_bfloat16(*)[HR + 8]>(sbuf + Y_BYTES + Z_BYTES);
-  auto part = reinterpret_cast<float(*)[128 + 1]>(sbuf);  // reused after the main loop
+                                                             int r, int RP, int mchunk) {
+  constexpr int S = kColStages, YS = kColYS;
+  extern __shared__ __align__(16) uint8_t col_smem[];
+  const int ZW = 2 * RP + 8;  // padded row of a 64 x 2RP split-Z tile
+  __nv_bfloat16* yring = reinterpret_cast<__nv_bfloat16*>(col_smem);
+  __nv_bfloat16* zring = yring + S * 64 * YS;
+  auto part = reinterpret_cast<float(*)[128 + 1]>(col_smem);  // reused after the main loop
   const bool second = (int)blockIdx.x >= nb0;
   const ColredProblem& P = second ? p1 : p0;
   const int c0 = (second ? (int)blockIdx.x - nb0 : (int)blockIdx.x) * 128;
@@ -526,53 +470,58 @@ __global__ void __launch_bounds__(128) colred_cluster_kernel(ColredProblem p0, C
   const int CS = gridDim.y;
   const int lo = (int)rank * mchunk;
   const int hi = min(M, lo + mchunk);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, c = lane & 3;
+  const int ntiles = hi > lo ? (hi - lo + 63) / 64 : 0;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  auto issue = [&](int t) {
+    const int mb = lo + 64 * t;
+    const uint32_t ydst = smem_u32(yring + (t % S) * 64 * YS);
+#pragma unroll
+    for (int it = 0; it < 64 * 16 / 128; ++it) {
+      const int i = tid + 128 * it;
+      const int m = i >> 4, q = i & 15;
+      const bool v = (mb + m < hi) && (c0 + 8 * q < P.C);
+      cp_async16(ydst + (uint32_t)(m * YS + 8 * q) * 2, v ? (const void*)(P.Y + (long)(mb + m) * P.ldy + c0 + 8 * q) : (const void*)P.Y, v);
+    }
+    const uint32_t zdst = smem_u32(zring + (t % S) * 64 * ZW);
+    const int zq = 2 * RP / 8;  // 16-byte chunks per split-Z row
+    for (int i = tid; i < 64 * zq; i += 128) {
+      const int m = i / zq, q = i % zq;
+      const bool v = mb + m < hi;
+      cp_async16(zdst + (uint32_t)(m * ZW + 8 * q) * 2, v ? (const void*)(P.Zs + (long)(mb + m) * 2 * RP + 8 * q) : (const void*)P.Zs, v);
+    }
+  };
+#pragma unroll
+  for (int t = 0; t < S - 1; ++t) {
+    if (t < ntiles) issue(t);
+    cp_async_commit();
+  }
+
   float acc[JT][4][4];
 #pragma unroll
   for (int jt = 0; jt < JT; ++jt)
 #pragma unroll
     for (int t = 0; t < 4; ++t) acc[jt][t][0] = acc[jt][t][1] = acc[jt][t][2] = acc[jt][t][3] = 0.f;
   const int wc = warp * 32;
-  for (int mb = lo; mb < hi; mb += HR) {
-    const int n = min(HR, hi - mb);
-    uint4 yv[HR * 16 / 128];
-#pragma unroll
-    for (int it = 0; it < HR * 16 / 128; ++it) {
-      const int i = threadIdx.x + 128 * it;
-      const int m = i >> 4, q = i & 15;
-      yv[it] = (m < n && c0 + 8 * q < P.C)
-                   ? __ldg(reinterpret_cast<const uint4*>(P.Y + (long)(mb + m) * P.ldy + c0 + 8 * q))
-                   : make_uint4(0, 0, 0, 0);
-    }
+  // ldmatrix.trans lane addresses. B (Y, k = m, n = c): matrices (m 0-7 | 8-15) x (c 0-7 | 8-15).
+  // A (Z^T, rows j, k = m): matrices (j 0-7, m 0-7), (j 8-15, m 0-7), (j 0-7, m 8-15), (j 8-15, m 8-15).
+  const int mat = lane >> 3, rr = lane & 7;
+  const int yb_row = ((mat & 1) ? 8 : 0) + rr, yb_col = wc + ((mat & 2) ? 8 : 0);
+  const int za_row = rr + ((mat & 2) ? 8 : 0), za_col = (mat & 1) ? 8 : 0;
+  for (int t = 0; t < ntiles; ++t) {
+    cp_async_wait<S - 2>();
     __syncthreads();
+    if (t + S - 1 < ntiles) issue(t + S - 1);
+    cp_async_commit();
+    const uint32_t ybase = smem_u32(yring + (t % S) * 64 * YS + yb_row * YS + yb_col);
+    const uint32_t zbase = smem_u32(zring + (t % S) * 64 * ZW + za_row * ZW + za_col);
 #pragma unroll
-    for (int it = 0; it < HR * 16 / 128; ++it) {
-      const int i = threadIdx.x + 128 * it;
-      *reinterpret_cast<uint4*>(ys + (i >> 4) * YS + 8 * (i & 15)) = yv[it];
-    }
-    for (int i = threadIdx.x; i < JT * 16 * HR; i += 128) {
-      const int j = i / HR, m = i % HR;
-      float z = 0.f;
-      if (m < n && j < r) z = P.Z[(long)(mb + m) * r + j];
-      const __nv_bfloat16 h = __float2bfloat16_rn(z);
-      zh[j][m] = h;
-      zl[j][m] = __float2bfloat16_rn(z - __bfloat162float(h));
-    }
-    __syncthreads();
-#pragma unroll 2
-    for (int k = 0; k < HR; k += 16) {
+    for (int k = 0; k < 64; k += 16) {
       uint32_t b[4][2];
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
-        const int mat = lane >> 3, rr = lane & 7;
-        const int krow = k + ((mat & 1) ? 8 : 0) + rr;
-        const int ncol = wc + 16 * h2 + ((mat & 2) ? 8 : 0);
-        const uint32_t addr = smem_u32(ys + krow * YS + ncol);
         uint32_t x0, x1, x2, x3;
-        asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                     : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3)
-                     : "r"(addr));
+        ldsm_x4_t(ybase + (uint32_t)(k * YS + 16 * h2) * 2, x0, x1, x2, x3);
         b[2 * h2][0] = x0;
         b[2 * h2][1] = x1;
         b[2 * h2 + 1][0] = x2;
@@ -580,45 +529,42 @@ __global__ void __launch_bounds__(128) colred_cluster_kernel(ColredProblem p0, C
       }
 #pragma unroll
       for (int jt = 0; jt < JT; ++jt) {
-        const int j0 = 16 * jt;
-        const uint32_t ah0 = *reinterpret_cast<const uint32_t*>(&zh[j0 + g][k + 2 * c]);
-        const uint32_t ah1 = *reinterpret_cast<const uint32_t*>(&zh[j0 + g + 8][k + 2 * c]);
-        const uint32_t ah2 = *reinterpret_cast<const uint32_t*>(&zh[j0 + g][k + 2 * c + 8]);
-        const uint32_t ah3 = *reinterpret_cast<const uint32_t*>(&zh[j0 + g + 8][k + 2 * c + 8]);
-        const uint32_t al0 = *reinterpret_cast<const uint32_t*>(&zl[j0 + g][k + 2 * c]);
-        const uint32_t al1 = *reinterpret_cast<const uint32_t*>(&zl[j0 + g + 8][k + 2 * c]);
-        const uint32_t al2 = *reinterpret_cast<const uint32_t*>(&zl[j0 + g][k + 2 * c + 8]);
-        const uint32_t al3 = *reinterpret_cast<const uint32_t*>(&zl[j0 + g + 8][k + 2 * c + 8]);
+        uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
+        ldsm_x4_t(zbase + (uint32_t)(k * ZW + 16 * jt) * 2, h0, h1, h2, h3);
+        ldsm_x4_t(zbase + (uint32_t)(k * ZW + RP + 16 * jt) * 2, l0, l1, l2, l3);
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          mma_16816(acc[jt][t], ah0, ah1, ah2, ah3, b[t][0], b[t][1]);
-          mma_16816(acc[jt][t], al0, al1, al2, al3, b[t][0], b[t][1]);
+        for (int n = 0; n < 4; ++n) {
+          mma_16816(acc[jt][n], h0, h1, h2, h3, b[n][0], b[n][1]);
+          mma_16816(acc[jt][n], l0, l1, l2, l3, b[n][0], b[n][1]);
         }
       }
     }
   }
-  __syncthreads();  // the staging buffers become the partial tile
+  cp_async_wait<0>();
+  __syncthreads();  // the ring becomes the partial tile
+  {
+    const int g = lane >> 2, c = lane & 3;
 #pragma unroll
-  for (int jt = 0; jt < JT; ++jt)
+    for (int jt = 0; jt < JT; ++jt)
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const int col = wc + 8 * t + 2 * c;
-      const int j0 = 16 * jt + g;
-      part[j0][col] = acc[jt][t][0];
-      part[j0][col + 1] = acc[jt][t][1];
-      part[j0 + 8][col] = acc[jt][t][2];
-      part[j0 + 8][col + 1] = acc[jt][t][3];
-    }
+      for (int n = 0; n < 4; ++n) {
+        const int col = wc + 8 * n + 2 * c;
+        const int j0 = 16 * jt + g;
+        part[j0][col] = acc[jt][n][0];
+        part[j0][col + 1] = acc[jt][n][1];
+        part[j0 + 8][col] = acc[jt][n][2];
+        part[j0 + 8][col + 1] = acc[jt][n][3];
+      }
+  }
   cluster_sync_all();
   // rank q reduces columns [q*128/CS, (q+1)*128/CS) over ranks in order
   const int cols_per = (128 + CS - 1) / CS;
   const int cl0 = (int)rank * cols_per;
-  for (int i = threadIdx.x; i < cols_per * r; i += 128) {
+  for (int i = tid; i < cols_per * r; i += 128) {
     const int cl = cl0 + i / r, j = i % r;
     const int col = c0 + cl;
     if (cl >= 128 || col >= P.C) continue;
-    float v = 0.f;
-    for (int q = 0; q < CS; ++q) v += ld_dsmem_f32(&part[j][cl], (uint32_t)q);
+    const float v = cluster_sum_ordered(&part[j][cl], CS);
     const long o = P.transpose ? (long)j * P.C + col : (long)col * r + j;
     P.out[o] = P.scale * v;
   }
@@ -751,82 +697,6 @@ __global__ void lora_bop_vec_kernel(const __nv_bfloat16* __restrict__ Z, long zn
       v[q] = j < r ? Z[(long)e * zes + (long)n * zn + (long)j * zjs] : __float2bfloat16(0.f);
     }
     *reinterpret_cast<uint4*>(LB + rn * 2 * RP + j0) = *reinterpret_cast<const uint4*>(v);
-  }
-}
-
-// LB[e*rows + n][j] = LB[..][RP + j] = Z(e, n, j) = Z[e*zes + n*zn + j*zjs] for j < r, else 0.
-__global__ void lora_bop_kernel(const __nv_bfloat16* __restrict__ Z, long zn, long zjs, long zes, int rows,
-                                int nexp, int r, int RP, __nv_bfloat16* __restrict__ LB) {
-  const long total = (long)nexp * rows * 2 * RP;
-  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total; i += (long)gridDim.x * blockDim.x) {
-    const int j2 = (int)(i % (2 * RP));
-    const long rn = i / (2 * RP);
-    const int n = (int)(rn % rows);
-    const int e = (int)(rn / rows);
-    const int j = j2 < RP ? j2 : j2 - RP;
-    LB[i] = (j < r) ? Z[(long)e * zes + (long)n * zn + (long)j * zjs] : __float2bfloat16(0.f);
-  }
-}
-
-// Partial column reductions over one slice of rows: part[slice][c][j] = sum_m Y[m][c] * Z[m][j]
-// for m in [row_lo, row_hi) of the slice; 128 threads x 2 columns per CTA, grid (C/256, slices).
-// Slices: dense mode slice s = rows [128 s, 128 s + 128); grouped mode slice s = m-block s of the
-// routed batch (seg_off / mblk_off / E as in the GEMM), never crossing an expert boundary.
-// zw (nullable) scales row m of Z by zw[m] (routing weight).
-template <int RM>
-__global__ void __launch_bounds__(128) colred_partial_kernel(const __nv_bfloat16* __restrict__ Y, long ldy, int Ccols,
-                                                             const float* __restrict__ Z, int r, int M,
-                                                             const float* __restrict__ zw, const int* __restrict__ seg_off,
-                                                             const int* __restrict__ mblk_off, int E,
-                                                             float* __restrict__ part) {
-  __shared__ float zs[128 * RM];
-  const int slice = blockIdx.y;
-  int lo, hi;
-  if (E == 0) {
-    lo = slice * 128;
-    hi = min(M, lo + 128);
-  } else {
-    const int total = __ldg(mblk_off + E);
-    if (slice >= total) return;
-    int a = 0, b = E - 1;
-    while (a < b) {
-      const int mid = (a + b + 1) >> 1;
-      if (__ldg(mblk_off + mid) <= slice) a = mid; else b = mid - 1;
-    }
-    lo = __ldg(seg_off + a) + (slice - __ldg(mblk_off + a)) * 128;
-    hi = min(__ldg(seg_off + a + 1), lo + 128);
-  }
-  const int n = hi - lo;
-  for (int i = threadIdx.x; i < n * r; i += 128) {
-    const int m = i / r, j = i % r;
-    float z = Z[(long)(lo + m) * r + j];
-    if (zw != nullptr) z *= zw[lo + m];
-    zs[m * RM + j] = z;
-  }
-  __syncthreads();
-  const int c = blockIdx.x * 256 + 2 * threadIdx.x;
-  if (c >= Ccols) return;
-  float a0[RM], a1[RM];
-#pragma unroll
-  for (int j = 0; j < RM; ++j) { a0[j] = 0.f; a1[j] = 0.f; }
-  for (int m = 0; m < n; ++m) {
-    const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(Y + (long)(lo + m) * ldy + c));
-#pragma unroll
-    for (int j = 0; j < RM; ++j) {
-      if (j < r) {
-        const float z = zs[m * RM + j];
-        a0[j] = fmaf(y.x, z, a0[j]);
-        a1[j] = fmaf(y.y, z, a1[j]);
-      }
-    }
-  }
-  float* o = part + ((long)slice * Ccols + c) * r;
-#pragma unroll
-  for (int j = 0; j < RM; ++j) {
-    if (j < r) {
-      o[j] = a0[j];
-      o[r + j] = a1[j];
-    }
   }
 }
 

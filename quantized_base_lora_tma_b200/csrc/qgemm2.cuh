@@ -37,17 +37,22 @@ __device__ __forceinline__ int gemm2_dq_warp(int warp) {  // ordinal of a dequan
   return q - (q + 1) / 4;
 }
 
-template <int QT, bool TRANS>
+// MS = 1: 256 x 256 pair tiles (each CTA 128 A rows), double-buffered accumulators.
+// MS = 2: 512 x 256 pair tiles: each CTA holds two 128-row A blocks per stage and every dequantized
+// B half feeds two pair MMAs (half the dequant work per FLOP); the two accumulators fill TMEM, so
+// the epilogue of a tile is not overlapped with the next tile's main loop.
+template <int QT, bool TRANS, int MS>
 struct Gemm2Cfg {
   static constexpr int BN = 256;                 // pair tile N (output columns)
   static constexpr int HN = 128;                 // this CTA's half of N
+  static constexpr int BM = 256 * MS;            // pair tile M
   static constexpr int GB = QTraits<QT>::kGroupBytes;
-  static constexpr int A_BYTES = 128 * kBK * 2;  // 16 KB
+  static constexpr int A_BYTES = MS * 128 * kBK * 2;  // 16 / 32 KB
   static constexpr int B_BYTES = HN * kBK * 2;   // 16 KB
   static constexpr int RAW_ROWS = TRANS ? 64 : 128;
   static constexpr int RAW_BYTES = RAW_ROWS * GB;
-  static constexpr int STAGES = TRANS ? (GB > 200 ? 4 : 5) : (GB > 200 ? 4 : 5);
-  static constexpr int RAW_SLOTS = TRANS ? (GB > 200 ? 5 : 6) : (GB > 200 ? 2 : 3);
+  static constexpr int STAGES = MS == 2 ? 3 : (GB > 200 ? 4 : 5);
+  static constexpr int RAW_SLOTS = TRANS ? (GB > 200 ? (MS == 2 ? 4 : 5) : 6) : (GB > 200 ? 2 : 3);
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
   static constexpr int OFF_RAW = OFF_B + STAGES * B_BYTES;
@@ -56,13 +61,16 @@ struct Gemm2Cfg {
   static constexpr int SIG_BYTES = 16 * (kNumDqWarps / 2);  // peer dequant signals per quantized step
   static constexpr int OFF_SIG = (OFF_BAR + NUM_BARS * 8 + 16 + 127) / 128 * 128;  // signal landing area
   static constexpr int SMEM_BYTES = OFF_SIG + 16 * kNumDqWarps + 1024;
-  static constexpr int ACC_COLS = BN;
+  static constexpr int ACC_COLS = MS * BN;       // TMEM columns of one tile's accumulators
+  static constexpr int NBUF = MS == 1 ? 2 : 1;   // accumulator buffers
   static constexpr int TMEM_COLS = 512;
+  static_assert(NBUF * ACC_COLS <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(RAW_BYTES % 128 == 0, "raw slot alignment");
 };
 
-// Dense pair tiles: t -> (256-row block, 256-column block, K part).
+// Dense pair tiles: t -> (BM-row block, 256-column block, K part).
+template <int BM>
 __device__ __forceinline__ bool gemm2_tile(const GemmParams& p, int t, TileInfo& ti) {
   const int kb_main = p.Kd / kBK;
   if (t >= p.num_m_blocks * p.num_n_tiles * p.ksplit) return false;
@@ -70,7 +78,7 @@ __device__ __forceinline__ bool gemm2_tile(const GemmParams& p, int t, TileInfo&
   const int rest = t / p.ksplit;
   const int mb = rest % p.num_m_blocks;
   ti.nb = rest / p.num_m_blocks;
-  ti.row0 = mb * 256;
+  ti.row0 = mb * BM;
   ti.row_end = p.M;
   ti.e = 0;
   ti.kb_lo = ti.ks * p.kb_per_split;
@@ -79,12 +87,12 @@ __device__ __forceinline__ bool gemm2_tile(const GemmParams& p, int t, TileInfo&
   return true;
 }
 
-template <int QT, bool TRANS>
+template <int QT, bool TRANS, int MS>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm2Threads, 1)
     qgemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
                   const __grid_constant__ CUtensorMap tmLA, const __grid_constant__ CUtensorMap tmLB,
                   const GemmParams p) {
-  using C = Gemm2Cfg<QT, TRANS>;
+  using C = Gemm2Cfg<QT, TRANS, MS>;
   constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw_[];
   const uint32_t base_u32 = (smem_u32(smem_raw_) + 1023u) & ~1023u;
@@ -158,7 +166,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm2Threads, 1)
       bool ok = true;
       bool issued = false;
       TileInfo ti;
-      for (int t = cid; ok && gemm2_tile(p, t, ti); t += ncl) {
+      for (int t = cid; ok && gemm2_tile<C::BM>(p, t, ti); t += ncl) {
         const int nsteps = tile_steps(ti);
         const int arow = ti.row0 + 128 * (int)rank;
         for (int i = 0; i < nsteps; ++i, ++it) {
@@ -169,11 +177,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm2Threads, 1)
           const uint32_t fb = full_leader(s);
           if (kb < kb_main) {
             if (leader) mbar_arrive_expect_tx(full_bar(s), 2 * C::A_BYTES + C::SIG_BYTES);
-            tma_load_2d_pair(sA + s * C::A_BYTES, &tmA, fb, kb * kBK, arow);
+#pragma unroll
+            for (int h = 0; h < MS; ++h)
+              tma_load_2d_pair(sA + s * C::A_BYTES + h * 16384, &tmA, fb, kb * kBK, arow + 256 * h);
           } else {
             const int x = (kb - kb_main) * kBK;
             if (leader) mbar_arrive_expect_tx(full_bar(s), 2 * (C::A_BYTES + C::B_BYTES));
-            tma_load_2d_pair(sA + s * C::A_BYTES, &tmLA, fb, x, arow);
+#pragma unroll
+            for (int h = 0; h < MS; ++h)
+              tma_load_2d_pair(sA + s * C::A_BYTES + h * 16384, &tmLA, fb, x, arow + 256 * h);
             const int lb = ti.nb * BN + C::HN * (int)rank;
             tma_load_2d_pair(sB + s * C::B_BYTES, &tmLB, fb, x, lb);
             tma_load_2d_pair(sB + s * C::B_BYTES + 64 * 128, &tmLB, fb, x, lb + 64);
@@ -194,7 +206,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm2Threads, 1)
       for (int s = 0; s < C::RAW_SLOTS; ++s) last_phase[s] = -1;
       constexpr int GW = C::GB / 4;
       TileInfo ti;
-      for (int t = cid; ok && gemm2_tile(p, t, ti); t += ncl) {
+      for (int t = cid; ok && gemm2_tile<C::BM>(p, t, ti); t += ncl) {
         const int c_lo = TRANS ? ti.kb_lo : ti.kb_lo / 4;
         const int c_hi = TRANS ? ti.kb_hi : ti.kb_hi / 4;
         for (int c = c_lo; c < c_hi; ++c, ++rc) {
@@ -232,9 +244,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm2Threads, 1)
       const uint64_t adesc0 = smem_desc_sw128(sA, 16, 1024);
       const uint64_t bdesc0_k = smem_desc_sw128(sB, 16, 1024);
       const uint64_t bdesc0_mn = smem_desc_sw128(sB, 1024, 2048);
-      for (int t = cid; ok && gemm2_tile(p, t, ti); t += ncl, ++tc) {
-        const int buf = tc & 1;
-        if (!mbar_wait<true>(tempty_bar(buf), ((tc >> 1) & 1) ^ 1, 13)) { ok = false; break; }
+      for (int t = cid; ok && gemm2_tile<C::BM>(p, t, ti); t += ncl, ++tc) {
+        const int buf = tc % C::NBUF;
+        if (!mbar_wait<true>(tempty_bar(buf), ((tc / C::NBUF) & 1) ^ 1, 13)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * C::ACC_COLS;
         const int nq = ti.kb_hi - ti.kb_lo;
@@ -244,16 +256,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm2Threads, 1)
           tc_fence_after();
           const uint64_t ad = adesc0 + (uint64_t)(s * (C::A_BYTES >> 4));
           const bool kmaj = !TRANS || i >= nq;
+          // the MS A blocks of a stage are 16 KB (1024 descriptor units) apart and share the B half
           if (kmaj) {
             const uint64_t bd = bdesc0_k + (uint64_t)(s * (C::B_BYTES >> 4));
 #pragma unroll
             for (int k = 0; k < kBK / 16; ++k)
-              umma_bf16_pair(d_tmem, ad + 2 * k, bd + 2 * k, idesc_kmaj, (i | k) != 0);
+#pragma unroll
+              for (int h = 0; h < MS; ++h)
+                umma_bf16_pair(d_tmem + h * BN, ad + 1024 * h + 2 * k, bd + 2 * k, idesc_kmaj, (i | k) != 0);
           } else {
             const uint64_t bd = bdesc0_mn + (uint64_t)(s * (C::B_BYTES >> 4));
 #pragma unroll
             for (int k = 0; k < kBK / 16; ++k)
-              umma_bf16_pair(d_tmem, ad + 2 * k, bd + 256 * k, idesc_main, (i | k) != 0);
+#pragma unroll
+              for (int h = 0; h < MS; ++h)
+                umma_bf16_pair(d_tmem + h * BN, ad + 1024 * h + 2 * k, bd + 256 * k, idesc_main, (i | k) != 0);
           }
           umma_commit_pair_both(empty_bar(s));
           issued = true;
@@ -281,7 +298,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm2Threads, 1)
     int it = 0, rc = 0;
     bool ok = true;
     TileInfo ti;
-    for (int t = cid; ok && gemm2_tile(p, t, ti); t += ncl) {
+    for (int t = cid; ok && gemm2_tile<C::BM>(p, t, ti); t += ncl) {
       if (!TRANS) {
         for (int g = ti.kb_lo / 4; ok && g < ti.kb_hi / 4; ++g, ++rc) {
           const int rs = rc % C::RAW_SLOTS;
@@ -347,17 +364,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm2Threads, 1)
       }
     }
   } else if (warp < kNumEpiWarps) {
-    // ---------------- epilogue: this CTA's 128 rows x 256 columns ----------------
+    // ---------------- epilogue: this CTA's MS x 128 rows x 256 columns ----------------
     int tc = 0;
     TileInfo ti;
-    for (int t = cid; gemm2_tile(p, t, ti); t += ncl, ++tc) {
-      const int buf = tc & 1;
-      if (!warp_wait(tfull_bar(buf), (tc >> 1) & 1, 18)) break;
+    for (int t = cid; gemm2_tile<C::BM>(p, t, ti); t += ncl, ++tc) {
+      const int buf = tc % C::NBUF;
+      if (!warp_wait(tfull_bar(buf), (tc / C::NBUF) & 1, 18)) break;
       tc_fence_after();
-      const int row = ti.row0 + 128 * (int)rank + warp * 32 + lane;
-      const bool valid = row < ti.row_end;
-      const uint32_t tbase = tmem_base + ((uint32_t)(warp * 32) << 16) + buf * C::ACC_COLS;
-      epilogue_rows<EPI_STORE, BN>(p, ti, row, valid, tbase);
+#pragma unroll 1
+      for (int h = 0; h < MS; ++h) {
+        const int row = ti.row0 + 256 * h + 128 * (int)rank + warp * 32 + lane;
+        const bool valid = row < ti.row_end;
+        const uint32_t tbase = tmem_base + ((uint32_t)(warp * 32) << 16) + buf * C::ACC_COLS + h * BN;
+        epilogue_rows<EPI_STORE, BN>(p, ti, row, valid, tbase);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader(buf));

@@ -132,11 +132,11 @@ static int launch_qgemm_q(int qtype, const CUtensorMap& tA, const CUtensorMap& t
 // Pair-tile dense GEMM: clusters of two CTAs, one cluster per pair tile slot. The grid is capped at
 // the number of clusters that can be resident at once (a persistent kernel must never have CTAs
 // waiting for a free SM pair).
-template <int QT, bool TRANS>
+template <int QT, bool TRANS, int MS>
 static int launch_qgemm2(const CUtensorMap& tA, const CUtensorMap& tW, const CUtensorMap& tLA, const CUtensorMap& tLB,
                          const GemmParams& p, int tiles, cudaStream_t st, int slot) {
-  using C = Gemm2Cfg<QT, TRANS>;
-  auto k = qgemm2_kernel<QT, TRANS>;
+  using C = Gemm2Cfg<QT, TRANS, MS>;
+  auto k = qgemm2_kernel<QT, TRANS, MS>;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return QL_ERR_CUDA;
   static int max_clusters[16] = {};
@@ -167,13 +167,13 @@ static int launch_qgemm2(const CUtensorMap& tA, const CUtensorMap& tW, const CUt
   return launch_status();
 }
 
-template <bool TRANS>
+template <bool TRANS, int MS>
 static int launch_qgemm2_q(int qtype, const CUtensorMap& tA, const CUtensorMap& tW, const CUtensorMap& tLA,
                            const CUtensorMap& tLB, const GemmParams& p, int tiles, cudaStream_t st, int slot) {
   switch (qtype) {
-    case QL_Q8_0: return launch_qgemm2<QL_Q8_0, TRANS>(tA, tW, tLA, tLB, p, tiles, st, slot);
-    case QL_Q4_0: return launch_qgemm2<QL_Q4_0, TRANS>(tA, tW, tLA, tLB, p, tiles, st, slot);
-    case QL_Q4_K: return launch_qgemm2<QL_Q4_K, TRANS>(tA, tW, tLA, tLB, p, tiles, st, slot);
+    case QL_Q8_0: return launch_qgemm2<QL_Q8_0, TRANS, MS>(tA, tW, tLA, tLB, p, tiles, st, slot);
+    case QL_Q4_0: return launch_qgemm2<QL_Q4_0, TRANS, MS>(tA, tW, tLA, tLB, p, tiles, st, slot);
+    case QL_Q4_K: return launch_qgemm2<QL_Q4_K, TRANS, MS>(tA, tW, tLA, tLB, p, tiles, st, slot);
     default: return QL_ERR_UNSUPPORTED;
   }
 }
@@ -189,51 +189,35 @@ static void rows_split(int M, int Kin, int ks_cap, int* KS, int* kchunk) {
   *KS = (Kin + kc - 1) / kc;
 }
 
-// out = oscale * Y Z^T (fp32 [M x r]) and la = split(lscale * Y Z^T); dense Z(j, k) = Z[j*zj + k*zk].
-// Grouped use (row_exp != NULL, per-row expert) goes through the CUDA-core kernel.
-static int launch_lora_rows(const __nv_bfloat16* Y, long ldy, int M, int Kin, const __nv_bfloat16* Z, long zj, long zk,
-                            long zes, const int* row_exp, int r, float oscale, float lscale, float* out,
-                            __nv_bfloat16* la, float* part, cudaStream_t st, int ks_cap = 16) {
-  const int RP = lora_rp(r);
-  if (M <= 0) return QL_OK;
-  if (row_exp == nullptr) {
-    int KS, kchunk;
-    rows_split(M, Kin, ks_cap, &KS, &kchunk);
-    dim3 grid((M + 63) / 64, KS);
-    const int NT = r <= 16 ? 2 : (r <= 32 ? 4 : 8);
-    if (NT == 2) lora_rows_mma_kernel<2><<<grid, 128, 0, st>>>(Y, ldy, M, Kin, kchunk, Z, zj, zk, r, part);
-    else if (NT == 4) lora_rows_mma_kernel<4><<<grid, 128, 0, st>>>(Y, ldy, M, Kin, kchunk, Z, zj, zk, r, part);
-    else lora_rows_mma_kernel<8><<<grid, 128, 0, st>>>(Y, ldy, M, Kin, kchunk, Z, zj, zk, r, part);
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    if (launch_status() != QL_OK) return QL_ERR_CUDA;
-    const long total = (long)M * RP;
-    const int g2 = (int)std::min<long>((total + 255) / 256, 148L * 16);
-    lora_rows_reduce_kernel<<<g2, 256, 0, st>>>(part, KS, M, 8 * NT, r, oscale, lscale, out, la, RP);
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    return launch_status();
-  }
-  const int grid = (M + 7) / 8;
-  if (r <= 16)
-    lora_rows_kernel<16><<<grid, 256, 0, st>>>(Y, ldy, M, Kin, Z, zj, zk, zes, row_exp, r, oscale, lscale, out, la, RP);
-  else if (r <= 32)
-    lora_rows_kernel<32><<<grid, 256, 0, st>>>(Y, ldy, M, Kin, Z, zj, zk, zes, row_exp, r, oscale, lscale, out, la, RP);
-  else
-    lora_rows_kernel<64><<<grid, 256, 0, st>>>(Y, ldy, M, Kin, Z, zj, zk, zes, row_exp, r, oscale, lscale, out, la, RP);
-  g_launches.fetch_add(1, std::memory_order_relaxed);
-  return launch_status();
+// Dense row reduction with the in-cluster split-K sum: out = oscale * Y Z^T, la = split(lscale *
+// Y Z^T), optionally hs = split(hscale * hin) for the same rows, and, in the same launch,
+// LB = [Zb | Zb] (bop).
+template <int NT>
+static cudaError_t launch_rows_nt(cudaLaunchConfig_t& cfg, const __nv_bfloat16* Y, long ldy, int M, int Kin,
+                                  int kchunk, const __nv_bfloat16* Z, long zj, long zk, int r, float oscale,
+                                  float lscale, float* out, __nv_bfloat16* la, int RP, BopArgs bop, __nv_bfloat16* LB,
+                                  int row_blocks, const float* hin, float hscale, __nv_bfloat16* hs) {
+  auto k = lora_rows_cluster_kernel<NT>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cfg.dynamicSmemBytes);
+  if (e != cudaSuccess) return e;
+  return cudaLaunchKernelEx(&cfg, k, Y, ldy, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out, la, RP, bop, LB,
+                            row_blocks, hin, hscale, hs);
 }
 
-// Dense row reduction with the in-cluster split-K sum: out = oscale * Y Z^T, la = split(lscale *
-// Y Z^T) and, in the same launch, LB = [Zb | Zb] (bop).
 static int launch_rows_dense(const __nv_bfloat16* Y, long ldy, int M, int Kin, const __nv_bfloat16* Z, long zj,
                              long zk, int r, float oscale, float lscale, float* out, __nv_bfloat16* la, BopArgs bop,
-                             __nv_bfloat16* LB, cudaStream_t st) {
+                             __nv_bfloat16* LB, cudaStream_t st, const float* hin = nullptr, float hscale = 0.f,
+                             __nv_bfloat16* hs = nullptr) {
   if (M <= 0) return QL_OK;
   const int RP = lora_rp(r);
-  int KS = std::max(1, std::min(8, Kin / 32));
+  // k range per cluster rank: a multiple of the 128-wide streamed tile
+  int KS = std::max(1, std::min(8, (Kin + 127) / 128));
   int kchunk = (Kin + KS - 1) / KS;
-  kchunk = (kchunk + 31) / 32 * 32;
+  kchunk = (kchunk + 127) / 128 * 128;
   KS = (Kin + kchunk - 1) / kchunk;
+  const int NT = r <= 16 ? 2 : (r <= 32 ? 4 : 8);
+  const size_t smem = rows_smem_bytes(NT, kchunk);
+  if (smem > 232448) return QL_ERR_SHAPE;  // the staged adapter slice does not fit on chip
   // extra clusters for the LB operand when it outweighs the row work (small M)
   const int row_blocks = (M + 63) / 64;
   const long bop_items = bop.Z ? (long)bop.rows * (2 * RP / 8) : 0;
@@ -242,7 +226,7 @@ static int launch_rows_dense(const __nv_bfloat16* Y, long ldy, int M, int Kin, c
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(row_blocks + bop_blocks, KS, 1);
   cfg.blockDim = dim3(128, 1, 1);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -252,15 +236,15 @@ static int launch_rows_dense(const __nv_bfloat16* Y, long ldy, int M, int Kin, c
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e;
-  if (r <= 16)
-    e = cudaLaunchKernelEx(&cfg, lora_rows_cluster_kernel<2>, Y, ldy, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out,
-                           la, RP, bop, LB, row_blocks);
-  else if (r <= 32)
-    e = cudaLaunchKernelEx(&cfg, lora_rows_cluster_kernel<4>, Y, ldy, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out,
-                           la, RP, bop, LB, row_blocks);
+  if (NT == 2)
+    e = launch_rows_nt<2>(cfg, Y, ldy, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out, la, RP, bop, LB, row_blocks,
+                          hin, hscale, hs);
+  else if (NT == 4)
+    e = launch_rows_nt<4>(cfg, Y, ldy, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out, la, RP, bop, LB, row_blocks,
+                          hin, hscale, hs);
   else
-    e = cudaLaunchKernelEx(&cfg, lora_rows_cluster_kernel<8>, Y, ldy, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out,
-                           la, RP, bop, LB, row_blocks);
+    e = launch_rows_nt<8>(cfg, Y, ldy, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out, la, RP, bop, LB, row_blocks,
+                          hin, hscale, hs);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -270,7 +254,17 @@ static int launch_rows_dense(const __nv_bfloat16* Y, long ldy, int M, int Kin, c
 }
 
 // Two dense column reductions in one launch (dB and dA of the backward).
+template <int JT>
+static cudaError_t launch_colred_jt(cudaLaunchConfig_t& cfg, const ColredProblem& p0, const ColredProblem& p1, int nb0,
+                                    int M, int r, int RP, int mchunk) {
+  auto k = colred_cluster_kernel<JT>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cfg.dynamicSmemBytes);
+  if (e != cudaSuccess) return e;
+  return cudaLaunchKernelEx(&cfg, k, p0, p1, nb0, M, r, RP, mchunk);
+}
+
 static int launch_colred_dense(const ColredProblem& p0, const ColredProblem& p1, int M, int r, cudaStream_t st) {
+  const int RP = lora_rp(r);
   int CS = std::max(1, std::min(8, (M + 63) / 64));
   int mchunk = (M + CS - 1) / CS;
   mchunk = (mchunk + 63) / 64 * 64;
@@ -279,7 +273,7 @@ static int launch_colred_dense(const ColredProblem& p0, const ColredProblem& p1,
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nb0 + nb1, CS, 1);
   cfg.blockDim = dim3(128, 1, 1);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = colred_smem_bytes(RP);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -290,25 +284,15 @@ static int launch_colred_dense(const ColredProblem& p0, const ColredProblem& p1,
   cfg.numAttrs = 1;
   const int JT = (r + 15) / 16;
   cudaError_t e;
-  if (JT == 1) e = cudaLaunchKernelEx(&cfg, colred_cluster_kernel<1>, p0, p1, nb0, M, r, mchunk);
-  else if (JT == 2) e = cudaLaunchKernelEx(&cfg, colred_cluster_kernel<2>, p0, p1, nb0, M, r, mchunk);
-  else if (JT == 3) e = cudaLaunchKernelEx(&cfg, colred_cluster_kernel<3>, p0, p1, nb0, M, r, mchunk);
-  else e = cudaLaunchKernelEx(&cfg, colred_cluster_kernel<4>, p0, p1, nb0, M, r, mchunk);
+  if (JT == 1) e = launch_colred_jt<1>(cfg, p0, p1, nb0, M, r, RP, mchunk);
+  else if (JT == 2) e = launch_colred_jt<2>(cfg, p0, p1, nb0, M, r, RP, mchunk);
+  else if (JT == 3) e = launch_colred_jt<3>(cfg, p0, p1, nb0, M, r, RP, mchunk);
+  else e = launch_colred_jt<4>(cfg, p0, p1, nb0, M, r, RP, mchunk);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return QL_ERR_CUDA;
   }
-  return launch_status();
-}
-
-static int launch_lora_bop(const __nv_bfloat16* Z, long zn, long zjs, long zes, int rows, int nexp, int r,
-                           __nv_bfloat16* LB, cudaStream_t st) {
-  const int RP = lora_rp(r);
-  const long total = (long)nexp * rows * 2 * RP;
-  const int grid = (int)std::min<long>((total + 255) / 256, 148L * 16);
-  lora_bop_kernel<<<grid, 256, 0, st>>>(Z, zn, zjs, zes, rows, nexp, r, RP, LB);
-  g_launches.fetch_add(1, std::memory_order_relaxed);
   return launch_status();
 }
 
@@ -332,18 +316,19 @@ static int launch_colred(const __nv_bfloat16* Y, long ldy, int Ccols, const floa
   return launch_status();
 }
 
-// Tile plan of a dense GEMM. With more than 128 rows the tiles are pair tiles of 256 x 256 computed
-// by two CTAs (pair = true); otherwise 128 x 128 tiles on one CTA. K is split into ksplit parts of
+// Tile plan of a dense GEMM. More than 256 rows: 512 x 256 pair tiles (two CTAs, two 128-row A
+// blocks each, ms = 2); 129 to 256 rows: 256 x 256 pair tiles (ms = 1); otherwise 128 x 128 tiles on
+// one CTA (ms = 0). In that last, small-M, weight-streaming regime K is split into ksplit parts of
 // kb_per_split k-blocks (a multiple of 4 in forward mode) when the output has fewer tiles than there
-// are tile slots (SMs, or SM pairs): the small-M, weight-streaming regime.
+// are SMs.
 struct DensePlan {
-  bool pair;
+  int ms;
   int ksplit, kbs, mblocks, ntiles;
 };
 static DensePlan plan_dense(int64_t M, int64_t Nd, int64_t Kd, bool trans, bool allow_split) {
   DensePlan d;
-  d.pair = M > 128;
-  const int tm = d.pair ? 256 : 128, tn = d.pair ? 256 : 128;
+  d.ms = M > 256 ? 2 : (M > 128 ? 1 : 0);
+  const int tm = d.ms ? 256 * d.ms : 128, tn = d.ms ? 256 : 128;
   d.mblocks = (int)((M + tm - 1) / tm);
   d.ntiles = (int)((Nd + tn - 1) / tn);
   const int kb_main = (int)(Kd / 64);
@@ -351,8 +336,8 @@ static DensePlan plan_dense(int64_t M, int64_t Nd, int64_t Kd, bool trans, bool 
   d.ksplit = 1;
   d.kbs = kb_main;
   const int tiles = d.mblocks * d.ntiles;
-  const int slots = d.pair ? num_sms() / 2 : num_sms();
-  if (allow_split && tiles < slots) {
+  const int slots = num_sms();
+  if (allow_split && d.ms == 0 && tiles < slots) {
     int ks = std::min((4 * slots + tiles - 1) / tiles, std::min(kb_main / unit, 32));
     if (ks > 1) {
       int kbs = (kb_main + ks - 1) / ks;
@@ -411,16 +396,17 @@ static int launch_dense_gemm(int qtype, const void* A, int64_t M, int64_t Kd, co
     p.out_dtype = out_dtype;
   }
   const int tiles = d.mblocks * d.ntiles * d.ksplit;
-  int rc = d.pair ? launch_qgemm2_q<TRANS>(qtype, tA, tW, tLA, tLB, p, tiles, st, slot)
-                  : launch_qgemm_q<TRANS, EPI_STORE, 1>(qtype, tA, tW, tLA, tLB, p, std::min(tiles, num_sms()), st,
-                                                        slot);
+  int rc;
+  if (d.ms == 2) rc = launch_qgemm2_q<TRANS, 2>(qtype, tA, tW, tLA, tLB, p, tiles, st, slot);
+  else if (d.ms == 1) rc = launch_qgemm2_q<TRANS, 1>(qtype, tA, tW, tLA, tLB, p, tiles, st, slot);
+  else rc = launch_qgemm_q<TRANS, EPI_STORE, 1>(qtype, tA, tW, tLA, tLB, p, std::min(tiles, num_sms()), st, slot);
   if (rc || d.ksplit == 1) return rc;
   return launch_split_reduce(split_buf, d.ksplit, (long)M * Nd, (long)M * Nd, out, out_dtype, st);
 }
 
 // Workspace layout of the dense layer (byte offsets, 256-aligned).
 struct LinearWs {
-  size_t la, lb, g, split, total;
+  size_t la, lb, hs, split, total;
 };
 static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 static LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int r) {
@@ -430,7 +416,7 @@ static LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int r) {
   size_t o = 0;
   w.la = o; o = al256(o + (size_t)M * KL * 2);
   w.lb = o; o = al256(o + (size_t)NK * KL * 2);
-  w.g = o; o = al256(o + (size_t)M * r * 4);
+  w.hs = o; o = al256(o + (size_t)M * KL * 2);
   const size_t sf = split_bytes(plan_dense(M, N, K, false, true), M, N);
   const size_t sb = split_bytes(plan_dense(M, K, N, true, true), M, K);
   w.split = o; o = al256(o + std::max(sf, sb));
@@ -894,21 +880,23 @@ int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void
   uint8_t* wsb = (uint8_t*)ws;
   __nv_bfloat16* LA = (__nv_bfloat16*)(wsb + w.la);
   __nv_bfloat16* LB = (__nv_bfloat16*)(wsb + w.lb);
-  float* G = (float*)(wsb + w.g);
   const int KL = 2 * lora_rp(r);
 
-  // G = s dY B (kept in fp32), its split operand, and LB[k] = [A^T(k) | A^T(k)]
-  rc = launch_rows_dense((const __nv_bfloat16*)dY, N, (int)M, (int)N, (const __nv_bfloat16*)B, 1, r, r, scale, scale, G,
-                         LA, dX ? BopArgs{(const __nv_bfloat16*)A, 1, K, (int)K} : BopArgs{nullptr, 0, 0, 0}, LB, st);
+  __nv_bfloat16* HS = (__nv_bfloat16*)(wsb + w.hs);
+  // LA = split(G) with G = s dY B, HS = split(s H), and LB[k] = [A^T(k) | A^T(k)]
+  rc = launch_rows_dense((const __nv_bfloat16*)dY, N, (int)M, (int)N, (const __nv_bfloat16*)B, 1, r, r, scale, scale,
+                         nullptr,
+                         LA, dX ? BopArgs{(const __nv_bfloat16*)A, 1, K, (int)K} : BopArgs{nullptr, 0, 0, 0}, LB, st, H,
+                         scale, HS);
   if (rc) return rc;
   if (dX) {
     rc = launch_dense_gemm<true>(qtype, dY, M, N, wq, N, K, LA, LB, KL, K, dX, dx_dtype,
                                  (float*)(wsb + w.split), true, st, 1);
     if (rc) return rc;
   }
-  // dB = s dY^T H and dA = G^T X in one launch
-  const ColredProblem pb{(const __nv_bfloat16*)dY, N, (int)N, H, scale, 0, dB};
-  const ColredProblem pa{(const __nv_bfloat16*)X, K, (int)K, G, 1.0f, 1, dA};
+  // dB = dY^T split(s H) and dA = split(G)^T X in one launch
+  const ColredProblem pb{(const __nv_bfloat16*)dY, N, (int)N, HS, 1.0f, 0, dB};
+  const ColredProblem pa{(const __nv_bfloat16*)X, K, (int)K, LA, 1.0f, 1, dA};
   return launch_colred_dense(pb, pa, (int)M, r, st);
 }
 
