@@ -324,36 +324,63 @@ __global__ void __launch_bounds__(128) lora_rows_cluster_kernel(
                  v);
     }
   };
-  // the ring's first tiles are in flight while the LB share is written and Z is staged
+  // Z(j, k) contiguous in k: staged by cp.async in its own group, ahead of the ring's first tiles
+  if (zk == 1) {
+    const uint32_t zdst = smem_u32(zs);
+    for (int i = tid; i < RN * (kchunk / 8); i += 128) {
+      const int j = i / (kchunk / 8), q = i % (kchunk / 8);
+      const bool v = j < r && 8 * q < nk;
+      cp_async16(zdst + (uint32_t)(j * ZS + 8 * q) * 2, v ? (const void*)(Z + (long)j * zj + kb + 8 * q) : (const void*)Z,
+                 v);
+    }
+  }
+  cp_async_commit();
 #pragma unroll
   for (int t = 0; t < S - 1; ++t) {
     if (t < ntiles) issue(t);
     cp_async_commit();
   }
-  lora_bop_share(bop, r, RP, LB);
-  if (zk == 1) {
-    for (int i = tid; i < RN * (kchunk / 8); i += 128) {
-      const int j = i / (kchunk / 8), q = i % (kchunk / 8);
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (j < r && 8 * q < nk) v = __ldg(reinterpret_cast<const uint4*>(Z + (long)j * zj + kb + 8 * q));
-      *reinterpret_cast<uint4*>(zs + j * ZS + 8 * q) = v;
-    }
-  } else {
-    // strided Z: eight independent loads in flight per thread; consecutive threads read
-    // consecutive j of one k
-    const int total = kchunk * RN;
-    for (int i0 = tid; i0 < total; i0 += 128 * 8) {
-      __nv_bfloat16 v[8];
+  if (zk != 1) {
+    // Z(j, k) = Z[j*zj + k*zk] with unit zj (the transposed adapter): the r values of one k are
+    // contiguous; all of a thread's loads are issued before its first shared store
+    const bool vec = zj == 1 && (r & 7) == 0 && (zk & 7) == 0;
+    if (vec) {
+      const int cpr = r / 8;  // 16-byte chunks per k
+      const int total = kchunk * cpr;
+      for (int i0 = tid; i0 < total; i0 += 128 * 8) {
+        uint4 v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = i0 + 128 * u;
-        const int kk = i / RN, j = i % RN;
-        v[u] = (i < total && j < r && kk < nk) ? Z[(long)j * zj + (long)(kb + kk) * zk] : __float2bfloat16(0.f);
+        for (int u = 0; u < 8; ++u) {
+          const int i = i0 + 128 * u, kk = i / cpr, q = i % cpr;
+          v[u] = (i < total && kk < nk) ? __ldg(reinterpret_cast<const uint4*>(Z + (long)(kb + kk) * zk + 8 * q))
+                                        : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = i0 + 128 * u, kk = i / cpr, q = i % cpr;
+          if (i < total) {
+            const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&v[u]);
+#pragma unroll
+            for (int w = 0; w < 8; ++w) zs[(8 * q + w) * ZS + kk] = e[w];
+          }
+        }
       }
+      for (int i = tid; i < (RN - r) * kchunk; i += 128) zs[(r + i / kchunk) * ZS + i % kchunk] = __float2bfloat16(0.f);
+    } else {
+      const int total = kchunk * RN;
+      for (int i0 = tid; i0 < total; i0 += 128 * 16) {
+        __nv_bfloat16 v[16];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = i0 + 128 * u;
-        if (i < total) zs[(i % RN) * ZS + i / RN] = v[u];
+        for (int u = 0; u < 16; ++u) {
+          const int i = i0 + 128 * u;
+          const int kk = i / RN, j = i % RN;
+          v[u] = (i < total && j < r && kk < nk) ? Z[(long)j * zj + (long)(kb + kk) * zk] : __float2bfloat16(0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int i = i0 + 128 * u;
+          if (i < total) zs[(i % RN) * ZS + i / RN] = v[u];
+        }
       }
     }
   }
@@ -398,6 +425,7 @@ __global__ void __launch_bounds__(128) lora_rows_cluster_kernel(
       part[(lr + 8) * RN + j + 1] = acc[t][3];
     }
   }
+  lora_bop_share(bop, r, RP, LB);  // off the main loop's path: overlaps the wait for the cluster
   cluster_sync_all();
   // rank q reduces rows [q*64/KS, (q+1)*64/KS) of the cluster's 64 rows, over ranks in order
   const int rows_per = (64 + KS - 1) / KS;

@@ -265,11 +265,13 @@ static cudaError_t launch_colred_jt(cudaLaunchConfig_t& cfg, const ColredProblem
 
 static int launch_colred_dense(const ColredProblem& p0, const ColredProblem& p1, int M, int r, cudaStream_t st) {
   const int RP = lora_rp(r);
-  int CS = std::max(1, std::min(8, (M + 63) / 64));
+  const int nb0 = (p0.C + 127) / 128, nb1 = (p1.C + 127) / 128;
+  // row slices per column block: as many as keep every CTA resident in one wave (two per SM)
+  const int CS_max = std::max(1, std::min(8, 2 * num_sms() / (nb0 + nb1)));
+  int CS = std::max(1, std::min(CS_max, (M + 63) / 64));
   int mchunk = (M + CS - 1) / CS;
   mchunk = (mchunk + 63) / 64 * 64;
   CS = (M + mchunk - 1) / mchunk;
-  const int nb0 = (p0.C + 127) / 128, nb1 = (p1.C + 127) / 128;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nb0 + nb1, CS, 1);
   cfg.blockDim = dim3(128, 1, 1);
