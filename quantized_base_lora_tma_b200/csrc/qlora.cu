@@ -12,6 +12,7 @@
 #include "lora.cuh"
 #include "qgemm.cuh"
 #include "qgemm2.cuh"
+#include "gemv.cuh"
 #include "moe.cuh"
 
 namespace qlora {
@@ -406,6 +407,74 @@ static int launch_dense_gemm(int qtype, const void* A, int64_t M, int64_t Kd, co
   return launch_split_reduce(split_buf, d.ksplit, (long)M * Nd, (long)M * Nd, out, out_dtype, st);
 }
 
+// Small-M forward (M <= 16, Q4_0 / Q8_0, r <= 16): one launch of the weight-streaming kernel; the
+// KS CTAs of a cluster split K so that about two CTAs per SM are resident.
+template <int QT, int MT>
+static int launch_gemv_q(const CUtensorMap& tW, const CUtensorMap& tX, const GvParams& p, int KS, cudaStream_t st,
+                         int slot) {
+  using C = GvCfg<QT, MT>;
+  auto k = qgemv_fwd_kernel<QT, MT>;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+    return QL_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.N / kGvRows, KS, 1);
+  cfg.blockDim = dim3(kGvThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = KS;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  ev_record(slot, 0, st);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k, tW, tX, p);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  ev_record(slot, 1, st);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  return launch_status();
+}
+
+static bool gemv_fwd_applies(int qtype, int64_t M, int r) {
+  return M <= 16 && r <= kGvMaxRank && (qtype == QL_Q4_0 || qtype == QL_Q8_0);
+}
+
+static int launch_gemv_fwd(int qtype, const void* wq, int64_t N, int64_t K, const void* X, int64_t M, const void* A,
+                           const void* B, int r, float scale, void* Y, int y_dtype, float* H, cudaStream_t st,
+                           int slot) {
+  const int MT = M <= 8 ? 1 : 2;
+  CUtensorMap tW, tX;
+  if (!tmap_packed(&tW, wq, packed_row_bytes(qtype, K), N, group_bytes(qtype)) ||
+      !tmap_bf16_rows(&tX, X, K, M, 8u * MT))
+    return QL_ERR_CUDA;
+  const int row_blocks = (int)(N / kGvRows);
+  const int groups = (int)(K / 256);
+  int KS = std::max(1, std::min(std::min(8, groups), 2 * num_sms() / row_blocks));  // one resident wave
+  const int kgroups = (groups + KS - 1) / KS;
+  KS = (groups + kgroups - 1) / kgroups;
+  GvParams p;
+  p.N = (int)N;
+  p.K = (int)K;
+  p.M = (int)M;
+  p.r = r;
+  p.kgroups = kgroups;
+  p.scale = scale;
+  p.A = (const __nv_bfloat16*)A;
+  p.B = (const __nv_bfloat16*)B;
+  p.Y = Y;
+  p.y_dtype = y_dtype;
+  p.H = H;
+  if (qtype == QL_Q4_0)
+    return MT == 1 ? launch_gemv_q<QL_Q4_0, 1>(tW, tX, p, KS, st, slot)
+                   : launch_gemv_q<QL_Q4_0, 2>(tW, tX, p, KS, st, slot);
+  return MT == 1 ? launch_gemv_q<QL_Q8_0, 1>(tW, tX, p, KS, st, slot)
+                 : launch_gemv_q<QL_Q8_0, 2>(tW, tX, p, KS, st, slot);
+}
+
 // Workspace layout of the dense layer (byte offsets, 256-aligned).
 struct LinearWs {
   size_t la, lb, hs, split, total;
@@ -628,6 +697,8 @@ int qlora_linear_fwd(int qtype, const void* wq, int64_t N, int64_t K, const void
   if (!ws || ws_bytes < w.total) return QL_ERR_WORKSPACE;
   if (!aligned16(ws)) return QL_ERR_ALIGNMENT;
   cudaStream_t st = (cudaStream_t)stream;
+  if (gemv_fwd_applies(qtype, M, r))
+    return launch_gemv_fwd(qtype, wq, N, K, X, M, A, B, r, scale, Y, y_dtype, H, st, 0);
   uint8_t* wsb = (uint8_t*)ws;
   __nv_bfloat16* LA = (__nv_bfloat16*)(wsb + w.la);
   __nv_bfloat16* LB = (__nv_bfloat16*)(wsb + w.lb);

@@ -93,6 +93,8 @@ SMALL = [
     (3, 1024, 1024, 4),
     (1100, 512, 4096, 8),  # more pair tiles than SM pairs: forward without a K split
     (1100, 4096, 512, 8),  # the same for the input-gradient GEMM
+    (9, 1280, 192, 16),    # decode path: two token tiles, two adapter tiles, K steps not a multiple of the split
+    (13, 768, 64, 12),     # decode path: one row block, ragged rank
 ]
 
 
