@@ -44,7 +44,7 @@ struct GvCfg {
   static constexpr int X_BOX = XR * 128;              // one 64-wide k box
   static constexpr int X_BYTES = 4 * X_BOX;
   static constexpr int STAGE = W_BYTES + X_BYTES;
-  static constexpr int STAGES = GB > 200 ? 3 : 4;  // two CTAs per SM
+  static constexpr int STAGES = 3;
   static constexpr int OFF_PART = STAGES * STAGE;                 // [2][64][16] fp32 partial outputs
   static constexpr int OFF_HP = OFF_PART + 2 * kGvRows * 16 * 4;  // [9][16][16] fp32: 8 warps' H, their sum
   static constexpr int OFF_HF = OFF_HP + 9 * 16 * 16 * 4;         // [16][16] fp32 summed H

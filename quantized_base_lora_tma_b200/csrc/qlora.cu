@@ -453,7 +453,11 @@ static int launch_gemv_fwd(int qtype, const void* wq, int64_t N, int64_t K, cons
     return QL_ERR_CUDA;
   const int row_blocks = (int)(N / kGvRows);
   const int groups = (int)(K / 256);
-  int KS = std::max(1, std::min(std::min(8, groups), 2 * num_sms() / row_blocks));  // one resident wave
+  // K split: as many slices as keep every CTA resident in one wave
+  const size_t smem = qtype == QL_Q4_0 ? (MT == 1 ? GvCfg<QL_Q4_0, 1>::SMEM_BYTES : GvCfg<QL_Q4_0, 2>::SMEM_BYTES)
+                                       : (MT == 1 ? GvCfg<QL_Q8_0, 1>::SMEM_BYTES : GvCfg<QL_Q8_0, 2>::SMEM_BYTES);
+  const int per_sm = std::max(1, (int)(233472 / (smem + 1024)));
+  int KS = std::max(1, std::min(std::min(8, groups), per_sm * num_sms() / row_blocks));
   const int kgroups = (groups + KS - 1) / KS;
   KS = (groups + kgroups - 1) / kgroups;
   GvParams p;
