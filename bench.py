@@ -350,11 +350,18 @@ def run_ours(args, rank, world, local_rank):
     launches0 = ql.qlora_launch_count()
     sampler = ClockSampler(local_rank)
     wall0 = time.perf_counter()
+    # The GEMM events are recorded on every fourth step only: an event between two kernels of the
+    # step stops the next kernel from starting while the previous one drains (programmatic launch),
+    # so those steps are slower; they stay in the step mean, which is therefore slightly pessimistic.
+    ev_steps = list(range(0, K, 4))
     with sampler:
         for i in range(K):
             flush.zero_()
             for s in (0, 1):
-                ql.qlora_set_kernel_events(s, gev[s][i][0], gev[s][i][1])
+                if i % 4 == 0:
+                    ql.qlora_set_kernel_events(s, gev[s][i // 4][0], gev[s][i // 4][1])
+                else:
+                    ql.qlora_set_kernel_events(s, None, None)
             ev[i][0].record(stream)
             run.step()
             allreduce_grads()
@@ -371,7 +378,7 @@ def run_ours(args, rank, world, local_rank):
     if st != 0:
         raise RuntimeError(f"device status {st} at site {site}")
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    gemm_ms = {s: [a.elapsed_time(b) for a, b in gev[s]] for s in (0, 1)}
+    gemm_ms = {s: [gev[s][j][0].elapsed_time(gev[s][j][1]) for j in range(len(ev_steps))] for s in (0, 1)}
     ms = statistics.mean(step_ms)
     if world > 1:
         t = torch.tensor([ms], device="cuda")
@@ -415,8 +422,8 @@ def run_ours(args, rank, world, local_rank):
     # dominant kernel: the tensor-core GEMM with the larger share of the step
     g_mean = {s: statistics.mean(gemm_ms[s]) for s in (0, 1)}
     dom = max(g_mean, key=g_mean.get)
-    dom_name = {0: "qgemm_fwd (dequant-in-SMEM tcgen05 GEMM, K-major)",
-                1: "qgemm_dx (dequant-in-SMEM tcgen05 GEMM, MN-major)"}[dom]
+    dom_name = {0: "qgemm_fwd (dequant-in-SMEM tcgen05 cta_group::2 GEMM, 512x256 pair tiles, K-major B)",
+                1: "qgemm_dx (dequant-in-SMEM tcgen05 cta_group::2 GEMM, 512x256 pair tiles, MN-major B)"}[dom]
     achieved = run.gemm_flops(dom) / (g_mean[dom] / 1e3) / 1e12
     step_tflops = run.flops() / (ms / 1e3) / 1e12
     traffic = profiled_traffic(args.workload, "qgemm_fwd" if dom == 0 else "qgemm_dx")

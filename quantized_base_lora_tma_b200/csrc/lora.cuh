@@ -295,6 +295,8 @@ __global__ void __launch_bounds__(128) lora_rows_cluster_kernel(
   constexpr int RN = 8 * NT;
   constexpr int S = kRowsStages, TK = kRowsTileK, YS = kRowsYS;
   extern __shared__ __align__(16) uint8_t rows_smem[];
+  pdl_launch_dependents();
+  pdl_wait();
   if ((int)blockIdx.x >= row_blocks) {
     lora_bop_share(bop, r, RP, LB);
     return;
@@ -487,6 +489,8 @@ __global__ void __launch_bounds__(128) colred_cluster_kernel(ColredProblem p0, C
                                                              int r, int RP, int mchunk) {
   constexpr int S = kColStages, YS = kColYS;
   extern __shared__ __align__(16) uint8_t col_smem[];
+  pdl_launch_dependents();
+  pdl_wait();
   const int ZW = 2 * RP + 8;  // padded row of a 64 x 2RP split-Z tile
   __nv_bfloat16* yring = reinterpret_cast<__nv_bfloat16*>(col_smem);
   __nv_bfloat16* zring = yring + S * 64 * YS;
@@ -752,6 +756,8 @@ __global__ void colred_reduce_kernel(const float* __restrict__ part, int Ccols, 
 // Ordered sum of the split-K partials of a dense GEMM: out[m][n] = sum_ks part[ks][m][n].
 __global__ void split_reduce_kernel(const float* __restrict__ part, int ksplit, long stride, long count,
                                     void* __restrict__ out, int out_dtype) {
+  pdl_launch_dependents();
+  pdl_wait();
   for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; 4 * i < count; i += (long)gridDim.x * blockDim.x) {
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int ks = 0; ks < ksplit; ++ks) {

@@ -119,6 +119,14 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int sit
 }
 
 // ------------------------------------------------------------------------------------------------
+// Programmatic dependent launch. Kernels of the dense path let the next kernel in the stream start
+// its set-up early (launch_dependents) and wait for the previous kernel's completion and memory
+// (wait) before their first global-memory access; both are no-ops without a programmatic launch.
+// ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// ------------------------------------------------------------------------------------------------
 // CTA pairs (clusters of two)
 // ------------------------------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t cta_rank_in_cluster() {

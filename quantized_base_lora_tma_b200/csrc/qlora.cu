@@ -105,6 +105,40 @@ static inline int launch_status() {
 // ------------------------------------------------------------------------------------------------
 // Launch helpers
 // ------------------------------------------------------------------------------------------------
+// Launch configuration with programmatic stream serialization (the kernel may start while the
+// previous kernel in the stream finishes; the dense-path kernels wait on it in-kernel) and, when
+// cluster_y > 0, a (1, cluster_y, 1) cluster shape.
+struct PdlLaunch {
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[2];
+  PdlLaunch(dim3 grid, dim3 block, size_t smem, cudaStream_t st, int cluster_y = 0) {
+    cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    int n = 1;
+    if (cluster_y > 0) {
+      attr[1].id = cudaLaunchAttributeClusterDimension;
+      attr[1].val.clusterDim.x = 1;
+      attr[1].val.clusterDim.y = (unsigned)cluster_y;
+      attr[1].val.clusterDim.z = 1;
+      n = 2;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+  }
+};
+static int launch_result(cudaError_t e) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  return launch_status();
+}
 template <int QT, bool TRANS, int EPI, int MS>
 static int launch_qgemm(const CUtensorMap& tA, const CUtensorMap& tW, const CUtensorMap& tLA, const CUtensorMap& tLB,
                         const GemmParams& p, int grid, cudaStream_t st, int slot) {
@@ -112,11 +146,11 @@ static int launch_qgemm(const CUtensorMap& tA, const CUtensorMap& tW, const CUte
   auto k = qgemm_kernel<QT, TRANS, EPI, MS>;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return QL_ERR_CUDA;
+  PdlLaunch L(dim3(grid), dim3(kGemmThreads), C::SMEM_BYTES, st);
   ev_record(slot, 0, st);
-  k<<<grid, kGemmThreads, C::SMEM_BYTES, st>>>(tA, tW, tLA, tLB, p);
-  g_launches.fetch_add(1, std::memory_order_relaxed);
+  const cudaError_t e = cudaLaunchKernelEx(&L.cfg, k, tA, tW, tLA, tLB, p);
   ev_record(slot, 1, st);
-  return launch_status();
+  return launch_result(e);
 }
 
 template <bool TRANS, int EPI, int MS>
@@ -161,11 +195,11 @@ static int launch_qgemm2(const CUtensorMap& tA, const CUtensorMap& tW, const CUt
     mc = n;
   }
   const int clusters = std::min(tiles, mc);
+  PdlLaunch L(dim3(2 * clusters), dim3(kGemm2Threads), C::SMEM_BYTES, st);  // cluster shape from the kernel
   ev_record(slot, 0, st);
-  k<<<2 * clusters, kGemm2Threads, C::SMEM_BYTES, st>>>(tA, tW, tLA, tLB, p);
-  g_launches.fetch_add(1, std::memory_order_relaxed);
+  const cudaError_t e = cudaLaunchKernelEx(&L.cfg, k, tA, tW, tLA, tLB, p);
   ev_record(slot, 1, st);
-  return launch_status();
+  return launch_result(e);
 }
 
 template <bool TRANS, int MS>
@@ -224,18 +258,8 @@ static int launch_rows_dense(const __nv_bfloat16* Y, long ldy, int M, int Kin, c
   const long bop_items = bop.Z ? (long)bop.rows * (2 * RP / 8) : 0;
   const long per_cluster = (long)KS * 128 * 4;
   const int bop_blocks = (int)std::max<long>(0, (bop_items + per_cluster - 1) / per_cluster - row_blocks);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(row_blocks + bop_blocks, KS, 1);
-  cfg.blockDim = dim3(128, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = KS;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  PdlLaunch L(dim3(row_blocks + bop_blocks, KS, 1), dim3(128), smem, st, KS);
+  cudaLaunchConfig_t& cfg = L.cfg;
   cudaError_t e;
   if (NT == 2)
     e = launch_rows_nt<2>(cfg, Y, ldy, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out, la, RP, bop, LB, row_blocks,
@@ -273,18 +297,8 @@ static int launch_colred_dense(const ColredProblem& p0, const ColredProblem& p1,
   int mchunk = (M + CS - 1) / CS;
   mchunk = (mchunk + 63) / 64 * 64;
   CS = (M + mchunk - 1) / mchunk;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(nb0 + nb1, CS, 1);
-  cfg.blockDim = dim3(128, 1, 1);
-  cfg.dynamicSmemBytes = colred_smem_bytes(RP);
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = CS;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  PdlLaunch L(dim3(nb0 + nb1, CS, 1), dim3(128), colred_smem_bytes(RP), st, CS);
+  cudaLaunchConfig_t& cfg = L.cfg;
   const int JT = (r + 15) / 16;
   cudaError_t e;
   if (JT == 1) e = launch_colred_jt<1>(cfg, p0, p1, nb0, M, r, RP, mchunk);
@@ -359,9 +373,8 @@ static int launch_split_reduce(const float* part, int ksplit, long stride, long 
                                cudaStream_t st) {
   const long vec = count / 4;
   const int grid = (int)std::min<long>((vec + 255) / 256, (long)num_sms() * 8);
-  split_reduce_kernel<<<grid, 256, 0, st>>>(part, ksplit, stride, count, out, out_dtype);
-  g_launches.fetch_add(1, std::memory_order_relaxed);
-  return launch_status();
+  PdlLaunch L(dim3(grid), dim3(256), 0, st);
+  return launch_result(cudaLaunchKernelEx(&L.cfg, split_reduce_kernel, part, ksplit, stride, count, out, out_dtype));
 }
 
 
@@ -416,27 +429,11 @@ static int launch_gemv_q(const CUtensorMap& tW, const CUtensorMap& tX, const GvP
   auto k = qgemv_fwd_kernel<QT, MT>;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return QL_ERR_CUDA;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.N / kGvRows, KS, 1);
-  cfg.blockDim = dim3(kGvThreads, 1, 1);
-  cfg.dynamicSmemBytes = C::SMEM_BYTES;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = KS;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  PdlLaunch L(dim3(p.N / kGvRows, KS, 1), dim3(kGvThreads), C::SMEM_BYTES, st, KS);
   ev_record(slot, 0, st);
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, k, tW, tX, p);
-  g_launches.fetch_add(1, std::memory_order_relaxed);
+  const cudaError_t e = cudaLaunchKernelEx(&L.cfg, k, tW, tX, p);
   ev_record(slot, 1, st);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return QL_ERR_CUDA;
-  }
-  return launch_status();
+  return launch_result(e);
 }
 
 static bool gemv_fwd_applies(int qtype, int64_t M, int r) {
