@@ -532,6 +532,18 @@ def run_reference(args, rank, world):
     }
 
 
+def decode_calls(M, calls=3):
+    """Three forward calls of the decode-shaped linear (the launch a profiler captures)."""
+    import quantized_base_lora_tma_b200 as ql
+    from quantized_base_lora_tma_b200 import build
+    build.build()
+    c = inp.decode_q4_0_8192(M)
+    d = DenseLayerRun(c)
+    for _ in range(calls):
+        ql.qlora_linear_fwd(c.qtype, d.wq, c.N, c.K, d.X, d.A, d.B, c.r, c.scale, d.Y, d.H, d.ws)
+    device_status_ok(f"decode M={M}")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -543,8 +555,14 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-also", action="store_true", help="skip the other shapes of the benchmark set")
+    ap.add_argument("--decode-calls", type=int, default=0, metavar="M",
+                    help="profiling driver: run the decode-shaped Q4_0 8192x8192 forward with M tokens "
+                         "three times and exit (no timing, no JSON line)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.decode_calls:
+        decode_calls(args.decode_calls)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
