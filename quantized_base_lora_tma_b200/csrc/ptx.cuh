@@ -89,31 +89,53 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the thread may sleep (without issuing) until the phase
+// completes or about `hint_ns` pass, instead of spinning on the barrier.
+template <bool CLUSTER = false>
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  if (CLUSTER) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+  }
+  return ok != 0;
+}
+
 // Wait until the phase with the given parity has completed. Returns false (after recording a
-// timeout) if it has not within kWaitLimitNs, or at once if another wait already gave up.
-// With honour_abort = false it ignores other waits' failures (used to drain copies in flight).
+// timeout) if it has not within limit_ns, or at once if another wait already gave up. With
+// honour_abort = false it ignores other waits' failures (used to drain copies in flight).
+// Between polls the thread sleeps in the barrier (suspend hint of 0.2 ms) rather than spinning,
+// so waiting warps leave issue slots (and power) to the warps doing the work. Giving up needs
+// both the time limit and a floor of polls, so that a jump of the global timer alone can never
+// end a wait that is still making progress.
+constexpr uint32_t kSleepHintNs = 200000u;
 template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int site,
                                           bool honour_abort = true, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait<CLUSTER>(bar, parity)) return true;
-  // The abort flag (a global load) and the timer are read only every 1024 polls: both take hundreds
-  // of cycles, during which a completed phase would go unnoticed. Giving up needs both the time
-  // limit and a floor of failed polls, so that a jump of the global timer alone can never end a
-  // wait that is still making progress.
-  uint64_t t0 = 0;
-  uint32_t spins = 0;
-  const uint32_t min_spins = limit_ns >= 1000000ull ? 65536u : 2048u;
+  const uint64_t t0 = globaltimer_ns();
+  const uint32_t hint = limit_ns < 4ull * kSleepHintNs ? (uint32_t)(limit_ns / 4) : kSleepHintNs;
+  uint32_t polls = 0;
   while (true) {
-    if (mbar_try_wait<CLUSTER>(bar, parity)) return true;
-    if ((++spins & 1023u) == 0) {
-      if (honour_abort && dev_aborted()) return false;
-      const uint64_t now = globaltimer_ns();
-      if (t0 == 0) {
-        t0 = now;
-      } else if (spins >= min_spins && now - t0 > limit_ns) {
-        if (honour_abort) dev_fail(QL_ERR_TIMEOUT, site);
-        return false;
-      }
+    if (mbar_try_wait_sleep<CLUSTER>(bar, parity, hint)) return true;
+    ++polls;
+    if (honour_abort && dev_aborted()) return false;
+    if (polls >= 16u && globaltimer_ns() - t0 > limit_ns) {
+      if (honour_abort) dev_fail(QL_ERR_TIMEOUT, site);
+      return false;
     }
   }
 }
