@@ -72,17 +72,23 @@ struct GemmParams {
   float* dw_part;              // SWIGLU_BWD: [M x num_n_tiles] partial <dh_u, h>
 };
 
-template <int QT, bool TRANS, int MS>
+// BN = 128 or 256 output columns per tile. With BN = 256 every A tile feeds twice the columns and
+// each M = 128 MMA is N = 256, which needs a quarter less shared-memory operand bandwidth per FLOP:
+// the single-CTA tile is bound by shared-memory bandwidth (the MMAs' operand reads plus the TMA and
+// dequant traffic), not by the tensor pipe.
+template <int QT, bool TRANS, int MS, int BN_ = 128>
 struct GemmCfg {
   static constexpr int BM = 128 * MS;
-  static constexpr int BN = 128;
+  static constexpr int BN = BN_;
   static constexpr int GB = QTraits<QT>::kGroupBytes;
   static constexpr int A_BYTES = BM * kBK * 2;               // 16 / 32 KB
-  static constexpr int B_BYTES = BN * kBK * 2;               // 16 KB
-  static constexpr int RAW_ROWS = TRANS ? 64 : 128;          // W rows per raw chunk (one group each)
+  static constexpr int B_BYTES = BN * kBK * 2;               // 16 / 32 KB
+  static constexpr int RAW_ROWS = TRANS ? 64 : BN;           // W rows per raw chunk (one group each)
   static constexpr int RAW_BYTES = RAW_ROWS * GB;
-  static constexpr int STAGES = MS == 2 ? 3 : 4;
-  static constexpr int RAW_SLOTS = TRANS ? (GB > 200 ? 4 : 6) : (GB > 200 ? 2 : 3);
+  static constexpr int STAGES = (MS == 2 || BN == 256) ? 3 : 4;
+  static constexpr int RAW_SLOTS = TRANS ? (GB > 200 ? 4 : 6) : (GB > 200 ? 2 : (BN == 256 ? 2 : 3));
+  static constexpr int UNITS = BN / 128;                     // 32-weight units per dequant thread and stage
+  static constexpr int MN_SBO = BN / 64 * 1024;              // MN-major B: bytes per 8 k-rows
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
   static constexpr int OFF_RAW = OFF_B + STAGES * B_BYTES;
@@ -279,12 +285,12 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, const TileInf
   }
 }
 
-template <int QT, bool TRANS, int EPI, int MS>
+template <int QT, bool TRANS, int EPI, int MS, int BN_ = 128>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     qgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
                  const __grid_constant__ CUtensorMap tmLA, const __grid_constant__ CUtensorMap tmLB,
                  const GemmParams p) {
-  using C = GemmCfg<QT, TRANS, MS>;
+  using C = GemmCfg<QT, TRANS, MS, BN_>;
   constexpr int BN = C::BN;
   constexpr int BM = C::BM;
   extern __shared__ uint8_t smem_raw_[];
@@ -373,7 +379,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int i = 0; i < BN / 64; ++i) {
               int y;
-              if (EPI == EPI_SWIGLU) y = lb0 + (i == 0 ? ti.nb * 64 : p.I + ti.nb * 64);
+              // SWIGLU tiles: columns [0, BN/2) are gate rows, [BN/2, BN) the up rows of the same j
+              if (EPI == EPI_SWIGLU)
+                y = lb0 + (i < BN / 128 ? ti.nb * (BN / 2) + 64 * i : p.I + ti.nb * (BN / 2) + 64 * (i - BN / 128));
               else y = lb0 + ti.nb * BN + 64 * i;
               tma_load_2d(sB + s * C::B_BYTES + i * 64 * 128, &tmLB, full_bar(s), x, y);
             }
@@ -406,13 +414,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           mbar_arrive_expect_tx(rfull_bar(s), C::RAW_BYTES);
           const uint32_t dst = sRaw + s * C::RAW_BYTES;
           if (TRANS) {
-            tma_load_2d(dst, &tmW, rfull_bar(s), (ti.nb >> 1) * GW, wbase + c * 64);
+            // the 256-column group holding the tile's columns
+            tma_load_2d(dst, &tmW, rfull_bar(s), (ti.nb * BN / 256) * GW, wbase + c * 64);
           } else {
-            int y0, y1;
-            if (EPI == EPI_SWIGLU) { y0 = wbase + ti.nb * 64; y1 = wbase + p.I + ti.nb * 64; }
-            else { y0 = wbase + ti.nb * 128; y1 = y0 + 64; }
-            tma_load_2d(dst, &tmW, rfull_bar(s), c * GW, y0);
-            tma_load_2d(dst + 64 * C::GB, &tmW, rfull_bar(s), c * GW, y1);
+            // BN rows of W in 64-row boxes (SWIGLU: BN/2 gate rows, then the BN/2 up rows)
+#pragma unroll
+            for (int b = 0; b < BN / 64; ++b) {
+              int y;
+              if (EPI == EPI_SWIGLU)
+                y = wbase + (b < BN / 128 ? ti.nb * (BN / 2) + 64 * b : p.I + ti.nb * (BN / 2) + 64 * (b - BN / 128));
+              else y = wbase + ti.nb * BN + 64 * b;
+              tma_load_2d(dst + b * 64 * C::GB, &tmW, rfull_bar(s), c * GW, y);
+            }
           }
           last_phase[s] = (int)ph;
         }
@@ -450,7 +463,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int k = 0; k < kBK / 16; ++k) {
             uint64_t bd;
             if (kmaj) bd = smem_desc_sw128(b0 + 32 * k, 16, 1024);
-            else bd = smem_desc_sw128(b0 + 4096 * k, 1024, 2048);
+            else bd = smem_desc_sw128(b0 + 2 * C::MN_SBO * k, 1024, C::MN_SBO);
 #pragma unroll
             for (int h = 0; h < MS; ++h) {
               const uint64_t ad = smem_desc_sw128(a0 + h * 16384 + 32 * k, 16, 1024);
@@ -490,9 +503,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int s = it % C::STAGES;
             if (!warp_wait(empty_bar(s), ((it / C::STAGES) & 1) ^ 1, 6)) { ok = false; break; }
             uint8_t* sb = smem + C::OFF_B + s * C::B_BYTES;
-            {
-              // row gt/2 of the tile, 32-weight unit 2*sub + gt%2 of the group
-              const int row = gt >> 1, uh = gt & 1;
+#pragma unroll
+            for (int u = 0; u < C::UNITS; ++u) {
+              // row gt/2 (+ 128 u) of the tile, 32-weight unit 2*sub + gt%2 of the group
+              const int row = (gt >> 1) + 128 * u, uh = gt & 1;
               uint4 v[4];
               decode_unit_bf16<QT>(raw + row * C::GB, 2 * sub + uh, v);
 #pragma unroll
@@ -517,16 +531,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (!warp_wait(empty_bar(s), ((it / C::STAGES) & 1) ^ 1, 6)) { ok = false; break; }
           const uint8_t* raw = smem + C::OFF_RAW + rs * C::RAW_BYTES;
           uint8_t* sb = smem + C::OFF_B + s * C::B_BYTES;
-          {
-            // 32-column unit: row kk = gt/4 of the chunk, unit 4*(nb&1) + gt%4 of the group
-            // (the tile's 128 columns are half of the 256-column group)
-            const int kk = gt >> 2, ul = gt & 3;
+#pragma unroll
+          for (int u = 0; u < C::UNITS; ++u) {
+            // 32-column unit: row kk = gt/4 of the chunk, unit 4u + gt%4 of the tile's columns; the
+            // tile's BN columns are (part of) the 256-column group: unit 4 (nb & 1) + ... for BN = 128
+            const int kk = gt >> 2, ul = 4 * u + (gt & 3);
+            const int gunit = BN == 256 ? ul : 4 * (ti.nb & 1) + ul;
             uint4 v[4];
-            decode_unit_bf16<QT>(raw + kk * C::GB, 4 * (ti.nb & 1) + ul, v);
+            decode_unit_bf16<QT>(raw + kk * C::GB, gunit, v);
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
-              const int gc = 4 * ul + cc;  // 16-byte chunk within the tile's 128 columns
-              const int off = (kk >> 3) * 2048 + (gc >> 3) * 1024 + (kk & 7) * 128 + (((gc & 7) ^ (kk & 7)) << 4);
+              const int gc = 4 * ul + cc;  // 16-byte chunk within the tile's BN columns
+              const int off = (kk >> 3) * C::MN_SBO + (gc >> 3) * 1024 + (kk & 7) * 128 + (((gc & 7) ^ (kk & 7)) << 4);
               *reinterpret_cast<uint4*>(sb + off) = v[cc];
             }
           }

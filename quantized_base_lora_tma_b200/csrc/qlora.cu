@@ -139,11 +139,11 @@ static int launch_result(cudaError_t e) {
   }
   return launch_status();
 }
-template <int QT, bool TRANS, int EPI, int MS>
+template <int QT, bool TRANS, int EPI, int MS, int BN = 128>
 static int launch_qgemm(const CUtensorMap& tA, const CUtensorMap& tW, const CUtensorMap& tLA, const CUtensorMap& tLB,
                         const GemmParams& p, int grid, cudaStream_t st, int slot) {
-  using C = GemmCfg<QT, TRANS, MS>;
-  auto k = qgemm_kernel<QT, TRANS, EPI, MS>;
+  using C = GemmCfg<QT, TRANS, MS, BN>;
+  auto k = qgemm_kernel<QT, TRANS, EPI, MS, BN>;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return QL_ERR_CUDA;
   PdlLaunch L(dim3(grid), dim3(kGemmThreads), C::SMEM_BYTES, st);
@@ -155,13 +155,24 @@ static int launch_qgemm(const CUtensorMap& tA, const CUtensorMap& tW, const CUte
 
 template <bool TRANS, int EPI, int MS>
 static int launch_qgemm_q(int qtype, const CUtensorMap& tA, const CUtensorMap& tW, const CUtensorMap& tLA,
-                          const CUtensorMap& tLB, const GemmParams& p, int grid, cudaStream_t st, int slot) {
+                          const CUtensorMap& tLB, const GemmParams& p, int grid, cudaStream_t st, int slot,
+                          int bn = 128) {
   switch (qtype) {
     case QL_Q8_0: return launch_qgemm<QL_Q8_0, TRANS, EPI, MS>(tA, tW, tLA, tLB, p, grid, st, slot);
-    case QL_Q4_0: return launch_qgemm<QL_Q4_0, TRANS, EPI, MS>(tA, tW, tLA, tLB, p, grid, st, slot);
-    case QL_Q4_K: return launch_qgemm<QL_Q4_K, TRANS, EPI, MS>(tA, tW, tLA, tLB, p, grid, st, slot);
+    case QL_Q4_0:
+      return bn == 256 ? launch_qgemm<QL_Q4_0, TRANS, EPI, MS, 256>(tA, tW, tLA, tLB, p, grid, st, slot)
+                       : launch_qgemm<QL_Q4_0, TRANS, EPI, MS>(tA, tW, tLA, tLB, p, grid, st, slot);
+    case QL_Q4_K:
+      return bn == 256 ? launch_qgemm<QL_Q4_K, TRANS, EPI, MS, 256>(tA, tW, tLA, tLB, p, grid, st, slot)
+                       : launch_qgemm<QL_Q4_K, TRANS, EPI, MS>(tA, tW, tLA, tLB, p, grid, st, slot);
     default: return QL_ERR_UNSUPPORTED;
   }
+}
+
+// Tile width of a grouped GEMM: 256 columns where the 144-byte groups let the raw ring hold 256
+// rows and the output width divides (div = the column count per tile unit), else 128.
+static int grouped_bn(int qtype, int64_t cols, int64_t div256) {
+  return group_bytes(qtype) == 144 && cols % div256 == 0 ? 256 : 128;
 }
 
 // Pair-tile dense GEMM: clusters of two CTAs, one cluster per pair tile slot. The grid is capped at
@@ -793,11 +804,12 @@ int qlora_moe_fwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
       return QL_ERR_CUDA;
     GemmParams p;
     memset(&p, 0, sizeof(p));
-    p.M = P; p.Nd = (int)(2 * I); p.Kd = (int)H; p.n_lora_kb = KL / 64; p.num_n_tiles = (int)(I / 64);
+    const int bn = grouped_bn(qtype, I, 128);  // a tile holds bn/2 gate and bn/2 up columns
+    p.M = P; p.Nd = (int)(2 * I); p.Kd = (int)H; p.n_lora_kb = KL / 64; p.num_n_tiles = (int)(I / (bn / 2));
     p.w_rows_per_expert = (int)(2 * I); p.lb_rows_per_expert = (int)(2 * I); p.I = (int)I;
     p.E = E; p.seg_off = off; p.mblk_off = mblk; p.ksplit = 1;
     p.out_g = g; p.out_u = u; p.out_h = h; p.out_lo = (__nv_bfloat16*)(sb + sv.hlo);
-    rc = launch_qgemm_q<false, EPI_SWIGLU, 1>(qtype, tA, tW, tLA, tLB, p, nsm, st, 2);
+    rc = launch_qgemm_q<false, EPI_SWIGLU, 1>(qtype, tA, tW, tLA, tLB, p, nsm, st, 2, bn);
     if (rc) return rc;
   }
   // down: Hd = h A_d^T (saved), LA = split(s Hd), LB = [B_d | B_d]
@@ -814,11 +826,12 @@ int qlora_moe_fwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
       return QL_ERR_CUDA;
     GemmParams p;
     memset(&p, 0, sizeof(p));
-    p.M = P; p.Nd = (int)H; p.Kd = (int)I; p.n_lora_kb = KL / 64; p.num_n_tiles = (int)(H / 128);
+    const int bn = grouped_bn(qtype, H, 256);
+    p.M = P; p.Nd = (int)H; p.Kd = (int)I; p.n_lora_kb = KL / 64; p.num_n_tiles = (int)(H / bn);
     p.w_rows_per_expert = (int)H; p.lb_rows_per_expert = (int)H; p.I = (int)I;
     p.E = E; p.seg_off = off; p.mblk_off = mblk; p.ksplit = 1;
     p.out = pair_out; p.out_dtype = QL_F32; p.ldo = H; p.row_w = row_w;
-    rc = launch_qgemm_q<false, EPI_PAIR_OUT, 1>(qtype, tA, tW, tLA, tLB, p, nsm, st, 3);
+    rc = launch_qgemm_q<false, EPI_PAIR_OUT, 1>(qtype, tA, tW, tLA, tLB, p, nsm, st, 3, bn);
     if (rc) return rc;
   }
   return launch_combine(pair_out, (int)H, inv_perm, (int)T, k, Y, y_dtype, st);
@@ -875,6 +888,7 @@ int qlora_moe_bwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
   if (rc) return rc;
   rc = launch_gather((const __nv_bfloat16*)dY, (int)H, perm, P, k, dYp, nullptr, nullptr, st);
   if (rc) return rc;
+  int dw_tiles = 0;  // output-column tiles of the down input-gradient GEMM (dw partials per row)
   // down input-gradient: Gd = s dYp B_d, LA = split(Gd), LB[e][i] = [A_d^T | A_d^T]
   rc = launch_rows_seg(dYp, H, (int)H, (const __nv_bfloat16*)B_d, 1, r, (long)H * r, off, mblk, E, r, scale, scale, Gd,
                        LA, ms, st);
@@ -889,11 +903,12 @@ int qlora_moe_bwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
       return QL_ERR_CUDA;
     GemmParams p;
     memset(&p, 0, sizeof(p));
-    p.M = P; p.Nd = (int)I; p.Kd = (int)H; p.n_lora_kb = KL / 64; p.num_n_tiles = (int)(I / 128);
+    dw_tiles = (int)(I / grouped_bn(qtype, I, 256));
+    p.M = P; p.Nd = (int)I; p.Kd = (int)H; p.n_lora_kb = KL / 64; p.num_n_tiles = dw_tiles;
     p.w_rows_per_expert = (int)H; p.lb_rows_per_expert = (int)I; p.I = (int)I;
     p.E = E; p.seg_off = off; p.mblk_off = mblk; p.ksplit = 1;
     p.in_g = g; p.in_u = u; p.in_h = h; p.out_g = dgu; p.out_lo = dgu_lo; p.row_w = row_w; p.dw_part = dwp;
-    rc = launch_qgemm_q<true, EPI_SWIGLU_BWD, 1>(qtype, tA, tW, tLA, tLB, p, nsm, st, 4);
+    rc = launch_qgemm_q<true, EPI_SWIGLU_BWD, 1>(qtype, tA, tW, tLA, tLB, p, nsm, st, 4, grouped_bn(qtype, I, 256));
     if (rc) return rc;
   }
   // down adapter gradients: dA_d = sum_p w_p Gd_p^T h_p ; dB_d = s sum_p w_p dYp_p^T Hd_p
@@ -915,11 +930,12 @@ int qlora_moe_bwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
       return QL_ERR_CUDA;
     GemmParams p;
     memset(&p, 0, sizeof(p));
-    p.M = P; p.Nd = (int)H; p.Kd = (int)(2 * I); p.n_lora_kb = KL / 64; p.num_n_tiles = (int)(H / 128);
+    const int bn = grouped_bn(qtype, H, 256);
+    p.M = P; p.Nd = (int)H; p.Kd = (int)(2 * I); p.n_lora_kb = KL / 64; p.num_n_tiles = (int)(H / bn);
     p.w_rows_per_expert = (int)(2 * I); p.lb_rows_per_expert = (int)H; p.I = (int)I;
     p.E = E; p.seg_off = off; p.mblk_off = mblk; p.ksplit = 1;
     p.out = dxp; p.out_dtype = QL_F32; p.ldo = H;
-    rc = launch_qgemm_q<true, EPI_STORE, 1>(qtype, tA, tW, tLA, tLB, p, nsm, st, 5);
+    rc = launch_qgemm_q<true, EPI_STORE, 1>(qtype, tA, tW, tLA, tLB, p, nsm, st, 5, bn);
     if (rc) return rc;
   }
   rc = launch_combine(dxp, (int)H, inv_perm, (int)T, k, dX, dx_dtype, st);
@@ -930,7 +946,7 @@ int qlora_moe_bwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
   rc = launch_colred(dgu, 2 * I, (int)(2 * I), Hgu, r, P, nullptr, off, mblk, E, ms, part, scale, 0, dB_gu, st, dgu_lo);
   if (rc) return rc;
   if (d_logits != nullptr) {
-    moe_dw_dlogits_kernel<<<(int)((T + 127) / 128), 128, 0, st>>>(dwp, (int)(I / 128), inv_perm, topk_idx, topk_w,
+    moe_dw_dlogits_kernel<<<(int)((T + 127) / 128), 128, 0, st>>>(dwp, dw_tiles, inv_perm, topk_idx, topk_w,
                                                                   (int)T, E, k, nullptr, d_logits);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return launch_status();
