@@ -456,47 +456,58 @@ __global__ void __launch_bounds__(128) lora_rows_cluster_kernel(
   cluster_sync_all();  // no CTA leaves while a peer may still read its partials
 }
 
-// Two column-reduction problems in one launch (dense layer): problem p (blockIdx.x < nb0: p = 0)
-// computes out = scale * sum_m Y[m][c] Z[m][j] over all M rows, for the 128 columns c of this CTA
-// (warp w: columns 32w .. 32w+31). Z is given as its bf16 split [M x 2RP] = [hi | lo] (the sum of
-// the two carries Z to about 2^-16 relative). Cluster rank q takes rows [q * mchunk, (q + 1) *
-// mchunk); 64-row tiles of Y and of the split Z stream through a cp.async ring into mma.sync
-// (A = Z^T by ldmatrix.trans, B = Y by ldmatrix.trans) and the ranks' partials are summed through
-// distributed shared memory in rank order. transpose = 0: out[c][j]; 1: out[j][c].
-struct ColredProblem {
-  const __nv_bfloat16* Y;
-  long ldy;
+// One column-reduction problem of the TMA version: out = scale * sum_m Y[m][c] Z[m][j], Y and Z
+// read through tensor maps (128-byte swizzled 64 x 64 boxes).
+struct ColredOut {
   int C;
-  const __nv_bfloat16* Zs;
   float scale;
   int transpose;
   float* out;
 };
 
-constexpr int kColStages = 4;
-constexpr int kColYS = 128 + 8;  // padded row of a 64 x 128 Y tile (bf16)
-
-// Dynamic shared memory of colred_cluster_kernel: the ring, which later holds the partial tile
-// [16 * JT <= RP][129] fp32.
+constexpr int kColTmaStagesMax = 6;
+// Bytes of one ring stage: two 64 x 64 Y boxes and 2RP/64 boxes of the split operand.
+__host__ __device__ constexpr int colred_stage_bytes(int RP) { return 2 * 8192 + (2 * RP / 64) * 8192; }
+__host__ __device__ constexpr int colred_stages(int RP) { return RP > 32 ? 5 : kColTmaStagesMax; }
 __host__ __device__ constexpr size_t colred_smem_bytes(int RP) {
-  return (size_t)kColStages * 64 * (kColYS + 2 * RP + 8) * 2 > (size_t)RP * (128 + 1) * 4
-             ? (size_t)kColStages * 64 * (kColYS + 2 * RP + 8) * 2
-             : (size_t)RP * (128 + 1) * 4;
+  return (size_t)colred_stages(RP) * colred_stage_bytes(RP) + 2 * kColTmaStagesMax * 8 + 1024;
 }
 
+// Element (row, col) of a 128-byte-swizzled box of 64 bf16 columns: 16-byte chunk col/8 of row
+// `row` sits at chunk position (col/8) ^ (row % 8).
+__device__ __forceinline__ uint32_t sw128_addr(uint32_t box, int row, int col) {
+  return box + (uint32_t)(row * 128) + ((uint32_t)(((col >> 3) ^ (row & 7))) << 4) + (uint32_t)((col & 7) * 2);
+}
+
+// Two column reductions in one launch (dense layer): problem p (blockIdx.x < nb0: p = 0)
+// computes out = scale * sum_m Y[m][c] Z[m][j] for the 128 columns c of this CTA (warp w: columns
+// 32w .. 32w+31). Z is the split operand [M x 2RP] = [hi | lo] of an fp32 tensor (the sum of the
+// two carries it to about 2^-16 relative). Cluster rank q takes rows [q * mchunk, (q + 1) * mchunk);
+// one thread streams 64-row tiles of Y and Z by TMA into a ring of mbarrier-guarded stages, the
+// four warps feed them to mma.sync through ldmatrix.trans (A = Z^T, B = Y), and the ranks' partials
+// are summed through distributed shared memory in rank order. transpose = 0: out[c][j];
+// 1: out[j][c].
 template <int JT>
-__global__ void __launch_bounds__(128) colred_cluster_kernel(ColredProblem p0, ColredProblem p1, int nb0, int M,
-                                                             int r, int RP, int mchunk) {
-  constexpr int S = kColStages, YS = kColYS;
-  extern __shared__ __align__(16) uint8_t col_smem[];
+__global__ void __launch_bounds__(128) colred_cluster_kernel(const __grid_constant__ CUtensorMap tmY0,
+                                                             const __grid_constant__ CUtensorMap tmY1,
+                                                             const __grid_constant__ CUtensorMap tmZ0,
+                                                             const __grid_constant__ CUtensorMap tmZ1, ColredOut o0,
+                                                             ColredOut o1, int nb0, int M, int r, int RP, int mchunk) {
+  extern __shared__ uint8_t col_smem_raw[];
+  const uint32_t base = (smem_u32(col_smem_raw) + 1023u) & ~1023u;
+  uint8_t* smem = col_smem_raw + (base - smem_u32(col_smem_raw));
   pdl_launch_dependents();
-  pdl_wait();
-  const int ZW = 2 * RP + 8;  // padded row of a 64 x 2RP split-Z tile
-  __nv_bfloat16* yring = reinterpret_cast<__nv_bfloat16*>(col_smem);
-  __nv_bfloat16* zring = yring + S * 64 * YS;
-  auto part = reinterpret_cast<float(*)[128 + 1]>(col_smem);  // reused after the main loop
+  const int S = colred_stages(RP);
+  const int SB = colred_stage_bytes(RP);
+  const int zboxes = 2 * RP / 64;
+  const uint32_t bar0 = base + (uint32_t)(S * SB);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (kColTmaStagesMax + s); };
+  auto part = reinterpret_cast<float(*)[128 + 1]>(smem);  // reuses the ring after the main loop
   const bool second = (int)blockIdx.x >= nb0;
-  const ColredProblem& P = second ? p1 : p0;
+  const CUtensorMap* tmY = second ? &tmY1 : &tmY0;
+  const CUtensorMap* tmZ = second ? &tmZ1 : &tmZ0;
+  const ColredOut& P = second ? o1 : o0;
   const int c0 = (second ? (int)blockIdx.x - nb0 : (int)blockIdx.x) * 128;
   const uint32_t rank = cluster_ctarank();
   const int CS = gridDim.y;
@@ -505,55 +516,54 @@ __global__ void __launch_bounds__(128) colred_cluster_kernel(ColredProblem p0, C
   const int ntiles = hi > lo ? (hi - lo + 63) / 64 : 0;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  auto issue = [&](int t) {
-    const int mb = lo + 64 * t;
-    const uint32_t ydst = smem_u32(yring + (t % S) * 64 * YS);
-#pragma unroll
-    for (int it = 0; it < 64 * 16 / 128; ++it) {
-      const int i = tid + 128 * it;
-      const int m = i >> 4, q = i & 15;
-      const bool v = (mb + m < hi) && (c0 + 8 * q < P.C);
-      cp_async16(ydst + (uint32_t)(m * YS + 8 * q) * 2, v ? (const void*)(P.Y + (long)(mb + m) * P.ldy + c0 + 8 * q) : (const void*)P.Y, v);
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 4);
     }
-    const uint32_t zdst = smem_u32(zring + (t % S) * 64 * ZW);
-    const int zq = 2 * RP / 8;  // 16-byte chunks per split-Z row
-    for (int i = tid; i < 64 * zq; i += 128) {
-      const int m = i / zq, q = i % zq;
-      const bool v = mb + m < hi;
-      cp_async16(zdst + (uint32_t)(m * ZW + 8 * q) * 2, v ? (const void*)(P.Zs + (long)(mb + m) * 2 * RP + 8 * q) : (const void*)P.Zs, v);
-    }
-  };
-#pragma unroll
-  for (int t = 0; t < S - 1; ++t) {
-    if (t < ntiles) issue(t);
-    cp_async_commit();
+    fence_mbar_init();
+    prefetch_tmap(tmY);
+    prefetch_tmap(tmZ);
   }
+  __syncthreads();
+  pdl_wait();
+
+  auto issue = [&](int t) {
+    const int s = t % S;
+    const uint32_t st = base + (uint32_t)(s * SB);
+    const int mb = lo + 64 * t;
+    mbar_arrive_expect_tx(full_bar(s), (uint32_t)SB);
+    tma_load_2d(st, tmY, full_bar(s), c0, mb);
+    tma_load_2d(st + 8192, tmY, full_bar(s), c0 + 64, mb);
+    for (int zb = 0; zb < zboxes; ++zb) tma_load_2d(st + 16384 + 8192 * zb, tmZ, full_bar(s), 64 * zb, mb);
+  };
+  if (tid == 0)
+    for (int t = 0; t < min(ntiles, S); ++t) issue(t);
 
   float acc[JT][4][4];
 #pragma unroll
   for (int jt = 0; jt < JT; ++jt)
 #pragma unroll
     for (int t = 0; t < 4; ++t) acc[jt][t][0] = acc[jt][t][1] = acc[jt][t][2] = acc[jt][t][3] = 0.f;
-  const int wc = warp * 32;
   // ldmatrix.trans lane addresses. B (Y, k = m, n = c): matrices (m 0-7 | 8-15) x (c 0-7 | 8-15).
   // A (Z^T, rows j, k = m): matrices (j 0-7, m 0-7), (j 8-15, m 0-7), (j 0-7, m 8-15), (j 8-15, m 8-15).
   const int mat = lane >> 3, rr = lane & 7;
-  const int yb_row = ((mat & 1) ? 8 : 0) + rr, yb_col = wc + ((mat & 2) ? 8 : 0);
+  const int yb_row = ((mat & 1) ? 8 : 0) + rr, yb_col = 32 * (warp & 1) + ((mat & 2) ? 8 : 0);
   const int za_row = rr + ((mat & 2) ? 8 : 0), za_col = (mat & 1) ? 8 : 0;
+  bool ok = true;
   for (int t = 0; t < ntiles; ++t) {
-    cp_async_wait<S - 2>();
-    __syncthreads();
-    if (t + S - 1 < ntiles) issue(t + S - 1);
-    cp_async_commit();
-    const uint32_t ybase = smem_u32(yring + (t % S) * 64 * YS + yb_row * YS + yb_col);
-    const uint32_t zbase = smem_u32(zring + (t % S) * 64 * ZW + za_row * ZW + za_col);
+    const int s = t % S;
+    if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), (uint32_t)((t / S) & 1), 31))) { ok = false; break; }
+    const uint32_t st = base + (uint32_t)(s * SB);
+    const uint32_t ybox = st + 8192u * (uint32_t)(warp >> 1);
+    const uint32_t zbox = st + 16384u;
 #pragma unroll
     for (int k = 0; k < 64; k += 16) {
       uint32_t b[4][2];
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
         uint32_t x0, x1, x2, x3;
-        ldsm_x4_t(ybase + (uint32_t)(k * YS + 16 * h2) * 2, x0, x1, x2, x3);
+        ldsm_x4_t(sw128_addr(ybox, k + yb_row, yb_col + 16 * h2), x0, x1, x2, x3);
         b[2 * h2][0] = x0;
         b[2 * h2][1] = x1;
         b[2 * h2 + 1][0] = x2;
@@ -561,9 +571,10 @@ __global__ void __launch_bounds__(128) colred_cluster_kernel(ColredProblem p0, C
       }
 #pragma unroll
       for (int jt = 0; jt < JT; ++jt) {
+        const int ch = za_col + 16 * jt, cl = ch + RP;  // hi and lo columns of the split operand
         uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
-        ldsm_x4_t(zbase + (uint32_t)(k * ZW + 16 * jt) * 2, h0, h1, h2, h3);
-        ldsm_x4_t(zbase + (uint32_t)(k * ZW + RP + 16 * jt) * 2, l0, l1, l2, l3);
+        ldsm_x4_t(sw128_addr(zbox + 8192u * (uint32_t)(ch >> 6), k + za_row, ch & 63), h0, h1, h2, h3);
+        ldsm_x4_t(sw128_addr(zbox + 8192u * (uint32_t)(cl >> 6), k + za_row, cl & 63), l0, l1, l2, l3);
 #pragma unroll
         for (int n = 0; n < 4; ++n) {
           mma_16816(acc[jt][n], h0, h1, h2, h3, b[n][0], b[n][1]);
@@ -571,11 +582,23 @@ __global__ void __launch_bounds__(128) colred_cluster_kernel(ColredProblem p0, C
         }
       }
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty_bar(s));
+    if (warp == 0 && t + S < ntiles) {
+      // thread 0 refills this slot once all four warps have released it
+      bool w = true;
+      if (lane == 0) {
+        w = mbar_wait(empty_bar(s), (uint32_t)((t / S) & 1), 32);
+        if (w) issue(t + S);
+      }
+      if (!__shfl_sync(0xffffffffu, w ? 1 : 0, 0)) { ok = false; break; }
+    }
   }
-  cp_async_wait<0>();
+  if (!ok || dev_aborted()) spin_ns(2000000ull);  // copies issued before a wait gave up land first
   __syncthreads();  // the ring becomes the partial tile
   {
     const int g = lane >> 2, c = lane & 3;
+    const int wc = warp * 32;
 #pragma unroll
     for (int jt = 0; jt < JT; ++jt)
 #pragma unroll
@@ -597,8 +620,8 @@ __global__ void __launch_bounds__(128) colred_cluster_kernel(ColredProblem p0, C
     const int col = c0 + cl;
     if (cl >= 128 || col >= P.C) continue;
     const float v = cluster_sum_ordered(&part[j][cl], CS);
-    const long o = P.transpose ? (long)j * P.C + col : (long)col * r + j;
-    P.out[o] = P.scale * v;
+    const long oi = P.transpose ? (long)j * P.C + col : (long)col * r + j;
+    P.out[oi] = P.scale * v;
   }
   cluster_sync_all();
 }

@@ -289,33 +289,42 @@ static int launch_rows_dense(const __nv_bfloat16* Y, long ldy, int M, int Kin, c
   return launch_status();
 }
 
-// Two dense column reductions in one launch (dB and dA of the backward).
+// Two dense column reductions in one launch (dB and dA of the backward): out_p = scale_p *
+// Y_p^T Z_p for Y_p [M x C_p] bf16 and the split operands Z_p [M x 2RP] bf16.
 template <int JT>
-static cudaError_t launch_colred_jt(cudaLaunchConfig_t& cfg, const ColredProblem& p0, const ColredProblem& p1, int nb0,
-                                    int M, int r, int RP, int mchunk) {
+static cudaError_t launch_colred_jt(cudaLaunchConfig_t& cfg, const CUtensorMap* tm, const ColredOut& o0,
+                                    const ColredOut& o1, int nb0, int M, int r, int RP, int mchunk) {
   auto k = colred_cluster_kernel<JT>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cfg.dynamicSmemBytes);
   if (e != cudaSuccess) return e;
-  return cudaLaunchKernelEx(&cfg, k, p0, p1, nb0, M, r, RP, mchunk);
+  return cudaLaunchKernelEx(&cfg, k, tm[0], tm[1], tm[2], tm[3], o0, o1, nb0, M, r, RP, mchunk);
 }
 
-static int launch_colred_dense(const ColredProblem& p0, const ColredProblem& p1, int M, int r, cudaStream_t st) {
+static int launch_colred_dense(const __nv_bfloat16* Y0, int C0, const __nv_bfloat16* Z0, const ColredOut& o0,
+                               const __nv_bfloat16* Y1, int C1, const __nv_bfloat16* Z1, const ColredOut& o1, int M, int r,
+                               cudaStream_t st) {
   const int RP = lora_rp(r);
-  const int nb0 = (p0.C + 127) / 128, nb1 = (p1.C + 127) / 128;
-  // row slices per column block: as many as keep every CTA resident in one wave (two per SM)
-  const int CS_max = std::max(1, std::min(8, 2 * num_sms() / (nb0 + nb1)));
+  CUtensorMap tm[4];
+  if (!tmap_bf16_rows(&tm[0], Y0, C0, M, 64) || !tmap_bf16_rows(&tm[1], Y1, C1, M, 64) ||
+      !tmap_bf16_rows(&tm[2], Z0, 2 * RP, M, 64) || !tmap_bf16_rows(&tm[3], Z1, 2 * RP, M, 64))
+    return QL_ERR_CUDA;
+  const int nb0 = (C0 + 127) / 128, nb1 = (C1 + 127) / 128;
+  // row slices per column block: as many as keep every CTA resident in one wave
+  const size_t smem = colred_smem_bytes(RP);
+  const int per_sm = std::max(1, (int)(233472 / (smem + 1024)));
+  const int CS_max = std::max(1, std::min(8, per_sm * num_sms() / (nb0 + nb1)));
   int CS = std::max(1, std::min(CS_max, (M + 63) / 64));
   int mchunk = (M + CS - 1) / CS;
   mchunk = (mchunk + 63) / 64 * 64;
   CS = (M + mchunk - 1) / mchunk;
-  PdlLaunch L(dim3(nb0 + nb1, CS, 1), dim3(128), colred_smem_bytes(RP), st, CS);
+  PdlLaunch L(dim3(nb0 + nb1, CS, 1), dim3(128), smem, st, CS);
   cudaLaunchConfig_t& cfg = L.cfg;
   const int JT = (r + 15) / 16;
   cudaError_t e;
-  if (JT == 1) e = launch_colred_jt<1>(cfg, p0, p1, nb0, M, r, RP, mchunk);
-  else if (JT == 2) e = launch_colred_jt<2>(cfg, p0, p1, nb0, M, r, RP, mchunk);
-  else if (JT == 3) e = launch_colred_jt<3>(cfg, p0, p1, nb0, M, r, RP, mchunk);
-  else e = launch_colred_jt<4>(cfg, p0, p1, nb0, M, r, RP, mchunk);
+  if (JT == 1) e = launch_colred_jt<1>(cfg, tm, o0, o1, nb0, M, r, RP, mchunk);
+  else if (JT == 2) e = launch_colred_jt<2>(cfg, tm, o0, o1, nb0, M, r, RP, mchunk);
+  else if (JT == 3) e = launch_colred_jt<3>(cfg, tm, o0, o1, nb0, M, r, RP, mchunk);
+  else e = launch_colred_jt<4>(cfg, tm, o0, o1, nb0, M, r, RP, mchunk);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -985,9 +994,10 @@ int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void
     if (rc) return rc;
   }
   // dB = dY^T split(s H) and dA = split(G)^T X in one launch
-  const ColredProblem pb{(const __nv_bfloat16*)dY, N, (int)N, HS, 1.0f, 0, dB};
-  const ColredProblem pa{(const __nv_bfloat16*)X, K, (int)K, LA, 1.0f, 1, dA};
-  return launch_colred_dense(pb, pa, (int)M, r, st);
+  const ColredOut ob{(int)N, 1.0f, 0, dB};
+  const ColredOut oa{(int)K, 1.0f, 1, dA};
+  return launch_colred_dense((const __nv_bfloat16*)dY, (int)N, HS, ob, (const __nv_bfloat16*)X, (int)K, LA, oa, (int)M,
+                             r, st);
 }
 
 }  // extern "C"
