@@ -223,13 +223,13 @@ __global__ void __launch_bounds__(kGvThreads) qgemv_fwd_kernel(const __grid_cons
     }
     fence_mbar_init();
   }
-  pdl_launch_dependents();
   if (warp == kGvWarpA && lane == 0) {
     prefetch_tmap(&tmW);
     prefetch_tmap(&tmX);
   }
   __syncthreads();
   pdl_wait();  // inputs of the previous kernel in the stream are complete from here on
+  pdl_launch_dependents();  // after the wait: a dependent may rely on what this launch waited for
 
   auto issue = [&](int i) {  // stage i of this slice into slot i % STAGES
     const int s = i % C::STAGES;

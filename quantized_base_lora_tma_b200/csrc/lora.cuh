@@ -4,11 +4,12 @@
 //            and the tensor-core operand LA[m] = [hi(v) | lo(v)], v = lscale * sum
 //   bop      LB[n] = [Z(n, :) | Z(n, :)]                        B (forward) or A^T (dX)
 //   colred   out[c, j] = sum_m Y[m, c] Z[m, j] over row slices, then an ordered sum over the
-//            slices: dB = dY^T split(s H), dA = split(G)^T X (deterministic: no atomics)
+//            slices: dB = dY^T split(s H), dA = split(G)^T X (deterministic: no float atomics)
 //
-// Dense layer: lora_rows_cluster_kernel and colred_cluster_kernel stream their bf16 operand through
-// a cp.async ring and sum the slices in-cluster. Routed (grouped) layer: lora_rows_seg_kernel,
-// colred_mma_kernel + colred_reduce_kernel, lora_bop_vec_kernel.
+// Dense layer: lora_rows_cluster_kernel streams its bf16 operand through a cp.async ring and sums
+// its k slices in-cluster; colred_flow_kernel streams through a TMA ring, takes units of work from
+// a counter and sums a block's row slices in slice order. Routed (grouped) layer:
+// lora_rows_seg_kernel, colred_mma_kernel + colred_reduce_kernel, lora_bop_vec_kernel.
 //
 // The fast LoRA backward these implement is the plain chain rule of the layer (Show HN: LoRA over
 // GGUF, "Things involved in the training": "Fast LoRA bwd formula like Unsloth for linear layer
@@ -291,12 +292,14 @@ __global__ void __launch_bounds__(128) lora_rows_cluster_kernel(
     const __nv_bfloat16* __restrict__ Y, long ldy, int M, int Kin, int kchunk, const __nv_bfloat16* __restrict__ Z,
     long zj, long zk, int r, float oscale, float lscale, float* __restrict__ out, __nv_bfloat16* __restrict__ la,
     int RP, BopArgs bop, __nv_bfloat16* __restrict__ LB, int row_blocks, const float* __restrict__ hin, float hscale,
-    __nv_bfloat16* __restrict__ hs) {
+    __nv_bfloat16* __restrict__ hs, int* __restrict__ zc, int zn) {
   constexpr int RN = 8 * NT;
   constexpr int S = kRowsStages, TK = kRowsTileK, YS = kRowsYS;
   extern __shared__ __align__(16) uint8_t rows_smem[];
-  pdl_launch_dependents();
   pdl_wait();
+  pdl_launch_dependents();
+  if (blockIdx.x == 0 && blockIdx.y == 0)
+    for (int i = threadIdx.x; i < zn; i += blockDim.x) zc[i] = 0;  // counters of a later kernel
   if ((int)blockIdx.x >= row_blocks) {
     lora_bop_share(bop, r, RP, LB);
     return;
@@ -456,21 +459,46 @@ __global__ void __launch_bounds__(128) lora_rows_cluster_kernel(
   cluster_sync_all();  // no CTA leaves while a peer may still read its partials
 }
 
-// One column-reduction problem of the TMA version: out = scale * sum_m Y[m][c] Z[m][j], Y and Z
-// read through tensor maps (128-byte swizzled 64 x 64 boxes).
+// Dense column reductions (dB and dA of the backward) in one launch, as units of work claimed
+// from a counter: out_p = scale_p * sum_m Y_p[m][c] Z_p[m][j] for Y_p [M x C_p] and the split
+// operand Z_p [M x 2RP] = [hi | lo] bf16 of an fp32 tensor (the two together carry it to about
+// 2^-16 relative), both read through tensor maps (128-byte swizzled 64 x 64 boxes).
 struct ColredOut {
   int C;
   float scale;
-  int transpose;
+  int transpose;  // 0: out[c][j]; 1: out[j][c]
   float* out;
+};
+// The columns of both problems form nblk blocks of 128 (the first nb0 of problem 0); the rows form
+// csu chunks of mchunk (a multiple of the tile height tr, every chunk non-empty). A unit is one
+// (block, chunk),
+// u = block * csu + chunk. With csu > 1 each unit leaves its fp32 partial [16 JT][128] in part, and
+// whichever CTA finishes the last chunk of a block sums that block's partials in chunk order, so
+// the result does not depend on which CTA took which unit.
+struct ColredFlow {
+  ColredOut o0, o1;
+  int nb0, nblk, M, r, RP, mchunk, csu;
+  int tr;          // rows per streamed tile (64, 128 or 256): the height of every TMA box
+  int defer_wait;  // 1: the previous kernel in the stream already waited for this launch's inputs
+  float* part;     // [nblk * csu][16 JT][128]
+  int* ctr;        // [0]: next unit to claim, [1 + b]: chunks of block b finished; zero at launch
 };
 
 constexpr int kColTmaStagesMax = 6;
-// Bytes of one ring stage: two 64 x 64 Y boxes and 2RP/64 boxes of the split operand.
-__host__ __device__ constexpr int colred_stage_bytes(int RP) { return 2 * 8192 + (2 * RP / 64) * 8192; }
-__host__ __device__ constexpr int colred_stages(int RP) { return RP > 32 ? 5 : kColTmaStagesMax; }
-__host__ __device__ constexpr size_t colred_smem_bytes(int RP) {
-  return (size_t)colred_stages(RP) * colred_stage_bytes(RP) + 2 * kColTmaStagesMax * 8 + 1024;
+constexpr int kColWarps = 9;  // eight consumer warps and one producer warp
+constexpr int kColCombStride = 136;
+// Bytes of one ring stage: two tr x 64 Y boxes and 2RP/64 boxes of the split operand, 128-byte rows.
+__host__ __device__ constexpr int colred_stage_bytes(int RP, int tr) { return (2 + 2 * RP / 64) * tr * 128; }
+__host__ __device__ constexpr int colred_comb_bytes(int JT) { return 16 * JT * kColCombStride * 4; }
+// Ring stages: as many as fit beside the combine tile, the tags and barriers (256 bytes) and the
+// alignment slack, up to six.
+__host__ __device__ constexpr int colred_stages(int RP, int JT, int tr) {
+  return (232448 - 1024 - 256 - colred_comb_bytes(JT)) / colred_stage_bytes(RP, tr) < kColTmaStagesMax
+             ? (232448 - 1024 - 256 - colred_comb_bytes(JT)) / colred_stage_bytes(RP, tr)
+             : kColTmaStagesMax;
+}
+__host__ __device__ constexpr size_t colred_smem_bytes(int RP, int JT, int tr) {
+  return (size_t)colred_stages(RP, JT, tr) * colred_stage_bytes(RP, tr) + colred_comb_bytes(JT) + 256 + 1024;
 }
 
 // Element (row, col) of a 128-byte-swizzled box of 64 bf16 columns: 16-byte chunk col/8 of row
@@ -479,151 +507,275 @@ __device__ __forceinline__ uint32_t sw128_addr(uint32_t box, int row, int col) {
   return box + (uint32_t)(row * 128) + ((uint32_t)(((col >> 3) ^ (row & 7))) << 4) + (uint32_t)((col & 7) * 2);
 }
 
-// Two column reductions in one launch (dense layer): problem p (blockIdx.x < nb0: p = 0)
-// computes out = scale * sum_m Y[m][c] Z[m][j] for the 128 columns c of this CTA (warp w: columns
-// 32w .. 32w+31). Z is the split operand [M x 2RP] = [hi | lo] of an fp32 tensor (the sum of the
-// two carries it to about 2^-16 relative). Cluster rank q takes rows [q * mchunk, (q + 1) * mchunk);
-// one thread streams 64-row tiles of Y and Z by TMA into a ring of mbarrier-guarded stages, the
-// four warps feed them to mma.sync through ldmatrix.trans (A = Z^T, B = Y), and the ranks' partials
-// are summed through distributed shared memory in rank order. transpose = 0: out[c][j];
-// 1: out[j][c].
+__device__ __forceinline__ void colred_store(const ColredOut& O, int r, int j, int col, float v) {
+  if (j < r && col < O.C) O.out[O.transpose ? (long)j * O.C + col : (long)col * r + j] = O.scale * v;
+}
+
+// Sum of block d's partials in chunk order (the 256 consumer threads).
 template <int JT>
-__global__ void __launch_bounds__(128) colred_cluster_kernel(const __grid_constant__ CUtensorMap tmY0,
-                                                             const __grid_constant__ CUtensorMap tmY1,
-                                                             const __grid_constant__ CUtensorMap tmZ0,
-                                                             const __grid_constant__ CUtensorMap tmZ1, ColredOut o0,
-                                                             ColredOut o1, int nb0, int M, int r, int RP, int mchunk) {
+__device__ void colred_reduce_block(const ColredFlow& P, int d, int tid) {
+  const bool second = d >= P.nb0;
+  const ColredOut& O = second ? P.o1 : P.o0;
+  const int c0 = (second ? d - P.nb0 : d) * 128;
+  const float* src = P.part + (size_t)d * P.csu * (16 * JT * 128);
+  for (int i = tid; i < 16 * JT * 32; i += 256) {
+    const int j = i >> 5, c4 = (i & 31) * 4;
+    if (j >= P.r) continue;
+    float4 a = __ldcg(reinterpret_cast<const float4*>(src + j * 128 + c4));
+    for (int q = 1; q < P.csu; ++q) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(src + (size_t)q * (16 * JT * 128) + j * 128 + c4));
+      a.x += v.x;
+      a.y += v.y;
+      a.z += v.z;
+      a.w += v.w;
+    }
+    colred_store(O, P.r, j, c0 + c4, a.x);
+    colred_store(O, P.r, j, c0 + c4 + 1, a.y);
+    colred_store(O, P.r, j, c0 + c4 + 2, a.z);
+    colred_store(O, P.r, j, c0 + c4 + 3, a.w);
+  }
+}
+
+// Persistent column reduction. Warp 8 (one lane) claims units from ctr[0], one ahead, and streams
+// their 64-row tiles of Y and Z by TMA into a ring of mbarrier-guarded stages, each stage tagged
+// with its unit and whether it opens or closes it. Consumer warp w takes columns 32 (w % 4) ..
+// +31 of the block and rows 32 (w / 4) .. +31 of each tile, through ldmatrix.trans and mma.sync
+// (A = Z^T, B = Y); at a unit's end the two row halves are added through shared memory and the
+// result goes out (csu = 1) or to the unit's partial. With defer_wait the wait for the previous
+// kernel moves to the end, so that the launch can run beside it on SMs it leaves idle.
+template <int JT>
+__global__ void __launch_bounds__(32 * kColWarps) colred_flow_kernel(const __grid_constant__ CUtensorMap tmY0,
+                                                                     const __grid_constant__ CUtensorMap tmY1,
+                                                                     const __grid_constant__ CUtensorMap tmZ0,
+                                                                     const __grid_constant__ CUtensorMap tmZ1,
+                                                                     const ColredFlow P) {
   extern __shared__ uint8_t col_smem_raw[];
   const uint32_t base = (smem_u32(col_smem_raw) + 1023u) & ~1023u;
   uint8_t* smem = col_smem_raw + (base - smem_u32(col_smem_raw));
   pdl_launch_dependents();
-  const int S = colred_stages(RP);
-  const int SB = colred_stage_bytes(RP);
-  const int zboxes = 2 * RP / 64;
-  const uint32_t bar0 = base + (uint32_t)(S * SB);
+  const int S = colred_stages(P.RP, JT, P.tr);
+  const int SB = colred_stage_bytes(P.RP, P.tr);
+  const int YB = P.tr * 128;  // bytes of one box
+  const int zboxes = 2 * P.RP / 64;
+  float* comb = reinterpret_cast<float*>(smem + (size_t)S * SB);
+  volatile int* meta = reinterpret_cast<volatile int*>(smem + (size_t)S * SB + colred_comb_bytes(JT));
+  volatile int* pend_smem = meta + 2 * kColTmaStagesMax;
+  const uint32_t bar0 = base + (uint32_t)(S * SB + colred_comb_bytes(JT) + 64);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (kColTmaStagesMax + s); };
-  auto part = reinterpret_cast<float(*)[128 + 1]>(smem);  // reuses the ring after the main loop
-  const bool second = (int)blockIdx.x >= nb0;
-  const CUtensorMap* tmY = second ? &tmY1 : &tmY0;
-  const CUtensorMap* tmZ = second ? &tmZ1 : &tmZ0;
-  const ColredOut& P = second ? o1 : o0;
-  const int c0 = (second ? (int)blockIdx.x - nb0 : (int)blockIdx.x) * 128;
-  const uint32_t rank = cluster_ctarank();
-  const int CS = gridDim.y;
-  const int lo = (int)rank * mchunk;
-  const int hi = min(M, lo + mchunk);
-  const int ntiles = hi > lo ? (hi - lo + 63) / 64 : 0;
+  const uint32_t sync_bar = bar0 + 8u * (2 * kColTmaStagesMax);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int U = P.nblk * P.csu;
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 4);
+      mbar_init(empty_bar(s), 8);
     }
+    mbar_init(sync_bar, 8);
     fence_mbar_init();
-    prefetch_tmap(tmY);
-    prefetch_tmap(tmZ);
+  }
+  if (warp == 8 && lane == 0) {
+    prefetch_tmap(&tmY0);
+    prefetch_tmap(&tmY1);
+    prefetch_tmap(&tmZ0);
+    prefetch_tmap(&tmZ1);
   }
   __syncthreads();
-  pdl_wait();
+  if (!P.defer_wait) pdl_wait();
 
-  auto issue = [&](int t) {
-    const int s = t % S;
-    const uint32_t st = base + (uint32_t)(s * SB);
-    const int mb = lo + 64 * t;
-    mbar_arrive_expect_tx(full_bar(s), (uint32_t)SB);
-    tma_load_2d(st, tmY, full_bar(s), c0, mb);
-    tma_load_2d(st + 8192, tmY, full_bar(s), c0 + 64, mb);
-    for (int zb = 0; zb < zboxes; ++zb) tma_load_2d(st + 16384 + 8192 * zb, tmZ, full_bar(s), 64 * zb, mb);
-  };
-  if (tid == 0)
-    for (int t = 0; t < min(ntiles, S); ++t) issue(t);
-
-  float acc[JT][4][4];
-#pragma unroll
-  for (int jt = 0; jt < JT; ++jt)
-#pragma unroll
-    for (int t = 0; t < 4; ++t) acc[jt][t][0] = acc[jt][t][1] = acc[jt][t][2] = acc[jt][t][3] = 0.f;
-  // ldmatrix.trans lane addresses. B (Y, k = m, n = c): matrices (m 0-7 | 8-15) x (c 0-7 | 8-15).
-  // A (Z^T, rows j, k = m): matrices (j 0-7, m 0-7), (j 8-15, m 0-7), (j 0-7, m 8-15), (j 8-15, m 8-15).
-  const int mat = lane >> 3, rr = lane & 7;
-  const int yb_row = ((mat & 1) ? 8 : 0) + rr, yb_col = 32 * (warp & 1) + ((mat & 2) ? 8 : 0);
-  const int za_row = rr + ((mat & 2) ? 8 : 0), za_col = (mat & 1) ? 8 : 0;
   bool ok = true;
-  for (int t = 0; t < ntiles; ++t) {
-    const int s = t % S;
-    if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), (uint32_t)((t / S) & 1), 31))) { ok = false; break; }
-    const uint32_t st = base + (uint32_t)(s * SB);
-    const uint32_t ybox = st + 8192u * (uint32_t)(warp >> 1);
-    const uint32_t zbox = st + 16384u;
-#pragma unroll
-    for (int k = 0; k < 64; k += 16) {
-      uint32_t b[4][2];
-#pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        uint32_t x0, x1, x2, x3;
-        ldsm_x4_t(sw128_addr(ybox, k + yb_row, yb_col + 16 * h2), x0, x1, x2, x3);
-        b[2 * h2][0] = x0;
-        b[2 * h2][1] = x1;
-        b[2 * h2 + 1][0] = x2;
-        b[2 * h2 + 1][1] = x3;
-      }
-#pragma unroll
-      for (int jt = 0; jt < JT; ++jt) {
-        const int ch = za_col + 16 * jt, cl = ch + RP;  // hi and lo columns of the split operand
-        uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
-        ldsm_x4_t(sw128_addr(zbox + 8192u * (uint32_t)(ch >> 6), k + za_row, ch & 63), h0, h1, h2, h3);
-        ldsm_x4_t(sw128_addr(zbox + 8192u * (uint32_t)(cl >> 6), k + za_row, cl & 63), l0, l1, l2, l3);
-#pragma unroll
-        for (int n = 0; n < 4; ++n) {
-          mma_16816(acc[jt][n], h0, h1, h2, h3, b[n][0], b[n][1]);
-          mma_16816(acc[jt][n], l0, l1, l2, l3, b[n][0], b[n][1]);
+  if (warp == 8) {
+    if (lane == 0) {
+      int it = 0;
+      int u = atomicAdd(P.ctr, 1);
+      while (true) {
+        const int nxt = u < U ? atomicAdd(P.ctr, 1) : U;  // the next claim travels while this unit streams
+        if (u >= U) {
+          // no work left: a tile-less stage tagged -1 tells the consumers
+          const int s = it % S;
+          if (it >= S && !mbar_wait(empty_bar(s), (uint32_t)((it / S - 1) & 1), 33)) {
+            ok = false;
+            break;
+          }
+          meta[2 * s] = -1;
+          mbar_arrive(full_bar(s));
+          break;
         }
+        const int b = u / P.csu, q = u - b * P.csu;
+        const bool second = b >= P.nb0;
+        const CUtensorMap* tmY = second ? &tmY1 : &tmY0;
+        const CUtensorMap* tmZ = second ? &tmZ1 : &tmZ0;
+        const int c0 = (second ? b - P.nb0 : b) * 128;
+        const int lo = q * P.mchunk, hi = min(P.M, lo + P.mchunk);
+        const int nt = (hi - lo + P.tr - 1) / P.tr;
+        for (int t = 0; t < nt && ok; ++t, ++it) {
+          const int s = it % S;
+          if (it >= S && !mbar_wait(empty_bar(s), (uint32_t)((it / S - 1) & 1), 33)) {
+            ok = false;
+            break;
+          }
+          meta[2 * s] = u;
+          meta[2 * s + 1] = (t == 0 ? 1 : 0) | (t == nt - 1 ? 2 : 0);
+          const uint32_t st = base + (uint32_t)(s * SB);
+          const int mb = lo + P.tr * t;
+          mbar_arrive_expect_tx(full_bar(s), (uint32_t)SB);
+          tma_load_2d(st, tmY, full_bar(s), c0, mb);
+          tma_load_2d(st + YB, tmY, full_bar(s), c0 + 64, mb);
+          for (int zb = 0; zb < zboxes; ++zb) tma_load_2d(st + (2 + zb) * YB, tmZ, full_bar(s), 64 * zb, mb);
+        }
+        if (!ok) break;
+        u = nxt;
       }
     }
+    // the idle lanes must not run ahead to the final wait: griddepcontrol.wait would hold the
+    // whole warp, lane 0 included, until the previous kernel completes
     __syncwarp();
-    if (lane == 0) mbar_arrive(empty_bar(s));
-    if (warp == 0 && t + S < ntiles) {
-      // thread 0 refills this slot once all four warps have released it
-      bool w = true;
-      if (lane == 0) {
-        w = mbar_wait(empty_bar(s), (uint32_t)((t / S) & 1), 32);
-        if (w) issue(t + S);
+  } else {
+    const int cg = warp & 3, kh = warp >> 2;
+    float acc[JT][4][4];
+    // ldmatrix.trans lane addresses. B (Y, k = m, n = c): matrices (m 0-7 | 8-15) x (c 0-7 | 8-15).
+    // A (Z^T, rows j, k = m): matrices (j 0-7, m 0-7), (j 8-15, m 0-7), (j 0-7, m 8-15), (j 8-15, m 8-15).
+    const int mat = lane >> 3, rr = lane & 7;
+    const int yb_row = ((mat & 1) ? 8 : 0) + rr, yb_col = 32 * (cg & 1) + ((mat & 2) ? 8 : 0);
+    const int za_row = rr + ((mat & 2) ? 8 : 0), za_col = (mat & 1) ? 8 : 0;
+    const int g = lane >> 2, c = lane & 3;
+    uint32_t sync_par = 0;
+    auto consumer_sync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sync_bar);
+      const bool w = __all_sync(0xffffffffu, mbar_wait(sync_bar, sync_par, 34));
+      sync_par ^= 1u;
+      return w;
+    };
+    int pend_b = -1, pend_tok = 0;  // thread 0: the last unit's block and its count before this CTA's add
+    int it = 0;
+    while (true) {
+      const int s = it % S;
+      if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), (uint32_t)((it / S) & 1), 31))) {
+        ok = false;
+        break;
       }
-      if (!__shfl_sync(0xffffffffu, w ? 1 : 0, 0)) { ok = false; break; }
+      const int u = meta[2 * s], fl = meta[2 * s + 1];
+      if (u < 0) break;
+      if (fl & 1) {
+#pragma unroll
+        for (int jt = 0; jt < JT; ++jt)
+#pragma unroll
+          for (int n = 0; n < 4; ++n) acc[jt][n][0] = acc[jt][n][1] = acc[jt][n][2] = acc[jt][n][3] = 0.f;
+      }
+      const uint32_t st = base + (uint32_t)(s * SB);
+      const uint32_t ybox = st + (uint32_t)YB * (uint32_t)(cg >> 1);
+      const uint32_t zbox = st + 2u * (uint32_t)YB;
+      const int half = P.tr >> 1;
+#pragma unroll 2
+      for (int kk = 0; kk < half; kk += 16) {
+        const int k = half * kh + kk;
+        uint32_t bf[4][2];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t x0, x1, x2, x3;
+          ldsm_x4_t(sw128_addr(ybox, k + yb_row, yb_col + 16 * h2), x0, x1, x2, x3);
+          bf[2 * h2][0] = x0;
+          bf[2 * h2][1] = x1;
+          bf[2 * h2 + 1][0] = x2;
+          bf[2 * h2 + 1][1] = x3;
+        }
+#pragma unroll
+        for (int jt = 0; jt < JT; ++jt) {
+          const int ch = za_col + 16 * jt, cl = ch + P.RP;  // hi and lo columns of the split operand
+          uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
+          ldsm_x4_t(sw128_addr(zbox + (uint32_t)YB * (uint32_t)(ch >> 6), k + za_row, ch & 63), h0, h1, h2, h3);
+          ldsm_x4_t(sw128_addr(zbox + (uint32_t)YB * (uint32_t)(cl >> 6), k + za_row, cl & 63), l0, l1, l2, l3);
+#pragma unroll
+          for (int n = 0; n < 4; ++n) {
+            mma_16816(acc[jt][n], h0, h1, h2, h3, bf[n][0], bf[n][1]);
+            mma_16816(acc[jt][n], l0, l1, l2, l3, bf[n][0], bf[n][1]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty_bar(s));
+      ++it;
+      if (!(fl & 2)) continue;
+
+      // end of unit u: add the row halves, then the output or the partial
+      const int b = u / P.csu;
+      if (kh == 1) {
+#pragma unroll
+        for (int jt = 0; jt < JT; ++jt)
+#pragma unroll
+          for (int n = 0; n < 4; ++n) {
+            const int col = 32 * cg + 8 * n + 2 * c, j0 = 16 * jt + g;
+            *reinterpret_cast<float2*>(comb + j0 * kColCombStride + col) = make_float2(acc[jt][n][0], acc[jt][n][1]);
+            *reinterpret_cast<float2*>(comb + (j0 + 8) * kColCombStride + col) =
+                make_float2(acc[jt][n][2], acc[jt][n][3]);
+          }
+      }
+      if (!consumer_sync()) {
+        ok = false;
+        break;
+      }
+      if (kh == 0) {
+        const bool second = b >= P.nb0;
+        const ColredOut& O = second ? P.o1 : P.o0;
+        const int c0 = (second ? b - P.nb0 : b) * 128;
+        float* dst = P.part + (size_t)u * (16 * JT * 128);
+#pragma unroll
+        for (int jt = 0; jt < JT; ++jt)
+#pragma unroll
+          for (int n = 0; n < 4; ++n) {
+            const int col = 32 * cg + 8 * n + 2 * c, j0 = 16 * jt + g;
+            const float2 lo2 = *reinterpret_cast<const float2*>(comb + j0 * kColCombStride + col);
+            const float2 hi2 = *reinterpret_cast<const float2*>(comb + (j0 + 8) * kColCombStride + col);
+            const float v0 = acc[jt][n][0] + lo2.x, v1 = acc[jt][n][1] + lo2.y;
+            const float v2 = acc[jt][n][2] + hi2.x, v3 = acc[jt][n][3] + hi2.y;
+            if (P.csu == 1) {
+              colred_store(O, P.r, j0, c0 + col, v0);
+              colred_store(O, P.r, j0, c0 + col + 1, v1);
+              colred_store(O, P.r, j0 + 8, c0 + col, v2);
+              colred_store(O, P.r, j0 + 8, c0 + col + 1, v3);
+            } else {
+              *reinterpret_cast<float2*>(dst + j0 * 128 + col) = make_float2(v0, v1);
+              *reinterpret_cast<float2*>(dst + (j0 + 8) * 128 + col) = make_float2(v2, v3);
+            }
+          }
+        if (P.csu > 1) __threadfence();
+      }
+      if (P.csu > 1 && tid == 0) {
+        // the count taken at the previous unit's end has long arrived: was that the block's last chunk?
+        const int d = (pend_b >= 0 && pend_tok == P.csu - 1) ? pend_b : -1;
+        if (d >= 0) __threadfence();
+        *pend_smem = d;
+      }
+      if (!consumer_sync()) {
+        ok = false;
+        break;
+      }
+      if (P.csu > 1) {
+        const int d = *pend_smem;
+        if (tid == 0) {
+          __threadfence();
+          pend_b = b;
+          pend_tok = atomicAdd(P.ctr + 1 + b, 1);
+        }
+        if (d >= 0) colred_reduce_block<JT>(P, d, tid);
+      }
+    }
+    if (ok && P.csu > 1) {
+      if (tid == 0) {
+        const int d = (pend_b >= 0 && pend_tok == P.csu - 1) ? pend_b : -1;
+        if (d >= 0) __threadfence();
+        *pend_smem = d;
+      }
+      if (consumer_sync()) {
+        const int d = *pend_smem;
+        if (d >= 0) colred_reduce_block<JT>(P, d, tid);
+      }
     }
   }
   if (!ok || dev_aborted()) spin_ns(2000000ull);  // copies issued before a wait gave up land first
-  __syncthreads();  // the ring becomes the partial tile
-  {
-    const int g = lane >> 2, c = lane & 3;
-    const int wc = warp * 32;
-#pragma unroll
-    for (int jt = 0; jt < JT; ++jt)
-#pragma unroll
-      for (int n = 0; n < 4; ++n) {
-        const int col = wc + 8 * n + 2 * c;
-        const int j0 = 16 * jt + g;
-        part[j0][col] = acc[jt][n][0];
-        part[j0][col + 1] = acc[jt][n][1];
-        part[j0 + 8][col] = acc[jt][n][2];
-        part[j0 + 8][col + 1] = acc[jt][n][3];
-      }
-  }
-  cluster_sync_all();
-  // rank q reduces columns [q*128/CS, (q+1)*128/CS) over ranks in order
-  const int cols_per = (128 + CS - 1) / CS;
-  const int cl0 = (int)rank * cols_per;
-  for (int i = tid; i < cols_per * r; i += 128) {
-    const int cl = cl0 + i / r, j = i % r;
-    const int col = c0 + cl;
-    if (cl >= 128 || col >= P.C) continue;
-    const float v = cluster_sum_ordered(&part[j][cl], CS);
-    const long oi = P.transpose ? (long)j * P.C + col : (long)col * r + j;
-    P.out[oi] = P.scale * v;
-  }
-  cluster_sync_all();
+  if (P.defer_wait) pdl_wait();
 }
 
 // Grouped (routed) row products: one CTA per 128-row block of an expert segment (the grouped
@@ -779,8 +931,8 @@ __global__ void colred_reduce_kernel(const float* __restrict__ part, int Ccols, 
 // Ordered sum of the split-K partials of a dense GEMM: out[m][n] = sum_ks part[ks][m][n].
 __global__ void split_reduce_kernel(const float* __restrict__ part, int ksplit, long stride, long count,
                                     void* __restrict__ out, int out_dtype) {
-  pdl_launch_dependents();
   pdl_wait();
+  pdl_launch_dependents();
   for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; 4 * i < count; i += (long)gridDim.x * blockDim.x) {
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int ks = 0; ks < ksplit; ++ks) {

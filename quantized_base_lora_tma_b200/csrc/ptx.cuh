@@ -141,9 +141,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int sit
 }
 
 // ------------------------------------------------------------------------------------------------
-// Programmatic dependent launch. Kernels of the dense path let the next kernel in the stream start
-// its set-up early (launch_dependents) and wait for the previous kernel's completion and memory
-// (wait) before their first global-memory access; both are no-ops without a programmatic launch.
+// Programmatic dependent launch. Kernels of the dense path wait for the previous kernel's
+// completion and memory (wait) before their first global-memory access, and only then let the
+// next kernel in the stream start its set-up early (launch_dependents); both are no-ops without a
+// programmatic launch. Every kernel waits before it exits, so when a kernel starts, all kernels two
+// or more launches back have completed: a kernel whose inputs all come from there may defer its
+// own wait to its end and run beside the previous kernel.
 // ------------------------------------------------------------------------------------------------
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }

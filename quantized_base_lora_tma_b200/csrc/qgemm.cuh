@@ -299,7 +299,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  pdl_launch_dependents();
 
   const uint32_t sA = base_u32 + C::OFF_A;
   const uint32_t sB = base_u32 + C::OFF_B;
@@ -344,6 +343,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
   pdl_wait();  // inputs of the previous kernel in the stream are complete from here on
+  pdl_launch_dependents();  // after the wait: a dependent may rely on what this launch waited for
 
   const int kb_main = p.Kd / kBK;
   // k-block of step i of a tile: its quantized part first, then (if it carries them) the LoRA blocks

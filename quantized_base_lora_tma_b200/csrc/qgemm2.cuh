@@ -100,7 +100,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm2Threads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  pdl_launch_dependents();
   const uint32_t rank = cta_rank_in_cluster();  // 0 = leader
   const bool leader = rank == 0;
   const int cid = blockIdx.x >> 1;
@@ -150,6 +149,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm2Threads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
   pdl_wait();  // inputs of the previous kernel in the stream are complete from here on
+  pdl_launch_dependents();  // after the wait: a dependent may rely on what this launch waited for
 
   const int kb_main = p.Kd / kBK;
   auto tile_steps = [&](const TileInfo& ti) { return (ti.kb_hi - ti.kb_lo) + (ti.lora ? p.n_lora_kb : 0); };

@@ -97,6 +97,7 @@ static int group_bytes(int qtype) {
 static int64_t packed_row_bytes(int qtype, int64_t cols) { return cols / 256 * group_bytes(qtype); }
 
 static inline int lora_rp(int r) { return 32 * ((r + 31) / 32); }
+static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 static inline int launch_status() {
   return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
@@ -242,18 +243,18 @@ template <int NT>
 static cudaError_t launch_rows_nt(cudaLaunchConfig_t& cfg, const __nv_bfloat16* Y, long ldy, int M, int Kin,
                                   int kchunk, const __nv_bfloat16* Z, long zj, long zk, int r, float oscale,
                                   float lscale, float* out, __nv_bfloat16* la, int RP, BopArgs bop, __nv_bfloat16* LB,
-                                  int row_blocks, const float* hin, float hscale, __nv_bfloat16* hs) {
+                                  int row_blocks, const float* hin, float hscale, __nv_bfloat16* hs, int* zc, int zn) {
   auto k = lora_rows_cluster_kernel<NT>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cfg.dynamicSmemBytes);
   if (e != cudaSuccess) return e;
   return cudaLaunchKernelEx(&cfg, k, Y, ldy, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out, la, RP, bop, LB,
-                            row_blocks, hin, hscale, hs);
+                            row_blocks, hin, hscale, hs, zc, zn);
 }
 
 static int launch_rows_dense(const __nv_bfloat16* Y, long ldy, int M, int Kin, const __nv_bfloat16* Z, long zj,
                              long zk, int r, float oscale, float lscale, float* out, __nv_bfloat16* la, BopArgs bop,
                              __nv_bfloat16* LB, cudaStream_t st, const float* hin = nullptr, float hscale = 0.f,
-                             __nv_bfloat16* hs = nullptr) {
+                             __nv_bfloat16* hs = nullptr, int* zc = nullptr, int zn = 0) {
   if (M <= 0) return QL_OK;
   const int RP = lora_rp(r);
   // k range per cluster rank: a multiple of the 128-wide streamed tile
@@ -274,13 +275,13 @@ static int launch_rows_dense(const __nv_bfloat16* Y, long ldy, int M, int Kin, c
   cudaError_t e;
   if (NT == 2)
     e = launch_rows_nt<2>(cfg, Y, ldy, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out, la, RP, bop, LB, row_blocks,
-                          hin, hscale, hs);
+                          hin, hscale, hs, zc, zn);
   else if (NT == 4)
     e = launch_rows_nt<4>(cfg, Y, ldy, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out, la, RP, bop, LB, row_blocks,
-                          hin, hscale, hs);
+                          hin, hscale, hs, zc, zn);
   else
     e = launch_rows_nt<8>(cfg, Y, ldy, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out, la, RP, bop, LB, row_blocks,
-                          hin, hscale, hs);
+                          hin, hscale, hs, zc, zn);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -290,41 +291,75 @@ static int launch_rows_dense(const __nv_bfloat16* Y, long ldy, int M, int Kin, c
 }
 
 // Two dense column reductions in one launch (dB and dA of the backward): out_p = scale_p *
-// Y_p^T Z_p for Y_p [M x C_p] bf16 and the split operands Z_p [M x 2RP] bf16.
-template <int JT>
-static cudaError_t launch_colred_jt(cudaLaunchConfig_t& cfg, const CUtensorMap* tm, const ColredOut& o0,
-                                    const ColredOut& o1, int nb0, int M, int r, int RP, int mchunk) {
-  auto k = colred_cluster_kernel<JT>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cfg.dynamicSmemBytes);
-  if (e != cudaSuccess) return e;
-  return cudaLaunchKernelEx(&cfg, k, tm[0], tm[1], tm[2], tm[3], o0, o1, nb0, M, r, RP, mchunk);
+// Y_p^T Z_p for Y_p [M x C_p] bf16 and the split operands Z_p [M x 2RP] bf16. Tiles of 256 rows
+// (128 for r > 32, so that two stages still fit); rows go in chunks of at most 2048, so that a
+// launch at the bench shape has one unit per column block and no partials.
+struct ColredPlan {
+  int nb0, nblk, csu, mchunk, tr;
+};
+static ColredPlan plan_colred(int64_t M, int64_t C0, int64_t C1, int r) {
+  ColredPlan p;
+  p.nb0 = (int)((C0 + 127) / 128);
+  p.nblk = p.nb0 + (int)((C1 + 127) / 128);
+  p.tr = lora_rp(r) <= 32 ? 256 : 128;
+  const int csu = (int)std::max<int64_t>(1, std::min<int64_t>(8, (M + 2047) / 2048));
+  int mchunk = (int)((M + csu - 1) / csu);
+  mchunk = (mchunk + p.tr - 1) / p.tr * p.tr;
+  p.mchunk = mchunk;
+  p.csu = (int)((M + mchunk - 1) / mchunk);
+  return p;
+}
+// Counters and partials of the column reduction, for the workspace.
+static size_t colred_ctr_bytes(const ColredPlan& p) { return (size_t)(1 + p.nblk) * 4; }
+static size_t colred_ws_bytes(const ColredPlan& p, int r) {
+  const int JT = (r + 15) / 16;
+  return al256(colred_ctr_bytes(p)) + (p.csu > 1 ? (size_t)p.nblk * p.csu * JT * 16 * 128 * 4 : 0);
 }
 
+template <int JT>
+static cudaError_t launch_colred_jt(cudaLaunchConfig_t& cfg, const CUtensorMap* tm, const ColredFlow& P) {
+  auto k = colred_flow_kernel<JT>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cfg.dynamicSmemBytes);
+  if (e != cudaSuccess) return e;
+  return cudaLaunchKernelEx(&cfg, k, tm[0], tm[1], tm[2], tm[3], P);
+}
+
+// crws: the plan's workspace (counters zeroed by an earlier kernel of the same stream, then
+// partials). defer_wait: the previous kernel in the stream waited for this launch's inputs itself.
 static int launch_colred_dense(const __nv_bfloat16* Y0, int C0, const __nv_bfloat16* Z0, const ColredOut& o0,
                                const __nv_bfloat16* Y1, int C1, const __nv_bfloat16* Z1, const ColredOut& o1, int M, int r,
-                               cudaStream_t st) {
+                               uint8_t* crws, int defer_wait, cudaStream_t st) {
   const int RP = lora_rp(r);
-  CUtensorMap tm[4];
-  if (!tmap_bf16_rows(&tm[0], Y0, C0, M, 64) || !tmap_bf16_rows(&tm[1], Y1, C1, M, 64) ||
-      !tmap_bf16_rows(&tm[2], Z0, 2 * RP, M, 64) || !tmap_bf16_rows(&tm[3], Z1, 2 * RP, M, 64))
-    return QL_ERR_CUDA;
-  const int nb0 = (C0 + 127) / 128, nb1 = (C1 + 127) / 128;
-  // row slices per column block: as many as keep every CTA resident in one wave
-  const size_t smem = colred_smem_bytes(RP);
-  const int per_sm = std::max(1, (int)(233472 / (smem + 1024)));
-  const int CS_max = std::max(1, std::min(8, per_sm * num_sms() / (nb0 + nb1)));
-  int CS = std::max(1, std::min(CS_max, (M + 63) / 64));
-  int mchunk = (M + CS - 1) / CS;
-  mchunk = (mchunk + 63) / 64 * 64;
-  CS = (M + mchunk - 1) / mchunk;
-  PdlLaunch L(dim3(nb0 + nb1, CS, 1), dim3(128), smem, st, CS);
-  cudaLaunchConfig_t& cfg = L.cfg;
   const int JT = (r + 15) / 16;
+  CUtensorMap tm[4];
+  const ColredPlan pl = plan_colred(M, C0, C1, r);
+  if (!tmap_bf16_rows(&tm[0], Y0, C0, M, pl.tr) || !tmap_bf16_rows(&tm[1], Y1, C1, M, pl.tr) ||
+      !tmap_bf16_rows(&tm[2], Z0, 2 * RP, M, pl.tr) || !tmap_bf16_rows(&tm[3], Z1, 2 * RP, M, pl.tr))
+    return QL_ERR_CUDA;
+  ColredFlow P;
+  P.o0 = o0;
+  P.o1 = o1;
+  P.nb0 = pl.nb0;
+  P.nblk = pl.nblk;
+  P.M = M;
+  P.r = r;
+  P.RP = RP;
+  P.mchunk = pl.mchunk;
+  P.tr = pl.tr;
+  P.csu = pl.csu;
+  P.defer_wait = defer_wait;
+  P.ctr = reinterpret_cast<int*>(crws);
+  P.part = reinterpret_cast<float*>(crws + al256(colred_ctr_bytes(pl)));
+  const size_t smem = colred_smem_bytes(RP, JT, pl.tr);
+  const int per_sm = std::max(1, (int)(233472 / (smem + 1024)));
+  const int grid = std::min(pl.nblk * pl.csu, per_sm * num_sms());
+  PdlLaunch L(dim3(grid), dim3(32 * kColWarps), smem, st);
+  cudaLaunchConfig_t& cfg = L.cfg;
   cudaError_t e;
-  if (JT == 1) e = launch_colred_jt<1>(cfg, tm, o0, o1, nb0, M, r, RP, mchunk);
-  else if (JT == 2) e = launch_colred_jt<2>(cfg, tm, o0, o1, nb0, M, r, RP, mchunk);
-  else if (JT == 3) e = launch_colred_jt<3>(cfg, tm, o0, o1, nb0, M, r, RP, mchunk);
-  else e = launch_colred_jt<4>(cfg, tm, o0, o1, nb0, M, r, RP, mchunk);
+  if (JT == 1) e = launch_colred_jt<1>(cfg, tm, P);
+  else if (JT == 2) e = launch_colred_jt<2>(cfg, tm, P);
+  else if (JT == 3) e = launch_colred_jt<3>(cfg, tm, P);
+  else e = launch_colred_jt<4>(cfg, tm, P);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -333,7 +368,6 @@ static int launch_colred_dense(const __nv_bfloat16* Y0, int C0, const __nv_bfloa
   return launch_status();
 }
 
-// out = scale * sum over slices of Y[m, c] Z[m, j]
 static int launch_colred(const __nv_bfloat16* Y, long ldy, int Ccols, const float* Z, int r, int M, const float* zw,
                          const int* seg_off, const int* mblk_off, int E, int max_slices, float* part, float scale,
                          int transpose, float* out, cudaStream_t st, const __nv_bfloat16* Ylo = nullptr) {
@@ -498,9 +532,8 @@ static int launch_gemv_fwd(int qtype, const void* wq, int64_t N, int64_t K, cons
 
 // Workspace layout of the dense layer (byte offsets, 256-aligned).
 struct LinearWs {
-  size_t la, lb, hs, split, total;
+  size_t la, lb, hs, split, cr, total;
 };
-static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 static LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int r) {
   LinearWs w;
   const int KL = 2 * lora_rp(r);
@@ -512,6 +545,7 @@ static LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int r) {
   const size_t sf = split_bytes(plan_dense(M, N, K, false, true), M, N);
   const size_t sb = split_bytes(plan_dense(M, K, N, true, true), M, K);
   w.split = o; o = al256(o + std::max(sf, sb));
+  w.cr = o; o = al256(o + colred_ws_bytes(plan_colred(M, N, K, r), r));
   w.total = o;
   return w;
 }
@@ -982,22 +1016,26 @@ int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void
   const int KL = 2 * lora_rp(r);
 
   __nv_bfloat16* HS = (__nv_bfloat16*)(wsb + w.hs);
-  // LA = split(G) with G = s dY B, HS = split(s H), and LB[k] = [A^T(k) | A^T(k)]
+  uint8_t* crws = wsb + w.cr;
+  const int ncr = (int)(colred_ctr_bytes(plan_colred(M, N, K, r)) / 4);
+  // LA = split(G) with G = s dY B, HS = split(s H), and LB[k] = [A^T(k) | A^T(k)]; the column
+  // reduction's counters are zeroed on the way
   rc = launch_rows_dense((const __nv_bfloat16*)dY, N, (int)M, (int)N, (const __nv_bfloat16*)B, 1, r, r, scale, scale,
                          nullptr,
                          LA, dX ? BopArgs{(const __nv_bfloat16*)A, 1, K, (int)K} : BopArgs{nullptr, 0, 0, 0}, LB, st, H,
-                         scale, HS);
+                         scale, HS, (int*)crws, ncr);
   if (rc) return rc;
   if (dX) {
     rc = launch_dense_gemm<true>(qtype, dY, M, N, wq, N, K, LA, LB, KL, K, dX, dx_dtype,
                                  (float*)(wsb + w.split), true, st, 1);
     if (rc) return rc;
   }
-  // dB = dY^T split(s H) and dA = split(G)^T X in one launch
+  // dB = dY^T split(s H) and dA = split(G)^T X in one launch; after the dX GEMM (which waited for
+  // the row kernel) it runs beside the GEMM on the SMs the GEMM leaves idle
   const ColredOut ob{(int)N, 1.0f, 0, dB};
   const ColredOut oa{(int)K, 1.0f, 1, dA};
   return launch_colred_dense((const __nv_bfloat16*)dY, (int)N, HS, ob, (const __nv_bfloat16*)X, (int)K, LA, oa, (int)M,
-                             r, st);
+                             r, crws, dX ? 1 : 0, st);
 }
 
 }  // extern "C"

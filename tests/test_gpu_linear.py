@@ -95,6 +95,8 @@ SMALL = [
     (1100, 4096, 512, 8),  # the same for the input-gradient GEMM
     (9, 1280, 192, 16),    # decode path: two token tiles, two adapter tiles, K steps not a multiple of the split
     (13, 768, 64, 12),     # decode path: one row block, ragged rank
+    (4500, 256, 320, 8),   # adapter gradients from three row chunks (partials summed in chunk order)
+    (2600, 256, 192, 40),  # the same with r > 32 (128-row tiles)
 ]
 
 
@@ -127,6 +129,18 @@ def test_linear_b_zero_gives_exact_zero_dA():
     Yr, Hr, dXr, dAr, dBr = oracle_linear(c)
     assert_close(f64(Y), Yr, "Y")
     assert_close(f64(dB), dBr, "dB")
+
+
+@pytest.mark.parametrize("shape", [(300, 512, 384, 4), (2600, 256, 192, 40)])
+def test_linear_bwd_without_dx(shape):
+    """Without dX the adapter gradients follow the row kernel directly: the same values, bit for bit."""
+    M, K, N, r = shape
+    c = inp.linear_case(M, K, N, inp.Q8_0, r, 2.0 * r, seed=M + r)
+    a = [t.clone() for t in run_linear(c)]
+    b = run_linear(c, with_dx=False)
+    assert b[2] is None
+    for i in (0, 1, 3, 4):
+        assert torch.equal(a[i], b[i])
 
 
 def test_linear_deterministic():
