@@ -86,8 +86,13 @@ def _p(t):
     return _c_vp(t.data_ptr())
 
 
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _s(stream):
     if stream is None:
+        if _raw_stream is not None:  # the current stream's handle without building a Stream object
+            return _c_vp(_raw_stream(torch.cuda.current_device()))
         stream = torch.cuda.current_stream()
     return _c_vp(stream.cuda_stream)
 

@@ -1,26 +1,31 @@
 // Small-M forward of the layer (M <= 16 tokens, decode-shaped): Y = X deq(W)^T + s (X A^T) B^T and
-// H = X A^T, in one launch. This is the weight-streaming regime of the layer ("MMQ" for a few
-// tokens, Show HN: LoRA over GGUF, "Things involved in the training"): every packed weight byte is
-// read once and each weight is used M times, so the kernel is built to keep HBM busy rather than
-// the tensor cores:
+// H = X A^T. This is the weight-streaming regime of the layer ("MMQ" for a few tokens, Show HN:
+// LoRA over GGUF, "Things involved in the training"): every packed weight byte is read once and
+// each weight is used M times, so the kernels are built to keep HBM busy with as few instructions
+// per weight as the decode allows. Three launches:
 //
-//   * A CTA owns 64 rows of W and a K slice; the KS CTAs of a cluster share the row block and split
-//     K. One producer thread streams, per 256-wide K step, the 64 packed groups of the rows and the
-//     X tile (tokens padded to 8 or 16 rows by the copy's zero fill) into a shared-memory ring by
-//     TMA (no multicast).
-//   * Eight warps share the 64 rows: two per 16-row set, each taking half of the eight 32-weight
-//     blocks of a K step. A thread decodes its two rows' 8-weight runs straight into the A
-//     fragments of mma.sync (bf16 in, fp32 accumulate; B = the X tile): the Q4_0 / Q8_0 block's
-//     integers q - 8 / q are exact in bf16, so each 32-weight block is one exact integer-by-X
-//     product pair of MMAs, scaled by the block's fp16 scale d in fp32 afterwards. The dequantized
-//     weight never exists in any memory.
-//   * The same warps accumulate H = X A^T over the slice on the tensor cores (two of the sixteen
-//     k16 steps of a K step each); a ninth warp only issues the copies.
-//   * Partials of the K slices (and of H) are summed through distributed shared memory in rank
-//     order (deterministic); the adapter term s H B^T is added in fp32 in the same epilogue.
+//   * gemv_h_kernel: H in one CTA. The weight stream does not need it and runs beside it.
+//   * qgemv_fwd_kernel: persistent, two CTAs per SM, each a balanced range of steps (ROWS rows of W
+//     x 256 k) that may span the end of one row block and the start of the next (stream-K). One
+//     producer thread streams the packed groups and the X tile (tokens padded to 8 or 16 rows by
+//     the copy's zero fill) into a shared-memory ring by TMA (no multicast), each stage tagged with
+//     its row block. Warp w takes the block pair w % 4 of every step (two 32-weight blocks, 4-byte
+//     aligned) for half of the rows; it builds the X fragments of its two blocks once per step and
+//     reuses them for all its row tiles, and decodes its rows' bytes straight into the A
+//     fragments of mma.sync (bf16 in, fp32 accumulate). The k order inside a block is free (X
+//     follows it), so a bf16 pair costs one shift and one LOP3:
+//       Q4_0: a 32-bit word of qs holds bytes 4c .. 4c + 3; (w >> 8s) & 0x000F000F | 0x43004300
+//       puts two nibbles n into two bf16 lanes reading 128 + n, exactly. The offset (136 per
+//       weight, i.e. 128 + 8) is removed through the accumulator input of the block's first MMA:
+//       -136 times the block's sum of X, itself an MMA of the X fragments with a constant -136.
+//       Q8_0: q via the 2^23 magic float, exact, then to bf16.
+//     Each 32-weight block's exact integer-by-X sum is scaled by its fp16 scale d in fp32. At the
+//     end of a row block's piece the four block pairs' partials are summed in order into the
+//     piece's slot in global memory.
+//   * gemv_finish_kernel: per 32 rows, the row block's slots in order plus s H B^T (fp32).
 //
-// Numerics: sum over blocks of d * (sum_k (q - 8) x) with fp32 accumulation, i.e. the exact decode
-// d (q - 8) is applied without an intermediate bf16 rounding of the weight.
+// Numerics: sum over blocks of d * (sum_k (q - 8) x) (Q4_0) or d * (sum_k q x) (Q8_0), fp32
+// accumulation in a fixed order; the decoded weight is never rounded.
 #pragma once
 #include <cuda_bf16.h>
 
@@ -30,40 +35,52 @@
 
 namespace qlora {
 
-constexpr int kGvRows = 64;                    // W rows per CTA
-constexpr int kGvWarps = 9;                    // 8 compute warps + producer / adapter warp
-constexpr int kGvWarpA = 8;                    // the producer / adapter warp
+constexpr int kGvCompute = 8;     // compute warps
+constexpr int kGvWarpP = 8;       // the producer warp
+constexpr int kGvWarpL = 9;       // the warp that releases the next launch
+constexpr int kGvWarps = 10;
 constexpr int kGvThreads = kGvWarps * 32;
-constexpr int kGvMaxRank = 16;                 // adapter ranks this path takes (RN = 8 or 16)
+constexpr int kGvMaxRank = 16;    // adapter ranks this path takes
 
 template <int QT, int MT>
 struct GvCfg {
-  static constexpr int GB = QTraits<QT>::kGroupBytes;
-  static constexpr int W_BYTES = kGvRows * GB;        // 64 packed groups
-  static constexpr int XR = 8 * MT;                   // token rows of the X tile
-  static constexpr int X_BOX = XR * 128;              // one 64-wide k box
+  static constexpr int ROWS = QT == QL_Q4_0 ? 128 : 64;  // W rows per K step
+  static constexpr int RT = ROWS / 32;                    // row tiles (16 rows) per warp
+  static constexpr int GB = QTraits<QT>::kGroupBytes;     // bytes per 256 weights of a row
+  static constexpr int PB = GB / 4;                       // bytes per block pair
+  static constexpr int W_BYTES = ROWS * GB;
+  static constexpr int XR = 8 * MT;                       // token rows of the X tile
+  static constexpr int X_BOX = XR * 128;                  // one 64-wide k box
   static constexpr int X_BYTES = 4 * X_BOX;
   static constexpr int STAGE = W_BYTES + X_BYTES;
-  static constexpr int STAGES = 3;
-  static constexpr int OFF_PART = STAGES * STAGE;                 // [2][64][16] fp32 partial outputs
-  static constexpr int OFF_HP = OFF_PART + 2 * kGvRows * 16 * 4;  // [9][16][16] fp32: 8 warps' H, their sum
-  static constexpr int OFF_HF = OFF_HP + 9 * 16 * 16 * 4;         // [16][16] fp32 summed H
-  static constexpr int OFF_BAR = OFF_HF + 16 * 16 * 4;
-  static constexpr int SMEM_BYTES = OFF_BAR + 2 * STAGES * 8 + 1024;  // + alignment slack
+  static constexpr int STAGES = MT == 2 ? 3 : 4;
+  static constexpr int OFF_PART = STAGES * STAGE;         // [4 pairs][XR tokens][ROWS] fp32
+  static constexpr int OFF_META = OFF_PART + 4 * XR * ROWS * 4;  // per stage: row block, piece flags
+  static constexpr int OFF_BAR = OFF_META + 2 * 4 * STAGES + 16;
+  static constexpr int SMEM_BYTES = OFF_BAR + (2 * STAGES + 1) * 8 + 1024;  // + alignment slack
   static_assert(W_BYTES % 1024 == 0 && X_BOX % 1024 == 0, "128-byte-swizzled boxes need 1 KB alignment");
-  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(SMEM_BYTES <= 116 * 1024, "two CTAs per SM");
 };
 
+// Work of the weight-streaming kernel: T = NRB * KSTEPS steps (ROWS rows x 256 k each), step
+// t = row block * KSTEPS + K step; CTA i of G takes steps [i T / G, (i + 1) T / G). The part of a
+// row block inside one CTA's range is a piece; its fp32 partial goes to slot (CTA - first CTA of
+// the row block), and gemv_finish_kernel sums a row block's slots in order.
 struct GvParams {
   int N, K, M, r;
-  int kgroups;     // 256-wide K steps per cluster rank
-  float scale;
-  const __nv_bfloat16* A;  // [r x K]
-  const __nv_bfloat16* B;  // [N x r]
-  void* Y;                 // [M x N]
-  int y_dtype;
-  float* H;                // [M x r]
+  uint32_t nib_mask, bf16_magic;  // 0x000F000F, 0x43004300 (registers for the Q4_0 decode)
+  int ksteps, T, maxslots;
+  float* gpart;            // [NRB][maxslots][XR][ROWS] piece partials
 };
+
+// First step of CTA i's range, and the CTA whose range holds step s.
+__host__ __device__ __forceinline__ long gv_start(int i, int T, int G) { return (long)i * T / G; }
+__host__ __device__ __forceinline__ int gv_cta_of(long s, int T, int G) {
+  int i = (int)(s * G / T);
+  while (i + 1 < G && gv_start(i + 1, T, G) <= s) ++i;
+  while (i > 0 && gv_start(i, T, G) > s) --i;
+  return i;
+}
 
 // mma.sync m16n8k16 with a zero accumulator input.
 __device__ __forceinline__ void mma_16816_z(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -75,127 +92,141 @@ __device__ __forceinline__ void mma_16816_z(float (&d)[4], uint32_t a0, uint32_t
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
 }
 
-// 8 bytes at p (2-byte aligned; MIS = p % 4 known at compile time) as two words.
-template <int MIS>
-__device__ __forceinline__ void lds8(const uint8_t* p, uint32_t& x0, uint32_t& x1) {
-  if (MIS == 0) {
-    const uint2 v = *reinterpret_cast<const uint2*>(p);  // 8-byte aligned here (see callers)
-    x0 = v.x;
-    x1 = v.y;
-  } else {
-    const uint32_t* w = reinterpret_cast<const uint32_t*>(p - 2);
-    const uint32_t w0 = w[0], w1 = w[1], w2 = w[2];
-    x0 = __funnelshift_r(w0, w1, 16);
-    x1 = __funnelshift_r(w1, w2, 16);
-  }
+// mma.sync m16n8k16 with a separate accumulator input.
+__device__ __forceinline__ void mma_16816_c(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                            uint32_t b0, uint32_t b1, const float (&c)[4]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%11,%12,%13};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]), "f"(c[2]), "f"(c[3]));
 }
 
-// Low-nibble pair -> exact bf16 pair: the bytes picked by sel land in the low and high halves;
-// with the bf16 exponent of 128 OR-ed in, a nibble n reads 128 + n (bf16 has 7 mantissa bits, so
-// only a low nibble can be placed this way), and one subtraction of 136 gives n - 8 exactly.
-__device__ __forceinline__ uint32_t nib2_bf16(uint32_t x, uint32_t sel) {
-  const uint32_t t = __byte_perm(x, 0u, sel);
-  return bf16x2_sub((t & 0x000F000Fu) | 0x43004300u, 0x43084308u /* bf16 (136, 136) */);
+// Element k of token row `row` of a 128-byte-swizzled box of 64 k (row pitch 128 bytes).
+__device__ __forceinline__ const uint8_t* gv_x_at(const uint8_t* box, int row, int k) {
+  return box + row * 128 + ((((k >> 3) ^ (row & 7))) << 4) + (k & 7) * 2;
 }
 
-// Integers of weights [8c, 8c + 8) of block `blk` of a packed 256-weight group at g, as four bf16
-// pairs (consecutive k), and the block's scale. Q4_0: q - 8; Q8_0: q.
-template <int QT, int BLK>
-__device__ __forceinline__ void gv_decode(const uint8_t* g, int c, uint32_t (&a)[4], float& d);
+// (a & b) | c in one LOP3. The masks come in as registers (kernel parameters): with both as
+// immediates the compiler would split the operation in two.
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
 
-template <int QT, int BLK>
-__device__ __forceinline__ void gv_decode(const uint8_t* g, int c, uint32_t (&a)[4], float& d) {
+// Q4_0: w holds qs bytes 4c .. 4c + 3 of a block (low nibbles: weights 4c .. 4c + 3, high nibbles:
+// 16 + 4c ..). p[0] = (4c, 4c + 2), p[1] = (4c + 1, 4c + 3), p[2] = (16 + 4c, 16 + 4c + 2),
+// p[3] = (16 + 4c + 1, 16 + 4c + 3), each lane the bf16 128 + n (nm = 0x000F000F,
+// mg = 0x43004300).
+__device__ __forceinline__ void gv_q4_pairs(uint32_t w, uint32_t nm, uint32_t mg, uint32_t (&p)[4]) {
+  p[0] = and_or(w, nm, mg);
+  p[1] = and_or(w >> 8, nm, mg);
+  p[2] = and_or(w >> 4, nm, mg);
+  p[3] = and_or(w >> 12, nm, mg);
+}
+
+// Q8_0: w holds 4 int8 weights (k, k + 1, k + 2, k + 3) -> bf16 pairs (k, k + 1), (k + 2, k + 3).
+__device__ __forceinline__ void gv_q8_pairs(uint32_t w, uint32_t& p01, uint32_t& p23) {
+  float f[4];
+  magic4(w ^ 0x80808080u, f);
+  const float2 bias = make_float2(-8388736.0f, -8388736.0f);  // -(2^23 + 128)
+  const float2 a = __fadd2_rn(make_float2(f[0], f[1]), bias);
+  const float2 b = __fadd2_rn(make_float2(f[2], f[3]), bias);
+  p01 = bf16x2_bits(a.x, a.y);
+  p23 = bf16x2_bits(b.x, b.y);
+}
+
+__device__ __forceinline__ float half_lo(uint32_t w) { return __low2float(*reinterpret_cast<const __half2*>(&w)); }
+__device__ __forceinline__ float half_hi(uint32_t w) { return __high2float(*reinterpret_cast<const __half2*>(&w)); }
+
+// One row's registers for the block pair at rb (4-byte aligned; rbc = rb + 4c): fr[blk] = the
+// A-fragment words of the block's two MMAs in order (MMA0 k slots 2c.., 2c+8..; MMA1 the same), and
+// the blocks' scales.
+template <int QT>
+__device__ __forceinline__ void gv_row_pair(const uint8_t* rb, const uint8_t* rbc, uint32_t nm, uint32_t mg,
+                                            uint32_t (&fr)[2][4], float (&d)[2]) {
+  const uint32_t* W = reinterpret_cast<const uint32_t*>(rb);
+  const uint32_t* Wc = reinterpret_cast<const uint32_t*>(rbc);
   if (QT == QL_Q4_0) {
-    // block: fp16 d, 16 bytes; byte j = weight j (low nibble) and j + 16 (high nibble).
-    // weights [8c, 8c + 8): bytes 8 (c & 1) .. + 8, nibble c >> 1. Block start 18 BLK: the bytes
-    // start at 18 BLK + 2 + 8 (c & 1), which is 4-aligned for odd BLK (the group is 16-aligned).
-    const uint8_t* b = g + 18 * BLK;
-    d = __half2float(*reinterpret_cast<const __half*>(b));
-    uint32_t x0, x1;
-    const uint8_t* p = b + 2 + 8 * (c & 1);
-    if (BLK & 1) {
-      x0 = *reinterpret_cast<const uint32_t*>(p);
-      x1 = *reinterpret_cast<const uint32_t*>(p + 4);
-    } else {
-      lds8<2>(p, x0, x1);
-    }
-    // lanes taking high nibbles shift them down first (a per-lane amount: no divergence)
-    const uint32_t sh = (uint32_t)(c >> 1) * 4u;
-    x0 >>= sh;
-    x1 >>= sh;
-    a[0] = nib2_bf16(x0, 0x4140u);
-    a[1] = nib2_bf16(x0, 0x4342u);
-    a[2] = nib2_bf16(x1, 0x4140u);
-    a[3] = nib2_bf16(x1, 0x4342u);
+    // block A: fp16 d at 0, qs at 2 .. 17; block B: d at 18, qs at 20 .. 35
+    d[0] = half_lo(W[0]);
+    d[1] = half_hi(W[4]);
+    gv_q4_pairs(__funnelshift_r(Wc[0], Wc[1], 16), nm, mg, fr[0]);
+    gv_q4_pairs(Wc[5], nm, mg, fr[1]);
   } else {
-    // Q8_0 block: fp16 d, 32 int8; weights [8c, 8c + 8) are bytes 2 + 8c .. + 8 (4-aligned for
-    // odd BLK). int8 -> exact fp32 by the 2^23 magic (q + 128 biased byte), then to bf16.
-    const uint8_t* b = g + 34 * BLK;
-    d = __half2float(*reinterpret_cast<const __half*>(b));
-    uint32_t x0, x1;
-    const uint8_t* p = b + 2 + 8 * c;
-    if (BLK & 1) {
-      x0 = *reinterpret_cast<const uint32_t*>(p);
-      x1 = *reinterpret_cast<const uint32_t*>(p + 4);
-    } else {
-      lds8<2>(p, x0, x1);
-    }
-    const float2 bias = make_float2(-8388736.0f, -8388736.0f);  // -(2^23 + 128)
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint32_t x = (h ? x1 : x0) ^ 0x80808080u;
-      float f[4];
-      magic4(x, f);
-      const float2 p0 = __fadd2_rn(make_float2(f[0], f[1]), bias);
-      const float2 p1 = __fadd2_rn(make_float2(f[2], f[3]), bias);
-      a[2 * h] = bf16x2_bits(p0.x, p0.y);
-      a[2 * h + 1] = bf16x2_bits(p1.x, p1.y);
-    }
+    // block A: d at 0, qs at 2 .. 33; block B: d at 34, qs at 36 .. 67
+    d[0] = half_lo(W[0]);
+    d[1] = half_hi(W[8]);
+    gv_q8_pairs(__funnelshift_r(Wc[0], Wc[1], 16), fr[0][0], fr[0][1]);  // weights 4c .. 4c + 3
+    gv_q8_pairs(__funnelshift_r(Wc[4], Wc[5], 16), fr[0][2], fr[0][3]);  // 16 + 4c ..
+    gv_q8_pairs(Wc[9], fr[1][0], fr[1][1]);
+    gv_q8_pairs(Wc[13], fr[1][2], fr[1][3]);
   }
 }
 
-// X or adapter-A element pair (row, k, k + 1) of a 128-byte-swizzled box of 64 k (row pitch 128 B).
-__device__ __forceinline__ uint32_t sw128_pair(const uint8_t* box, int row, int kk) {
-  return *reinterpret_cast<const uint32_t*>(box + row * 128 + ((((kk >> 3) ^ (row & 7))) << 4) + (kk & 7) * 2);
-}
-__device__ __forceinline__ uint4 sw128_chunk(const uint8_t* box, int row, int chunk) {
-  return *reinterpret_cast<const uint4*>(box + row * 128 + ((chunk ^ (row & 7)) << 4));
-}
-
-// One 256-wide K step of rows g0 and g1 (= g0 + 8 rows): eight 32-weight blocks, each two exact
-// integer MMAs per token tile and one fp32 scale-accumulate per output.
-template <int QT, int MT, int BLK>
-__device__ __forceinline__ void gv_block(const uint8_t* g0, const uint8_t* g1, const uint8_t* xs, int c, int g,
-                                         float (&acc)[MT][4]) {
-  uint32_t a[4], b[4];
-  float d0, d1;
-  gv_decode<QT, BLK>(g0, c, a, d0);
-  gv_decode<QT, BLK>(g1, c, b, d1);
-  const uint8_t* xb = xs + (BLK >> 1) * GvCfg<QT, MT>::X_BOX;
+// H = X A^T for m < M <= 16, j < r <= 16, in one CTA: warp w takes the k16 steps w, w + 32, .. (mma.sync,
+// A = X rows, B = adapter rows; four steps' loads in flight at a time) and the 32 warps' sums are
+// added in order. Writes hf [16][16] (zero past M and r) for the finish kernel and H [M x r].
+// It runs beside the weight stream.
+constexpr int kGvHWarps = 32;
+__global__ void __launch_bounds__(kGvHWarps * 32) gemv_h_kernel(const __nv_bfloat16* __restrict__ X,
+                                                                const __nv_bfloat16* __restrict__ A, int M, int K,
+                                                                int r, float* __restrict__ hf, float* __restrict__ H) {
+  __shared__ float red[kGvHWarps][256];
+  pdl_wait();
+  pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+  float acc[2][4];
 #pragma unroll
-  for (int t = 0; t < MT; ++t) {
-    const uint4 xv = sw128_chunk(xb, 8 * t + g, 4 * (BLK & 1) + c);
-    float dblk[4];
-    mma_16816_z(dblk, a[0], b[0], a[1], b[1], xv.x, xv.y);
-    mma_16816(dblk, a[2], b[2], a[3], b[3], xv.z, xv.w);
-    acc[t][0] = fmaf(d0, dblk[0], acc[t][0]);
-    acc[t][1] = fmaf(d0, dblk[1], acc[t][1]);
-    acc[t][2] = fmaf(d1, dblk[2], acc[t][2]);
-    acc[t][3] = fmaf(d1, dblk[3], acc[t][3]);
+  for (int jt = 0; jt < 2; ++jt) acc[jt][0] = acc[jt][1] = acc[jt][2] = acc[jt][3] = 0.f;
+  auto ld = [&](const __nv_bfloat16* p, int row, int rows, int k) -> uint32_t {
+    return row < rows ? __ldg(reinterpret_cast<const unsigned int*>(p + (long)row * K + k)) : 0u;
+  };
+  constexpr int U = 4;
+  for (int k0 = 16 * warp; k0 < K; k0 += 16 * kGvHWarps * U) {
+    uint32_t a[U][4], b[U][2][2];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int k = k0 + 16 * kGvHWarps * u;
+      const bool in = k < K;
+      a[u][0] = in ? ld(X, g, M, k + 2 * c) : 0u;
+      a[u][1] = in ? ld(X, g + 8, M, k + 2 * c) : 0u;
+      a[u][2] = in ? ld(X, g, M, k + 2 * c + 8) : 0u;
+      a[u][3] = in ? ld(X, g + 8, M, k + 2 * c + 8) : 0u;
+#pragma unroll
+      for (int jt = 0; jt < 2; ++jt) {
+        b[u][jt][0] = in ? ld(A, 8 * jt + g, r, k + 2 * c) : 0u;
+        b[u][jt][1] = in ? ld(A, 8 * jt + g, r, k + 2 * c + 8) : 0u;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int jt = 0; jt < 2; ++jt) mma_16816(acc[jt], a[u][0], a[u][1], a[u][2], a[u][3], b[u][jt][0], b[u][jt][1]);
+  }
+  // acc[jt]: (m = g, j = 8 jt + 2c, + 1) and (m = g + 8, same j)
+#pragma unroll
+  for (int jt = 0; jt < 2; ++jt) {
+    const int j = 8 * jt + 2 * c;
+    red[warp][g * 16 + j] = acc[jt][0];
+    red[warp][g * 16 + j + 1] = acc[jt][1];
+    red[warp][(g + 8) * 16 + j] = acc[jt][2];
+    red[warp][(g + 8) * 16 + j + 1] = acc[jt][3];
+  }
+  __syncthreads();
+  if (threadIdx.x < 256) {
+    float v = 0.f;
+    for (int w = 0; w < kGvHWarps; ++w) v += red[w][threadIdx.x];
+    hf[threadIdx.x] = v;
+    const int m = threadIdx.x >> 4, j = threadIdx.x & 15;
+    if (H != nullptr && m < M && j < r) H[m * r + j] = v;
   }
 }
-// Blocks [4 HALF, 4 HALF + 4) of a K step (two warps share a row set, one half each).
-template <int QT, int MT, int HALF>
-__device__ __forceinline__ void gv_block_half(const uint8_t* g0, const uint8_t* g1, const uint8_t* xs, int c, int g,
-                                              float (&acc)[MT][4]) {
-  gv_block<QT, MT, 4 * HALF + 0>(g0, g1, xs, c, g, acc);
-  gv_block<QT, MT, 4 * HALF + 1>(g0, g1, xs, c, g, acc);
-  gv_block<QT, MT, 4 * HALF + 2>(g0, g1, xs, c, g, acc);
-  gv_block<QT, MT, 4 * HALF + 3>(g0, g1, xs, c, g, acc);
-}
 
+// The weight-streaming kernel (stream-K over row blocks x K steps; see GvParams).
 template <int QT, int MT>
-__global__ void __launch_bounds__(kGvThreads) qgemv_fwd_kernel(const __grid_constant__ CUtensorMap tmW,
+__global__ void __launch_bounds__(kGvThreads, 2) qgemv_fwd_kernel(const __grid_constant__ CUtensorMap tmW,
                                                                const __grid_constant__ CUtensorMap tmX,
                                                                const GvParams p) {
   using C = GvCfg<QT, MT>;
@@ -204,156 +235,203 @@ __global__ void __launch_bounds__(kGvThreads) qgemv_fwd_kernel(const __grid_cons
   uint8_t* smem = gv_smem_raw + (base_u32 - smem_u32(gv_smem_raw));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
-  const uint32_t rank = cluster_ctarank();
-  const int KS = gridDim.y;
-  const int n0 = blockIdx.x * kGvRows;
-  const int kg0 = (int)rank * p.kgroups;                        // first 256-wide K step of the slice
-  const int nst = max(0, min(p.kgroups, p.K / 256 - kg0));      // steps of this slice
+  const int G = gridDim.x;
+  const long s0 = gv_start(blockIdx.x, p.T, G), s1 = gv_start(blockIdx.x + 1, p.T, G);
+  const int nsteps = (int)(s1 - s0);
   const uint32_t bar0 = base_u32 + C::OFF_BAR;
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
+  const uint32_t sync_bar = bar0 + 8u * (2 * C::STAGES);
   float* part = reinterpret_cast<float*>(smem + C::OFF_PART);
-  float* hp = reinterpret_cast<float*>(smem + C::OFF_HP);
-  float* hf = reinterpret_cast<float*>(smem + C::OFF_HF);
+  volatile int* meta = reinterpret_cast<volatile int*>(smem + C::OFF_META);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), kGvWarps - 1);  // the compute warps
+      mbar_init(empty_bar(s), kGvCompute);
     }
+    mbar_init(sync_bar, kGvCompute);
     fence_mbar_init();
   }
-  if (warp == kGvWarpA && lane == 0) {
+  if (warp == kGvWarpP && lane == 0) {
     prefetch_tmap(&tmW);
     prefetch_tmap(&tmX);
   }
   __syncthreads();
-  pdl_wait();  // inputs of the previous kernel in the stream are complete from here on
-  pdl_launch_dependents();  // after the wait: a dependent may rely on what this launch waited for
-
-  auto issue = [&](int i) {  // stage i of this slice into slot i % STAGES
-    const int s = i % C::STAGES;
-    const uint32_t st = base_u32 + s * C::STAGE;
-    const int kg = kg0 + i;
-    mbar_arrive_expect_tx(full_bar(s), C::STAGE);
-    tma_load_2d(st, &tmW, full_bar(s), kg * (C::GB / 4), n0);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      tma_load_2d(st + C::W_BYTES + q * C::X_BOX, &tmX, full_bar(s), kg * 256 + 64 * q, 0);
-    }
-  };
+  // W and X come from before the H kernel that precedes this launch (it waited for its predecessor
+  // before it let this launch start), so the stream needs no wait.
 
   bool ok = true;
-  float acc[MT][4];
-#pragma unroll
-  for (int t = 0; t < MT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-  float hacc[2][4];
-#pragma unroll
-  for (int t = 0; t < 2; ++t) hacc[t][0] = hacc[t][1] = hacc[t][2] = hacc[t][3] = 0.f;
-
-  if (warp == kGvWarpA) {
-    // ---- producer: lane 0 refills each slot as soon as the compute warps release it ----
+  if (warp == kGvWarpP) {
+    // ---- producer: lane 0 streams the range's steps, tagging each stage with its row block and
+    // whether it opens or closes a piece ----
     if (lane == 0) {
-      for (int i = 0; i < nst; ++i) {
-        if (i >= C::STAGES && !mbar_wait(empty_bar(i % C::STAGES), ((i / C::STAGES) & 1) ^ 1, 41)) {
+      for (int it = 0; it < nsteps; ++it) {
+        const int s = it % C::STAGES;
+        if (it >= C::STAGES && !mbar_wait(empty_bar(s), ((it / C::STAGES) & 1) ^ 1, 41)) {
           ok = false;
           break;
         }
-        issue(i);
+        // ramp: stages 2 and 3 only once stages 0 and 1 have landed, so that the first data of
+        // every CTA is not queued behind the whole ring's worth of every other CTA
+        if (it >= 2 && it < C::STAGES && !mbar_wait(full_bar(it - 2), 0u, 42)) {
+          ok = false;
+          break;
+        }
+        const long t = s0 + it;
+        const int rb = (int)(t / p.ksteps), ks = (int)(t - (long)rb * p.ksteps);
+        meta[2 * s] = rb;
+        meta[2 * s + 1] = (it == 0 || ks == 0 ? 1 : 0) | (it == nsteps - 1 || ks == p.ksteps - 1 ? 2 : 0);
+        const uint32_t st = base_u32 + s * C::STAGE;
+        mbar_arrive_expect_tx(full_bar(s), C::STAGE);
+        tma_load_2d(st, &tmW, full_bar(s), ks * (C::GB / 4), rb * C::ROWS);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          tma_load_2d(st + C::W_BYTES + q * C::X_BOX, &tmX, full_bar(s), ks * 256 + 64 * q, 0);
       }
     }
-  } else {
-    // ---- weight rows 16 (warp % 4) + g and + 8; blocks of half warp / 4 of each K step; and
-    // H = X A^T over k16 steps warp and warp + 8 of each K step ----
-    const int R0 = 16 * (warp & 3) + g;
-    const int half = warp >> 2;
-    for (int i = 0; i < nst; ++i) {
-      const int s = i % C::STAGES;
-      if (!warp_wait(full_bar(s), (i / C::STAGES) & 1, 43)) { ok = false; break; }
+    __syncwarp();  // the idle lanes wait here, not at the final wait (which would hold lane 0)
+  } else if (warp < kGvCompute) {
+    const int tid = threadIdx.x;                   // 0 .. 255
+    const int bp = warp & 3;                       // block pair of every K step
+    const int rbase = (warp >> 2) * (C::ROWS / 2);  // first row of this warp's half
+    const int thr_off = (rbase + g) * C::GB + bp * C::PB;
+    const uint32_t nm = p.nib_mask, mg = p.bf16_magic;
+    uint32_t sync_par = 0;
+    auto consumer_sync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sync_bar);
+      const bool w = __all_sync(0xffffffffu, mbar_wait(sync_bar, sync_par, 44));
+      sync_par ^= 1u;
+      return w;
+    };
+    float acc[C::RT][MT][4];
+    for (int it = 0; it < nsteps; ++it) {
+      const int s = it % C::STAGES;
+      if (!warp_wait(full_bar(s), (it / C::STAGES) & 1, 43)) { ok = false; break; }
+      const int rb = meta[2 * s], fl = meta[2 * s + 1];
+      if (fl & 1) {
+#pragma unroll
+        for (int t = 0; t < C::RT; ++t)
+#pragma unroll
+          for (int tt = 0; tt < MT; ++tt) acc[t][tt][0] = acc[t][tt][1] = acc[t][tt][2] = acc[t][tt][3] = 0.f;
+      }
       const uint8_t* ws = smem + s * C::STAGE;
-      const uint8_t* xs = ws + C::W_BYTES;
-      const uint8_t* g0 = ws + R0 * C::GB;
-      const uint8_t* g1 = g0 + 8 * C::GB;
-      if (half == 0) gv_block_half<QT, MT, 0>(g0, g1, xs, c, g, acc);
-      else gv_block_half<QT, MT, 1>(g0, g1, xs, c, g, acc);
+      const uint8_t* xbox = ws + C::W_BYTES + bp * C::X_BOX;  // blocks 2bp, 2bp + 1: k 64 bp .. + 63
+      // X fragments of the two blocks (per token tile) in the k order of the A fragments, and for
+      // Q4_0 the offset term -136 * (block sum of X) in accumulator layout
+      uint32_t xf[2][MT][4];
+      float cz[2][MT][4];
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        const int k16 = warp + 8 * h2;
-        const int q = k16 >> 2, kk = (k16 & 3) * 16;
-        const uint8_t* xb = xs + q * C::X_BOX;
-        const long kglob = (long)(kg0 + i) * 256 + 64 * q + kk;  // this k16 step of the adapter A
-        const uint32_t a0 = sw128_pair(xb, g, kk + 2 * c);
-        const uint32_t a2 = sw128_pair(xb, g, kk + 2 * c + 8);
-        const uint32_t a1 = MT == 2 ? sw128_pair(xb, g + 8, kk + 2 * c) : 0u;
-        const uint32_t a3 = MT == 2 ? sw128_pair(xb, g + 8, kk + 2 * c + 8) : 0u;
+      for (int blk = 0; blk < 2; ++blk)
 #pragma unroll
-        for (int jt = 0; jt < 2; ++jt) {
-          if (jt == 1 && p.r <= 8) break;
-          const int j = 8 * jt + g;
-          uint32_t b0 = 0u, b1 = 0u;
-          if (j < p.r) {
-            const __nv_bfloat16* ar = p.A + (long)j * p.K + kglob + 2 * c;
-            b0 = __ldg(reinterpret_cast<const unsigned int*>(ar));
-            b1 = __ldg(reinterpret_cast<const unsigned int*>(ar + 8));
+        for (int tt = 0; tt < MT; ++tt) {
+          const int row = 8 * tt + g;
+          const uint2 u0 = *reinterpret_cast<const uint2*>(gv_x_at(xbox, row, 32 * blk + 4 * c));
+          const uint2 u1 = *reinterpret_cast<const uint2*>(gv_x_at(xbox, row, 32 * blk + 16 + 4 * c));
+          if (QT == QL_Q4_0) {
+            xf[blk][tt][0] = __byte_perm(u0.x, u0.y, 0x5410);  // x(4c), x(4c + 2)
+            xf[blk][tt][1] = __byte_perm(u0.x, u0.y, 0x7632);  // x(4c + 1), x(4c + 3)
+            xf[blk][tt][2] = __byte_perm(u1.x, u1.y, 0x5410);
+            xf[blk][tt][3] = __byte_perm(u1.x, u1.y, 0x7632);
+            const uint32_t m136 = 0xC308C308u;  // bf16 (-136, -136)
+            mma_16816_z(cz[blk][tt], m136, m136, m136, m136, xf[blk][tt][0], xf[blk][tt][1]);
+            mma_16816(cz[blk][tt], m136, m136, m136, m136, xf[blk][tt][2], xf[blk][tt][3]);
+          } else {
+            xf[blk][tt][0] = u0.x;
+            xf[blk][tt][1] = u0.y;
+            xf[blk][tt][2] = u1.x;
+            xf[blk][tt][3] = u1.y;
           }
-          mma_16816(hacc[jt], a0, a1, a2, a3, b0, b1);
         }
+      const uint8_t* rbp = ws + thr_off;  // the thread's first row, its block pair
+#pragma unroll
+      for (int t = 0; t < C::RT; ++t) {
+        uint32_t f0[2][4], f1[2][4];
+        float d0[2], d1[2];
+        gv_row_pair<QT>(rbp + 16 * t * C::GB, rbp + 16 * t * C::GB + 4 * c, nm, mg, f0, d0);
+        gv_row_pair<QT>(rbp + (16 * t + 8) * C::GB, rbp + (16 * t + 8) * C::GB + 4 * c, nm, mg, f1, d1);
+#pragma unroll
+        for (int blk = 0; blk < 2; ++blk)
+#pragma unroll
+          for (int tt = 0; tt < MT; ++tt) {
+            float dblk[4];
+            if (QT == QL_Q4_0)
+              mma_16816_c(dblk, f0[blk][0], f1[blk][0], f0[blk][1], f1[blk][1], xf[blk][tt][0], xf[blk][tt][1],
+                          cz[blk][tt]);
+            else
+              mma_16816_z(dblk, f0[blk][0], f1[blk][0], f0[blk][1], f1[blk][1], xf[blk][tt][0], xf[blk][tt][1]);
+            mma_16816(dblk, f0[blk][2], f1[blk][2], f0[blk][3], f1[blk][3], xf[blk][tt][2], xf[blk][tt][3]);
+            acc[t][tt][0] = fmaf(d0[blk], dblk[0], acc[t][tt][0]);
+            acc[t][tt][1] = fmaf(d0[blk], dblk[1], acc[t][tt][1]);
+            acc[t][tt][2] = fmaf(d1[blk], dblk[2], acc[t][tt][2]);
+            acc[t][tt][3] = fmaf(d1[blk], dblk[3], acc[t][tt][3]);
+          }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(empty_bar(s));
-    }
-    // this warp's H partial: rows m = g, g + 8; cols j = 8 jt + 2c, + 1
-    float* hw = hp + warp * 256;
+      if (!(fl & 2)) continue;
+
+      // ---- end of a piece of row block rb: the four pairs' partials, summed in order, go to the
+      // piece's slot ----
+      {
+        float* pw = part + bp * (C::XR * C::ROWS);
 #pragma unroll
-    for (int jt = 0; jt < 2; ++jt) {
-      const int j = 8 * jt + 2 * c;
-      hw[g * 16 + j] = hacc[jt][0];
-      hw[g * 16 + j + 1] = hacc[jt][1];
-      hw[(g + 8) * 16 + j] = hacc[jt][2];
-      hw[(g + 8) * 16 + j + 1] = hacc[jt][3];
-    }
-    // partial outputs of this half: rows R0, R0 + 8; tokens 8t + 2c, + 1
-    float* ph = part + half * kGvRows * 16;
+        for (int t = 0; t < C::RT; ++t)
 #pragma unroll
-    for (int t = 0; t < MT; ++t) {
-      const int m = 8 * t + 2 * c;
-      ph[R0 * 16 + m] = acc[t][0];
-      ph[R0 * 16 + m + 1] = acc[t][1];
-      ph[(R0 + 8) * 16 + m] = acc[t][2];
-      ph[(R0 + 8) * 16 + m + 1] = acc[t][3];
+          for (int tt = 0; tt < MT; ++tt) {
+            const int R0 = rbase + 16 * t + g, m = 8 * tt + 2 * c;
+            pw[m * C::ROWS + R0] = acc[t][tt][0];
+            pw[(m + 1) * C::ROWS + R0] = acc[t][tt][1];
+            pw[m * C::ROWS + R0 + 8] = acc[t][tt][2];
+            pw[(m + 1) * C::ROWS + R0 + 8] = acc[t][tt][3];
+          }
+      }
+      if (!consumer_sync()) { ok = false; break; }
+      constexpr int SZ = C::XR * C::ROWS;
+      const int cfirst = gv_cta_of((long)rb * p.ksteps, p.T, G);
+      float* gp = p.gpart + ((long)rb * p.maxslots + (blockIdx.x - cfirst)) * SZ;
+      for (int i = tid; i < p.M * C::ROWS; i += kGvCompute * 32)  // i = m ROWS + R
+        gp[i] = ((part[i] + part[SZ + i]) + part[2 * SZ + i]) + part[3 * SZ + i];
+      if (!consumer_sync()) { ok = false; break; }  // part is free for the next piece
     }
   }
   if (!ok || dev_aborted()) spin_ns(2000000ull);  // copies issued before a wait gave up land first
-  __syncthreads();
-  // the two halves of every K step, and the eight warps' H partials, in a fixed order
-  for (int i = threadIdx.x; i < kGvRows * 16; i += kGvThreads) part[i] += part[kGvRows * 16 + i];
-  for (int i = threadIdx.x; i < 256; i += kGvThreads) {
-    float v = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) v += hp[w * 256 + i];
-    hp[8 * 256 + i] = v;
+  if (warp == kGvWarpL && lane == 0) {
+    // the next launch may start once every CTA has seen the H kernel complete
+    pdl_wait();
+    pdl_launch_dependents();
   }
-  cluster_sync_all();
-  // H = sum over the cluster's slices, in rank order
-  for (int i = threadIdx.x; i < 16 * 16; i += kGvThreads) hf[i] = cluster_sum_ordered(&hp[8 * 256 + i], KS);
-  __syncthreads();
-  if (blockIdx.x == 0 && rank == 0 && p.H != nullptr)
-    for (int i = threadIdx.x; i < p.M * p.r; i += kGvThreads) p.H[i] = hf[(i / p.r) * 16 + i % p.r];
-  // rank q finishes rows [q * rows_per, (q + 1) * rows_per) of the block
-  const int rows_per = (kGvRows + KS - 1) / KS;
-  const int rlo = (int)rank * rows_per;
-  const int rhi = min(kGvRows, rlo + rows_per);
-  for (int i = threadIdx.x; i < (rhi - rlo) * p.M; i += kGvThreads) {
-    const int m = i / (rhi - rlo), R = rlo + i % (rhi - rlo);
-    const int n = n0 + R;
-    float y = cluster_sum_ordered(&part[R * 16 + m], KS);
+  pdl_wait();  // this launch completes only after the H kernel has
+}
+
+// Y[m][n] = sum over the row block's slots in order + s sum_j H[m][j] B[n][j], for the 32 rows
+// [32 blockIdx.x, + 32) of the block's row block (of `rows` rows).
+__global__ void __launch_bounds__(128) gemv_finish_kernel(const float* __restrict__ gpart, int maxslots, int xr,
+                                                          int rows, int ksteps, int T, int G,
+                                                          const float* __restrict__ hf,
+                                                          const __nv_bfloat16* __restrict__ B, int N, int M, int r,
+                                                          float scale, void* __restrict__ Y, int y_dtype) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int n0 = 32 * blockIdx.x;
+  const int rb = n0 / rows, R0 = n0 - rb * rows;
+  const long t0 = (long)rb * ksteps;
+  const int cfirst = gv_cta_of(t0, T, G);
+  const int np = gv_cta_of(t0 + ksteps - 1, T, G) - cfirst + 1;
+  const long sz = (long)xr * rows;
+  const float* gb = gpart + (long)rb * maxslots * sz;
+  for (int i = threadIdx.x; i < M * 32; i += blockDim.x) {
+    const int m = i >> 5, R = R0 + (i & 31), n = rb * rows + R;
+    if (n >= N) continue;  // rows past N (zero filled by the copy) of the last row block
+    float y = 0.f;
+    for (int q = 0; q < np; ++q) y += gb[q * sz + m * rows + R];
     float l = 0.f;
-    for (int j = 0; j < p.r; ++j) l = fmaf(hf[m * 16 + j], __bfloat162float(p.B[(long)n * p.r + j]), l);
-    y = fmaf(p.scale, l, y);
-    if (p.y_dtype == QL_F32) reinterpret_cast<float*>(p.Y)[(long)m * p.N + n] = y;
-    else reinterpret_cast<__nv_bfloat16*>(p.Y)[(long)m * p.N + n] = __float2bfloat16_rn(y);
+    for (int j = 0; j < r; ++j) l = fmaf(hf[m * 16 + j], __bfloat162float(B[(long)n * r + j]), l);
+    y = fmaf(scale, l, y);
+    if (y_dtype == QL_F32) reinterpret_cast<float*>(Y)[(long)m * N + n] = y;
+    else reinterpret_cast<__nv_bfloat16*>(Y)[(long)m * N + n] = __float2bfloat16_rn(y);
   }
-  cluster_sync_all();  // no CTA leaves while a peer may still read its partials
 }
 
 }  // namespace qlora

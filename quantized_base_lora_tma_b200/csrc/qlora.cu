@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "qlora.h"
 #include "lora.cuh"
@@ -71,16 +72,55 @@ static bool tmap_bf16_rows(CUtensorMap* m, const void* ptr, uint64_t cols, uint6
                    CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-static bool tmap_packed(CUtensorMap* m, const void* ptr, uint64_t row_bytes, uint64_t rows, uint32_t group_bytes) {
-  return make_tmap(m, ptr, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, row_bytes / 4, rows, row_bytes, group_bytes / 4, 64,
+static bool tmap_packed(CUtensorMap* m, const void* ptr, uint64_t row_bytes, uint64_t rows, uint32_t group_bytes,
+                        uint32_t box_rows = 64) {
+  return make_tmap(m, ptr, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, row_bytes / 4, rows, row_bytes, group_bytes / 4, box_rows,
                    CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
+// Per-device host state that launches look up on every call: the SM count and which kernels have
+// had their dynamic shared-memory limit raised (cudaFuncSetAttribute costs microseconds).
+constexpr int kHostDevices = 64;
+static std::atomic<int> g_num_sms[kHostDevices];
+
 static int num_sms() {
-  int dev = 0, n = 148;
+  int dev = 0;
   cudaGetDevice(&dev);
+  if (dev >= 0 && dev < kHostDevices) {
+    const int c = g_num_sms[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int n = 148;
   cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
+  n = n > 0 ? n : 148;
+  if (dev >= 0 && dev < kHostDevices) g_num_sms[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+static std::mutex g_smem_attr_mu;
+static std::vector<std::pair<std::pair<const void*, int>, int>> g_smem_attr;  // (kernel, device) -> bytes set
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per kernel, device and size.
+template <typename Kernel>
+static cudaError_t set_smem(Kernel k, int bytes) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const void* key = reinterpret_cast<const void*>(k);
+  {
+    std::lock_guard<std::mutex> lock(g_smem_attr_mu);
+    for (const auto& e : g_smem_attr)
+      if (e.first.first == key && e.first.second == dev && e.second >= bytes) return cudaSuccess;
+  }
+  const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_smem_attr_mu);
+  for (auto& x : g_smem_attr)
+    if (x.first.first == key && x.first.second == dev) {
+      x.second = std::max(x.second, bytes);
+      return cudaSuccess;
+    }
+  g_smem_attr.push_back({{key, dev}, bytes});
+  return cudaSuccess;
 }
 
 static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -145,7 +185,7 @@ static int launch_qgemm(const CUtensorMap& tA, const CUtensorMap& tW, const CUte
                         const GemmParams& p, int grid, cudaStream_t st, int slot) {
   using C = GemmCfg<QT, TRANS, MS, BN>;
   auto k = qgemm_kernel<QT, TRANS, EPI, MS, BN>;
-  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+  if (set_smem(k, C::SMEM_BYTES) != cudaSuccess)
     return QL_ERR_CUDA;
   PdlLaunch L(dim3(grid), dim3(kGemmThreads), C::SMEM_BYTES, st);
   ev_record(slot, 0, st);
@@ -184,7 +224,7 @@ static int launch_qgemm2(const CUtensorMap& tA, const CUtensorMap& tW, const CUt
                          const GemmParams& p, int tiles, cudaStream_t st, int slot) {
   using C = Gemm2Cfg<QT, TRANS, MS>;
   auto k = qgemm2_kernel<QT, TRANS, MS>;
-  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+  if (set_smem(k, C::SMEM_BYTES) != cudaSuccess)
     return QL_ERR_CUDA;
   static int max_clusters[16] = {};
   int dev = 0;
@@ -245,7 +285,7 @@ static cudaError_t launch_rows_nt(cudaLaunchConfig_t& cfg, const __nv_bfloat16* 
                                   float lscale, float* out, __nv_bfloat16* la, int RP, BopArgs bop, __nv_bfloat16* LB,
                                   int row_blocks, const float* hin, float hscale, __nv_bfloat16* hs, int* zc, int zn) {
   auto k = lora_rows_cluster_kernel<NT>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cfg.dynamicSmemBytes);
+  cudaError_t e = set_smem(k, (int)cfg.dynamicSmemBytes);
   if (e != cudaSuccess) return e;
   return cudaLaunchKernelEx(&cfg, k, Y, ldy, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out, la, RP, bop, LB,
                             row_blocks, hin, hscale, hs, zc, zn);
@@ -319,7 +359,7 @@ static size_t colred_ws_bytes(const ColredPlan& p, int r) {
 template <int JT>
 static cudaError_t launch_colred_jt(cudaLaunchConfig_t& cfg, const CUtensorMap* tm, const ColredFlow& P) {
   auto k = colred_flow_kernel<JT>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cfg.dynamicSmemBytes);
+  cudaError_t e = set_smem(k, (int)cfg.dynamicSmemBytes);
   if (e != cudaSuccess) return e;
   return cudaLaunchKernelEx(&cfg, k, tm[0], tm[1], tm[2], tm[3], P);
 }
@@ -474,16 +514,45 @@ static int launch_dense_gemm(int qtype, const void* A, int64_t M, int64_t Kd, co
   return launch_split_reduce(split_buf, d.ksplit, (long)M * Nd, (long)M * Nd, out, out_dtype, st);
 }
 
-// Small-M forward (M <= 16, Q4_0 / Q8_0, r <= 16): one launch of the weight-streaming kernel; the
-// KS CTAs of a cluster split K so that about two CTAs per SM are resident.
+// Small-M forward (M <= 16, Q4_0 / Q8_0, r <= 16): the H partial kernel, then the weight-streaming
+// kernel over G = (CTAs per SM) x SMs persistent CTAs, each a balanced range of steps.
+struct GvPlan {
+  int rows, mt, xr, nrb, ksteps, T, G, maxslots;
+  size_t smem;
+  size_t hp_bytes, part_bytes;  // workspace: H [16][16], piece partials
+};
+static GvPlan gemv_plan(int qtype, int64_t N, int64_t K, int64_t M) {
+  GvPlan g;
+  g.mt = M <= 8 ? 1 : 2;
+  g.xr = 8 * g.mt;
+  g.rows = qtype == QL_Q4_0 ? GvCfg<QL_Q4_0, 1>::ROWS : GvCfg<QL_Q8_0, 1>::ROWS;
+  g.smem = qtype == QL_Q4_0 ? (g.mt == 1 ? GvCfg<QL_Q4_0, 1>::SMEM_BYTES : GvCfg<QL_Q4_0, 2>::SMEM_BYTES)
+                            : (g.mt == 1 ? GvCfg<QL_Q8_0, 1>::SMEM_BYTES : GvCfg<QL_Q8_0, 2>::SMEM_BYTES);
+  g.nrb = (int)((N + g.rows - 1) / g.rows);
+  g.ksteps = (int)(K / 256);
+  g.T = g.nrb * g.ksteps;
+  const int per_sm = std::max(1, (int)(233472 / (g.smem + 1024)));
+  // one SM is left to the H kernel that runs beside the stream: a persistent CTA that could not be
+  // placed until it finished would hold up the whole launch
+  g.G = std::max(1, std::min(g.T, per_sm * std::max(1, num_sms() - 1)));
+  g.maxslots = 1;
+  for (int rb = 0; rb < g.nrb; ++rb) {
+    const long t0 = (long)rb * g.ksteps;
+    g.maxslots = std::max(g.maxslots, gv_cta_of(t0 + g.ksteps - 1, g.T, g.G) - gv_cta_of(t0, g.T, g.G) + 1);
+  }
+  g.hp_bytes = al256((size_t)256 * 4);
+  g.part_bytes = (size_t)g.nrb * g.maxslots * g.xr * g.rows * 4;
+  return g;
+}
+
 template <int QT, int MT>
-static int launch_gemv_q(const CUtensorMap& tW, const CUtensorMap& tX, const GvParams& p, int KS, cudaStream_t st,
+static int launch_gemv_q(const CUtensorMap& tW, const CUtensorMap& tX, const GvParams& p, int G, cudaStream_t st,
                          int slot) {
   using C = GvCfg<QT, MT>;
   auto k = qgemv_fwd_kernel<QT, MT>;
-  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+  if (set_smem(k, C::SMEM_BYTES) != cudaSuccess)
     return QL_ERR_CUDA;
-  PdlLaunch L(dim3(p.N / kGvRows, KS, 1), dim3(kGvThreads), C::SMEM_BYTES, st, KS);
+  PdlLaunch L(dim3(G), dim3(kGvThreads), C::SMEM_BYTES, st);
   ev_record(slot, 0, st);
   const cudaError_t e = cudaLaunchKernelEx(&L.cfg, k, tW, tX, p);
   ev_record(slot, 1, st);
@@ -494,45 +563,52 @@ static bool gemv_fwd_applies(int qtype, int64_t M, int r) {
   return M <= 16 && r <= kGvMaxRank && (qtype == QL_Q4_0 || qtype == QL_Q8_0);
 }
 
+// ws: the plan's workspace (H [16][16], then piece partials). Three launches: H (one CTA), the
+// weight stream (runs beside it), the row-block sums with the adapter term.
 static int launch_gemv_fwd(int qtype, const void* wq, int64_t N, int64_t K, const void* X, int64_t M, const void* A,
-                           const void* B, int r, float scale, void* Y, int y_dtype, float* H, cudaStream_t st,
-                           int slot) {
-  const int MT = M <= 8 ? 1 : 2;
+                           const void* B, int r, float scale, void* Y, int y_dtype, float* H, uint8_t* ws,
+                           cudaStream_t st, int slot) {
+  const GvPlan g = gemv_plan(qtype, N, K, M);
   CUtensorMap tW, tX;
-  if (!tmap_packed(&tW, wq, packed_row_bytes(qtype, K), N, group_bytes(qtype)) ||
-      !tmap_bf16_rows(&tX, X, K, M, 8u * MT))
+  if (!tmap_packed(&tW, wq, packed_row_bytes(qtype, K), N, group_bytes(qtype), (uint32_t)g.rows) ||
+      !tmap_bf16_rows(&tX, X, K, M, (uint32_t)g.xr))
     return QL_ERR_CUDA;
-  const int row_blocks = (int)(N / kGvRows);
-  const int groups = (int)(K / 256);
-  // K split: as many slices as keep every CTA resident in one wave
-  const size_t smem = qtype == QL_Q4_0 ? (MT == 1 ? GvCfg<QL_Q4_0, 1>::SMEM_BYTES : GvCfg<QL_Q4_0, 2>::SMEM_BYTES)
-                                       : (MT == 1 ? GvCfg<QL_Q8_0, 1>::SMEM_BYTES : GvCfg<QL_Q8_0, 2>::SMEM_BYTES);
-  const int per_sm = std::max(1, (int)(233472 / (smem + 1024)));
-  int KS = std::max(1, std::min(std::min(8, groups), per_sm * num_sms() / row_blocks));
-  const int kgroups = (groups + KS - 1) / KS;
-  KS = (groups + kgroups - 1) / kgroups;
+  float* hf = reinterpret_cast<float*>(ws);
+  float* gpart = reinterpret_cast<float*>(ws + g.hp_bytes);
+  {
+    PdlLaunch L(dim3(1), dim3(kGvHWarps * 32), 0, st);
+    const int rc = launch_result(cudaLaunchKernelEx(&L.cfg, gemv_h_kernel, (const __nv_bfloat16*)X,
+                                                    (const __nv_bfloat16*)A, (int)M, (int)K, r, hf, H));
+    if (rc) return rc;
+  }
   GvParams p;
   p.N = (int)N;
   p.K = (int)K;
   p.M = (int)M;
   p.r = r;
-  p.kgroups = kgroups;
-  p.scale = scale;
-  p.A = (const __nv_bfloat16*)A;
-  p.B = (const __nv_bfloat16*)B;
-  p.Y = Y;
-  p.y_dtype = y_dtype;
-  p.H = H;
+  p.nib_mask = 0x000F000Fu;
+  p.bf16_magic = 0x43004300u;
+  p.ksteps = g.ksteps;
+  p.T = g.T;
+  p.maxslots = g.maxslots;
+  p.gpart = gpart;
+  int rc;
   if (qtype == QL_Q4_0)
-    return MT == 1 ? launch_gemv_q<QL_Q4_0, 1>(tW, tX, p, KS, st, slot)
-                   : launch_gemv_q<QL_Q4_0, 2>(tW, tX, p, KS, st, slot);
-  return MT == 1 ? launch_gemv_q<QL_Q8_0, 1>(tW, tX, p, KS, st, slot)
-                 : launch_gemv_q<QL_Q8_0, 2>(tW, tX, p, KS, st, slot);
+    rc = g.mt == 1 ? launch_gemv_q<QL_Q4_0, 1>(tW, tX, p, g.G, st, slot)
+                   : launch_gemv_q<QL_Q4_0, 2>(tW, tX, p, g.G, st, slot);
+  else
+    rc = g.mt == 1 ? launch_gemv_q<QL_Q8_0, 1>(tW, tX, p, g.G, st, slot)
+                   : launch_gemv_q<QL_Q8_0, 2>(tW, tX, p, g.G, st, slot);
+  if (rc) return rc;
+  PdlLaunch L(dim3((unsigned)(g.nrb * g.rows / 32)), dim3(128), 0, st);
+  return launch_result(cudaLaunchKernelEx(&L.cfg, gemv_finish_kernel, (const float*)gpart, g.maxslots, g.xr, g.rows,
+                                          g.ksteps, g.T, g.G, (const float*)hf, (const __nv_bfloat16*)B, (int)N,
+                                          (int)M, r, scale, Y, y_dtype));
 }
 
 // Workspace layout of the dense layer (byte offsets, 256-aligned).
 struct LinearWs {
-  size_t la, lb, hs, split, cr, total;
+  size_t la, lb, hs, split, cr, hp, total;
 };
 static LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int r) {
   LinearWs w;
@@ -546,6 +622,13 @@ static LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int r) {
   const size_t sb = split_bytes(plan_dense(M, K, N, true, true), M, K);
   w.split = o; o = al256(o + std::max(sf, sb));
   w.cr = o; o = al256(o + colred_ws_bytes(plan_colred(M, N, K, r), r));
+  if (M <= 16) {
+    const GvPlan g = gemv_plan(QL_Q4_0, N, K, M), g8 = gemv_plan(QL_Q8_0, N, K, M);
+    const size_t gv = std::max(g.hp_bytes + g.part_bytes, g8.hp_bytes + g8.part_bytes);
+    w.hp = o; o = al256(o + gv);
+  } else {
+    w.hp = o;
+  }
   w.total = o;
   return w;
 }
@@ -752,9 +835,9 @@ int qlora_linear_fwd(int qtype, const void* wq, int64_t N, int64_t K, const void
   if (!ws || ws_bytes < w.total) return QL_ERR_WORKSPACE;
   if (!aligned16(ws)) return QL_ERR_ALIGNMENT;
   cudaStream_t st = (cudaStream_t)stream;
-  if (gemv_fwd_applies(qtype, M, r))
-    return launch_gemv_fwd(qtype, wq, N, K, X, M, A, B, r, scale, Y, y_dtype, H, st, 0);
   uint8_t* wsb = (uint8_t*)ws;
+  if (gemv_fwd_applies(qtype, M, r))
+    return launch_gemv_fwd(qtype, wq, N, K, X, M, A, B, r, scale, Y, y_dtype, H, wsb + w.hp, st, 0);
   __nv_bfloat16* LA = (__nv_bfloat16*)(wsb + w.la);
   __nv_bfloat16* LB = (__nv_bfloat16*)(wsb + w.lb);
   const int KL = 2 * lora_rp(r);
