@@ -231,12 +231,11 @@ struct BopArgs {            // LB[n] = [Z(n, :) | Z(n, :)], zero padded (nullptr
   int rows;
 };
 
-// This CTA's share (by its linear index in the grid) of LB, 8 columns per item.
-__device__ __forceinline__ void lora_bop_share(const BopArgs& bop, int r, int RP, __nv_bfloat16* __restrict__ LB) {
+// Share cta of ncta CTAs of LB, 8 columns per item.
+__device__ __forceinline__ void lora_bop_share(const BopArgs& bop, int r, int RP, __nv_bfloat16* __restrict__ LB,
+                                               long cta, long ncta) {
   if (bop.Z == nullptr) return;
   const long items = (long)bop.rows * (2 * RP / 8);
-  const long cta = (long)blockIdx.y * gridDim.x + blockIdx.x;
-  const long ncta = (long)gridDim.x * gridDim.y;
   for (long i = cta * blockDim.x + threadIdx.x; i < items; i += ncta * blockDim.x) {
     const int n = (int)(i / (2 * RP / 8));
     const int j0 = (int)(i % (2 * RP / 8)) * 8;
@@ -276,17 +275,24 @@ constexpr int kRowsTileK = 128;   // k per streamed tile (64 rows x 128 bf16)
 constexpr int kRowsYS = kRowsTileK + 8;  // padded tile row: ldmatrix rows land in distinct banks
 
 // Dynamic shared memory of lora_rows_cluster_kernel<NT> for a k range of kchunk.
-__host__ __device__ constexpr size_t rows_smem_bytes(int NT, int kchunk) {
-  return (size_t)kRowsStages * 64 * kRowsYS * 2 + (size_t)8 * NT * (kchunk + 8) * 2 + (size_t)64 * 8 * NT * 4;
+// Z slice: [RN][kchunk + 8] (k contiguous) or, ztr, [kchunk][RN + 8] (j contiguous).
+__host__ __device__ constexpr size_t rows_zs_halves(int NT, int kchunk, bool ztr) {
+  return ztr ? (size_t)kchunk * (8 * NT + 8) : (size_t)8 * NT * (kchunk + 8);
+}
+__host__ __device__ constexpr size_t rows_smem_bytes(int NT, int kchunk, bool ztr) {
+  return (size_t)kRowsStages * 64 * kRowsYS * 2 + rows_zs_halves(NT, kchunk, ztr) * 2 + (size_t)64 * 8 * NT * 4;
 }
 
 // Rows of out = Y Z^T for 64 rows per cluster column (warp w owns rows 16w .. 16w+15); cluster rank
-// q sums k in [q * kchunk, (q + 1) * kchunk). Z(j, k) = Z[j*zj + k*zk] is staged once per CTA; the
-// rows of Y stream through a ring of 64 x 128 tiles (cp.async, kRowsStages deep) into ldmatrix-fed
-// mma.sync. The ranks' partials are summed through distributed shared memory in rank order.
-// Writes out = oscale * sum (fp32 [M x r]) and la = split(lscale * sum) ([M x 2RP] bf16); when
-// hin is given also hs = split(hscale * hin) for the same rows; every CTA also writes its share of
-// the LB operand (bop). CTAs with blockIdx.x >= row_blocks (whole clusters) only write LB.
+// q sums k in [q * kchunk, (q + 1) * kchunk). Z(j, k) = Z[j*zj + k*zk] is staged once per CTA as
+// it lies in memory: [j][k] when k is contiguous (read by ldmatrix), [k][j] when j is (read by
+// ldmatrix.trans, no transpose on the way in). The rows of Y stream through a ring of 64 x 128
+// tiles (cp.async, kRowsStages deep) into mma.sync. The ranks' partials are summed through
+// distributed shared memory in rank order. Writes out = oscale * sum (fp32 [M x r]) and
+// la = split(lscale * sum) ([M x 2RP] bf16). The aux CTAs (blockIdx.x >= row_blocks, whole
+// clusters, when the launch has room for them in its one wave) write the LB operand (bop) and,
+// when hin is given, hs = split(hscale * hin), beside the row CTAs; without them every CTA takes a
+// share of that before its cluster sync.
 template <int NT>
 __global__ void __launch_bounds__(128) lora_rows_cluster_kernel(
     const __nv_bfloat16* __restrict__ Y, long ldy, int M, int Kin, int kchunk, const __nv_bfloat16* __restrict__ Z,
@@ -300,14 +306,29 @@ __global__ void __launch_bounds__(128) lora_rows_cluster_kernel(
   pdl_launch_dependents();
   if (blockIdx.x == 0 && blockIdx.y == 0)
     for (int i = threadIdx.x; i < zn; i += blockDim.x) zc[i] = 0;  // counters of a later kernel
+  // LB and hs: by the aux CTAs when the launch has them, else by every CTA before its cluster sync
+  auto aux_share = [&](long cta, long ncta) {
+    lora_bop_share(bop, r, RP, LB, cta, ncta);
+    if (hs != nullptr)
+      for (long i = cta * blockDim.x + threadIdx.x; i < (long)M * RP; i += ncta * blockDim.x) {
+        const long m = i / RP;
+        const int j = (int)(i % RP);
+        const float x = j < r ? hscale * hin[m * r + j] : 0.f;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+        hs[m * 2 * RP + j] = hi;
+        hs[m * 2 * RP + RP + j] = __float2bfloat16_rn(x - __bfloat162float(hi));
+      }
+  };
+  const bool aux_ctas = (int)gridDim.x > row_blocks;
   if ((int)blockIdx.x >= row_blocks) {
-    lora_bop_share(bop, r, RP, LB);
+    aux_share((long)(blockIdx.x - row_blocks) * gridDim.y + blockIdx.y, (long)(gridDim.x - row_blocks) * gridDim.y);
     return;
   }
-  const int ZS = kchunk + 8;
+  const bool ztr = zk != 1;  // Z staged [k][j]
+  const int ZS = kchunk + 8, ZT = RN + 8;
   __nv_bfloat16* ring = reinterpret_cast<__nv_bfloat16*>(rows_smem);
   __nv_bfloat16* zs = ring + S * 64 * YS;
-  float* part = reinterpret_cast<float*>(zs + RN * ZS);
+  float* part = reinterpret_cast<float*>(zs + rows_zs_halves(NT, kchunk, ztr));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int KS = gridDim.y;
   const uint32_t rank = cluster_ctarank();
@@ -329,14 +350,27 @@ __global__ void __launch_bounds__(128) lora_rows_cluster_kernel(
                  v);
     }
   };
-  // Z(j, k) contiguous in k: staged by cp.async in its own group, ahead of the ring's first tiles
-  if (zk == 1) {
-    const uint32_t zdst = smem_u32(zs);
+  // the Z slice by cp.async in its own group, ahead of the ring's first tiles, where rows are whole
+  // 16-byte chunks; otherwise element by element
+  const uint32_t zdst = smem_u32(zs);
+  if (!ztr) {
     for (int i = tid; i < RN * (kchunk / 8); i += 128) {
       const int j = i / (kchunk / 8), q = i % (kchunk / 8);
       const bool v = j < r && 8 * q < nk;
       cp_async16(zdst + (uint32_t)(j * ZS + 8 * q) * 2, v ? (const void*)(Z + (long)j * zj + kb + 8 * q) : (const void*)Z,
                  v);
+    }
+  } else if (zj == 1 && (r & 7) == 0 && (zk & 7) == 0) {
+    for (int i = tid; i < kchunk * (RN / 8); i += 128) {
+      const int kk = i / (RN / 8), q = i % (RN / 8);
+      const bool v = 8 * q < r && kk < nk;
+      cp_async16(zdst + (uint32_t)(kk * ZT + 8 * q) * 2, v ? (const void*)(Z + (long)(kb + kk) * zk + 8 * q) : (const void*)Z,
+                 v);
+    }
+  } else {
+    for (int i = tid; i < kchunk * RN; i += 128) {
+      const int kk = i / RN, j = i % RN;
+      zs[kk * ZT + j] = (j < r && kk < nk) ? Z[(long)j * zj + (long)(kb + kk) * zk] : __float2bfloat16(0.f);
     }
   }
   cp_async_commit();
@@ -345,65 +379,23 @@ __global__ void __launch_bounds__(128) lora_rows_cluster_kernel(
     if (t < ntiles) issue(t);
     cp_async_commit();
   }
-  if (zk != 1) {
-    // Z(j, k) = Z[j*zj + k*zk] with unit zj (the transposed adapter): the r values of one k are
-    // contiguous; all of a thread's loads are issued before its first shared store
-    const bool vec = zj == 1 && (r & 7) == 0 && (zk & 7) == 0;
-    if (vec) {
-      const int cpr = r / 8;  // 16-byte chunks per k
-      const int total = kchunk * cpr;
-      for (int i0 = tid; i0 < total; i0 += 128 * 8) {
-        uint4 v[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int i = i0 + 128 * u, kk = i / cpr, q = i % cpr;
-          v[u] = (i < total && kk < nk) ? __ldg(reinterpret_cast<const uint4*>(Z + (long)(kb + kk) * zk + 8 * q))
-                                        : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int i = i0 + 128 * u, kk = i / cpr, q = i % cpr;
-          if (i < total) {
-            const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&v[u]);
-#pragma unroll
-            for (int w = 0; w < 8; ++w) zs[(8 * q + w) * ZS + kk] = e[w];
-          }
-        }
-      }
-      for (int i = tid; i < (RN - r) * kchunk; i += 128) zs[(r + i / kchunk) * ZS + i % kchunk] = __float2bfloat16(0.f);
-    } else {
-      const int total = kchunk * RN;
-      for (int i0 = tid; i0 < total; i0 += 128 * 16) {
-        __nv_bfloat16 v[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int i = i0 + 128 * u;
-          const int kk = i / RN, j = i % RN;
-          v[u] = (i < total && j < r && kk < nk) ? Z[(long)j * zj + (long)(kb + kk) * zk] : __float2bfloat16(0.f);
-        }
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int i = i0 + 128 * u;
-          if (i < total) zs[(i % RN) * ZS + i / RN] = v[u];
-        }
-      }
-    }
-  }
 
   float acc[NT][4];
 #pragma unroll
   for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-  // ldmatrix lane addresses: A = rows 16w + lane%16, k offset 8*(lane/16); B = Z rows (n) lane%8 +
-  // 8*(lane/16) of an n-tile pair, k offset 8*((lane/8)%2)
+  // ldmatrix lane addresses: A = rows 16w + lane%16, k offset 8*(lane/16). B, [j][k]: Z rows (n)
+  // lane%8 + 8*(lane/16) of an n-tile pair, k offset 8*((lane/8)%2); B, [k][j] (.trans): k rows
+  // lane%8 + 8*((lane/8)%2), j offset 8*(lane/16). Both give (tile 0: k 0-7, k 8-15; tile 1: ..).
   const int a_row = 16 * warp + (lane & 15), a_col = 8 * (lane >> 4);
   const int b_row = (lane & 7) + 8 * (lane >> 4), b_col = 8 * ((lane >> 3) & 1);
+  const int t_k = (lane & 7) + 8 * ((lane >> 3) & 1), t_j = 8 * (lane >> 4);
   for (int t = 0; t < ntiles; ++t) {
     cp_async_wait<S - 2>();
     __syncthreads();  // tile t visible to all; every thread is done with tile t - 1's slot
     if (t + S - 1 < ntiles) issue(t + S - 1);
     cp_async_commit();
     const uint32_t abase = smem_u32(ring + (t % S) * 64 * YS + a_row * YS + a_col);
-    const uint32_t bbase = smem_u32(zs + b_row * ZS + t * TK + b_col);
+    const uint32_t bbase = ztr ? smem_u32(zs + (t * TK + t_k) * ZT + t_j) : smem_u32(zs + b_row * ZS + t * TK + b_col);
 #pragma unroll
     for (int k16 = 0; k16 < TK / 16; ++k16) {
       uint32_t a0, a1, a2, a3;
@@ -411,7 +403,8 @@ __global__ void __launch_bounds__(128) lora_rows_cluster_kernel(
 #pragma unroll
       for (int tp = 0; tp < NT / 2; ++tp) {
         uint32_t b0, b1, b2, b3;
-        ldsm_x4(bbase + (uint32_t)(16 * tp * ZS) * 2 + 32 * k16, b0, b1, b2, b3);
+        if (ztr) ldsm_x4_t(bbase + (uint32_t)(16 * k16 * ZT) * 2 + 32 * tp, b0, b1, b2, b3);
+        else ldsm_x4(bbase + (uint32_t)(16 * tp * ZS) * 2 + 32 * k16, b0, b1, b2, b3);
         mma_16816(acc[2 * tp], a0, a1, a2, a3, b0, b1);
         mma_16816(acc[2 * tp + 1], a0, a1, a2, a3, b2, b3);
       }
@@ -430,7 +423,7 @@ __global__ void __launch_bounds__(128) lora_rows_cluster_kernel(
       part[(lr + 8) * RN + j + 1] = acc[t][3];
     }
   }
-  lora_bop_share(bop, r, RP, LB);  // off the main loop's path: overlaps the wait for the cluster
+  if (!aux_ctas) aux_share((long)blockIdx.y * gridDim.x + blockIdx.x, (long)gridDim.x * gridDim.y);
   cluster_sync_all();
   // rank q reduces rows [q*64/KS, (q+1)*64/KS) of the cluster's 64 rows, over ranks in order
   const int rows_per = (64 + KS - 1) / KS;
@@ -448,12 +441,6 @@ __global__ void __launch_bounds__(128) lora_rows_cluster_kernel(
       const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
       la[(long)m * 2 * RP + j] = j < r ? hi : __float2bfloat16(0.f);
       la[(long)m * 2 * RP + RP + j] = j < r ? lo : __float2bfloat16(0.f);
-    }
-    if (hs != nullptr) {
-      const float x = j < r ? hscale * hin[(long)m * r + j] : 0.f;
-      const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-      hs[(long)m * 2 * RP + j] = hi;
-      hs[(long)m * 2 * RP + RP + j] = __float2bfloat16_rn(x - __bfloat162float(hi));
     }
   }
   cluster_sync_all();  // no CTA leaves while a peer may still read its partials

@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <array>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -291,6 +292,50 @@ static cudaError_t launch_rows_nt(cudaLaunchConfig_t& cfg, const __nv_bfloat16* 
                             row_blocks, hin, hscale, hs, zc, zn);
 }
 
+// Clusters of KS CTAs of the row kernel (NT, smem) that are resident at once (cached).
+static int rows_cluster_capacity(int NT, size_t smem, int KS) {
+  static std::mutex mu;
+  static std::vector<std::pair<std::array<long, 4>, int>> cache;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const std::array<long, 4> key{NT, (long)smem, KS, dev};
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (const auto& e : cache)
+      if (e.first == key) return e.second;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1, KS, 1);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 1;
+  at[0].val.clusterDim.y = KS;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  cudaError_t e;
+  if (NT == 2) {
+    set_smem(lora_rows_cluster_kernel<2>, (int)smem);
+    e = cudaOccupancyMaxActiveClusters(&n, lora_rows_cluster_kernel<2>, &cfg);
+  } else if (NT == 4) {
+    set_smem(lora_rows_cluster_kernel<4>, (int)smem);
+    e = cudaOccupancyMaxActiveClusters(&n, lora_rows_cluster_kernel<4>, &cfg);
+  } else {
+    set_smem(lora_rows_cluster_kernel<8>, (int)smem);
+    e = cudaOccupancyMaxActiveClusters(&n, lora_rows_cluster_kernel<8>, &cfg);
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  cache.push_back({key, n});
+  return n;
+}
+
 static int launch_rows_dense(const __nv_bfloat16* Y, long ldy, int M, int Kin, const __nv_bfloat16* Z, long zj,
                              long zk, int r, float oscale, float lscale, float* out, __nv_bfloat16* la, BopArgs bop,
                              __nv_bfloat16* LB, cudaStream_t st, const float* hin = nullptr, float hscale = 0.f,
@@ -303,14 +348,16 @@ static int launch_rows_dense(const __nv_bfloat16* Y, long ldy, int M, int Kin, c
   kchunk = (kchunk + 127) / 128 * 128;
   KS = (Kin + kchunk - 1) / kchunk;
   const int NT = r <= 16 ? 2 : (r <= 32 ? 4 : 8);
-  const size_t smem = rows_smem_bytes(NT, kchunk);
+  const size_t smem = rows_smem_bytes(NT, kchunk, zk != 1);
   if (smem > 232448) return QL_ERR_SHAPE;  // the staged adapter slice does not fit on chip
-  // extra clusters for the LB operand when it outweighs the row work (small M)
+  // aux clusters beside the row clusters for the LB operand and hs (about 8 items per thread, at
+  // most 32 CTAs) when they all fit in the same wave; otherwise the row CTAs share that work
   const int row_blocks = (M + 63) / 64;
-  const long bop_items = bop.Z ? (long)bop.rows * (2 * RP / 8) : 0;
-  const long per_cluster = (long)KS * 128 * 4;
-  const int bop_blocks = (int)std::max<long>(0, (bop_items + per_cluster - 1) / per_cluster - row_blocks);
-  PdlLaunch L(dim3(row_blocks + bop_blocks, KS, 1), dim3(128), smem, st, KS);
+  const long aux_items = (bop.Z ? (long)bop.rows * (2 * RP / 8) : 0) + (hs ? (long)M * RP / 4 : 0);
+  const int aux_ctas = aux_items ? (int)std::min<long>(32, std::max<long>(1, (aux_items + 1023) / 1024)) : 0;
+  int aux_blocks = (aux_ctas + KS - 1) / KS;
+  if (aux_blocks > 0 && row_blocks + aux_blocks > rows_cluster_capacity(NT, smem, KS)) aux_blocks = 0;
+  PdlLaunch L(dim3(row_blocks + aux_blocks, KS, 1), dim3(128), smem, st, KS);
   cudaLaunchConfig_t& cfg = L.cfg;
   cudaError_t e;
   if (NT == 2)
