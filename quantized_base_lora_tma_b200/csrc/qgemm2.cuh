@@ -148,8 +148,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm2Threads, 1)
   cluster_arrive_wait();  // both CTAs' barriers exist before any cross-CTA arrival
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
-  pdl_wait();  // inputs of the previous kernel in the stream are complete from here on
-  pdl_launch_dependents();  // after the wait: a dependent may rely on what this launch waited for
+  // A and W come from before the previous kernel in the stream (the row kernel, which waited for
+  // its own predecessor before it let this launch start), so the main loop streams them at once;
+  // only the LoRA operands are that kernel's output: the A producer waits for it before their
+  // first copy, and epilogue warp 0 waits for it before it lets the next launch start (which may
+  // rely on what this launch waited for) and so that this launch completes only after it.
 
   const int kb_main = p.Kd / kBK;
   auto tile_steps = [&](const TileInfo& ti) { return (ti.kb_hi - ti.kb_lo) + (ti.lora ? p.n_lora_kb : 0); };
@@ -167,6 +170,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm2Threads, 1)
       int it = 0;
       bool ok = true;
       bool issued = false;
+      bool waited = false;
       TileInfo ti;
       for (int t = cid; ok && gemm2_tile<C::BM>(p, t, ti); t += ncl) {
         const int nsteps = tile_steps(ti);
@@ -183,6 +187,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm2Threads, 1)
             for (int h = 0; h < MS; ++h)
               tma_load_2d_pair(sA + s * C::A_BYTES + h * 16384, &tmA, fb, kb * kBK, arow + 256 * h);
           } else {
+            if (!waited) {
+              pdl_wait();  // the LoRA operands are the previous kernel's output
+              waited = true;
+            }
             const int x = (kb - kb_main) * kBK;
             if (leader) mbar_arrive_expect_tx(full_bar(s), 2 * (C::A_BYTES + C::B_BYTES));
 #pragma unroll
@@ -367,6 +375,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm2Threads, 1)
     }
   } else if (warp < kNumEpiWarps) {
     // ---------------- epilogue: this CTA's MS x 128 rows x 256 columns ----------------
+    if (warp == 0) {
+      pdl_wait();
+      pdl_launch_dependents();
+    }
     int tc = 0;
     TileInfo ti;
     for (int t = cid; gemm2_tile<C::BM>(p, t, ti); t += ncl, ++tc) {
