@@ -6,8 +6,8 @@
 //   colred   out[c, j] = sum_m Y[m, c] Z[m, j] over row slices, then an ordered sum over the
 //            slices: dB = dY^T split(s H), dA = split(G)^T X (deterministic: no float atomics)
 //
-// Dense layer: lora_rows_cluster_kernel streams its bf16 operand through a cp.async ring and sums
-// its k slices in-cluster; colred_flow_kernel streams through a TMA ring, takes units of work from
+// Dense layer: lora_rows_cluster_kernel streams its bf16 operand through a TMA ring and sums its k
+// slices in-cluster; colred_flow_kernel streams through a TMA ring, takes units of work from
 // a counter and sums a block's row slices in slice order. Routed (grouped) layer:
 // lora_rows_seg_kernel, colred_mma_kernel + colred_reduce_kernel, lora_bop_vec_kernel.
 //
@@ -270,38 +270,49 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
                : "r"(addr));
 }
 
-constexpr int kRowsStages = 4;    // cp.async ring depth of the dense row products
-constexpr int kRowsTileK = 128;   // k per streamed tile (64 rows x 128 bf16)
-constexpr int kRowsYS = kRowsTileK + 8;  // padded tile row: ldmatrix rows land in distinct banks
+// Element (row, col) of a 128-byte-swizzled box of 64 bf16 columns: 16-byte chunk col/8 of row
+// `row` sits at chunk position (col/8) ^ (row % 8).
+__device__ __forceinline__ uint32_t sw128_addr(uint32_t box, int row, int col) {
+  return box + (uint32_t)(row * 128) + ((uint32_t)(((col >> 3) ^ (row & 7))) << 4) + (uint32_t)((col & 7) * 2);
+}
 
-// Dynamic shared memory of lora_rows_cluster_kernel<NT> for a k range of kchunk.
-// Z slice: [RN][kchunk + 8] (k contiguous) or, ztr, [kchunk][RN + 8] (j contiguous).
+constexpr int kRowsStages = 4;    // TMA ring depth of the dense row products
+constexpr int kRowsTileK = 128;   // k per streamed tile: 64 rows x 128 bf16, two 128-byte-swizzled boxes
+constexpr int kRowsStageBytes = 64 * kRowsTileK * 2;
+
+// Dynamic shared memory of lora_rows_cluster_kernel<NT> for a k range of kchunk: the ring, the Z
+// slice ([RN][kchunk + 8], k contiguous, or ztr: [kchunk][RN + 8], j contiguous), the partials, the
+// ring's barriers and the alignment slack.
 __host__ __device__ constexpr size_t rows_zs_halves(int NT, int kchunk, bool ztr) {
   return ztr ? (size_t)kchunk * (8 * NT + 8) : (size_t)8 * NT * (kchunk + 8);
 }
 __host__ __device__ constexpr size_t rows_smem_bytes(int NT, int kchunk, bool ztr) {
-  return (size_t)kRowsStages * 64 * kRowsYS * 2 + rows_zs_halves(NT, kchunk, ztr) * 2 + (size_t)64 * 8 * NT * 4;
+  return (size_t)kRowsStages * kRowsStageBytes + rows_zs_halves(NT, kchunk, ztr) * 2 + (size_t)64 * 8 * NT * 4 +
+         2 * kRowsStages * 8 + 1024;
 }
 
 // Rows of out = Y Z^T for 64 rows per cluster column (warp w owns rows 16w .. 16w+15); cluster rank
 // q sums k in [q * kchunk, (q + 1) * kchunk). Z(j, k) = Z[j*zj + k*zk] is staged once per CTA as
 // it lies in memory: [j][k] when k is contiguous (read by ldmatrix), [k][j] when j is (read by
-// ldmatrix.trans, no transpose on the way in). The rows of Y stream through a ring of 64 x 128
-// tiles (cp.async, kRowsStages deep) into mma.sync. The ranks' partials are summed through
+// ldmatrix.trans, no transpose on the way in). The rows of Y (tensor map tmY, 64 x 64 boxes,
+// 128-byte swizzle) stream by TMA through a ring of 64 x 128 tiles (kRowsStages deep, mbarrier
+// guarded; thread 0 refills a slot once the four warps have released it) into mma.sync. The ranks' partials are summed through
 // distributed shared memory in rank order. Writes out = oscale * sum (fp32 [M x r]) and
 // la = split(lscale * sum) ([M x 2RP] bf16). The aux CTAs (blockIdx.x >= row_blocks, whole
 // clusters, when the launch has room for them in its one wave) write the LB operand (bop) and,
 // when hin is given, hs = split(hscale * hin), beside the row CTAs; without them every CTA takes a
-// share of that before its cluster sync.
+// share of that while its first copies are in flight.
 template <int NT>
 __global__ void __launch_bounds__(128) lora_rows_cluster_kernel(
-    const __nv_bfloat16* __restrict__ Y, long ldy, int M, int Kin, int kchunk, const __nv_bfloat16* __restrict__ Z,
+    const __grid_constant__ CUtensorMap tmY, int M, int Kin, int kchunk, const __nv_bfloat16* __restrict__ Z,
     long zj, long zk, int r, float oscale, float lscale, float* __restrict__ out, __nv_bfloat16* __restrict__ la,
     int RP, BopArgs bop, __nv_bfloat16* __restrict__ LB, int row_blocks, const float* __restrict__ hin, float hscale,
     __nv_bfloat16* __restrict__ hs, int* __restrict__ zc, int zn) {
   constexpr int RN = 8 * NT;
-  constexpr int S = kRowsStages, TK = kRowsTileK, YS = kRowsYS;
-  extern __shared__ __align__(16) uint8_t rows_smem[];
+  constexpr int S = kRowsStages, TK = kRowsTileK, SB = kRowsStageBytes;
+  extern __shared__ uint8_t rows_smem_raw[];
+  const uint32_t base = (smem_u32(rows_smem_raw) + 1023u) & ~1023u;
+  uint8_t* smem = rows_smem_raw + (base - smem_u32(rows_smem_raw));
   pdl_wait();
   pdl_launch_dependents();
   if (blockIdx.x == 0 && blockIdx.y == 0)
@@ -326,9 +337,11 @@ __global__ void __launch_bounds__(128) lora_rows_cluster_kernel(
   }
   const bool ztr = zk != 1;  // Z staged [k][j]
   const int ZS = kchunk + 8, ZT = RN + 8;
-  __nv_bfloat16* ring = reinterpret_cast<__nv_bfloat16*>(rows_smem);
-  __nv_bfloat16* zs = ring + S * 64 * YS;
+  __nv_bfloat16* zs = reinterpret_cast<__nv_bfloat16*>(smem + S * SB);
   float* part = reinterpret_cast<float*>(zs + rows_zs_halves(NT, kchunk, ztr));
+  const uint32_t bar0 = smem_u32(part + 64 * RN);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int KS = gridDim.y;
   const uint32_t rank = cluster_ctarank();
@@ -338,20 +351,25 @@ __global__ void __launch_bounds__(128) lora_rows_cluster_kernel(
   const int nk = max(0, ke - kb);
   const int ntiles = (nk + TK - 1) / TK;
 
-  auto issue = [&](int t) {
-    const uint32_t dst0 = smem_u32(ring + (t % S) * 64 * YS);
-#pragma unroll
-    for (int it = 0; it < 64 * (TK / 8) / 128; ++it) {
-      const int i = tid + 128 * it;
-      const int row = i / (TK / 8), q = i % (TK / 8);
-      const int k = kb + t * TK + 8 * q;
-      const bool v = (m0 + row < M) && (k < ke);
-      cp_async16(dst0 + (uint32_t)(row * YS + 8 * q) * 2, v ? (const void*)(Y + (long)(m0 + row) * ldy + k) : (const void*)Y,
-                 v);
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 4);
     }
+    fence_mbar_init();
+    prefetch_tmap(&tmY);
+  }
+  __syncthreads();
+  auto issue = [&](int t) {  // tile t into slot t % S: k [kb + 128 t, + 128) of rows [m0, m0 + 64)
+    const int s = t % S;
+    const uint32_t st = base + (uint32_t)(s * SB);
+    mbar_arrive_expect_tx(full_bar(s), (uint32_t)SB);
+    tma_load_2d(st, &tmY, full_bar(s), kb + t * TK, m0);
+    tma_load_2d(st + SB / 2, &tmY, full_bar(s), kb + t * TK + 64, m0);
   };
-  // the Z slice by cp.async in its own group, ahead of the ring's first tiles, where rows are whole
-  // 16-byte chunks; otherwise element by element
+  // the Z slice by cp.async where rows are whole 16-byte chunks, otherwise element by element; its
+  // requests go out ahead of the ring's first tiles, which would otherwise queue them behind the
+  // whole grid's tile traffic
   const uint32_t zdst = smem_u32(zs);
   if (!ztr) {
     for (int i = tid; i < RN * (kchunk / 8); i += 128) {
@@ -374,32 +392,37 @@ __global__ void __launch_bounds__(128) lora_rows_cluster_kernel(
     }
   }
   cp_async_commit();
-#pragma unroll
-  for (int t = 0; t < S - 1; ++t) {
-    if (t < ntiles) issue(t);
-    cp_async_commit();
-  }
+  if (tid == 0)
+    for (int t = 0; t < min(ntiles, S); ++t) issue(t);
+  // without aux CTAs, this CTA's share of LB and hs while the first copies are in flight
+  if (!aux_ctas) aux_share((long)blockIdx.y * gridDim.x + blockIdx.x, (long)gridDim.x * gridDim.y);
+  cp_async_wait<0>();
+  __syncthreads();  // the Z slice is visible to every warp
 
   float acc[NT][4];
 #pragma unroll
   for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-  // ldmatrix lane addresses: A = rows 16w + lane%16, k offset 8*(lane/16). B, [j][k]: Z rows (n)
-  // lane%8 + 8*(lane/16) of an n-tile pair, k offset 8*((lane/8)%2); B, [k][j] (.trans): k rows
-  // lane%8 + 8*((lane/8)%2), j offset 8*(lane/16). Both give (tile 0: k 0-7, k 8-15; tile 1: ..).
+  // ldmatrix lane addresses: A = rows 16w + lane%16, k offset 8*(lane/16) (in the swizzled boxes).
+  // B, [j][k]: Z rows (n) lane%8 + 8*(lane/16) of an n-tile pair, k offset 8*((lane/8)%2); B, [k][j]
+  // (.trans): k rows lane%8 + 8*((lane/8)%2), j offset 8*(lane/16). Both give (tile 0: k 0-7,
+  // k 8-15; tile 1: ..).
   const int a_row = 16 * warp + (lane & 15), a_col = 8 * (lane >> 4);
   const int b_row = (lane & 7) + 8 * (lane >> 4), b_col = 8 * ((lane >> 3) & 1);
   const int t_k = (lane & 7) + 8 * ((lane >> 3) & 1), t_j = 8 * (lane >> 4);
+  bool ok = true;
   for (int t = 0; t < ntiles; ++t) {
-    cp_async_wait<S - 2>();
-    __syncthreads();  // tile t visible to all; every thread is done with tile t - 1's slot
-    if (t + S - 1 < ntiles) issue(t + S - 1);
-    cp_async_commit();
-    const uint32_t abase = smem_u32(ring + (t % S) * 64 * YS + a_row * YS + a_col);
+    const int s = t % S;
+    if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), (uint32_t)((t / S) & 1), 51))) {
+      ok = false;
+      break;
+    }
+    const uint32_t st = base + (uint32_t)(s * SB);
     const uint32_t bbase = ztr ? smem_u32(zs + (t * TK + t_k) * ZT + t_j) : smem_u32(zs + b_row * ZS + t * TK + b_col);
 #pragma unroll
     for (int k16 = 0; k16 < TK / 16; ++k16) {
+      const int kk = 16 * k16 + a_col;  // k within the tile
       uint32_t a0, a1, a2, a3;
-      ldsm_x4(abase + 32 * k16, a0, a1, a2, a3);
+      ldsm_x4(sw128_addr(st + (uint32_t)((kk >> 6) * (SB / 2)), a_row, kk & 63), a0, a1, a2, a3);
 #pragma unroll
       for (int tp = 0; tp < NT / 2; ++tp) {
         uint32_t b0, b1, b2, b3;
@@ -409,8 +432,19 @@ __global__ void __launch_bounds__(128) lora_rows_cluster_kernel(
         mma_16816(acc[2 * tp + 1], a0, a1, a2, a3, b2, b3);
       }
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty_bar(s));
+    if (warp == 0 && t + S < ntiles) {
+      // thread 0 refills this slot once all four warps have released it
+      bool w = true;
+      if (lane == 0) {
+        w = mbar_wait(empty_bar(s), (uint32_t)((t / S) & 1), 52);
+        if (w) issue(t + S);
+      }
+      if (!__shfl_sync(0xffffffffu, w ? 1 : 0, 0)) { ok = false; break; }
+    }
   }
-  cp_async_wait<0>();
+  if (!ok || dev_aborted()) spin_ns(2000000ull);  // copies issued before a wait gave up land first
   {
     const int g = lane >> 2, c = lane & 3;
 #pragma unroll
@@ -423,7 +457,6 @@ __global__ void __launch_bounds__(128) lora_rows_cluster_kernel(
       part[(lr + 8) * RN + j + 1] = acc[t][3];
     }
   }
-  if (!aux_ctas) aux_share((long)blockIdx.y * gridDim.x + blockIdx.x, (long)gridDim.x * gridDim.y);
   cluster_sync_all();
   // rank q reduces rows [q*64/KS, (q+1)*64/KS) of the cluster's 64 rows, over ranks in order
   const int rows_per = (64 + KS - 1) / KS;
@@ -488,11 +521,6 @@ __host__ __device__ constexpr size_t colred_smem_bytes(int RP, int JT, int tr) {
   return (size_t)colred_stages(RP, JT, tr) * colred_stage_bytes(RP, tr) + colred_comb_bytes(JT) + 256 + 1024;
 }
 
-// Element (row, col) of a 128-byte-swizzled box of 64 bf16 columns: 16-byte chunk col/8 of row
-// `row` sits at chunk position (col/8) ^ (row % 8).
-__device__ __forceinline__ uint32_t sw128_addr(uint32_t box, int row, int col) {
-  return box + (uint32_t)(row * 128) + ((uint32_t)(((col >> 3) ^ (row & 7))) << 4) + (uint32_t)((col & 7) * 2);
-}
 
 __device__ __forceinline__ void colred_store(const ColredOut& O, int r, int j, int col, float v) {
   if (j < r && col < O.C) O.out[O.transpose ? (long)j * O.C + col : (long)col * r + j] = O.scale * v;

@@ -281,14 +281,14 @@ static void rows_split(int M, int Kin, int ks_cap, int* KS, int* kchunk) {
 // Y Z^T), optionally hs = split(hscale * hin) for the same rows, and, in the same launch,
 // LB = [Zb | Zb] (bop).
 template <int NT>
-static cudaError_t launch_rows_nt(cudaLaunchConfig_t& cfg, const __nv_bfloat16* Y, long ldy, int M, int Kin,
-                                  int kchunk, const __nv_bfloat16* Z, long zj, long zk, int r, float oscale,
-                                  float lscale, float* out, __nv_bfloat16* la, int RP, BopArgs bop, __nv_bfloat16* LB,
+static cudaError_t launch_rows_nt(cudaLaunchConfig_t& cfg, const CUtensorMap& tmY, int M, int Kin, int kchunk,
+                                  const __nv_bfloat16* Z, long zj, long zk, int r, float oscale, float lscale,
+                                  float* out, __nv_bfloat16* la, int RP, BopArgs bop, __nv_bfloat16* LB,
                                   int row_blocks, const float* hin, float hscale, __nv_bfloat16* hs, int* zc, int zn) {
   auto k = lora_rows_cluster_kernel<NT>;
   cudaError_t e = set_smem(k, (int)cfg.dynamicSmemBytes);
   if (e != cudaSuccess) return e;
-  return cudaLaunchKernelEx(&cfg, k, Y, ldy, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out, la, RP, bop, LB,
+  return cudaLaunchKernelEx(&cfg, k, tmY, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out, la, RP, bop, LB,
                             row_blocks, hin, hscale, hs, zc, zn);
 }
 
@@ -349,6 +349,9 @@ static int launch_rows_dense(const __nv_bfloat16* Y, long ldy, int M, int Kin, c
   KS = (Kin + kchunk - 1) / kchunk;
   const int NT = r <= 16 ? 2 : (r <= 32 ? 4 : 8);
   const size_t smem = rows_smem_bytes(NT, kchunk, zk != 1);
+  CUtensorMap tmY;
+  if (!make_tmap(&tmY, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Kin, M, ldy * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+    return QL_ERR_CUDA;
   if (smem > 232448) return QL_ERR_SHAPE;  // the staged adapter slice does not fit on chip
   // aux clusters beside the row clusters for the LB operand and hs (about 8 items per thread, at
   // most 32 CTAs) when they all fit in the same wave; otherwise the row CTAs share that work
@@ -361,13 +364,13 @@ static int launch_rows_dense(const __nv_bfloat16* Y, long ldy, int M, int Kin, c
   cudaLaunchConfig_t& cfg = L.cfg;
   cudaError_t e;
   if (NT == 2)
-    e = launch_rows_nt<2>(cfg, Y, ldy, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out, la, RP, bop, LB, row_blocks,
+    e = launch_rows_nt<2>(cfg, tmY, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out, la, RP, bop, LB, row_blocks,
                           hin, hscale, hs, zc, zn);
   else if (NT == 4)
-    e = launch_rows_nt<4>(cfg, Y, ldy, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out, la, RP, bop, LB, row_blocks,
+    e = launch_rows_nt<4>(cfg, tmY, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out, la, RP, bop, LB, row_blocks,
                           hin, hscale, hs, zc, zn);
   else
-    e = launch_rows_nt<8>(cfg, Y, ldy, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out, la, RP, bop, LB, row_blocks,
+    e = launch_rows_nt<8>(cfg, tmY, M, Kin, kchunk, Z, zj, zk, r, oscale, lscale, out, la, RP, bop, LB, row_blocks,
                           hin, hscale, hs, zc, zn);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (e != cudaSuccess) {
