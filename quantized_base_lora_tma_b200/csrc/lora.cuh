@@ -901,24 +901,149 @@ __global__ void __launch_bounds__(256) lora_rows_seg_kernel(const __nv_bfloat16*
   }
 }
 
+// Bytes of shared memory of lora_rows_seg_z_kernel: the whole adapter slice [RN][Kin + 8].
+__host__ __device__ constexpr size_t rows_seg_z_smem(int NT, int Kin) { return (size_t)8 * NT * (Kin + 8) * 2; }
+
+// The grouped row products of lora_rows_seg_kernel with the expert's whole adapter slice resident
+// in shared memory ([RN][Kin + 8], k contiguous; staged once, transposed on the way in when j is the
+// contiguous index), so the stream of Y needs no barrier: each thread keeps the next 128-wide
+// chunk of its two rows in flight while it multiplies the current one. Kin % 8 == 0.
+template <int NT>
+__global__ void __launch_bounds__(256, 2) lora_rows_seg_z_kernel(
+    const __nv_bfloat16* __restrict__ Y, long ldy, int Kin, const __nv_bfloat16* __restrict__ Z, long zj, long zk,
+    long zes, const int* __restrict__ seg_off, const int* __restrict__ mblk_off, int E, int r, float oscale,
+    float lscale, float* __restrict__ out, __nv_bfloat16* __restrict__ la, int RP) {
+  constexpr int RN = 8 * NT;
+  constexpr int SK = 128;
+  extern __shared__ __align__(16) __nv_bfloat16 zsd[];
+  const int ZS = Kin + 8;
+  const int total = __ldg(mblk_off + E);
+  const int blk = blockIdx.x;
+  if (blk >= total) return;
+  int a = 0, b = E - 1;
+  while (a < b) {
+    const int mid = (a + b + 1) >> 1;
+    if (__ldg(mblk_off + mid) <= blk) a = mid; else b = mid - 1;
+  }
+  const int e = a;
+  const int row_lo = __ldg(seg_off + e) + (blk - __ldg(mblk_off + e)) * 128;
+  const int row_hi = min(__ldg(seg_off + e + 1), row_lo + 128);
+  const __nv_bfloat16* Ze = Z + (long)e * zes;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, c = lane & 3;
+  const int r0 = row_lo + warp * 16 + g, r1 = r0 + 8;
+  const bool v0 = r0 < row_hi, v1 = r1 < row_hi;
+  const __nv_bfloat16* y0 = Y + (long)(v0 ? r0 : row_lo) * ldy;
+  const __nv_bfloat16* y1 = Y + (long)(v1 ? r1 : row_lo) * ldy;
+  auto load = [&](uint4 (&xa)[SK / 32], uint4 (&xb)[SK / 32], int k0) {
+#pragma unroll
+    for (int q = 0; q < SK / 32; ++q) {
+      const int k = k0 + 32 * q + 8 * c;
+      const bool in = k < Kin;
+      xa[q] = (v0 && in) ? __ldg(reinterpret_cast<const uint4*>(y0 + k)) : make_uint4(0, 0, 0, 0);
+      xb[q] = (v1 && in) ? __ldg(reinterpret_cast<const uint4*>(y1 + k)) : make_uint4(0, 0, 0, 0);
+    }
+  };
+  // the first chunk is on its way while the adapter slice is staged
+  uint4 xa0[SK / 32], xb0[SK / 32], xa1[SK / 32], xb1[SK / 32];
+  load(xa0, xb0, 0);
+  if (zk == 1) {
+    for (int i = tid; i < RN * (Kin / 8); i += 256) {
+      const int j = i / (Kin / 8), q = i - j * (Kin / 8);
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (j < r) v = __ldg(reinterpret_cast<const uint4*>(Ze + (long)j * zj + 8 * q));
+      *reinterpret_cast<uint4*>(zsd + j * ZS + 8 * q) = v;
+    }
+  } else {
+    for (int i = tid; i < Kin * RN; i += 256) {
+      const int kk = i / RN, j = i - kk * RN;
+      zsd[j * ZS + kk] = j < r ? Ze[(long)j * zj + (long)kk * zk] : __float2bfloat16(0.f);
+    }
+  }
+  __syncthreads();
+  float acc[NT][4];
+#pragma unroll
+  for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+  auto compute = [&](const uint4 (&xa)[SK / 32], const uint4 (&xb)[SK / 32], int k0) {
+#pragma unroll
+    for (int q = 0; q < SK / 32; ++q) {
+      const int k = k0 + 32 * q + 8 * c;
+      const bool in = k < Kin;
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        const uint4 zq = in ? *reinterpret_cast<const uint4*>(zsd + (8 * t + g) * ZS + k) : make_uint4(0, 0, 0, 0);
+        mma_16816(acc[t], xa[q].x, xb[q].x, xa[q].y, xb[q].y, zq.x, zq.y);
+        mma_16816(acc[t], xa[q].z, xb[q].z, xa[q].w, xb[q].w, zq.z, zq.w);
+      }
+    }
+  };
+  for (int k0 = 0; k0 < Kin; k0 += 2 * SK) {
+    if (k0 + SK < Kin) load(xa1, xb1, k0 + SK);
+    compute(xa0, xb0, k0);
+    if (k0 + SK < Kin) {
+      if (k0 + 2 * SK < Kin) load(xa0, xb0, k0 + 2 * SK);
+      compute(xa1, xb1, k0 + SK);
+    }
+  }
+  // C fragment: rows r0 / r1, columns 8t + 2c (+1)
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int row = hh ? r1 : r0;
+      if (!(hh ? v1 : v0)) continue;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int j = 8 * t + 2 * c + q;
+        const float v = acc[t][2 * hh + q];
+        if (out != nullptr && j < r) out[(long)row * r + j] = oscale * v;
+        if (la != nullptr && j < RP) {
+          const float x = lscale * v;
+          const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+          const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+          la[(long)row * 2 * RP + j] = j < r ? hi : __float2bfloat16(0.f);
+          la[(long)row * 2 * RP + RP + j] = j < r ? lo : __float2bfloat16(0.f);
+        }
+      }
+    }
+  }
+  // padding columns of la beyond RN (RP > RN happens for r <= 16: RN = 16, RP = 32)
+  if (la != nullptr && RP > RN) {
+    for (int i = tid; i < 128 * (RP - RN); i += 256) {
+      const int lr = i / (RP - RN), j = RN + i % (RP - RN);
+      const int row = row_lo + lr;
+      if (row < row_hi) {
+        la[(long)row * 2 * RP + j] = __float2bfloat16(0.f);
+        la[(long)row * 2 * RP + RP + j] = __float2bfloat16(0.f);
+      }
+    }
+  }
+}
+
 // LB[e][n] = [Z_e(n, :) | Z_e(n, :)] zero padded to 2*RP columns; Z_e(n, j) = Z[e*zes + n*zn + j*zjs].
 // One thread per 8 output columns.
 __global__ void lora_bop_vec_kernel(const __nv_bfloat16* __restrict__ Z, long zn, long zjs, long zes, int rows, int nexp,
                                     int r, int RP, __nv_bfloat16* __restrict__ LB) {
+  // 32-bit index arithmetic (the host keeps nexp * rows * 2RP / 8 below 2^31): a 64-bit division
+  // per item would cost more than the item
   const int per_row = 2 * RP / 8;
-  const long items = (long)nexp * rows * per_row;
-  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < items; i += (long)gridDim.x * blockDim.x) {
-    const long rn = i / per_row;
-    const int j0 = (int)(i % per_row) * 8;
-    const int n = (int)(rn % rows);
-    const int e = (int)(rn / rows);
+  const int items = nexp * rows * per_row;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < items; i += gridDim.x * blockDim.x) {
+    const int rn = i / per_row;
+    const int j0 = (i - rn * per_row) * 8;
+    const int e = rn / rows;
+    const int n = rn - e * rows;
+    const int jb = j0 % RP;  // first rank column of the chunk (both halves repeat Z)
     __nv_bfloat16 v[8];
+    if (jb < r) {
+      const __nv_bfloat16* zp = Z + (long)e * zes + (long)n * zn;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int j = (j0 + q) % RP;
-      v[q] = j < r ? Z[(long)e * zes + (long)n * zn + (long)j * zjs] : __float2bfloat16(0.f);
+      for (int q = 0; q < 8; ++q) v[q] = jb + q < r ? zp[(long)(jb + q) * zjs] : __float2bfloat16(0.f);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = __float2bfloat16(0.f);
     }
-    *reinterpret_cast<uint4*>(LB + rn * 2 * RP + j0) = *reinterpret_cast<const uint4*>(v);
+    *reinterpret_cast<uint4*>(LB + (long)rn * 2 * RP + j0) = *reinterpret_cast<const uint4*>(v);
   }
 }
 
@@ -927,19 +1052,28 @@ __global__ void lora_bop_vec_kernel(const __nv_bfloat16* __restrict__ Z, long zn
 __global__ void colred_reduce_kernel(const float* __restrict__ part, int Ccols, int r, int nslices_dense,
                                      const int* __restrict__ mblk_off, int E, float scale, int transpose,
                                      float* __restrict__ out) {
+  // i runs over the output in its own order (consecutive threads write consecutive floats), with
+  // 32-bit index arithmetic (the host keeps the count below 2^31)
   const int nexp = E == 0 ? 1 : E;
-  const long total = (long)nexp * Ccols * r;
-  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total; i += (long)gridDim.x * blockDim.x) {
-    const int e = (int)(i / ((long)Ccols * r));
-    const long cj = i % ((long)Ccols * r);
+  const int per_e = Ccols * r;
+  const int total = nexp * per_e;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+    const int e = i / per_e;
+    const int w = i - e * per_e;
+    int c, j;
+    if (transpose) {
+      j = w / Ccols;
+      c = w - j * Ccols;
+    } else {
+      c = w / r;
+      j = w - c * r;
+    }
     int s0, s1;
     if (E == 0) { s0 = 0; s1 = nslices_dense; }
     else { s0 = __ldg(mblk_off + e); s1 = __ldg(mblk_off + e + 1); }
     float acc = 0.f;
-    for (int s = s0; s < s1; ++s) acc += part[(long)s * Ccols * r + cj];
-    const int c = (int)(cj / r), j = (int)(cj % r);
-    const long o = transpose ? ((long)e * r + j) * Ccols + c : ((long)e * Ccols + c) * r + j;
-    out[o] = scale * acc;
+    for (int s = s0; s < s1; ++s) acc += part[(long)s * per_e + c * r + j];
+    out[i] = scale * acc;
   }
 }
 

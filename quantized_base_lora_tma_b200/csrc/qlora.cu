@@ -471,6 +471,7 @@ static int launch_colred(const __nv_bfloat16* Y, long ldy, int Ccols, const floa
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (launch_status() != QL_OK) return QL_ERR_CUDA;
   const long total = (long)(E == 0 ? 1 : E) * Ccols * r;
+  if (total >= (1L << 31)) return QL_ERR_SHAPE;
   const int g2 = (int)std::min<long>((total + 255) / 256, 148L * 16);
   colred_reduce_kernel<<<g2, 256, 0, st>>>(part, Ccols, r, max_slices, mblk_off, E, scale, transpose, out);
   g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -759,6 +760,31 @@ static int launch_rows_seg(const __nv_bfloat16* Y, long ldy, int Kin, const __nv
                            const int* seg_off, const int* mblk, int E, int r, float oscale, float lscale, float* out,
                            __nv_bfloat16* la, int max_slices, cudaStream_t st) {
   const int RP = lora_rp(r);
+  const int NT = r <= 16 ? 2 : (r <= 32 ? 4 : 8);
+  const size_t zsm = rows_seg_z_smem(NT, Kin);
+  if (Kin % 8 == 0 && zsm <= 110 * 1024) {
+    // the expert's whole adapter slice resident in shared memory (two CTAs per SM)
+    cudaError_t e;
+    if (NT == 2) {
+      e = set_smem(lora_rows_seg_z_kernel<2>, (int)zsm);
+      if (e == cudaSuccess)
+        lora_rows_seg_z_kernel<2><<<max_slices, 256, zsm, st>>>(Y, ldy, Kin, Z, zj, zk, zes, seg_off, mblk, E, r, oscale,
+                                                                lscale, out, la, RP);
+    } else if (NT == 4) {
+      e = set_smem(lora_rows_seg_z_kernel<4>, (int)zsm);
+      if (e == cudaSuccess)
+        lora_rows_seg_z_kernel<4><<<max_slices, 256, zsm, st>>>(Y, ldy, Kin, Z, zj, zk, zes, seg_off, mblk, E, r, oscale,
+                                                                lscale, out, la, RP);
+    } else {
+      e = set_smem(lora_rows_seg_z_kernel<8>, (int)zsm);
+      if (e == cudaSuccess)
+        lora_rows_seg_z_kernel<8><<<max_slices, 256, zsm, st>>>(Y, ldy, Kin, Z, zj, zk, zes, seg_off, mblk, E, r, oscale,
+                                                                lscale, out, la, RP);
+    }
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (e != cudaSuccess) return QL_ERR_CUDA;
+    return launch_status();
+  }
   if (r <= 16)
     lora_rows_seg_kernel<2><<<max_slices, 256, 0, st>>>(Y, ldy, Kin, Z, zj, zk, zes, seg_off, mblk, E, r, oscale, lscale,
                                                         out, la, RP);
@@ -776,6 +802,7 @@ static int launch_bop_vec(const __nv_bfloat16* Z, long zn, long zjs, long zes, i
                           __nv_bfloat16* LB, cudaStream_t st) {
   const int RP = lora_rp(r);
   const long items = (long)nexp * rows * (2 * RP / 8);
+  if (items >= (1L << 31)) return QL_ERR_SHAPE;
   const int grid = (int)std::min<long>((items + 255) / 256, (long)num_sms() * 8);
   lora_bop_vec_kernel<<<grid, 256, 0, st>>>(Z, zn, zjs, zes, rows, nexp, r, RP, LB);
   g_launches.fetch_add(1, std::memory_order_relaxed);
