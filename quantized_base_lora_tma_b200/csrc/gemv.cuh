@@ -435,3 +435,224 @@ __global__ void __launch_bounds__(128) gemv_finish_kernel(const float* __restric
 }
 
 }  // namespace qlora
+
+namespace qlora {
+
+// ------------------------------------------------------------------------------------------------
+// Small-M input gradient (M <= 16, Q4_0): dX = dY deq(W) + G A with G = s dY B (from the row kernel,
+// as its split operand LA = [hi | lo]). Two launches:
+//   * qgemv_dx_kernel: persistent, stream-K over steps (k group of 256 columns of W, 128 rows of W),
+//     t = k group * NB + row block, so that a CTA's range walks down the rows of one k group (a
+//     piece) into the next. Warp w owns block w of the k group (32 columns of W = 32 outputs) and
+//     all 128 rows of a step; the reduction runs over the rows of W, so the MMA is
+//     D[k][token] += sum_n W[n][k] dY[token][n] with A = W^T (16 k x 16 rows) and B = dY^T.
+//     The k order inside an MMA tile is free: tile row g is byte 2g of the block's qs and tile row
+//     g + 8 byte 2g + 1 (low nibbles in the first k tile, high nibbles in the second), so one byte
+//     permute of two rows' byte pairs gives a word that decodes like a forward word (one shift and
+//     one LOP3 per bf16 pair, 128 + q). The row scale d[n] cannot come out of a sum over rows: it
+//     multiplies the B operand in fp32 (dY[token][n] d[n], fed as a bf16 hi + lo pair, so the
+//     whole product is fp32-accurate), and the offset (136 per weight) enters as MMAs of a
+//     constant -136 with that B. Each warp writes its 32
+//     columns of the piece's partial straight from its accumulators.
+//   * qgemv_dx_finish_kernel: per 256 columns, the k group's slots in CTA order plus G A (fp32).
+// ------------------------------------------------------------------------------------------------
+template <int MT>
+struct GvdCfg {
+  static constexpr int ROWS = 128;                        // rows of W per step
+  static constexpr int GB = QTraits<QL_Q4_0>::kGroupBytes;  // 144
+  static constexpr int W_BYTES = ROWS * GB;
+  static constexpr int XR = 8 * MT;                       // token rows of the dY tile
+  static constexpr int Y_BOX = XR * 128;                  // 64 rows of W (n) x XR tokens
+  static constexpr int Y_BYTES = 2 * Y_BOX;
+  static constexpr int STAGE = W_BYTES + Y_BYTES;
+  static constexpr int STAGES = 4;
+  static constexpr int OFF_META = STAGES * STAGE;
+  static constexpr int OFF_BAR = OFF_META + 2 * 4 * STAGES + 16;
+  static constexpr int SMEM_BYTES = OFF_BAR + 2 * STAGES * 8 + 1024;
+  static_assert(W_BYTES % 1024 == 0 && Y_BOX % 1024 == 0, "128-byte-swizzled boxes need 1 KB alignment");
+  static_assert(SMEM_BYTES <= 116 * 1024, "two CTAs per SM");
+};
+
+struct GvdParams {
+  int N, K, M;
+  uint32_t nib_mask, bf16_magic;  // 0x000F000F, 0x43004300
+  int nb, T, maxslots;            // row blocks of 128, steps, slots per k group
+  float* gpart;                   // [K/256][maxslots][XR][256] piece partials
+};
+
+template <int MT>
+__global__ void __launch_bounds__(kGvThreads, 2) qgemv_dx_kernel(const __grid_constant__ CUtensorMap tmW,
+                                                                 const __grid_constant__ CUtensorMap tmY,
+                                                                 const GvdParams p) {
+  using C = GvdCfg<MT>;
+  extern __shared__ uint8_t gvd_smem_raw[];
+  const uint32_t base_u32 = (smem_u32(gvd_smem_raw) + 1023u) & ~1023u;
+  uint8_t* smem = gvd_smem_raw + (base_u32 - smem_u32(gvd_smem_raw));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  const int G = gridDim.x;
+  const long s0 = gv_start(blockIdx.x, p.T, G), s1 = gv_start(blockIdx.x + 1, p.T, G);
+  const int nsteps = (int)(s1 - s0);
+  const uint32_t bar0 = base_u32 + C::OFF_BAR;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
+  volatile int* meta = reinterpret_cast<volatile int*>(smem + C::OFF_META);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), kGvCompute);
+    }
+    fence_mbar_init();
+  }
+  if (warp == kGvWarpP && lane == 0) {
+    prefetch_tmap(&tmW);
+    prefetch_tmap(&tmY);
+  }
+  __syncthreads();
+  // W and dY come from before the row kernel that precedes this launch (it waited for its
+  // predecessor before it let this launch start): the stream needs no wait.
+
+  bool ok = true;
+  if (warp == kGvWarpP) {
+    if (lane == 0) {
+      for (int it = 0; it < nsteps; ++it) {
+        const int s = it % C::STAGES;
+        if (it >= C::STAGES && !mbar_wait(empty_bar(s), ((it / C::STAGES) & 1) ^ 1, 45)) {
+          ok = false;
+          break;
+        }
+        if (it >= 2 && it < C::STAGES && !mbar_wait(full_bar(it - 2), 0u, 46)) {
+          ok = false;
+          break;
+        }
+        const long t = s0 + it;
+        const int kg = (int)(t / p.nb), nbk = (int)(t - (long)kg * p.nb);
+        meta[2 * s] = kg;
+        meta[2 * s + 1] = (it == 0 || nbk == 0 ? 1 : 0) | (it == nsteps - 1 || nbk == p.nb - 1 ? 2 : 0);
+        const uint32_t st = base_u32 + s * C::STAGE;
+        mbar_arrive_expect_tx(full_bar(s), C::STAGE);
+        tma_load_2d(st, &tmW, full_bar(s), kg * (C::GB / 4), nbk * C::ROWS);
+        tma_load_2d(st + C::W_BYTES, &tmY, full_bar(s), nbk * C::ROWS, 0);
+        tma_load_2d(st + C::W_BYTES + C::Y_BOX, &tmY, full_bar(s), nbk * C::ROWS + 64, 0);
+      }
+    }
+    __syncwarp();  // the idle lanes wait here, not at the final wait (which would hold lane 0)
+  } else if (warp < kGvCompute) {
+    const uint32_t nm = p.nib_mask, mg = p.bf16_magic;
+    const int b = warp;                        // block of the k group
+    const uint32_t m136 = 0xC308C308u;         // bf16 (-136, -136)
+    float acc[2][MT][4];                       // k tiles (low / high nibbles) x token tiles
+    for (int it = 0; it < nsteps; ++it) {
+      const int s = it % C::STAGES;
+      if (!warp_wait(full_bar(s), (it / C::STAGES) & 1, 47)) { ok = false; break; }
+      const int kg = meta[2 * s], fl = meta[2 * s + 1];
+      if (fl & 1) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int tt = 0; tt < MT; ++tt) acc[h][tt][0] = acc[h][tt][1] = acc[h][tt][2] = acc[h][tt][3] = 0.f;
+      }
+      const uint8_t* ws = smem + s * C::STAGE;
+      const uint8_t* ys = ws + C::W_BYTES;
+#pragma unroll 2
+      for (int nt = 0; nt < C::ROWS / 16; ++nt) {
+        // this thread's rows of W: n0 = 16 nt + 2c, n0 + 1, n0 + 8, n0 + 9 (the MMA's k columns)
+        const int n0 = 16 * nt + 2 * c;
+        const uint8_t* r0 = ws + n0 * C::GB + 18 * b;
+        const uint32_t q0 = *reinterpret_cast<const uint16_t*>(r0 + 2 + 2 * g);
+        const uint32_t q1 = *reinterpret_cast<const uint16_t*>(r0 + C::GB + 2 + 2 * g);
+        const uint32_t q2 = *reinterpret_cast<const uint16_t*>(r0 + 8 * C::GB + 2 + 2 * g);
+        const uint32_t q3 = *reinterpret_cast<const uint16_t*>(r0 + 9 * C::GB + 2 + 2 * g);
+        const float d0 = __half2float(*reinterpret_cast<const __half*>(r0));
+        const float d1 = __half2float(*reinterpret_cast<const __half*>(r0 + C::GB));
+        const float d2 = __half2float(*reinterpret_cast<const __half*>(r0 + 8 * C::GB));
+        const float d3 = __half2float(*reinterpret_cast<const __half*>(r0 + 9 * C::GB));
+        // bytes (2g, 2g + 1) of rows n0, n0 + 1 -> tile rows g, g + 8 of columns 2c, 2c + 1
+        uint32_t pa[4], pb[4];
+        gv_q4_pairs(__byte_perm(q0, q1, 0x5410), nm, mg, pa);  // pa: a0 t0, a1 t0, a0 t1, a1 t1
+        gv_q4_pairs(__byte_perm(q2, q3, 0x5410), nm, mg, pb);  // pb: a2 t0, a3 t0, a2 t1, a3 t1
+#pragma unroll
+        for (int tt = 0; tt < MT; ++tt) {
+          const int row = 8 * tt + g;  // token
+          const uint8_t* yb = ys + (n0 >> 6) * C::Y_BOX;
+          const uint32_t y01 = *reinterpret_cast<const uint32_t*>(gv_x_at(yb, row, n0 & 63));
+          const uint32_t y23 = *reinterpret_cast<const uint32_t*>(gv_x_at(yb, row, (n0 + 8) & 63));
+          const float2 f01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&y01));
+          const float2 f23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&y23));
+          // B = dY d as a bf16 hi + lo pair (fp32-accurate): the weight integers are exact, so the
+          // sum over rows carries no rounding of its own beyond fp32
+          const float e0 = f01.x * d0, e1 = f01.y * d1, e2 = f23.x * d2, e3 = f23.y * d3;
+          const uint32_t h0 = bf16x2_bits(e0, e1), h1 = bf16x2_bits(e2, e3);
+          const float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&h0));
+          const float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&h1));
+          const uint32_t l0 = bf16x2_bits(e0 - g01.x, e1 - g01.y), l1 = bf16x2_bits(e2 - g23.x, e3 - g23.y);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            mma_16816(acc[h][tt], m136, m136, m136, m136, h0, h1);
+            mma_16816(acc[h][tt], m136, m136, m136, m136, l0, l1);
+            mma_16816(acc[h][tt], pa[2 * h], pa[2 * h + 1], pb[2 * h], pb[2 * h + 1], h0, h1);
+            mma_16816(acc[h][tt], pa[2 * h], pa[2 * h + 1], pb[2 * h], pb[2 * h + 1], l0, l1);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty_bar(s));
+      if (!(fl & 2)) continue;
+      // end of a piece of k group kg: this warp's 32 columns x tokens straight to the slot.
+      // acc[h][tt]: rows (k) g, g + 8 of tile h -> columns 32b + 16h + 2g, + 1; tokens 8tt + 2c, + 1
+      const int cfirst = gv_cta_of((long)kg * p.nb, p.T, G);
+      float* gp = p.gpart + ((long)kg * p.maxslots + (blockIdx.x - cfirst)) * (C::XR * 256);
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int tt = 0; tt < MT; ++tt) {
+          const int col = 32 * b + 16 * h + 2 * g, m = 8 * tt + 2 * c;
+          *reinterpret_cast<float2*>(gp + m * 256 + col) = make_float2(acc[h][tt][0], acc[h][tt][2]);
+          *reinterpret_cast<float2*>(gp + (m + 1) * 256 + col) = make_float2(acc[h][tt][1], acc[h][tt][3]);
+        }
+    }
+  }
+  if (!ok || dev_aborted()) spin_ns(2000000ull);  // copies issued before a wait gave up land first
+  if (warp == kGvWarpL && lane == 0) {
+    pdl_wait();
+    pdl_launch_dependents();
+  }
+  pdl_wait();
+}
+
+// dX[m][k] = the k group's slots in CTA order + sum_j G[m][j] A[j][k], G = hi + lo of LA [M x 2RP];
+// one CTA per k group (256 columns).
+__global__ void __launch_bounds__(256) qgemv_dx_finish_kernel(const float* __restrict__ gpart, int maxslots, int xr,
+                                                              int nb, int T, int G, const __nv_bfloat16* __restrict__ LA,
+                                                              int RP, const __nv_bfloat16* __restrict__ A, int r, int M,
+                                                              int K, void* __restrict__ dX, int dx_dtype) {
+  __shared__ float gs[16][64];
+  pdl_wait();
+  pdl_launch_dependents();
+  for (int i = threadIdx.x; i < 16 * 64; i += blockDim.x) {
+    const int m = i >> 6, j = i & 63;
+    gs[m][j] = (m < M && j < r)
+                   ? __bfloat162float(LA[(long)m * 2 * RP + j]) + __bfloat162float(LA[(long)m * 2 * RP + RP + j])
+                   : 0.f;
+  }
+  __syncthreads();
+  const int kg = blockIdx.x;
+  const long t0 = (long)kg * nb;
+  const int cfirst = gv_cta_of(t0, T, G);
+  const int np = gv_cta_of(t0 + nb - 1, T, G) - cfirst + 1;
+  const long sz = (long)xr * 256;
+  const float* gb = gpart + (long)kg * maxslots * sz;
+  for (int i = threadIdx.x; i < M * 256; i += blockDim.x) {
+    const int m = i >> 8, kk = i & 255, k = kg * 256 + kk;
+    float y = 0.f;
+    for (int q = 0; q < np; ++q) y += gb[q * sz + m * 256 + kk];
+    float l = 0.f;
+    for (int j = 0; j < r; ++j) l = fmaf(gs[m][j], __bfloat162float(A[(long)j * K + k]), l);
+    y += l;
+    if (dx_dtype == QL_F32) reinterpret_cast<float*>(dX)[(long)m * K + k] = y;
+    else reinterpret_cast<__nv_bfloat16*>(dX)[(long)m * K + k] = __float2bfloat16_rn(y);
+  }
+}
+
+}  // namespace qlora

@@ -657,9 +657,73 @@ static int launch_gemv_fwd(int qtype, const void* wq, int64_t N, int64_t K, cons
                                           (int)M, r, scale, Y, y_dtype));
 }
 
+// Small-M input gradient (M <= 16, Q4_0): the dX weight stream, then the k-group sums with G A.
+struct GvdPlan {
+  int mt, xr, nb, groups, T, G, maxslots;
+  size_t smem, part_bytes;
+};
+static bool gemv_dx_applies(int qtype, int64_t M) { return M <= 16 && qtype == QL_Q4_0; }
+static GvdPlan gemv_dx_plan(int64_t N, int64_t K, int64_t M) {
+  GvdPlan g;
+  g.mt = M <= 8 ? 1 : 2;
+  g.xr = 8 * g.mt;
+  g.smem = g.mt == 1 ? GvdCfg<1>::SMEM_BYTES : GvdCfg<2>::SMEM_BYTES;
+  g.nb = (int)((N + 127) / 128);
+  g.groups = (int)(K / 256);
+  g.T = g.nb * g.groups;
+  const int per_sm = std::max(1, (int)(233472 / (g.smem + 1024)));
+  g.G = std::max(1, std::min(g.T, per_sm * num_sms()));
+  g.maxslots = 1;
+  for (int kg = 0; kg < g.groups; ++kg) {
+    const long t0 = (long)kg * g.nb;
+    g.maxslots = std::max(g.maxslots, gv_cta_of(t0 + g.nb - 1, g.T, g.G) - gv_cta_of(t0, g.T, g.G) + 1);
+  }
+  g.part_bytes = (size_t)g.groups * g.maxslots * g.xr * 256 * 4;
+  return g;
+}
+
+template <int MT>
+static int launch_gemv_dx_q(const CUtensorMap& tW, const CUtensorMap& tY, const GvdParams& p, int G, cudaStream_t st,
+                            int slot) {
+  using C = GvdCfg<MT>;
+  auto k = qgemv_dx_kernel<MT>;
+  if (set_smem(k, C::SMEM_BYTES) != cudaSuccess) return QL_ERR_CUDA;
+  PdlLaunch L(dim3(G), dim3(kGvThreads), C::SMEM_BYTES, st);
+  ev_record(slot, 0, st);
+  const cudaError_t e = cudaLaunchKernelEx(&L.cfg, k, tW, tY, p);
+  ev_record(slot, 1, st);
+  return launch_result(e);
+}
+
+// dX (the caller's dtype) from W, dY and the row kernel's LA = split(G); part: the plan's partials.
+static int launch_gemv_dx(const void* wq, int64_t N, int64_t K, const void* dY, int64_t M, const __nv_bfloat16* LA,
+                          int RP, const void* A, int r, void* dX, int dx_dtype, float* part, cudaStream_t st,
+                          int slot) {
+  const GvdPlan g = gemv_dx_plan(N, K, M);
+  CUtensorMap tW, tY;
+  if (!tmap_packed(&tW, wq, packed_row_bytes(QL_Q4_0, K), N, group_bytes(QL_Q4_0), 128u) ||
+      !tmap_bf16_rows(&tY, dY, N, M, (uint32_t)g.xr))
+    return QL_ERR_CUDA;
+  GvdParams p;
+  p.N = (int)N;
+  p.K = (int)K;
+  p.M = (int)M;
+  p.nib_mask = 0x000F000Fu;
+  p.bf16_magic = 0x43004300u;
+  p.nb = g.nb;
+  p.T = g.T;
+  p.maxslots = g.maxslots;
+  p.gpart = part;
+  const int rc = g.mt == 1 ? launch_gemv_dx_q<1>(tW, tY, p, g.G, st, slot) : launch_gemv_dx_q<2>(tW, tY, p, g.G, st, slot);
+  if (rc) return rc;
+  PdlLaunch L(dim3(g.groups), dim3(256), 0, st);
+  return launch_result(cudaLaunchKernelEx(&L.cfg, qgemv_dx_finish_kernel, (const float*)part, g.maxslots, g.xr, g.nb,
+                                          g.T, g.G, LA, RP, (const __nv_bfloat16*)A, r, (int)M, (int)K, dX, dx_dtype));
+}
+
 // Workspace layout of the dense layer (byte offsets, 256-aligned).
 struct LinearWs {
-  size_t la, lb, hs, split, cr, hp, total;
+  size_t la, lb, hs, split, cr, hp, dxp, total;
 };
 static LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int r) {
   LinearWs w;
@@ -677,8 +741,10 @@ static LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int r) {
     const GvPlan g = gemv_plan(QL_Q4_0, N, K, M), g8 = gemv_plan(QL_Q8_0, N, K, M);
     const size_t gv = std::max(g.hp_bytes + g.part_bytes, g8.hp_bytes + g8.part_bytes);
     w.hp = o; o = al256(o + gv);
+    w.dxp = o; o = al256(o + gemv_dx_plan(N, K, M).part_bytes);
   } else {
     w.hp = o;
+    w.dxp = o;
   }
   w.total = o;
   return w;
@@ -1180,12 +1246,18 @@ int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void
   const int ncr = (int)(colred_ctr_bytes(plan_colred(M, N, K, r)) / 4);
   // LA = split(G) with G = s dY B, HS = split(s H), and LB[k] = [A^T(k) | A^T(k)]; the column
   // reduction's counters are zeroed on the way
+  // (LB only for the tensor-core dX GEMM: the small-M dX path reads A itself)
+  const bool need_lb = dX != nullptr && !gemv_dx_applies(qtype, M);
   rc = launch_rows_dense((const __nv_bfloat16*)dY, N, (int)M, (int)N, (const __nv_bfloat16*)B, 1, r, r, scale, scale,
-                         nullptr,
-                         LA, dX ? BopArgs{(const __nv_bfloat16*)A, 1, K, (int)K} : BopArgs{nullptr, 0, 0, 0}, LB, st, H,
-                         scale, HS, (int*)crws, ncr);
+                         nullptr, LA,
+                         need_lb ? BopArgs{(const __nv_bfloat16*)A, 1, K, (int)K} : BopArgs{nullptr, 0, 0, 0}, LB, st,
+                         H, scale, HS, (int*)crws, ncr);
   if (rc) return rc;
-  if (dX) {
+  if (dX && gemv_dx_applies(qtype, M)) {
+    // weight streaming: W read once, G A added in the finish launch
+    rc = launch_gemv_dx(wq, N, K, dY, M, LA, lora_rp(r), A, r, dX, dx_dtype, (float*)(wsb + w.dxp), st, 1);
+    if (rc) return rc;
+  } else if (dX) {
     rc = launch_dense_gemm<true>(qtype, dY, M, N, wq, N, K, LA, LB, KL, K, dX, dx_dtype,
                                  (float*)(wsb + w.split), true, st, 1);
     if (rc) return rc;
