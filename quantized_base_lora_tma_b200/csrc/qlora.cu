@@ -662,12 +662,14 @@ struct GvdPlan {
   int mt, xr, nb, groups, T, G, maxslots;
   size_t smem, part_bytes;
 };
-static bool gemv_dx_applies(int qtype, int64_t M) { return M <= 16 && qtype == QL_Q4_0; }
+// (at 9..16 tokens the doubled B operand work makes it no faster than the tensor-core GEMM)
+static bool gemv_dx_applies(int qtype, int64_t M) { return M <= 8 && qtype == QL_Q4_0; }
 static GvdPlan gemv_dx_plan(int64_t N, int64_t K, int64_t M) {
+  (void)M;  // M <= 8: one token tile
   GvdPlan g;
-  g.mt = M <= 8 ? 1 : 2;
-  g.xr = 8 * g.mt;
-  g.smem = g.mt == 1 ? GvdCfg<1>::SMEM_BYTES : GvdCfg<2>::SMEM_BYTES;
+  g.mt = 1;
+  g.xr = 8;
+  g.smem = GvdCfg<1>::SMEM_BYTES;
   g.nb = (int)((N + 127) / 128);
   g.groups = (int)(K / 256);
   g.T = g.nb * g.groups;
@@ -714,7 +716,7 @@ static int launch_gemv_dx(const void* wq, int64_t N, int64_t K, const void* dY, 
   p.T = g.T;
   p.maxslots = g.maxslots;
   p.gpart = part;
-  const int rc = g.mt == 1 ? launch_gemv_dx_q<1>(tW, tY, p, g.G, st, slot) : launch_gemv_dx_q<2>(tW, tY, p, g.G, st, slot);
+  const int rc = launch_gemv_dx_q<1>(tW, tY, p, g.G, st, slot);
   if (rc) return rc;
   PdlLaunch L(dim3(g.groups), dim3(256), 0, st);
   return launch_result(cudaLaunchKernelEx(&L.cfg, qgemv_dx_finish_kernel, (const float*)part, g.maxslots, g.xr, g.nb,
