@@ -266,17 +266,6 @@ static int launch_qgemm2_q(int qtype, const CUtensorMap& tA, const CUtensorMap& 
   }
 }
 
-// Split-K configuration of the row reductions (H = X A^T, G = s dY B).
-static void rows_split(int M, int Kin, int ks_cap, int* KS, int* kchunk) {
-  const int mblocks = (M + 63) / 64;
-  int ks = (4 * 148 + mblocks - 1) / mblocks;
-  ks = std::max(1, std::min(std::min(ks, ks_cap), std::min(16, Kin / 256)));
-  int kc = (Kin + ks - 1) / ks;
-  kc = (kc + 15) / 16 * 16;
-  *kchunk = kc;
-  *KS = (Kin + kc - 1) / kc;
-}
-
 // Dense row reduction with the in-cluster split-K sum: out = oscale * Y Z^T, la = split(lscale *
 // Y Z^T), optionally hs = split(hscale * hin) for the same rows, and, in the same launch,
 // LB = [Zb | Zb] (bop).
