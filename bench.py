@@ -169,13 +169,21 @@ class DenseLayerRun:
         self.dA = torch.empty(r, K, dtype=torch.float32, device="cuda")
         self.dB = torch.empty(N, r, dtype=torch.float32, device="cuda")
 
-    def step(self, X=None, dY=None):
+    def fwd(self, X=None):
+        c, ql = self.c, self.ql
+        X = self.X if X is None else X
+        ql.qlora_linear_fwd(c.qtype, self.wq, c.N, c.K, X, self.A, self.B, c.r, c.scale, self.Y, self.H, self.ws)
+
+    def bwd(self, X=None, dY=None):
         c, ql = self.c, self.ql
         X = self.X if X is None else X
         dY = self.dY if dY is None else dY
-        ql.qlora_linear_fwd(c.qtype, self.wq, c.N, c.K, X, self.A, self.B, c.r, c.scale, self.Y, self.H, self.ws)
         ql.qlora_linear_bwd(c.qtype, self.wq, c.N, c.K, X, dY, self.A, self.B, c.r, c.scale, self.H, self.dX,
                             self.dA, self.dB, self.ws)
+
+    def step(self, X=None, dY=None):
+        self.fwd(X)
+        self.bwd(X, dY)
 
     def flops(self):
         c = self.c
@@ -395,14 +403,24 @@ def run_ours(args, rank, world, local_rank):
     Xd = torch.empty_like(run.X)
     dYd = torch.empty_like(run.dY)
     e2e_ms = []
+    # X first on the compute stream; dY on a copy stream once X is in, so that its transfer
+    # overlaps the forward; the backward waits for it
+    copy_stream = torch.cuda.Stream()
     for i in range(E + 2):
         flush.zero_()
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev_x, ev_dy = torch.cuda.Event(), torch.cuda.Event()
         a.record(stream)
         Xd.copy_(X_h, non_blocking=True)
-        dYd.copy_(dY_h, non_blocking=True)
-        run.step(Xd, dYd)
+        ev_x.record(stream)
+        copy_stream.wait_event(ev_x)
+        with torch.cuda.stream(copy_stream):
+            dYd.copy_(dY_h, non_blocking=True)
+        ev_dy.record(copy_stream)
+        run.fwd(Xd)
+        stream.wait_event(ev_dy)
+        run.bwd(Xd, dYd)
         allreduce_grads()
         dA_h.copy_(run.dA, non_blocking=True)
         dB_h.copy_(run.dB, non_blocking=True)
