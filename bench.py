@@ -551,15 +551,16 @@ def run_reference(args, rank, world):
     }
 
 
-def decode_calls(M, calls=3):
-    """Three forward calls of the decode-shaped linear (the launch a profiler captures)."""
+def decode_calls(M, calls=3, bwd=False):
+    """Three forward (and, with bwd, backward) calls of the decode-shaped linear (the launches a
+    profiler captures)."""
     import quantized_base_lora_tma_b200 as ql
     from quantized_base_lora_tma_b200 import build
     build.build()
     c = inp.decode_q4_0_8192(M)
     d = DenseLayerRun(c)
     for _ in range(calls):
-        ql.qlora_linear_fwd(c.qtype, d.wq, c.N, c.K, d.X, d.A, d.B, c.r, c.scale, d.Y, d.H, d.ws)
+        d.fwd() if not bwd else d.step()
     device_status_ok(f"decode M={M}")
 
 
@@ -577,10 +578,11 @@ def main():
     ap.add_argument("--decode-calls", type=int, default=0, metavar="M",
                     help="profiling driver: run the decode-shaped Q4_0 8192x8192 forward with M tokens "
                          "three times and exit (no timing, no JSON line)")
+    ap.add_argument("--decode-bwd", action="store_true", help="with --decode-calls: forward and backward")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.decode_calls:
-        decode_calls(args.decode_calls)
+        decode_calls(args.decode_calls, bwd=args.decode_bwd)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

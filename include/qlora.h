@@ -72,6 +72,13 @@ uint64_t qlora_launch_count(void);
  * thread-safe with concurrent calls that launch into the same slot. */
 int qlora_set_kernel_events(int slot, void* start, void* stop);
 
+/* Which of the dense linear's pair GEMMs may compute the adapter row products (H = X A^T in the
+ * forward, G = s dY B in the input gradient, and the operands built from them) inside their own
+ * launch, on the SM pairs their tiles leave idle, instead of in a separate launch before them: bit 0
+ * the forward GEMM, bit 1 the input-gradient GEMM (default 1). Either way the results obey the same
+ * bounds. Process-wide; returns the previous mask. */
+int qlora_set_rows_fusion(int mask);
+
 /* Reads the device status word of the current device (synchronises the device first). Returns
  * QL_OK or the first recorded device-side error (QL_ERR_TIMEOUT); *site (nullable) receives the
  * code of the wait that gave up. reset != 0 clears the word afterwards. */

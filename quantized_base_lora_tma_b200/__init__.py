@@ -8,5 +8,6 @@ from ._lib import (Q4_0, Q4_K, Q8_0, QL_BF16, QL_F32, QloraError, gguf_dequant, 
                    qlora_device_status, qlora_launch_count, qlora_linear_bwd, qlora_linear_fwd,
                    qlora_linear_fwd_noalloc,
                    qlora_linear_workspace_bytes, qlora_selftest_wait_timeout, qlora_set_kernel_events,
+                   qlora_set_rows_fusion,
                    qlora_status_string, MoeRoute, qlora_moe_route, qlora_moe_saved_bytes,
                    qlora_moe_workspace_bytes, qlora_moe_fwd, qlora_moe_bwd)

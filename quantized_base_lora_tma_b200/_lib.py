@@ -32,6 +32,7 @@ SIGNATURES = {
     "qlora_launch_count": (ctypes.c_uint64, []),
     "qlora_device_status": (_c_int, [ctypes.POINTER(_c_int), _c_int]),
     "qlora_set_kernel_events": (_c_int, [_c_int, _c_vp, _c_vp]),
+    "qlora_set_rows_fusion": (_c_int, [_c_int]),
     "qlora_selftest_wait_timeout": (_c_int, [_c_i64, _c_vp]),
     "gguf_dequant": (_c_int, [_c_int, _c_vp, _c_i64, _c_i64, _c_vp, _c_int, _c_vp]),
     "qlora_linear_workspace_bytes": (_c_sz, [_c_i64, _c_i64, _c_i64, _c_int]),
@@ -122,6 +123,13 @@ def qlora_device_status(reset: bool = False):
     site = _c_int(0)
     rc = lib().qlora_device_status(ctypes.byref(site), 1 if reset else 0)
     return rc, site.value
+
+
+def qlora_set_rows_fusion(mask) -> int:
+    """Which dense pair GEMMs compute the adapter row products in their own launch: bit 0 the
+    forward, bit 1 the input gradient (True = both, False = neither); returns the previous mask."""
+    m = 3 if mask is True else (0 if mask is False else int(mask))
+    return int(lib().qlora_set_rows_fusion(m))
 
 
 def qlora_set_kernel_events(slot: int, start=None, stop=None):

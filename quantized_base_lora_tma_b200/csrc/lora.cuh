@@ -502,6 +502,8 @@ struct ColredFlow {
   int defer_wait;  // 1: the previous kernel in the stream already waited for this launch's inputs
   float* part;     // [nblk * csu][16 JT][128]
   int* ctr;        // [0]: next unit to claim, [1 + b]: chunks of block b finished; zero at launch
+  const int* gate; // with defer_wait: a count of the previous launch that reaches gate_target once
+  int gate_target; // the split operands and the zeroed counters are written (nullable)
 };
 
 constexpr int kColTmaStagesMax = 6;
@@ -601,7 +603,11 @@ __global__ void __launch_bounds__(32 * kColWarps) colred_flow_kernel(const __gri
 
   bool ok = true;
   if (warp == 8) {
-    if (lane == 0) {
+    if (lane == 0 && P.gate != nullptr) {
+      ok = wait_count(P.gate, P.gate_target, 65);
+      fence_proxy_async_global();
+    }
+    if (lane == 0 && ok) {
       int it = 0;
       int u = atomicAdd(P.ctr, 1);
       while (true) {

@@ -198,6 +198,43 @@ __device__ __forceinline__ void cluster_arrive_wait() {
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// The same for global memory: generic-proxy writes (or reads acquired from another CTA) ordered
+// against this thread's later TMA copies.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// ------------------------------------------------------------------------------------------------
+// Counters between CTAs of one grid, or towards a later launch: a producer CTA makes its global
+// writes visible (every writer fences, a CTA barrier, then one thread's release add); a consumer
+// thread acquires the count and fences before its TMA copies read the data. The producers are
+// CTAs of lower index in the same launch (dispatched no later than the waiters, and waiting on
+// nothing themselves) or of an earlier launch, so every wait ends; it is bounded all the same.
+// ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void release_add_gpu(int* p, int v) {
+  __threadfence();
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ bool wait_count(const int* p, int target, int site) {
+  if (ld_acquire_gpu(p) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  uint32_t polls = 0;
+  while (true) {
+    __nanosleep(500);
+    if (ld_acquire_gpu(p) >= target) return true;
+    ++polls;
+    if (dev_aborted()) return false;
+    if (polls >= 16u && globaltimer_ns() - t0 > kWaitLimitNs) {
+      dev_fail(QL_ERR_TIMEOUT, site);
+      return false;
+    }
+  }
+}
 
 // ------------------------------------------------------------------------------------------------
 // TMA (tiled, no multicast)

@@ -39,6 +39,29 @@ constexpr int kWarpDq0 = 7;
 constexpr int kNumDqWarps = 16;  // two groups of eight, taking alternate stages
 constexpr int kGemmThreads = (kWarpDq0 + kNumDqWarps) * 32;  // 736
 
+// Adapter row products computed inside a dense pair-GEMM launch, by the clusters the tiles leave
+// idle (see gemm2_rows_role): out = oscale Y Z^T and la = split(lscale Y Z^T) for the GEMM's A
+// operand Y, plus LB and hs, with counters the LoRA k-blocks (and a later column reduction) wait on.
+struct RowsFuse {
+  int r, RP, nt;               // rank, padded rank (LA / LB are 2RP wide), 8-column tiles of Z^T
+  int ztr;                     // the adapter box is [k][j] (j contiguous) rather than [j][k]
+  int stages;                  // TMA ring depth
+  float oscale, lscale;
+  float* out;                  // fp32 [M x r] (nullable)
+  __nv_bfloat16* la;           // [M x 2RP] = [hi | lo]
+  const __nv_bfloat16* lbz;    // LB[n] = [Z(n, :) | Z(n, :)], Z(n, j) = lbz[n lbzn + j lbzj] (nullable)
+  long lbzn, lbzj;
+  int lb_rows;
+  __nv_bfloat16* lb;
+  const float* hin;            // hs = split(hscale hin), [M x 2RP] (nullable)
+  float hscale;
+  __nv_bfloat16* hs;
+  int* ctr;  // [0] CTAs whose LB / hs share is written, [1] CTAs done, [2 + mb] 128-row blocks of
+             // M block mb written; zero at launch
+  int* zc;   // counters of a later launch, zeroed here (nullable)
+  int zn;
+};
+
 struct GemmParams {
   int M;           // rows of the A operand (tokens; routed pairs in grouped mode)
   int Nd;          // output columns
@@ -70,6 +93,10 @@ struct GemmParams {
   const __nv_bfloat16* in_h;
   const float* row_w;          // PAIR_OUT, SWIGLU_BWD: routing weight per row
   float* dw_part;              // SWIGLU_BWD: [M x num_n_tiles] partial <dh_u, h>
+  // dense pair GEMM: clusters [0, rx) compute the adapter row products (0 = none: the LoRA
+  // operands are the previous launch's output)
+  int rx;
+  RowsFuse rf;
 };
 
 // BN = 128 or 256 output columns per tile. With BN = 256 every A tile feeds twice the columns and

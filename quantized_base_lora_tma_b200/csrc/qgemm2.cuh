@@ -21,6 +21,7 @@
 //   tfull[b]  each CTA: one pair commit arriving on both; tempty[b] leader: 4 + 4 epilogue warps
 // Every wait is bounded (ptx.cuh); both CTAs always reach the final cluster barrier.
 #pragma once
+#include "lora.cuh"
 #include "qgemm.cuh"
 
 namespace qlora {
@@ -87,23 +88,177 @@ __device__ __forceinline__ bool gemm2_tile(const GemmParams& p, int t, TileInfo&
   return true;
 }
 
+// ---------------- adapter row products inside the GEMM's launch ----------------
+// The pair tiles of a dense GEMM often leave SM pairs idle (64 tiles of 512 x 256 on 74 pairs).
+// In a fused launch the first rx clusters take those SMs and compute, for the GEMM's own A operand
+// Y (X in the forward, dY in the input gradient), out = oscale Y Z^T and la = split(lscale Y Z^T)
+// by 128-row blocks, plus LB and hs, while the tiles' main loops run; the tiles' LoRA k-blocks
+// come last and wait for the counters. Every CTA first writes its share of LB and hs, then streams
+// its blocks through a TMA ring: Y's 128 x 64 boxes (the GEMM's tensor map) and the adapter's
+// 64-wide boxes (tmZ: RN x 64 with 128-byte swizzle for Z stored [j][k], or 64 x RN unswizzled
+// for Z stored [k][j]). Warps 0..7 own 16 rows each (ldmatrix, mma.sync, fp32 accumulation over
+// the whole k range in order), warp 8 lane 0 produces.
+template <int NT>
+__device__ __forceinline__ constexpr int rows_fuse_stage_bytes() {
+  return 128 * 128 + 8 * NT * 128;
+}
+template <int NT, int MS>
+__device__ __noinline__ void gemm2_rows_role(const CUtensorMap* tmY, const CUtensorMap* tmZ, const GemmParams& p, uint32_t base) {
+  const RowsFuse& f = p.rf;
+  constexpr int RN = 8 * NT;
+  constexpr int XB = 128 * 128;
+  constexpr int SB = rows_fuse_stage_bytes<NT>();
+  const int S = f.stages;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int cta = blockIdx.x, ncta = 2 * p.rx;
+  pdl_wait();  // Y and the adapters may be the previous launch's output
+  pdl_launch_dependents();
+  if (cta == 0 && f.zc != nullptr)
+    for (int i = tid; i < f.zn; i += blockDim.x) f.zc[i] = 0;
+  lora_bop_share(BopArgs{f.lbz, f.lbzn, f.lbzj, f.lb_rows}, f.r, f.RP, f.lb, cta, ncta);
+  if (f.hs != nullptr)
+    for (long i = (long)cta * blockDim.x + tid; i < (long)p.M * f.RP; i += (long)ncta * blockDim.x) {
+      const long m = i / f.RP;
+      const int j = (int)(i % f.RP);
+      const float x = j < f.r ? f.hscale * f.hin[m * f.r + j] : 0.f;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+      f.hs[m * 2 * f.RP + j] = hi;
+      f.hs[m * 2 * f.RP + f.RP + j] = __float2bfloat16_rn(x - __bfloat162float(hi));
+    }
+  fence_proxy_async_global();
+  const uint32_t bar0 = base + (uint32_t)(S * SB);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 8);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0) release_add_gpu(f.ctr, 1);  // this CTA's LB and hs share is out
+
+  const int nblk = (p.M + 127) / 128;
+  const int ksteps = p.Kd / kBK;
+  if (warp == 8) {
+    if (lane == 0) {
+      prefetch_tmap(tmY);
+      prefetch_tmap(tmZ);
+      int it = 0;
+      bool ok = true;
+      for (int b = cta; ok && b < nblk; b += ncta)
+        for (int kt = 0; kt < ksteps; ++kt, ++it) {
+          const int s = it % S;
+          if (!mbar_wait(empty_bar(s), ((it / S) & 1) ^ 1, 61)) {
+            ok = false;
+            break;
+          }
+          const uint32_t st = base + (uint32_t)(s * SB);
+          mbar_arrive_expect_tx(full_bar(s), (uint32_t)SB);
+          tma_load_2d(st, tmY, full_bar(s), kt * kBK, b * 128);
+          if (f.ztr) tma_load_2d(st + XB, tmZ, full_bar(s), 0, kt * kBK);
+          else tma_load_2d(st + XB, tmZ, full_bar(s), kt * kBK, 0);
+        }
+      if (!ok && it > 0) spin_ns(2000000ull);  // copies in flight land before the CTA exits
+    }
+  } else if (warp < 8) {
+    const int a_row = 16 * warp + (lane & 15), a_col = 8 * (lane >> 4);
+    const int b_row = (lane & 7) + 8 * (lane >> 4), b_col = 8 * ((lane >> 3) & 1);
+    const int t_k = (lane & 7) + 8 * ((lane >> 3) & 1), t_j = 8 * (lane >> 4);
+    const int g = lane >> 2, c = lane & 3;
+    // after a failed wait a warp skips the work but keeps taking the same named-barrier steps
+    int it = 0;
+    bool ok = true;
+    for (int b = cta; b < nblk; b += ncta) {
+      float acc[NT][4];
+#pragma unroll
+      for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+      for (int kt = 0; ok && kt < ksteps; ++kt, ++it) {
+        const int s = it % S;
+        if (!warp_wait(full_bar(s), (it / S) & 1, 62)) {
+          ok = false;
+          break;
+        }
+        const uint32_t xs = base + (uint32_t)(s * SB), zs = xs + XB;
+#pragma unroll
+        for (int k16 = 0; k16 < kBK / 16; ++k16) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(sw128_addr(xs, a_row, 16 * k16 + a_col), a0, a1, a2, a3);
+#pragma unroll
+          for (int tp = 0; tp < NT / 2; ++tp) {
+            uint32_t b0, b1, b2, b3;
+            if (f.ztr) ldsm_x4_t(zs + (uint32_t)(((16 * k16 + t_k) * RN + 16 * tp + t_j) * 2), b0, b1, b2, b3);
+            else ldsm_x4(sw128_addr(zs, 16 * tp + b_row, 16 * k16 + b_col), b0, b1, b2, b3);
+            mma_16816(acc[2 * tp], a0, a1, a2, a3, b0, b1);
+            mma_16816(acc[2 * tp + 1], a0, a1, a2, a3, b2, b3);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty_bar(s));
+      }
+      // rows 16 warp + g and + 8 of the block: out, and la = [hi | lo] zero past r
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int m = b * 128 + 16 * warp + g + 8 * h;
+        if (!ok || m >= p.M) continue;
+        __nv_bfloat16* lam = f.la + (long)m * 2 * f.RP;
+#pragma unroll
+        for (int t = 0; t < NT; ++t)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int j = 8 * t + 2 * c + e;
+            if (j >= f.RP) continue;
+            const float v = acc[t][2 * h + e];
+            if (f.out != nullptr && j < f.r) f.out[(long)m * f.r + j] = f.oscale * v;
+            const float x = j < f.r ? f.lscale * v : 0.f;
+            const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+            lam[j] = hi;
+            lam[f.RP + j] = __float2bfloat16_rn(x - __bfloat162float(hi));
+          }
+        for (int j = RN + c; j < f.RP; j += 4) {
+          lam[j] = __float2bfloat16(0.f);
+          lam[f.RP + j] = __float2bfloat16(0.f);
+        }
+      }
+      fence_proxy_async_global();
+      asm volatile("bar.sync 1, 256;" ::: "memory");  // the eight row warps
+      if (tid == 0 && !dev_aborted()) release_add_gpu(f.ctr + 2 + b / (2 * MS), 1);
+    }
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    if (tid == 0 && !dev_aborted()) release_add_gpu(f.ctr + 1, 1);
+  }
+}
+
 template <int QT, bool TRANS, int MS>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm2Threads, 1)
     qgemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
                   const __grid_constant__ CUtensorMap tmLA, const __grid_constant__ CUtensorMap tmLB,
-                  const GemmParams p) {
+                  const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ GemmParams p) {
   using C = Gemm2Cfg<QT, TRANS, MS>;
   constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw_[];
   const uint32_t base_u32 = (smem_u32(smem_raw_) + 1023u) & ~1023u;
   uint8_t* smem = smem_raw_ + (base_u32 - smem_u32(smem_raw_));
 
+  if ((int)(blockIdx.x >> 1) < p.rx) {  // a cluster of the fused adapter row products
+    if (p.rf.nt == 2) gemm2_rows_role<2, MS>(&tmA, &tmZ, p, base_u32);
+    else if (p.rf.nt == 4) gemm2_rows_role<4, MS>(&tmA, &tmZ, p, base_u32);
+    else gemm2_rows_role<8, MS>(&tmA, &tmZ, p, base_u32);
+    return;
+  }
+  if (p.rx > 0) {
+    // fused: A and W may be the previous launch's output too
+    pdl_wait();
+    pdl_launch_dependents();
+  }
+
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cta_rank_in_cluster();  // 0 = leader
   const bool leader = rank == 0;
-  const int cid = blockIdx.x >> 1;
-  const int ncl = gridDim.x >> 1;
+  const int cid = (int)(blockIdx.x >> 1) - p.rx;  // tile clusters follow the row clusters
+  const int ncl = (int)(gridDim.x >> 1) - p.rx;
 
   const uint32_t sA = base_u32 + C::OFF_A;
   const uint32_t sB = base_u32 + C::OFF_B;
@@ -148,11 +303,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm2Threads, 1)
   cluster_arrive_wait();  // both CTAs' barriers exist before any cross-CTA arrival
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
-  // A and W come from before the previous kernel in the stream (the row kernel, which waited for
-  // its own predecessor before it let this launch start), so the main loop streams them at once;
-  // only the LoRA operands are that kernel's output: the A producer waits for it before their
-  // first copy, and epilogue warp 0 waits for it before it lets the next launch start (which may
-  // rely on what this launch waited for) and so that this launch completes only after it.
+  // Unfused, A and W come from before the previous kernel in the stream (the row kernel, which
+  // waited for its own predecessor before it let this launch start), so the main loop streams them
+  // at once; only the LoRA operands are that kernel's output: the A producer waits for it before
+  // their first copy, and epilogue warp 0 waits for it before it lets the next launch start (which
+  // may rely on what this launch waited for) and so that this launch completes only after it.
+  // Fused, everything waited above, and the A producer waits for the row clusters' counters
+  // (LB and hs shares, then the 128-row blocks of the tile's M block) before the LoRA copies.
 
   const int kb_main = p.Kd / kBK;
   auto tile_steps = [&](const TileInfo& ti) { return (ti.kb_hi - ti.kb_lo) + (ti.lora ? p.n_lora_kb : 0); };
@@ -171,10 +328,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm2Threads, 1)
       bool ok = true;
       bool issued = false;
       bool waited = false;
+      int mb_ready = -1;
       TileInfo ti;
       for (int t = cid; ok && gemm2_tile<C::BM>(p, t, ti); t += ncl) {
         const int nsteps = tile_steps(ti);
         const int arow = ti.row0 + 128 * (int)rank;
+        const int mb = ti.row0 / C::BM;
         for (int i = 0; i < nsteps; ++i, ++it) {
           const int kb = step_kb(ti, i);
           const int s = it % C::STAGES;
@@ -188,8 +347,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm2Threads, 1)
               tma_load_2d_pair(sA + s * C::A_BYTES + h * 16384, &tmA, fb, kb * kBK, arow + 256 * h);
           } else {
             if (!waited) {
-              pdl_wait();  // the LoRA operands are the previous kernel's output
+              if (p.rx == 0) pdl_wait();  // the LoRA operands are the previous kernel's output
+              else if (!wait_count(p.rf.ctr, 2 * p.rx, 63)) { ok = false; break; }
               waited = true;
+            }
+            if (p.rx > 0 && mb != mb_ready) {
+              const int blocks = min(2 * MS, (p.M + 127) / 128 - 2 * MS * mb);
+              if (!wait_count(p.rf.ctr + 2 + mb, blocks, 64)) { ok = false; break; }
+              fence_proxy_async_global();
+              mb_ready = mb;
             }
             const int x = (kb - kb_main) * kBK;
             if (leader) mbar_arrive_expect_tx(full_bar(s), 2 * (C::A_BYTES + C::B_BYTES));

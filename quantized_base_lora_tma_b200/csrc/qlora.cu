@@ -220,13 +220,12 @@ static int grouped_bn(int qtype, int64_t cols, int64_t div256) {
 // Pair-tile dense GEMM: clusters of two CTAs, one cluster per pair tile slot. The grid is capped at
 // the number of clusters that can be resident at once (a persistent kernel must never have CTAs
 // waiting for a free SM pair).
+// Clusters of the pair GEMM that are resident at once (cached per device; 0 on error).
 template <int QT, bool TRANS, int MS>
-static int launch_qgemm2(const CUtensorMap& tA, const CUtensorMap& tW, const CUtensorMap& tLA, const CUtensorMap& tLB,
-                         const GemmParams& p, int tiles, cudaStream_t st, int slot) {
+static int qgemm2_max_clusters() {
   using C = Gemm2Cfg<QT, TRANS, MS>;
   auto k = qgemm2_kernel<QT, TRANS, MS>;
-  if (set_smem(k, C::SMEM_BYTES) != cudaSuccess)
-    return QL_ERR_CUDA;
+  if (set_smem(k, C::SMEM_BYTES) != cudaSuccess) return 0;
   static int max_clusters[16] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -244,25 +243,54 @@ static int launch_qgemm2(const CUtensorMap& tA, const CUtensorMap& tW, const CUt
     cfg.attrs = at;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, k, &cfg) != cudaSuccess || n <= 0) return QL_ERR_CUDA;
+    if (cudaOccupancyMaxActiveClusters(&n, k, &cfg) != cudaSuccess || n <= 0) return 0;
     mc = n;
   }
-  const int clusters = std::min(tiles, mc);
+  return mc;
+}
+
+// With p.rx row clusters (fused adapter row products) in front of the tile clusters.
+template <int QT, bool TRANS, int MS>
+static int launch_qgemm2(const CUtensorMap& tA, const CUtensorMap& tW, const CUtensorMap& tLA, const CUtensorMap& tLB,
+                         const CUtensorMap& tZ, const GemmParams& p, int tiles, cudaStream_t st, int slot) {
+  using C = Gemm2Cfg<QT, TRANS, MS>;
+  auto k = qgemm2_kernel<QT, TRANS, MS>;
+  const int mc = qgemm2_max_clusters<QT, TRANS, MS>();
+  if (mc <= p.rx) return QL_ERR_CUDA;
+  const int clusters = p.rx + std::min(tiles, mc - p.rx);
   PdlLaunch L(dim3(2 * clusters), dim3(kGemm2Threads), C::SMEM_BYTES, st);  // cluster shape from the kernel
   ev_record(slot, 0, st);
-  const cudaError_t e = cudaLaunchKernelEx(&L.cfg, k, tA, tW, tLA, tLB, p);
+  const cudaError_t e = cudaLaunchKernelEx(&L.cfg, k, tA, tW, tLA, tLB, tZ, p);
   ev_record(slot, 1, st);
   return launch_result(e);
 }
 
 template <bool TRANS, int MS>
 static int launch_qgemm2_q(int qtype, const CUtensorMap& tA, const CUtensorMap& tW, const CUtensorMap& tLA,
-                           const CUtensorMap& tLB, const GemmParams& p, int tiles, cudaStream_t st, int slot) {
+                           const CUtensorMap& tLB, const CUtensorMap& tZ, const GemmParams& p, int tiles,
+                           cudaStream_t st, int slot) {
   switch (qtype) {
-    case QL_Q8_0: return launch_qgemm2<QL_Q8_0, TRANS, MS>(tA, tW, tLA, tLB, p, tiles, st, slot);
-    case QL_Q4_0: return launch_qgemm2<QL_Q4_0, TRANS, MS>(tA, tW, tLA, tLB, p, tiles, st, slot);
-    case QL_Q4_K: return launch_qgemm2<QL_Q4_K, TRANS, MS>(tA, tW, tLA, tLB, p, tiles, st, slot);
+    case QL_Q8_0: return launch_qgemm2<QL_Q8_0, TRANS, MS>(tA, tW, tLA, tLB, tZ, p, tiles, st, slot);
+    case QL_Q4_0: return launch_qgemm2<QL_Q4_0, TRANS, MS>(tA, tW, tLA, tLB, tZ, p, tiles, st, slot);
+    case QL_Q4_K: return launch_qgemm2<QL_Q4_K, TRANS, MS>(tA, tW, tLA, tLB, tZ, p, tiles, st, slot);
     default: return QL_ERR_UNSUPPORTED;
+  }
+}
+template <bool TRANS, int MS>
+static int qgemm2_max_clusters_q(int qtype) {
+  switch (qtype) {
+    case QL_Q8_0: return qgemm2_max_clusters<QL_Q8_0, TRANS, MS>();
+    case QL_Q4_0: return qgemm2_max_clusters<QL_Q4_0, TRANS, MS>();
+    case QL_Q4_K: return qgemm2_max_clusters<QL_Q4_K, TRANS, MS>();
+    default: return 0;
+  }
+}
+template <bool TRANS, int MS>
+static int qgemm2_smem_q(int qtype) {
+  switch (qtype) {
+    case QL_Q8_0: return Gemm2Cfg<QL_Q8_0, TRANS, MS>::SMEM_BYTES;
+    case QL_Q4_0: return Gemm2Cfg<QL_Q4_0, TRANS, MS>::SMEM_BYTES;
+    default: return Gemm2Cfg<QL_Q4_K, TRANS, MS>::SMEM_BYTES;
   }
 }
 
@@ -405,9 +433,12 @@ static cudaError_t launch_colred_jt(cudaLaunchConfig_t& cfg, const CUtensorMap* 
 
 // crws: the plan's workspace (counters zeroed by an earlier kernel of the same stream, then
 // partials). defer_wait: the previous kernel in the stream waited for this launch's inputs itself.
+// gate: with defer_wait, a count of the previous launch's that reaches gate_target once the inputs
+// Z0 and Z1 (and the zeroed counters) are written; the producer waits for it before its first claim.
 static int launch_colred_dense(const __nv_bfloat16* Y0, int C0, const __nv_bfloat16* Z0, const ColredOut& o0,
                                const __nv_bfloat16* Y1, int C1, const __nv_bfloat16* Z1, const ColredOut& o1, int M, int r,
-                               uint8_t* crws, int defer_wait, cudaStream_t st) {
+                               uint8_t* crws, int defer_wait, cudaStream_t st, const int* gate = nullptr,
+                               int gate_target = 0) {
   const int RP = lora_rp(r);
   const int JT = (r + 15) / 16;
   CUtensorMap tm[4];
@@ -429,6 +460,8 @@ static int launch_colred_dense(const __nv_bfloat16* Y0, int C0, const __nv_bfloa
   P.defer_wait = defer_wait;
   P.ctr = reinterpret_cast<int*>(crws);
   P.part = reinterpret_cast<float*>(crws + al256(colred_ctr_bytes(pl)));
+  P.gate = gate;
+  P.gate_target = gate_target;
   const size_t smem = colred_smem_bytes(RP, JT, pl.tr);
   const int per_sm = std::max(1, (int)(233472 / (smem + 1024)));
   const int grid = std::min(pl.nblk * pl.csu, per_sm * num_sms());
@@ -512,13 +545,42 @@ static int launch_split_reduce(const float* part, int ksplit, long stride, long 
 }
 
 
+// Which dense pair GEMMs compute the adapter row products in their own launch when they can
+// (qlora_set_rows_fusion): bit 0 the forward, bit 1 the input gradient. The input gradient is not
+// fused by default: there the column reductions that follow need the SMs the row clusters hold.
+static std::atomic<int> g_rows_fusion{1};
+
+// Row clusters of a fused dense pair GEMM (0: the row kernel runs before the GEMM). The tiles take
+// one wave of clusters and leave at least one idle; the row clusters take the idle ones, as many as
+// give every CTA one 128-row block, and fusion is used only when no CTA gets more than three (so
+// the row products end well before the tiles' main loops). The input-gradient direction stages the
+// adapter B [N x r] by TMA, whose rows must be a multiple of 16 bytes: r % 8 == 0.
+static int dense_fuse_rx(int qtype, int64_t M, int64_t Nd, int64_t Kd, bool trans, int r) {
+  if (!(g_rows_fusion.load(std::memory_order_relaxed) & (trans ? 2 : 1))) return 0;
+  const DensePlan d = plan_dense(M, Nd, Kd, trans, true);
+  if (d.ms == 0 || d.ksplit != 1) return 0;
+  if (trans && r % 8 != 0) return 0;
+  const int mc = trans ? (d.ms == 2 ? qgemm2_max_clusters_q<true, 2>(qtype) : qgemm2_max_clusters_q<true, 1>(qtype))
+                       : (d.ms == 2 ? qgemm2_max_clusters_q<false, 2>(qtype) : qgemm2_max_clusters_q<false, 1>(qtype));
+  const int idle = mc - d.mblocks * d.ntiles;
+  const int nblk = (int)((M + 127) / 128);
+  const int rx = std::min(idle, (nblk + 1) / 2);
+  if (rx < 1 || (nblk + 2 * rx - 1) / (2 * rx) > 3) return 0;
+  return rx;
+}
+// Counters of a fused launch: [0], [1], then one per M block of the pair tiles (at most M / 256).
+static size_t fuse_ctr_bytes(int64_t M) { return (size_t)(2 + (M + 255) / 256) * 4; }
+static int lora_nt(int r) { return r <= 16 ? 2 : (r <= 32 ? 4 : 8); }
+
 // One dense dequant GEMM (forward: TRANS = false, D = A deq(W)^T; input-gradient: TRANS = true,
 // D = A deq(W)) with its LoRA k-blocks, planned by plan_dense; with a K split the fp32 partials go
-// to split_buf and are summed in order into `out`.
+// to split_buf and are summed in order into `out`. With rx > 0 (from dense_fuse_rx) the launch also
+// computes the adapter row products (rf, the adapter's tensor map tZ; rf->ctr zeroed beforehand).
 template <bool TRANS>
 static int launch_dense_gemm(int qtype, const void* A, int64_t M, int64_t Kd, const void* wq, int64_t w_rows,
                              int64_t w_cols, const __nv_bfloat16* LA, const __nv_bfloat16* LB, int KL, int64_t Nd,
-                             void* out, int out_dtype, float* split_buf, bool allow_split, cudaStream_t st, int slot) {
+                             void* out, int out_dtype, float* split_buf, bool allow_split, cudaStream_t st, int slot,
+                             int rx = 0, const RowsFuse* rf = nullptr, const CUtensorMap* tZ = nullptr) {
   const DensePlan d = plan_dense(M, Nd, Kd, TRANS, allow_split && split_buf != nullptr);
   const uint32_t box = 128u;
   CUtensorMap tA, tW, tLA, tLB;
@@ -546,9 +608,19 @@ static int launch_dense_gemm(int qtype, const void* A, int64_t M, int64_t Kd, co
     p.out_dtype = out_dtype;
   }
   const int tiles = d.mblocks * d.ntiles * d.ksplit;
+  if (rx > 0) {
+    if (d.ms == 0 || d.ksplit != 1 || rf == nullptr || tZ == nullptr) return QL_ERR_INVALID_ARG;
+    p.rx = rx;
+    p.rf = *rf;
+    const int smem = d.ms == 2 ? qgemm2_smem_q<TRANS, 2>(qtype) : qgemm2_smem_q<TRANS, 1>(qtype);
+    const int sb = 128 * 128 + 8 * rf->nt * 128;
+    p.rf.stages = std::min(8, (smem - 1024) / (sb + 16));
+    if (p.rf.stages < 2) return QL_ERR_SHAPE;
+  }
+  const CUtensorMap& tZr = tZ != nullptr ? *tZ : tA;
   int rc;
-  if (d.ms == 2) rc = launch_qgemm2_q<TRANS, 2>(qtype, tA, tW, tLA, tLB, p, tiles, st, slot);
-  else if (d.ms == 1) rc = launch_qgemm2_q<TRANS, 1>(qtype, tA, tW, tLA, tLB, p, tiles, st, slot);
+  if (d.ms == 2) rc = launch_qgemm2_q<TRANS, 2>(qtype, tA, tW, tLA, tLB, tZr, p, tiles, st, slot);
+  else if (d.ms == 1) rc = launch_qgemm2_q<TRANS, 1>(qtype, tA, tW, tLA, tLB, tZr, p, tiles, st, slot);
   else rc = launch_qgemm_q<TRANS, EPI_STORE, 1>(qtype, tA, tW, tLA, tLB, p, std::min(tiles, num_sms()), st, slot);
   if (rc || d.ksplit == 1) return rc;
   return launch_split_reduce(split_buf, d.ksplit, (long)M * Nd, (long)M * Nd, out, out_dtype, st);
@@ -714,7 +786,7 @@ static int launch_gemv_dx(const void* wq, int64_t N, int64_t K, const void* dY, 
 
 // Workspace layout of the dense layer (byte offsets, 256-aligned).
 struct LinearWs {
-  size_t la, lb, hs, split, cr, hp, dxp, total;
+  size_t la, lb, hs, split, cr, fz, hp, dxp, total;
 };
 static LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int r) {
   LinearWs w;
@@ -728,6 +800,7 @@ static LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int r) {
   const size_t sb = split_bytes(plan_dense(M, K, N, true, true), M, K);
   w.split = o; o = al256(o + std::max(sf, sb));
   w.cr = o; o = al256(o + colred_ws_bytes(plan_colred(M, N, K, r), r));
+  w.fz = o; o = al256(o + fuse_ctr_bytes(M));
   if (M <= 16) {
     const GvPlan g = gemv_plan(QL_Q4_0, N, K, M), g8 = gemv_plan(QL_Q8_0, N, K, M);
     const size_t gv = std::max(g.hp_bytes + g.part_bytes, g8.hp_bytes + g8.part_bytes);
@@ -906,6 +979,8 @@ const char* qlora_status_string(int s) {
 
 uint64_t qlora_launch_count(void) { return g_launches.load(); }
 
+int qlora_set_rows_fusion(int enable) { return g_rows_fusion.exchange(enable & 3); }
+
 int qlora_set_kernel_events(int slot, void* start, void* stop) {
   if (slot < 0 || slot >= kEventSlots) return QL_ERR_INVALID_ARG;
   if ((start == nullptr) != (stop == nullptr)) return QL_ERR_INVALID_ARG;
@@ -975,6 +1050,34 @@ int qlora_linear_fwd(int qtype, const void* wq, int64_t N, int64_t K, const void
   __nv_bfloat16* LA = (__nv_bfloat16*)(wsb + w.la);
   __nv_bfloat16* LB = (__nv_bfloat16*)(wsb + w.lb);
   const int KL = 2 * lora_rp(r);
+
+  CUtensorMap tZ;  // A [r x K]: 64-wide boxes of all RN rows (rows past r read as zero)
+  int rx = dense_fuse_rx(qtype, M, N, K, false, r);
+  if (rx > 0 && !make_tmap(&tZ, A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, r, K * 2, 64, 8 * lora_nt(r),
+                           CU_TENSOR_MAP_SWIZZLE_128B))
+    rx = 0;  // the map is refused: the row kernel instead
+  if (rx > 0) {
+    // one launch: the GEMM's idle clusters compute H, split(s H) and LB beside the tiles
+    RowsFuse f;
+    memset(&f, 0, sizeof(f));
+    f.r = r;
+    f.RP = lora_rp(r);
+    f.nt = lora_nt(r);
+    f.ztr = 0;
+    f.oscale = 1.0f;
+    f.lscale = scale;
+    f.out = H;
+    f.la = LA;
+    f.lbz = (const __nv_bfloat16*)B;
+    f.lbzn = r;
+    f.lbzj = 1;
+    f.lb_rows = (int)N;
+    f.lb = LB;
+    f.ctr = (int*)(wsb + w.fz);
+    if (cudaMemsetAsync(f.ctr, 0, fuse_ctr_bytes(M), st) != cudaSuccess) return QL_ERR_CUDA;
+    return launch_dense_gemm<false>(qtype, X, M, K, wq, N, K, LA, LB, KL, N, Y, y_dtype, (float*)(wsb + w.split),
+                                    true, st, 0, rx, &f, &tZ);
+  }
 
   // H = X A^T (saved), the split operand of s*H, and LB = [B | B]
   rc = launch_rows_dense((const __nv_bfloat16*)X, K, (int)M, (int)K, (const __nv_bfloat16*)A, K, 1, r, 1.0f, scale, H,
@@ -1235,6 +1338,45 @@ int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void
   __nv_bfloat16* HS = (__nv_bfloat16*)(wsb + w.hs);
   uint8_t* crws = wsb + w.cr;
   const int ncr = (int)(colred_ctr_bytes(plan_colred(M, N, K, r)) / 4);
+  const ColredOut ob{(int)N, 1.0f, 0, dB};
+  const ColredOut oa{(int)K, 1.0f, 1, dA};
+
+  CUtensorMap tZ;  // B [N x r]: boxes of 64 rows x RN (columns past r read as zero)
+  int rx = dX != nullptr && !gemv_dx_applies(qtype, M) ? dense_fuse_rx(qtype, M, K, N, true, r) : 0;
+  if (rx > 0 && !make_tmap(&tZ, B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, N, (uint64_t)r * 2, 8 * lora_nt(r), 64,
+                           CU_TENSOR_MAP_SWIZZLE_NONE))
+    rx = 0;  // the map is refused: the row kernel instead
+  if (rx > 0) {
+    // one launch for G = s dY B (as LA = split(G)), HS = split(s H), LB = [A^T | A^T] and the dX
+    // GEMM; the column reduction then waits for the row clusters' count, not for the GEMM
+    RowsFuse f;
+    memset(&f, 0, sizeof(f));
+    f.r = r;
+    f.RP = lora_rp(r);
+    f.nt = lora_nt(r);
+    f.ztr = 1;
+    f.oscale = scale;
+    f.lscale = scale;
+    f.out = nullptr;
+    f.la = LA;
+    f.lbz = (const __nv_bfloat16*)A;
+    f.lbzn = 1;
+    f.lbzj = K;
+    f.lb_rows = (int)K;
+    f.lb = LB;
+    f.hin = H;
+    f.hscale = scale;
+    f.hs = HS;
+    f.ctr = (int*)(wsb + w.fz);
+    f.zc = (int*)crws;
+    f.zn = ncr;
+    if (cudaMemsetAsync(f.ctr, 0, fuse_ctr_bytes(M), st) != cudaSuccess) return QL_ERR_CUDA;
+    rc = launch_dense_gemm<true>(qtype, dY, M, N, wq, N, K, LA, LB, KL, K, dX, dx_dtype, (float*)(wsb + w.split),
+                                 true, st, 1, rx, &f, &tZ);
+    if (rc) return rc;
+    return launch_colred_dense((const __nv_bfloat16*)dY, (int)N, HS, ob, (const __nv_bfloat16*)X, (int)K, LA, oa,
+                               (int)M, r, crws, 1, st, f.ctr + 1, 2 * rx);
+  }
   // LA = split(G) with G = s dY B, HS = split(s H), and LB[k] = [A^T(k) | A^T(k)]; the column
   // reduction's counters are zeroed on the way
   // (LB only for the tensor-core dX GEMM: the small-M dX path reads A itself)
@@ -1255,8 +1397,6 @@ int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void
   }
   // dB = dY^T split(s H) and dA = split(G)^T X in one launch; after the dX GEMM (which waited for
   // the row kernel) it runs beside the GEMM on the SMs the GEMM leaves idle
-  const ColredOut ob{(int)N, 1.0f, 0, dB};
-  const ColredOut oa{(int)K, 1.0f, 1, dA};
   return launch_colred_dense((const __nv_bfloat16*)dY, (int)N, HS, ob, (const __nv_bfloat16*)X, (int)K, LA, oa, (int)M,
                              r, crws, dX ? 1 : 0, st);
 }

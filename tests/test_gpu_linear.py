@@ -131,9 +131,63 @@ def test_linear_b_zero_gives_exact_zero_dA():
     assert_close(f64(dB), dBr, "dB")
 
 
+@pytest.fixture
+def unfused():
+    """Row products in their own launch before each pair GEMM (the path without idle clusters)."""
+    prev = ql.qlora_set_rows_fusion(False)
+    try:
+        yield
+    finally:
+        ql.qlora_set_rows_fusion(prev)
+
+
+PAIR_SHAPES = [(300, 512, 384, 4), (129, 768, 320, 16), (200, 256, 448, 40), (1100, 512, 4096, 8),
+               (4500, 256, 320, 8)]
+
+
+@pytest.mark.parametrize("mask", [0, 3])
+@pytest.mark.parametrize("qtype", [inp.Q8_0, inp.Q4_K])
+@pytest.mark.parametrize("shape", PAIR_SHAPES)
+def test_linear_parity_fusion_modes(qtype, shape, mask):
+    """Row products in their own launches (mask 0) and inside both GEMMs (mask 3); the default
+    (forward only) is what the other parity tests run."""
+    M, K, N, r = shape
+    c = inp.linear_case(M, K, N, qtype, r, 2.0 * r, seed=M + K + N + r)
+    prev = ql.qlora_set_rows_fusion(mask)
+    try:
+        Y, H, dX, dA, dB = run_linear(c)
+    finally:
+        ql.qlora_set_rows_fusion(prev)
+    Yr, Hr, dXr, dAr, dBr = oracle_linear(c)
+    for got, ref, name in [(Y, Yr, "Y"), (H, Hr, "H"), (dX, dXr, "dX"), (dA, dAr, "dA"), (dB, dBr, "dB")]:
+        assert_close(f64(got), ref, name)
+
+
+def test_rows_fusion_engages():
+    """With idle SM pairs the fused forward is one launch (GEMM with the row products) instead of two,
+    and the fused backward two (GEMM, column reductions) instead of three; the results agree within
+    the bar."""
+    c = inp.linear_case(700, 1024, 768, inp.Q8_0, 16, 32.0, seed=5)
+    counts, outs = [], []
+    for mask in (3, 1, 0):
+        prev = ql.qlora_set_rows_fusion(mask)
+        try:
+            n0 = ql.qlora_launch_count()
+            outs.append([t.clone() for t in run_linear(c)])
+            counts.append(ql.qlora_launch_count() - n0)
+        finally:
+            ql.qlora_set_rows_fusion(prev)
+    assert counts == [3, 4, 5], counts
+    refs = oracle_linear(c)
+    for got in outs:
+        for g, ref, name in zip(got, refs, ["Y", "H", "dX", "dA", "dB"]):
+            assert_close(f64(g), ref, name)
+
+
 @pytest.mark.parametrize("shape", [(300, 512, 384, 4), (2600, 256, 192, 40)])
-def test_linear_bwd_without_dx(shape):
-    """Without dX the adapter gradients follow the row kernel directly: the same values, bit for bit."""
+def test_linear_bwd_without_dx(shape, unfused):
+    """Without dX the adapter gradients follow the row kernel directly: with the row products in
+    their own launch in both runs, the same values, bit for bit."""
     M, K, N, r = shape
     c = inp.linear_case(M, K, N, inp.Q8_0, r, 2.0 * r, seed=M + r)
     a = [t.clone() for t in run_linear(c)]
@@ -141,6 +195,24 @@ def test_linear_bwd_without_dx(shape):
     assert b[2] is None
     for i in (0, 1, 3, 4):
         assert torch.equal(a[i], b[i])
+
+
+@pytest.mark.parametrize("shape", [(300, 512, 384, 8), (2600, 256, 192, 40)])
+def test_linear_bwd_without_dx_fused(shape):
+    """The input-gradient GEMM computes G itself when fused; without dX the row kernel does: both
+    sets of adapter gradients are within the bar of the oracle."""
+    M, K, N, r = shape
+    c = inp.linear_case(M, K, N, inp.Q8_0, r, 2.0 * r, seed=M + r)
+    prev = ql.qlora_set_rows_fusion(3)
+    try:
+        a = [t.clone() for t in run_linear(c)]
+        b = run_linear(c, with_dx=False)
+    finally:
+        ql.qlora_set_rows_fusion(prev)
+    refs = oracle_linear(c)
+    for run in (a, b):
+        for i, name in [(3, "dA"), (4, "dB")]:
+            assert_close(f64(run[i]), refs[i], name)
 
 
 def test_linear_deterministic():
