@@ -502,8 +502,9 @@ struct ColredFlow {
   int defer_wait;  // 1: the previous kernel in the stream already waited for this launch's inputs
   float* part;     // [nblk * csu][16 JT][128]
   int* ctr;        // [0]: next unit to claim, [1 + b]: chunks of block b finished; zero at launch
-  const int* gate; // with defer_wait: a count of the previous launch that reaches gate_target once
-  int gate_target; // the split operands and the zeroed counters are written (nullable)
+  const unsigned long long* gate;  // with defer_wait: a tagged count (gate_seq) of the previous
+  unsigned gate_seq;               // launch that reaches gate_target once the split operands and
+  int gate_target;                 // the zeroed counters are written (nullable)
 };
 
 constexpr int kColTmaStagesMax = 6;
@@ -604,7 +605,7 @@ __global__ void __launch_bounds__(32 * kColWarps) colred_flow_kernel(const __gri
   bool ok = true;
   if (warp == 8) {
     if (lane == 0 && P.gate != nullptr) {
-      ok = wait_count(P.gate, P.gate_target, 65);
+      ok = wait_tagged(P.gate, P.gate_seq, P.gate_target, 65);
       fence_proxy_async_global();
     }
     if (lane == 0 && ok) {

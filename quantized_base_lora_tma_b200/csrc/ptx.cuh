@@ -206,27 +206,41 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 
 // ------------------------------------------------------------------------------------------------
 // Counters between CTAs of one grid, or towards a later launch: a producer CTA makes its global
-// writes visible (every writer fences, a CTA barrier, then one thread's release add); a consumer
-// thread acquires the count and fences before its TMA copies read the data. The producers are
-// CTAs of lower index in the same launch (dispatched no later than the waiters, and waiting on
-// nothing themselves) or of an earlier launch, so every wait ends; it is bounded all the same.
+// writes visible (every writer fences for the async proxy, a CTA barrier, then one thread's fenced
+// add); a consumer thread acquires the count and fences before its TMA copies read the data. The
+// producers are CTAs of lower index in the same launch (dispatched no later than the waiters, and
+// waiting on nothing themselves) or of an earlier launch, so every wait ends; it is bounded all
+// the same.
 // ------------------------------------------------------------------------------------------------
-__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+// Tagged counters: a 64-bit word (tag << 32 | count) whose tag is the launch's sequence number, so
+// that a launch needs no zeroed counters. The first add of a launch replaces a word left with another
+// tag by (seq, 1); waits count only words carrying their own tag.
+__device__ __forceinline__ unsigned long long ld_acquire_gpu_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
 }
-__device__ __forceinline__ void release_add_gpu(int* p, int v) {
-  __threadfence();
-  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+__device__ __forceinline__ void tagged_add(unsigned long long* p, unsigned seq) {
+  __threadfence();  // release: the writes this add publishes come first
+  unsigned long long old = ld_acquire_gpu_u64(p);
+  while (true) {  // lock-free: each retry means another CTA's add went in
+    const unsigned long long nv = (unsigned)(old >> 32) == seq ? old + 1ull : (((unsigned long long)seq << 32) | 1ull);
+    const unsigned long long prev = atomicCAS(p, old, nv);
+    if (prev == old) return;
+    old = prev;
+  }
 }
-__device__ __forceinline__ bool wait_count(const int* p, int target, int site) {
-  if (ld_acquire_gpu(p) >= target) return true;
+__device__ __forceinline__ bool tagged_reached(const unsigned long long* p, unsigned seq, int target) {
+  const unsigned long long v = ld_acquire_gpu_u64(p);
+  return (unsigned)(v >> 32) == seq && (int)(unsigned)(v & 0xffffffffull) >= target;
+}
+__device__ __forceinline__ bool wait_tagged(const unsigned long long* p, unsigned seq, int target, int site) {
+  if (tagged_reached(p, seq, target)) return true;
   const uint64_t t0 = globaltimer_ns();
   uint32_t polls = 0;
   while (true) {
     __nanosleep(500);
-    if (ld_acquire_gpu(p) >= target) return true;
+    if (tagged_reached(p, seq, target)) return true;
     ++polls;
     if (dev_aborted()) return false;
     if (polls >= 16u && globaltimer_ns() - t0 > kWaitLimitNs) {
@@ -245,6 +259,14 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
       "[%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y,
+                                            int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
+      "[%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
 // Bring the box at (x, y) into L2 without touching shared memory (no completion to wait for).

@@ -45,6 +45,7 @@ constexpr int kGemmThreads = (kWarpDq0 + kNumDqWarps) * 32;  // 736
 struct RowsFuse {
   int r, RP, nt;               // rank, padded rank (LA / LB are 2RP wide), 8-column tiles of Z^T
   int ztr;                     // the adapter box is [k][j] (j contiguous) rather than [j][k]
+  int kc;                      // 64-wide k chunks per ring stage
   int stages;                  // TMA ring depth
   float oscale, lscale;
   float* out;                  // fp32 [M x r] (nullable)
@@ -56,9 +57,10 @@ struct RowsFuse {
   const float* hin;            // hs = split(hscale hin), [M x 2RP] (nullable)
   float hscale;
   __nv_bfloat16* hs;
-  int* ctr;  // [0] CTAs whose LB / hs share is written, [1] CTAs done, [2 + mb] 128-row blocks of
-             // M block mb written; zero at launch
-  int* zc;   // counters of a later launch, zeroed here (nullable)
+  unsigned long long* ctr;  // tagged counters (seq): [0] CTAs whose LB / hs share is written,
+                            // [1] CTAs done, [2 + mb] 128-row blocks of M block mb written
+  unsigned seq;             // this launch's tag
+  int* zc;                  // counters of a later launch, zeroed here (nullable)
   int zn;
 };
 

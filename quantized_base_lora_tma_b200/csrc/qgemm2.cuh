@@ -94,21 +94,20 @@ __device__ __forceinline__ bool gemm2_tile(const GemmParams& p, int t, TileInfo&
 // Y (X in the forward, dY in the input gradient), out = oscale Y Z^T and la = split(lscale Y Z^T)
 // by 128-row blocks, plus LB and hs, while the tiles' main loops run; the tiles' LoRA k-blocks
 // come last and wait for the counters. Every CTA first writes its share of LB and hs, then streams
-// its blocks through a TMA ring: Y's 128 x 64 boxes (the GEMM's tensor map) and the adapter's
-// 64-wide boxes (tmZ: RN x 64 with 128-byte swizzle for Z stored [j][k], or 64 x RN unswizzled
-// for Z stored [k][j]). Warps 0..7 own 16 rows each (ldmatrix, mma.sync, fp32 accumulation over
-// the whole k range in order), warp 8 lane 0 produces.
-template <int NT>
-__device__ __forceinline__ constexpr int rows_fuse_stage_bytes() {
-  return 128 * 128 + 8 * NT * 128;
-}
+// its blocks through a TMA ring, kc 64-wide k chunks per stage in one copy of each operand.
+// tmY views Y as [rows][k chunk][64] with a 128 x kc x 64 box, 128-byte swizzled, so a stage holds
+// 128-byte lines (row y, chunk z) at line y kc + z; tmZ views the adapter Z stored [j][k] the same
+// way (RN x kc x 64), or, stored [k][j], as 64 kc k-rows of RN unswizzled. Warps 0..7 own 16 rows
+// each (ldmatrix, mma.sync, fp32 accumulation over the whole k range in order), warp 8 lane 0
+// produces.
 template <int NT, int MS>
 __device__ __noinline__ void gemm2_rows_role(const CUtensorMap* tmY, const CUtensorMap* tmZ, const GemmParams& p, uint32_t base) {
   const RowsFuse& f = p.rf;
   constexpr int RN = 8 * NT;
-  constexpr int XB = 128 * 128;
-  constexpr int SB = rows_fuse_stage_bytes<NT>();
-  const int S = f.stages;
+  constexpr int XB = 128 * 128;  // one chunk of Y: 128 rows x 64 k
+  constexpr int ZB = RN * 128;   // one chunk of Z: RN x 64
+  const int S = f.stages, KC = f.kc;
+  const int SB = KC * (XB + ZB);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cta = blockIdx.x, ncta = 2 * p.rx;
   pdl_wait();  // Y and the adapters may be the previous launch's output
@@ -137,10 +136,10 @@ __device__ __noinline__ void gemm2_rows_role(const CUtensorMap* tmY, const CUten
     fence_mbar_init();
   }
   __syncthreads();
-  if (tid == 0) release_add_gpu(f.ctr, 1);  // this CTA's LB and hs share is out
+  if (tid == 0) tagged_add(f.ctr, f.seq);  // this CTA's LB and hs share is out
 
   const int nblk = (p.M + 127) / 128;
-  const int ksteps = p.Kd / kBK;
+  const int ksteps = (p.Kd / kBK + KC - 1) / KC;  // stages per block (chunks past the end read as zero)
   if (warp == 8) {
     if (lane == 0) {
       prefetch_tmap(tmY);
@@ -156,9 +155,9 @@ __device__ __noinline__ void gemm2_rows_role(const CUtensorMap* tmY, const CUten
           }
           const uint32_t st = base + (uint32_t)(s * SB);
           mbar_arrive_expect_tx(full_bar(s), (uint32_t)SB);
-          tma_load_2d(st, tmY, full_bar(s), kt * kBK, b * 128);
-          if (f.ztr) tma_load_2d(st + XB, tmZ, full_bar(s), 0, kt * kBK);
-          else tma_load_2d(st + XB, tmZ, full_bar(s), kt * kBK, 0);
+          tma_load_3d(st, tmY, full_bar(s), 0, kt * KC, b * 128);
+          if (f.ztr) tma_load_2d(st + KC * XB, tmZ, full_bar(s), 0, kt * KC * kBK);
+          else tma_load_3d(st + KC * XB, tmZ, full_bar(s), 0, kt * KC, 0);
         }
       if (!ok && it > 0) spin_ns(2000000ull);  // copies in flight land before the CTA exits
     }
@@ -180,18 +179,22 @@ __device__ __noinline__ void gemm2_rows_role(const CUtensorMap* tmY, const CUten
           ok = false;
           break;
         }
-        const uint32_t xs = base + (uint32_t)(s * SB), zs = xs + XB;
+        const uint32_t xs = base + (uint32_t)(s * SB), zs = xs + (uint32_t)(KC * XB);
+        for (int z = 0; z < KC; ++z) {
 #pragma unroll
-        for (int k16 = 0; k16 < kBK / 16; ++k16) {
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4(sw128_addr(xs, a_row, 16 * k16 + a_col), a0, a1, a2, a3);
+          for (int k16 = 0; k16 < kBK / 16; ++k16) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(sw128_addr(xs, a_row * KC + z, 16 * k16 + a_col), a0, a1, a2, a3);
 #pragma unroll
-          for (int tp = 0; tp < NT / 2; ++tp) {
-            uint32_t b0, b1, b2, b3;
-            if (f.ztr) ldsm_x4_t(zs + (uint32_t)(((16 * k16 + t_k) * RN + 16 * tp + t_j) * 2), b0, b1, b2, b3);
-            else ldsm_x4(sw128_addr(zs, 16 * tp + b_row, 16 * k16 + b_col), b0, b1, b2, b3);
-            mma_16816(acc[2 * tp], a0, a1, a2, a3, b0, b1);
-            mma_16816(acc[2 * tp + 1], a0, a1, a2, a3, b2, b3);
+            for (int tp = 0; tp < NT / 2; ++tp) {
+              uint32_t b0, b1, b2, b3;
+              if (f.ztr)
+                ldsm_x4_t(zs + (uint32_t)(((z * kBK + 16 * k16 + t_k) * RN + 16 * tp + t_j) * 2), b0, b1, b2, b3);
+              else
+                ldsm_x4(sw128_addr(zs, (16 * tp + b_row) * KC + z, 16 * k16 + b_col), b0, b1, b2, b3);
+              mma_16816(acc[2 * tp], a0, a1, a2, a3, b0, b1);
+              mma_16816(acc[2 * tp + 1], a0, a1, a2, a3, b2, b3);
+            }
           }
         }
         __syncwarp();
@@ -223,10 +226,10 @@ __device__ __noinline__ void gemm2_rows_role(const CUtensorMap* tmY, const CUten
       }
       fence_proxy_async_global();
       asm volatile("bar.sync 1, 256;" ::: "memory");  // the eight row warps
-      if (tid == 0 && !dev_aborted()) release_add_gpu(f.ctr + 2 + b / (2 * MS), 1);
+      if (tid == 0 && !dev_aborted()) tagged_add(f.ctr + 2 + b / (2 * MS), f.seq);
     }
     asm volatile("bar.sync 1, 256;" ::: "memory");
-    if (tid == 0 && !dev_aborted()) release_add_gpu(f.ctr + 1, 1);
+    if (tid == 0 && !dev_aborted()) tagged_add(f.ctr + 1, f.seq);
   }
 }
 
@@ -234,7 +237,8 @@ template <int QT, bool TRANS, int MS>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm2Threads, 1)
     qgemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
                   const __grid_constant__ CUtensorMap tmLA, const __grid_constant__ CUtensorMap tmLB,
-                  const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ GemmParams p) {
+                  const __grid_constant__ CUtensorMap tmRY, const __grid_constant__ CUtensorMap tmZ,
+                  const __grid_constant__ GemmParams p) {
   using C = Gemm2Cfg<QT, TRANS, MS>;
   constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw_[];
@@ -242,9 +246,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm2Threads, 1)
   uint8_t* smem = smem_raw_ + (base_u32 - smem_u32(smem_raw_));
 
   if ((int)(blockIdx.x >> 1) < p.rx) {  // a cluster of the fused adapter row products
-    if (p.rf.nt == 2) gemm2_rows_role<2, MS>(&tmA, &tmZ, p, base_u32);
-    else if (p.rf.nt == 4) gemm2_rows_role<4, MS>(&tmA, &tmZ, p, base_u32);
-    else gemm2_rows_role<8, MS>(&tmA, &tmZ, p, base_u32);
+    if (p.rf.nt == 2) gemm2_rows_role<2, MS>(&tmRY, &tmZ, p, base_u32);
+    else if (p.rf.nt == 4) gemm2_rows_role<4, MS>(&tmRY, &tmZ, p, base_u32);
+    else gemm2_rows_role<8, MS>(&tmRY, &tmZ, p, base_u32);
     return;
   }
   if (p.rx > 0) {
@@ -348,12 +352,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm2Threads, 1)
           } else {
             if (!waited) {
               if (p.rx == 0) pdl_wait();  // the LoRA operands are the previous kernel's output
-              else if (!wait_count(p.rf.ctr, 2 * p.rx, 63)) { ok = false; break; }
+              else if (!wait_tagged(p.rf.ctr, p.rf.seq, 2 * p.rx, 63)) { ok = false; break; }
               waited = true;
             }
             if (p.rx > 0 && mb != mb_ready) {
               const int blocks = min(2 * MS, (p.M + 127) / 128 - 2 * MS * mb);
-              if (!wait_count(p.rf.ctr + 2 + mb, blocks, 64)) { ok = false; break; }
+              if (!wait_tagged(p.rf.ctr + 2 + mb, p.rf.seq, blocks, 64)) { ok = false; break; }
               fence_proxy_async_global();
               mb_ready = mb;
             }

@@ -8,6 +8,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <random>
 #include <vector>
 
 #include "qlora.h"
@@ -65,6 +66,22 @@ static bool make_tmap(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, i
   (void)esize;
   CUresult r = fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// bf16 rows [rows x cols] (cols a multiple of 64) seen as [rows][cols / 64][64]: box [box_rows][kc][64],
+// 128-byte swizzled, landing as 128-byte lines (row y, chunk z) at line y kc + z.
+static bool tmap_bf16_chunks(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint32_t box_rows,
+                             uint32_t kc) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {64, cols / 64, rows};
+  cuuint64_t strides[2] = {128, cols * 2};
+  cuuint32_t box[3] = {64, kc, box_rows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -252,7 +269,8 @@ static int qgemm2_max_clusters() {
 // With p.rx row clusters (fused adapter row products) in front of the tile clusters.
 template <int QT, bool TRANS, int MS>
 static int launch_qgemm2(const CUtensorMap& tA, const CUtensorMap& tW, const CUtensorMap& tLA, const CUtensorMap& tLB,
-                         const CUtensorMap& tZ, const GemmParams& p, int tiles, cudaStream_t st, int slot) {
+                         const CUtensorMap& tRY, const CUtensorMap& tZ, const GemmParams& p, int tiles, cudaStream_t st,
+                         int slot) {
   using C = Gemm2Cfg<QT, TRANS, MS>;
   auto k = qgemm2_kernel<QT, TRANS, MS>;
   const int mc = qgemm2_max_clusters<QT, TRANS, MS>();
@@ -260,19 +278,19 @@ static int launch_qgemm2(const CUtensorMap& tA, const CUtensorMap& tW, const CUt
   const int clusters = p.rx + std::min(tiles, mc - p.rx);
   PdlLaunch L(dim3(2 * clusters), dim3(kGemm2Threads), C::SMEM_BYTES, st);  // cluster shape from the kernel
   ev_record(slot, 0, st);
-  const cudaError_t e = cudaLaunchKernelEx(&L.cfg, k, tA, tW, tLA, tLB, tZ, p);
+  const cudaError_t e = cudaLaunchKernelEx(&L.cfg, k, tA, tW, tLA, tLB, tRY, tZ, p);
   ev_record(slot, 1, st);
   return launch_result(e);
 }
 
 template <bool TRANS, int MS>
 static int launch_qgemm2_q(int qtype, const CUtensorMap& tA, const CUtensorMap& tW, const CUtensorMap& tLA,
-                           const CUtensorMap& tLB, const CUtensorMap& tZ, const GemmParams& p, int tiles,
-                           cudaStream_t st, int slot) {
+                           const CUtensorMap& tLB, const CUtensorMap& tRY, const CUtensorMap& tZ, const GemmParams& p,
+                           int tiles, cudaStream_t st, int slot) {
   switch (qtype) {
-    case QL_Q8_0: return launch_qgemm2<QL_Q8_0, TRANS, MS>(tA, tW, tLA, tLB, tZ, p, tiles, st, slot);
-    case QL_Q4_0: return launch_qgemm2<QL_Q4_0, TRANS, MS>(tA, tW, tLA, tLB, tZ, p, tiles, st, slot);
-    case QL_Q4_K: return launch_qgemm2<QL_Q4_K, TRANS, MS>(tA, tW, tLA, tLB, tZ, p, tiles, st, slot);
+    case QL_Q8_0: return launch_qgemm2<QL_Q8_0, TRANS, MS>(tA, tW, tLA, tLB, tRY, tZ, p, tiles, st, slot);
+    case QL_Q4_0: return launch_qgemm2<QL_Q4_0, TRANS, MS>(tA, tW, tLA, tLB, tRY, tZ, p, tiles, st, slot);
+    case QL_Q4_K: return launch_qgemm2<QL_Q4_K, TRANS, MS>(tA, tW, tLA, tLB, tRY, tZ, p, tiles, st, slot);
     default: return QL_ERR_UNSUPPORTED;
   }
 }
@@ -437,8 +455,8 @@ static cudaError_t launch_colred_jt(cudaLaunchConfig_t& cfg, const CUtensorMap* 
 // Z0 and Z1 (and the zeroed counters) are written; the producer waits for it before its first claim.
 static int launch_colred_dense(const __nv_bfloat16* Y0, int C0, const __nv_bfloat16* Z0, const ColredOut& o0,
                                const __nv_bfloat16* Y1, int C1, const __nv_bfloat16* Z1, const ColredOut& o1, int M, int r,
-                               uint8_t* crws, int defer_wait, cudaStream_t st, const int* gate = nullptr,
-                               int gate_target = 0) {
+                               uint8_t* crws, int defer_wait, cudaStream_t st,
+                               const unsigned long long* gate = nullptr, unsigned gate_seq = 0, int gate_target = 0) {
   const int RP = lora_rp(r);
   const int JT = (r + 15) / 16;
   CUtensorMap tm[4];
@@ -461,6 +479,7 @@ static int launch_colred_dense(const __nv_bfloat16* Y0, int C0, const __nv_bfloa
   P.ctr = reinterpret_cast<int*>(crws);
   P.part = reinterpret_cast<float*>(crws + al256(colred_ctr_bytes(pl)));
   P.gate = gate;
+  P.gate_seq = gate_seq;
   P.gate_target = gate_target;
   const size_t smem = colred_smem_bytes(RP, JT, pl.tr);
   const int per_sm = std::max(1, (int)(233472 / (smem + 1024)));
@@ -568,9 +587,26 @@ static int dense_fuse_rx(int qtype, int64_t M, int64_t Nd, int64_t Kd, bool tran
   if (rx < 1 || (nblk + 2 * rx - 1) / (2 * rx) > 3) return 0;
   return rx;
 }
-// Counters of a fused launch: [0], [1], then one per M block of the pair tiles (at most M / 256).
-static size_t fuse_ctr_bytes(int64_t M) { return (size_t)(2 + (M + 255) / 256) * 4; }
+// Tagged counters of a fused launch: [0], [1], then one per M block of the pair tiles (at most
+// M / 256), 8 bytes each. Tags are launch sequence numbers, unique within the process (the start is
+// random, so a reloaded library does not meet its predecessor's tags in a reused workspace).
+static size_t fuse_ctr_bytes(int64_t M) { return (size_t)(2 + (M + 255) / 256) * 8; }
+static unsigned next_fuse_seq() {
+  static std::atomic<unsigned> seq{(unsigned)std::random_device{}()};
+  return seq.fetch_add(1, std::memory_order_relaxed) + 1u;
+}
 static int lora_nt(int r) { return r <= 16 ? 2 : (r <= 32 ? 4 : 8); }
+// The row clusters' ring in the pair GEMM's shared memory: two 64-wide k chunks per stage when at
+// least three such stages fit, else one.
+static void fuse_ring(int qtype, bool trans, int ms, int nt, int& kc, int& stages) {
+  const int smem = trans ? (ms == 2 ? qgemm2_smem_q<true, 2>(qtype) : qgemm2_smem_q<true, 1>(qtype))
+                         : (ms == 2 ? qgemm2_smem_q<false, 2>(qtype) : qgemm2_smem_q<false, 1>(qtype));
+  for (kc = 2;; --kc) {
+    const int sb = kc * (128 * 128 + 8 * nt * 128);
+    stages = std::min(8, (smem - 1024) / (sb + 16));
+    if (stages >= 3 || kc == 1) return;
+  }
+}
 
 // One dense dequant GEMM (forward: TRANS = false, D = A deq(W)^T; input-gradient: TRANS = true,
 // D = A deq(W)) with its LoRA k-blocks, planned by plan_dense; with a K split the fp32 partials go
@@ -580,7 +616,8 @@ template <bool TRANS>
 static int launch_dense_gemm(int qtype, const void* A, int64_t M, int64_t Kd, const void* wq, int64_t w_rows,
                              int64_t w_cols, const __nv_bfloat16* LA, const __nv_bfloat16* LB, int KL, int64_t Nd,
                              void* out, int out_dtype, float* split_buf, bool allow_split, cudaStream_t st, int slot,
-                             int rx = 0, const RowsFuse* rf = nullptr, const CUtensorMap* tZ = nullptr) {
+                             int rx = 0, const RowsFuse* rf = nullptr, const CUtensorMap* tRY = nullptr,
+                             const CUtensorMap* tZ = nullptr) {
   const DensePlan d = plan_dense(M, Nd, Kd, TRANS, allow_split && split_buf != nullptr);
   const uint32_t box = 128u;
   CUtensorMap tA, tW, tLA, tLB;
@@ -609,18 +646,16 @@ static int launch_dense_gemm(int qtype, const void* A, int64_t M, int64_t Kd, co
   }
   const int tiles = d.mblocks * d.ntiles * d.ksplit;
   if (rx > 0) {
-    if (d.ms == 0 || d.ksplit != 1 || rf == nullptr || tZ == nullptr) return QL_ERR_INVALID_ARG;
+    if (d.ms == 0 || d.ksplit != 1 || rf == nullptr || tRY == nullptr || tZ == nullptr) return QL_ERR_INVALID_ARG;
     p.rx = rx;
     p.rf = *rf;
-    const int smem = d.ms == 2 ? qgemm2_smem_q<TRANS, 2>(qtype) : qgemm2_smem_q<TRANS, 1>(qtype);
-    const int sb = 128 * 128 + 8 * rf->nt * 128;
-    p.rf.stages = std::min(8, (smem - 1024) / (sb + 16));
     if (p.rf.stages < 2) return QL_ERR_SHAPE;
   }
+  const CUtensorMap& tRYr = tRY != nullptr ? *tRY : tA;
   const CUtensorMap& tZr = tZ != nullptr ? *tZ : tA;
   int rc;
-  if (d.ms == 2) rc = launch_qgemm2_q<TRANS, 2>(qtype, tA, tW, tLA, tLB, tZr, p, tiles, st, slot);
-  else if (d.ms == 1) rc = launch_qgemm2_q<TRANS, 1>(qtype, tA, tW, tLA, tLB, tZr, p, tiles, st, slot);
+  if (d.ms == 2) rc = launch_qgemm2_q<TRANS, 2>(qtype, tA, tW, tLA, tLB, tRYr, tZr, p, tiles, st, slot);
+  else if (d.ms == 1) rc = launch_qgemm2_q<TRANS, 1>(qtype, tA, tW, tLA, tLB, tRYr, tZr, p, tiles, st, slot);
   else rc = launch_qgemm_q<TRANS, EPI_STORE, 1>(qtype, tA, tW, tLA, tLB, p, std::min(tiles, num_sms()), st, slot);
   if (rc || d.ksplit == 1) return rc;
   return launch_split_reduce(split_buf, d.ksplit, (long)M * Nd, (long)M * Nd, out, out_dtype, st);
@@ -1051,11 +1086,15 @@ int qlora_linear_fwd(int qtype, const void* wq, int64_t N, int64_t K, const void
   __nv_bfloat16* LB = (__nv_bfloat16*)(wsb + w.lb);
   const int KL = 2 * lora_rp(r);
 
-  CUtensorMap tZ;  // A [r x K]: 64-wide boxes of all RN rows (rows past r read as zero)
+  // X and A [r x K] in kc-chunk boxes (A's rows past r read as zero)
+  CUtensorMap tRY, tZ;
+  int kc = 1, stages = 0;
   int rx = dense_fuse_rx(qtype, M, N, K, false, r);
-  if (rx > 0 && !make_tmap(&tZ, A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, r, K * 2, 64, 8 * lora_nt(r),
-                           CU_TENSOR_MAP_SWIZZLE_128B))
-    rx = 0;  // the map is refused: the row kernel instead
+  if (rx > 0) {
+    fuse_ring(qtype, false, plan_dense(M, N, K, false, true).ms, lora_nt(r), kc, stages);
+    if (!tmap_bf16_chunks(&tRY, X, K, M, 128, kc) || !tmap_bf16_chunks(&tZ, A, K, r, 8 * lora_nt(r), kc))
+      rx = 0;  // a map is refused: the row kernel instead
+  }
   if (rx > 0) {
     // one launch: the GEMM's idle clusters compute H, split(s H) and LB beside the tiles
     RowsFuse f;
@@ -1064,6 +1103,8 @@ int qlora_linear_fwd(int qtype, const void* wq, int64_t N, int64_t K, const void
     f.RP = lora_rp(r);
     f.nt = lora_nt(r);
     f.ztr = 0;
+    f.kc = kc;
+    f.stages = stages;
     f.oscale = 1.0f;
     f.lscale = scale;
     f.out = H;
@@ -1073,10 +1114,10 @@ int qlora_linear_fwd(int qtype, const void* wq, int64_t N, int64_t K, const void
     f.lbzj = 1;
     f.lb_rows = (int)N;
     f.lb = LB;
-    f.ctr = (int*)(wsb + w.fz);
-    if (cudaMemsetAsync(f.ctr, 0, fuse_ctr_bytes(M), st) != cudaSuccess) return QL_ERR_CUDA;
+    f.ctr = (unsigned long long*)(wsb + w.fz);
+    f.seq = next_fuse_seq();
     return launch_dense_gemm<false>(qtype, X, M, K, wq, N, K, LA, LB, KL, N, Y, y_dtype, (float*)(wsb + w.split),
-                                    true, st, 0, rx, &f, &tZ);
+                                    true, st, 0, rx, &f, &tRY, &tZ);
   }
 
   // H = X A^T (saved), the split operand of s*H, and LB = [B | B]
@@ -1341,11 +1382,17 @@ int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void
   const ColredOut ob{(int)N, 1.0f, 0, dB};
   const ColredOut oa{(int)K, 1.0f, 1, dA};
 
-  CUtensorMap tZ;  // B [N x r]: boxes of 64 rows x RN (columns past r read as zero)
+  // dY in kc-chunk boxes, and B [N x r] as boxes of 64 kc rows x RN (columns past r read as zero)
+  CUtensorMap tRY, tZ;
+  int kc = 1, stages = 0;
   int rx = dX != nullptr && !gemv_dx_applies(qtype, M) ? dense_fuse_rx(qtype, M, K, N, true, r) : 0;
-  if (rx > 0 && !make_tmap(&tZ, B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, N, (uint64_t)r * 2, 8 * lora_nt(r), 64,
-                           CU_TENSOR_MAP_SWIZZLE_NONE))
-    rx = 0;  // the map is refused: the row kernel instead
+  if (rx > 0) {
+    fuse_ring(qtype, true, plan_dense(M, K, N, true, true).ms, lora_nt(r), kc, stages);
+    if (!tmap_bf16_chunks(&tRY, dY, N, M, 128, kc) ||
+        !make_tmap(&tZ, B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, N, (uint64_t)r * 2, 8 * lora_nt(r), 64 * kc,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+      rx = 0;  // a map is refused: the row kernel instead
+  }
   if (rx > 0) {
     // one launch for G = s dY B (as LA = split(G)), HS = split(s H), LB = [A^T | A^T] and the dX
     // GEMM; the column reduction then waits for the row clusters' count, not for the GEMM
@@ -1355,6 +1402,8 @@ int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void
     f.RP = lora_rp(r);
     f.nt = lora_nt(r);
     f.ztr = 1;
+    f.kc = kc;
+    f.stages = stages;
     f.oscale = scale;
     f.lscale = scale;
     f.out = nullptr;
@@ -1367,15 +1416,15 @@ int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void
     f.hin = H;
     f.hscale = scale;
     f.hs = HS;
-    f.ctr = (int*)(wsb + w.fz);
+    f.ctr = (unsigned long long*)(wsb + w.fz);
+    f.seq = next_fuse_seq();
     f.zc = (int*)crws;
     f.zn = ncr;
-    if (cudaMemsetAsync(f.ctr, 0, fuse_ctr_bytes(M), st) != cudaSuccess) return QL_ERR_CUDA;
     rc = launch_dense_gemm<true>(qtype, dY, M, N, wq, N, K, LA, LB, KL, K, dX, dx_dtype, (float*)(wsb + w.split),
-                                 true, st, 1, rx, &f, &tZ);
+                                 true, st, 1, rx, &f, &tRY, &tZ);
     if (rc) return rc;
     return launch_colred_dense((const __nv_bfloat16*)dY, (int)N, HS, ob, (const __nv_bfloat16*)X, (int)K, LA, oa,
-                               (int)M, r, crws, 1, st, f.ctr + 1, 2 * rx);
+                               (int)M, r, crws, 1, st, f.ctr + 1, f.seq, 2 * rx);
   }
   // LA = split(G) with G = s dY B, HS = split(s H), and LB[k] = [A^T(k) | A^T(k)]; the column
   // reduction's counters are zeroed on the way
