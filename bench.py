@@ -359,16 +359,17 @@ def run_ours(args, rank, world, local_rank):
     launches0 = ql.qlora_launch_count()
     sampler = ClockSampler(local_rank)
     wall0 = time.perf_counter()
-    # The GEMM events are recorded on every fourth step only: an event between two kernels of the
+    # The GEMM events are recorded on every eighth step only: an event between two kernels of the
     # step stops the next kernel from starting while the previous one drains (programmatic launch),
     # so those steps are slower; they stay in the step mean, which is therefore slightly pessimistic.
-    ev_steps = list(range(0, K, 4))
+    EV_EVERY = 8
+    ev_steps = list(range(0, K, EV_EVERY))
     with sampler:
         for i in range(K):
             flush.zero_()
             for s in (0, 1):
-                if i % 4 == 0:
-                    ql.qlora_set_kernel_events(s, gev[s][i // 4][0], gev[s][i // 4][1])
+                if i % EV_EVERY == 0:
+                    ql.qlora_set_kernel_events(s, gev[s][i // EV_EVERY][0], gev[s][i // EV_EVERY][1])
                 else:
                     ql.qlora_set_kernel_events(s, None, None)
             ev[i][0].record(stream)
