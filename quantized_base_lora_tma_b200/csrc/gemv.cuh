@@ -224,6 +224,88 @@ __global__ void __launch_bounds__(kGvHWarps * 32) gemv_h_kernel(const __nv_bfloa
   }
 }
 
+// The backward's row products for m < M <= 16, j < r <= 16, in one CTA like gemv_h_kernel:
+// G = s dY B with B [N x r] (j contiguous: each B fragment pairs two rows of B), written as
+// la = split(G) [M x 2RP] (zero past r); hs = split(s H) [M x 2RP] for the column reductions,
+// whose counters (zc, zn) it zeroes.
+__global__ void __launch_bounds__(kGvHWarps * 32) gemv_g_kernel(const __nv_bfloat16* __restrict__ dY,
+                                                                const __nv_bfloat16* __restrict__ B,
+                                                                const float* __restrict__ H, int M, int N, int r,
+                                                                float scale, int RP, __nv_bfloat16* __restrict__ la,
+                                                                __nv_bfloat16* __restrict__ hs, int* __restrict__ zc,
+                                                                int zn) {
+  __shared__ float red[kGvHWarps][256];
+  pdl_wait();
+  pdl_launch_dependents();
+  for (int i = threadIdx.x; i < zn; i += blockDim.x) zc[i] = 0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+  float acc[2][4];
+#pragma unroll
+  for (int jt = 0; jt < 2; ++jt) acc[jt][0] = acc[jt][1] = acc[jt][2] = acc[jt][3] = 0.f;
+  auto ldy = [&](int row, int k) -> uint32_t {
+    return row < M ? __ldg(reinterpret_cast<const unsigned int*>(dY + (long)row * N + k)) : 0u;
+  };
+  auto ldb = [&](int j, int k) -> uint32_t {  // (B[k][j], B[k + 1][j])
+    if (j >= r) return 0u;
+    const unsigned short lo = __ldg(reinterpret_cast<const unsigned short*>(B + (long)k * r + j));
+    const unsigned short hi = __ldg(reinterpret_cast<const unsigned short*>(B + (long)(k + 1) * r + j));
+    return (uint32_t)lo | ((uint32_t)hi << 16);
+  };
+  constexpr int U = 4;
+  for (int k0 = 16 * warp; k0 < N; k0 += 16 * kGvHWarps * U) {
+    uint32_t a[U][4], b[U][2][2];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int k = k0 + 16 * kGvHWarps * u;
+      const bool in = k < N;
+      a[u][0] = in ? ldy(g, k + 2 * c) : 0u;
+      a[u][1] = in ? ldy(g + 8, k + 2 * c) : 0u;
+      a[u][2] = in ? ldy(g, k + 2 * c + 8) : 0u;
+      a[u][3] = in ? ldy(g + 8, k + 2 * c + 8) : 0u;
+#pragma unroll
+      for (int jt = 0; jt < 2; ++jt) {
+        b[u][jt][0] = in ? ldb(8 * jt + g, k + 2 * c) : 0u;
+        b[u][jt][1] = in ? ldb(8 * jt + g, k + 2 * c + 8) : 0u;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int jt = 0; jt < 2; ++jt) mma_16816(acc[jt], a[u][0], a[u][1], a[u][2], a[u][3], b[u][jt][0], b[u][jt][1]);
+  }
+#pragma unroll
+  for (int jt = 0; jt < 2; ++jt) {
+    const int j = 8 * jt + 2 * c;
+    red[warp][g * 16 + j] = acc[jt][0];
+    red[warp][g * 16 + j + 1] = acc[jt][1];
+    red[warp][(g + 8) * 16 + j] = acc[jt][2];
+    red[warp][(g + 8) * 16 + j + 1] = acc[jt][3];
+  }
+  __syncthreads();
+  if (threadIdx.x < 256) {
+    float v = 0.f;
+    for (int w = 0; w < kGvHWarps; ++w) v += red[w][threadIdx.x];
+    const int m = threadIdx.x >> 4, j = threadIdx.x & 15;
+    if (m < M) {
+      const float x = j < r ? scale * v : 0.f;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+      la[(long)m * 2 * RP + j] = hi;
+      la[(long)m * 2 * RP + RP + j] = __float2bfloat16_rn(x - __bfloat162float(hi));
+      for (int jj = 16 + j; jj < RP; jj += 16) {
+        la[(long)m * 2 * RP + jj] = __float2bfloat16(0.f);
+        la[(long)m * 2 * RP + RP + jj] = __float2bfloat16(0.f);
+      }
+    }
+  }
+  for (int i = threadIdx.x; i < M * RP; i += blockDim.x) {
+    const int m = i / RP, j = i % RP;
+    const float x = j < r ? scale * H[m * r + j] : 0.f;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+    hs[(long)m * 2 * RP + j] = hi;
+    hs[(long)m * 2 * RP + RP + j] = __float2bfloat16_rn(x - __bfloat162float(hi));
+  }
+}
+
 // The weight-streaming kernel (stream-K over row blocks x K steps; see GvParams).
 template <int QT, int MT>
 __global__ void __launch_bounds__(kGvThreads, 2) qgemv_fwd_kernel(const __grid_constant__ CUtensorMap tmW,
@@ -627,31 +709,47 @@ __global__ void __launch_bounds__(256) qgemv_dx_finish_kernel(const float* __res
                                                               int nb, int T, int G, const __nv_bfloat16* __restrict__ LA,
                                                               int RP, const __nv_bfloat16* __restrict__ A, int r, int M,
                                                               int K, void* __restrict__ dX, int dx_dtype) {
-  __shared__ float gs[16][64];
+  __shared__ float gs[8][64];
   pdl_wait();
   pdl_launch_dependents();
-  for (int i = threadIdx.x; i < 16 * 64; i += blockDim.x) {
+  for (int i = threadIdx.x; i < 8 * 64; i += blockDim.x) {
     const int m = i >> 6, j = i & 63;
     gs[m][j] = (m < M && j < r)
                    ? __bfloat162float(LA[(long)m * 2 * RP + j]) + __bfloat162float(LA[(long)m * 2 * RP + RP + j])
                    : 0.f;
   }
-  __syncthreads();
   const int kg = blockIdx.x;
   const long t0 = (long)kg * nb;
   const int cfirst = gv_cta_of(t0, T, G);
   const int np = gv_cta_of(t0 + nb - 1, T, G) - cfirst + 1;
   const long sz = (long)xr * 256;
-  const float* gb = gpart + (long)kg * maxslots * sz;
-  for (int i = threadIdx.x; i < M * 256; i += blockDim.x) {
-    const int m = i >> 8, kk = i & 255, k = kg * 256 + kk;
-    float y = 0.f;
-    for (int q = 0; q < np; ++q) y += gb[q * sz + m * 256 + kk];
-    float l = 0.f;
-    for (int j = 0; j < r; ++j) l = fmaf(gs[m][j], __bfloat162float(A[(long)j * K + k]), l);
-    y += l;
-    if (dx_dtype == QL_F32) reinterpret_cast<float*>(dX)[(long)m * K + k] = y;
-    else reinterpret_cast<__nv_bfloat16*>(dX)[(long)m * K + k] = __float2bfloat16_rn(y);
+  const float* gb = gpart + (long)kg * maxslots * sz + threadIdx.x;
+  const int k = kg * 256 + threadIdx.x;
+  // thread = output column k for every token (M <= 8): the slot loads of all tokens, then the
+  // adapter column, go out together
+  float y[8];
+#pragma unroll
+  for (int m = 0; m < 8; ++m) y[m] = 0.f;
+  for (int q = 0; q < np; ++q)
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+      if (m < M) y[m] += gb[q * sz + m * 256];
+  float l[8];
+#pragma unroll
+  for (int m = 0; m < 8; ++m) l[m] = 0.f;
+  __syncthreads();  // gs
+#pragma unroll 8
+  for (int j = 0; j < r; ++j) {
+    const float av = __bfloat162float(A[(long)j * K + k]);
+#pragma unroll
+    for (int m = 0; m < 8; ++m) l[m] = fmaf(gs[m][j], av, l[m]);
+  }
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    if (m >= M) break;
+    const float v = y[m] + l[m];
+    if (dx_dtype == QL_F32) reinterpret_cast<float*>(dX)[(long)m * K + k] = v;
+    else reinterpret_cast<__nv_bfloat16*>(dX)[(long)m * K + k] = __float2bfloat16_rn(v);
   }
 }
 

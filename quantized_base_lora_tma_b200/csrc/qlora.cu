@@ -1430,10 +1430,17 @@ int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void
   // reduction's counters are zeroed on the way
   // (LB only for the tensor-core dX GEMM: the small-M dX path reads A itself)
   const bool need_lb = dX != nullptr && !gemv_dx_applies(qtype, M);
-  rc = launch_rows_dense((const __nv_bfloat16*)dY, N, (int)M, (int)N, (const __nv_bfloat16*)B, 1, r, r, scale, scale,
-                         nullptr, LA,
-                         need_lb ? BopArgs{(const __nv_bfloat16*)A, 1, K, (int)K} : BopArgs{nullptr, 0, 0, 0}, LB, st,
-                         H, scale, HS, (int*)crws, ncr);
+  if (dX != nullptr && gemv_dx_applies(qtype, M) && r <= 16) {
+    // a handful of token rows: one CTA (the weight stream after it does not need LB)
+    PdlLaunch L(dim3(1), dim3(kGvHWarps * 32), 0, st);
+    rc = launch_result(cudaLaunchKernelEx(&L.cfg, gemv_g_kernel, (const __nv_bfloat16*)dY, (const __nv_bfloat16*)B, H,
+                                          (int)M, (int)N, r, scale, lora_rp(r), LA, HS, (int*)crws, ncr));
+  } else {
+    rc = launch_rows_dense((const __nv_bfloat16*)dY, N, (int)M, (int)N, (const __nv_bfloat16*)B, 1, r, r, scale,
+                           scale, nullptr, LA,
+                           need_lb ? BopArgs{(const __nv_bfloat16*)A, 1, K, (int)K} : BopArgs{nullptr, 0, 0, 0}, LB,
+                           st, H, scale, HS, (int*)crws, ncr);
+  }
   if (rc) return rc;
   if (dX && gemv_dx_applies(qtype, M)) {
     // weight streaming: W read once, G A added in the finish launch

@@ -95,6 +95,8 @@ SMALL = [
     (1100, 4096, 512, 8),  # the same for the input-gradient GEMM
     (9, 1280, 192, 16),    # decode path: two token tiles, two adapter tiles, K steps not a multiple of the split
     (13, 768, 64, 12),     # decode path: one row block, ragged rank
+    (7, 512, 384, 16),     # small-M backward: G in one CTA (Q4_0), full adapter tile
+    (5, 768, 256, 12),     # the same with a ragged rank
     (4500, 256, 320, 8),   # adapter gradients from three row chunks (partials summed in chunk order)
     (2600, 256, 192, 40),  # the same with r > 32 (128-row tiles)
 ]
