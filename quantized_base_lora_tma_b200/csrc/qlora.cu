@@ -573,9 +573,13 @@ static std::atomic<int> g_rows_fusion{1};
 // one wave of clusters and leave at least one idle; the row clusters take the idle ones, as many as
 // give every CTA one 128-row block, and fusion is used only when no CTA gets more than three (so
 // the row products end well before the tiles' main loops). The input-gradient direction stages the
-// adapter B [N x r] by TMA, whose rows must be a multiple of 16 bytes: r % 8 == 0.
-static int dense_fuse_rx(int qtype, int64_t M, int64_t Nd, int64_t Kd, bool trans, int r) {
+// adapter B [N x r] by TMA, whose rows must be a multiple of 16 bytes: r % 8 == 0. Not while the
+// stream is being captured into a graph: the launch's counter tag is a kernel argument, and every
+// replay of the graph would reuse it.
+static int dense_fuse_rx(int qtype, int64_t M, int64_t Nd, int64_t Kd, bool trans, int r, cudaStream_t st) {
   if (!(g_rows_fusion.load(std::memory_order_relaxed) & (trans ? 2 : 1))) return 0;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return 0;
   const DensePlan d = plan_dense(M, Nd, Kd, trans, true);
   if (d.ms == 0 || d.ksplit != 1) return 0;
   if (trans && r % 8 != 0) return 0;
@@ -1089,7 +1093,7 @@ int qlora_linear_fwd(int qtype, const void* wq, int64_t N, int64_t K, const void
   // X and A [r x K] in kc-chunk boxes (A's rows past r read as zero)
   CUtensorMap tRY, tZ;
   int kc = 1, stages = 0;
-  int rx = dense_fuse_rx(qtype, M, N, K, false, r);
+  int rx = dense_fuse_rx(qtype, M, N, K, false, r, st);
   if (rx > 0) {
     fuse_ring(qtype, false, plan_dense(M, N, K, false, true).ms, lora_nt(r), kc, stages);
     if (!tmap_bf16_chunks(&tRY, X, K, M, 128, kc) || !tmap_bf16_chunks(&tZ, A, K, r, 8 * lora_nt(r), kc))
@@ -1385,7 +1389,7 @@ int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void
   // dY in kc-chunk boxes, and B [N x r] as boxes of 64 kc rows x RN (columns past r read as zero)
   CUtensorMap tRY, tZ;
   int kc = 1, stages = 0;
-  int rx = dX != nullptr && !gemv_dx_applies(qtype, M) ? dense_fuse_rx(qtype, M, K, N, true, r) : 0;
+  int rx = dX != nullptr && !gemv_dx_applies(qtype, M) ? dense_fuse_rx(qtype, M, K, N, true, r, st) : 0;
   if (rx > 0) {
     fuse_ring(qtype, true, plan_dense(M, K, N, true, true).ms, lora_nt(r), kc, stages);
     if (!tmap_bf16_chunks(&tRY, dY, N, M, 128, kc) ||

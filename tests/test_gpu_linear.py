@@ -302,3 +302,46 @@ def test_linear_repeated_launches_complete(qtype):
     rc, site = ql.qlora_device_status(reset=False)
     assert rc == 0, f"bounded wait gave up at site {site}"
     assert torch.equal(first[0], Y) and torch.equal(first[1], dX)
+
+
+def test_linear_cuda_graph_replay():
+    """Forward and backward captured once into a CUDA graph and replayed with new inputs copied into
+    the same buffers: every replay matches the oracle of its own inputs. (Under capture the row
+    products run in their own launch: a fused launch's counter tag would repeat on every replay.)"""
+    cases = [inp.linear_case(700, 1024, 768, inp.Q8_0, 16, 32.0, seed=s) for s in (21, 22)]
+    c0 = cases[0]
+    M, N, K, r = c0.M, c0.N, c0.K, c0.r
+    X, dY, A, B = dev_bf16(c0.X), dev_bf16(c0.dY), dev_bf16(c0.A), dev_bf16(c0.B)
+    wq = dev_u8(c0.wq)
+    ws = torch.empty(ql.qlora_linear_workspace_bytes(M, N, K, r), dtype=torch.uint8, device="cuda")
+    Y = torch.empty(M, N, dtype=torch.float32, device="cuda")
+    H = torch.empty(M, r, dtype=torch.float32, device="cuda")
+    dX = torch.empty(M, K, dtype=torch.float32, device="cuda")
+    dA = torch.empty(r, K, dtype=torch.float32, device="cuda")
+    dB = torch.empty(N, r, dtype=torch.float32, device="cuda")
+
+    def step():
+        ql.qlora_linear_fwd(c0.qtype, wq, N, K, X, A, B, r, c0.scale, Y, H, ws)
+        ql.qlora_linear_bwd(c0.qtype, wq, N, K, X, dY, A, B, r, c0.scale, H, dX, dA, dB, ws)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step()  # warm-up outside the capture (lazy per-kernel set-up)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    for c in cases + cases[:1]:
+        X.copy_(dev_bf16(c.X))
+        dY.copy_(dev_bf16(c.dY))
+        A.copy_(dev_bf16(c.A))
+        B.copy_(dev_bf16(c.B))
+        wq.copy_(dev_u8(c.wq))
+        g.replay()
+        torch.cuda.synchronize()
+        refs = oracle_linear(c)
+        for got, ref, name in zip([Y, H, dX, dA, dB], refs, ["Y", "H", "dX", "dA", "dB"]):
+            assert_close(f64(got), ref, name)
+    del g
