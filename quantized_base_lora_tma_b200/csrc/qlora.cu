@@ -5,6 +5,7 @@
 
 #include <array>
 #include <atomic>
+#include <chrono>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -595,8 +596,15 @@ static int dense_fuse_rx(int qtype, int64_t M, int64_t Nd, int64_t Kd, bool tran
 // M / 256), 8 bytes each. Tags are launch sequence numbers, unique within the process (the start is
 // random, so a reloaded library does not meet its predecessor's tags in a reused workspace).
 static size_t fuse_ctr_bytes(int64_t M) { return (size_t)(2 + (M + 255) / 256) * 8; }
+static unsigned fuse_seq_start() {
+  try {
+    return (unsigned)std::random_device{}();
+  } catch (...) {  // no entropy source: the clock will do
+    return (unsigned)std::chrono::steady_clock::now().time_since_epoch().count();
+  }
+}
 static unsigned next_fuse_seq() {
-  static std::atomic<unsigned> seq{(unsigned)std::random_device{}()};
+  static std::atomic<unsigned> seq{fuse_seq_start()};
   return seq.fetch_add(1, std::memory_order_relaxed) + 1u;
 }
 static int lora_nt(int r) { return r <= 16 ? 2 : (r <= 32 ? 4 : 8); }
