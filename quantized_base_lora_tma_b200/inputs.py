@@ -280,6 +280,61 @@ def moe_case(T, H, I, E, k, qtype, r, alpha, seed=0, zipf_s=0.0, w_std=0.02, b_s
                    to_bf16_bits(A_gu), to_bf16_bits(B_gu), to_bf16_bits(A_d), to_bf16_bits(B_d))
 
 
+def synth_q4_k(rng, rows: int, cols: int) -> np.ndarray:
+    """Valid Q4_K superblocks drawn directly as bytes, [rows x cols/256 x 144]: fp16 d uniform in
+    [1.0e-4, 1.6e-4), fp16 dmin uniform in [0.8e-3, 1.2e-3), 6-bit sc and m uniform in [32, 64), 4-bit
+    codes uniform. The weights d sc q - dmin m then spread over about +-0.05 (std near 0.027), the
+    scale of an N(0, 0.02) weight, without encoding the fp32 weights first."""
+    nb = rows * (cols // 256)
+    out = np.empty((nb, 144), np.uint8)
+    d16 = rng.uniform(1.0e-4, 1.6e-4, nb).astype(np.float16)
+    dm16 = rng.uniform(0.8e-3, 1.2e-3, nb).astype(np.float16)
+    sc = rng.integers(32, 64, (nb, 8), dtype=np.uint8)
+    m = rng.integers(32, 64, (nb, 8), dtype=np.uint8)
+    out[:, 0:2] = d16.view(np.uint8).reshape(-1, 2)
+    out[:, 2:4] = dm16.view(np.uint8).reshape(-1, 2)
+    for j in range(4):
+        out[:, 4 + j] = (sc[:, j] & 63) | ((sc[:, j + 4] >> 4) << 6)
+        out[:, 8 + j] = (m[:, j] & 63) | ((m[:, j + 4] >> 4) << 6)
+        out[:, 12 + j] = (sc[:, j + 4] & 15) | ((m[:, j + 4] & 15) << 4)
+    out[:, 16:] = rng.integers(0, 256, (nb, 128), dtype=np.uint8)
+    return out.reshape(rows, -1)
+
+
+_MOE256 = {}
+
+
+def moe_q4_k_256x4096x1536(T, seed=0):
+    """Skewed, weight-bound MoE: T tokens, hidden 4096, 256 experts of intermediate 1536, top-8,
+    Q4_K, Zipf(1.1) popularity bias on the logits, rank 4, alpha 8 on gate/up and down.
+
+    The layer shape is fixed and its weights are the same for every T: they and the adapters come
+    from default_rng(seed), in the order W_gu_e, W_d_e for e = 0..255 (drawn as Q4_K blocks by
+    synth_q4_k), then A_gu, B_gu, A_d, B_d; X, dY and the logits come from default_rng([seed, T]).
+    The packed weights are kept between calls (2.7 GB)."""
+    H, I, E, k, r = 4096, 1536, 256, 8, 4
+    if seed not in _MOE256:
+        rng = np.random.default_rng(seed)
+        w_gu = np.empty((E, 2 * I, row_bytes(Q4_K, H)), np.uint8)
+        w_d = np.empty((E, H, row_bytes(Q4_K, I)), np.uint8)
+        for e in range(E):
+            w_gu[e] = synth_q4_k(rng, 2 * I, H)
+            w_d[e] = synth_q4_k(rng, H, I)
+        A_gu = to_bf16_bits(_normal(rng, (E, r, H), 1.0 / math.sqrt(H)))
+        B_gu = to_bf16_bits(_normal(rng, (E, 2 * I, r), 0.01))
+        A_d = to_bf16_bits(_normal(rng, (E, r, I), 1.0 / math.sqrt(I)))
+        B_d = to_bf16_bits(_normal(rng, (E, H, r), 0.01))
+        _MOE256.clear()
+        _MOE256[seed] = (w_gu, w_d, A_gu, B_gu, A_d, B_d)
+    w_gu, w_d, A_gu, B_gu, A_d, B_d = _MOE256[seed]
+    rng = np.random.default_rng([seed, T])
+    X = _normal(rng, (T, H), 1.0)
+    dY = _normal(rng, (T, H), 1.0)
+    logits = _normal(rng, (T, E), 1.0) - np.float32(1.1) * np.log(np.arange(1, E + 1, dtype=np.float32))[None, :]
+    return MoECase(f"moe_q4_k_T{T}_H4096_E256_I1536_k8_zipf", Q4_K, T, H, I, E, k, r, 8.0, to_bf16_bits(X),
+                   to_bf16_bits(dY), to_bf16_bits(logits), w_gu, w_d, A_gu, B_gu, A_d, B_d)
+
+
 def moe_q4_0_2048tok_128x768(seed=0):
     """Grouped MoE layer: 2048 tokens, hidden 2048, 128 experts of intermediate 768, top-8, Q4_0,
     rank 4, alpha 8 on gate/up and down."""

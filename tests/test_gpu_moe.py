@@ -159,3 +159,32 @@ def test_moe_q4_0_2048tok_128x768_sampled():
         g = f64(got[name])
         for e in idx0:
             assert_close(g[e], ref[name][e], f"{name}[{e}]")
+
+
+_MOE256_GAP = ("at 8 tokens, routing, Y[0], dX[0] and d_logits[0] are within the bar, but dB_gu of the most "
+               "popular expert is at 1.16e-2 RMS against the 1e-2 bar; the cause is not yet found")
+
+
+@pytest.mark.parametrize("T", [
+    pytest.param(8, marks=pytest.mark.xfail(reason=_MOE256_GAP, strict=False)),
+    pytest.param(64, marks=pytest.mark.skip(reason="not yet run on a GPU: first the 8-token gap")),
+    pytest.param(4096, marks=pytest.mark.skip(reason="not yet run on a GPU: first the 8-token gap")),
+])
+def test_moe_q4_k_256x4096x1536_zipf_sampled(T):
+    """The skewed, weight-bound MoE shape (256 experts of 1536, hidden 4096, top-8, Q4_K, Zipf(1.1)
+    popularity, rank 4) at 8, 64 and 4096 tokens: exact routing for every token; the oracle decodes
+    only token 0's 8 experts and checks token 0's output, input gradient and router-logit gradient
+    and those experts' adapter gradients (each summed over every pair the expert received)."""
+    c = inp.moe_q4_k_256x4096x1536(T)
+    R, got = run_moe(c)
+    L = gb.bf16_bits_to_f64(c.logits)
+    idx0 = [int(e) for e in om.route(L[:1], c.k)[0][0]]
+    ref, route = oracle_moe(c, experts=idx0)
+    _check_route(R, c.logits, c.k)
+    assert_close(f64(got["Y"])[0], ref["Y"][0], "Y[0]")
+    assert_close(f64(got["dX"])[0], ref["dX"][0], "dX[0]")
+    assert_close(f64(got["d_logits"])[0], ref["d_logits"][0], "d_logits[0]")
+    for name in ["dA_gu", "dB_gu", "dA_d", "dB_d"]:
+        g = f64(got[name])
+        for e in idx0:
+            assert_close(g[e], ref[name][e], f"{name}[{e}]")
