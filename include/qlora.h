@@ -50,7 +50,7 @@ typedef enum { QL_F32 = 0, QL_BF16 = 1 } ql_dtype;
 typedef enum {
   QL_OK = 0,
   QL_ERR_INVALID_ARG = 1, /* null pointer, bad enum, non-positive size */
-  QL_ERR_UNSUPPORTED = 2, /* a qtype / rank / expert count this build does not handle */
+  QL_ERR_UNSUPPORTED = 2, /* a qtype / rank / expert count the library does not handle */
   QL_ERR_SHAPE = 3,       /* a size rule is broken (e.g. K % 256 != 0) */
   QL_ERR_ALIGNMENT = 4,   /* a pointer is not 16-byte aligned */
   QL_ERR_WORKSPACE = 5,   /* ws is NULL or smaller than the query says */
