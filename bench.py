@@ -497,6 +497,18 @@ def _blas_threads():
         return os.cpu_count()
 
 
+def _cpu_model():
+    """The host CPU's model name (first processor entry of /proc/cpuinfo), or None."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def oracle_step(case, rows):
     """The oracle's forward + backward restricted to a sample of token rows (dA, dB over those rows)."""
     from oracle import gguf_blocks as gb
@@ -520,8 +532,8 @@ def cpu_baseline(case, target_s=15.0, max_rows=None):
     t0 = time.perf_counter()
     oracle_step(case, np.arange(n))
     dt = time.perf_counter() - t0
-    return {"value": n / dt, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
-            "sample": f"fp64 numpy oracle fwd+bwd on the first {n} of {rows_total} token rows "
+    return {"value": n / dt, "unit": "tokens/s", "cores": _blas_threads(), "cpu_model": _cpu_model(),
+            "kind": "oracle", "sample": f"fp64 numpy oracle fwd+bwd on the first {n} of {rows_total} token rows "
                       f"(weights decoded once per call), {dt:.1f} s"}
 
 
@@ -546,8 +558,8 @@ def run_reference(args, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl_name, "tokens_per_step_sample": n},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": f"fp64 numpy oracle fwd+bwd on {n} token rows per step"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "cpu_model": _cpu_model(),
+                         "kind": "oracle", "sample": f"fp64 numpy oracle fwd+bwd on {n} token rows per step"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
