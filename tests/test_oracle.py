@@ -337,3 +337,30 @@ def test_moe_grads_finite_differences():
             fd = (out[0] - out[1]) / (2 * h)
             g = grads[name][i]
             assert abs(fd - g) <= 1e-5 * max(1.0, abs(g)), (name, i, fd, g)
+
+
+def test_synth_q4_k_blocks_have_the_stated_fields():
+    """The 256-expert workload's weights are drawn directly as Q4_K blocks: every 6-bit scale and
+    min decodes in [32, 64), d and dmin in their stated ranges, and the weights spread over about
+    +-0.05 with a std near 0.027 (checked through the oracle's decoder and gguf-py's)."""
+    rng = np.random.default_rng(3)
+    raw = inp.synth_q4_k(rng, 64, 1024)
+    assert raw.shape == (64, 4 * 144)
+    b = raw.reshape(-1, 144)
+    sc, m = gb.q4_k_scales(b[:, 4:16])
+    assert sc.min() >= 32 and sc.max() < 64 and m.min() >= 32 and m.max() < 64
+    d = b[:, 0:2].copy().view(np.float16).astype(np.float64).ravel()
+    dmin = b[:, 2:4].copy().view(np.float16).astype(np.float64).ravel()
+    assert d.min() >= 0.99e-4 and d.max() <= 1.61e-4
+    assert dmin.min() >= 0.79e-3 and dmin.max() <= 1.21e-3
+    w = gb.decode_exact(inp.Q4_K, raw, 64, 1024)
+    assert 0.02 < w.std() < 0.035
+    assert -0.08 < w.min() and w.max() < 0.16
+    try:
+        import gguf
+        from gguf import quants
+    except ImportError:
+        return
+    want = quants.dequantize(raw, gguf.GGMLQuantizationType.Q4_K).astype(np.float32)
+    got = gb.deq_f32(inp.Q4_K, raw, 64, 1024).astype(np.float32)
+    assert np.array_equal(got.view(np.uint32), want.reshape(64, 1024).view(np.uint32))
