@@ -98,3 +98,18 @@ def test_linear_argument_errors(lib):
     assert bwd(H=None) == 1
     assert bwd(wsb=16) == 5
     assert ql.qlora_launch_count() == 0    # nothing above reached a launch
+
+
+def test_rows_fusion_switch(lib):
+    """The fusion mask is process-wide host state: set, read back through the previous value, and
+    restored (no launch, no device call)."""
+    prev = ql.qlora_set_rows_fusion(0)
+    try:
+        assert ql.qlora_set_rows_fusion(3) == 0
+        assert ql.qlora_set_rows_fusion(True) == 3
+        assert ql.qlora_set_rows_fusion(False) == 3
+        assert ql.qlora_set_rows_fusion(6) == 0      # only bits 0 and 1 are kept
+        assert ql.qlora_set_rows_fusion(1) == 2
+    finally:
+        ql.qlora_set_rows_fusion(prev)
+    assert prev == 1  # the default: the forward only
