@@ -30,14 +30,21 @@ weight), dw_tj = <dh_u, h>, dh = w_tj dh_u, sigma = 1/(1+exp(-g)):
   dA_d_e  = sum_p (s w_p dY_t B_d)^T h_p       dB_d_e  = s sum_p (w_p dY_t)^T (h_p A_d^T)
   d_logits on the k selected logits of token t: w_j (dw_j - sum_i w_i dw_i); zero elsewhere.
 
-Rounding points (``mirror=True``): the layer stores g, u, h and d[g|u] in bf16 and uses the stored
-g, u in the backward, and the bf16 h and d[g|u] in the matmuls that take them (the down projection
-and its adapter input h A_d^T; the gate/up input-gradient and its adapter input s d[g|u] B_gu); the
-oracle rounds the same values at the same places. The adapter gradients dA_d and dB_gu, which sum
-over an expert's pairs only, take h and d[g|u] at fp32 accuracy (the layer carries them as a bf16
-pair there), so the oracle uses the unrounded values for those two. The weighted pair outputs w*o
-and the pair input-gradients dx_pair are kept in fp32 (no rounding point). Weights are the bf16 decode. With
-``mirror=False`` and ``round_weights=False`` the function is smooth (finite-difference checks).
+Rounding points (``mirror=True``): the layer stores h and d[g|u] in bf16 and feeds those stored
+values to the matmuls that take them (h: the down projection, its adapter input h A_d^T and the
+routing-weight gradient <dh_u, h>; d[g|u]: the gate/up input-gradient and its adapter input
+s d[g|u] B_gu); the oracle rounds the same values at the same places. g and u are kept at fp32
+accuracy (the layer saves them in fp32), so the SwiGLU derivative takes them unrounded. The adapter
+gradients dA_d and dB_gu, which sum over an expert's pairs only, take h and d[g|u] at fp32 accuracy
+(the layer carries them as a bf16 pair there), so the oracle uses the unrounded values for those
+two. The weighted pair outputs w*o and the pair input-gradients dx_pair are kept in fp32 (no
+rounding point). Weights are the bf16 decode. With ``mirror=False`` and ``round_weights=False`` the
+function is smooth (finite-difference checks).
+
+Why g and u are not rounding points: a bf16 rounding of g or u is a decision, and an fp32 and an
+fp64 evaluation of the same value land on neighbouring bf16 values now and then; the derivative of
+SwiGLU then differs by about 2^-8 relative in that entry, and for an expert with few pairs one
+such entry can dominate an element of dB_gu (a sum over those pairs only).
 """
 from __future__ import annotations
 
@@ -114,8 +121,8 @@ def moe_fwd(Wgu, Wd, X, idx, w, counts, offsets, perm, A_gu, B_gu, A_d, B_d, s, 
         ge, ue = gu[:, :I], gu[:, I:]
         h_exact[a:b] = _silu(ge) * ue
         h[a:b] = rb(h_exact[a:b])
-        g[a:b] = rb(ge)
-        u[a:b] = rb(ue)
+        g[a:b] = ge
+        u[a:b] = ue
         Hd[a:b] = h[a:b] @ A_d[e].T
         o = h[a:b] @ Wd[e].T + s * (Hd[a:b] @ B_d[e].T)
         pair_out[a:b] = wp[a:b, None] * o

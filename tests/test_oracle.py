@@ -364,3 +364,145 @@ def test_synth_q4_k_blocks_have_the_stated_fields():
     want = quants.dequantize(raw, gguf.GGMLQuantizationType.Q4_K).astype(np.float32)
     got = gb.deq_f32(inp.Q4_K, raw, 64, 1024).astype(np.float32)
     assert np.array_equal(got.view(np.uint32), want.reshape(64, 1024).view(np.uint32))
+
+
+# ------------------------------------------------------------------------------------------------
+# MoE rounding points (mirror=True)
+# ------------------------------------------------------------------------------------------------
+def _bf16_torch(v):
+    """bf16 rounding of fp64 values through torch's own casts (fp64 -> fp32 -> bf16, nearest even):
+    an implementation that shares nothing with the oracle's bit arithmetic."""
+    return torch.from_numpy(np.asarray(v, dtype=np.float64)).to(torch.float32).to(torch.bfloat16).to(
+        torch.float64).numpy()
+
+
+def _brute_moe_rounded(X, dY, L, k, Wgu, Wd, Agu, Bgu, Ad, Bd, s, rb):
+    """The routed SwiGLU layer, forward and backward, token by token and pair by pair with explicit
+    scalar sums (no matmul, no sorting of pairs), with bf16 rounding `rb` applied where the layer
+    stores a bf16 value that a later matmul reads: h (down projection, h A_d^T, <dh_u, h>) and
+    d[g|u] (gate/up input gradient, s d[g|u] B_gu). The adapter gradients dA_d and dB_gu take the
+    unrounded h and d[g|u]; g and u are never rounded."""
+    T, H = X.shape
+    E, I, r = Wgu.shape[0], Wd.shape[2], Agu.shape[1]
+    Y = np.zeros((T, H)); dX = np.zeros((T, H)); dL = np.zeros((T, E))
+    dAgu = np.zeros_like(Agu); dBgu = np.zeros_like(Bgu); dAd = np.zeros_like(Ad); dBd = np.zeros_like(Bd)
+    for t in range(T):
+        sel = sorted(range(E), key=lambda e: (-L[t, e], e))[:k]
+        z = [math.exp(L[t, e] - L[t, sel[0]]) for e in sel]
+        w = [zi / sum(z) for zi in z]
+        x, dy = X[t], dY[t]
+        dws = []
+        for j, e in enumerate(sel):
+            hg = [sum(x[q] * Agu[e, a, q] for q in range(H)) for a in range(r)]
+            gu = [sum(x[q] * Wgu[e, n, q] for q in range(H)) + s * sum(hg[a] * Bgu[e, n, a] for a in range(r))
+                  for n in range(2 * I)]
+            g, u = gu[:I], gu[I:]
+            hx = [g[i] / (1.0 + math.exp(-g[i])) * u[i] for i in range(I)]
+            h = list(rb(hx))
+            hd = [sum(h[i] * Ad[e, a, i] for i in range(I)) for a in range(r)]
+            for n in range(H):
+                o = sum(h[i] * Wd[e, n, i] for i in range(I)) + s * sum(hd[a] * Bd[e, n, a] for a in range(r))
+                Y[t, n] += w[j] * o
+            Gd = [s * sum(dy[n] * Bd[e, n, a] for n in range(H)) for a in range(r)]
+            dhu = [sum(dy[n] * Wd[e, n, i] for n in range(H)) + sum(Gd[a] * Ad[e, a, i] for a in range(r))
+                   for i in range(I)]
+            dws.append(sum(dhu[i] * h[i] for i in range(I)))
+            sg = [1.0 / (1.0 + math.exp(-g[i])) for i in range(I)]
+            dgx = ([w[j] * dhu[i] * u[i] * sg[i] * (1.0 + g[i] * (1.0 - sg[i])) for i in range(I)]
+                   + [w[j] * dhu[i] * g[i] * sg[i] for i in range(I)])
+            dgr = list(rb(dgx))
+            Ggu = [s * sum(dgr[n] * Bgu[e, n, a] for n in range(2 * I)) for a in range(r)]
+            for q in range(H):
+                dX[t, q] += (sum(dgr[n] * Wgu[e, n, q] for n in range(2 * I))
+                             + sum(Ggu[a] * Agu[e, a, q] for a in range(r)))
+            for a in range(r):
+                for i in range(I):
+                    dAd[e, a, i] += w[j] * Gd[a] * hx[i]
+                for n in range(H):
+                    dBd[e, n, a] += s * w[j] * dy[n] * hd[a]
+                for q in range(H):
+                    dAgu[e, a, q] += Ggu[a] * x[q]
+                for n in range(2 * I):
+                    dBgu[e, n, a] += s * dgx[n] * hg[a]
+        tot = sum(w[i] * dws[i] for i in range(k))
+        for j, e in enumerate(sel):
+            dL[t, e] = w[j] * (dws[j] - tot)
+    return dict(Y=Y, dX=dX, dA_gu=dAgu, dB_gu=dBgu, dA_d=dAd, dB_d=dBd, d_logits=dL)
+
+
+def _tiny_moe_f64(seed=11, T=3, H=12, I=6, E=3, k=2, r=2):
+    rng = np.random.default_rng(seed)
+    n = lambda *shape, sd=1.0: rng.standard_normal(shape) * sd  # noqa: E731
+    return dict(X=n(T, H), dY=n(T, H), L=n(T, E), Wgu=n(E, 2 * I, H, sd=0.4), Wd=n(E, H, I, sd=0.4),
+                Agu=n(E, r, H, sd=0.3), Bgu=n(E, 2 * I, r, sd=0.3), Ad=n(E, r, I, sd=0.3), Bd=n(E, H, r, sd=0.3),
+                s=1.5, k=k)
+
+
+def _oracle_moe_f64(d, mirror):
+    idx, w, counts, offsets, perm, inv = om.route(d["L"], d["k"])
+    Y, saved = om.moe_fwd(d["Wgu"], d["Wd"], d["X"], idx, w, counts, offsets, perm, d["Agu"], d["Bgu"], d["Ad"],
+                          d["Bd"], d["s"], mirror=mirror)
+    gr = om.moe_bwd(d["Wgu"], d["Wd"], d["X"], d["dY"], idx, w, counts, offsets, perm, d["Agu"], d["Bgu"],
+                    d["Ad"], d["Bd"], d["s"], saved, mirror=mirror)
+    gr["Y"] = Y
+    gr["d_logits"] = om.scatter_d_logits(idx, gr["d_logits_sel"], d["L"].shape[1])
+    return gr, saved, (idx, w, perm)
+
+
+@pytest.mark.parametrize("mirror", [True, False])
+def test_moe_rounding_points_vs_brute_force(mirror):
+    """Each bf16 rounding point of the MoE oracle, pinned by a scalar brute-force evaluation that
+    applies torch's bf16 cast at the layer's storage points (or none, for mirror=False). Moving a
+    rounding point (rounded h into dA_d, rounded d[g|u] into dB_gu, a rounded g or u in the SwiGLU
+    derivative, a rounded pair output) changes some output by about 2^-9 relative, far above the
+    1e-12 agreement asked here."""
+    d = _tiny_moe_f64()
+    rb = _bf16_torch if mirror else (lambda v: np.asarray(v, dtype=np.float64))
+    want = _brute_moe_rounded(d["X"], d["dY"], d["L"], d["k"], d["Wgu"], d["Wd"], d["Agu"], d["Bgu"], d["Ad"],
+                              d["Bd"], d["s"], rb)
+    got, _, _ = _oracle_moe_f64(d, mirror)
+    for name in want:
+        scale = max(1.0, float(np.abs(want[name]).max()))
+        assert np.allclose(got[name], want[name], rtol=1e-12, atol=1e-12 * scale), name
+
+
+def test_moe_rounding_points_are_live_and_bounded():
+    """mirror=True differs from mirror=False (the rounding points are live), and by no more than
+    the bf16 bound: Y depends on the rounding of h only through a linear map, so
+    |Y_m - Y_x| <= sum_j w_j sum_i |dh_i| |Wd[:, i] + s Bd Ad[:, i]| with |dh_i| <= 2^-8 (1 + 2^-15) |h_i|
+    (bf16 unit roundoff 2^-8, plus the fp32 step before it); dX likewise through the rounding of
+    d[g|u] and W_gu + s B_gu A_gu."""
+    d = _tiny_moe_f64(seed=12)
+    gm, sm, (idx, w, perm) = _oracle_moe_f64(d, True)
+    gx, sx, _ = _oracle_moe_f64(d, False)
+    k = d["k"]
+    u = 2.0 ** -8 * (1 + 2.0 ** -15)
+    T, H = d["X"].shape
+    for name in ["Y", "dX", "dA_gu", "dB_d", "d_logits"]:
+        assert np.abs(gm[name] - gx[name]).max() > 1e-9, name      # the rounding reaches every output
+    # g and u are not rounding points
+    assert np.array_equal(sm["g"], sx["g"]) and np.array_equal(sm["u"], sx["u"])
+    bY = np.zeros((T, H))
+    bX = np.zeros((T, H))
+    hx = sx["h"]
+    for pos, pair in enumerate(perm):
+        t, j = divmod(int(pair), k)
+        e = idx[t, j]
+        Md = np.abs(d["Wd"][e] + d["s"] * d["Bd"][e] @ d["Ad"][e])          # [H, I]
+        bY[t] += w[t, j] * (Md @ (u * np.abs(hx[pos])))
+        Mgu = np.abs(d["Wgu"][e] + d["s"] * d["Bgu"][e] @ d["Agu"][e])      # [2I, H]
+        # d[g|u] of the pair without rounding: the smooth backward's value
+        dgu_x = _pair_dgu(d, sx, pos, t, e, w[t, j])
+        bX[t] += (u * np.abs(dgu_x)) @ Mgu
+    assert np.all(np.abs(gm["Y"] - gx["Y"]) <= bY * (1 + 1e-9) + 1e-15)
+    assert np.all(np.abs(gm["dX"] - gx["dX"]) <= bX * (1 + 1e-9) + 1e-15)
+
+
+def _pair_dgu(d, saved, pos, t, e, w):
+    """d[g|u] of one pair from the smooth (unrounded) forward values, written out elementwise."""
+    g, uu = saved["g"][pos], saved["u"][pos]
+    dy = d["dY"][t]
+    Gd = d["s"] * (dy @ d["Bd"][e])
+    dhu = dy @ d["Wd"][e] + Gd @ d["Ad"][e]
+    sg = 1.0 / (1.0 + np.exp(-g))
+    return np.concatenate([w * dhu * uu * sg * (1 + g * (1 - sg)), w * dhu * g * sg])
