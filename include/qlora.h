@@ -154,16 +154,17 @@ int qlora_moe_route(const void* logits, int64_t T, int E, int k, int32_t* topk_i
                     void* stream);
 
 /* Bytes of the activations the forward saves for the backward (caller-owned buffer `saved`):
- * g, u, h [P x I] bf16, the bf16 residual h - bf16(h) [P x I] and X A_gu^T, h A_d^T [P x r] fp32,
- * in pair order. */
+ * g, u [P x I] fp32, h [P x I] bf16, the bf16 residual h - bf16(h) [P x I] and X A_gu^T, h A_d^T
+ * [P x r] fp32, in pair order. */
 size_t qlora_moe_saved_bytes(int64_t T, int k, int64_t H, int64_t I, int r);
 
 /* Scratch bytes for qlora_moe_fwd / qlora_moe_bwd with these sizes. */
 size_t qlora_moe_workspace_bytes(int64_t T, int k, int E, int64_t H, int64_t I, int r);
 
 /* Forward. X [T x H] bf16; the routing buffers as written by qlora_moe_route; Y [T x H] of y_dtype.
- * The weighted per-pair outputs stay fp32 up to the slot-ordered fp32 sum; g, u, h are saved in
- * bf16 (h from the fp32 g, u). */
+ * The weighted per-pair outputs stay fp32 up to the slot-ordered fp32 sum; g and u are saved in
+ * fp32 (the backward's SwiGLU derivative takes them unrounded), h in bf16 (from the fp32 g, u) with
+ * its bf16 residual. */
 int qlora_moe_fwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H, int64_t I,
                   const void* X, int64_t T, int k, const int32_t* topk_idx, const float* topk_w,
                   const int32_t* offsets, const int32_t* perm, const int32_t* inv_perm,
@@ -198,11 +199,16 @@ int qlora_moe_bwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
  * return QL_ERR_WORKSPACE before any launch.
  * It calls no allocation routine of any kind.
  *
- * The first call on each device looks up the array's device address (cudaGetSymbolAddress) while
- * that device is current; make that first call before any stream capture. All calls on a device
+ * The first call in each context (per device) looks up the array's device address
+ * (cudaGetSymbolAddress) while that device is current, and looks it up again when a call finds
+ * another context current (after a device reset the library image is loaded anew and the array
+ * may move); make the first call in a context before any stream capture. All calls on a device
  * share the one array and leave their operands in it: two calls whose kernels overlap on the GPU
  * (different streams, no ordering between them) race on it and may produce wrong results; calls
- * on one stream, or otherwise ordered, are fine. Each call rewrites everything it reads. */
+ * on one stream, or otherwise ordered, are fine. Each call rewrites everything it reads.
+ * It always runs the tensor-core GEMM without a K split (the split's fp32 partials would not fit
+ * the array), also where qlora_linear_fwd would take the small-M weight stream or a K split, so
+ * decode-shaped calls (a few tokens) are slower here than through qlora_linear_fwd. */
 int qlora_linear_fwd_noalloc(int qtype, const void* wq, int64_t N, int64_t K, const void* X, int64_t M,
                              const void* A, const void* B, int r, float scale, void* Y, int y_dtype,
                              float* H, void* stream);

@@ -31,20 +31,22 @@ weight), dw_tj = <dh_u, h>, dh = w_tj dh_u, sigma = 1/(1+exp(-g)):
   d_logits on the k selected logits of token t: w_j (dw_j - sum_i w_i dw_i); zero elsewhere.
 
 Rounding points (``mirror=True``): the layer stores h and d[g|u] in bf16 and feeds those stored
-values to the matmuls that take them (h: the down projection, its adapter input h A_d^T and the
-routing-weight gradient <dh_u, h>; d[g|u]: the gate/up input-gradient and its adapter input
-s d[g|u] B_gu); the oracle rounds the same values at the same places. g and u are kept at fp32
-accuracy (the layer saves them in fp32), so the SwiGLU derivative takes them unrounded. The adapter
-gradients dA_d and dB_gu, which sum over an expert's pairs only, take h and d[g|u] at fp32 accuracy
-(the layer carries them as a bf16 pair there), so the oracle uses the unrounded values for those
-two. The weighted pair outputs w*o and the pair input-gradients dx_pair are kept in fp32 (no
+values to the matmuls that take them (h: the down projection and its adapter input h A_d^T;
+d[g|u]: the gate/up input-gradient and its adapter input s d[g|u] B_gu); the oracle rounds the same
+values at the same places. g and u are kept at fp32 accuracy (the layer saves them in fp32), so the
+SwiGLU derivative takes them unrounded. The routing-weight gradient <dh_u, h> and the adapter
+gradients dA_d and dB_gu (sums over an expert's pairs only) take h and d[g|u] at fp32 accuracy
+(the layer carries them as a bf16 pair there), so the oracle uses the unrounded values for those. The weighted pair outputs w*o and the pair input-gradients dx_pair are kept in fp32 (no
 rounding point). Weights are the bf16 decode. With ``mirror=False`` and ``round_weights=False`` the
 function is smooth (finite-difference checks).
 
-Why g and u are not rounding points: a bf16 rounding of g or u is a decision, and an fp32 and an
-fp64 evaluation of the same value land on neighbouring bf16 values now and then; the derivative of
-SwiGLU then differs by about 2^-8 relative in that entry, and for an expert with few pairs one
-such entry can dominate an element of dB_gu (a sum over those pairs only).
+Why these are not rounding points: a bf16 rounding is a decision, and an fp32 and an fp64
+evaluation of the same value land on neighbouring bf16 values now and then. A flipped g or u moves
+the SwiGLU derivative by about 2^-8 relative in that entry, and for an expert with few pairs one
+such entry can dominate an element of dB_gu (a sum over those pairs only). A flipped h moves one
+term of <dh_u, h> by 2^-8 of itself, and single terms h_i dh_u_i are heavy-tailed (products of
+near-Gaussian values): one flip can move a token's router-logit gradient by more than 1e-2 of its
+RMS.
 """
 from __future__ import annotations
 
@@ -82,11 +84,33 @@ def _sigmoid(g):
     return 1.0 / (1.0 + np.exp(-g))
 
 
-def expert_weights(qtype, w_gu, w_d, H, I, round_weights=True, experts=None):
+class LazyExpertWeights:
+    """One expert's decoded weight matrix on demand (``W[e]``), keeping only the last one decoded:
+    bounds host memory when the layer is evaluated at full size, where all experts' decoded
+    weights would not fit."""
+
+    def __init__(self, qtype, packed, rows, cols, round_weights=True):
+        self.qtype, self.packed, self.rows, self.cols = qtype, packed, rows, cols
+        self.dec = deq_bf16 if round_weights else decode_exact
+        self._e, self._w = None, None
+
+    def __getitem__(self, e):
+        if e != self._e:
+            self._w = None
+            self._w = self.dec(self.qtype, self.packed[e], self.rows, self.cols)
+            self._e = e
+        return self._w
+
+
+def expert_weights(qtype, w_gu, w_d, H, I, round_weights=True, experts=None, lazy=False):
     """Decoded (W_gu [E,2I,H], W_d [E,H,I]). With `experts`, only those are decoded (the others
-    stay zero and must then be skipped by moe_fwd / moe_bwd through the same `experts`)."""
+    stay zero and must then be skipped by moe_fwd / moe_bwd through the same `experts`). With
+    `lazy`, each expert is decoded when moe_fwd / moe_bwd reach it."""
     dec = deq_bf16 if round_weights else decode_exact
     E = w_gu.shape[0]
+    if lazy:
+        return (LazyExpertWeights(qtype, w_gu, 2 * I, H, round_weights),
+                LazyExpertWeights(qtype, w_d, H, I, round_weights))
     if experts is None:
         Wgu = np.stack([dec(qtype, w_gu[e], 2 * I, H) for e in range(E)])
         Wd = np.stack([dec(qtype, w_d[e], H, I) for e in range(E)])
@@ -160,7 +184,7 @@ def moe_bwd(Wgu, Wd, X, dY, idx, w, counts, offsets, perm, A_gu, B_gu, A_d, B_d,
         dy = dY[tok[a:b]]
         Gd = s * (dy @ B_d[e])
         dh_u = dy @ Wd[e] + Gd @ A_d[e]
-        dw_p[a:b] = (dh_u * h[a:b]).sum(axis=1)
+        dw_p[a:b] = (dh_u * saved["h_exact"][a:b]).sum(axis=1)
         dh = wp[a:b, None] * dh_u
         sg = _sigmoid(g[a:b])
         dg = dh * u[a:b] * sg * (1.0 + g[a:b] * (1.0 - sg))

@@ -86,13 +86,15 @@ struct GemmParams {
   void* out;
   int out_dtype;
   long ldo;
-  __nv_bfloat16* out_g;        // SWIGLU: g, u, h [M x I]; SWIGLU_BWD: d[g|u] [M x 2I] in out_g
-  __nv_bfloat16* out_u;
-  __nv_bfloat16* out_h;
+  float* out_gf;               // SWIGLU: g, u [M x I] in fp32 (the SwiGLU derivative takes them unrounded)
+  float* out_uf;
+  __nv_bfloat16* out_h;        // SWIGLU: bf16 h [M x I]
+  __nv_bfloat16* out_g;        // SWIGLU_BWD: bf16 d[g|u] [M x 2I]
   __nv_bfloat16* out_lo;       // SWIGLU: h - bf16(h); SWIGLU_BWD: d[g|u] - bf16(d[g|u]) (nullable)
-  const __nv_bfloat16* in_g;   // SWIGLU_BWD: saved g, u, h [M x I]
-  const __nv_bfloat16* in_u;
+  const float* in_gf;          // SWIGLU_BWD: saved fp32 g, u and bf16 h, h - bf16(h) [M x I]
+  const float* in_uf;
   const __nv_bfloat16* in_h;
+  const __nv_bfloat16* in_hlo;
   const float* row_w;          // PAIR_OUT, SWIGLU_BWD: routing weight per row
   float* dw_part;              // SWIGLU_BWD: [M x num_n_tiles] partial <dh_u, h>
   // dense pair GEMM: clusters [0, rx) compute the adapter row products (0 = none: the LoRA
@@ -257,8 +259,12 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, const TileInf
             u[j] = __uint_as_float(vu[8 * i + j]);
             h[j] = silu_f(g[j]) * u[j];
           }
-          *reinterpret_cast<uint4*>(p.out_g + o + 8 * i) = pack_bf16x8(g);
-          *reinterpret_cast<uint4*>(p.out_u + o + 8 * i) = pack_bf16x8(u);
+          float4* gq = reinterpret_cast<float4*>(p.out_gf + o + 8 * i);
+          float4* uq = reinterpret_cast<float4*>(p.out_uf + o + 8 * i);
+          gq[0] = make_float4(g[0], g[1], g[2], g[3]);
+          gq[1] = make_float4(g[4], g[5], g[6], g[7]);
+          uq[0] = make_float4(u[0], u[1], u[2], u[3]);
+          uq[1] = make_float4(u[4], u[5], u[6], u[7]);
           uint4 hh, hl;
           split_bf16x8(h, hh, hl);
           *reinterpret_cast<uint4*>(p.out_h + o + 8 * i) = hh;
@@ -279,19 +285,25 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, const TileInf
         const long o = (long)row * p.I + j0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const uint4 gq = *reinterpret_cast<const uint4*>(p.in_g + o + 8 * i);
-          const uint4 uq = *reinterpret_cast<const uint4*>(p.in_u + o + 8 * i);
+          const float4 g0 = *reinterpret_cast<const float4*>(p.in_gf + o + 8 * i);
+          const float4 g1 = *reinterpret_cast<const float4*>(p.in_gf + o + 8 * i + 4);
+          const float4 u0 = *reinterpret_cast<const float4*>(p.in_uf + o + 8 * i);
+          const float4 u1 = *reinterpret_cast<const float4*>(p.in_uf + o + 8 * i + 4);
           const uint4 hq = *reinterpret_cast<const uint4*>(p.in_h + o + 8 * i);
-          const __nv_bfloat16* gb = reinterpret_cast<const __nv_bfloat16*>(&gq);
-          const __nv_bfloat16* ub = reinterpret_cast<const __nv_bfloat16*>(&uq);
+          const uint4 hlq = *reinterpret_cast<const uint4*>(p.in_hlo + o + 8 * i);
+          const float gb[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+          const float ub[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
           const __nv_bfloat16* hb = reinterpret_cast<const __nv_bfloat16*>(&hq);
+          const __nv_bfloat16* hlb = reinterpret_cast<const __nv_bfloat16*>(&hlq);
           float dg[8], du[8];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const float a = __uint_as_float(v[8 * i + j]);
-            const float g = __bfloat162float(gb[j]);
-            const float u = __bfloat162float(ub[j]);
-            dwp = fmaf(a, __bfloat162float(hb[j]), dwp);
+            const float g = gb[j];
+            const float u = ub[j];
+            // <dh_u, h> with h at fp32 accuracy (the bf16 pair): a flip of the bf16 h alone would
+            // move a heavy-tailed term by 2^-8 of itself
+            dwp = fmaf(a, __bfloat162float(hb[j]) + __bfloat162float(hlb[j]), dwp);
             const float dh = wr * a;
             const float sg = 1.0f / (1.0f + expf(-g));
             dg[j] = dh * u * sg * (1.0f + g * (1.0f - sg));

@@ -884,8 +884,8 @@ static MoeSaved moe_saved(int64_t T, int k, int64_t H, int64_t I, int r) {
   const size_t P = (size_t)T * k;
   MoeSaved m;
   size_t o = 0;
-  m.g = o; o = al256(o + P * I * 2);
-  m.u = o; o = al256(o + P * I * 2);
+  m.g = o; o = al256(o + P * I * 4);
+  m.u = o; o = al256(o + P * I * 4);
   m.h = o; o = al256(o + P * I * 2);
   m.hlo = o; o = al256(o + P * I * 2);
   m.hgu = o; o = al256(o + P * r * 4);
@@ -1196,8 +1196,8 @@ int qlora_moe_fwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
   float* row_w = (float*)(wb + w.row_w);
   __nv_bfloat16* LA = (__nv_bfloat16*)(wb + w.la);
   __nv_bfloat16* LB = (__nv_bfloat16*)(wb + w.lb);
-  __nv_bfloat16* g = (__nv_bfloat16*)(sb + sv.g);
-  __nv_bfloat16* u = (__nv_bfloat16*)(sb + sv.u);
+  float* g = (float*)(sb + sv.g);
+  float* u = (float*)(sb + sv.u);
   __nv_bfloat16* h = (__nv_bfloat16*)(sb + sv.h);
   float* Hgu = (float*)(sb + sv.hgu);
   float* Hd = (float*)(sb + sv.hd);
@@ -1224,7 +1224,7 @@ int qlora_moe_fwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
     p.M = P; p.Nd = (int)(2 * I); p.Kd = (int)H; p.n_lora_kb = KL / 64; p.num_n_tiles = (int)(I / (bn / 2));
     p.w_rows_per_expert = (int)(2 * I); p.lb_rows_per_expert = (int)(2 * I); p.I = (int)I;
     p.E = E; p.seg_off = off; p.mblk_off = mblk; p.ksplit = 1;
-    p.out_g = g; p.out_u = u; p.out_h = h; p.out_lo = (__nv_bfloat16*)(sb + sv.hlo);
+    p.out_gf = g; p.out_uf = u; p.out_h = h; p.out_lo = (__nv_bfloat16*)(sb + sv.hlo);
     rc = launch_qgemm_q<false, EPI_SWIGLU, 1>(qtype, tA, tW, tLA, tLB, p, nsm, st, 2, bn);
     if (rc) return rc;
   }
@@ -1291,8 +1291,8 @@ int qlora_moe_bwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
   float* dwp = (float*)(wb + w.dwp);
   float* dxp = (float*)(wb + w.dxp);
   float* part = (float*)(wb + w.part);
-  const __nv_bfloat16* g = (const __nv_bfloat16*)(sb + sv.g);
-  const __nv_bfloat16* u = (const __nv_bfloat16*)(sb + sv.u);
+  const float* g = (const float*)(sb + sv.g);
+  const float* u = (const float*)(sb + sv.u);
   const __nv_bfloat16* h = (const __nv_bfloat16*)(sb + sv.h);
   const __nv_bfloat16* h_lo = (const __nv_bfloat16*)(sb + sv.hlo);
   const float* Hgu = (const float*)(sb + sv.hgu);
@@ -1323,7 +1323,7 @@ int qlora_moe_bwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
     p.M = P; p.Nd = (int)I; p.Kd = (int)H; p.n_lora_kb = KL / 64; p.num_n_tiles = dw_tiles;
     p.w_rows_per_expert = (int)H; p.lb_rows_per_expert = (int)I; p.I = (int)I;
     p.E = E; p.seg_off = off; p.mblk_off = mblk; p.ksplit = 1;
-    p.in_g = g; p.in_u = u; p.in_h = h; p.out_g = dgu; p.out_lo = dgu_lo; p.row_w = row_w; p.dw_part = dwp;
+    p.in_gf = g; p.in_uf = u; p.in_h = h; p.in_hlo = h_lo; p.out_g = dgu; p.out_lo = dgu_lo; p.row_w = row_w; p.dw_part = dwp;
     rc = launch_qgemm_q<true, EPI_SWIGLU_BWD, 1>(qtype, tA, tW, tLA, tLB, p, nsm, st, 4, grouped_bn(qtype, I, 256));
     if (rc) return rc;
   }
@@ -1483,18 +1483,43 @@ static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
 constexpr int kMaxDevices = 64;
 static std::mutex g_static_scratch_mu;
+// per device: the context the address was looked up in, and the address
+static void* g_static_scratch_ctx[kMaxDevices] = {};
 static void* g_static_scratch_dev[kMaxDevices] = {};
 
-// Device address of g_static_scratch on the current device; looked up on the first use per device.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+static CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+// Device address of g_static_scratch in the current device's current context. It is looked up
+// (cudaGetSymbolAddress) on the first use in a context and again whenever the context differs
+// from the one it was looked up in: after a device reset the module is loaded anew and the array
+// may sit elsewhere.
 static int static_scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return QL_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return QL_ERR_UNSUPPORTED;
+  CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+  CUcontext ctx = nullptr;
+  if (get_ctx == nullptr || get_ctx(&ctx) != CUDA_SUCCESS) return QL_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_static_scratch_mu);
-  if (g_static_scratch_dev[dev] == nullptr) {
+  if (ctx == nullptr || g_static_scratch_dev[dev] == nullptr || g_static_scratch_ctx[dev] != (void*)ctx) {
     void* ptr = nullptr;
+    // also makes the device's primary context current if no context was
     if (cudaGetSymbolAddress((void**)&ptr, g_static_scratch) != cudaSuccess || ptr == nullptr) return QL_ERR_CUDA;
+    if (ctx == nullptr && (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr)) return QL_ERR_CUDA;
     g_static_scratch_dev[dev] = ptr;
+    g_static_scratch_ctx[dev] = (void*)ctx;
   }
   *out = g_static_scratch_dev[dev];
   return QL_OK;

@@ -282,15 +282,16 @@ def moe_case(T, H, I, E, k, qtype, r, alpha, seed=0, zipf_s=0.0, w_std=0.02, b_s
 
 def synth_q4_k(rng, rows: int, cols: int) -> np.ndarray:
     """Valid Q4_K superblocks drawn directly as bytes, [rows x cols/256 x 144]: fp16 d uniform in
-    [1.0e-4, 1.6e-4), fp16 dmin uniform in [0.8e-3, 1.2e-3), 6-bit sc and m uniform in [32, 64), 4-bit
-    codes uniform. The weights d sc q - dmin m then spread over about +-0.05 (std near 0.027), the
-    scale of an N(0, 0.02) weight, without encoding the fp32 weights first."""
+    [1.0e-4, 1.6e-4), fp16 dmin uniform in [0.8e-3, 1.2e-3), 6-bit sc and m uniform over all 64
+    values (so both halves of the split of sub-blocks 4..7, whose top two bits live in bytes 0..7,
+    occur), 4-bit codes uniform. The weights d sc q - dmin m then spread over about -0.07..0.14
+    (std near 0.035), the scale of an N(0, 0.02) weight, without encoding the fp32 weights first."""
     nb = rows * (cols // 256)
     out = np.empty((nb, 144), np.uint8)
     d16 = rng.uniform(1.0e-4, 1.6e-4, nb).astype(np.float16)
     dm16 = rng.uniform(0.8e-3, 1.2e-3, nb).astype(np.float16)
-    sc = rng.integers(32, 64, (nb, 8), dtype=np.uint8)
-    m = rng.integers(32, 64, (nb, 8), dtype=np.uint8)
+    sc = rng.integers(0, 64, (nb, 8), dtype=np.uint8)
+    m = rng.integers(0, 64, (nb, 8), dtype=np.uint8)
     out[:, 0:2] = d16.view(np.uint8).reshape(-1, 2)
     out[:, 2:4] = dm16.view(np.uint8).reshape(-1, 2)
     for j in range(4):

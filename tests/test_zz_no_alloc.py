@@ -1,5 +1,5 @@
 """The forward entry point that allocates nothing (qlora_linear_fwd_noalloc) against the regular
-forward with a caller-provided workspace.
+forward with a caller-provided workspace and against the oracle.
 
 Some callers cannot allocate device memory (their device pool is owned by a caching allocator, or
 an allocation's device-wide synchronisation is not acceptable where they run), so they cannot pass a
@@ -17,6 +17,9 @@ if torch.cuda.is_available():
     import quantized_base_lora_tma_b200 as ql
     from tests.gpu_util import assert_close, dev_bf16, dev_u8, f64
 
+from oracle import gguf_blocks as gb
+from oracle import lora_linear as ll
+
 
 def _forward_both(c):
     X, A, B = dev_bf16(c.X), dev_bf16(c.A), dev_bf16(c.B)
@@ -33,15 +36,30 @@ def _forward_both(c):
     return f64(Y_ws), f64(H_ws), f64(Y_na), f64(H_na)
 
 
+def _oracle_fwd(c):
+    W = ll.weights(c.qtype, c.wq, c.N, c.K)
+    f = gb.bf16_bits_to_f64
+    return ll.linear_fwd(W, f(c.X), f(c.A), f(c.B), c.scale)
+
+
+# (M, K, N, qtype, r): pair-tile sizes, the decode-sized and single-tile sizes where the regular
+# forward takes the weight stream or a K split and this one the plain single-CTA GEMM, and a size
+# whose adapter operands fill the 4 MiB array exactly ((512 + 32256) rows x 128 bytes).
+NOALLOC_CASES = [(300, 512, 384, inp.Q4_K, 16), (129, 768, 320, inp.Q8_0, 40), (4, 1024, 512, inp.Q4_0, 16),
+                 (64, 512, 640, inp.Q4_K, 8), (512, 256, 32256, inp.Q4_0, 4)]
+
+
 def test_noalloc_forward_matches_workspace_forward_twice():
     ql.qlora_device_status(reset=True)
-    # two calls in a row, the second with other sizes and values than the first
-    cases = [inp.linear_case(300, 512, 384, inp.Q4_K, 16, 32.0, seed=21),
-             inp.linear_case(129, 768, 320, inp.Q8_0, 40, 80.0, seed=22)]
-    for c in cases:
+    # calls in a row, each with other sizes and values than the one before
+    for i, (M, K, N, qt, r) in enumerate(NOALLOC_CASES):
+        c = inp.linear_case(M, K, N, qt, r, 2.0 * r, seed=21 + i)
         Y_ws, H_ws, Y_na, H_na = _forward_both(c)
-        assert_close(Y_na, Y_ws, "Y")
-        assert_close(H_na, H_ws, "H")
+        assert_close(Y_na, Y_ws, f"Y vs workspace forward {M}x{K}x{N}")
+        assert_close(H_na, H_ws, f"H vs workspace forward {M}x{K}x{N}")
+        Yr, Hr = _oracle_fwd(c)
+        assert_close(Y_na, Yr, f"Y vs oracle {M}x{K}x{N}")
+        assert_close(H_na, Hr, f"H vs oracle {M}x{K}x{N}")
     rc, site = ql.qlora_device_status(reset=True)
     assert rc == 0, (rc, site)
 
@@ -52,6 +70,10 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     # M + N far beyond the 4 MiB of static scratch: refused before any launch
     before = ql.qlora_launch_count()
     rc = lib.qlora_linear_fwd_noalloc(inp.Q4_0, fake, 65536, 256, fake, 65536, fake, fake, 16, 2.0, fake, 0,
+                                      fake, None)
+    assert rc == 5
+    # one 64-row block past the exact fit of the last case above
+    rc = lib.qlora_linear_fwd_noalloc(inp.Q4_0, fake, 32320, 256, fake, 512, fake, fake, 4, 2.0, fake, 0,
                                       fake, None)
     assert rc == 5
     assert ql.qlora_launch_count() == before
