@@ -199,14 +199,19 @@ class DenseLayerRun:
 class MoERun:
     """Device buffers and one step (route + forward + backward) of the routed MoE layer."""
 
+    _dev_weights = {}  # packed expert stacks already on the device, by host array identity
+
     def __init__(self, case):
         import quantized_base_lora_tma_b200 as ql
         self.ql = ql
         self.c = c = case
         T, H, I, E, k, r = c.T, c.H, c.I, c.E, c.k, c.r
         self.X, self.dY, self.logits = bf16_dev(c.X), bf16_dev(c.dY), bf16_dev(c.logits)
-        self.w_gu = torch.from_numpy(c.w_gu).cuda()
-        self.w_d = torch.from_numpy(c.w_d).cuda()
+        key = (id(c.w_gu), id(c.w_d))
+        if key not in MoERun._dev_weights:
+            MoERun._dev_weights.clear()
+            MoERun._dev_weights[key] = (torch.from_numpy(c.w_gu).cuda(), torch.from_numpy(c.w_d).cuda())
+        self.w_gu, self.w_d = MoERun._dev_weights[key]
         self.A_gu, self.B_gu = bf16_dev(c.A_gu), bf16_dev(c.B_gu)
         self.A_d, self.B_d = bf16_dev(c.A_d), bf16_dev(c.B_d)
         self.route = ql.MoeRoute(T, E, k)
@@ -221,19 +226,34 @@ class MoERun:
         self.dB_d = torch.empty(E, H, r, **f32)
         self.dL = torch.empty(T, E, **f32)
 
-    def step(self):
+    def fwd(self):
+        """Routing and the forward: one pass over the touched experts' weights."""
         c, ql = self.c, self.ql
         ql.qlora_moe_route(self.logits, c.k, self.route)
         ql.qlora_moe_fwd(c.qtype, self.w_gu, self.w_d, c.E, c.H, c.I, self.X, self.route, self.A_gu, self.B_gu,
                          self.A_d, self.B_d, c.r, c.scale, self.Y, self.saved, self.ws)
+
+    def bwd(self):
+        """The backward (second pass over the touched experts' weights)."""
+        c, ql = self.c, self.ql
         ql.qlora_moe_bwd(c.qtype, self.w_gu, self.w_d, c.E, c.H, c.I, self.X, self.dY, self.route, self.A_gu,
                          self.B_gu, self.A_d, self.B_d, c.r, c.scale, self.saved, self.dX, self.dA_gu, self.dB_gu,
                          self.dA_d, self.dB_d, self.dL, self.ws)
+
+    def step(self):
+        self.fwd()
+        self.bwd()
 
     def flops(self):
         c = self.c
         P = c.T * c.k
         return 12.0 * P * c.H * c.I + 6.0 * c.r * (2 * c.H + 3 * c.I) * P
+
+    def touched_weight_bytes(self):
+        """Packed weight bytes of the experts that received at least one pair (one pass)."""
+        c = self.c
+        used = int((self.route.counts > 0).sum().item())
+        return used, used * (c.w_gu[0].nbytes + c.w_d[0].nbytes)
 
 
 def allreduce_adapter_grads(grads):
@@ -243,20 +263,30 @@ def allreduce_adapter_grads(grads):
         torch.distributed.all_reduce(g, op=torch.distributed.ReduceOp.SUM)
 
 
+EV_EVERY = 8  # kernel events on one timed step in this many (as for the headline)
+
+
 def time_steps(fn, steps, warmup, flush, slots=()):
-    """Mean device time (ms) of fn() over `steps` calls, L2 flushed before each; per-slot GEMM means."""
+    """Mean device time (ms) of fn() over `steps` calls, L2 flushed before each, and per-slot GEMM
+    means. The GEMM events are recorded on one step in EV_EVERY only: an event between two kernels
+    stops the next one from starting while the previous one drains (programmatic launch), so those
+    steps are slower; they stay in the step mean, as in the headline."""
     import quantized_base_lora_tma_b200 as ql
     stream = torch.cuda.current_stream()
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-    gev = {s: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    nev = (steps + EV_EVERY - 1) // EV_EVERY
+    gev = {s: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nev)]
            for s in slots}
     for i in range(steps):
         flush.zero_()
         for s in slots:
-            ql.qlora_set_kernel_events(s, gev[s][i][0], gev[s][i][1])
+            if i % EV_EVERY == 0:
+                ql.qlora_set_kernel_events(s, gev[s][i // EV_EVERY][0], gev[s][i // EV_EVERY][1])
+            else:
+                ql.qlora_set_kernel_events(s, None, None)
         ev[i][0].record(stream)
         fn()
         ev[i][1].record(stream)
@@ -288,6 +318,31 @@ def also_measurements(flush, steps, pk):
         "experts_touched": int((m.route.counts > 0).sum().item())}
     device_status_ok("moe")
     del m
+    torch.cuda.empty_cache()
+    # skewed 256-expert Q4_K MoE: weight-bound at 8 and 64 tokens, tensor-bound at 4096
+    for T in (8, 64, 4096):
+        c = inp.moe_q4_k_256x4096x1536(T)
+        m = MoERun(c)
+        n = max(5, steps // 4) if T == 4096 else steps
+        ms, g = time_steps(m.step, n, 3, flush, slots=(2, 3, 4, 5))
+        ms_f, _ = time_steps(m.fwd, n, 3, flush)
+        ms_b, _ = time_steps(m.bwd, n, 3, flush)
+        used, wb = m.touched_weight_bytes()
+        counts = m.route.counts.cpu().numpy()
+        tf = m.flops() / (ms / 1e3) / 1e12
+        out[f"moe_q4_k_T{T}_H4096_E256_I1536_k8_r4_zipf"] = {
+            "tokens_per_s": T / (ms / 1e3), "ms_per_step": ms, "fwd_ms": ms_f, "bwd_ms": ms_b,
+            "tflops": tf, "frac_of_bf16_peak": tf / pk["bf16_tflops"],
+            "experts_touched": used, "weight_bytes_per_pass": wb,
+            "fwd_weight_gbs": wb / (ms_f / 1e3) / 1e9, "bwd_weight_gbs": wb / (ms_b / 1e3) / 1e9,
+            "fwd_frac_of_hbm": wb / (ms_f / 1e3) / 1e9 / pk["hbm_gbs"],
+            "bwd_frac_of_hbm": wb / (ms_b / 1e3) / 1e9 / pk["hbm_gbs"],
+            "gemm_ms": {"gate_up": g[2], "down": g[3], "down_dx": g[4], "gate_up_dx": g[5]},
+            "top_expert_counts": sorted((int(x) for x in counts), reverse=True)[:8]}
+        device_status_ok(f"moe256 T={T}")
+        del m
+        torch.cuda.empty_cache()
+    MoERun._dev_weights.clear()
     torch.cuda.empty_cache()
     # decode-shaped linear: weight streaming
     for M in (1, 4, 16):
@@ -564,17 +619,30 @@ def run_reference(args, rank, world):
     }
 
 
-def decode_calls(M, calls=3, bwd=False):
-    """Three forward (and, with bwd, backward) calls of the decode-shaped linear (the launches a
-    profiler captures)."""
-    import quantized_base_lora_tma_b200 as ql
+PROFILE_CASES = {
+    "dense_q8_0": lambda: DenseLayerRun(inp.dense_proj_2048x4096x4096(inp.Q8_0)),
+    "dense_q4_0": lambda: DenseLayerRun(inp.dense_proj_2048x4096x4096(inp.Q4_0)),
+    "gate_up_q4_k": lambda: DenseLayerRun(inp.gate_up_q4_k_2048x2048x12288()),
+    "moe_q4_0": lambda: MoERun(inp.moe_q4_0_2048tok_128x768()),
+    "moe256_t8": lambda: MoERun(inp.moe_q4_k_256x4096x1536(8)),
+    "moe256_t64": lambda: MoERun(inp.moe_q4_k_256x4096x1536(64)),
+    "moe256_t4096": lambda: MoERun(inp.moe_q4_k_256x4096x1536(4096)),
+    "decode_m1": lambda: DenseLayerRun(inp.decode_q4_0_8192(1)),
+    "decode_m4": lambda: DenseLayerRun(inp.decode_q4_0_8192(4)),
+    "decode_m16": lambda: DenseLayerRun(inp.decode_q4_0_8192(16)),
+}
+
+
+def profile_calls(name, calls=3, fwd_only=False):
+    """`calls` steps (or forwards) of a named workload and nothing else: the launches a profiler
+    captures. No timing, no JSON line."""
     from quantized_base_lora_tma_b200 import build
     build.build()
-    c = inp.decode_q4_0_8192(M)
-    d = DenseLayerRun(c)
+    run = PROFILE_CASES[name]()
     for _ in range(calls):
-        d.fwd() if not bwd else d.step()
-    device_status_ok(f"decode M={M}")
+        run.fwd() if fwd_only else run.step()
+    torch.cuda.synchronize()
+    device_status_ok(name)
 
 
 def main():
@@ -588,14 +656,20 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-also", action="store_true", help="skip the other shapes of the benchmark set")
-    ap.add_argument("--decode-calls", type=int, default=0, metavar="M",
-                    help="profiling driver: run the decode-shaped Q4_0 8192x8192 forward with M tokens "
-                         "three times and exit (no timing, no JSON line)")
+    ap.add_argument("--calls", default=None, choices=sorted(PROFILE_CASES),
+                    help="profiling driver: run three steps of the named workload and exit (no timing, no JSON line)")
+    ap.add_argument("--fwd-only", action="store_true", help="with --calls: forwards only")
+    ap.add_argument("--ncalls", type=int, default=3, help="with --calls: how many")
+    ap.add_argument("--decode-calls", type=int, default=0, choices=[0, 1, 4, 16], metavar="M",
+                    help="profiling driver: three forwards of the decode-shaped Q4_0 8192x8192 linear with M "
+                         "tokens (same as --calls decode_mM --fwd-only)")
     ap.add_argument("--decode-bwd", action="store_true", help="with --decode-calls: forward and backward")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.decode_calls:
-        decode_calls(args.decode_calls, bwd=args.decode_bwd)
+        args.calls, args.fwd_only = f"decode_m{args.decode_calls}", not args.decode_bwd
+    if args.calls:
+        profile_calls(args.calls, args.ncalls, args.fwd_only)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -91,10 +91,8 @@ struct GemmParams {
   __nv_bfloat16* out_h;        // SWIGLU: bf16 h [M x I]
   __nv_bfloat16* out_g;        // SWIGLU_BWD: bf16 d[g|u] [M x 2I]
   __nv_bfloat16* out_lo;       // SWIGLU: h - bf16(h); SWIGLU_BWD: d[g|u] - bf16(d[g|u]) (nullable)
-  const float* in_gf;          // SWIGLU_BWD: saved fp32 g, u and bf16 h, h - bf16(h) [M x I]
+  const float* in_gf;          // SWIGLU_BWD: saved fp32 g, u [M x I]
   const float* in_uf;
-  const __nv_bfloat16* in_h;
-  const __nv_bfloat16* in_hlo;
   const float* row_w;          // PAIR_OUT, SWIGLU_BWD: routing weight per row
   float* dw_part;              // SWIGLU_BWD: [M x num_n_tiles] partial <dh_u, h>
   // dense pair GEMM: clusters [0, rx) compute the adapter row products (0 = none: the LoRA
@@ -168,8 +166,9 @@ __device__ __forceinline__ bool gemm_tile(const GemmParams& p, int t, TileInfo& 
   ti.lora = 1;
   const int total_mb = __ldg(p.mblk_off + p.E);
   if (t >= total_mb * p.num_n_tiles) return false;
-  const int gm = t % total_mb;
-  ti.nb = t / total_mb;
+  // the output-column tiles of one 128-row block are consecutive: their A rows are read from L2
+  const int gm = t / p.num_n_tiles;
+  ti.nb = t - gm * p.num_n_tiles;
   // last expert e with mblk_off[e] <= gm
   int lo = 0, hi = p.E - 1;
   while (lo < hi) {
@@ -240,18 +239,18 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, const TileInf
       }
     }
   } else if (EPI == EPI_SWIGLU) {
-    // tile columns [0, BN/2) are gate j = nb*BN/2 + c, [BN/2, BN) are up for the same j
+    // tile columns [0, BN/2) are gate j = nb*BN/2 + c, [BN/2, BN) are up for the same j; 16 j at a time
 #pragma unroll 1
-    for (int jp = 0; jp < BN / 64; ++jp) {
-      uint32_t vg[32], vu[32];
-      tmem_ld32(tbase + 32 * jp, vg);
-      tmem_ld32(tbase + BN / 2 + 32 * jp, vu);
+    for (int jp = 0; jp < BN / 32; ++jp) {
+      uint32_t vg[16], vu[16];
+      tmem_ld16(tbase + 16 * jp, vg);
+      tmem_ld16(tbase + BN / 2 + 16 * jp, vu);
       tmem_ld_wait();
-      const int j0 = ti.nb * (BN / 2) + 32 * jp;
+      const int j0 = ti.nb * (BN / 2) + 16 * jp;
       if (valid && j0 < p.I) {
         const long o = (long)row * p.I + j0;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 2; ++i) {
           float g[8], u[8], h[8];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
@@ -273,51 +272,58 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, const TileInf
       }
     }
   } else if (EPI == EPI_SWIGLU_BWD) {
+    // dh_u = accumulator; dh = w dh_u; the SwiGLU derivative from the saved fp32 g, u; <dh_u, h>
+    // with h = silu(g) u recomputed at fp32 accuracy. The saved g, u are read-only here: 16 columns
+    // of both are loaded together ahead of the arithmetic and stores, one memory latency per batch.
+    const float* __restrict__ gin = p.in_gf;
+    const float* __restrict__ uin = p.in_uf;
+    __nv_bfloat16* __restrict__ go = p.out_g;
+    __nv_bfloat16* __restrict__ gl = p.out_lo;
     float wr = 0.0f, dwp = 0.0f;
     if (valid) wr = __ldg(p.row_w + row);
 #pragma unroll 1
-    for (int jc = 0; jc < BN / 32; ++jc) {
-      uint32_t v[32];
-      tmem_ld32(tbase + 32 * jc, v);
-      tmem_ld_wait();
-      const int j0 = ti.nb * BN + 32 * jc;
-      if (valid && j0 < p.I) {
-        const long o = (long)row * p.I + j0;
+    for (int jc = 0; jc < BN / 16; ++jc) {
+      uint32_t v[16];
+      tmem_ld16(tbase + 16 * jc, v);
+      const int j0 = ti.nb * BN + 16 * jc;
+      const bool act = valid && j0 < p.I;
+      float4 gq[4], uq[4];
+      if (act) {
+        const float4* g4 = reinterpret_cast<const float4*>(gin + (long)row * p.I + j0);
+        const float4* u4 = reinterpret_cast<const float4*>(uin + (long)row * p.I + j0);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float4 g0 = *reinterpret_cast<const float4*>(p.in_gf + o + 8 * i);
-          const float4 g1 = *reinterpret_cast<const float4*>(p.in_gf + o + 8 * i + 4);
-          const float4 u0 = *reinterpret_cast<const float4*>(p.in_uf + o + 8 * i);
-          const float4 u1 = *reinterpret_cast<const float4*>(p.in_uf + o + 8 * i + 4);
-          const uint4 hq = *reinterpret_cast<const uint4*>(p.in_h + o + 8 * i);
-          const uint4 hlq = *reinterpret_cast<const uint4*>(p.in_hlo + o + 8 * i);
-          const float gb[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-          const float ub[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-          const __nv_bfloat16* hb = reinterpret_cast<const __nv_bfloat16*>(&hq);
-          const __nv_bfloat16* hlb = reinterpret_cast<const __nv_bfloat16*>(&hlq);
+        for (int q = 0; q < 4; ++q) {
+          gq[q] = __ldg(g4 + q);
+          uq[q] = __ldg(u4 + q);
+        }
+      }
+      tmem_ld_wait();
+      if (act) {
+        const float* gf = reinterpret_cast<const float*>(gq);
+        const float* uf = reinterpret_cast<const float*>(uq);
+        const long od = (long)row * 2 * p.I + j0;
+#pragma unroll
+        for (int hlf = 0; hlf < 2; ++hlf) {
           float dg[8], du[8];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const float a = __uint_as_float(v[8 * i + j]);
-            const float g = gb[j];
-            const float u = ub[j];
-            // <dh_u, h> with h at fp32 accuracy (the bf16 pair): a flip of the bf16 h alone would
-            // move a heavy-tailed term by 2^-8 of itself
-            dwp = fmaf(a, __bfloat162float(hb[j]) + __bfloat162float(hlb[j]), dwp);
-            const float dh = wr * a;
+            const float a = __uint_as_float(v[8 * hlf + j]);
+            const float g = gf[8 * hlf + j], u = uf[8 * hlf + j];
             const float sg = 1.0f / (1.0f + expf(-g));
+            const float dh = wr * a;
             dg[j] = dh * u * sg * (1.0f + g * (1.0f - sg));
             du[j] = dh * g * sg;
+            // <dh_u, h> with h at fp32 accuracy: a flip of a bf16 h would move a heavy-tailed term
+            dwp = fmaf(a, silu_f(g) * u, dwp);
           }
-          const long od = (long)row * 2 * p.I + j0 + 8 * i;
-          uint4 gh, gl, uh, ul;
-          split_bf16x8(dg, gh, gl);
-          split_bf16x8(du, uh, ul);
-          *reinterpret_cast<uint4*>(p.out_g + od) = gh;
-          *reinterpret_cast<uint4*>(p.out_g + od + p.I) = uh;
-          if (p.out_lo != nullptr) {
-            *reinterpret_cast<uint4*>(p.out_lo + od) = gl;
-            *reinterpret_cast<uint4*>(p.out_lo + od + p.I) = ul;
+          uint4 gh, glo, uh, ulo;
+          split_bf16x8(dg, gh, glo);
+          split_bf16x8(du, uh, ulo);
+          *reinterpret_cast<uint4*>(go + od + 8 * hlf) = gh;
+          *reinterpret_cast<uint4*>(go + od + p.I + 8 * hlf) = uh;
+          if (gl != nullptr) {
+            *reinterpret_cast<uint4*>(gl + od + 8 * hlf) = glo;
+            *reinterpret_cast<uint4*>(gl + od + p.I + 8 * hlf) = ulo;
           }
         }
       }

@@ -1323,7 +1323,7 @@ int qlora_moe_bwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
     p.M = P; p.Nd = (int)I; p.Kd = (int)H; p.n_lora_kb = KL / 64; p.num_n_tiles = dw_tiles;
     p.w_rows_per_expert = (int)H; p.lb_rows_per_expert = (int)I; p.I = (int)I;
     p.E = E; p.seg_off = off; p.mblk_off = mblk; p.ksplit = 1;
-    p.in_gf = g; p.in_uf = u; p.in_h = h; p.in_hlo = h_lo; p.out_g = dgu; p.out_lo = dgu_lo; p.row_w = row_w; p.dw_part = dwp;
+    p.in_gf = g; p.in_uf = u; p.out_g = dgu; p.out_lo = dgu_lo; p.row_w = row_w; p.dw_part = dwp;
     rc = launch_qgemm_q<true, EPI_SWIGLU_BWD, 1>(qtype, tA, tW, tLA, tLB, p, nsm, st, 4, grouped_bn(qtype, I, 256));
     if (rc) return rc;
   }
