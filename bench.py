@@ -319,6 +319,15 @@ def also_measurements(flush, steps, pk):
     device_status_ok("moe")
     del m
     torch.cuda.empty_cache()
+    # routing alone at 4096 tokens, 256 experts, top-8 (the skewed workload's logits)
+    import quantized_base_lora_tma_b200 as ql
+    c = inp.moe_q4_k_256x4096x1536(4096)
+    lg = bf16_dev(c.logits)
+    R = ql.MoeRoute(c.T, c.E, c.k)
+    ms_r, _ = time_steps(lambda: ql.qlora_moe_route(lg, c.k, R), steps, 3, flush)
+    out["moe_route_T4096_E256_k8"] = {"ms": ms_r, "logit_gbs": c.logits.nbytes / (ms_r / 1e3) / 1e9}
+    device_status_ok("route")
+    del R, lg
     # skewed 256-expert Q4_K MoE: weight-bound at 8 and 64 tokens, tensor-bound at 4096
     for T in (8, 64, 4096):
         c = inp.moe_q4_k_256x4096x1536(T)

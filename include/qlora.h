@@ -141,6 +141,9 @@ int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void
  * P = T * k routed pairs.
  * ------------------------------------------------------------------------------------------- */
 
+/* Scratch bytes for qlora_moe_route: ceil(T / 32) x E int32 (the expert histograms of 32-token rows). */
+size_t qlora_moe_route_workspace_bytes(int64_t T, int E, int k);
+
 /* Routing. logits [T x E] bf16. Writes (device buffers of the caller):
  *   topk_idx [T x k] int32   selected experts, descending logit, equal logits -> lower index
  *   topk_w   [T x k] fp32    softmax over the k selected logits
@@ -148,10 +151,14 @@ int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void
  *   perm     [P] int32       pairs t*k+j sorted by (expert, token, slot); inv_perm [P] its inverse
  *   mblk     [E+1] int32     sum over earlier experts of ceil(counts/128): the grouped GEMMs' block list
  * Indices, counts, offsets, perm, inv_perm and mblk are exact (no floating point decides them
- * beyond comparisons of the bf16 logits). */
+ * beyond comparisons of the bf16 logits). Three launches: per row of 32 tokens, the top-k (a warp
+ * per token) and the row's expert histogram by warp match (no global atomics); one scan over rows
+ * and experts; per row, each pair's position from the scanned counts and the row's lane masks.
+ * ws (ws_bytes >= qlora_moe_route_workspace_bytes) holds the histograms; its contents on entry do
+ * not matter. */
 int qlora_moe_route(const void* logits, int64_t T, int E, int k, int32_t* topk_idx, float* topk_w,
                     int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv_perm, int32_t* mblk,
-                    void* stream);
+                    void* ws, size_t ws_bytes, void* stream);
 
 /* Bytes of the activations the forward saves for the backward (caller-owned buffer `saved`):
  * g, u [P x I] fp32, h [P x I] bf16, the bf16 residual h - bf16(h) [P x I] and X A_gu^T, h A_d^T

@@ -38,8 +38,9 @@ SIGNATURES = {
     "qlora_linear_workspace_bytes": (_c_sz, [_c_i64, _c_i64, _c_i64, _c_int]),
     "qlora_linear_fwd": (_c_int, [_c_int, _c_vp, _c_i64, _c_i64, _c_vp, _c_i64, _c_vp, _c_vp, _c_int, _c_f,
                                   _c_vp, _c_int, _c_vp, _c_vp, _c_sz, _c_vp]),
+    "qlora_moe_route_workspace_bytes": (_c_sz, [_c_i64, _c_int, _c_int]),
     "qlora_moe_route": (_c_int, [_c_vp, _c_i64, _c_int, _c_int, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp,
-                                 _c_vp]),
+                                 _c_vp, _c_sz, _c_vp]),
     "qlora_moe_saved_bytes": (_c_sz, [_c_i64, _c_int, _c_i64, _c_i64, _c_int]),
     "qlora_moe_workspace_bytes": (_c_sz, [_c_i64, _c_int, _c_int, _c_i64, _c_i64, _c_int]),
     "qlora_moe_fwd": (_c_int, [_c_int, _c_vp, _c_vp, _c_int, _c_i64, _c_i64, _c_vp, _c_i64, _c_int, _c_vp, _c_vp,
@@ -190,6 +191,8 @@ class MoeRoute:
         self.perm = torch.empty(P, dtype=i32, device=device)
         self.inv_perm = torch.empty(P, dtype=i32, device=device)
         self.mblk = torch.empty(E + 1, dtype=i32, device=device)
+        self.ws = torch.empty(max(1, int(lib().qlora_moe_route_workspace_bytes(T, E, k))), dtype=torch.uint8,
+                              device=device)
 
 
 def qlora_moe_route(logits, k, route=None, stream=None) -> MoeRoute:
@@ -197,7 +200,8 @@ def qlora_moe_route(logits, k, route=None, stream=None) -> MoeRoute:
     if route is None:
         route = MoeRoute(T, E, k, logits.device)
     _check(lib().qlora_moe_route(_p(logits), T, E, k, _p(route.topk_idx), _p(route.topk_w), _p(route.counts),
-                                 _p(route.offsets), _p(route.perm), _p(route.inv_perm), _p(route.mblk), _s(stream)),
+                                 _p(route.offsets), _p(route.perm), _p(route.inv_perm), _p(route.mblk),
+                                 _p(route.ws), route.ws.numel(), _s(stream)),
            "qlora_moe_route")
     return route
 

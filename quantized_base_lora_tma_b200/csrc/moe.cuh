@@ -18,118 +18,156 @@ namespace qlora {
 constexpr int kMaxExperts = 256;
 constexpr int kMaxTopK = 16;
 
-// One warp per token. E <= 256, k <= 16.
-__global__ void moe_topk_kernel(const __nv_bfloat16* __restrict__ logits, int T, int E, int k,
-                                int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
-                                int32_t* __restrict__ counts) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (warp >= T) return;
-  const __nv_bfloat16* l = logits + (long)warp * E;
-  float v[kMaxExperts / 32];
-#pragma unroll
-  for (int i = 0; i < kMaxExperts / 32; ++i) {
-    const int e = lane + 32 * i;
-    v[i] = e < E ? __bfloat162float(l[e]) : -INFINITY;
-  }
-  float sel_v[kMaxTopK];
-  int sel_e[kMaxTopK];
-  for (int j = 0; j < k; ++j) {
-    // lane-local best: larger value, then lower index (indices increase with i)
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
+constexpr int kRouteRow = 32;  // tokens per histogram row: one warp's lanes
+
+// Routing, first pass: one CTA of 32 warps per row of 32 tokens, one token per warp. The warp
+// chooses the token's top-k (lane-local best of 8 logits, then a butterfly over the lanes: larger
+// value wins, equal values go to the lower expert index); the weights are the softmax over the k
+// selected logits. The row's per-expert histogram is built without atomics on global memory: for
+// each slot, the lanes of warp 0 (one token each) that picked the same expert find each other with
+// __match_any_sync and their leader adds the group's size to the shared histogram, which becomes
+// row `blockIdx.x` of hist [rows x E].
+__global__ void __launch_bounds__(1024) moe_route_select_kernel(const __nv_bfloat16* __restrict__ logits, int T,
+                                                                int E, int k, int32_t* __restrict__ topk_idx,
+                                                                float* __restrict__ topk_w,
+                                                                int32_t* __restrict__ hist) {
+  __shared__ int s_hist[kMaxExperts];
+  __shared__ uint8_t s_sel[kRouteRow][kMaxTopK];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kRouteRow + warp;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
+  if (t < T) {
+    const __nv_bfloat16* l = logits + (long)t * E;
+    float v[kMaxExperts / 32];
 #pragma unroll
     for (int i = 0; i < kMaxExperts / 32; ++i) {
       const int e = lane + 32 * i;
-      if (e < E && (v[i] > bv || (v[i] == bv && e < be))) { bv = v[i]; be = e; }
+      v[i] = e < E ? __bfloat162float(l[e]) : -INFINITY;
     }
+    float sel_v[kMaxTopK];
+    int sel_e[kMaxTopK];
+    for (int j = 0; j < k; ++j) {
+      float bv = -INFINITY;
+      int be = 0x7fffffff;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+      for (int i = 0; i < kMaxExperts / 32; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E && (v[i] > bv || (v[i] == bv && e < be))) { bv = v[i]; be = e; }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+      }
+      sel_v[j] = bv;
+      sel_e[j] = be;
+#pragma unroll
+      for (int i = 0; i < kMaxExperts / 32; ++i)  // never selected again
+        if (lane + 32 * i == be) v[i] = -INFINITY;
     }
-    sel_v[j] = bv;
-    sel_e[j] = be;
-    // a selected expert can never be selected again: mark it below every finite logit
-#pragma unroll
-    for (int i = 0; i < kMaxExperts / 32; ++i)
-      if (lane + 32 * i == be) v[i] = -INFINITY;
+    if (lane == 0) {
+      const float vmax = sel_v[0];
+      float w[kMaxTopK];
+      float sum = 0.f;
+      for (int j = 0; j < k; ++j) {
+        w[j] = expf(sel_v[j] - vmax);
+        sum += w[j];
+      }
+      const float inv = 1.0f / sum;
+      for (int j = 0; j < k; ++j) {
+        topk_idx[(long)t * k + j] = sel_e[j];
+        topk_w[(long)t * k + j] = w[j] * inv;
+        s_sel[warp][j] = (uint8_t)sel_e[j];
+      }
+    }
   }
-  if (lane == 0) {
-    const float vmax = sel_v[0];
-    float w[kMaxTopK];
-    float sum = 0.f;
+  __syncthreads();
+  if (warp == 0) {  // lane = token of the row
+    const bool has = blockIdx.x * kRouteRow + lane < T;
     for (int j = 0; j < k; ++j) {
-      w[j] = expf(sel_v[j] - vmax);
-      sum += w[j];
+      const int e = has ? (int)s_sel[lane][j] : -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, e);
+      if (has && lane == __ffs(peers) - 1) atomicAdd(&s_hist[e], __popc(peers));
     }
-    const float inv = 1.0f / sum;
-    for (int j = 0; j < k; ++j) {
-      topk_idx[(long)warp * k + j] = sel_e[j];
-      topk_w[(long)warp * k + j] = w[j] * inv;
-      atomicAdd(counts + sel_e[j], 1);  // a count: the order of the additions does not matter
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(long)blockIdx.x * E + e] = s_hist[e];
+}
+
+// Routing, second pass (one CTA of 256 threads): thread e turns column e of the histogram table into
+// its exclusive prefix over the rows (in place) and keeps the total; block scans over the experts
+// give counts, offsets (offsets[E] = T k) and mblk.
+__global__ void __launch_bounds__(kMaxExperts) moe_route_scan_kernel(int32_t* __restrict__ hist, int E, int nrow,
+                                                                     int32_t* __restrict__ counts,
+                                                                     int32_t* __restrict__ offsets,
+                                                                     int32_t* __restrict__ mblk) {
+  __shared__ int s_scan[kMaxExperts / 32 * 2];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int tot = 0;
+  if (tid < E)
+    for (int q0 = 0; q0 < nrow; q0 += 16) {  // 16 rows loaded together, then their prefixes stored
+      int c[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) c[i] = q0 + i < nrow ? hist[(long)(q0 + i) * E + tid] : 0;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        if (q0 + i < nrow) hist[(long)(q0 + i) * E + tid] = tot;
+        tot += c[i];
+      }
+    }
+  // exclusive scans over e of tot and of ceil(tot / 128): warp scans, then over the 8 warps
+  const int nb = (tot + 127) / 128;
+  int x = tot, y = nb;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int xo = __shfl_up_sync(0xffffffffu, x, o), yo = __shfl_up_sync(0xffffffffu, y, o);
+    if (lane >= o) { x += xo; y += yo; }
+  }
+  if (lane == 31) { s_scan[warp] = x; s_scan[kMaxExperts / 32 + warp] = y; }
+  __syncthreads();
+  int wx = 0, wy = 0;
+  for (int w = 0; w < warp; ++w) { wx += s_scan[w]; wy += s_scan[kMaxExperts / 32 + w]; }
+  if (tid < E) {
+    const int off_e = wx + x - tot, mb_e = wy + y - nb;
+    counts[tid] = tot;
+    offsets[tid] = off_e;
+    mblk[tid] = mb_e;
+    if (tid == E - 1) {
+      offsets[E] = off_e + tot;
+      mblk[E] = mb_e + nb;
     }
   }
 }
 
-// One CTA (1024 threads) per expert e: offsets[e] and mblk[e] from the counts of the experts before
-// it, then e's pairs in token order: perm[offsets[e] + rank] = t*k + j and its inverse, where rank
-// counts the earlier tokens that selected e (block-wide ballot prefix sums over 1024 tokens at a
-// time). CTA 0 also writes offsets[E] and mblk[E].
-__global__ void __launch_bounds__(1024) moe_place_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
-                                                         const int32_t* __restrict__ counts,
-                                                         int32_t* __restrict__ offsets, int32_t* __restrict__ mblk,
-                                                         int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm) {
-  __shared__ int s_base;
-  __shared__ int s_warp[32];
-  const int e = blockIdx.x;
-  if (threadIdx.x == 0) {
-    int o = 0, mb = 0;
-    for (int q = 0; q < e; ++q) {
-      const int c = counts[q];
-      o += c;
-      mb += (c + 127) / 128;
-    }
-    offsets[e] = o;
-    mblk[e] = mb;
-    if (e == 0) {
-      int ot = 0, mt = 0;
-      for (int q = 0; q < E; ++q) {
-        const int c = counts[q];
-        ot += c;
-        mt += (c + 127) / 128;
-      }
-      offsets[E] = ot;
-      mblk[E] = mt;
-    }
-    s_base = o;
+// Routing, third pass: 8 warps per CTA, warp = one row of 32 tokens (lane = token), placing the
+// row's pairs in (expert, token, slot) order. A token picks an expert at most once, so the rank of
+// pair (t, j) with expert e among e's pairs is the number of earlier tokens that picked e:
+// offsets[e], plus e's pairs in the earlier rows (the scanned table), plus the earlier lanes of this
+// row that picked e (the popcount of the row's lane mask of e, set by shared atomicOr).
+__global__ void __launch_bounds__(256) moe_route_place_kernel(
+    const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ hist, const int32_t* __restrict__ offsets,
+    int T, int E, int k, int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm) {
+  __shared__ uint32_t s_bits[8][kMaxExperts];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int row = blockIdx.x * 8 + warp;
+  const int t = row * kRouteRow + lane;
+  const bool has = t < T;
+  for (int i = lane; i < kMaxExperts; i += 32) s_bits[warp][i] = 0u;
+  __syncwarp();
+  int sel[kMaxTopK];
+  for (int j = 0; j < k; ++j) {
+    sel[j] = has ? __ldg(topk_idx + (long)t * k + j) : 0;
+    if (has) atomicOr(&s_bits[warp][sel[j]], 1u << lane);
   }
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int t0 = 0; t0 < T; t0 += 1024) {
-    const int t = t0 + threadIdx.x;
-    int slot = -1;
-    if (t < T)
-      for (int j = 0; j < k; ++j)
-        if (topk_idx[(long)t * k + j] == e) slot = j;
-    const uint32_t b = __ballot_sync(0xffffffffu, slot >= 0);
-    if (lane == 0) s_warp[warp] = __popc(b);
-    __syncthreads();
-    int before = 0, total = 0;
-    for (int w = 0; w < 32; ++w) {
-      const int c = s_warp[w];
-      if (w < warp) before += c;
-      total += c;
-    }
-    if (slot >= 0) {
-      const int pos = s_base + before + __popc(b & ((1u << lane) - 1u));
-      perm[pos] = t * k + slot;
-      inv_perm[t * k + slot] = pos;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) s_base += total;
-    __syncthreads();
+  __syncwarp();
+  if (!has) return;
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int j = 0; j < k; ++j) {
+    const int e = sel[j];
+    const int r = __ldg(offsets + e) + __ldg(hist + (long)row * E + e) + __popc(s_bits[warp][e] & lt);
+    perm[r] = t * k + j;
+    inv_perm[(long)t * k + j] = r;
   }
 }
 

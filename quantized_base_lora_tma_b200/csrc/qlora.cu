@@ -1141,19 +1141,33 @@ int qlora_linear_fwd(int qtype, const void* wq, int64_t N, int64_t K, const void
                                   st, 0);
 }
 
+static size_t moe_route_ws(int64_t T, int E) { return al256((size_t)((T + kRouteRow - 1) / kRouteRow) * E * 4); }
+
+size_t qlora_moe_route_workspace_bytes(int64_t T, int E, int k) {
+  if (T < 1 || E < 1 || E > kMaxExperts || k < 1 || k > kMaxTopK || k > E) return 0;
+  return moe_route_ws(T, E);
+}
+
 int qlora_moe_route(const void* logits, int64_t T, int E, int k, int32_t* topk_idx, float* topk_w, int32_t* counts,
-                    int32_t* offsets, int32_t* perm, int32_t* inv_perm, int32_t* mblk, void* stream) {
+                    int32_t* offsets, int32_t* perm, int32_t* inv_perm, int32_t* mblk, void* ws, size_t ws_bytes,
+                    void* stream) {
   if (!logits || !topk_idx || !topk_w || !counts || !offsets || !perm || !inv_perm || !mblk) return QL_ERR_INVALID_ARG;
   if (E < 1 || E > kMaxExperts || k < 1 || k > kMaxTopK || k > E) return QL_ERR_UNSUPPORTED;
   if (T < 1) return QL_ERR_INVALID_ARG;
   if (T > (1 << 24)) return QL_ERR_SHAPE;
+  if (!ws || ws_bytes < moe_route_ws(T, E)) return QL_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QL_ERR_ALIGNMENT;
   cudaStream_t st = (cudaStream_t)stream;
-  if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, st) != cudaSuccess) return QL_ERR_CUDA;
-  const int grid = (int)((T * 32 + 255) / 256);
-  moe_topk_kernel<<<grid, 256, 0, st>>>((const __nv_bfloat16*)logits, (int)T, E, k, topk_idx, topk_w, counts);
+  const int nrow = (int)((T + kRouteRow - 1) / kRouteRow);
+  int32_t* hist = (int32_t*)ws;
+  moe_route_select_kernel<<<nrow, 32 * kRouteRow, 0, st>>>((const __nv_bfloat16*)logits, (int)T, E, k, topk_idx,
+                                                           topk_w, hist);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (launch_status() != QL_OK) return QL_ERR_CUDA;
-  moe_place_kernel<<<E, 1024, 0, st>>>(topk_idx, (int)T, E, k, counts, offsets, mblk, perm, inv_perm);
+  moe_route_scan_kernel<<<1, kMaxExperts, 0, st>>>(hist, E, nrow, counts, offsets, mblk);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (launch_status() != QL_OK) return QL_ERR_CUDA;
+  moe_route_place_kernel<<<(nrow + 7) / 8, 256, 0, st>>>(topk_idx, hist, offsets, (int)T, E, k, perm, inv_perm);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return launch_status();
 }

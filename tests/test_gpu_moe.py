@@ -38,7 +38,8 @@ def _check_route(R, logits_bits, k):
     return idx, w, counts, offsets, perm, inv
 
 
-@pytest.mark.parametrize("T,E,k,zipf", [(2048, 128, 8, 0.0), (4096, 256, 8, 1.1), (37, 16, 3, 0.0), (5, 4, 4, 0.0)])
+@pytest.mark.parametrize("T,E,k,zipf", [(2048, 128, 8, 0.0), (4096, 256, 8, 1.1), (37, 16, 3, 0.0), (5, 4, 4, 0.0),
+                                        (1000, 256, 16, 1.1), (777, 33, 1, 0.0)])
 def test_route_exact(T, E, k, zipf):
     rng = np.random.default_rng(T + E)
     L = rng.standard_normal((T, E)).astype(np.float32)
