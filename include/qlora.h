@@ -17,7 +17,8 @@
  *     results are valid after the caller synchronises that stream.
  *   - bf16 tensors are IEEE bfloat16 (uint16 storage). Packed weights are GGUF blocks in file
  *     order: a weight [rows x cols] is `rows` packed rows of cols/QK blocks each (QK = 32 for
- *     Q4_0/Q8_0, 256 for Q4_K; 18, 34, 144 bytes per block). Expert stacks are [E][rows][...].
+ *     Q4_0/Q8_0, 256 for the K-quants; 18, 34 bytes per Q4_0 / Q8_0 block, 144, 176, 210 per
+ *     Q4_K / Q5_K / Q6_K superblock). Expert stacks are [E][rows][...].
  *   - Every pointer must be 16-byte aligned; the packed weight rows, X, dY, A and B rows must make
  *     every row start 16-byte aligned (guaranteed by the shape rules below).
  *   - Return value: a ql_status. Argument errors are detected on the host before anything is
@@ -41,8 +42,10 @@ extern "C" {
 #pragma GCC visibility push(default)
 #endif
 
-/* GGML type ids of the supported block formats. */
-typedef enum { QL_Q4_0 = 2, QL_Q8_0 = 8, QL_Q4_K = 12 } ql_qtype;
+/* GGML type ids of the supported block formats. Q6_K (210-byte superblocks, not a multiple of 16
+ * bytes, so not copied by TMA) is supported by gguf_dequant only; the layer entry points return
+ * QL_ERR_UNSUPPORTED for it. */
+typedef enum { QL_Q4_0 = 2, QL_Q8_0 = 8, QL_Q4_K = 12, QL_Q5_K = 13, QL_Q6_K = 14 } ql_qtype;
 
 /* Element type of an output tensor. */
 typedef enum { QL_F32 = 0, QL_BF16 = 1 } ql_dtype;
@@ -93,7 +96,7 @@ int qlora_selftest_wait_timeout(int64_t limit_us, void* stream);
  * gguf_dequant — expand packed GGUF rows to fp32 or bf16.
  * The pages' recipe runs a standalone GGUF dequant function (Show HN: LoRA over GGUF, "Other
  * notes"); the layer's own kernels never call this: they expand blocks in shared memory.
- *   qtype     QL_Q4_0 | QL_Q8_0 | QL_Q4_K
+ *   qtype     QL_Q4_0 | QL_Q8_0 | QL_Q4_K | QL_Q5_K | QL_Q6_K
  *   wq        [rows][cols/QK blocks] packed bytes
  *   rows      > 0
  *   cols      > 0, multiple of 256

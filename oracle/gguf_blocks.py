@@ -15,8 +15,17 @@ definitions:
         sc_j = S[j] & 63 and m_j = S[j+4] & 63; for j >= 4, sc_j = (S[j+4] & 15) | (S[j-4] >> 6) << 4
         and m_j = (S[j+4] >> 4) | (S[j] >> 6) << 4. Nibble group i (32 bytes) holds sub-block 2i
         in its low nibbles and sub-block 2i+1 in its high nibbles.
+  Q5_K  176-byte superblock of 256: fp16 d, fp16 dmin, the same 12 scale bytes as Q4_K, 32 bytes
+        qh, 128 bytes of nibbles laid out as in Q4_K. Weight l of sub-block j takes its fifth bit
+        from bit j of qh[l]: q = nibble + 16 * ((qh[l] >> j) & 1) in [0, 32); w = d*sc_j*q - dmin*m_j.
+  Q6_K  210-byte superblock of 256: 128 bytes ql, 64 bytes qh, 16 int8 scales, fp16 d (last).
+        Each half h of 128 weights uses ql[64h:64h+64], qh[32h:32h+32] and scales[8h:8h+8]; its
+        weight 32a + l (a in 0..3, l in 0..31) has low bits from ql[64h + 32(a & 1) + l] (low nibble
+        for a < 2, high nibble otherwise), high bits (qh[32h + l] >> 2a) & 3, and scale
+        scales[8h + 2a + l // 16]: q = low | high << 4 in [0, 64), w = d * scale * (q - 32).
 
-Every decoded value is exact in fp64. ``deq_f32`` rounds the exact value once to fp32 (round to
+Every decoded value is exact in fp64 (and, except the Q4_K / Q5_K difference, already in fp32:
+at most 24 significant bits). ``deq_f32`` rounds the exact value once to fp32 (round to
 nearest even); ``deq_bf16`` rounds that fp32 value to bf16 (round to nearest even). The layer
 multiplies bf16 weight tiles, so ``deq_bf16`` is what the matmul oracles use.
 """
@@ -24,9 +33,9 @@ from __future__ import annotations
 
 import numpy as np
 
-Q4_0, Q8_0, Q4_K = 2, 8, 12
-_QK = {Q4_0: 32, Q8_0: 32, Q4_K: 256}
-_BB = {Q4_0: 18, Q8_0: 34, Q4_K: 144}
+Q4_0, Q8_0, Q4_K, Q5_K, Q6_K = 2, 8, 12, 13, 14
+_QK = {Q4_0: 32, Q8_0: 32, Q4_K: 256, Q5_K: 256, Q6_K: 256}
+_BB = {Q4_0: 18, Q8_0: 34, Q4_K: 144, Q5_K: 176, Q6_K: 210}
 
 
 def _fp16_at(blocks: np.ndarray, off: int) -> np.ndarray:
@@ -87,7 +96,40 @@ def decode_q4_k(raw, rows, cols) -> np.ndarray:
     return w.reshape(rows, cols)
 
 
-_DECODERS = {Q4_0: decode_q4_0, Q8_0: decode_q8_0, Q4_K: decode_q4_k}
+def decode_q5_k(raw, rows, cols) -> np.ndarray:
+    b = _blocks(Q5_K, raw, rows, cols)
+    d = _fp16_at(b, 0)
+    dmin = _fp16_at(b, 2)
+    sc, m = q4_k_scales(b[:, 4:16])
+    qh = b[:, 16:48].astype(np.int64)                  # [nb, 32]: bit j of qh[l] -> sub-block j
+    qs = b[:, 48:176].reshape(-1, 4, 32).astype(np.int64)
+    q = np.empty((b.shape[0], 8, 32), np.float64)
+    for j in range(8):
+        nib = (qs[:, j // 2, :] >> (4 * (j % 2))) & 0x0F
+        q[:, j, :] = nib + 16 * ((qh >> j) & 1)
+    w = d[:, None, None] * sc[:, :, None] * q - dmin[:, None, None] * m[:, :, None]
+    return w.reshape(rows, cols)
+
+
+def decode_q6_k(raw, rows, cols) -> np.ndarray:
+    b = _blocks(Q6_K, raw, rows, cols)
+    ql = b[:, 0:128].astype(np.int64)
+    qh = b[:, 128:192].astype(np.int64)
+    scales = b[:, 192:208].copy().view(np.int8).astype(np.float64)
+    d = _fp16_at(b, 208)
+    w = np.empty((b.shape[0], 256), np.float64)
+    l = np.arange(32)
+    for h in range(2):
+        for a in range(4):
+            low = (ql[:, 64 * h + 32 * (a & 1) + l] >> (4 * (a >> 1))) & 0x0F
+            high = (qh[:, 32 * h + l] >> (2 * a)) & 3
+            q = (low | (high << 4)).astype(np.float64)
+            s = scales[:, 8 * h + 2 * a + l // 16]
+            w[:, 128 * h + 32 * a + l] = d[:, None] * s * (q - 32.0)
+    return w.reshape(rows, cols)
+
+
+_DECODERS = {Q4_0: decode_q4_0, Q8_0: decode_q8_0, Q4_K: decode_q4_k, Q5_K: decode_q5_k, Q6_K: decode_q6_k}
 
 
 def decode_exact(qtype, raw, rows, cols) -> np.ndarray:

@@ -1,12 +1,12 @@
 // GGUF block decode on the device: 8 consecutive weights of one 256-weight group of a packed row.
 //
 // A "group" is the packed bytes of 256 consecutive weights of one row: 8 Q8_0 blocks (272 B),
-// 8 Q4_0 blocks (144 B) or one Q4_K superblock (144 B). Groups are the unit every kernel here
-// moves: their byte size is a multiple of 16, so they can be copied by TMA and rows of K % 256 == 0
-// weights start 16-byte aligned.
+// 8 Q4_0 blocks (144 B), or one Q4_K (144 B), Q5_K (176 B) or Q6_K (210 B) superblock. Groups are the
+// unit every kernel here moves: except Q6_K's, their byte size is a multiple of 16, so they can be
+// copied by TMA and rows of K % 256 == 0 weights start 16-byte aligned.
 //
-// Values are the exact decode rounded once to fp32 (each product below is exact in fp32; the Q4_K
-// difference is formed by one fused multiply-add, i.e. one rounding), which a caller then rounds
+// Values are the exact decode rounded once to fp32 (each product below is exact in fp32; the Q4_K /
+// Q5_K difference is formed by one fused multiply-add, i.e. one rounding), which a caller then rounds
 // to bf16 (nearest even) for the tensor cores.
 #pragma once
 #include <cuda_bf16.h>
@@ -30,6 +30,16 @@ struct QTraits<QL_Q4_0> {
 template <>
 struct QTraits<QL_Q4_K> {
   static constexpr int kGroupBytes = 144;
+};
+template <>
+struct QTraits<QL_Q5_K> {
+  static constexpr int kGroupBytes = 176;
+};
+// 210 bytes is not a multiple of 16: Q6_K groups cannot be TMA-copied one by one, so only the
+// standalone dequant (byte and half-word loads) reads them.
+template <>
+struct QTraits<QL_Q6_K> {
+  static constexpr int kGroupBytes = 210;
 };
 
 __device__ __forceinline__ uint32_t pack2_same(__nv_bfloat16 h) {
@@ -110,9 +120,64 @@ __device__ __forceinline__ void decode8<QL_Q4_K>(const uint8_t* g, int c, float 
   }
 }
 
+// The 6-bit (sc, m) pair of sub-block j from the 12 scale bytes S shared by Q4_K and Q5_K.
+__device__ __forceinline__ void k_scale_min(const uint8_t* S, int j, int& sc, int& m) {
+  if (j < 4) {
+    sc = S[j] & 63;
+    m = S[j + 4] & 63;
+  } else {
+    sc = (S[j + 4] & 15) | ((S[j - 4] >> 6) << 4);
+    m = (S[j + 4] >> 4) | ((S[j] >> 6) << 4);
+  }
+}
+
+// Q5_K superblock (176 B): fp16 d, fp16 dmin, the 12 scale bytes, 32 bytes qh, 128 bytes of nibbles
+// (as Q4_K); weight l of sub-block j: q = nibble + 16 * bit j of qh[l]; w = d*sc*q - dmin*m.
+template <>
+__device__ __forceinline__ void decode8<QL_Q5_K>(const uint8_t* g, int c, float (&w)[8]) {
+  const float d = half_at(g);
+  const float dmin = half_at(g + 2);
+  const int j = c >> 2, l0 = 8 * (c & 3);
+  int sc, m;
+  k_scale_min(g + 4, j, sc, m);
+  const float ds = d * (float)sc;       // exact (11 + 6 bits)
+  const float dm = -(dmin * (float)m);  // exact
+  const uint2 q = *reinterpret_cast<const uint2*>(g + 48 + 32 * (j >> 1) + l0);
+  const uint2 h = *reinterpret_cast<const uint2*>(g + 16 + l0);
+  const int sh = (j & 1) * 4;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int q0 = (int)((q.x >> (8 * i + sh)) & 15u) | (int)(((h.x >> (8 * i + j)) & 1u) << 4);
+    const int q1 = (int)((q.y >> (8 * i + sh)) & 15u) | (int)(((h.y >> (8 * i + j)) & 1u) << 4);
+    w[i] = fmaf(ds, (float)q0, dm);
+    w[4 + i] = fmaf(ds, (float)q1, dm);
+  }
+}
+
+// Q6_K superblock (210 B): 128 bytes ql, 64 bytes qh, 16 int8 scales, fp16 d. Weight 32a + l of half
+// h: q = (nibble (a >> 1) of ql[64h + 32(a & 1) + l]) | ((qh[32h + l] >> 2a) & 3) << 4, scale
+// scales[8h + 2a + l / 16]; w = d * scale * (q - 32), exact in fp32 (at most 11 + 7 + 6 bits). The
+// superblocks are only 2-byte aligned.
+template <>
+__device__ __forceinline__ void decode8<QL_Q6_K>(const uint8_t* g, int c, float (&w)[8]) {
+  const int h = c >> 4, p0 = 8 * (c & 15);
+  const int a = p0 >> 5, l0 = p0 & 31;
+  const float ds = half_at(g + 208) * (float)(int8_t)g[192 + 8 * h + 2 * a + (l0 >> 4)];
+  const uint2 lo = load8_a2(g + 64 * h + 32 * (a & 1) + l0);
+  const uint2 hi = load8_a2(g + 128 + 32 * h + l0);
+  const int sl = 4 * (a >> 1), shh = 2 * a;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int q0 = (int)((lo.x >> (8 * i + sl)) & 15u) | (int)(((hi.x >> (8 * i + shh)) & 3u) << 4);
+    const int q1 = (int)((lo.y >> (8 * i + sl)) & 15u) | (int)(((hi.y >> (8 * i + shh)) & 3u) << 4);
+    w[i] = ds * (float)(q0 - 32);
+    w[4 + i] = ds * (float)(q1 - 32);
+  }
+}
+
 // ------------------------------------------------------------------------------------------------
 // Whole-unit decode to bf16 for the tensor-core producers: weights [32u, 32u + 32) of a group
-// (one Q8_0 / Q4_0 block, or one 32-weight sub-block of a Q4_K superblock) as four 16-byte chunks
+// (one Q8_0 / Q4_0 block, or 32 weights of a K-quant superblock) as four 16-byte chunks
 // of 8 bf16. Every result equals RNE_bf16 of the exact decoded value (which is exact in fp32).
 // Integer-to-float conversion uses the 2^23 magic: the float with bit pattern 0x4B000000 | b is
 // 2^23 + b for a byte b, so one byte permute plus one subtraction yields an exact small integer.
@@ -266,6 +331,66 @@ __device__ __forceinline__ void decode_unit_bf16<QL_Q4_K>(const uint8_t* g, int 
     const float2 c = __ffma2_rn(__fadd2_rn(make_float2(f[2], f[3]), bias), dsv, dmv);
     o[2 * i] = bf16x2_bits(a.x, a.y);
     o[2 * i + 1] = bf16x2_bits(c.x, c.y);
+  }
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) out[cc] = make_uint4(o[4 * cc], o[4 * cc + 1], o[4 * cc + 2], o[4 * cc + 3]);
+}
+
+// Q5_K sub-block u: as Q4_K with the fifth bit of each code from bit u of the 32 qh bytes; one fp32
+// FMA rounds d*sc*q - dmin*m once, then one bf16 rounding.
+template <>
+__device__ __forceinline__ void decode_unit_bf16<QL_Q5_K>(const uint8_t* g, int u, uint4 (&out)[4]) {
+  const float d = half_at(g);
+  const float dmin = half_at(g + 2);
+  int sc, m;
+  k_scale_min(g + 4, u, sc, m);
+  const float ds = d * (float)sc;
+  const float dm = -(dmin * (float)m);
+  const uint4* qp = reinterpret_cast<const uint4*>(g + 48 + 32 * (u >> 1));
+  const uint4* hp = reinterpret_cast<const uint4*>(g + 16);
+  const uint4 q0 = qp[0], q1 = qp[1], h0 = hp[0], h1 = hp[1];
+  const uint32_t xs[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+  const uint32_t hs[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+  const uint32_t sh = (uint32_t)(u & 1) * 4u;
+  const float2 dsv = make_float2(ds, ds), dmv = make_float2(dm, dm);
+  const float2 bias = make_float2(-8388608.0f, -8388608.0f);  // -2^23
+  uint32_t o[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float f[4];
+    magic4(((xs[i] >> sh) & 0x0F0F0F0Fu) | (((hs[i] >> u) & 0x01010101u) << 4), f);
+    const float2 a = __ffma2_rn(__fadd2_rn(make_float2(f[0], f[1]), bias), dsv, dmv);
+    const float2 c = __ffma2_rn(__fadd2_rn(make_float2(f[2], f[3]), bias), dsv, dmv);
+    o[2 * i] = bf16x2_bits(a.x, a.y);
+    o[2 * i + 1] = bf16x2_bits(c.x, c.y);
+  }
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) out[cc] = make_uint4(o[4 * cc], o[4 * cc + 1], o[4 * cc + 2], o[4 * cc + 3]);
+}
+
+// Q6_K unit u (32 weights 32a + l of half h = u / 4, a = u % 4): two scales (l < 16, l >= 16);
+// d * scale * (q - 32) is exact in fp32, then one bf16 rounding. 2-byte aligned loads.
+template <>
+__device__ __forceinline__ void decode_unit_bf16<QL_Q6_K>(const uint8_t* g, int u, uint4 (&out)[4]) {
+  const int h = u >> 2, a = u & 3;
+  const float d = half_at(g + 208);
+  const float ds0 = d * (float)(int8_t)g[192 + 8 * h + 2 * a];
+  const float ds1 = d * (float)(int8_t)g[192 + 8 * h + 2 * a + 1];
+  uint32_t lo[8], hi[8];
+  load32_a2(g + 64 * h + 32 * (a & 1), lo);
+  load32_a2(g + 128 + 32 * h, hi);
+  const uint32_t sl = 4u * (uint32_t)(a >> 1), shh = 2u * (uint32_t)a;
+  const float2 bias = make_float2(-8388640.0f, -8388640.0f);  // -(2^23 + 32)
+  uint32_t o[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float2 dsv = i < 4 ? make_float2(ds0, ds0) : make_float2(ds1, ds1);
+    float f[4];
+    magic4(((lo[i] >> sl) & 0x0F0F0F0Fu) | (((hi[i] >> shh) & 0x03030303u) << 4), f);
+    const float2 x = __fmul2_rn(__fadd2_rn(make_float2(f[0], f[1]), bias), dsv);
+    const float2 y = __fmul2_rn(__fadd2_rn(make_float2(f[2], f[3]), bias), dsv);
+    o[2 * i] = bf16x2_bits(x.x, x.y);
+    o[2 * i + 1] = bf16x2_bits(y.x, y.y);
   }
 #pragma unroll
   for (int cc = 0; cc < 4; ++cc) out[cc] = make_uint4(o[4 * cc], o[4 * cc + 1], o[4 * cc + 2], o[4 * cc + 3]);

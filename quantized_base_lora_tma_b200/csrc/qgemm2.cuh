@@ -52,7 +52,7 @@ struct Gemm2Cfg {
   static constexpr int B_BYTES = HN * kBK * 2;   // 16 KB
   static constexpr int RAW_ROWS = TRANS ? 64 : 128;
   static constexpr int RAW_BYTES = RAW_ROWS * GB;
-  static constexpr int STAGES = MS == 2 ? 3 : (GB > 200 ? 4 : 5);
+  static constexpr int STAGES = MS == 2 ? 3 : (GB > 150 ? 4 : 5);
   static constexpr int RAW_SLOTS = TRANS ? (GB > 200 ? (MS == 2 ? 4 : 5) : 6) : (GB > 200 ? 2 : 3);
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;

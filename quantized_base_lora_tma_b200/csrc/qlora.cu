@@ -144,11 +144,13 @@ static cudaError_t set_smem(Kernel k, int bytes) {
 
 static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Packed bytes of 256 weights of a row, for the types the layer's GEMMs take (0 otherwise).
 static int group_bytes(int qtype) {
   switch (qtype) {
     case QL_Q8_0: return 272;
     case QL_Q4_0: return 144;
     case QL_Q4_K: return 144;
+    case QL_Q5_K: return 176;
     default: return 0;
   }
 }
@@ -225,6 +227,7 @@ static int launch_qgemm_q(int qtype, const CUtensorMap& tA, const CUtensorMap& t
     case QL_Q4_K:
       return bn == 256 ? launch_qgemm<QL_Q4_K, TRANS, EPI, MS, 256>(tA, tW, tLA, tLB, p, grid, st, slot)
                        : launch_qgemm<QL_Q4_K, TRANS, EPI, MS>(tA, tW, tLA, tLB, p, grid, st, slot);
+    case QL_Q5_K: return launch_qgemm<QL_Q5_K, TRANS, EPI, MS>(tA, tW, tLA, tLB, p, grid, st, slot);
     default: return QL_ERR_UNSUPPORTED;
   }
 }
@@ -292,6 +295,7 @@ static int launch_qgemm2_q(int qtype, const CUtensorMap& tA, const CUtensorMap& 
     case QL_Q8_0: return launch_qgemm2<QL_Q8_0, TRANS, MS>(tA, tW, tLA, tLB, tRY, tZ, p, tiles, st, slot);
     case QL_Q4_0: return launch_qgemm2<QL_Q4_0, TRANS, MS>(tA, tW, tLA, tLB, tRY, tZ, p, tiles, st, slot);
     case QL_Q4_K: return launch_qgemm2<QL_Q4_K, TRANS, MS>(tA, tW, tLA, tLB, tRY, tZ, p, tiles, st, slot);
+    case QL_Q5_K: return launch_qgemm2<QL_Q5_K, TRANS, MS>(tA, tW, tLA, tLB, tRY, tZ, p, tiles, st, slot);
     default: return QL_ERR_UNSUPPORTED;
   }
 }
@@ -301,6 +305,7 @@ static int qgemm2_max_clusters_q(int qtype) {
     case QL_Q8_0: return qgemm2_max_clusters<QL_Q8_0, TRANS, MS>();
     case QL_Q4_0: return qgemm2_max_clusters<QL_Q4_0, TRANS, MS>();
     case QL_Q4_K: return qgemm2_max_clusters<QL_Q4_K, TRANS, MS>();
+    case QL_Q5_K: return qgemm2_max_clusters<QL_Q5_K, TRANS, MS>();
     default: return 0;
   }
 }
@@ -309,6 +314,7 @@ static int qgemm2_smem_q(int qtype) {
   switch (qtype) {
     case QL_Q8_0: return Gemm2Cfg<QL_Q8_0, TRANS, MS>::SMEM_BYTES;
     case QL_Q4_0: return Gemm2Cfg<QL_Q4_0, TRANS, MS>::SMEM_BYTES;
+    case QL_Q5_K: return Gemm2Cfg<QL_Q5_K, TRANS, MS>::SMEM_BYTES;
     default: return Gemm2Cfg<QL_Q4_K, TRANS, MS>::SMEM_BYTES;
   }
 }
@@ -1057,7 +1063,7 @@ int qlora_selftest_wait_timeout(int64_t limit_us, void* stream) {
 
 int gguf_dequant(int qtype, const void* wq, int64_t rows, int64_t cols, void* out, int out_dtype, void* stream) {
   if (!wq || !out) return QL_ERR_INVALID_ARG;
-  if (group_bytes(qtype) == 0) return QL_ERR_UNSUPPORTED;
+  if (group_bytes(qtype) == 0 && qtype != QL_Q6_K) return QL_ERR_UNSUPPORTED;
   if (out_dtype != QL_F32 && out_dtype != QL_BF16) return QL_ERR_INVALID_ARG;
   if (rows < 1 || cols < 1) return QL_ERR_INVALID_ARG;
   if (cols % 256 != 0) return QL_ERR_SHAPE;
@@ -1069,6 +1075,8 @@ int gguf_dequant(int qtype, const void* wq, int64_t rows, int64_t cols, void* ou
     case QL_Q8_0: gguf_dequant_kernel<QL_Q8_0><<<grid, 256, 0, st>>>((const uint8_t*)wq, rows, cols, out, out_dtype); break;
     case QL_Q4_0: gguf_dequant_kernel<QL_Q4_0><<<grid, 256, 0, st>>>((const uint8_t*)wq, rows, cols, out, out_dtype); break;
     case QL_Q4_K: gguf_dequant_kernel<QL_Q4_K><<<grid, 256, 0, st>>>((const uint8_t*)wq, rows, cols, out, out_dtype); break;
+    case QL_Q5_K: gguf_dequant_kernel<QL_Q5_K><<<grid, 256, 0, st>>>((const uint8_t*)wq, rows, cols, out, out_dtype); break;
+    case QL_Q6_K: gguf_dequant_kernel<QL_Q6_K><<<grid, 256, 0, st>>>((const uint8_t*)wq, rows, cols, out, out_dtype); break;
   }
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return launch_status();

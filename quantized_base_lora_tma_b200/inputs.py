@@ -26,10 +26,12 @@ import numpy as np
 Q4_0 = 2
 Q8_0 = 8
 Q4_K = 12
+Q5_K = 13
+Q6_K = 14
 
-QK = {Q4_0: 32, Q8_0: 32, Q4_K: 256}          # elements per block
-BLOCK_BYTES = {Q4_0: 18, Q8_0: 34, Q4_K: 144}  # bytes per block
-QTYPE_NAMES = {Q4_0: "q4_0", Q8_0: "q8_0", Q4_K: "q4_k"}
+QK = {Q4_0: 32, Q8_0: 32, Q4_K: 256, Q5_K: 256, Q6_K: 256}          # elements per block
+BLOCK_BYTES = {Q4_0: 18, Q8_0: 34, Q4_K: 144, Q5_K: 176, Q6_K: 210}  # bytes per block
+QTYPE_NAMES = {Q4_0: "q4_0", Q8_0: "q8_0", Q4_K: "q4_k", Q5_K: "q5_k", Q6_K: "q6_k"}
 QTYPE_BY_NAME = {v: k for k, v in QTYPE_NAMES.items()}
 
 
@@ -137,7 +139,92 @@ def pack_q4_k(w: np.ndarray) -> np.ndarray:
     return out.reshape(rows, -1)
 
 
-PACKERS = {Q4_0: pack_q4_0, Q8_0: pack_q8_0, Q4_K: pack_q4_k}
+def _k_scale_bytes(sc: np.ndarray, m: np.ndarray) -> np.ndarray:
+    """The 12 bytes of eight 6-bit (sc, m) pairs shared by Q4_K and Q5_K, [nb, 12]."""
+    S = np.zeros((sc.shape[0], 12), np.uint8)
+    for j in range(4):
+        S[:, j] = (sc[:, j] & 63) | ((sc[:, j + 4] >> 4) << 6)
+        S[:, j + 4] = (m[:, j] & 63) | ((m[:, j + 4] >> 4) << 6)
+        S[:, j + 8] = (sc[:, j + 4] & 15) | ((m[:, j + 4] & 15) << 4)
+    return S
+
+
+def pack_q5_k(w: np.ndarray) -> np.ndarray:
+    """Q5_K with a plain min/max encoder, as pack_q4_k but with 5-bit codes (31 steps).
+
+    Per 32-weight sub-block j: lo = min(0, min x), scale_j = (max x - lo)/31, min_j = -lo; d, dmin,
+    sc_j, m_j as in pack_q4_k; q = round((x + dmin*m_j)/(d*sc_j)) clamped to [0, 31]. Byte layout:
+    fp16 d, fp16 dmin, 12 scale bytes, 32 bytes qh (bit j of byte l = bit 4 of q of weight l of
+    sub-block j), 128 bytes of low nibbles (group i: sub-block 2i low, 2i+1 high).
+    """
+    rows, cols = w.shape
+    x = np.ascontiguousarray(w, dtype=np.float32).reshape(-1, 8, 32)
+    nb = x.shape[0]
+    lo = np.minimum(np.float32(0), x.min(axis=2))
+    scale = (x.max(axis=2) - lo) / np.float32(31)
+    mn = -lo
+    d16 = (scale.max(axis=1) / np.float32(63)).astype(np.float16)
+    dm16 = (mn.max(axis=1) / np.float32(63)).astype(np.float16)
+    d = d16.astype(np.float32)[:, None]
+    dm = dm16.astype(np.float32)[:, None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        sc = np.where(d > 0, _round_half_away(scale / d), 0)
+        m = np.where(dm > 0, _round_half_away(mn / dm), 0)
+    sc = np.clip(sc, 0, 63).astype(np.uint8)
+    m = np.clip(m, 0, 63).astype(np.uint8)
+    step = d * sc.astype(np.float32)
+    off = dm * m.astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = np.where(step[:, :, None] > 0, _round_half_away((x + off[:, :, None]) / step[:, :, None]), 0)
+    q = np.clip(q, 0, 31).astype(np.uint8)
+    out = np.zeros((nb, 176), np.uint8)
+    out[:, 0:2] = d16.view(np.uint8).reshape(-1, 2)
+    out[:, 2:4] = dm16.view(np.uint8).reshape(-1, 2)
+    out[:, 4:16] = _k_scale_bytes(sc, m)
+    qh = np.zeros((nb, 32), np.uint8)
+    for j in range(8):
+        qh |= ((q[:, j, :] >> 4) & 1) << j
+    out[:, 16:48] = qh
+    for i in range(4):
+        out[:, 48 + 32 * i:80 + 32 * i] = (q[:, 2 * i, :] & 15) | ((q[:, 2 * i + 1, :] & 15) << 4)
+    return out.reshape(rows, -1)
+
+
+def pack_q6_k(w: np.ndarray) -> np.ndarray:
+    """Q6_K with a plain absmax encoder.
+
+    Per 16-weight group g: scale_g = max|x| / 32; d = max scale_g / 127 (fp16); sc_g =
+    round(scale_g / d) clamped to [-128, 127] (int8); q = round(x / (d*sc_g)) + 32 clamped to
+    [0, 63] (32 where d*sc_g = 0). Byte layout: 128 bytes ql, 64 bytes qh, 16 int8 scales, fp16 d;
+    weight 32a + l of half h (a in 0..3): low 4 bits in ql[64h + 32(a & 1) + l] (low nibble for
+    a < 2), high 2 bits at bit 2a of qh[32h + l].
+    """
+    rows, cols = w.shape
+    x = np.ascontiguousarray(w, dtype=np.float32).reshape(-1, 16, 16)
+    nb = x.shape[0]
+    scale = np.abs(x).max(axis=2) / np.float32(32)
+    d16 = (scale.max(axis=1) / np.float32(127)).astype(np.float16)
+    d = d16.astype(np.float32)[:, None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        sc = np.where(d > 0, _round_half_away(scale / d), 0)
+    sc = np.clip(sc, -128, 127).astype(np.int8)
+    step = d * sc.astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = np.where(step[:, :, None] != 0, _round_half_away(x / step[:, :, None]), 0) + 32
+    q = np.clip(q, 0, 63).astype(np.uint8).reshape(nb, 256)
+    out = np.zeros((nb, 210), np.uint8)
+    l = np.arange(32)
+    for h in range(2):
+        for a in range(4):
+            qa = q[:, 128 * h + 32 * a + l]
+            out[:, 64 * h + 32 * (a & 1) + l] |= (qa & 15) << (4 * (a >> 1))
+            out[:, 128 + 32 * h + l] |= (qa >> 4) << (2 * a)
+    out[:, 192:208] = sc.view(np.uint8)
+    out[:, 208:210] = d16.view(np.uint8).reshape(-1, 2)
+    return out.reshape(rows, -1)
+
+
+PACKERS = {Q4_0: pack_q4_0, Q8_0: pack_q8_0, Q4_K: pack_q4_k, Q5_K: pack_q5_k, Q6_K: pack_q6_k}
 
 
 def pack(qtype: int, w: np.ndarray) -> np.ndarray:

@@ -26,15 +26,17 @@ def _reset_status():
 def _random_packed(qtype, rows, cols, rng):
     w = (rng.standard_normal((rows, cols)) * 0.02).astype(np.float32)
     raw = inp.pack(qtype, w)
-    if qtype != inp.Q4_K:  # sprinkle subnormal and zero scales
+    # sprinkle subnormal and zero scales (d of Q4_0 / Q8_0 blocks, d of Q6_K superblocks)
+    off = {inp.Q4_0: 0, inp.Q8_0: 0, inp.Q6_K: 208}.get(qtype)
+    if off is not None:
         bb = inp.BLOCK_BYTES[qtype]
         v = raw.reshape(-1, bb)
-        v[::5, 0:2] = np.frombuffer(np.float16(3.0e-6).tobytes(), np.uint8)
-        v[::13, 0:2] = 0
+        v[::5, off:off + 2] = np.frombuffer(np.float16(3.0e-6).tobytes(), np.uint8)
+        v[::13, off:off + 2] = 0
     return raw
 
 
-@pytest.mark.parametrize("qtype", [inp.Q4_0, inp.Q8_0, inp.Q4_K])
+@pytest.mark.parametrize("qtype", [inp.Q4_0, inp.Q8_0, inp.Q4_K, inp.Q5_K, inp.Q6_K])
 def test_dequant_bit_exact(qtype):
     rng = np.random.default_rng(qtype)
     rows, cols = 37, 768
@@ -102,7 +104,7 @@ SMALL = [
 ]
 
 
-@pytest.mark.parametrize("qtype", [inp.Q4_0, inp.Q8_0, inp.Q4_K])
+@pytest.mark.parametrize("qtype", [inp.Q4_0, inp.Q8_0, inp.Q4_K, inp.Q5_K])
 @pytest.mark.parametrize("shape", SMALL)
 def test_linear_parity_small(qtype, shape):
     M, K, N, r = shape

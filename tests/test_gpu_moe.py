@@ -118,6 +118,7 @@ SMALL = [
     (600, 256, 512, 4, 2, inp.Q8_0, 16, 0.0),     # segments spanning several 128-row blocks
     (33, 256, 256, 1, 1, inp.Q4_0, 4, 0.0),       # one expert, k = 1: a dense SwiGLU layer
     (64, 256, 256, 8, 8, inp.Q4_K, 40, 0.0),      # k = E (every expert every token), r > 32
+    (300, 512, 256, 8, 4, inp.Q5_K, 8, 1.0),      # Q5_K experts, skewed
 ]
 
 

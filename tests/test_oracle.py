@@ -65,27 +65,74 @@ def test_hand_packed_q4_k_high_bit_split():
     assert np.array_equal(got, want)
 
 
+def test_hand_packed_q5_k():
+    """A Q5_K superblock written byte by byte from chosen (sc, m, q): the scales in the Q4_K packing,
+    the fifth bit of weight l of sub-block j at bit j of qh[l], the low nibbles as in Q4_K."""
+    sc = [1, 5, 9, 13, 17, 40, 51, 63]
+    m = [2, 0, 7, 30, 33, 16, 48, 62]
+    q = [[(3 * l + 5 * j) % 32 for l in range(32)] for j in range(8)]
+    S = [0] * 12
+    for j in range(4):
+        S[j] = (sc[j] & 63) | ((sc[j + 4] >> 4) << 6)
+        S[j + 4] = (m[j] & 63) | ((m[j + 4] >> 4) << 6)
+        S[j + 8] = (sc[j + 4] & 15) | ((m[j + 4] & 15) << 4)
+    qh = [sum(((q[j][l] >> 4) & 1) << j for j in range(8)) for l in range(32)]
+    qs = []
+    for i in range(4):
+        qs += [(q[2 * i][l] & 15) | ((q[2 * i + 1][l] & 15) << 4) for l in range(32)]
+    raw = np.frombuffer(bytes([0x00, 0x3C, 0x00, 0x38] + S + qh + qs), np.uint8)   # d = 1.0, dmin = 0.5
+    assert raw.size == 176
+    got = gb.decode_exact(gb.Q5_K, raw, 1, 256)[0].reshape(8, 32)
+    want = np.array([[1.0 * sc[j] * q[j][l] - 0.5 * m[j] for l in range(32)] for j in range(8)])
+    assert np.array_equal(got, want)
+
+
+def test_hand_packed_q6_k():
+    """A Q6_K superblock written byte by byte from chosen int8 scales and 6-bit codes: weight
+    32a + l of half h has its low nibble in ql[64h + 32(a & 1) + l] (high nibble for a >= 2), its two
+    high bits at bit 2a of qh[32h + l], and the scale scales[8h + 2a + l // 16]; d is the last fp16."""
+    scales = [-128, -3, 0, 1, 7, 64, 127, -77, 5, -5, 33, -33, 100, 2, -1, 9]
+    q = [(7 * i + 3) % 64 for i in range(256)]
+    ql = [0] * 128
+    qh = [0] * 64
+    for h in range(2):
+        for a in range(4):
+            for l in range(32):
+                v = q[128 * h + 32 * a + l]
+                ql[64 * h + 32 * (a & 1) + l] |= (v & 15) << (4 * (a >> 1))
+                qh[32 * h + l] |= (v >> 4) << (2 * a)
+    sc_bytes = [x & 255 for x in scales]
+    raw = np.frombuffer(bytes(ql + qh + sc_bytes + [0x00, 0x34]), np.uint8)          # d = 0.25
+    assert raw.size == 210
+    got = gb.decode_exact(gb.Q6_K, raw, 1, 256)[0]
+    want = np.array([0.25 * scales[8 * (i // 128) + 2 * ((i % 128) // 32) + (i % 32) // 16] * (q[i] - 32)
+                     for i in range(256)])
+    assert np.array_equal(got, want)
+
+
 def _random_blocks(qtype, nblocks, rng):
-    bb = {gb.Q4_0: 18, gb.Q8_0: 34, gb.Q4_K: 144}[qtype]
+    bb = {gb.Q4_0: 18, gb.Q8_0: 34, gb.Q4_K: 144, gb.Q5_K: 176, gb.Q6_K: 210}[qtype]
     raw = rng.integers(0, 256, size=(nblocks, bb), dtype=np.uint8)
-    # finite fp16 scales only (random bytes could spell Inf/NaN)
-    n_h = 2 if qtype == gb.Q4_K else 1
-    for h in range(n_h):
+    # finite fp16 scales only (random bytes could spell Inf/NaN): bytes 0-1 (and 2-3 for the
+    # superblocks with a dmin), or the last two bytes of a Q6_K superblock
+    offs = {gb.Q4_K: [0, 2], gb.Q5_K: [0, 2], gb.Q6_K: [208]}.get(qtype, [0])
+    for o in offs:
         d = (rng.standard_normal(nblocks) * 0.01).astype(np.float16)
         d[::7] = np.float16(6.0e-8)                    # include subnormal scales
-        raw[:, 2 * h:2 * h + 2] = d.view(np.uint8).reshape(-1, 2)
+        raw[:, o:o + 2] = d.view(np.uint8).reshape(-1, 2)
     return raw
 
 
-@pytest.mark.parametrize("qtype,gtype", [(gb.Q4_0, "Q4_0"), (gb.Q8_0, "Q8_0"), (gb.Q4_K, "Q4_K")])
+@pytest.mark.parametrize("qtype,gtype", [(gb.Q4_0, "Q4_0"), (gb.Q8_0, "Q8_0"), (gb.Q4_K, "Q4_K"),
+                                         (gb.Q5_K, "Q5_K"), (gb.Q6_K, "Q6_K")])
 def test_decode_matches_gguf_py(qtype, gtype):
     """Independent codebase: gguf-py's dequantize (fp32) must equal the fp32 rounding of the exact
     decode, element by element."""
     gguf = pytest.importorskip("gguf")
     from gguf import quants
     rng = np.random.default_rng(7)
-    qk = {gb.Q4_0: 32, gb.Q8_0: 32, gb.Q4_K: 256}[qtype]
-    rows, cols = 16, 4 * qk if qtype == gb.Q4_K else 16 * qk
+    qk = {gb.Q4_0: 32, gb.Q8_0: 32}.get(qtype, 256)
+    rows, cols = 16, 4 * qk if qk == 256 else 16 * qk
     raw = _random_blocks(qtype, rows * cols // qk, rng).reshape(rows, -1)
     want = quants.dequantize(raw, getattr(gguf.GGMLQuantizationType, gtype)).astype(np.float32)
     got = gb.deq_f32(qtype, raw, rows, cols).astype(np.float32)
@@ -115,7 +162,7 @@ def test_packers_match_gguf_py_bytes(gtype):
     assert np.array_equal(inp.pack(qt, x), quants.quantize(x, getattr(gguf.GGMLQuantizationType, gtype)))
 
 
-@pytest.mark.parametrize("qtype", [inp.Q4_0, inp.Q8_0, inp.Q4_K])
+@pytest.mark.parametrize("qtype", [inp.Q4_0, inp.Q8_0, inp.Q4_K, inp.Q5_K, inp.Q6_K])
 def test_pack_roundtrip_error_bound(qtype):
     rng = np.random.default_rng(5)
     x = (rng.standard_normal((8, 512)) * 0.02).astype(np.float32)
@@ -123,6 +170,23 @@ def test_pack_roundtrip_error_bound(qtype):
     err = np.abs(w - x)
     if qtype == inp.Q4_K:
         assert err.max() < 0.2 * (x.max() - x.min()) / 15 * 8
+    elif qtype == inp.Q5_K:
+        # per 32-weight sub-block: half a step of (max - min(0, min)) / 31, widened for the 6-bit
+        # scale and min and their fp16 super-scales
+        xs = x.reshape(-1, 32)
+        step = (xs.max(axis=1) - np.minimum(0, xs.min(axis=1))) / 31
+        assert np.all(err.reshape(-1, 32) <= step[:, None] * 1.5 + 1e-7)
+    elif qtype == inp.Q6_K:
+        # per 16-weight group with step = d * scale read from the packed bytes: half a step where
+        # the code is not clipped, and the clipped excess |x| - 31 step (codes - 32 end at +31) or
+        # |x| - 32 step (at -32) where it is
+        b = inp.pack(qtype, x).reshape(-1, 210)
+        d = b[:, 208:210].copy().view(np.float16).astype(np.float64).ravel()
+        step = np.abs(d[:, None] * b[:, 192:208].copy().view(np.int8).astype(np.float64)).ravel()
+        xs = x.reshape(-1, 16).astype(np.float64)
+        clip = np.maximum(xs.max(axis=1) - 31 * step, -xs.min(axis=1) - 32 * step)
+        bound = np.maximum(0.5 * step, clip)
+        assert np.all(err.reshape(-1, 16) <= bound[:, None] * (1 + 1e-9) + 1e-9)
     else:
         qk = 32
         d = np.abs(inp.pack(qtype, x).reshape(-1, 18 if qtype == inp.Q4_0 else 34)[:, :2].copy()
