@@ -547,14 +547,20 @@ static DensePlan plan_dense(int64_t M, int64_t Nd, int64_t Kd, bool trans, bool 
   d.kbs = kb_main;
   const int tiles = d.mblocks * d.ntiles;
   const int slots = num_sms();
+  int ks = 1;
   if (allow_split && d.ms == 0 && tiles < slots) {
-    int ks = std::min((4 * slots + tiles - 1) / tiles, std::min(kb_main / unit, 32));
-    if (ks > 1) {
-      int kbs = (kb_main + ks - 1) / ks;
-      kbs = (kbs + unit - 1) / unit * unit;
-      d.kbs = kbs;
-      d.ksplit = (kb_main + kbs - 1) / kbs;
-    }
+    ks = std::min((4 * slots + tiles - 1) / tiles, std::min(kb_main / unit, 32));
+  } else if (allow_split && d.ms > 0 && 2 * tiles <= slots / 2) {
+    // pair tiles filling at most half of the SM pairs (e.g. a 2048 x 2048 input gradient over a
+    // long reduction: 32 tiles on 74 pairs): split K so that one wave fills most pairs; the fp32
+    // parts are summed in part order afterwards
+    ks = std::min((slots / 2) / tiles, std::min(kb_main / unit / 8, 4));
+  }
+  if (ks > 1) {
+    int kbs = (kb_main + ks - 1) / ks;
+    kbs = (kbs + unit - 1) / unit * unit;
+    d.kbs = kbs;
+    d.ksplit = (kb_main + kbs - 1) / kbs;
   }
   return d;
 }
@@ -635,7 +641,7 @@ static int launch_dense_gemm(int qtype, const void* A, int64_t M, int64_t Kd, co
                              int64_t w_cols, const __nv_bfloat16* LA, const __nv_bfloat16* LB, int KL, int64_t Nd,
                              void* out, int out_dtype, float* split_buf, bool allow_split, cudaStream_t st, int slot,
                              int rx = 0, const RowsFuse* rf = nullptr, const CUtensorMap* tRY = nullptr,
-                             const CUtensorMap* tZ = nullptr) {
+                             const CUtensorMap* tZ = nullptr, bool* sum_pending = nullptr) {
   const DensePlan d = plan_dense(M, Nd, Kd, TRANS, allow_split && split_buf != nullptr);
   const uint32_t box = 128u;
   CUtensorMap tA, tW, tLA, tLB;
@@ -676,6 +682,10 @@ static int launch_dense_gemm(int qtype, const void* A, int64_t M, int64_t Kd, co
   else if (d.ms == 1) rc = launch_qgemm2_q<TRANS, 1>(qtype, tA, tW, tLA, tLB, tRYr, tZr, p, tiles, st, slot);
   else rc = launch_qgemm_q<TRANS, EPI_STORE, 1>(qtype, tA, tW, tLA, tLB, p, std::min(tiles, num_sms()), st, slot);
   if (rc || d.ksplit == 1) return rc;
+  if (sum_pending != nullptr) {  // the caller launches the part sum (launch_split_reduce) itself
+    *sum_pending = true;
+    return QL_OK;
+  }
   return launch_split_reduce(split_buf, d.ksplit, (long)M * Nd, (long)M * Nd, out, out_dtype, st);
 }
 
@@ -1480,15 +1490,22 @@ int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void
     // weight streaming: W read once, G A added in the finish launch
     rc = launch_gemv_dx(wq, N, K, dY, M, LA, lora_rp(r), A, r, dX, dx_dtype, (float*)(wsb + w.dxp), st, 1);
     if (rc) return rc;
-  } else if (dX) {
+  }
+  bool sum_pending = false;
+  if (dX && !gemv_dx_applies(qtype, M)) {
     rc = launch_dense_gemm<true>(qtype, dY, M, N, wq, N, K, LA, LB, KL, K, dX, dx_dtype,
-                                 (float*)(wsb + w.split), true, st, 1);
+                                 (float*)(wsb + w.split), true, st, 1, 0, nullptr, nullptr, nullptr, &sum_pending);
     if (rc) return rc;
   }
   // dB = dY^T split(s H) and dA = split(G)^T X in one launch; after the dX GEMM (which waited for
   // the row kernel) it runs beside the GEMM on the SMs the GEMM leaves idle
-  return launch_colred_dense((const __nv_bfloat16*)dY, (int)N, HS, ob, (const __nv_bfloat16*)X, (int)K, LA, oa, (int)M,
-                             r, crws, dX ? 1 : 0, st);
+  rc = launch_colred_dense((const __nv_bfloat16*)dY, (int)N, HS, ob, (const __nv_bfloat16*)X, (int)K, LA, oa, (int)M,
+                           r, crws, dX ? 1 : 0, st);
+  if (rc || !sum_pending) return rc;
+  // the dX GEMM split K: its fp32 parts are summed after the column reductions (two launches after
+  // the GEMM, which has completed by then), so those still run beside the GEMM
+  const DensePlan d = plan_dense(M, K, N, true, true);
+  return launch_split_reduce((float*)(wsb + w.split), d.ksplit, (long)M * K, (long)M * K, dX, dx_dtype, st);
 }
 
 }  // extern "C"
