@@ -306,6 +306,7 @@ def device_status_ok(where):
 
 def also_measurements(flush, steps, pk):
     """Single-GPU measurements of the other shapes of the benchmark set (not the headline)."""
+    import quantized_base_lora_tma_b200 as ql
     out = {}
     # routed MoE layer, fwd + bwd incl. routing
     c = inp.moe_q4_0_2048tok_128x768()
@@ -319,8 +320,23 @@ def also_measurements(flush, steps, pk):
     device_status_ok("moe")
     del m
     torch.cuda.empty_cache()
+    # 8-bit AdamW on the headline layer's adapters (A [16 x 4096] and B [4096 x 16])
+    n = 2 * 16 * 4096
+    st = ql.Adamw8State(n)
+    pp = torch.zeros(n, dtype=torch.float32, device="cuda")
+    gg = torch.randn(n, dtype=torch.float32, device="cuda") * 0.01
+    pb = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+    t_ = [0]
+
+    def adam_step():
+        t_[0] += 1
+        ql.qlora_adamw8_step(pp, gg, st, t_[0], 1e-4, 0.9, 0.999, 1e-8, 0.01, p_bf16=pb)
+    ms_a, _ = time_steps(adam_step, steps, 3, flush)
+    abytes = n * (4 + 4 + 4 + 1 + 1 + 1 + 1 + 2) + 4 * 4 * ((n + 255) // 256)  # p r/w, g, codes r/w, bf16 copy
+    out["adamw8_adapters_r16_4096x4096"] = {"params": n, "ms": ms_a, "gbs": abytes / (ms_a / 1e3) / 1e9}
+    device_status_ok("adamw8")
+    del st, pp, gg, pb
     # routing alone at 4096 tokens, 256 experts, top-8 (the skewed workload's logits)
-    import quantized_base_lora_tma_b200 as ql
     c = inp.moe_q4_k_256x4096x1536(4096)
     lg = bf16_dev(c.logits)
     R = ql.MoeRoute(c.T, c.E, c.k)

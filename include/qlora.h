@@ -196,6 +196,28 @@ int qlora_moe_bwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
                   float* dA_d, float* dB_d, float* d_logits, void* ws, size_t ws_bytes,
                   void* stream);
 
+/* ---------------------------------------------------------------------------------------------
+ * 8-bit AdamW step on the adapter parameters (the recipe's bitsandbytes 8-bit AdamW optimizer,
+ * Show HN: LoRA over GGUF, "Things involved in the training"): AdamW with decoupled weight decay
+ * whose moments are kept in 8 bits, block-wise.
+ *   p        [n] fp32 master parameters, updated in place
+ *   grad     [n] fp32 gradient (e.g. dA or dB of this layer)
+ *   m_q, v_q [n] uint8 codes of the first and second moment; m_absmax, v_absmax [ceil(n / 256)] fp32
+ *            scales, one per block of 256 values; all four updated in place. Zeros everywhere is the
+ *            state before the first step.
+ *   step     t >= 1 (the bias corrections use 1 - beta^t)
+ *   p_bf16   [n] bf16 (nullable): receives the updated parameters rounded to bf16 (the layer's A, B)
+ * Update, in fp32: m = b1 m + (1 - b1) g; v = b2 v + (1 - b2) g^2;
+ *   p = p - lr (m / c1 / (sqrt(v / c2) + eps) + weight_decay p), c1 = 1 - b1^t, c2 = 1 - b2^t.
+ * A code q of a block with scale a stands for a * T[q]. T is the dynamic tree table: after the sign
+ * bit (m only), E zero bits give the decade 10^-E, then an indicator bit, then B bits F of linear
+ * fraction: |T| = (0.1 + 0.9 (F + 1/2) / 2^B) / 10^E; no indicator codes 0. After the update each
+ * block's scale is max |value| over the block and each value takes the code of the nearest entry to
+ * value / scale (equal distances: the smaller entry). No workspace; one launch. */
+int qlora_adamw8_step(float* p, const float* grad, uint8_t* m_q, float* m_absmax, uint8_t* v_q, float* v_absmax,
+                      int64_t n, float lr, float beta1, float beta2, float eps, float weight_decay, int64_t step,
+                      void* p_bf16, void* stream);
+
 /* Forward without allocation (no counterpart in the method's sources; a convenience of this
  * library). Same arguments, results and rules as qlora_linear_fwd, minus (ws, ws_bytes).
  *

@@ -14,7 +14,7 @@ import torch
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libqlora.so")
 
-Q4_0, Q8_0, Q4_K = 2, 8, 12
+Q4_0, Q8_0, Q4_K, Q5_K, Q6_K = 2, 8, 12, 13, 14
 QL_F32, QL_BF16 = 0, 1
 QL_OK = 0
 STATUS = {0: "QL_OK", 1: "QL_ERR_INVALID_ARG", 2: "QL_ERR_UNSUPPORTED", 3: "QL_ERR_SHAPE",
@@ -49,6 +49,8 @@ SIGNATURES = {
     "qlora_moe_bwd": (_c_int, [_c_int, _c_vp, _c_vp, _c_int, _c_i64, _c_i64, _c_vp, _c_vp, _c_i64, _c_int, _c_vp,
                                _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_f, _c_vp,
                                _c_sz, _c_vp, _c_int, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_sz, _c_vp]),
+    "qlora_adamw8_step": (_c_int, [_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_f, _c_f, _c_f, _c_f, _c_f,
+                                   _c_i64, _c_vp, _c_vp]),
     "qlora_linear_fwd_noalloc": (_c_int, [_c_int, _c_vp, _c_i64, _c_i64, _c_vp, _c_i64, _c_vp, _c_vp, _c_int,
                                           _c_f, _c_vp, _c_int, _c_vp, _c_vp]),
     "qlora_linear_bwd": (_c_int, [_c_int, _c_vp, _c_i64, _c_i64, _c_vp, _c_vp, _c_i64, _c_vp, _c_vp, _c_int,
@@ -236,3 +238,23 @@ def qlora_moe_bwd(qtype, w_gu, w_d, E, H, I, X, dY, route, A_gu, B_gu, A_d, B_d,
                                _p(A_d), _p(B_d), r, scale, _p(saved), _nb(saved), _p(dX), _dt(dX), _p(dA_gu),
                                _p(dB_gu), _p(dA_d), _p(dB_d), _p(d_logits), _p(ws), _nb(ws), _s(stream)),
            "qlora_moe_bwd")
+
+
+class Adamw8State:
+    """Device buffers of the 8-bit AdamW moments for n parameters (zeros: before the first step)."""
+
+    def __init__(self, n, device="cuda"):
+        nb = (n + 255) // 256
+        self.n = n
+        self.m_q = torch.zeros(n, dtype=torch.uint8, device=device)
+        self.v_q = torch.zeros(n, dtype=torch.uint8, device=device)
+        self.m_absmax = torch.zeros(nb, dtype=torch.float32, device=device)
+        self.v_absmax = torch.zeros(nb, dtype=torch.float32, device=device)
+
+
+def qlora_adamw8_step(p, grad, state, step, lr=1e-4, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0,
+                      p_bf16=None, stream=None):
+    _check(lib().qlora_adamw8_step(_p(p), _p(grad), _p(state.m_q), _p(state.m_absmax), _p(state.v_q),
+                                   _p(state.v_absmax), p.numel(), lr, beta1, beta2, eps, weight_decay, step,
+                                   _p(p_bf16) if p_bf16 is not None else None, _s(stream)),
+           "qlora_adamw8_step")

@@ -3,7 +3,9 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <array>
+#include <cmath>
 #include <atomic>
 #include <chrono>
 #include <cstdint>
@@ -18,6 +20,7 @@
 #include "qgemm2.cuh"
 #include "gemv.cuh"
 #include "moe.cuh"
+#include "adamw8.cuh"
 
 namespace qlora {
 
@@ -1565,6 +1568,83 @@ static int static_scratch_address(void** out) {
 }
 
 }  // namespace qlora
+
+// ------------------------------------------------------------------------------------------------
+// 8-bit AdamW on the adapters
+// ------------------------------------------------------------------------------------------------
+namespace qlora {
+
+// The dynamic tree code tables: after the optional sign bit, E zero bits (the decade 10^-E), an
+// indicator bit and B fraction bits F; |entry| = (0.1 + 0.9 (F + 1/2) / 2^B) / 10^E; no indicator
+// codes 0. Entries are formed in fp64 and rounded once to fp32.
+static void build_adamw8_tables(Adamw8Tables& T) {
+  static const double p10[9] = {1.0, 10.0, 100.0, 1000.0, 1e4, 1e5, 1e6, 1e7, 1e8};
+  for (int sg = 0; sg < 2; ++sg) {
+    const bool is_signed = sg == 0;
+    const int nbits = is_signed ? 7 : 8;
+    float* dec = is_signed ? T.dec_s : T.dec_u;
+    for (int q = 0; q < 256; ++q) {
+      const int bits = q & ((1 << nbits) - 1);
+      const bool neg = is_signed && ((q >> 7) & 1);
+      double v = 0.0;
+      if (bits != 0) {
+        int top = 0;
+        while ((bits >> (top + 1)) != 0) ++top;          // index of the highest set bit
+        const int E = nbits - 1 - top;
+        const int B = nbits - E - 1;
+        const int F = bits & ((1 << B) - 1);
+        v = (0.1 + 0.9 * (F + 0.5) / std::ldexp(1.0, B)) / p10[E];
+      }
+      dec[q] = (float)(neg ? -v : v);
+    }
+    // distinct entries ascending (the signed -0 code 0x80 never produced), with their codes
+    std::vector<std::pair<float, int>> e;
+    for (int q = 0; q < 256; ++q)
+      if (!(is_signed && q == 0x80)) e.push_back({dec[q], q});
+    std::stable_sort(e.begin(), e.end(), [](const std::pair<float, int>& x, const std::pair<float, int>& y) {
+      return x.first < y.first;
+    });
+    float* srt = is_signed ? T.srt_s : T.srt_u;
+    uint8_t* cod = is_signed ? T.cod_s : T.cod_u;
+    for (int k = 0; k < 256; ++k) {
+      srt[k] = k < (int)e.size() ? e[k].first : 2.0f;
+      cod[k] = k < (int)e.size() ? (uint8_t)e[k].second : 0;
+    }
+    (is_signed ? T.ns : T.nu) = (int)e.size();
+  }
+}
+
+static const Adamw8Tables& adamw8_tables() {
+  static Adamw8Tables T;
+  static std::once_flag once;
+  std::call_once(once, [] { build_adamw8_tables(T); });
+  return T;
+}
+
+}  // namespace qlora
+
+extern "C" int qlora_adamw8_step(float* p, const float* grad, uint8_t* m_q, float* m_absmax, uint8_t* v_q,
+                                 float* v_absmax, int64_t n, float lr, float beta1, float beta2, float eps,
+                                 float weight_decay, int64_t step, void* p_bf16, void* stream) {
+  if (!p || !grad || !m_q || !m_absmax || !v_q || !v_absmax) return QL_ERR_INVALID_ARG;
+  if (n < 1 || step < 1) return QL_ERR_INVALID_ARG;
+  if (!(beta1 >= 0.f && beta1 < 1.f) || !(beta2 >= 0.f && beta2 < 1.f) || !(eps > 0.f)) return QL_ERR_INVALID_ARG;
+  if (n > ((int64_t)1 << 40)) return QL_ERR_SHAPE;
+  Adamw8Args a;
+  a.lr = lr;
+  a.b1 = beta1;
+  a.b2 = beta2;
+  a.eps = eps;
+  a.wd = weight_decay;
+  a.c1 = (float)(1.0 - std::pow((double)beta1, (double)step));
+  a.c2 = (float)(1.0 - std::pow((double)beta2, (double)step));
+  const long nblk = (long)((n + kAdamBlock - 1) / kAdamBlock);
+  adamw8_kernel<<<(unsigned)nblk, kAdamBlock, 0, (cudaStream_t)stream>>>(p, grad, m_q, m_absmax, v_q, v_absmax, (long)n,
+                                                                        a, adamw8_tables(),
+                                                                        (__nv_bfloat16*)p_bf16);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return launch_status();
+}
 
 extern "C" int qlora_linear_fwd_noalloc(int qtype, const void* wq, int64_t N, int64_t K, const void* X, int64_t M,
                                         const void* A, const void* B, int r, float scale, void* Y, int y_dtype,
