@@ -336,6 +336,22 @@ def also_measurements(flush, steps, pk):
     out["adamw8_adapters_r16_4096x4096"] = {"params": n, "ms": ms_a, "gbs": abytes / (ms_a / 1e3) / 1e9}
     device_status_ok("adamw8")
     del st, pp, gg, pb
+    # RMSNorm before the headline projection: 2048 tokens x 4096, forward (x -> bf16 x_n, rstd) and
+    # backward (fp32 d -> fp32 dx)
+    M_, K_ = 2048, 4096
+    xr = torch.randn(M_, K_, device="cuda").to(torch.bfloat16)
+    gr = torch.ones(K_, device="cuda").to(torch.bfloat16)
+    xn_ = torch.empty(M_, K_, dtype=torch.bfloat16, device="cuda")
+    rs_ = torch.empty(M_, dtype=torch.float32, device="cuda")
+    dxn_ = torch.randn(M_, K_, device="cuda")
+    dx_ = torch.empty(M_, K_, dtype=torch.float32, device="cuda")
+    ms_nf, _ = time_steps(lambda: ql.qlora_rmsnorm_fwd(xr, gr, 1e-6, xn_, rs_), steps, 3, flush)
+    ms_nb, _ = time_steps(lambda: ql.qlora_rmsnorm_bwd(xr, gr, rs_, dxn_, dx_), steps, 3, flush)
+    out["rmsnorm_2048x4096"] = {"fwd_ms": ms_nf, "bwd_ms": ms_nb,
+                                "fwd_gbs": (M_ * K_ * 4) / (ms_nf / 1e3) / 1e9,
+                                "bwd_gbs": (M_ * K_ * (2 + 4 + 4)) / (ms_nb / 1e3) / 1e9}
+    device_status_ok("rmsnorm")
+    del xr, gr, xn_, rs_, dxn_, dx_
     # routing alone at 4096 tokens, 256 experts, top-8 (the skewed workload's logits)
     c = inp.moe_q4_k_256x4096x1536(4096)
     lg = bf16_dev(c.logits)

@@ -197,6 +197,18 @@ int qlora_moe_bwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
                   void* stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * RMSNorm in front of the first projection ("RMSNorm from Liger Kernel", Show HN: LoRA over GGUF,
+ * "Things involved in the training"). X [M x K] bf16, gamma [K] bf16 (frozen), K % 8 == 0.
+ * Forward: rstd[m] = 1 / sqrt(mean_k X[m][k]^2 + eps) (fp32), Xn = bf16(X rstd gamma) [M x K]: the
+ * bf16 input of qlora_linear_fwd / qlora_linear_bwd. One pass per row (a warp per row).
+ * Backward: dX = rstd gamma d - (rstd^3 X / K) sum_k X gamma d, d = dXn [M x K] (dxn_dtype, e.g. the
+ * dX of qlora_linear_bwd) -> dX of dx_dtype. gamma is not trained (no gradient for it). */
+int qlora_rmsnorm_fwd(const void* X, const void* gamma, int64_t M, int64_t K, float eps, void* Xn, float* rstd,
+                      void* stream);
+int qlora_rmsnorm_bwd(const void* X, const void* gamma, const float* rstd, const void* dXn, int dxn_dtype,
+                      int64_t M, int64_t K, void* dX, int dx_dtype, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
  * 8-bit AdamW step on the adapter parameters (the recipe's bitsandbytes 8-bit AdamW optimizer,
  * Show HN: LoRA over GGUF, "Things involved in the training"): AdamW with decoupled weight decay
  * whose moments are kept in 8 bits, block-wise.

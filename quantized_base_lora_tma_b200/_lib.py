@@ -49,6 +49,8 @@ SIGNATURES = {
     "qlora_moe_bwd": (_c_int, [_c_int, _c_vp, _c_vp, _c_int, _c_i64, _c_i64, _c_vp, _c_vp, _c_i64, _c_int, _c_vp,
                                _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_f, _c_vp,
                                _c_sz, _c_vp, _c_int, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_sz, _c_vp]),
+    "qlora_rmsnorm_fwd": (_c_int, [_c_vp, _c_vp, _c_i64, _c_i64, _c_f, _c_vp, _c_vp, _c_vp]),
+    "qlora_rmsnorm_bwd": (_c_int, [_c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_i64, _c_i64, _c_vp, _c_int, _c_vp]),
     "qlora_adamw8_step": (_c_int, [_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_f, _c_f, _c_f, _c_f, _c_f,
                                    _c_i64, _c_vp, _c_vp]),
     "qlora_linear_fwd_noalloc": (_c_int, [_c_int, _c_vp, _c_i64, _c_i64, _c_vp, _c_i64, _c_vp, _c_vp, _c_int,
@@ -258,3 +260,14 @@ def qlora_adamw8_step(p, grad, state, step, lr=1e-4, beta1=0.9, beta2=0.999, eps
                                    _p(state.v_absmax), p.numel(), lr, beta1, beta2, eps, weight_decay, step,
                                    _p(p_bf16) if p_bf16 is not None else None, _s(stream)),
            "qlora_adamw8_step")
+
+
+def qlora_rmsnorm_fwd(X, gamma, eps, Xn, rstd, stream=None):
+    M, K = X.shape
+    _check(lib().qlora_rmsnorm_fwd(_p(X), _p(gamma), M, K, eps, _p(Xn), _p(rstd), _s(stream)), "qlora_rmsnorm_fwd")
+
+
+def qlora_rmsnorm_bwd(X, gamma, rstd, dXn, dX, stream=None):
+    M, K = X.shape
+    _check(lib().qlora_rmsnorm_bwd(_p(X), _p(gamma), _p(rstd), _p(dXn), _dt(dXn), M, K, _p(dX), _dt(dX), _s(stream)),
+           "qlora_rmsnorm_bwd")

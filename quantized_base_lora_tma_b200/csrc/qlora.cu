@@ -21,6 +21,7 @@
 #include "gemv.cuh"
 #include "moe.cuh"
 #include "adamw8.cuh"
+#include "rmsnorm.cuh"
 
 namespace qlora {
 
@@ -1622,6 +1623,34 @@ static const Adamw8Tables& adamw8_tables() {
 }
 
 }  // namespace qlora
+
+extern "C" int qlora_rmsnorm_fwd(const void* X, const void* gamma, int64_t M, int64_t K, float eps, void* Xn,
+                                 float* rstd, void* stream) {
+  if (!X || !gamma || !Xn || !rstd) return QL_ERR_INVALID_ARG;
+  if (M < 1 || K < 8 || !(eps >= 0.f)) return QL_ERR_INVALID_ARG;
+  if (K % 8 != 0 || M > (1 << 28) || K > (1 << 24)) return QL_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(gamma) || !aligned16(Xn)) return QL_ERR_ALIGNMENT;
+  const long threads = M * 32L;
+  rmsnorm_fwd_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, (cudaStream_t)stream>>>(
+      (const __nv_bfloat16*)X, (const __nv_bfloat16*)gamma, (int)M, (int)K, eps, (__nv_bfloat16*)Xn, rstd);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return launch_status();
+}
+
+extern "C" int qlora_rmsnorm_bwd(const void* X, const void* gamma, const float* rstd, const void* dXn, int dxn_dtype,
+                                 int64_t M, int64_t K, void* dX, int dx_dtype, void* stream) {
+  if (!X || !gamma || !rstd || !dXn || !dX) return QL_ERR_INVALID_ARG;
+  if ((dxn_dtype != QL_F32 && dxn_dtype != QL_BF16) || (dx_dtype != QL_F32 && dx_dtype != QL_BF16))
+    return QL_ERR_INVALID_ARG;
+  if (M < 1 || K < 8) return QL_ERR_INVALID_ARG;
+  if (K % 8 != 0 || M > (1 << 28) || K > (1 << 24)) return QL_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(gamma) || !aligned16(dXn) || !aligned16(dX)) return QL_ERR_ALIGNMENT;
+  const long threads = M * 32L;
+  rmsnorm_bwd_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, (cudaStream_t)stream>>>(
+      (const __nv_bfloat16*)X, (const __nv_bfloat16*)gamma, rstd, dXn, dxn_dtype, (int)M, (int)K, dX, dx_dtype);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return launch_status();
+}
 
 extern "C" int qlora_adamw8_step(float* p, const float* grad, uint8_t* m_q, float* m_absmax, uint8_t* v_q,
                                  float* v_absmax, int64_t n, float lr, float beta1, float beta2, float eps,
