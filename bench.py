@@ -352,6 +352,24 @@ def also_measurements(flush, steps, pk):
                                 "bwd_gbs": (M_ * K_ * (2 + 4 + 4)) / (ms_nb / 1e3) / 1e9}
     device_status_ok("rmsnorm")
     del xr, gr, xn_, rs_, dxn_, dx_
+    # quantized lm_head with chunked cross-entropy: 2048 tokens, hidden 2048, 128K vocabulary, Q8_0
+    lm = inp.lm_head_q8_0_128k()
+    lw = torch.from_numpy(lm["wq"]).cuda()
+    lx = bf16_dev(lm["X"])
+    llab = torch.from_numpy(lm["labels"]).cuda()
+    lws = torch.empty(ql.qlora_lm_head_ce_workspace_bytes(lm["M"], lm["V"], lm["K"], 256), dtype=torch.uint8,
+                      device="cuda")
+    lloss = torch.empty(lm["M"], dtype=torch.float32, device="cuda")
+    ldx = torch.empty(lm["M"], lm["K"], dtype=torch.bfloat16, device="cuda")
+    ms_l, _ = time_steps(lambda: ql.qlora_lm_head_ce(lm["qtype"], lw, lm["V"], lm["K"], lx, llab, 256, 1.0 / lm["M"],
+                                                   lloss, ldx, lws), max(5, steps // 4), 3, flush)
+    lflops = 4.0 * lm["M"] * lm["V"] * lm["K"]
+    out["lm_head_ce_q8_0_2048x2048x131072_chunk256"] = {
+        "ms": ms_l, "tokens_per_s": lm["M"] / (ms_l / 1e3), "tflops": lflops / (ms_l / 1e3) / 1e12,
+        "frac_of_bf16_peak": lflops / (ms_l / 1e3) / 1e12 / pk["bf16_tflops"]}
+    device_status_ok("lm_head")
+    del lm, lw, lx, llab, lws, lloss, ldx
+    torch.cuda.empty_cache()
     # routing alone at 4096 tokens, 256 experts, top-8 (the skewed workload's logits)
     c = inp.moe_q4_k_256x4096x1536(4096)
     lg = bf16_dev(c.logits)

@@ -197,6 +197,21 @@ int qlora_moe_bwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
                   void* stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * Quantized lm_head with chunked cross-entropy ("Chunked cross entropy loss like Liger Kernel, which
+ * works with MMQ", Show HN: LoRA over GGUF, "Things involved in the training"). W packed [V rows x K]
+ * (a type the layer's GEMMs take), X [M x K] bf16 (the final hidden states), labels [M] int32 in
+ * [0, V) or negative (ignored token). Rules: K % 256 == 0, V % 64 == 0.
+ * Per chunk of `chunk` token rows: fp32 logits = X_c deq(W)^T in the workspace (the dequant GEMM,
+ * no adapter); per row lse = log sum exp(logits), loss[m] = lse - logits[label] (0 if ignored); if
+ * dX is not NULL, D = (softmax - onehot(label)) grad_scale in bf16 (zero rows for ignored tokens) and
+ * dX_c = D deq(W) (dx_dtype): the gradient of grad_scale times the summed loss. The full [M x V]
+ * logits never exist: the workspace holds one chunk's fp32 logits and bf16 D. */
+size_t qlora_lm_head_ce_workspace_bytes(int64_t M, int64_t V, int64_t K, int64_t chunk);
+int qlora_lm_head_ce(int qtype, const void* wq, int64_t V, int64_t K, const void* X, int64_t M,
+                     const int32_t* labels, int64_t chunk, float grad_scale, float* loss, void* dX, int dx_dtype,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
  * RMSNorm in front of the first projection ("RMSNorm from Liger Kernel", Show HN: LoRA over GGUF,
  * "Things involved in the training"). X [M x K] bf16, gamma [K] bf16 (frozen), K % 8 == 0.
  * Forward: rstd[m] = 1 / sqrt(mean_k X[m][k]^2 + eps) (fp32), Xn = bf16(X rstd gamma) [M x K]: the

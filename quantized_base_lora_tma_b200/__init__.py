@@ -11,4 +11,5 @@ from ._lib import (Q4_0, Q4_K, Q8_0, QL_BF16, QL_F32, QloraError, gguf_dequant, 
                    qlora_set_rows_fusion,
                    qlora_status_string, MoeRoute, qlora_moe_route, qlora_moe_saved_bytes,
                    qlora_moe_workspace_bytes, qlora_moe_fwd, qlora_moe_bwd, Adamw8State, qlora_adamw8_step,
-                   qlora_rmsnorm_fwd, qlora_rmsnorm_bwd)
+                   qlora_rmsnorm_fwd, qlora_rmsnorm_bwd,
+                   qlora_lm_head_ce_workspace_bytes, qlora_lm_head_ce)

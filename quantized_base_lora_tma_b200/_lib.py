@@ -49,6 +49,9 @@ SIGNATURES = {
     "qlora_moe_bwd": (_c_int, [_c_int, _c_vp, _c_vp, _c_int, _c_i64, _c_i64, _c_vp, _c_vp, _c_i64, _c_int, _c_vp,
                                _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_f, _c_vp,
                                _c_sz, _c_vp, _c_int, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_sz, _c_vp]),
+    "qlora_lm_head_ce_workspace_bytes": (_c_sz, [_c_i64, _c_i64, _c_i64, _c_i64]),
+    "qlora_lm_head_ce": (_c_int, [_c_int, _c_vp, _c_i64, _c_i64, _c_vp, _c_i64, _c_vp, _c_i64, _c_f, _c_vp, _c_vp,
+                                  _c_int, _c_vp, _c_sz, _c_vp]),
     "qlora_rmsnorm_fwd": (_c_int, [_c_vp, _c_vp, _c_i64, _c_i64, _c_f, _c_vp, _c_vp, _c_vp]),
     "qlora_rmsnorm_bwd": (_c_int, [_c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_i64, _c_i64, _c_vp, _c_int, _c_vp]),
     "qlora_adamw8_step": (_c_int, [_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_f, _c_f, _c_f, _c_f, _c_f,
@@ -271,3 +274,15 @@ def qlora_rmsnorm_bwd(X, gamma, rstd, dXn, dX, stream=None):
     M, K = X.shape
     _check(lib().qlora_rmsnorm_bwd(_p(X), _p(gamma), _p(rstd), _p(dXn), _dt(dXn), M, K, _p(dX), _dt(dX), _s(stream)),
            "qlora_rmsnorm_bwd")
+
+
+def qlora_lm_head_ce_workspace_bytes(M, V, K, chunk) -> int:
+    return int(lib().qlora_lm_head_ce_workspace_bytes(M, V, K, chunk))
+
+
+def qlora_lm_head_ce(qtype, wq, V, K, X, labels, chunk, grad_scale, loss, dX, ws, stream=None):
+    M = X.shape[0]
+    _check(lib().qlora_lm_head_ce(qtype, _p(wq), V, K, _p(X), M, _p(labels), chunk, grad_scale, _p(loss),
+                                  _p(dX) if dX is not None else None, _dt(dX) if dX is not None else QL_F32,
+                                  _p(ws), _nb(ws), _s(stream)),
+           "qlora_lm_head_ce")

@@ -22,6 +22,7 @@
 #include "moe.cuh"
 #include "adamw8.cuh"
 #include "rmsnorm.cuh"
+#include "lmhead.cuh"
 
 namespace qlora {
 
@@ -171,6 +172,16 @@ static inline int launch_status() {
 // ------------------------------------------------------------------------------------------------
 // Launch helpers
 // ------------------------------------------------------------------------------------------------
+// While a NoEarlyStart is alive on a thread, PdlLaunch launches from that thread without programmatic
+// stream serialization: the kernel starts only once the previous kernel in the stream has completed
+// (for a GEMM whose A operand the immediately preceding kernel writes: the unfused pair GEMM streams
+// A before it waits for its predecessor).
+static thread_local int t_no_early_start = 0;
+struct NoEarlyStart {
+  NoEarlyStart() { ++t_no_early_start; }
+  ~NoEarlyStart() { --t_no_early_start; }
+};
+
 // Launch configuration with programmatic stream serialization (the kernel may start while the
 // previous kernel in the stream finishes; the dense-path kernels wait on it in-kernel) and, when
 // cluster_y > 0, a (1, cluster_y, 1) cluster shape.
@@ -184,7 +195,7 @@ struct PdlLaunch {
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[0].val.programmaticStreamSerializationAllowed = t_no_early_start ? 0 : 1;
     int n = 1;
     if (cluster_y > 0) {
       attr[1].id = cudaLaunchAttributeClusterDimension;
@@ -650,9 +661,14 @@ static int launch_dense_gemm(int qtype, const void* A, int64_t M, int64_t Kd, co
   const uint32_t box = 128u;
   CUtensorMap tA, tW, tLA, tLB;
   if (!tmap_bf16_rows(&tA, A, Kd, M, box) ||
-      !tmap_packed(&tW, wq, packed_row_bytes(qtype, w_cols), w_rows, group_bytes(qtype)) ||
-      !tmap_bf16_rows(&tLA, LA, KL, M, box) || !tmap_bf16_rows(&tLB, LB, KL, Nd, 64))
+      !tmap_packed(&tW, wq, packed_row_bytes(qtype, w_cols), w_rows, group_bytes(qtype)))
     return QL_ERR_CUDA;
+  if (KL == 0) {  // no adapter k-blocks (the kernels never read these maps then)
+    tLA = tA;
+    tLB = tA;
+  } else if (!tmap_bf16_rows(&tLA, LA, KL, M, box) || !tmap_bf16_rows(&tLB, LB, KL, Nd, 64)) {
+    return QL_ERR_CUDA;
+  }
   GemmParams p;
   memset(&p, 0, sizeof(p));
   p.M = (int)M;
@@ -1623,6 +1639,81 @@ static const Adamw8Tables& adamw8_tables() {
 }
 
 }  // namespace qlora
+
+// ------------------------------------------------------------------------------------------------
+// Quantized lm_head with chunked cross-entropy
+// ------------------------------------------------------------------------------------------------
+namespace qlora {
+
+struct LmWs {
+  size_t logits, dlog, split_f, split_x, total;
+};
+static LmWs lm_ws(int64_t M, int64_t V, int64_t K, int64_t chunk) {
+  const int64_t C = std::min(chunk, M);
+  const int64_t tail = M % C;
+  size_t sf = 0, sx = 0;
+  for (int64_t rows : {C, tail}) {
+    if (rows < 1) continue;
+    sf = std::max(sf, split_bytes(plan_dense(rows, V, K, false, true), rows, V));
+    sx = std::max(sx, split_bytes(plan_dense(rows, K, V, true, true), rows, K));
+  }
+  LmWs w;
+  size_t o = 0;
+  w.logits = o; o = al256(o + (size_t)C * V * 4);
+  w.dlog = o; o = al256(o + (size_t)C * V * 2);
+  w.split_f = o; o = al256(o + sf);
+  w.split_x = o; o = al256(o + sx);
+  w.total = o;
+  return w;
+}
+
+}  // namespace qlora
+
+extern "C" size_t qlora_lm_head_ce_workspace_bytes(int64_t M, int64_t V, int64_t K, int64_t chunk) {
+  if (M < 1 || V < 1 || K < 1 || chunk < 1) return 0;
+  return lm_ws(M, V, K, chunk).total;
+}
+
+extern "C" int qlora_lm_head_ce(int qtype, const void* wq, int64_t V, int64_t K, const void* X, int64_t M,
+                                const int32_t* labels, int64_t chunk, float grad_scale, float* loss, void* dX,
+                                int dx_dtype, void* ws, size_t ws_bytes, void* stream) {
+  if (!wq || !X || !labels || !loss) return QL_ERR_INVALID_ARG;
+  if (group_bytes(qtype) == 0) return QL_ERR_UNSUPPORTED;
+  if (M < 1 || V < 64 || K < 256 || chunk < 1) return QL_ERR_INVALID_ARG;
+  if (K % 256 != 0 || V % 64 != 0 || M > (1 << 26) || K > (1 << 16) || V > (1 << 22)) return QL_ERR_SHAPE;
+  if (dX && dx_dtype != QL_F32 && dx_dtype != QL_BF16) return QL_ERR_INVALID_ARG;
+  if (!aligned16(wq) || !aligned16(X) || !aligned16(loss) || (dX && !aligned16(dX))) return QL_ERR_ALIGNMENT;
+  const LmWs w = lm_ws(M, V, K, chunk);
+  if (!ws || ws_bytes < w.total) return QL_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QL_ERR_ALIGNMENT;
+  cudaStream_t st = (cudaStream_t)stream;
+  uint8_t* wsb = (uint8_t*)ws;
+  float* logits = (float*)(wsb + w.logits);
+  __nv_bfloat16* dlog = (__nv_bfloat16*)(wsb + w.dlog);
+  const int64_t C = std::min(chunk, M);
+  const size_t xes = dx_dtype == QL_F32 ? 4 : 2;
+  for (int64_t c0 = 0; c0 < M; c0 += C) {
+    const int64_t rows = std::min(C, M - c0);
+    const __nv_bfloat16* Xc = (const __nv_bfloat16*)X + c0 * K;
+    // logits = X_c deq(W)^T, fp32, no adapter
+    int rc = launch_dense_gemm<false>(qtype, Xc, rows, K, wq, V, K, nullptr, nullptr, 0, V, logits, QL_F32,
+                                      (float*)(wsb + w.split_f), true, st, 0);
+    if (rc) return rc;
+    // the CE kernel and the input-gradient GEMM each read what the launch right before them wrote:
+    // they start only once it has completed
+    NoEarlyStart serial;
+    lm_ce_kernel<<<(unsigned)rows, kCeThreads, 0, st>>>(logits, (int)V, labels + c0, grad_scale, loss + c0,
+                                                        dX ? dlog : nullptr);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (launch_status() != QL_OK) return QL_ERR_CUDA;
+    if (dX) {
+      rc = launch_dense_gemm<true>(qtype, dlog, rows, V, wq, V, K, nullptr, nullptr, 0, K,
+                                   (uint8_t*)dX + c0 * K * xes, dx_dtype, (float*)(wsb + w.split_x), true, st, 1);
+      if (rc) return rc;
+    }
+  }
+  return QL_OK;
+}
 
 extern "C" int qlora_rmsnorm_fwd(const void* X, const void* gamma, int64_t M, int64_t K, float eps, void* Xn,
                                  float* rstd, void* stream) {

@@ -389,6 +389,28 @@ def synth_q4_k(rng, rows: int, cols: int) -> np.ndarray:
     return out.reshape(rows, -1)
 
 
+def synth_q8_0(rng, rows: int, cols: int) -> np.ndarray:
+    """Valid Q8_0 blocks drawn directly as bytes, [rows x cols/32 x 34]: fp16 d uniform in
+    [1.0e-4, 3.0e-4), int8 codes uniform in [-127, 127]. The weights d q then spread over about
+    +-0.04 (std near 0.0135), without encoding fp32 weights first."""
+    nb = rows * (cols // 32)
+    out = np.empty((nb, 34), np.uint8)
+    out[:, 0:2] = rng.uniform(1.0e-4, 3.0e-4, nb).astype(np.float16).view(np.uint8).reshape(-1, 2)
+    out[:, 2:] = rng.integers(-127, 128, (nb, 32), dtype=np.int8).view(np.uint8)
+    return out.reshape(rows, -1)
+
+
+def lm_head_q8_0_128k(M=2048, seed=0):
+    """Quantized lm_head workload: M tokens of hidden 2048, a 131072-entry vocabulary, Q8_0 weights
+    drawn as blocks (synth_q8_0), labels uniform over the vocabulary. Draw order: W, X, labels."""
+    V, K = 131072, 2048
+    rng = np.random.default_rng(seed)
+    wq = synth_q8_0(rng, V, K)
+    X = to_bf16_bits(_normal(rng, (M, K), 1.0))
+    labels = rng.integers(0, V, M).astype(np.int32)
+    return dict(V=V, K=K, M=M, qtype=Q8_0, wq=wq, X=X, labels=labels)
+
+
 _MOE256 = {}
 
 

@@ -574,3 +574,24 @@ def _pair_dgu(d, saved, pos, t, e, w):
     dhu = dy @ d["Wd"][e] + Gd @ d["Ad"][e]
     sg = 1.0 / (1.0 + np.exp(-g))
     return np.concatenate([w * dhu * uu * sg * (1 + g * (1 - sg)), w * dhu * g * sg])
+
+
+def test_synth_q8_0_blocks_have_the_stated_fields():
+    """The lm_head workload's Q8_0 blocks are drawn as bytes: d in its range, codes in [-127, 127],
+    and gguf-py decodes them to the oracle's values."""
+    rng = np.random.default_rng(4)
+    raw = inp.synth_q8_0(rng, 16, 512)
+    b = raw.reshape(-1, 34)
+    d = b[:, 0:2].copy().view(np.float16).astype(np.float64).ravel()
+    q = b[:, 2:].view(np.int8)
+    assert d.min() >= 0.99e-4 and d.max() <= 3.01e-4 and q.min() >= -127 and q.max() <= 127
+    w = gb.decode_exact(inp.Q8_0, raw, 16, 512)
+    assert 0.008 < w.std() < 0.02
+    try:
+        import gguf
+        from gguf import quants
+    except ImportError:
+        return
+    want = quants.dequantize(raw, gguf.GGMLQuantizationType.Q8_0).astype(np.float32)
+    assert np.array_equal(gb.deq_f32(inp.Q8_0, raw, 16, 512).astype(np.float32).view(np.uint32),
+                          want.reshape(16, 512).view(np.uint32))
