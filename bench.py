@@ -678,7 +678,31 @@ def run_reference(args, rank, world):
     }
 
 
+class LmHeadRun:
+    """Device buffers and one call of the quantized lm_head with chunked cross-entropy."""
+
+    def __init__(self, lm, chunk=256):
+        import quantized_base_lora_tma_b200 as ql
+        self.ql, self.lm, self.chunk = ql, lm, chunk
+        self.w = torch.from_numpy(lm["wq"]).cuda()
+        self.x = bf16_dev(lm["X"])
+        self.lab = torch.from_numpy(lm["labels"]).cuda()
+        self.ws = torch.empty(ql.qlora_lm_head_ce_workspace_bytes(lm["M"], lm["V"], lm["K"], chunk),
+                              dtype=torch.uint8, device="cuda")
+        self.loss = torch.empty(lm["M"], dtype=torch.float32, device="cuda")
+        self.dx = torch.empty(lm["M"], lm["K"], dtype=torch.bfloat16, device="cuda")
+
+    def step(self):
+        lm = self.lm
+        self.ql.qlora_lm_head_ce(lm["qtype"], self.w, lm["V"], lm["K"], self.x, self.lab, self.chunk, 1.0 / lm["M"],
+                                 self.loss, self.dx, self.ws)
+
+    fwd = step
+
+
 PROFILE_CASES = {
+    "moe_q4_k_e32_t4096": lambda: MoERun(inp.moe_q4_k_256x4096x1536(4096, E=32)),
+    "lm_head": lambda: LmHeadRun(inp.lm_head_q8_0_128k()),
     "dense_q8_0": lambda: DenseLayerRun(inp.dense_proj_2048x4096x4096(inp.Q8_0)),
     "dense_q4_0": lambda: DenseLayerRun(inp.dense_proj_2048x4096x4096(inp.Q4_0)),
     "gate_up_q4_k": lambda: DenseLayerRun(inp.gate_up_q4_k_2048x2048x12288()),

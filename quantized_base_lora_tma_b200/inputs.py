@@ -414,16 +414,18 @@ def lm_head_q8_0_128k(M=2048, seed=0):
 _MOE256 = {}
 
 
-def moe_q4_k_256x4096x1536(T, seed=0):
+def moe_q4_k_256x4096x1536(T, seed=0, E=256):
     """Skewed, weight-bound MoE: T tokens, hidden 4096, 256 experts of intermediate 1536, top-8,
     Q4_K, Zipf(1.1) popularity bias on the logits, rank 4, alpha 8 on gate/up and down.
 
     The layer shape is fixed and its weights are the same for every T: they and the adapters come
-    from default_rng(seed), in the order W_gu_e, W_d_e for e = 0..255 (drawn as Q4_K blocks by
+    from default_rng(seed), in the order W_gu_e, W_d_e for e = 0..E-1 (drawn as Q4_K blocks by
     synth_q4_k), then A_gu, B_gu, A_d, B_d; X, dY and the logits come from default_rng([seed, T]).
-    The packed weights are kept between calls (2.7 GB)."""
-    H, I, E, k, r = 4096, 1536, 256, 8, 4
-    if seed not in _MOE256:
+    The packed weights are kept between calls (2.7 GB). E < 256 gives the same expert shape with
+    fewer experts (a profiling case small enough to capture with every counter)."""
+    H, I, k, r = 4096, 1536, 8, 4
+    key = (seed, E)
+    if key not in _MOE256:
         rng = np.random.default_rng(seed)
         w_gu = np.empty((E, 2 * I, row_bytes(Q4_K, H)), np.uint8)
         w_d = np.empty((E, H, row_bytes(Q4_K, I)), np.uint8)
@@ -435,13 +437,13 @@ def moe_q4_k_256x4096x1536(T, seed=0):
         A_d = to_bf16_bits(_normal(rng, (E, r, I), 1.0 / math.sqrt(I)))
         B_d = to_bf16_bits(_normal(rng, (E, H, r), 0.01))
         _MOE256.clear()
-        _MOE256[seed] = (w_gu, w_d, A_gu, B_gu, A_d, B_d)
-    w_gu, w_d, A_gu, B_gu, A_d, B_d = _MOE256[seed]
+        _MOE256[key] = (w_gu, w_d, A_gu, B_gu, A_d, B_d)
+    w_gu, w_d, A_gu, B_gu, A_d, B_d = _MOE256[key]
     rng = np.random.default_rng([seed, T])
     X = _normal(rng, (T, H), 1.0)
     dY = _normal(rng, (T, H), 1.0)
     logits = _normal(rng, (T, E), 1.0) - np.float32(1.1) * np.log(np.arange(1, E + 1, dtype=np.float32))[None, :]
-    return MoECase(f"moe_q4_k_T{T}_H4096_E256_I1536_k8_zipf", Q4_K, T, H, I, E, k, r, 8.0, to_bf16_bits(X),
+    return MoECase(f"moe_q4_k_T{T}_H4096_E{E}_I1536_k8_zipf", Q4_K, T, H, I, E, k, r, 8.0, to_bf16_bits(X),
                    to_bf16_bits(dY), to_bf16_bits(logits), w_gu, w_d, A_gu, B_gu, A_d, B_d)
 
 
