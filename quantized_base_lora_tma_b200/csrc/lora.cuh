@@ -914,7 +914,13 @@ __host__ __device__ constexpr size_t rows_seg_z_smem(int NT, int Kin) { return (
 // The grouped row products of lora_rows_seg_kernel with the expert's whole adapter slice resident
 // in shared memory ([RN][Kin + 8], k contiguous; staged once, transposed on the way in when j is the
 // contiguous index), so the stream of Y needs no barrier: each thread keeps the next 128-wide
-// chunk of its two rows in flight while it multiplies the current one. Kin % 8 == 0.
+// chunk of its two rows in flight while it multiplies the current one. Kin % 256 == 0.
+//
+// The block's rows make nrt = ceil(rows / 16) row tiles; the 8 warps split into 8 / nrt groups
+// that take interleaved 128-wide k chunks of every tile, so a short segment (a tiny expert) keeps
+// all warps streaming instead of one. The groups' partials are summed in group order through
+// shared memory (the adapter slice is no longer needed by then), so the result does not depend on
+// timing.
 template <int NT>
 __global__ void __launch_bounds__(256, 2) lora_rows_seg_z_kernel(
     const __nv_bfloat16* __restrict__ Y, long ldy, int Kin, const __nv_bfloat16* __restrict__ Z, long zj, long zk,
@@ -935,11 +941,15 @@ __global__ void __launch_bounds__(256, 2) lora_rows_seg_z_kernel(
   const int e = a;
   const int row_lo = __ldg(seg_off + e) + (blk - __ldg(mblk_off + e)) * 128;
   const int row_hi = min(__ldg(seg_off + e + 1), row_lo + 128);
+  const int nrt = (row_hi - row_lo + 15) >> 4;  // 1..8
+  const int ngrp = 8 / nrt;
   const __nv_bfloat16* Ze = Z + (long)e * zes;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int rt = warp % nrt, grp = warp / nrt;
+  const bool active = grp < ngrp;
   const int g = lane >> 2, c = lane & 3;
-  const int r0 = row_lo + warp * 16 + g, r1 = r0 + 8;
-  const bool v0 = r0 < row_hi, v1 = r1 < row_hi;
+  const int r0 = row_lo + rt * 16 + g, r1 = r0 + 8;
+  const bool v0 = active && r0 < row_hi, v1 = active && r1 < row_hi;
   const __nv_bfloat16* y0 = Y + (long)(v0 ? r0 : row_lo) * ldy;
   const __nv_bfloat16* y1 = Y + (long)(v1 ? r1 : row_lo) * ldy;
   auto load = [&](uint4 (&xa)[SK / 32], uint4 (&xb)[SK / 32], int k0) {
@@ -951,15 +961,29 @@ __global__ void __launch_bounds__(256, 2) lora_rows_seg_z_kernel(
       xb[q] = (v1 && in) ? __ldg(reinterpret_cast<const uint4*>(y1 + k)) : make_uint4(0, 0, 0, 0);
     }
   };
+  const int kstep = ngrp * SK;
   // the first chunk is on its way while the adapter slice is staged
   uint4 xa0[SK / 32], xb0[SK / 32], xa1[SK / 32], xb1[SK / 32];
-  load(xa0, xb0, 0);
+  load(xa0, xb0, grp * SK);
   if (zk == 1) {
     for (int i = tid; i < RN * (Kin / 8); i += 256) {
       const int j = i / (Kin / 8), q = i - j * (Kin / 8);
       uint4 v = make_uint4(0, 0, 0, 0);
       if (j < r) v = __ldg(reinterpret_cast<const uint4*>(Ze + (long)j * zj + 8 * q));
       *reinterpret_cast<uint4*>(zsd + j * ZS + 8 * q) = v;
+    }
+  } else if (zj == 1 && zk == r && (reinterpret_cast<uintptr_t>(Ze) & 15) == 0) {
+    // [Kin][r] contiguous: 16-byte loads, scattered to [j][k]
+    for (int i = tid; i < RN * ZS / 2; i += 256) reinterpret_cast<uint32_t*>(zsd)[i] = 0u;
+    __syncthreads();
+    for (int i = tid; i < Kin * r / 8; i += 256) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(Ze) + i);
+      const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&v);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int f = 8 * i + q, kk = f / r, j = f - kk * r;
+        zsd[j * ZS + kk] = h[q];
+      }
     }
   } else {
     for (int i = tid; i < Kin * RN; i += 256) {
@@ -984,32 +1008,61 @@ __global__ void __launch_bounds__(256, 2) lora_rows_seg_z_kernel(
       }
     }
   };
-  for (int k0 = 0; k0 < Kin; k0 += 2 * SK) {
-    if (k0 + SK < Kin) load(xa1, xb1, k0 + SK);
-    compute(xa0, xb0, k0);
-    if (k0 + SK < Kin) {
-      if (k0 + 2 * SK < Kin) load(xa0, xb0, k0 + 2 * SK);
-      compute(xa1, xb1, k0 + SK);
+  if (active) {
+    for (int k0 = grp * SK; k0 < Kin; k0 += 2 * kstep) {
+      if (k0 + kstep < Kin) load(xa1, xb1, k0 + kstep);
+      compute(xa0, xb0, k0);
+      if (k0 + kstep < Kin) {
+        if (k0 + 2 * kstep < Kin) load(xa0, xb0, k0 + 2 * kstep);
+        compute(xa1, xb1, k0 + kstep);
+      }
     }
   }
-  // C fragment: rows r0 / r1, columns 8t + 2c (+1)
+  if (ngrp > 1) {
+    // partials of groups 1.. through shared memory: red[grp - 1][rt][lane][NT * 4]
+    float* red = reinterpret_cast<float*>(zsd);
+    __syncthreads();
+    if (active && grp > 0) {
+      float* dst = red + ((long)((grp - 1) * nrt + rt) * 32 + lane) * (NT * 4);
 #pragma unroll
-  for (int t = 0; t < NT; ++t) {
+      for (int t = 0; t < NT; ++t)
+        *reinterpret_cast<float4*>(dst + 4 * t) = make_float4(acc[t][0], acc[t][1], acc[t][2], acc[t][3]);
+    }
+    __syncthreads();
+    if (grp == 0) {
+      for (int o = 1; o < ngrp; ++o) {
+        const float* src = red + ((long)((o - 1) * nrt + rt) * 32 + lane) * (NT * 4);
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int row = hh ? r1 : r0;
-      if (!(hh ? v1 : v0)) continue;
+        for (int t = 0; t < NT; ++t) {
+          const float4 v = *reinterpret_cast<const float4*>(src + 4 * t);
+          acc[t][0] += v.x;
+          acc[t][1] += v.y;
+          acc[t][2] += v.z;
+          acc[t][3] += v.w;
+        }
+      }
+    }
+  }
+  // C fragment: rows r0 / r1, columns 8t + 2c (+1); written by the first group
+  if (grp == 0) {
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const int j = 8 * t + 2 * c + q;
-        const float v = acc[t][2 * hh + q];
-        if (out != nullptr && j < r) out[(long)row * r + j] = oscale * v;
-        if (la != nullptr && j < RP) {
-          const float x = lscale * v;
-          const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-          const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
-          la[(long)row * 2 * RP + j] = j < r ? hi : __float2bfloat16(0.f);
-          la[(long)row * 2 * RP + RP + j] = j < r ? lo : __float2bfloat16(0.f);
+    for (int t = 0; t < NT; ++t) {
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int row = hh ? r1 : r0;
+        if (!(hh ? v1 : v0)) continue;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int j = 8 * t + 2 * c + q;
+          const float v = acc[t][2 * hh + q];
+          if (out != nullptr && j < r) out[(long)row * r + j] = oscale * v;
+          if (la != nullptr && j < RP) {
+            const float x = lscale * v;
+            const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+            la[(long)row * 2 * RP + j] = j < r ? hi : __float2bfloat16(0.f);
+            la[(long)row * 2 * RP + RP + j] = j < r ? lo : __float2bfloat16(0.f);
+          }
         }
       }
     }
@@ -1028,59 +1081,64 @@ __global__ void __launch_bounds__(256, 2) lora_rows_seg_z_kernel(
 }
 
 // LB[e][n] = [Z_e(n, :) | Z_e(n, :)] zero padded to 2*RP columns; Z_e(n, j) = Z[e*zes + n*zn + j*zjs].
-// One thread per 8 output columns.
-__global__ void lora_bop_vec_kernel(const __nv_bfloat16* __restrict__ Z, long zn, long zjs, long zes, int rows, int nexp,
-                                    int r, int RP, __nv_bfloat16* __restrict__ LB) {
-  // 32-bit index arithmetic (the host keeps nexp * rows * 2RP / 8 below 2^31): a 64-bit division
-  // per item would cost more than the item
+// blockIdx.y is the expert; an expert whose segment is empty (seg_off given) is skipped, since no
+// GEMM tile reads its rows. One thread per 8 output columns.
+__global__ void lora_bop_vec_kernel(const __nv_bfloat16* __restrict__ Z, long zn, long zjs, long zes, int rows,
+                                    const int* __restrict__ seg_off, int r, int RP, __nv_bfloat16* __restrict__ LB) {
+  const int e = blockIdx.y;
+  if (seg_off != nullptr && __ldg(seg_off + e) == __ldg(seg_off + e + 1)) return;
+  // 32-bit index arithmetic within an expert (the host keeps rows * 2RP / 8 below 2^31)
   const int per_row = 2 * RP / 8;
-  const int items = nexp * rows * per_row;
+  const int items = rows * per_row;
+  const __nv_bfloat16* Ze = Z + (long)e * zes;
+  __nv_bfloat16* LBe = LB + (long)e * rows * 2 * RP;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < items; i += gridDim.x * blockDim.x) {
-    const int rn = i / per_row;
-    const int j0 = (i - rn * per_row) * 8;
-    const int e = rn / rows;
-    const int n = rn - e * rows;
+    const int n = i / per_row;
+    const int j0 = (i - n * per_row) * 8;
     const int jb = j0 % RP;  // first rank column of the chunk (both halves repeat Z)
     __nv_bfloat16 v[8];
     if (jb < r) {
-      const __nv_bfloat16* zp = Z + (long)e * zes + (long)n * zn;
+      const __nv_bfloat16* zp = Ze + (long)n * zn;
 #pragma unroll
       for (int q = 0; q < 8; ++q) v[q] = jb + q < r ? zp[(long)(jb + q) * zjs] : __float2bfloat16(0.f);
     } else {
 #pragma unroll
       for (int q = 0; q < 8; ++q) v[q] = __float2bfloat16(0.f);
     }
-    *reinterpret_cast<uint4*>(LB + (long)rn * 2 * RP + j0) = *reinterpret_cast<const uint4*>(v);
+    *reinterpret_cast<uint4*>(LBe + (long)n * 2 * RP + j0) = *reinterpret_cast<const uint4*>(v);
   }
 }
 
-// out = scale * ordered sum over the slices of each expert (dense: all slices, E = 1 output).
-// transpose = 0: out[e][c][j]; transpose = 1: out[e][j][c].
+// out = scale * ordered sum over the slices of each expert (dense: all slices, E = 0, one output).
+// transpose = 0: out[e][c][j]; transpose = 1: out[e][j][c]. blockIdx.y is the expert; an expert
+// without slices (no tokens) gets exact zeros, 16 bytes per store (Ccols * r % 4 == 0).
 __global__ void colred_reduce_kernel(const float* __restrict__ part, int Ccols, int r, int nslices_dense,
                                      const int* __restrict__ mblk_off, int E, float scale, int transpose,
                                      float* __restrict__ out) {
-  // i runs over the output in its own order (consecutive threads write consecutive floats), with
-  // 32-bit index arithmetic (the host keeps the count below 2^31)
-  const int nexp = E == 0 ? 1 : E;
+  const int e = blockIdx.y;
   const int per_e = Ccols * r;
-  const int total = nexp * per_e;
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
-    const int e = i / per_e;
-    const int w = i - e * per_e;
+  int s0, s1;
+  if (E == 0) { s0 = 0; s1 = nslices_dense; }
+  else { s0 = __ldg(mblk_off + e); s1 = __ldg(mblk_off + e + 1); }
+  float* oe = out + (long)e * per_e;
+  if (s0 == s1) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < per_e / 4; i += gridDim.x * blockDim.x)
+      reinterpret_cast<float4*>(oe)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    return;
+  }
+  // i runs over the expert's output in its own order (consecutive threads write consecutive floats)
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < per_e; i += gridDim.x * blockDim.x) {
     int c, j;
     if (transpose) {
-      j = w / Ccols;
-      c = w - j * Ccols;
+      j = i / Ccols;
+      c = i - j * Ccols;
     } else {
-      c = w / r;
-      j = w - c * r;
+      c = i / r;
+      j = i - c * r;
     }
-    int s0, s1;
-    if (E == 0) { s0 = 0; s1 = nslices_dense; }
-    else { s0 = __ldg(mblk_off + e); s1 = __ldg(mblk_off + e + 1); }
     float acc = 0.f;
     for (int s = s0; s < s1; ++s) acc += part[(long)s * per_e + c * r + j];
-    out[i] = scale * acc;
+    oe[i] = scale * acc;
   }
 }
 

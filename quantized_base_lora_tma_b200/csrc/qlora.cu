@@ -533,9 +533,9 @@ static int launch_colred(const __nv_bfloat16* Y, long ldy, int Ccols, const floa
   else colred_mma_kernel<4><<<grid, 128, 0, st>>>(Y, ldy, Ccols, Z, r, M, zw, seg_off, mblk_off, E, part, Ylo);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (launch_status() != QL_OK) return QL_ERR_CUDA;
-  const long total = (long)(E == 0 ? 1 : E) * Ccols * r;
-  if (total >= (1L << 31)) return QL_ERR_SHAPE;
-  const int g2 = (int)std::min<long>((total + 255) / 256, 148L * 16);
+  const long per_e = (long)Ccols * r;
+  if (per_e >= (1L << 31) || per_e % 4 != 0) return QL_ERR_SHAPE;
+  const dim3 g2((unsigned)std::min<long>((per_e + 255) / 256, 64L), E == 0 ? 1 : E);
   colred_reduce_kernel<<<g2, 256, 0, st>>>(part, Ccols, r, max_slices, mblk_off, E, scale, transpose, out);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return launch_status();
@@ -975,8 +975,8 @@ static int launch_rows_seg(const __nv_bfloat16* Y, long ldy, int Kin, const __nv
   const int RP = lora_rp(r);
   const int NT = r <= 16 ? 2 : (r <= 32 ? 4 : 8);
   const size_t zsm = rows_seg_z_smem(NT, Kin);
-  if (Kin % 8 == 0 && zsm <= 110 * 1024) {
-    // the expert's whole adapter slice resident in shared memory (two CTAs per SM)
+  if (Kin % 256 == 0 && zsm <= 220 * 1024) {
+    // the expert's whole adapter slice resident in shared memory (two CTAs per SM up to 110 KB)
     cudaError_t e;
     if (NT == 2) {
       e = set_smem(lora_rows_seg_z_kernel<2>, (int)zsm);
@@ -1012,12 +1012,14 @@ static int launch_rows_seg(const __nv_bfloat16* Y, long ldy, int Kin, const __nv
 }
 
 static int launch_bop_vec(const __nv_bfloat16* Z, long zn, long zjs, long zes, int rows, int nexp, int r,
-                          __nv_bfloat16* LB, cudaStream_t st) {
+                          __nv_bfloat16* LB, cudaStream_t st, const int* seg_off = nullptr) {
   const int RP = lora_rp(r);
-  const long items = (long)nexp * rows * (2 * RP / 8);
+  const long items = (long)rows * (2 * RP / 8);
   if (items >= (1L << 31)) return QL_ERR_SHAPE;
-  const int grid = (int)std::min<long>((items + 255) / 256, (long)num_sms() * 8);
-  lora_bop_vec_kernel<<<grid, 256, 0, st>>>(Z, zn, zjs, zes, rows, nexp, r, RP, LB);
+  // per expert about one CTA per 1024 items, at most one wave over all experts' CTAs
+  const long per_e = std::max(1L, std::min((items + 1023) / 1024, (long)num_sms() * 8 / nexp + 1));
+  const dim3 grid((unsigned)std::min(per_e, (items + 255) / 256), nexp);
+  lora_bop_vec_kernel<<<grid, 256, 0, st>>>(Z, zn, zjs, zes, rows, seg_off, r, RP, LB);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return launch_status();
 }
@@ -1261,7 +1263,7 @@ int qlora_moe_fwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
   rc = launch_rows_seg(Xp, H, (int)H, (const __nv_bfloat16*)A_gu, H, 1, (long)r * H, off, mblk, E, r, 1.0f, scale, Hgu,
                        LA, ms, st);
   if (rc) return rc;
-  rc = launch_bop_vec((const __nv_bfloat16*)B_gu, r, 1, (long)2 * I * r, (int)(2 * I), E, r, LB, st);
+  rc = launch_bop_vec((const __nv_bfloat16*)B_gu, r, 1, (long)2 * I * r, (int)(2 * I), E, r, LB, st, off);
   if (rc) return rc;
   const int nsm = num_sms();
   {
@@ -1284,7 +1286,7 @@ int qlora_moe_fwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
   rc = launch_rows_seg(h, I, (int)I, (const __nv_bfloat16*)A_d, I, 1, (long)r * I, off, mblk, E, r, 1.0f, scale, Hd, LA,
                        ms, st);
   if (rc) return rc;
-  rc = launch_bop_vec((const __nv_bfloat16*)B_d, r, 1, (long)H * r, (int)H, E, r, LB, st);
+  rc = launch_bop_vec((const __nv_bfloat16*)B_d, r, 1, (long)H * r, (int)H, E, r, LB, st, off);
   if (rc) return rc;
   {
     CUtensorMap tA, tW, tLA, tLB;
@@ -1361,7 +1363,7 @@ int qlora_moe_bwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
   rc = launch_rows_seg(dYp, H, (int)H, (const __nv_bfloat16*)B_d, 1, r, (long)H * r, off, mblk, E, r, scale, scale, Gd,
                        LA, ms, st);
   if (rc) return rc;
-  rc = launch_bop_vec((const __nv_bfloat16*)A_d, 1, I, (long)r * I, (int)I, E, r, LB, st);
+  rc = launch_bop_vec((const __nv_bfloat16*)A_d, 1, I, (long)r * I, (int)I, E, r, LB, st, off);
   if (rc) return rc;
   {
     CUtensorMap tA, tW, tLA, tLB;
@@ -1388,7 +1390,7 @@ int qlora_moe_bwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
   rc = launch_rows_seg(dgu, 2 * I, (int)(2 * I), (const __nv_bfloat16*)B_gu, 1, r, (long)2 * I * r, off, mblk, E, r,
                        scale, scale, Ggu, LA, ms, st);
   if (rc) return rc;
-  rc = launch_bop_vec((const __nv_bfloat16*)A_gu, 1, H, (long)r * H, (int)H, E, r, LB, st);
+  rc = launch_bop_vec((const __nv_bfloat16*)A_gu, 1, H, (long)r * H, (int)H, E, r, LB, st, off);
   if (rc) return rc;
   {
     CUtensorMap tA, tW, tLA, tLB;
