@@ -321,6 +321,7 @@ def also_measurements(flush, steps, pk):
     del m
     torch.cuda.empty_cache()
     # 8-bit AdamW on the headline layer's adapters (A [16 x 4096] and B [4096 x 16])
+    torch.manual_seed(0)
     n = 2 * 16 * 4096
     st = ql.Adamw8State(n)
     pp = torch.zeros(n, dtype=torch.float32, device="cuda")
