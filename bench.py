@@ -263,6 +263,7 @@ def allreduce_adapter_grads(grads):
         torch.distributed.all_reduce(g, op=torch.distributed.ReduceOp.SUM)
 
 
+LM_CHUNK = 1024  # token rows per cross-entropy chunk of the lm_head workload
 EV_EVERY = 8  # kernel events on one timed step in this many (as for the headline)
 
 
@@ -353,23 +354,17 @@ def also_measurements(flush, steps, pk):
                                 "bwd_gbs": (M_ * K_ * (2 + 4 + 4)) / (ms_nb / 1e3) / 1e9}
     device_status_ok("rmsnorm")
     del xr, gr, xn_, rs_, dxn_, dx_
-    # quantized lm_head with chunked cross-entropy: 2048 tokens, hidden 2048, 128K vocabulary, Q8_0
+    # quantized lm_head with chunked cross-entropy: 2048 tokens, hidden 2048, 128K vocabulary, Q8_0, in
+    # chunks of 1024 tokens (512-row pair tiles for the logits GEMM; 0.8 GB of workspace)
     lm = inp.lm_head_q8_0_128k()
-    lw = torch.from_numpy(lm["wq"]).cuda()
-    lx = bf16_dev(lm["X"])
-    llab = torch.from_numpy(lm["labels"]).cuda()
-    lws = torch.empty(ql.qlora_lm_head_ce_workspace_bytes(lm["M"], lm["V"], lm["K"], 256), dtype=torch.uint8,
-                      device="cuda")
-    lloss = torch.empty(lm["M"], dtype=torch.float32, device="cuda")
-    ldx = torch.empty(lm["M"], lm["K"], dtype=torch.bfloat16, device="cuda")
-    ms_l, _ = time_steps(lambda: ql.qlora_lm_head_ce(lm["qtype"], lw, lm["V"], lm["K"], lx, llab, 256, 1.0 / lm["M"],
-                                                   lloss, ldx, lws), max(5, steps // 4), 3, flush)
+    lr_ = LmHeadRun(lm, LM_CHUNK)
+    ms_l, _ = time_steps(lr_.step, max(5, steps // 4), 3, flush)
     lflops = 4.0 * lm["M"] * lm["V"] * lm["K"]
-    out["lm_head_ce_q8_0_2048x2048x131072_chunk256"] = {
+    out[f"lm_head_ce_q8_0_2048x2048x131072_chunk{LM_CHUNK}"] = {
         "ms": ms_l, "tokens_per_s": lm["M"] / (ms_l / 1e3), "tflops": lflops / (ms_l / 1e3) / 1e12,
         "frac_of_bf16_peak": lflops / (ms_l / 1e3) / 1e12 / pk["bf16_tflops"]}
     device_status_ok("lm_head")
-    del lm, lw, lx, llab, lws, lloss, ldx
+    del lm, lr_
     torch.cuda.empty_cache()
     # routing alone at 4096 tokens, 256 experts, top-8 (the skewed workload's logits)
     c = inp.moe_q4_k_256x4096x1536(4096)
@@ -682,7 +677,8 @@ def run_reference(args, rank, world):
 class LmHeadRun:
     """Device buffers and one call of the quantized lm_head with chunked cross-entropy."""
 
-    def __init__(self, lm, chunk=256):
+    def __init__(self, lm, chunk=None):
+        chunk = LM_CHUNK if chunk is None else chunk
         import quantized_base_lora_tma_b200 as ql
         self.ql, self.lm, self.chunk = ql, lm, chunk
         self.w = torch.from_numpy(lm["wq"]).cuda()

@@ -52,25 +52,58 @@ __device__ __forceinline__ uint32_t pack2_bf16(__nv_bfloat16 lo, __nv_bfloat16 h
   return (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
 }
 
+// ---- streamed tiles: 16-byte cp.async copies into a shared-memory ring ----------------------------
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  // src-size 0 fills the 16 bytes with zeros and reads nothing
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
 // Column reductions on tensor cores: part[slice][c][j] = sum_{m in slice} Y[m][c] * Zs[m][j], where
 // Zs = Z * zw (optional per-row weight) is fed as a bf16 hi + lo pair (fp32-accurate).
 // A operand: Zs^T (rows j, k = m); B operand: Y (k = m, n = c) through ldmatrix.trans.
-// Grid (ceil(C/128), slices), 128 threads: warp w owns columns 128*bx + 32w .. +31.
-// Slices as in colred_partial_kernel. JT = ceil(r/16) tiles of 16 rows of j.
+// Grid (ceil(C/128), slices), 128 threads: warp w owns columns 128*bx + 32w .. +31. A slice is one
+// 128-row block of an expert segment (E > 0) or of the rows (E == 0). Its whole 128 x 128 tile of Y
+// (and of Ylo) goes to shared memory in one round of 16-byte asynchronous copies (rows past the
+// segment zero-filled), while the threads stage Zs^T, so a CTA waits for memory once.
+// JT = ceil(r/16) tiles of 16 rows of j.
+constexpr int kCrYS = 128 + 8;  // padded row (bf16): 272 bytes, ldmatrix rows hit distinct banks
+__host__ __device__ constexpr int colred_mma_smem(int JT, bool two) {
+  return (two ? 2 : 1) * 128 * kCrYS * 2 + 2 * JT * 16 * kCrYS * 2;
+}
 template <int JT>
 __global__ void __launch_bounds__(128) colred_mma_kernel(const __nv_bfloat16* __restrict__ Y, long ldy, int Ccols,
                                                          const float* __restrict__ Z, int r, int M,
                                                          const float* __restrict__ zw, const int* __restrict__ seg_off,
                                                          const int* __restrict__ mblk_off, int E,
                                                          float* __restrict__ part,
-                                                         const __nv_bfloat16* __restrict__ Ylo) {
+                                                         const __nv_bfloat16* __restrict__ Ylo,
+                                                         const int32_t* __restrict__ rowmap, int rk) {
+  pdl_wait();  // inputs come from earlier launches in the stream
+  pdl_launch_dependents();
   // Ylo (nullable): a second bf16 term of Y (Y = Y + Ylo to ~2^-16), same layout.
-  constexpr int YS = 128 + 8;  // padded row (bf16): 272 bytes, ldmatrix rows hit distinct banks
-  constexpr int HR = 32;       // rows staged per step
-  __shared__ __align__(16) __nv_bfloat16 ys[HR * YS];
-  __shared__ __align__(16) __nv_bfloat16 ysl[HR * YS];
-  __shared__ __align__(16) __nv_bfloat16 zh[JT * 16][HR + 8];
-  __shared__ __align__(16) __nv_bfloat16 zl[JT * 16][HR + 8];
+  // rowmap (nullable): row m of the slice is row rowmap[m] / rk of Y (a pair's token row read in
+  // place, instead of from a gathered copy).
+  constexpr int YS = kCrYS;
+  extern __shared__ __align__(16) uint8_t crm_smem[];
+  __nv_bfloat16* zh = reinterpret_cast<__nv_bfloat16*>(crm_smem);  // [JT*16][YS]: Zs^T hi
+  __nv_bfloat16* zl = zh + JT * 16 * YS;                           // lo
+  __nv_bfloat16* ys = zl + JT * 16 * YS;                           // [128][YS]
+  __nv_bfloat16* ysl = ys + 128 * YS;                              // [128][YS] (two terms only)
   const int slice = blockIdx.y;
   int lo, hi;
   if (E == 0) {
@@ -87,94 +120,74 @@ __global__ void __launch_bounds__(128) colred_mma_kernel(const __nv_bfloat16* __
     lo = __ldg(seg_off + a) + (slice - __ldg(mblk_off + a)) * 128;
     hi = min(__ldg(seg_off + a + 1), lo + 128);
   }
+  const int n = max(0, hi - lo);
   const int c0 = blockIdx.x * 128;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, c = lane & 3;
   const bool two = Ylo != nullptr;
+  const int kmax = (n + 15) & ~15;  // rows past n are zero in both operands
+  for (int i = tid; i < (kmax << 4); i += 128) {
+    const int m = i >> 4, q = i & 15;
+    const bool in = m < n && c0 + 8 * q < Ccols;
+    const long yrow = rowmap != nullptr ? (long)(in ? __ldg(rowmap + lo + m) / rk : 0) : (long)(lo + m);
+    const long o = in ? yrow * ldy + c0 + 8 * q : 0;
+    cp_async16(smem_u32(ys + m * YS + 8 * q), Y + o, in);
+    if (two) cp_async16(smem_u32(ysl + m * YS + 8 * q), Ylo + o, in);
+  }
+  cp_async_commit();
+  // stage Zs^T as hi / lo bf16 while the copies are in flight
+  for (int i = tid; i < JT * 16 * kmax; i += 128) {
+    const int j = i / kmax, m = i - j * kmax;
+    float z = 0.f;
+    if (m < n && j < r) {
+      z = __ldg(Z + (long)(lo + m) * r + j);
+      if (zw != nullptr) z *= __ldg(zw + lo + m);
+    }
+    const __nv_bfloat16 h = __float2bfloat16_rn(z);
+    zh[j * YS + m] = h;
+    zl[j * YS + m] = __float2bfloat16_rn(z - __bfloat162float(h));
+  }
+  cp_async_wait<0>();
+  __syncthreads();
   float acc[JT][4][4];
 #pragma unroll
   for (int jt = 0; jt < JT; ++jt)
 #pragma unroll
     for (int t = 0; t < 4; ++t) acc[jt][t][0] = acc[jt][t][1] = acc[jt][t][2] = acc[jt][t][3] = 0.f;
   const int wc = warp * 32;  // warp's first column within the CTA tile
-  for (int step = 0; step < 128 / HR; ++step) {
-    const int mb = lo + step * HR;
-    const int n = min(HR, hi - mb);
-    if (n <= 0) break;
-    uint4 yv[HR * 16 / 128], yl[HR * 16 / 128];
+  for (int k = 0; k < kmax; k += 16) {
 #pragma unroll
-    for (int it = 0; it < HR * 16 / 128; ++it) {
-      const int i = threadIdx.x + 128 * it;
-      const int m = i >> 4, q = i & 15;
-      const bool in = m < n && c0 + 8 * q < Ccols;
-      const long o = (long)(mb + m) * ldy + c0 + 8 * q;
-      yv[it] = in ? __ldg(reinterpret_cast<const uint4*>(Y + o)) : make_uint4(0, 0, 0, 0);
-      yl[it] = (in && two) ? __ldg(reinterpret_cast<const uint4*>(Ylo + o)) : make_uint4(0, 0, 0, 0);
-    }
-    __syncthreads();
+    for (int term = 0; term < 2; ++term) {
+      if (term == 1 && !two) break;
+      const __nv_bfloat16* src = term ? ysl : ys;
+      // B fragments for 4 n8 tiles: two ldmatrix.x4.trans, each covering 2 tiles x k16
+      uint32_t b[4][2];
 #pragma unroll
-    for (int it = 0; it < HR * 16 / 128; ++it) {
-      const int i = threadIdx.x + 128 * it;
-      *reinterpret_cast<uint4*>(ys + (i >> 4) * YS + 8 * (i & 15)) = yv[it];
-      *reinterpret_cast<uint4*>(ysl + (i >> 4) * YS + 8 * (i & 15)) = yl[it];
-    }
-    // stage Z^T as hi / lo bf16
-    for (int i = threadIdx.x; i < JT * 16 * HR; i += 128) {
-      const int j = i / HR, m = i % HR;
-      float z = 0.f;
-      if (m < n && j < r) {
-        z = Z[(long)(mb + m) * r + j];
-        if (zw != nullptr) z *= zw[mb + m];
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int mat = lane >> 3, rr = lane & 7;
+        const int krow = k + ((mat & 1) ? 8 : 0) + rr;
+        const int ncol = wc + 16 * h2 + ((mat & 2) ? 8 : 0);
+        ldsm_x4_t(smem_u32(src + krow * YS + ncol), b[2 * h2][0], b[2 * h2][1], b[2 * h2 + 1][0], b[2 * h2 + 1][1]);
       }
-      const __nv_bfloat16 h = __float2bfloat16_rn(z);
-      zh[j][m] = h;
-      zl[j][m] = __float2bfloat16_rn(z - __bfloat162float(h));
-    }
-    __syncthreads();
 #pragma unroll
-    for (int k = 0; k < HR; k += 16) {
+      for (int jt = 0; jt < JT; ++jt) {
+        const int j0 = 16 * jt;
+        const uint32_t ah0 = *reinterpret_cast<const uint32_t*>(zh + (j0 + g) * YS + k + 2 * c);
+        const uint32_t ah1 = *reinterpret_cast<const uint32_t*>(zh + (j0 + g + 8) * YS + k + 2 * c);
+        const uint32_t ah2 = *reinterpret_cast<const uint32_t*>(zh + (j0 + g) * YS + k + 2 * c + 8);
+        const uint32_t ah3 = *reinterpret_cast<const uint32_t*>(zh + (j0 + g + 8) * YS + k + 2 * c + 8);
 #pragma unroll
-      for (int term = 0; term < 2; ++term) {
-        if (term == 1 && !two) break;
-        const __nv_bfloat16* src = term ? ysl : ys;
-        // B fragments for 4 n8 tiles: two ldmatrix.x4.trans, each covering 2 tiles x k16
-        uint32_t b[4][2];
+        for (int t = 0; t < 4; ++t) mma_16816(acc[jt][t], ah0, ah1, ah2, ah3, b[t][0], b[t][1]);
+        if (term == 0) {  // Z_lo * Y (Z_lo * Y_lo is below fp32 resolution)
+          const uint32_t al0 = *reinterpret_cast<const uint32_t*>(zl + (j0 + g) * YS + k + 2 * c);
+          const uint32_t al1 = *reinterpret_cast<const uint32_t*>(zl + (j0 + g + 8) * YS + k + 2 * c);
+          const uint32_t al2 = *reinterpret_cast<const uint32_t*>(zl + (j0 + g) * YS + k + 2 * c + 8);
+          const uint32_t al3 = *reinterpret_cast<const uint32_t*>(zl + (j0 + g + 8) * YS + k + 2 * c + 8);
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          const int mat = lane >> 3, rr = lane & 7;
-          const int krow = k + ((mat & 1) ? 8 : 0) + rr;
-          const int ncol = wc + 16 * h2 + ((mat & 2) ? 8 : 0);
-          const uint32_t addr = smem_u32(src + krow * YS + ncol);
-          uint32_t x0, x1, x2, x3;
-          asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                       : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3)
-                       : "r"(addr));
-          b[2 * h2][0] = x0;
-          b[2 * h2][1] = x1;
-          b[2 * h2 + 1][0] = x2;
-          b[2 * h2 + 1][1] = x3;
-        }
-#pragma unroll
-        for (int jt = 0; jt < JT; ++jt) {
-          const int j0 = 16 * jt;
-          const uint32_t ah0 = *reinterpret_cast<const uint32_t*>(&zh[j0 + g][k + 2 * c]);
-          const uint32_t ah1 = *reinterpret_cast<const uint32_t*>(&zh[j0 + g + 8][k + 2 * c]);
-          const uint32_t ah2 = *reinterpret_cast<const uint32_t*>(&zh[j0 + g][k + 2 * c + 8]);
-          const uint32_t ah3 = *reinterpret_cast<const uint32_t*>(&zh[j0 + g + 8][k + 2 * c + 8]);
-#pragma unroll
-          for (int t = 0; t < 4; ++t) mma_16816(acc[jt][t], ah0, ah1, ah2, ah3, b[t][0], b[t][1]);
-          if (term == 0) {  // Z_lo * Y (Z_lo * Y_lo is below fp32 resolution)
-            const uint32_t al0 = *reinterpret_cast<const uint32_t*>(&zl[j0 + g][k + 2 * c]);
-            const uint32_t al1 = *reinterpret_cast<const uint32_t*>(&zl[j0 + g + 8][k + 2 * c]);
-            const uint32_t al2 = *reinterpret_cast<const uint32_t*>(&zl[j0 + g][k + 2 * c + 8]);
-            const uint32_t al3 = *reinterpret_cast<const uint32_t*>(&zl[j0 + g + 8][k + 2 * c + 8]);
-#pragma unroll
-            for (int t = 0; t < 4; ++t) mma_16816(acc[jt][t], al0, al1, al2, al3, b[t][0], b[t][1]);
-          }
+          for (int t = 0; t < 4; ++t) mma_16816(acc[jt][t], al0, al1, al2, al3, b[t][0], b[t][1]);
         }
       }
     }
-    __syncthreads();
   }
   // acc[jt][t]: rows j = 16jt + g (+8), columns c0 + wc + 8t + 2c (+1)
 #pragma unroll
@@ -249,26 +262,6 @@ __device__ __forceinline__ void lora_bop_share(const BopArgs& bop, int r, int RP
   }
 }
 
-// ---- streamed tiles: 16-byte cp.async copies into a shared-memory ring ----------------------------
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
-  // src-size 0 fills the 16 bytes with zeros and reads nothing
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
 
 // Element (row, col) of a 128-byte-swizzled box of 64 bf16 columns: 16-byte chunk col/8 of row
 // `row` sits at chunk position (col/8) ^ (row % 8).
@@ -811,6 +804,8 @@ __global__ void __launch_bounds__(256) lora_rows_seg_kernel(const __nv_bfloat16*
                                                             const int* __restrict__ mblk_off, int E, int r, float oscale,
                                                             float lscale, float* __restrict__ out,
                                                             __nv_bfloat16* __restrict__ la, int RP) {
+  pdl_wait();  // inputs come from earlier launches in the stream
+  pdl_launch_dependents();
   constexpr int RN = 8 * NT;
   constexpr int SK = 128;
   constexpr int ZS = SK + 8;
@@ -926,6 +921,8 @@ __global__ void __launch_bounds__(256, 2) lora_rows_seg_z_kernel(
     const __nv_bfloat16* __restrict__ Y, long ldy, int Kin, const __nv_bfloat16* __restrict__ Z, long zj, long zk,
     long zes, const int* __restrict__ seg_off, const int* __restrict__ mblk_off, int E, int r, float oscale,
     float lscale, float* __restrict__ out, __nv_bfloat16* __restrict__ la, int RP) {
+  pdl_wait();  // inputs come from earlier launches in the stream
+  pdl_launch_dependents();
   constexpr int RN = 8 * NT;
   constexpr int SK = 128;
   extern __shared__ __align__(16) __nv_bfloat16 zsd[];
@@ -965,17 +962,18 @@ __global__ void __launch_bounds__(256, 2) lora_rows_seg_z_kernel(
   // the first chunk is on its way while the adapter slice is staged
   uint4 xa0[SK / 32], xb0[SK / 32], xa1[SK / 32], xb1[SK / 32];
   load(xa0, xb0, grp * SK);
+  // Only rows j < r of the slice are staged: a row j >= r of the shared tile only feeds accumulator
+  // column j, which is never written out, so its contents do not matter.
   if (zk == 1) {
-    for (int i = tid; i < RN * (Kin / 8); i += 256) {
+    const int n8 = r * (Kin / 8);
+#pragma unroll 4
+    for (int i = tid; i < n8; i += 256) {
       const int j = i / (Kin / 8), q = i - j * (Kin / 8);
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (j < r) v = __ldg(reinterpret_cast<const uint4*>(Ze + (long)j * zj + 8 * q));
-      *reinterpret_cast<uint4*>(zsd + j * ZS + 8 * q) = v;
+      *reinterpret_cast<uint4*>(zsd + j * ZS + 8 * q) = __ldg(reinterpret_cast<const uint4*>(Ze + (long)j * zj + 8 * q));
     }
   } else if (zj == 1 && zk == r && (reinterpret_cast<uintptr_t>(Ze) & 15) == 0) {
     // [Kin][r] contiguous: 16-byte loads, scattered to [j][k]
-    for (int i = tid; i < RN * ZS / 2; i += 256) reinterpret_cast<uint32_t*>(zsd)[i] = 0u;
-    __syncthreads();
+#pragma unroll 4
     for (int i = tid; i < Kin * r / 8; i += 256) {
       const uint4 v = __ldg(reinterpret_cast<const uint4*>(Ze) + i);
       const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&v);
@@ -986,12 +984,13 @@ __global__ void __launch_bounds__(256, 2) lora_rows_seg_z_kernel(
       }
     }
   } else {
-    for (int i = tid; i < Kin * RN; i += 256) {
-      const int kk = i / RN, j = i - kk * RN;
-      zsd[j * ZS + kk] = j < r ? Ze[(long)j * zj + (long)kk * zk] : __float2bfloat16(0.f);
+    for (int i = tid; i < Kin * r; i += 256) {
+      const int kk = i / r, j = i - kk * r;
+      zsd[j * ZS + kk] = Ze[(long)j * zj + (long)kk * zk];
     }
   }
   __syncthreads();
+  const int nt_used = (r + 7) >> 3;  // tiles of 8 adapter columns holding a column j < r
   float acc[NT][4];
 #pragma unroll
   for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
@@ -1002,6 +1001,7 @@ __global__ void __launch_bounds__(256, 2) lora_rows_seg_z_kernel(
       const bool in = k < Kin;
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
+        if (t >= nt_used) break;
         const uint4 zq = in ? *reinterpret_cast<const uint4*>(zsd + (8 * t + g) * ZS + k) : make_uint4(0, 0, 0, 0);
         mma_16816(acc[t], xa[q].x, xb[q].x, xa[q].y, xb[q].y, zq.x, zq.y);
         mma_16816(acc[t], xa[q].z, xb[q].z, xa[q].w, xb[q].w, zq.z, zq.w);
@@ -1082,30 +1082,27 @@ __global__ void __launch_bounds__(256, 2) lora_rows_seg_z_kernel(
 
 // LB[e][n] = [Z_e(n, :) | Z_e(n, :)] zero padded to 2*RP columns; Z_e(n, j) = Z[e*zes + n*zn + j*zjs].
 // blockIdx.y is the expert; an expert whose segment is empty (seg_off given) is skipped, since no
-// GEMM tile reads its rows. One thread per 8 output columns.
+// GEMM tile reads its rows. One thread per row n: its r values are loaded together, then the
+// 2*RP-wide row goes out as 16-byte stores.
 __global__ void lora_bop_vec_kernel(const __nv_bfloat16* __restrict__ Z, long zn, long zjs, long zes, int rows,
                                     const int* __restrict__ seg_off, int r, int RP, __nv_bfloat16* __restrict__ LB) {
+  pdl_wait();  // inputs come from earlier launches in the stream
+  pdl_launch_dependents();
   const int e = blockIdx.y;
   if (seg_off != nullptr && __ldg(seg_off + e) == __ldg(seg_off + e + 1)) return;
-  // 32-bit index arithmetic within an expert (the host keeps rows * 2RP / 8 below 2^31)
-  const int per_row = 2 * RP / 8;
-  const int items = rows * per_row;
   const __nv_bfloat16* Ze = Z + (long)e * zes;
   __nv_bfloat16* LBe = LB + (long)e * rows * 2 * RP;
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < items; i += gridDim.x * blockDim.x) {
-    const int n = i / per_row;
-    const int j0 = (i - n * per_row) * 8;
-    const int jb = j0 % RP;  // first rank column of the chunk (both halves repeat Z)
-    __nv_bfloat16 v[8];
-    if (jb < r) {
-      const __nv_bfloat16* zp = Ze + (long)n * zn;
+  for (int n = blockIdx.x * blockDim.x + threadIdx.x; n < rows; n += gridDim.x * blockDim.x) {
+    const __nv_bfloat16* zp = Ze + (long)n * zn;
+    uint4* out = reinterpret_cast<uint4*>(LBe + (long)n * 2 * RP);
+    for (int j0 = 0; j0 < RP; j0 += 8) {  // 8 rank columns at a time, written to both halves
+      __nv_bfloat16 v[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) v[q] = jb + q < r ? zp[(long)(jb + q) * zjs] : __float2bfloat16(0.f);
-    } else {
-#pragma unroll
-      for (int q = 0; q < 8; ++q) v[q] = __float2bfloat16(0.f);
+      for (int q = 0; q < 8; ++q) v[q] = j0 + q < r ? zp[(long)(j0 + q) * zjs] : __float2bfloat16(0.f);
+      const uint4 w = *reinterpret_cast<const uint4*>(v);
+      out[j0 / 8] = w;
+      out[(RP + j0) / 8] = w;
     }
-    *reinterpret_cast<uint4*>(LBe + (long)n * 2 * RP + j0) = *reinterpret_cast<const uint4*>(v);
   }
 }
 
@@ -1115,6 +1112,8 @@ __global__ void lora_bop_vec_kernel(const __nv_bfloat16* __restrict__ Z, long zn
 __global__ void colred_reduce_kernel(const float* __restrict__ part, int Ccols, int r, int nslices_dense,
                                      const int* __restrict__ mblk_off, int E, float scale, int transpose,
                                      float* __restrict__ out) {
+  pdl_wait();  // inputs come from earlier launches in the stream
+  pdl_launch_dependents();
   const int e = blockIdx.y;
   const int per_e = Ccols * r;
   int s0, s1;

@@ -31,6 +31,8 @@ __global__ void __launch_bounds__(1024) moe_route_select_kernel(const __nv_bfloa
                                                                 int E, int k, int32_t* __restrict__ topk_idx,
                                                                 float* __restrict__ topk_w,
                                                                 int32_t* __restrict__ hist) {
+  pdl_wait();  // inputs come from earlier launches in the stream
+  pdl_launch_dependents();
   __shared__ int s_hist[kMaxExperts];
   __shared__ uint8_t s_sel[kRouteRow][kMaxTopK];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -102,6 +104,8 @@ __global__ void __launch_bounds__(kMaxExperts) moe_route_scan_kernel(int32_t* __
                                                                      int32_t* __restrict__ counts,
                                                                      int32_t* __restrict__ offsets,
                                                                      int32_t* __restrict__ mblk) {
+  pdl_wait();  // inputs come from earlier launches in the stream
+  pdl_launch_dependents();
   __shared__ int s_scan[kMaxExperts / 32 * 2];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int tot = 0;
@@ -148,6 +152,8 @@ __global__ void __launch_bounds__(kMaxExperts) moe_route_scan_kernel(int32_t* __
 __global__ void __launch_bounds__(256) moe_route_place_kernel(
     const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ hist, const int32_t* __restrict__ offsets,
     int T, int E, int k, int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm) {
+  pdl_wait();  // inputs come from earlier launches in the stream
+  pdl_launch_dependents();
   __shared__ uint32_t s_bits[8][kMaxExperts];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int row = blockIdx.x * 8 + warp;
@@ -176,6 +182,8 @@ __global__ void __launch_bounds__(256) moe_route_place_kernel(
 __global__ void moe_gather_rows_kernel(const __nv_bfloat16* __restrict__ src, int cols, const int32_t* __restrict__ perm,
                                        int P, int k, __nv_bfloat16* __restrict__ dst, const float* __restrict__ topk_w,
                                        float* __restrict__ row_w) {
+  pdl_wait();  // inputs come from earlier launches in the stream
+  pdl_launch_dependents();
   const int vec = cols / 8;
   const long total = (long)P * vec;
   for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total; i += (long)gridDim.x * blockDim.x) {
@@ -191,6 +199,8 @@ __global__ void moe_gather_rows_kernel(const __nv_bfloat16* __restrict__ src, in
 // slot order).
 __global__ void moe_combine_kernel(const float* __restrict__ rows, int cols, const int32_t* __restrict__ inv_perm,
                                    int T, int k, void* __restrict__ out, int out_dtype) {
+  pdl_wait();  // inputs come from earlier launches in the stream
+  pdl_launch_dependents();
   const int vec = cols / 4;
   const long total = (long)T * vec;
   for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total; i += (long)gridDim.x * blockDim.x) {
@@ -223,24 +233,29 @@ __global__ void moe_combine_kernel(const float* __restrict__ rows, int cols, con
 __global__ void moe_dw_dlogits_kernel(const float* __restrict__ dw_part, int ntiles, const int32_t* __restrict__ inv_perm,
                                       const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_w, int T, int E,
                                       int k, float* __restrict__ dw_pair_out, float* __restrict__ d_logits) {
-  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  pdl_wait();  // inputs come from earlier launches in the stream
+  pdl_launch_dependents();
+  // one warp per token: lane j < k takes slot j (its tile partials summed in tile order), the
+  // weighted sum over slots is a fixed butterfly, and the lanes write the token's logit row
+  const int t = (int)((blockIdx.x * (long)blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
   if (t >= T) return;
-  float dw[kMaxTopK];
-  float s = 0.f;
-  for (int j = 0; j < k; ++j) {
-    const int p = inv_perm[(long)t * k + j];
-    float a = 0.f;
+  float a = 0.f, w = 0.f;
+  int sel = 0;
+  if (lane < k) {
+    const int p = inv_perm[(long)t * k + lane];
     for (int q = 0; q < ntiles; ++q) a += dw_part[(long)p * ntiles + q];
-    dw[j] = a;
-    if (dw_pair_out) dw_pair_out[(long)t * k + j] = a;
-    s += topk_w[(long)t * k + j] * a;
+    w = topk_w[(long)t * k + lane];
+    sel = topk_idx[(long)t * k + lane];
+    if (dw_pair_out) dw_pair_out[(long)t * k + lane] = a;
   }
+  float s = w * a;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   if (d_logits != nullptr) {
-    for (int e = 0; e < E; ++e) d_logits[(long)t * E + e] = 0.f;
-    for (int j = 0; j < k; ++j) {
-      const float w = topk_w[(long)t * k + j];
-      d_logits[(long)t * E + topk_idx[(long)t * k + j]] = w * (dw[j] - s);
-    }
+    for (int e = lane; e < E; e += 32) d_logits[(long)t * E + e] = 0.f;
+    __syncwarp();  // the zeros are ordered before the selected entries
+    if (lane < k) d_logits[(long)t * E + sel] = w * (a - s);
   }
 }
 

@@ -115,25 +115,33 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 }
 
 // Wait until the phase with the given parity has completed. Returns false (after recording a
-// timeout) if it has not within limit_ns, or at once if another wait already gave up. With
+// timeout) if it has not within limit_ns, or soon after another wait gave up. With
 // honour_abort = false it ignores other waits' failures (used to drain copies in flight).
 // Between polls the thread sleeps in the barrier (suspend hint of 0.2 ms) rather than spinning,
-// so waiting warps leave issue slots (and power) to the warps doing the work. Giving up needs
-// both the time limit and a floor of polls, so that a jump of the global timer alone can never
-// end a wait that is still making progress.
+// so waiting warps leave issue slots (and power) to the warps doing the work. A sleeping try_wait
+// may return early without the phase having completed, so the device status word (a global load,
+// an L2 round trip) and the time limit are checked only once per kAbortCheckNs of waiting: a load
+// in flight when the phase completes would delay the waiter by that round trip. Giving up needs
+// both the time limit and a floor of polls, so that a jump of the global timer alone can never end
+// a wait that is still making progress.
 constexpr uint32_t kSleepHintNs = 200000u;
+constexpr uint64_t kAbortCheckNs = 20000u;
 template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int site,
                                           bool honour_abort = true, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait<CLUSTER>(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   const uint32_t hint = limit_ns < 4ull * kSleepHintNs ? (uint32_t)(limit_ns / 4) : kSleepHintNs;
+  uint64_t next_check = t0 + kAbortCheckNs;
   uint32_t polls = 0;
   while (true) {
     if (mbar_try_wait_sleep<CLUSTER>(bar, parity, hint)) return true;
     ++polls;
+    const uint64_t now = globaltimer_ns();
+    if (now < next_check) continue;
+    next_check = now + kAbortCheckNs;
     if (honour_abort && dev_aborted()) return false;
-    if (polls >= 16u && globaltimer_ns() - t0 > limit_ns) {
+    if (polls >= 16u && now - t0 > limit_ns) {
       if (honour_abort) dev_fail(QL_ERR_TIMEOUT, site);
       return false;
     }
@@ -274,6 +282,10 @@ __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int x
   asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(map)),
                "r"(x), "r"(y)
                : "memory");
+}
+// Ask L2 for the line holding p (no register result, no wait).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
 }
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -201,7 +201,11 @@ __device__ __forceinline__ void split_bf16x8(const float (&f)[8], uint4& hi, uin
   lo = pack_bf16x8(l);
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
+// sigma(g) = 1 / (1 + e^-g) from the fast exponential and a fast reciprocal: relative error of order
+// 1e-6 for the gate values that occur, far below the bf16 resolution of what the epilogues store;
+// e^-g = inf (g < -88) gives 0 and e^-g = 0 gives 1.
+__device__ __forceinline__ float sigmoid_fast(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
+__device__ __forceinline__ float silu_f(float g) { return g * sigmoid_fast(g); }
 
 // Epilogue of one accumulator row block: this thread owns output row `row` (valid or not: the
 // TMEM loads are warp-collective) and reads BN fp32 columns starting at TMEM address tbase.
@@ -281,8 +285,21 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, const TileInf
     __nv_bfloat16* __restrict__ gl = p.out_lo;
     float wr = 0.0f, dwp = 0.0f;
     if (valid) wr = __ldg(p.row_w + row);
+    // the g and u of a batch are asked of L2 kPf batches ahead, so each batch's loads find them
+    // there instead of waiting a full memory latency (64 bytes of each per batch and row)
+    constexpr int kPf = 3;
+    auto prefetch_batch = [&](int jc) {
+      const int j0 = ti.nb * BN + 16 * jc;
+      if (valid && jc < BN / 16 && j0 < p.I) {
+        prefetch_l2(gin + (long)row * p.I + j0);
+        prefetch_l2(uin + (long)row * p.I + j0);
+      }
+    };
+#pragma unroll
+    for (int jc = 0; jc < kPf; ++jc) prefetch_batch(jc);
 #pragma unroll 1
     for (int jc = 0; jc < BN / 16; ++jc) {
+      prefetch_batch(jc + kPf);
       uint32_t v[16];
       tmem_ld16(tbase + 16 * jc, v);
       const int j0 = ti.nb * BN + 16 * jc;
@@ -309,12 +326,13 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, const TileInf
           for (int j = 0; j < 8; ++j) {
             const float a = __uint_as_float(v[8 * hlf + j]);
             const float g = gf[8 * hlf + j], u = uf[8 * hlf + j];
-            const float sg = 1.0f / (1.0f + expf(-g));
+            const float sg = sigmoid_fast(g);
             const float dh = wr * a;
+            const float sl = g * sg;  // silu(g)
             dg[j] = dh * u * sg * (1.0f + g * (1.0f - sg));
-            du[j] = dh * g * sg;
+            du[j] = dh * sl;
             // <dh_u, h> with h at fp32 accuracy: a flip of a bf16 h would move a heavy-tailed term
-            dwp = fmaf(a, silu_f(g) * u, dwp);
+            dwp = fmaf(a, sl * u, dwp);
           }
           uint4 gh, glo, uh, ulo;
           split_bf16x8(dg, gh, glo);

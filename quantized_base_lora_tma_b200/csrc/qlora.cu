@@ -208,6 +208,14 @@ struct PdlLaunch {
     cfg.numAttrs = n;
   }
 };
+// A launch that may start while the previous kernel in the stream finishes (the kernel itself
+// waits for it with griddepcontrol.wait before touching memory).
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+  PdlLaunch L(grid, block, smem, st);
+  return cudaLaunchKernelEx(&L.cfg, kern, static_cast<KArgs>(args)...);
+}
 static int launch_result(cudaError_t e) {
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (e != cudaSuccess) {
@@ -523,20 +531,38 @@ static int launch_colred_dense(const __nv_bfloat16* Y0, int C0, const __nv_bfloa
 
 static int launch_colred(const __nv_bfloat16* Y, long ldy, int Ccols, const float* Z, int r, int M, const float* zw,
                          const int* seg_off, const int* mblk_off, int E, int max_slices, float* part, float scale,
-                         int transpose, float* out, cudaStream_t st, const __nv_bfloat16* Ylo = nullptr) {
+                         int transpose, float* out, cudaStream_t st, const __nv_bfloat16* Ylo = nullptr,
+                         const int32_t* rowmap = nullptr, int rk = 1) {
   if (max_slices <= 0) return QL_OK;
   dim3 grid((Ccols + 127) / 128, max_slices);
   const int JT = (r + 15) / 16;
-  if (JT == 1) colred_mma_kernel<1><<<grid, 128, 0, st>>>(Y, ldy, Ccols, Z, r, M, zw, seg_off, mblk_off, E, part, Ylo);
-  else if (JT == 2) colred_mma_kernel<2><<<grid, 128, 0, st>>>(Y, ldy, Ccols, Z, r, M, zw, seg_off, mblk_off, E, part, Ylo);
-  else if (JT == 3) colred_mma_kernel<3><<<grid, 128, 0, st>>>(Y, ldy, Ccols, Z, r, M, zw, seg_off, mblk_off, E, part, Ylo);
-  else colred_mma_kernel<4><<<grid, 128, 0, st>>>(Y, ldy, Ccols, Z, r, M, zw, seg_off, mblk_off, E, part, Ylo);
+  const size_t sm = colred_mma_smem(JT, Ylo != nullptr);
+  cudaError_t e;
+  if (JT == 1) {
+    e = set_smem(colred_mma_kernel<1>, (int)sm);
+    if (e == cudaSuccess) e = launch_pdl(colred_mma_kernel<1>, grid, 128, sm, st, Y, ldy, Ccols, Z, r, M, zw, seg_off, mblk_off, E, part, Ylo, rowmap, rk);
+  } else if (JT == 2) {
+    e = set_smem(colred_mma_kernel<2>, (int)sm);
+    if (e == cudaSuccess) e = launch_pdl(colred_mma_kernel<2>, grid, 128, sm, st, Y, ldy, Ccols, Z, r, M, zw, seg_off, mblk_off, E, part, Ylo, rowmap, rk);
+  } else if (JT == 3) {
+    e = set_smem(colred_mma_kernel<3>, (int)sm);
+    if (e == cudaSuccess) e = launch_pdl(colred_mma_kernel<3>, grid, 128, sm, st, Y, ldy, Ccols, Z, r, M, zw, seg_off, mblk_off, E, part, Ylo, rowmap, rk);
+  } else {
+    e = set_smem(colred_mma_kernel<4>, (int)sm);
+    if (e == cudaSuccess) e = launch_pdl(colred_mma_kernel<4>, grid, 128, sm, st, Y, ldy, Ccols, Z, r, M, zw, seg_off, mblk_off, E, part, Ylo, rowmap, rk);
+  }
   g_launches.fetch_add(1, std::memory_order_relaxed);
-  if (launch_status() != QL_OK) return QL_ERR_CUDA;
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
   const long per_e = (long)Ccols * r;
   if (per_e >= (1L << 31) || per_e % 4 != 0) return QL_ERR_SHAPE;
-  const dim3 g2((unsigned)std::min<long>((per_e + 255) / 256, 64L), E == 0 ? 1 : E);
-  colred_reduce_kernel<<<g2, 256, 0, st>>>(part, Ccols, r, max_slices, mblk_off, E, scale, transpose, out);
+  // per expert a few CTAs of 256 threads (about eight outputs per thread): most experts of a
+  // skewed batch are empty, and their CTAs only store zeros
+  const long per_cta = E == 0 ? 256 : 2048;
+  const dim3 g2((unsigned)std::min<long>((per_e + per_cta - 1) / per_cta, 64L), E == 0 ? 1 : E);
+  launch_pdl(colred_reduce_kernel, g2, 256, 0, st, part, Ccols, r, max_slices, mblk_off, E, scale, transpose, out);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return launch_status();
 }
@@ -981,17 +1007,17 @@ static int launch_rows_seg(const __nv_bfloat16* Y, long ldy, int Kin, const __nv
     if (NT == 2) {
       e = set_smem(lora_rows_seg_z_kernel<2>, (int)zsm);
       if (e == cudaSuccess)
-        lora_rows_seg_z_kernel<2><<<max_slices, 256, zsm, st>>>(Y, ldy, Kin, Z, zj, zk, zes, seg_off, mblk, E, r, oscale,
+        launch_pdl(lora_rows_seg_z_kernel<2>, max_slices, 256, zsm, st, Y, ldy, Kin, Z, zj, zk, zes, seg_off, mblk, E, r, oscale,
                                                                 lscale, out, la, RP);
     } else if (NT == 4) {
       e = set_smem(lora_rows_seg_z_kernel<4>, (int)zsm);
       if (e == cudaSuccess)
-        lora_rows_seg_z_kernel<4><<<max_slices, 256, zsm, st>>>(Y, ldy, Kin, Z, zj, zk, zes, seg_off, mblk, E, r, oscale,
+        launch_pdl(lora_rows_seg_z_kernel<4>, max_slices, 256, zsm, st, Y, ldy, Kin, Z, zj, zk, zes, seg_off, mblk, E, r, oscale,
                                                                 lscale, out, la, RP);
     } else {
       e = set_smem(lora_rows_seg_z_kernel<8>, (int)zsm);
       if (e == cudaSuccess)
-        lora_rows_seg_z_kernel<8><<<max_slices, 256, zsm, st>>>(Y, ldy, Kin, Z, zj, zk, zes, seg_off, mblk, E, r, oscale,
+        launch_pdl(lora_rows_seg_z_kernel<8>, max_slices, 256, zsm, st, Y, ldy, Kin, Z, zj, zk, zes, seg_off, mblk, E, r, oscale,
                                                                 lscale, out, la, RP);
     }
     g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -999,13 +1025,13 @@ static int launch_rows_seg(const __nv_bfloat16* Y, long ldy, int Kin, const __nv
     return launch_status();
   }
   if (r <= 16)
-    lora_rows_seg_kernel<2><<<max_slices, 256, 0, st>>>(Y, ldy, Kin, Z, zj, zk, zes, seg_off, mblk, E, r, oscale, lscale,
+    launch_pdl(lora_rows_seg_kernel<2>, max_slices, 256, 0, st, Y, ldy, Kin, Z, zj, zk, zes, seg_off, mblk, E, r, oscale, lscale,
                                                         out, la, RP);
   else if (r <= 32)
-    lora_rows_seg_kernel<4><<<max_slices, 256, 0, st>>>(Y, ldy, Kin, Z, zj, zk, zes, seg_off, mblk, E, r, oscale, lscale,
+    launch_pdl(lora_rows_seg_kernel<4>, max_slices, 256, 0, st, Y, ldy, Kin, Z, zj, zk, zes, seg_off, mblk, E, r, oscale, lscale,
                                                         out, la, RP);
   else
-    lora_rows_seg_kernel<8><<<max_slices, 256, 0, st>>>(Y, ldy, Kin, Z, zj, zk, zes, seg_off, mblk, E, r, oscale, lscale,
+    launch_pdl(lora_rows_seg_kernel<8>, max_slices, 256, 0, st, Y, ldy, Kin, Z, zj, zk, zes, seg_off, mblk, E, r, oscale, lscale,
                                                         out, la, RP);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return launch_status();
@@ -1014,12 +1040,9 @@ static int launch_rows_seg(const __nv_bfloat16* Y, long ldy, int Kin, const __nv
 static int launch_bop_vec(const __nv_bfloat16* Z, long zn, long zjs, long zes, int rows, int nexp, int r,
                           __nv_bfloat16* LB, cudaStream_t st, const int* seg_off = nullptr) {
   const int RP = lora_rp(r);
-  const long items = (long)rows * (2 * RP / 8);
-  if (items >= (1L << 31)) return QL_ERR_SHAPE;
-  // per expert about one CTA per 1024 items, at most one wave over all experts' CTAs
-  const long per_e = std::max(1L, std::min((items + 1023) / 1024, (long)num_sms() * 8 / nexp + 1));
-  const dim3 grid((unsigned)std::min(per_e, (items + 255) / 256), nexp);
-  lora_bop_vec_kernel<<<grid, 256, 0, st>>>(Z, zn, zjs, zes, rows, seg_off, r, RP, LB);
+  // one thread per row of an expert
+  const dim3 grid((unsigned)((rows + 255) / 256), nexp);
+  launch_pdl(lora_bop_vec_kernel, grid, 256, 0, st, Z, zn, zjs, zes, rows, seg_off, r, RP, LB);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return launch_status();
 }
@@ -1028,7 +1051,7 @@ static int launch_gather(const __nv_bfloat16* src, int cols, const int32_t* perm
                          const float* topk_w, float* row_w, cudaStream_t st) {
   const long total = (long)P * (cols / 8);
   const int grid = (int)std::min<long>((total + 255) / 256, (long)num_sms() * 16);
-  moe_gather_rows_kernel<<<grid, 256, 0, st>>>(src, cols, perm, P, k, dst, topk_w, row_w);
+  launch_pdl(moe_gather_rows_kernel, grid, 256, 0, st, src, cols, perm, P, k, dst, topk_w, row_w);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return launch_status();
 }
@@ -1037,7 +1060,7 @@ static int launch_combine(const float* rows, int cols, const int32_t* inv_perm, 
                           int out_dtype, cudaStream_t st) {
   const long total = (long)T * (cols / 4);
   const int grid = (int)std::min<long>((total + 255) / 256, (long)num_sms() * 16);
-  moe_combine_kernel<<<grid, 256, 0, st>>>(rows, cols, inv_perm, T, k, out, out_dtype);
+  launch_pdl(moe_combine_kernel, grid, 256, 0, st, rows, cols, inv_perm, T, k, out, out_dtype);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return launch_status();
 }
@@ -1200,14 +1223,14 @@ int qlora_moe_route(const void* logits, int64_t T, int E, int k, int32_t* topk_i
   cudaStream_t st = (cudaStream_t)stream;
   const int nrow = (int)((T + kRouteRow - 1) / kRouteRow);
   int32_t* hist = (int32_t*)ws;
-  moe_route_select_kernel<<<nrow, 32 * kRouteRow, 0, st>>>((const __nv_bfloat16*)logits, (int)T, E, k, topk_idx,
+  launch_pdl(moe_route_select_kernel, nrow, 32 * kRouteRow, 0, st, (const __nv_bfloat16*)logits, (int)T, E, k, topk_idx,
                                                            topk_w, hist);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (launch_status() != QL_OK) return QL_ERR_CUDA;
-  moe_route_scan_kernel<<<1, kMaxExperts, 0, st>>>(hist, E, nrow, counts, offsets, mblk);
+  launch_pdl(moe_route_scan_kernel, 1, kMaxExperts, 0, st, hist, E, nrow, counts, offsets, mblk);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (launch_status() != QL_OK) return QL_ERR_CUDA;
-  moe_route_place_kernel<<<(nrow + 7) / 8, 256, 0, st>>>(topk_idx, hist, offsets, (int)T, E, k, perm, inv_perm);
+  launch_pdl(moe_route_place_kernel, (nrow + 7) / 8, 256, 0, st, topk_idx, hist, offsets, (int)T, E, k, perm, inv_perm);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return launch_status();
 }
@@ -1333,7 +1356,6 @@ int qlora_moe_bwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
   const int ms = moe_max_slices(P, E);
   uint8_t* wb = (uint8_t*)ws;
   const uint8_t* sb = (const uint8_t*)saved;
-  __nv_bfloat16* Xp = (__nv_bfloat16*)(wb + w.xp);
   __nv_bfloat16* dYp = (__nv_bfloat16*)(wb + w.yp);
   float* row_w = (float*)(wb + w.row_w);
   __nv_bfloat16* LA = (__nv_bfloat16*)(wb + w.la);
@@ -1354,9 +1376,8 @@ int qlora_moe_bwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
   const int* off = offsets;
   const int nsm = num_sms();
 
-  rc = launch_gather((const __nv_bfloat16*)X, (int)H, perm, P, k, Xp, topk_w, row_w, st);
-  if (rc) return rc;
-  rc = launch_gather((const __nv_bfloat16*)dY, (int)H, perm, P, k, dYp, nullptr, nullptr, st);
+  // dY in pair order (and each pair's routing weight); X is read in place by its one consumer
+  rc = launch_gather((const __nv_bfloat16*)dY, (int)H, perm, P, k, dYp, topk_w, row_w, st);
   if (rc) return rc;
   int dw_tiles = 0;  // output-column tiles of the down input-gradient GEMM (dw partials per row)
   // down input-gradient: Gd = s dYp B_d, LA = split(Gd), LB[e][i] = [A_d^T | A_d^T]
@@ -1410,13 +1431,15 @@ int qlora_moe_bwd(int qtype, const void* w_gu, const void* w_d, int E, int64_t H
   }
   rc = launch_combine(dxp, (int)H, inv_perm, (int)T, k, dX, dx_dtype, st);
   if (rc) return rc;
-  // gate/up adapter gradients: dA_gu = sum_p Ggu_p^T Xp_p ; dB_gu = s sum_p dgu_p^T Hgu_p
-  rc = launch_colred(Xp, H, (int)H, Ggu, r, P, nullptr, off, mblk, E, ms, part, 1.0f, 1, dA_gu, st);
+  // gate/up adapter gradients: dA_gu = sum_p Ggu_p^T x_p (x_p = X row perm[p] / k, read in place);
+  // dB_gu = s sum_p dgu_p^T Hgu_p
+  rc = launch_colred((const __nv_bfloat16*)X, H, (int)H, Ggu, r, P, nullptr, off, mblk, E, ms, part, 1.0f, 1, dA_gu, st,
+                     nullptr, perm, k);
   if (rc) return rc;
   rc = launch_colred(dgu, 2 * I, (int)(2 * I), Hgu, r, P, nullptr, off, mblk, E, ms, part, scale, 0, dB_gu, st, dgu_lo);
   if (rc) return rc;
   if (d_logits != nullptr) {
-    moe_dw_dlogits_kernel<<<(int)((T + 127) / 128), 128, 0, st>>>(dwp, dw_tiles, inv_perm, topk_idx, topk_w,
+    launch_pdl(moe_dw_dlogits_kernel, (int)((T + 7) / 8), 256, 0, st, dwp, dw_tiles, inv_perm, topk_idx, topk_w,
                                                                   (int)T, E, k, nullptr, d_logits);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return launch_status();
@@ -1704,8 +1727,8 @@ extern "C" int qlora_lm_head_ce(int qtype, const void* wq, int64_t V, int64_t K,
     // the CE kernel and the input-gradient GEMM each read what the launch right before them wrote:
     // they start only once it has completed
     NoEarlyStart serial;
-    lm_ce_kernel<<<(unsigned)rows, kCeThreads, 0, st>>>(logits, (int)V, labels + c0, grad_scale, loss + c0,
-                                                        dX ? dlog : nullptr);
+    lm_ce_kernel<<<(unsigned)std::min<int64_t>(rows, num_sms()), kCeThreads, 0, st>>>(
+        logits, (int)V, (int)rows, labels + c0, grad_scale, loss + c0, dX ? dlog : nullptr);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     if (launch_status() != QL_OK) return QL_ERR_CUDA;
     if (dX) {
