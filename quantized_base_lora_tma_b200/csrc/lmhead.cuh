@@ -4,8 +4,10 @@
 // exponentials over the row (float4 loads), lse = max + log(sum), loss = lse - logit[label]; then, if
 // asked, the gradient of the summed loss times grad_scale, (softmax - onehot(label)) * grad_scale, in
 // bf16 for the input-gradient GEMM. A negative label marks an ignored token: loss 0 and a zero
-// gradient row. One CTA per SM keeps the rows in flight (one per SM, 4 bytes x V each) well inside
-// L2, so the second pass over a row reads it from L2 rather than from DRAM.
+// gradient row. Given the logits GEMM's per-tile row statistics (max, sum exp per 256 columns),
+// the first pass is a merge of those and the logits are read once. Otherwise, one CTA per SM
+// keeps the rows in flight (one per SM, 4 bytes x V each) well inside L2, so the second pass over
+// a row reads it from L2 rather than from DRAM.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -22,6 +24,7 @@ __device__ __forceinline__ void ce_merge(float& m, float& s, float m2, float s2)
 }
 
 __global__ void __launch_bounds__(kCeThreads, 1) lm_ce_kernel(const float* __restrict__ logits, int V, int rows,
+                                                              const float2* __restrict__ stats, int ntiles,
                                                               const int32_t* __restrict__ labels, float grad_scale,
                                                               float* __restrict__ loss,
                                                               __nv_bfloat16* __restrict__ dlog) {
@@ -31,8 +34,16 @@ __global__ void __launch_bounds__(kCeThreads, 1) lm_ce_kernel(const float* __res
     const float4* l4 = reinterpret_cast<const float4*>(logits + (long)row * V);
     const int lab = labels[row];
     float m = -INFINITY, s = 0.f;
+    // with stats: the row's (max, sum exp) per column tile, merged in tile order per thread and
+    // then across lanes and warps in a fixed order; without: one pass over the row
+    if (stats != nullptr) {
+      for (int i = tid; i < ntiles; i += kCeThreads) {
+        const float2 t = __ldg(stats + (long)row * ntiles + i);
+        ce_merge(m, s, t.x, t.y);
+      }
+    }
     // kCeUnroll independent 16-byte loads per thread in flight before any is used
-    for (int c0 = tid; c0 < V / 4; c0 += kCeUnroll * kCeThreads) {
+    for (int c0 = tid; stats == nullptr && c0 < V / 4; c0 += kCeUnroll * kCeThreads) {
       float4 xv[kCeUnroll];
 #pragma unroll
       for (int u = 0; u < kCeUnroll; ++u) {

@@ -95,6 +95,8 @@ struct GemmParams {
   const float* in_uf;
   const float* row_w;          // PAIR_OUT, SWIGLU_BWD: routing weight per row
   float* dw_part;              // SWIGLU_BWD: [M x num_n_tiles] partial <dh_u, h>
+  float2* row_stats;           // pair GEMM, fp32 output without K split (nullable): per row and
+                               // column tile, (max, sum of exp(x - max)) of the tile's outputs
   // dense pair GEMM: clusters [0, rx) compute the adapter row products (0 = none: the LoRA
   // operands are the previous launch's output)
   int rx;
@@ -207,146 +209,227 @@ __device__ __forceinline__ void split_bf16x8(const float (&f)[8], uint4& hi, uin
 __device__ __forceinline__ float sigmoid_fast(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
 __device__ __forceinline__ float silu_f(float g) { return g * sigmoid_fast(g); }
 
-// Epilogue of one accumulator row block: this thread owns output row `row` (valid or not: the
-// TMEM loads are warp-collective) and reads BN fp32 columns starting at TMEM address tbase.
+// Store epilogue of the pair GEMM: this thread owns output row `row` (valid or not: the TMEM loads
+// are warp-collective) and reads BN fp32 columns starting at TMEM address tbase; 64 bytes of bf16
+// (or 128 of fp32) of its row per 32 columns.
+template <int BN>
+__device__ __forceinline__ void epilogue_rows_store(const GemmParams& p, const TileInfo& ti, int row, bool valid,
+                                                  uint32_t tbase) {
+  const bool split = p.ksplit > 1;  // fp32 partial of K part ti.ks
+  const bool stats = p.row_stats != nullptr;
+  float sm = -INFINITY, ss = 0.0f;  // the row's running max and sum of exp(x - max) over the tile
+#pragma unroll 1
+  for (int jc = 0; jc < BN / 32; ++jc) {
+    uint32_t v[32];
+    tmem_ld32(tbase + 32 * jc, v);
+    tmem_ld_wait();
+    const int col0 = ti.nb * BN + 32 * jc;
+    if (stats && valid && col0 < p.Nd) {
+      float bm = __uint_as_float(v[0]);
+#pragma unroll
+      for (int i = 1; i < 32; ++i) bm = fmaxf(bm, __uint_as_float(v[i]));
+      const float nm = fmaxf(sm, bm);
+      float acc = sm == -INFINITY ? 0.0f : ss * expf(sm - nm);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) acc += expf(__uint_as_float(v[i]) - nm);
+      sm = nm;
+      ss = acc;
+    }
+    if (valid && col0 < p.Nd) {
+      if (p.out_dtype == QL_F32 || split) {
+        float* base = reinterpret_cast<float*>(p.out) + (split ? ti.ks * p.split_stride : 0);
+        float4* o = reinterpret_cast<float4*>(base + (long)row * p.ldo + col0);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          o[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                             __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+      } else {
+        uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + (long)row * p.ldo + col0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float f[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) f[j] = __uint_as_float(v[8 * i + j]);
+          o[i] = pack_bf16x8(f);
+        }
+      }
+    }
+  }
+  if (stats && valid) p.row_stats[(long)row * p.num_n_tiles + ti.nb] = make_float2(sm, ss);
+}
+
+// SwiGLU-backward epilogue, one accumulator row per thread (32x32b TMEM loads, 16 columns per
+// batch): its outputs are bf16, for which the 16x256b shape gains nothing per byte stored and
+// needs twice the store instructions.
+template <int BN>
+__device__ __forceinline__ void epilogue_rows_swiglu_bwd(const GemmParams& p, const TileInfo& ti, int row, bool valid,
+                                                         uint32_t tbase) {
+  // dh_u = accumulator; dh = w dh_u; the SwiGLU derivative from the saved fp32 g, u; <dh_u, h>
+  // with h = silu(g) u recomputed at fp32 accuracy. The saved g, u are read-only here: 16 columns
+  // of both are loaded together ahead of the arithmetic and stores, one memory latency per batch.
+  const float* __restrict__ gin = p.in_gf;
+  const float* __restrict__ uin = p.in_uf;
+  __nv_bfloat16* __restrict__ go = p.out_g;
+  __nv_bfloat16* __restrict__ gl = p.out_lo;
+  float wr = 0.0f, dwp = 0.0f;
+  if (valid) wr = __ldg(p.row_w + row);
+  // the g and u of a batch are asked of L2 kPf batches ahead, so each batch's loads find them
+  // there instead of waiting a full memory latency (64 bytes of each per batch and row)
+  constexpr int kPf = 3;
+  auto prefetch_batch = [&](int jc) {
+    const int j0 = ti.nb * BN + 16 * jc;
+    if (valid && jc < BN / 16 && j0 < p.I) {
+      prefetch_l2(gin + (long)row * p.I + j0);
+      prefetch_l2(uin + (long)row * p.I + j0);
+    }
+  };
+#pragma unroll
+  for (int jc = 0; jc < kPf; ++jc) prefetch_batch(jc);
+#pragma unroll 1
+  for (int jc = 0; jc < BN / 16; ++jc) {
+    prefetch_batch(jc + kPf);
+    uint32_t v[16];
+    tmem_ld16(tbase + 16 * jc, v);
+    const int j0 = ti.nb * BN + 16 * jc;
+    const bool act = valid && j0 < p.I;
+    float4 gq[4], uq[4];
+    if (act) {
+      const float4* g4 = reinterpret_cast<const float4*>(gin + (long)row * p.I + j0);
+      const float4* u4 = reinterpret_cast<const float4*>(uin + (long)row * p.I + j0);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        gq[q] = __ldg(g4 + q);
+        uq[q] = __ldg(u4 + q);
+      }
+    }
+    tmem_ld_wait();
+    if (act) {
+      const float* gf = reinterpret_cast<const float*>(gq);
+      const float* uf = reinterpret_cast<const float*>(uq);
+      const long od = (long)row * 2 * p.I + j0;
+#pragma unroll
+      for (int hlf = 0; hlf < 2; ++hlf) {
+        float dg[8], du[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float a = __uint_as_float(v[8 * hlf + j]);
+          const float g = gf[8 * hlf + j], u = uf[8 * hlf + j];
+          const float sg = sigmoid_fast(g);
+          const float dh = wr * a;
+          const float sl = g * sg;  // silu(g)
+          dg[j] = dh * u * sg * (1.0f + g * (1.0f - sg));
+          du[j] = dh * sl;
+          // <dh_u, h> with h at fp32 accuracy: a flip of a bf16 h would move a heavy-tailed term
+          dwp = fmaf(a, sl * u, dwp);
+        }
+        uint4 gh, glo, uh, ulo;
+        split_bf16x8(dg, gh, glo);
+        split_bf16x8(du, uh, ulo);
+        *reinterpret_cast<uint4*>(go + od + 8 * hlf) = gh;
+        *reinterpret_cast<uint4*>(go + od + p.I + 8 * hlf) = uh;
+        if (gl != nullptr) {
+          *reinterpret_cast<uint4*>(gl + od + 8 * hlf) = glo;
+          *reinterpret_cast<uint4*>(gl + od + p.I + 8 * hlf) = ulo;
+        }
+      }
+    }
+  }
+  if (valid) p.dw_part[(long)row * p.num_n_tiles + ti.nb] = dwp;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_of(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Epilogue of one warp's 32 accumulator rows (rows rbase .. rbase + 31 of the tile, TMEM address tw
+// at the first of them and the tile's first column). The rows are read as two halves of 16 lanes
+// with the 16x256b shape: a thread holds rows a = rbase + 16 half + lane/4 and b = a + 8, two
+// adjacent columns 2(lane%4), +1 of every group of 8. Four consecutive lanes thus cover 8
+// consecutive columns of a row, so every global access of a warp moves whole 32-byte sectors of
+// 8 rows rather than half sectors of 32 rows.
 template <int EPI, int BN>
-__device__ __forceinline__ void epilogue_rows(const GemmParams& p, const TileInfo& ti, int row, bool valid,
-                                              uint32_t tbase) {
-  if (EPI == EPI_STORE || EPI == EPI_PAIR_OUT) {
-    float wr = 1.0f;
-    if (EPI == EPI_PAIR_OUT && valid) wr = __ldg(p.row_w + row);
-    const bool split = p.ksplit > 1;  // fp32 partial of K part ti.ks
+__device__ __forceinline__ void epilogue_warp(const GemmParams& p, const TileInfo& ti, int rbase, uint32_t tw) {
+  const int lane = threadIdx.x & 31;
+  const int cc = 2 * (lane & 3);
 #pragma unroll 1
-    for (int jc = 0; jc < BN / 32; ++jc) {
-      uint32_t v[32];
-      tmem_ld32(tbase + 32 * jc, v);
-      tmem_ld_wait();
-      const int col0 = ti.nb * BN + 32 * jc;
-      if (valid && col0 < p.Nd) {
-        if (p.out_dtype == QL_F32 || split) {
+  for (int half = 0; half < 2; ++half) {
+    const int ra = rbase + 16 * half + (lane >> 2), rb = ra + 8;
+    const bool va = ra < ti.row_end, vb = rb < ti.row_end;
+    const uint32_t th = tw + ((uint32_t)(16 * half) << 16);
+    if (EPI == EPI_STORE || EPI == EPI_PAIR_OUT) {
+      float wa = 1.0f, wb = 1.0f;
+      if (EPI == EPI_PAIR_OUT) {
+        if (va) wa = __ldg(p.row_w + ra);
+        if (vb) wb = __ldg(p.row_w + rb);
+      }
+      const bool split = p.ksplit > 1;  // fp32 partial of K part ti.ks
+      const bool f32 = p.out_dtype == QL_F32 || split;
+#pragma unroll 1
+      for (int jc = 0; jc < BN / 32; ++jc) {
+        uint32_t v[16];
+        tmem_ld_16x256_x4(th + 32 * jc, v);
+        tmem_ld_wait();
+        const int col0 = ti.nb * BN + 32 * jc;
+        if (col0 >= p.Nd) continue;
+        if (f32) {
           float* base = reinterpret_cast<float*>(p.out) + (split ? ti.ks * p.split_stride : 0);
-          float4* o = reinterpret_cast<float4*>(base + (long)row * p.ldo + col0);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            o[i] = make_float4(wr * __uint_as_float(v[4 * i]), wr * __uint_as_float(v[4 * i + 1]),
-                               wr * __uint_as_float(v[4 * i + 2]), wr * __uint_as_float(v[4 * i + 3]));
+          for (int q = 0; q < 4; ++q) {
+            const int col = col0 + 8 * q + cc;
+            if (va)
+              *reinterpret_cast<float2*>(base + (long)ra * p.ldo + col) =
+                  make_float2(wa * __uint_as_float(v[4 * q]), wa * __uint_as_float(v[4 * q + 1]));
+            if (vb)
+              *reinterpret_cast<float2*>(base + (long)rb * p.ldo + col) =
+                  make_float2(wb * __uint_as_float(v[4 * q + 2]), wb * __uint_as_float(v[4 * q + 3]));
+          }
         } else {
-          uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + (long)row * p.ldo + col0);
+          __nv_bfloat16* base = reinterpret_cast<__nv_bfloat16*>(p.out);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            float f[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) f[j] = wr * __uint_as_float(v[8 * i + j]);
-            o[i] = pack_bf16x8(f);
+          for (int q = 0; q < 4; ++q) {
+            const int col = col0 + 8 * q + cc;
+            if (va)
+              *reinterpret_cast<uint32_t*>(base + (long)ra * p.ldo + col) =
+                  bf16x2_of(wa * __uint_as_float(v[4 * q]), wa * __uint_as_float(v[4 * q + 1]));
+            if (vb)
+              *reinterpret_cast<uint32_t*>(base + (long)rb * p.ldo + col) =
+                  bf16x2_of(wb * __uint_as_float(v[4 * q + 2]), wb * __uint_as_float(v[4 * q + 3]));
           }
         }
       }
-    }
-  } else if (EPI == EPI_SWIGLU) {
-    // tile columns [0, BN/2) are gate j = nb*BN/2 + c, [BN/2, BN) are up for the same j; 16 j at a time
+    } else if (EPI == EPI_SWIGLU) {
+      // tile columns [0, BN/2) are gate j = nb*BN/2 + c, [BN/2, BN) are up for the same j; 32 j at a time
 #pragma unroll 1
-    for (int jp = 0; jp < BN / 32; ++jp) {
-      uint32_t vg[16], vu[16];
-      tmem_ld16(tbase + 16 * jp, vg);
-      tmem_ld16(tbase + BN / 2 + 16 * jp, vu);
-      tmem_ld_wait();
-      const int j0 = ti.nb * (BN / 2) + 16 * jp;
-      if (valid && j0 < p.I) {
-        const long o = (long)row * p.I + j0;
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          float g[8], u[8], h[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            g[j] = __uint_as_float(vg[8 * i + j]);
-            u[j] = __uint_as_float(vu[8 * i + j]);
-            h[j] = silu_f(g[j]) * u[j];
-          }
-          float4* gq = reinterpret_cast<float4*>(p.out_gf + o + 8 * i);
-          float4* uq = reinterpret_cast<float4*>(p.out_uf + o + 8 * i);
-          gq[0] = make_float4(g[0], g[1], g[2], g[3]);
-          gq[1] = make_float4(g[4], g[5], g[6], g[7]);
-          uq[0] = make_float4(u[0], u[1], u[2], u[3]);
-          uq[1] = make_float4(u[4], u[5], u[6], u[7]);
-          uint4 hh, hl;
-          split_bf16x8(h, hh, hl);
-          *reinterpret_cast<uint4*>(p.out_h + o + 8 * i) = hh;
-          if (p.out_lo != nullptr) *reinterpret_cast<uint4*>(p.out_lo + o + 8 * i) = hl;
-        }
-      }
-    }
-  } else if (EPI == EPI_SWIGLU_BWD) {
-    // dh_u = accumulator; dh = w dh_u; the SwiGLU derivative from the saved fp32 g, u; <dh_u, h>
-    // with h = silu(g) u recomputed at fp32 accuracy. The saved g, u are read-only here: 16 columns
-    // of both are loaded together ahead of the arithmetic and stores, one memory latency per batch.
-    const float* __restrict__ gin = p.in_gf;
-    const float* __restrict__ uin = p.in_uf;
-    __nv_bfloat16* __restrict__ go = p.out_g;
-    __nv_bfloat16* __restrict__ gl = p.out_lo;
-    float wr = 0.0f, dwp = 0.0f;
-    if (valid) wr = __ldg(p.row_w + row);
-    // the g and u of a batch are asked of L2 kPf batches ahead, so each batch's loads find them
-    // there instead of waiting a full memory latency (64 bytes of each per batch and row)
-    constexpr int kPf = 3;
-    auto prefetch_batch = [&](int jc) {
-      const int j0 = ti.nb * BN + 16 * jc;
-      if (valid && jc < BN / 16 && j0 < p.I) {
-        prefetch_l2(gin + (long)row * p.I + j0);
-        prefetch_l2(uin + (long)row * p.I + j0);
-      }
-    };
-#pragma unroll
-    for (int jc = 0; jc < kPf; ++jc) prefetch_batch(jc);
-#pragma unroll 1
-    for (int jc = 0; jc < BN / 16; ++jc) {
-      prefetch_batch(jc + kPf);
-      uint32_t v[16];
-      tmem_ld16(tbase + 16 * jc, v);
-      const int j0 = ti.nb * BN + 16 * jc;
-      const bool act = valid && j0 < p.I;
-      float4 gq[4], uq[4];
-      if (act) {
-        const float4* g4 = reinterpret_cast<const float4*>(gin + (long)row * p.I + j0);
-        const float4* u4 = reinterpret_cast<const float4*>(uin + (long)row * p.I + j0);
+      for (int jp = 0; jp < BN / 64; ++jp) {
+        uint32_t vg[16], vu[16];
+        tmem_ld_16x256_x4(th + 32 * jp, vg);
+        tmem_ld_16x256_x4(th + BN / 2 + 32 * jp, vu);
+        tmem_ld_wait();
+        const int j0 = ti.nb * (BN / 2) + 32 * jp;
+        if (j0 >= p.I) continue;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          gq[q] = __ldg(g4 + q);
-          uq[q] = __ldg(u4 + q);
-        }
-      }
-      tmem_ld_wait();
-      if (act) {
-        const float* gf = reinterpret_cast<const float*>(gq);
-        const float* uf = reinterpret_cast<const float*>(uq);
-        const long od = (long)row * 2 * p.I + j0;
 #pragma unroll
-        for (int hlf = 0; hlf < 2; ++hlf) {
-          float dg[8], du[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float a = __uint_as_float(v[8 * hlf + j]);
-            const float g = gf[8 * hlf + j], u = uf[8 * hlf + j];
-            const float sg = sigmoid_fast(g);
-            const float dh = wr * a;
-            const float sl = g * sg;  // silu(g)
-            dg[j] = dh * u * sg * (1.0f + g * (1.0f - sg));
-            du[j] = dh * sl;
-            // <dh_u, h> with h at fp32 accuracy: a flip of a bf16 h would move a heavy-tailed term
-            dwp = fmaf(a, sl * u, dwp);
-          }
-          uint4 gh, glo, uh, ulo;
-          split_bf16x8(dg, gh, glo);
-          split_bf16x8(du, uh, ulo);
-          *reinterpret_cast<uint4*>(go + od + 8 * hlf) = gh;
-          *reinterpret_cast<uint4*>(go + od + p.I + 8 * hlf) = uh;
-          if (gl != nullptr) {
-            *reinterpret_cast<uint4*>(gl + od + 8 * hlf) = glo;
-            *reinterpret_cast<uint4*>(gl + od + p.I + 8 * hlf) = ulo;
+          for (int rr = 0; rr < 2; ++rr) {
+            const int row = rr ? rb : ra;
+            if (!(rr ? vb : va)) continue;
+            const float g0 = __uint_as_float(vg[4 * q + 2 * rr]), g1 = __uint_as_float(vg[4 * q + 2 * rr + 1]);
+            const float u0 = __uint_as_float(vu[4 * q + 2 * rr]), u1 = __uint_as_float(vu[4 * q + 2 * rr + 1]);
+            const float h0 = silu_f(g0) * u0, h1 = silu_f(g1) * u1;
+            const long o = (long)row * p.I + j0 + 8 * q + cc;
+            *reinterpret_cast<float2*>(p.out_gf + o) = make_float2(g0, g1);
+            *reinterpret_cast<float2*>(p.out_uf + o) = make_float2(u0, u1);
+            const __nv_bfloat162 hh = __floats2bfloat162_rn(h0, h1);
+            *reinterpret_cast<__nv_bfloat162*>(p.out_h + o) = hh;
+            if (p.out_lo != nullptr)
+              *reinterpret_cast<uint32_t*>(p.out_lo + o) =
+                  bf16x2_of(h0 - __low2float(hh), h1 - __high2float(hh));
           }
         }
       }
+
     }
-    if (valid) p.dw_part[(long)row * p.num_n_tiles + ti.nb] = dwp;
   }
 }
 
@@ -638,10 +721,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
 #pragma unroll 1
       for (int h = 0; h < MS; ++h) {
-        const int row = ti.row0 + h * 128 + warp * 32 + lane;
-        const bool valid = row < ti.row_end;
-        const uint32_t tbase = tmem_base + ((uint32_t)(warp * 32) << 16) + buf * C::ACC_COLS + h * BN;
-        epilogue_rows<EPI, BN>(p, ti, row, valid, tbase);
+        const uint32_t tw = tmem_base + ((uint32_t)(warp * 32) << 16) + buf * C::ACC_COLS + h * BN;
+        if (EPI == EPI_SWIGLU_BWD) {
+          const int row = ti.row0 + h * 128 + warp * 32 + lane;
+          epilogue_rows_swiglu_bwd<BN>(p, ti, row, row < ti.row_end, tw);
+        } else {
+          epilogue_warp<EPI, BN>(p, ti, ti.row0 + h * 128 + warp * 32, tw);
+        }
       }
       tc_fence_before();
       __syncwarp();

@@ -560,7 +560,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm2Threads, 1)
         const int row = ti.row0 + 256 * h + 128 * (int)rank + warp * 32 + lane;
         const bool valid = row < ti.row_end;
         const uint32_t tbase = tmem_base + ((uint32_t)(warp * 32) << 16) + buf * C::ACC_COLS + h * BN;
-        epilogue_rows<EPI_STORE, BN>(p, ti, row, valid, tbase);
+        epilogue_rows_store<BN>(p, ti, row, valid, tbase);
       }
       tc_fence_before();
       __syncwarp();

@@ -682,8 +682,11 @@ static int launch_dense_gemm(int qtype, const void* A, int64_t M, int64_t Kd, co
                              int64_t w_cols, const __nv_bfloat16* LA, const __nv_bfloat16* LB, int KL, int64_t Nd,
                              void* out, int out_dtype, float* split_buf, bool allow_split, cudaStream_t st, int slot,
                              int rx = 0, const RowsFuse* rf = nullptr, const CUtensorMap* tRY = nullptr,
-                             const CUtensorMap* tZ = nullptr, bool* sum_pending = nullptr) {
+                             const CUtensorMap* tZ = nullptr, bool* sum_pending = nullptr,
+                             float2* row_stats = nullptr) {
   const DensePlan d = plan_dense(M, Nd, Kd, TRANS, allow_split && split_buf != nullptr);
+  // per-row softmax statistics come from the pair GEMM's fp32 store epilogue, without a K split
+  if (row_stats != nullptr && (d.ms == 0 || d.ksplit != 1 || out_dtype != QL_F32)) return QL_ERR_INVALID_ARG;
   const uint32_t box = 128u;
   CUtensorMap tA, tW, tLA, tLB;
   if (!tmap_bf16_rows(&tA, A, Kd, M, box) ||
@@ -706,6 +709,7 @@ static int launch_dense_gemm(int qtype, const void* A, int64_t M, int64_t Kd, co
   p.ksplit = d.ksplit;
   p.kb_per_split = d.kbs;
   p.ldo = Nd;
+  p.row_stats = row_stats;
   if (d.ksplit > 1) {
     p.out = split_buf;
     p.out_dtype = QL_F32;
@@ -1671,7 +1675,7 @@ static const Adamw8Tables& adamw8_tables() {
 namespace qlora {
 
 struct LmWs {
-  size_t logits, dlog, split_f, split_x, total;
+  size_t logits, dlog, stats, split_f, split_x, total;
 };
 static LmWs lm_ws(int64_t M, int64_t V, int64_t K, int64_t chunk) {
   const int64_t C = std::min(chunk, M);
@@ -1686,6 +1690,7 @@ static LmWs lm_ws(int64_t M, int64_t V, int64_t K, int64_t chunk) {
   size_t o = 0;
   w.logits = o; o = al256(o + (size_t)C * V * 4);
   w.dlog = o; o = al256(o + (size_t)C * V * 2);
+  w.stats = o; o = al256(o + (size_t)C * ((V + 255) / 256) * 8);  // (max, sum exp) per row and 256 columns
   w.split_f = o; o = al256(o + sf);
   w.split_x = o; o = al256(o + sx);
   w.total = o;
@@ -1720,15 +1725,21 @@ extern "C" int qlora_lm_head_ce(int qtype, const void* wq, int64_t V, int64_t K,
   for (int64_t c0 = 0; c0 < M; c0 += C) {
     const int64_t rows = std::min(C, M - c0);
     const __nv_bfloat16* Xc = (const __nv_bfloat16*)X + c0 * K;
-    // logits = X_c deq(W)^T, fp32, no adapter
+    // logits = X_c deq(W)^T, fp32, no adapter; the pair GEMM (more than 128 rows, no K split) also
+    // leaves each row's (max, sum exp) per 256 columns, so the CE kernel reads the logits once
+    const DensePlan d = plan_dense(rows, V, K, false, true);
+    const bool with_stats = d.ms != 0 && d.ksplit == 1 && d.ntiles == (int)((V + 255) / 256);
+    float2* stats = with_stats ? (float2*)(wsb + w.stats) : nullptr;
     int rc = launch_dense_gemm<false>(qtype, Xc, rows, K, wq, V, K, nullptr, nullptr, 0, V, logits, QL_F32,
-                                      (float*)(wsb + w.split_f), true, st, 0);
+                                      (float*)(wsb + w.split_f), true, st, 0, 0, nullptr, nullptr, nullptr,
+                                      nullptr, stats);
     if (rc) return rc;
     // the CE kernel and the input-gradient GEMM each read what the launch right before them wrote:
     // they start only once it has completed
     NoEarlyStart serial;
     lm_ce_kernel<<<(unsigned)std::min<int64_t>(rows, num_sms()), kCeThreads, 0, st>>>(
-        logits, (int)V, (int)rows, labels + c0, grad_scale, loss + c0, dX ? dlog : nullptr);
+        logits, (int)V, (int)rows, stats, with_stats ? d.ntiles : 0, labels + c0, grad_scale, loss + c0,
+        dX ? dlog : nullptr);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     if (launch_status() != QL_OK) return QL_ERR_CUDA;
     if (dX) {

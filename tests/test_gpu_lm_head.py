@@ -24,7 +24,8 @@ def _status():
 
 
 @pytest.mark.parametrize("M,V,K,chunk,qtype", [(300, 1024, 512, 128, inp.Q8_0), (600, 32000, 1024, 256, inp.Q4_K),
-                                               (5, 4096, 256, 64, inp.Q5_K), (260, 2048, 256, 260, inp.Q4_0)])
+                                               (5, 4096, 256, 64, inp.Q5_K), (260, 2048, 256, 260, inp.Q4_0),
+                                               (700, 4160, 512, 384, inp.Q8_0)])  # a partial last column tile
 def test_lm_head_ce_matches_oracle(M, V, K, chunk, qtype):
     rng = np.random.default_rng(M + V)
     W = (rng.standard_normal((V, K)) * 0.05).astype(np.float32)
