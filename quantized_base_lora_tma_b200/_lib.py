@@ -198,7 +198,7 @@ class MoeRoute:
         self.perm = torch.empty(P, dtype=i32, device=device)
         self.inv_perm = torch.empty(P, dtype=i32, device=device)
         self.mblk = torch.empty(E + 1, dtype=i32, device=device)
-        self.ws = torch.empty(max(1, int(lib().qlora_moe_route_workspace_bytes(T, E, k))), dtype=torch.uint8,
+        self.ws = torch.empty(max(1, qlora_moe_route_workspace_bytes(T, E, k)), dtype=torch.uint8,
                               device=device)
 
 
@@ -211,6 +211,10 @@ def qlora_moe_route(logits, k, route=None, stream=None) -> MoeRoute:
                                  _p(route.ws), route.ws.numel(), _s(stream)),
            "qlora_moe_route")
     return route
+
+
+def qlora_moe_route_workspace_bytes(T, E, k) -> int:
+    return int(lib().qlora_moe_route_workspace_bytes(T, E, k))
 
 
 def qlora_moe_saved_bytes(T, k, H, I, r) -> int:

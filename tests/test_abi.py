@@ -38,6 +38,11 @@ def test_every_declared_symbol_is_exported_and_bound(lib):
     assert names == set(_lib.SIGNATURES), names ^ set(_lib.SIGNATURES)
 
 
+def test_every_entry_point_has_a_binding_of_the_same_name(lib):
+    missing = [n for n in _lib.SIGNATURES if not callable(getattr(ql, n, None))]
+    assert not missing, missing
+
+
 def test_status_strings(lib):
     for code, name in _lib.STATUS.items():
         assert ql.qlora_status_string(code) == name
@@ -114,3 +119,93 @@ def test_rows_fusion_switch(lib):
     finally:
         ql.qlora_set_rows_fusion(prev)
     assert prev == 1  # the default: the forward only
+
+
+def test_moe_argument_errors(lib):
+    """Routing and the MoE layer reject bad arguments on the host (no launch)."""
+    L = lib
+    s = None
+    before = ql.qlora_launch_count()
+    wsr = ql.qlora_moe_route_workspace_bytes(64, 8, 2)
+    r6 = [FAKE] * 7  # topk_idx, topk_w, counts, offsets, perm, inv_perm, mblk
+
+    def route(**kw):
+        a = dict(lg=FAKE, T=64, E=8, k=2, ws=FAKE, wsb=wsr)
+        a.update(kw)
+        return L.qlora_moe_route(a["lg"], a["T"], a["E"], a["k"], *r6, a["ws"], a["wsb"], s)
+
+    assert route(lg=None) == 1
+    assert route(E=257) == 2 and route(k=17) == 2 and route(k=9) == 2 and route(k=0) == 2
+    assert route(T=0) == 1
+    assert route(wsb=wsr - 1) == 5 and route(ws=None) == 5
+    assert route(ws=FAKE + 4) == 4
+
+    T, k, E, H, I, r = 64, 2, 8, 256, 256, 4
+    sv = ql.qlora_moe_saved_bytes(T, k, H, I, r)
+    wsm = ql.qlora_moe_workspace_bytes(T, k, E, H, I, r)
+
+    def fwd(**kw):
+        a = dict(qt=2, E=E, H=H, I=I, X=FAKE, T=T, k=k, r=r, Y=FAKE, yd=0, sv=FAKE, svb=sv, ws=FAKE, wsb=wsm)
+        a.update(kw)
+        return L.qlora_moe_fwd(a["qt"], FAKE, FAKE, a["E"], a["H"], a["I"], a["X"], a["T"], a["k"], FAKE, FAKE,
+                               FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, a["r"], 2.0, a["Y"], a["yd"],
+                               a["sv"], a["svb"], a["ws"], a["wsb"], s)
+
+    assert fwd(qt=14) == 2          # Q6_K: dequantization only
+    assert fwd(E=300) == 2 and fwd(k=9) == 2 and fwd(r=65) == 2
+    assert fwd(H=300) == 3 and fwd(I=128) == 3
+    assert fwd(X=FAKE + 2) == 4
+    assert fwd(Y=None) == 1 and fwd(yd=5) == 1
+    assert fwd(svb=sv - 1) == 5 and fwd(wsb=wsm - 1) == 5
+
+    def bwd(**kw):
+        a = dict(dX=FAKE, dxd=0, dl=FAKE, svb=sv, wsb=wsm)
+        a.update(kw)
+        return L.qlora_moe_bwd(2, FAKE, FAKE, E, H, I, FAKE, FAKE, T, k, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                               FAKE, FAKE, FAKE, r, 2.0, FAKE, a["svb"], a["dX"], a["dxd"], FAKE, FAKE, FAKE, FAKE,
+                               a["dl"], FAKE, a["wsb"], s)
+
+    assert bwd(dX=None) == 1 and bwd(dxd=4) == 1
+    assert bwd(dl=FAKE + 4) == 4
+    assert bwd(svb=16) == 5 and bwd(wsb=16) == 5
+    assert ql.qlora_launch_count() == before
+
+
+def test_lm_head_rmsnorm_adamw_argument_errors(lib):
+    """The lm_head, RMSNorm and 8-bit AdamW entry points reject bad arguments on the host."""
+    L = lib
+    s = None
+    before = ql.qlora_launch_count()
+    M, V, K, C = 300, 1024, 512, 128
+    wsl = ql.qlora_lm_head_ce_workspace_bytes(M, V, K, C)
+    assert wsl > 0 and ql.qlora_lm_head_ce_workspace_bytes(0, V, K, C) == 0
+
+    def lm(**kw):
+        a = dict(qt=8, V=V, K=K, X=FAKE, M=M, lab=FAKE, C=C, loss=FAKE, dX=FAKE, dxd=0, ws=FAKE, wsb=wsl)
+        a.update(kw)
+        return L.qlora_lm_head_ce(a["qt"], FAKE, a["V"], a["K"], a["X"], a["M"], a["lab"], a["C"], 1.0, a["loss"],
+                                  a["dX"], a["dxd"], a["ws"], a["wsb"], s)
+
+    assert lm(lab=None) == 1 and lm(loss=None) == 1 and lm(C=0) == 1
+    assert lm(qt=5) == 2
+    assert lm(V=1000) == 3 and lm(K=300) == 3
+    assert lm(dxd=3) == 1
+    assert lm(X=FAKE + 8) == 4
+    assert lm(wsb=wsl - 1) == 5 and lm(ws=None) == 5
+
+    assert L.qlora_rmsnorm_fwd(None, FAKE, 4, 64, 1e-6, FAKE, FAKE, s) == 1
+    assert L.qlora_rmsnorm_fwd(FAKE, FAKE, 4, 60, 1e-6, FAKE, FAKE, s) == 3
+    assert L.qlora_rmsnorm_fwd(FAKE, FAKE, 4, 64, -1.0, FAKE, FAKE, s) == 1
+    assert L.qlora_rmsnorm_fwd(FAKE + 2, FAKE, 4, 64, 1e-6, FAKE, FAKE, s) == 4
+    assert L.qlora_rmsnorm_bwd(FAKE, FAKE, FAKE, FAKE, 7, 4, 64, FAKE, 0, s) == 1
+    assert L.qlora_rmsnorm_bwd(FAKE, FAKE, FAKE, FAKE, 0, 4, 68, FAKE, 0, s) == 3
+
+    def adam(**kw):
+        a = dict(p=FAKE, n=1000, b1=0.9, b2=0.999, eps=1e-8, t=1)
+        a.update(kw)
+        return L.qlora_adamw8_step(a["p"], FAKE, FAKE, FAKE, FAKE, FAKE, a["n"], 1e-3, a["b1"], a["b2"], a["eps"],
+                                   0.01, a["t"], None, s)
+
+    assert adam(p=None) == 1 and adam(n=0) == 1 and adam(t=0) == 1
+    assert adam(b1=1.0) == 1 and adam(b2=-0.1) == 1 and adam(eps=0.0) == 1
+    assert ql.qlora_launch_count() == before
