@@ -740,14 +740,8 @@ def main():
                     help="profiling driver: run three steps of the named workload and exit (no timing, no JSON line)")
     ap.add_argument("--fwd-only", action="store_true", help="with --calls: forwards only")
     ap.add_argument("--ncalls", type=int, default=3, help="with --calls: how many")
-    ap.add_argument("--decode-calls", type=int, default=0, choices=[0, 1, 4, 16], metavar="M",
-                    help="profiling driver: three forwards of the decode-shaped Q4_0 8192x8192 linear with M "
-                         "tokens (same as --calls decode_mM --fwd-only)")
-    ap.add_argument("--decode-bwd", action="store_true", help="with --decode-calls: forward and backward")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
-    if args.decode_calls:
-        args.calls, args.fwd_only = f"decode_m{args.decode_calls}", not args.decode_bwd
     if args.calls:
         profile_calls(args.calls, args.ncalls, args.fwd_only)
         return
