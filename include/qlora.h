@@ -133,8 +133,8 @@ int qlora_linear_bwd(int qtype, const void* wq, int64_t N, int64_t K, const void
                      void* stream);
 
 /* ---------------------------------------------------------------------------------------------
- * Routed MoE layer with SwiGLU experts ("MoE routing", "grouped MMQ" and the fast LoRA backward
- * "for linear layer and MoE layer" of Show HN: LoRA over GGUF, "Things involved in the training").
+ * Routed MoE layer with SwiGLU experts (the recipe's MoE routing, grouped quantized matmul and fast
+ * LoRA backward for the MoE layer: Show HN: LoRA over GGUF, "Things involved in the training").
  * Expert e: gate/up weight Wgu_e [2I x H] (rows [0, I) gate, [I, 2I) up), down weight Wd_e [H x I],
  * packed and stacked [E][rows][...]; adapters A_gu [E][r][H], B_gu [E][2I][r], A_d [E][r][I],
  * B_d [E][H][r] (bf16); s = scale.
@@ -212,7 +212,7 @@ int qlora_lm_head_ce(int qtype, const void* wq, int64_t V, int64_t K, const void
                      void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------------------
- * RMSNorm in front of the first projection ("RMSNorm from Liger Kernel", Show HN: LoRA over GGUF,
+ * RMSNorm in front of the first projection (the recipe's Liger RMSNorm, Show HN: LoRA over GGUF,
  * "Things involved in the training"). X [M x K] bf16, gamma [K] bf16 (frozen), K % 8 == 0.
  * Forward: rstd[m] = 1 / sqrt(mean_k X[m][k]^2 + eps) (fp32), Xn = bf16(X rstd gamma) [M x K]: the
  * bf16 input of qlora_linear_fwd / qlora_linear_bwd. One pass per row (a warp per row).

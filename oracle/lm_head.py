@@ -2,7 +2,7 @@
 
 Test infrastructure only: nothing in the library calls this module.
 
-The recipe trains with "chunked cross entropy loss like Liger Kernel, which works with MMQ" (Show HN:
+The recipe trains with a Liger-style chunked cross-entropy over the quantized matmul's logits (Show HN:
 LoRA over GGUF, "Things involved in the training"): the logits of the quantized output projection
 feed a per-token cross-entropy, chunked over tokens so the full logits never exist at once. Chunking
 changes where the work happens, not what is computed, so the oracle is the plain definition:

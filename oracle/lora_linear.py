@@ -3,7 +3,7 @@
 Test infrastructure only: nothing in the library calls this module.
 
 What it computes (the method's layer: a frozen GGUF base weight plus a trainable low-rank adapter,
-"Fast LoRA bwd formula like Unsloth for linear layer and MoE layer", Show HN: LoRA over GGUF,
+whose backward the recipe takes from an Unsloth-style fast LoRA formula, Show HN: LoRA over GGUF,
 "Things involved in the training"; the pages print no formula, so the one below is the plain chain
 rule of the layer's definition):
 

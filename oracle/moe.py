@@ -2,9 +2,9 @@
 
 Test infrastructure only: nothing in the library calls this module.
 
-Sources on the pages: MoE routing "like OpenAI triton-kernels", grouped MMQ for the quantized
-experts, "AITER gmm/ptgmm" for the non-quantized per-expert LoRA products, and the fast LoRA
-backward "for linear layer and MoE layer" (Show HN: LoRA over GGUF, "Things involved in the
+Sources on the pages: MoE routing after OpenAI's Triton kernels, a grouped quantized matmul for the
+experts, AITER's grouped matmuls for the non-quantized per-expert LoRA products, and the fast LoRA
+backward for both the linear and the MoE layer (Show HN: LoRA over GGUF, "Things involved in the
 training"); only active experts are loaded and their outputs are aggregated by a sparse reduce
 (ai-manual.ru, "Fused dequant-matmul и MoE kernels: как это работает"); the load-balancing loss is
 disabled (same Show HN list), so no auxiliary router loss appears here.

@@ -2,7 +2,7 @@
 
 Test infrastructure only: nothing in the library calls this module.
 
-The recipe's training stack normalizes each token with RMSNorm ("RMSNorm from Liger Kernel", Show HN:
+The recipe's training stack normalizes each token with Liger's RMSNorm (Show HN:
 LoRA over GGUF, "Things involved in the training") before the projections the layer implements. The
 pages print no formula; this is the standard definition. For a token row x of K values, a frozen
 gain g (part of the base model, never updated) and eps:

@@ -1,5 +1,5 @@
 // Small-M forward of the layer (M <= 16 tokens, decode-shaped): Y = X deq(W)^T + s (X A^T) B^T and
-// H = X A^T. This is the weight-streaming regime of the layer ("MMQ" for a few tokens, Show HN:
+// H = X A^T. This is the weight-streaming regime of the layer (the quantized matmul at a few tokens, Show HN:
 // LoRA over GGUF, "Things involved in the training"): every packed weight byte is read once and
 // each weight is used M times, so the kernels are built to keep HBM busy with as few instructions
 // per weight as the decode allows. Three launches:

@@ -1,5 +1,5 @@
 // Cross-entropy over the vocabulary for one chunk of token rows of an lm_head's fp32 logits (the
-// recipe's "chunked cross entropy loss like Liger Kernel, which works with MMQ", Show HN: LoRA over
+// recipe's chunked cross-entropy over the quantized matmul's logits, in the Liger manner, Show HN: LoRA over
 // GGUF, "Things involved in the training"). A CTA takes rows in turn: an online max / sum of
 // exponentials over the row (float4 loads), lse = max + log(sum), loss = lse - logit[label]; then, if
 // asked, the gradient of the summed loss times grad_scale, (softmax - onehot(label)) * grad_scale, in

@@ -12,8 +12,8 @@
 // lora_rows_seg_kernel, colred_mma_kernel + colred_reduce_kernel, lora_bop_vec_kernel.
 //
 // The fast LoRA backward these implement is the plain chain rule of the layer (Show HN: LoRA over
-// GGUF, "Things involved in the training": "Fast LoRA bwd formula like Unsloth for linear layer
-// and MoE layer"). Adapter gradients stay in fp32 end to end.
+// GGUF, "Things involved in the training", which names an Unsloth-style fast LoRA backward for the
+// linear and the MoE layer). Adapter gradients stay in fp32 end to end.
 #pragma once
 #include <cuda_bf16.h>
 

@@ -1,7 +1,7 @@
 // Routed MoE helpers: routing (top-k, counts, scan, permutation), gathers and the slot-ordered
-// combine. "MoE routing like OpenAI triton-kernels" (Show HN: LoRA over GGUF, "Things involved in
+// combine. The recipe's MoE routing, after OpenAI's Triton routing kernels (Show HN: LoRA over GGUF, "Things involved in
 // the training"); only the selected experts' weights are read and their outputs are summed per
-// token ("sparse reduce", ai-manual.ru, "Fused dequant-matmul и MoE kernels").
+// token (a sparse reduction, ai-manual.ru, "Fused dequant-matmul и MoE kernels").
 //
 // Routing of token t over E experts: the k largest logits, equal logits going to the lower expert
 // index, in descending order (slot 0 = largest); weight of slot j = softmax over the k selected

@@ -1,6 +1,6 @@
 // Dequant-in-shared-memory tcgen05 GEMM: D[M, Nd] = A[M, Kd] * deq(W)^T-or-deq(W) (+ LoRA k-blocks).
 //
-// This is the base matmul of the layer ("MMQ and grouped MMQ like llama.cpp", Show HN: LoRA over
+// This is the base matmul of the layer (the recipe's llama.cpp-style quantized and grouped matmuls, Show HN: LoRA over
 // GGUF, "Things involved in the training"; the fused dequant-matmul that expands packed weights on
 // chip without an fp16 intermediate in memory, ai-manual.ru, "Fused dequant-matmul и MoE kernels").
 // It is designed for sm_100a rather than after those kernels:

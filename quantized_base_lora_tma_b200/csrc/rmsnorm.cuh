@@ -1,4 +1,4 @@
-// RMSNorm in front of the layer's first projection ("RMSNorm from Liger Kernel", Show HN: LoRA over
+// RMSNorm in front of the layer's first projection (the recipe takes its RMSNorm from Liger, Show HN: LoRA over
 // GGUF, "Things involved in the training"): x_n = x r g with r = 1 / sqrt(mean(x^2) + eps) and a
 // frozen gain g. One warp per token row, 16-byte loads: the forward reads x once for the sum of
 // squares and once more (from L2) to write the projection's bf16 input x_n and r; the backward forms
