@@ -3,8 +3,8 @@
 Both sides of every parity test, and the benchmark, draw their inputs from here. This module holds
 no step of the layer's own arithmetic (no block decode, no matmul, no routing): it draws random
 tensors, stores them as bf16 bit patterns, and packs fp32 weights into GGUF blocks. Packing is the
-offline quantization that happens before training starts ("GGUF as the base model format for
-low-VRAM LoRA training", Show HN: LoRA over GGUF, opening paragraph); the layer itself only ever
+offline quantization that happens before training starts (the recipe trains LoRA over a GGUF base
+model to save memory, Show HN: LoRA over GGUF, opening paragraph); the layer itself only ever
 reads the packed bytes.
 
 Conventions
