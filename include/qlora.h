@@ -42,10 +42,10 @@ extern "C" {
 #pragma GCC visibility push(default)
 #endif
 
-/* GGML type ids of the supported block formats. Q6_K (210-byte superblocks, not a multiple of 16
- * bytes, so not copied by TMA) is supported by gguf_dequant only; the layer entry points return
- * QL_ERR_UNSUPPORTED for it. */
-typedef enum { QL_Q4_0 = 2, QL_Q8_0 = 8, QL_Q4_K = 12, QL_Q5_K = 13, QL_Q6_K = 14 } ql_qtype;
+/* GGML type ids of the supported block formats. Q2_K (84-byte superblocks) and Q6_K (210 bytes),
+ * whose superblocks are not a multiple of 16 bytes and so are not copied by TMA, are supported by
+ * gguf_dequant only; the layer entry points return QL_ERR_UNSUPPORTED for them. */
+typedef enum { QL_Q4_0 = 2, QL_Q8_0 = 8, QL_Q2_K = 10, QL_Q4_K = 12, QL_Q5_K = 13, QL_Q6_K = 14 } ql_qtype;
 
 /* Element type of an output tensor. */
 typedef enum { QL_F32 = 0, QL_BF16 = 1 } ql_dtype;
@@ -96,7 +96,7 @@ int qlora_selftest_wait_timeout(int64_t limit_us, void* stream);
  * gguf_dequant — expand packed GGUF rows to fp32 or bf16.
  * The pages' recipe runs a standalone GGUF dequant function (Show HN: LoRA over GGUF, "Other
  * notes"); the layer's own kernels never call this: they expand blocks in shared memory.
- *   qtype     QL_Q4_0 | QL_Q8_0 | QL_Q4_K | QL_Q5_K | QL_Q6_K
+ *   qtype     QL_Q4_0 | QL_Q8_0 | QL_Q2_K | QL_Q4_K | QL_Q5_K | QL_Q6_K
  *   wq        [rows][cols/QK blocks] packed bytes
  *   rows      > 0
  *   cols      > 0, multiple of 256

@@ -1,11 +1,11 @@
-"""Oracle: GGUF block decode (Q4_0, Q8_0, Q4_K), exact in fp64.
+"""Oracle: GGUF block decode (Q4_0, Q8_0, Q2_K, Q4_K, Q5_K, Q6_K), exact in fp64.
 
 Test infrastructure only: nothing in the library calls this module.
 
 The pages name GGUF as the frozen base format and say the training recipe runs a standalone
 dequant function over it (Show HN: LoRA over GGUF, "Other notes": the GGUF dequant function;
 aimodeling.com "GGUF steps up: a full kernel stack"). They do not print the block layouts; the
-layouts below are the public GGUF/ggml encodings of these three types, written out from their
+layouts below are the public GGUF/ggml encodings of these types, written out from their
 definitions:
 
   Q4_0  18-byte block of 32: fp16 d; 16 bytes, byte j = q[j] | q[j+16] << 4; w = d * (q - 8).
@@ -18,13 +18,18 @@ definitions:
   Q5_K  176-byte superblock of 256: fp16 d, fp16 dmin, the same 12 scale bytes as Q4_K, 32 bytes
         qh, 128 bytes of nibbles laid out as in Q4_K. Weight l of sub-block j takes its fifth bit
         from bit j of qh[l]: q = nibble + 16 * ((qh[l] >> j) & 1) in [0, 32); w = d*sc_j*q - dmin*m_j.
+  Q2_K  84-byte superblock of 256: 16 scale bytes (low nibble the scale, high nibble the min of one
+        16-weight group), 64 bytes of 2-bit codes, fp16 d, fp16 dmin (bytes 80, 82). Each half h of
+        128 weights uses qs[32h:32h+32]: its weight 32a + l (a in 0..3, l in 0..31) has the code
+        (qs[32h + l] >> 2a) & 3 and the scale byte S = scales[8h + 2a + l // 16]:
+        w = d * (S & 15) * q - dmin * (S >> 4).
   Q6_K  210-byte superblock of 256: 128 bytes ql, 64 bytes qh, 16 int8 scales, fp16 d (last).
         Each half h of 128 weights uses ql[64h:64h+64], qh[32h:32h+32] and scales[8h:8h+8]; its
         weight 32a + l (a in 0..3, l in 0..31) has low bits from ql[64h + 32(a & 1) + l] (low nibble
         for a < 2, high nibble otherwise), high bits (qh[32h + l] >> 2a) & 3, and scale
         scales[8h + 2a + l // 16]: q = low | high << 4 in [0, 64), w = d * scale * (q - 32).
 
-Every decoded value is exact in fp64 (and, except the Q4_K / Q5_K difference, already in fp32:
+Every decoded value is exact in fp64 (and, except the Q2_K / Q4_K / Q5_K difference, already in fp32:
 at most 24 significant bits). ``deq_f32`` rounds the exact value once to fp32 (round to
 nearest even); ``deq_bf16`` rounds that fp32 value to bf16 (round to nearest even). The layer
 multiplies bf16 weight tiles, so ``deq_bf16`` is what the matmul oracles use.
@@ -33,9 +38,9 @@ from __future__ import annotations
 
 import numpy as np
 
-Q4_0, Q8_0, Q4_K, Q5_K, Q6_K = 2, 8, 12, 13, 14
-_QK = {Q4_0: 32, Q8_0: 32, Q4_K: 256, Q5_K: 256, Q6_K: 256}
-_BB = {Q4_0: 18, Q8_0: 34, Q4_K: 144, Q5_K: 176, Q6_K: 210}
+Q4_0, Q8_0, Q2_K, Q4_K, Q5_K, Q6_K = 2, 8, 10, 12, 13, 14
+_QK = {Q4_0: 32, Q8_0: 32, Q2_K: 256, Q4_K: 256, Q5_K: 256, Q6_K: 256}
+_BB = {Q4_0: 18, Q8_0: 34, Q2_K: 84, Q4_K: 144, Q5_K: 176, Q6_K: 210}
 
 
 def _fp16_at(blocks: np.ndarray, off: int) -> np.ndarray:
@@ -129,7 +134,24 @@ def decode_q6_k(raw, rows, cols) -> np.ndarray:
     return w.reshape(rows, cols)
 
 
-_DECODERS = {Q4_0: decode_q4_0, Q8_0: decode_q8_0, Q4_K: decode_q4_k, Q5_K: decode_q5_k, Q6_K: decode_q6_k}
+def decode_q2_k(raw, rows, cols) -> np.ndarray:
+    b = _blocks(Q2_K, raw, rows, cols)
+    S = b[:, 0:16].astype(np.int64)
+    qs = b[:, 16:80].astype(np.int64)
+    d = _fp16_at(b, 80)
+    dmin = _fp16_at(b, 82)
+    w = np.empty((b.shape[0], 256), np.float64)
+    l = np.arange(32)
+    for h in range(2):
+        for a in range(4):
+            q = ((qs[:, 32 * h + l] >> (2 * a)) & 3).astype(np.float64)
+            sb = S[:, 8 * h + 2 * a + l // 16]
+            w[:, 128 * h + 32 * a + l] = d[:, None] * (sb & 15) * q - dmin[:, None] * (sb >> 4)
+    return w.reshape(rows, cols)
+
+
+_DECODERS = {Q4_0: decode_q4_0, Q8_0: decode_q8_0, Q2_K: decode_q2_k, Q4_K: decode_q4_k, Q5_K: decode_q5_k,
+             Q6_K: decode_q6_k}
 
 
 def decode_exact(qtype, raw, rows, cols) -> np.ndarray:

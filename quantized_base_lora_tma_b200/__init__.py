@@ -5,7 +5,7 @@ The kernels live in ``libqlora.so`` (built from ``csrc/`` by ``build.py``) behin
 marshalling only). ``inputs`` holds the seeded synthetic workloads and the offline GGUF packers.
 """
 from ._lib import (  # noqa: F401
-    Q4_0, Q4_K, Q5_K, Q6_K, Q8_0, QL_BF16, QL_F32, QloraError, lib,
+    Q2_K, Q4_0, Q4_K, Q5_K, Q6_K, Q8_0, QL_BF16, QL_F32, QloraError, lib,
     gguf_dequant,
     qlora_linear_workspace_bytes, qlora_linear_fwd, qlora_linear_bwd, qlora_linear_fwd_noalloc,
     MoeRoute, qlora_moe_route_workspace_bytes, qlora_moe_route, qlora_moe_saved_bytes, qlora_moe_workspace_bytes,

@@ -14,7 +14,7 @@ import torch
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libqlora.so")
 
-Q4_0, Q8_0, Q4_K, Q5_K, Q6_K = 2, 8, 12, 13, 14
+Q4_0, Q8_0, Q2_K, Q4_K, Q5_K, Q6_K = 2, 8, 10, 12, 13, 14
 QL_F32, QL_BF16 = 0, 1
 QL_OK = 0
 STATUS = {0: "QL_OK", 1: "QL_ERR_INVALID_ARG", 2: "QL_ERR_UNSUPPORTED", 3: "QL_ERR_SHAPE",

@@ -35,6 +35,11 @@ template <>
 struct QTraits<QL_Q5_K> {
   static constexpr int kGroupBytes = 176;
 };
+// 84 bytes is not a multiple of 16 either: like Q6_K, Q2_K is read by the standalone dequant only.
+template <>
+struct QTraits<QL_Q2_K> {
+  static constexpr int kGroupBytes = 84;
+};
 // 210 bytes is not a multiple of 16: Q6_K groups cannot be TMA-copied one by one, so only the
 // standalone dequant (byte and half-word loads) reads them.
 template <>
@@ -172,6 +177,27 @@ __device__ __forceinline__ void decode8<QL_Q6_K>(const uint8_t* g, int c, float 
     const int q1 = (int)((lo.y >> (8 * i + sl)) & 15u) | (int)(((hi.y >> (8 * i + shh)) & 3u) << 4);
     w[i] = ds * (float)(q0 - 32);
     w[4 + i] = ds * (float)(q1 - 32);
+  }
+}
+
+// Q2_K superblock (84 B): 16 scale bytes (low nibble scale, high nibble min, one per 16 weights),
+// 64 bytes of 2-bit codes, fp16 d at 80, fp16 dmin at 82. Weight 32a + l of half h: code
+// (qs[32h + l] >> 2a) & 3, scale byte S = scales[8h + 2a + l / 16]; w = d*(S & 15)*q - dmin*(S >> 4).
+// Both products are exact in fp32 (at most 11 + 4 + 2 bits); one fp32 FMA rounds the difference
+// once. The superblocks are 4-byte aligned; the 8 codes of a chunk are two aligned words.
+template <>
+__device__ __forceinline__ void decode8<QL_Q2_K>(const uint8_t* g, int c, float (&w)[8]) {
+  const int h = c >> 4, p0 = 8 * (c & 15);
+  const int a = p0 >> 5, l0 = p0 & 31;
+  const int S = g[8 * h + 2 * a + (l0 >> 4)];
+  const float ds = half_at(g + 80) * (float)(S & 15);
+  const float dm = -(half_at(g + 82) * (float)(S >> 4));
+  const uint32_t* qw = reinterpret_cast<const uint32_t*>(g + 16 + 32 * h + l0);
+  const uint32_t q0 = qw[0] >> (2 * a), q1 = qw[1] >> (2 * a);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    w[i] = __fmaf_rn(ds, (float)((q0 >> (8 * i)) & 3u), dm);
+    w[4 + i] = __fmaf_rn(ds, (float)((q1 >> (8 * i)) & 3u), dm);
   }
 }
 
@@ -416,6 +442,17 @@ __device__ __forceinline__ uint4 decode8_bf16(const uint8_t* g, int c) {
   float w[8];
   decode8<QT>(g, c, w);
   return pack_bf16x8(w);
+}
+
+// Q2_K unit u (weights 32u .. 32u + 31): the four 8-weight chunks of decode8, each rounded to bf16.
+template <>
+__device__ __forceinline__ void decode_unit_bf16<QL_Q2_K>(const uint8_t* g, int u, uint4 (&out)[4]) {
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    float w[8];
+    decode8<QL_Q2_K>(g, 4 * u + cc, w);
+    out[cc] = pack_bf16x8(w);
+  }
 }
 
 }  // namespace qlora

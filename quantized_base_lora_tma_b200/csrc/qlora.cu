@@ -1122,7 +1122,7 @@ int qlora_selftest_wait_timeout(int64_t limit_us, void* stream) {
 
 int gguf_dequant(int qtype, const void* wq, int64_t rows, int64_t cols, void* out, int out_dtype, void* stream) {
   if (!wq || !out) return QL_ERR_INVALID_ARG;
-  if (group_bytes(qtype) == 0 && qtype != QL_Q6_K) return QL_ERR_UNSUPPORTED;
+  if (group_bytes(qtype) == 0 && qtype != QL_Q6_K && qtype != QL_Q2_K) return QL_ERR_UNSUPPORTED;
   if (out_dtype != QL_F32 && out_dtype != QL_BF16) return QL_ERR_INVALID_ARG;
   if (rows < 1 || cols < 1) return QL_ERR_INVALID_ARG;
   if (cols % 256 != 0) return QL_ERR_SHAPE;
@@ -1136,6 +1136,7 @@ int gguf_dequant(int qtype, const void* wq, int64_t rows, int64_t cols, void* ou
     case QL_Q4_K: gguf_dequant_kernel<QL_Q4_K><<<grid, 256, 0, st>>>((const uint8_t*)wq, rows, cols, out, out_dtype); break;
     case QL_Q5_K: gguf_dequant_kernel<QL_Q5_K><<<grid, 256, 0, st>>>((const uint8_t*)wq, rows, cols, out, out_dtype); break;
     case QL_Q6_K: gguf_dequant_kernel<QL_Q6_K><<<grid, 256, 0, st>>>((const uint8_t*)wq, rows, cols, out, out_dtype); break;
+    case QL_Q2_K: gguf_dequant_kernel<QL_Q2_K><<<grid, 256, 0, st>>>((const uint8_t*)wq, rows, cols, out, out_dtype); break;
   }
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return launch_status();

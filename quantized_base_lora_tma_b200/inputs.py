@@ -25,13 +25,14 @@ import numpy as np
 # GGML type ids (the numbers the GGUF container uses for these block types).
 Q4_0 = 2
 Q8_0 = 8
+Q2_K = 10
 Q4_K = 12
 Q5_K = 13
 Q6_K = 14
 
-QK = {Q4_0: 32, Q8_0: 32, Q4_K: 256, Q5_K: 256, Q6_K: 256}          # elements per block
-BLOCK_BYTES = {Q4_0: 18, Q8_0: 34, Q4_K: 144, Q5_K: 176, Q6_K: 210}  # bytes per block
-QTYPE_NAMES = {Q4_0: "q4_0", Q8_0: "q8_0", Q4_K: "q4_k", Q5_K: "q5_k", Q6_K: "q6_k"}
+QK = {Q4_0: 32, Q8_0: 32, Q2_K: 256, Q4_K: 256, Q5_K: 256, Q6_K: 256}          # elements per block
+BLOCK_BYTES = {Q4_0: 18, Q8_0: 34, Q2_K: 84, Q4_K: 144, Q5_K: 176, Q6_K: 210}  # bytes per block
+QTYPE_NAMES = {Q4_0: "q4_0", Q8_0: "q8_0", Q2_K: "q2_k", Q4_K: "q4_k", Q5_K: "q5_k", Q6_K: "q6_k"}
 QTYPE_BY_NAME = {v: k for k, v in QTYPE_NAMES.items()}
 
 
@@ -224,7 +225,48 @@ def pack_q6_k(w: np.ndarray) -> np.ndarray:
     return out.reshape(rows, -1)
 
 
-PACKERS = {Q4_0: pack_q4_0, Q8_0: pack_q8_0, Q4_K: pack_q4_k, Q5_K: pack_q5_k, Q6_K: pack_q6_k}
+def pack_q2_k(w: np.ndarray) -> np.ndarray:
+    """Q2_K with a plain min/max encoder.
+
+    Per 16-weight group g: lo = min(0, min x), scale_g = (max x - lo) / 3, min_g = -lo; d = max
+    scale_g / 15 and dmin = max min_g / 15 (fp16); sc_g = round(scale_g / d) and m_g =
+    round(min_g / dmin), each clamped to [0, 15] with the fp16 d and dmin; q = round((x + dmin*m_g)
+    / (d*sc_g)) clamped to [0, 3] (0 where d*sc_g = 0). Byte layout: 16 bytes sc_g | m_g << 4, 64
+    bytes of codes (weight 32a + l of half h at bit 2a of qs[32h + l]), fp16 d, fp16 dmin.
+    """
+    rows, cols = w.shape
+    x = np.ascontiguousarray(w, dtype=np.float32).reshape(-1, 16, 16)
+    nb = x.shape[0]
+    lo = np.minimum(np.float32(0), x.min(axis=2))
+    scale = (x.max(axis=2) - lo) / np.float32(3)
+    mn = -lo
+    d16 = (scale.max(axis=1) / np.float32(15)).astype(np.float16)
+    m16 = (mn.max(axis=1) / np.float32(15)).astype(np.float16)
+    d = d16.astype(np.float32)[:, None]
+    dm = m16.astype(np.float32)[:, None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        sc = np.where(d > 0, _round_half_away(scale / d), 0)
+        m = np.where(dm > 0, _round_half_away(mn / dm), 0)
+    sc = np.clip(sc, 0, 15).astype(np.uint8)
+    m = np.clip(m, 0, 15).astype(np.uint8)
+    step = (d * sc.astype(np.float32))[:, :, None]
+    off = (dm * m.astype(np.float32))[:, :, None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = np.where(step != 0, _round_half_away((x + off) / step), 0)
+    q = np.clip(q, 0, 3).astype(np.uint8).reshape(nb, 256)
+    out = np.zeros((nb, 84), np.uint8)
+    out[:, 0:16] = sc | (m << 4)
+    l = np.arange(32)
+    for h in range(2):
+        for a in range(4):
+            out[:, 16 + 32 * h + l] |= q[:, 128 * h + 32 * a + l] << (2 * a)
+    out[:, 80:82] = d16.view(np.uint8).reshape(-1, 2)
+    out[:, 82:84] = m16.view(np.uint8).reshape(-1, 2)
+    return out.reshape(rows, -1)
+
+
+PACKERS = {Q4_0: pack_q4_0, Q8_0: pack_q8_0, Q2_K: pack_q2_k, Q4_K: pack_q4_k, Q5_K: pack_q5_k,
+           Q6_K: pack_q6_k}
 
 
 def pack(qtype: int, w: np.ndarray) -> np.ndarray:

@@ -88,6 +88,7 @@ def test_linear_argument_errors(lib):
     assert fwd(r=65) == 2
     assert fwd(qt=3) == 2
     assert fwd(qt=14) == 2  # Q6_K: gguf_dequant only (its 210-byte superblocks are not TMA-copied)
+    assert fwd(qt=10) == 2  # Q2_K: likewise (84-byte superblocks)
     assert fwd(X=None) == 1
     assert fwd(M=0) == 1
     assert fwd(X=FAKE + 8) == 4

@@ -26,8 +26,8 @@ def _reset_status():
 def _random_packed(qtype, rows, cols, rng):
     w = (rng.standard_normal((rows, cols)) * 0.02).astype(np.float32)
     raw = inp.pack(qtype, w)
-    # sprinkle subnormal and zero scales (d of Q4_0 / Q8_0 blocks, d of Q6_K superblocks)
-    off = {inp.Q4_0: 0, inp.Q8_0: 0, inp.Q6_K: 208}.get(qtype)
+    # sprinkle subnormal and zero scales (d of Q4_0 / Q8_0 blocks, d of Q6_K and Q2_K superblocks)
+    off = {inp.Q4_0: 0, inp.Q8_0: 0, inp.Q6_K: 208, inp.Q2_K: 80}.get(qtype)
     if off is not None:
         bb = inp.BLOCK_BYTES[qtype]
         v = raw.reshape(-1, bb)
@@ -36,7 +36,7 @@ def _random_packed(qtype, rows, cols, rng):
     return raw
 
 
-@pytest.mark.parametrize("qtype", [inp.Q4_0, inp.Q8_0, inp.Q4_K, inp.Q5_K, inp.Q6_K])
+@pytest.mark.parametrize("qtype", [inp.Q4_0, inp.Q8_0, inp.Q4_K, inp.Q5_K, inp.Q6_K, inp.Q2_K])
 def test_dequant_bit_exact(qtype):
     rng = np.random.default_rng(qtype)
     rows, cols = 37, 768

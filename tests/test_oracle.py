@@ -110,12 +110,34 @@ def test_hand_packed_q6_k():
     assert np.array_equal(got, want)
 
 
+def test_hand_packed_q2_k():
+    """A Q2_K superblock written byte by byte from chosen 4-bit scales, 4-bit mins and 2-bit codes:
+    weight 32a + l of half h has its code at bit 2a of qs[32h + l] and the scale byte
+    scales[8h + 2a + l // 16] (low nibble the scale, high nibble the min); d and dmin are the fp16
+    values at bytes 80 and 82."""
+    sc = [0, 1, 2, 3, 5, 8, 13, 15, 7, 4, 9, 11, 6, 10, 12, 14]
+    mn = [15, 0, 3, 7, 1, 2, 9, 4, 0, 15, 5, 6, 8, 10, 11, 13]
+    q = [(5 * i + 2) % 4 for i in range(256)]
+    qs = [0] * 64
+    for h in range(2):
+        for a in range(4):
+            for l in range(32):
+                qs[32 * h + l] |= q[128 * h + 32 * a + l] << (2 * a)
+    scales = [s | (m << 4) for s, m in zip(sc, mn)]
+    raw = np.frombuffer(bytes(scales + qs + [0x00, 0x34, 0x00, 0x38]), np.uint8)  # d = 0.25, dmin = 0.5
+    assert raw.size == 84
+    got = gb.decode_exact(gb.Q2_K, raw, 1, 256)[0]
+    g = [8 * (i // 128) + 2 * ((i % 128) // 32) + (i % 32) // 16 for i in range(256)]
+    want = np.array([0.25 * sc[g[i]] * q[i] - 0.5 * mn[g[i]] for i in range(256)])
+    assert np.array_equal(got, want)
+
+
 def _random_blocks(qtype, nblocks, rng):
-    bb = {gb.Q4_0: 18, gb.Q8_0: 34, gb.Q4_K: 144, gb.Q5_K: 176, gb.Q6_K: 210}[qtype]
+    bb = {gb.Q4_0: 18, gb.Q8_0: 34, gb.Q2_K: 84, gb.Q4_K: 144, gb.Q5_K: 176, gb.Q6_K: 210}[qtype]
     raw = rng.integers(0, 256, size=(nblocks, bb), dtype=np.uint8)
     # finite fp16 scales only (random bytes could spell Inf/NaN): bytes 0-1 (and 2-3 for the
     # superblocks with a dmin), or the last two bytes of a Q6_K superblock
-    offs = {gb.Q4_K: [0, 2], gb.Q5_K: [0, 2], gb.Q6_K: [208]}.get(qtype, [0])
+    offs = {gb.Q2_K: [80, 82], gb.Q4_K: [0, 2], gb.Q5_K: [0, 2], gb.Q6_K: [208]}.get(qtype, [0])
     for o in offs:
         d = (rng.standard_normal(nblocks) * 0.01).astype(np.float16)
         d[::7] = np.float16(6.0e-8)                    # include subnormal scales
@@ -124,7 +146,7 @@ def _random_blocks(qtype, nblocks, rng):
 
 
 @pytest.mark.parametrize("qtype,gtype", [(gb.Q4_0, "Q4_0"), (gb.Q8_0, "Q8_0"), (gb.Q4_K, "Q4_K"),
-                                         (gb.Q5_K, "Q5_K"), (gb.Q6_K, "Q6_K")])
+                                         (gb.Q5_K, "Q5_K"), (gb.Q6_K, "Q6_K"), (gb.Q2_K, "Q2_K")])
 def test_decode_matches_gguf_py(qtype, gtype):
     """Independent codebase: gguf-py's dequantize (fp32) must equal the fp32 rounding of the exact
     decode, element by element."""
@@ -160,6 +182,28 @@ def test_packers_match_gguf_py_bytes(gtype):
     x[3, :32] = 0.0
     qt = {"Q4_0": inp.Q4_0, "Q8_0": inp.Q8_0}[gtype]
     assert np.array_equal(inp.pack(qt, x), quants.quantize(x, getattr(gguf.GGMLQuantizationType, gtype)))
+
+
+def test_pack_q2_k_picks_the_nearest_code():
+    """The Q2_K encoder: every weight decodes to the representable value d*sc*q - dmin*m (q in 0..3,
+    from the block's own packed scale and min) nearest to it."""
+    rng = np.random.default_rng(9)
+    x = (rng.standard_normal((8, 512)) * 0.02).astype(np.float32)
+    x[2, :16] = 0.0
+    x[5, 16:32] = np.abs(x[5, 16:32])        # a group with no negative values (min 0)
+    raw = inp.pack(inp.Q2_K, x)
+    w = gb.decode_exact(gb.Q2_K, raw, 8, 512)
+    b = raw.reshape(-1, 84)
+    d = b[:, 80:82].copy().view(np.float16).astype(np.float64).ravel()
+    dm = b[:, 82:84].copy().view(np.float16).astype(np.float64).ravel()
+    S = b[:, 0:16].astype(np.int64)
+    step = d[:, None] * (S & 15)                           # [superblock, group]
+    off = dm[:, None] * (S >> 4)
+    grid = step[:, :, None] * np.arange(4) - off[:, :, None]   # [sb, group, 4]
+    xs = x.astype(np.float64).reshape(-1, 16, 16)
+    nearest = np.abs(xs[:, :, :, None] - grid[:, :, None, :]).min(axis=3)
+    err = np.abs(w.reshape(-1, 16, 16) - xs)
+    assert np.all(err <= nearest + 1e-6 * (step[:, :, None] + 1e-12))
 
 
 @pytest.mark.parametrize("qtype", [inp.Q4_0, inp.Q8_0, inp.Q4_K, inp.Q5_K, inp.Q6_K])
